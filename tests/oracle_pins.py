@@ -1,0 +1,414 @@
+"""Pins for the float64 oracle: checks against facts that do not come from the
+oracle itself (library special cases, closed forms, brute force, invariants and
+the values printed on the GQA glossary page).
+
+Each ``pin_*`` function raises AssertionError on failure.  They are collected
+as tests by ``test_oracle_pins.py`` and re-run against deliberately broken
+copies of the oracle by ``test_oracle_mutations.py``.
+"""
+from __future__ import annotations
+
+import math
+import os
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+
+import oracle.ccgqa as O
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def read_golden(name: str) -> dict:
+    vals = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            k, v = (s.strip() for s in line.split("=", 1))
+            vals[k] = v
+    return vals
+
+
+def _close(a, b, tol=1e-12, what=""):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, f"{what}: shape {a.shape} != {b.shape}"
+    err = float(np.max(np.abs(a - b))) if a.size else 0.0
+    scale = max(1.0, float(np.max(np.abs(b))) if b.size else 1.0)
+    assert err <= tol * scale, f"{what}: max abs err {err:.3e} > {tol:.1e}"
+
+
+def _rng(seed=0):
+    return np.random.default_rng(seed)
+
+
+def _small_layer(E=64, C=2, Hq=4, Hkv=2, K=4, seed=3, qk=True, vs=True, base=100.0,
+                 causal=True, chan=True, packed=False):
+    sh = O.Shape(E, C, Hq, Hkv)
+    r = _rng(seed)
+    d = sh.d
+    return O.Layer(
+        sh=sh,
+        W_qkv=None if packed else r.standard_normal((sh.n_qkv, E)) / math.sqrt(E),
+        conv_width=K,
+        conv_q_seq=r.standard_normal((Hq * d, K)) * 0.5 if K else None,
+        conv_q_chan=(r.standard_normal((Hq, d, d)) / math.sqrt(d)) if (K and chan) else None,
+        conv_k_seq=r.standard_normal((Hkv * d, K)) * 0.5 if K else None,
+        conv_k_chan=(r.standard_normal((Hkv, d, d)) / math.sqrt(d)) if (K and chan) else None,
+        qk_mean=qk, value_shift=vs, rope_base=base, causal=causal)
+
+
+# --------------------------------------------------------------------------
+# Attention core
+# --------------------------------------------------------------------------
+def brute_force_attention(q, k, v, G, causal, q_pos):
+    """Pure-Python loops, written from the definition of softmax attention."""
+    T, Hq, d = q.shape
+    L = k.shape[0]
+    out = np.zeros((T, Hq, d))
+    for ti in range(T):
+        for h in range(Hq):
+            g = h // G
+            scores = []
+            for s in range(L):
+                if causal and s > q_pos[ti]:
+                    continue
+                dot = 0.0
+                for i in range(d):
+                    dot += q[ti, h, i] * k[s, g, i]
+                scores.append((s, dot / math.sqrt(d)))
+            top = max(sc for _, sc in scores)
+            w = [(s, math.exp(sc - top)) for s, sc in scores]
+            tot = sum(x for _, x in w)
+            for s, x in w:
+                for i in range(d):
+                    out[ti, h, i] += x / tot * v[s, g, i]
+    return out
+
+
+def pin_gqa_glossary_example():
+    """The GQA page's example: grouped attention equals attention on copied
+    key/value heads; shape and cached-value counts as printed."""
+    g = read_golden("gqa_glossary_example.txt")
+    B, Hq, Hkv, T, d = (int(g[k]) for k in ("batch", "query_heads", "kv_heads", "tokens", "head_dim"))
+    gen = torch.Generator().manual_seed(0)
+    q = torch.randn(B, Hq, T, d, generator=gen, dtype=torch.float64)
+    k = torch.randn(B, Hkv, T, d, generator=gen, dtype=torch.float64)
+    v = torch.randn(B, Hkv, T, d, generator=gen, dtype=torch.float64)
+    grouped = F.scaled_dot_product_attention(q, k, v, is_causal=True, enable_gqa=True)
+    copied = F.scaled_dot_product_attention(
+        q, k.repeat_interleave(Hq // Hkv, dim=1), v.repeat_interleave(Hq // Hkv, dim=1),
+        is_causal=True)
+    assert tuple(grouped.shape) == tuple(int(s) for s in g["output_shape"].split())
+    assert (bool(torch.allclose(grouped, copied, atol=1e-6)) == (g["matches_copied_heads"] == "True"))
+    # the oracle on the same tensors ([T, H, d] layout)
+    o = O.attention(q[0].permute(1, 0, 2).numpy(), k[0].permute(1, 0, 2).numpy(),
+                    v[0].permute(1, 0, 2).numpy(), Hq // Hkv, True)
+    _close(o, grouped[0].permute(1, 0, 2).numpy(), 1e-12, "oracle vs SDPA(enable_gqa)")
+    _close(o, copied[0].permute(1, 0, 2).numpy(), 1e-12, "oracle vs SDPA(copied heads)")
+    assert O.cache_values_per_token(Hkv, d) == int(g["cached_values_per_token_gqa"])
+    assert O.cache_values_per_token(Hq, d) == int(g["cached_values_per_token_mha"])
+
+
+def pin_mqa_and_mha_reductions():
+    """One kv group is MQA; as many kv heads as query heads is MHA
+    (GQA page, "Cómo funciona GQA")."""
+    r = _rng(1)
+    T, Hq, d = 7, 4, 8
+    q = r.standard_normal((T, Hq, d))
+    k1 = r.standard_normal((T, 1, d))
+    v1 = r.standard_normal((T, 1, d))
+    mqa = O.attention(q, k1, v1, Hq, True)
+    for h in range(Hq):
+        ref = F.scaled_dot_product_attention(
+            torch.from_numpy(q[:, h][None]), torch.from_numpy(k1[:, 0][None]),
+            torch.from_numpy(v1[:, 0][None]), is_causal=True)[0].numpy()
+        _close(mqa[:, h], ref, 1e-12, f"MQA head {h}")
+    kf = r.standard_normal((T, Hq, d))
+    vf = r.standard_normal((T, Hq, d))
+    mha = O.attention(q, kf, vf, 1, False)
+    ref = F.scaled_dot_product_attention(
+        torch.from_numpy(q.transpose(1, 0, 2)), torch.from_numpy(kf.transpose(1, 0, 2)),
+        torch.from_numpy(vf.transpose(1, 0, 2)), is_causal=False).numpy().transpose(1, 0, 2)
+    _close(mha, ref, 1e-12, "MHA")
+
+
+def pin_attention_brute_force():
+    """Tiny shapes against pure-Python loops, causal and not, with offset
+    query positions and a group size of 3."""
+    r = _rng(2)
+    for causal in (True, False):
+        T, L, Hq, Hkv, d = 5, 9, 6, 2, 4
+        q = r.standard_normal((T, Hq, d))
+        k = r.standard_normal((L, Hkv, d))
+        v = r.standard_normal((L, Hkv, d))
+        pos = np.array([0, 2, 3, 7, 8])
+        _close(O.attention(q, k, v, 3, causal, q_pos=pos),
+               brute_force_attention(q, k, v, 3, causal, pos), 1e-12, f"brute causal={causal}")
+
+
+def pin_attention_closed_forms():
+    """Single visible key returns its value; scores ln 3 apart give weights
+    3/4 and 1/4; all-ones values give ones."""
+    d = 4
+    k = np.zeros((2, 1, d))
+    k[0, 0, 0] = 1.0
+    v = np.zeros((2, 1, d))
+    v[0, 0, :] = [1, 2, 3, 4]
+    v[1, 0, :] = [5, 6, 7, 8]
+    q = np.zeros((2, 1, d))
+    q[:, 0, 0] = math.sqrt(d) * math.log(3.0)   # score(key 0) - score(key 1) = ln 3
+    o = O.attention(q, k, v, 1, True)
+    _close(o[0, 0], v[0, 0], 1e-12, "first position sees only key 0")
+    _close(o[1, 0], 0.75 * v[0, 0] + 0.25 * v[1, 0], 1e-12, "weights 3/4, 1/4")
+    r = _rng(4)
+    q = r.standard_normal((6, 4, 8)) * 3
+    k = r.standard_normal((6, 2, 8)) * 3
+    _close(O.attention(q, k, np.ones((6, 2, 8)), 2, True), np.ones((6, 4, 8)), 1e-12, "V = 1")
+
+
+# --------------------------------------------------------------------------
+# RoPE
+# --------------------------------------------------------------------------
+def pin_rope_closed_form():
+    """d = 2: the single pair turns by t radians whatever the base.
+    d = 4, base 100: pairs (0, 2) and (1, 3) turn by t and t / 10."""
+    t = np.array([0.0, 1.0, 2.5, 40.0])
+    z = np.zeros((4, 1, 2))
+    z[:, 0, 0] = 1.0
+    r = O.rope(z, t, 12345.0)
+    _close(r[:, 0, 0], np.cos(t), 1e-14, "d=2 cos")
+    _close(r[:, 0, 1], np.sin(t), 1e-14, "d=2 sin")
+    z = np.zeros((4, 1, 4))
+    z[:, 0, 1] = 1.0              # second pair, first component
+    r = O.rope(z, t, 100.0)
+    _close(r[:, 0, 1], np.cos(t / 10), 1e-14, "pair 1 cos")
+    _close(r[:, 0, 3], np.sin(t / 10), 1e-14, "pair 1 sin")
+    _close(r[:, 0, 0], 0 * t, 0, "pair 0 untouched")
+    _close(r[:, 0, 2], 0 * t, 0, "pair 0 untouched")
+    z = np.zeros((4, 1, 4))
+    z[:, 0, 2] = 1.0              # first pair, second component: (0,1) -> (-sin, cos)
+    r = O.rope(z, t, 100.0)
+    _close(r[:, 0, 0], -np.sin(t), 1e-14, "rotate-half sign")
+    _close(r[:, 0, 2], np.cos(t), 1e-14, "rotate-half cos")
+    # position 0 is the identity; base 0 disables
+    zz = _rng(5).standard_normal((3, 2, 8))
+    _close(O.rope(zz, np.zeros(3), 1e4), zz, 0, "position 0")
+    _close(O.rope(zz, np.arange(3), 0.0), zz, 0, "base 0")
+
+
+def pin_rope_relative_offset():
+    """Scores after RoPE depend only on the position difference."""
+    r = _rng(6)
+    q = r.standard_normal((1, 3, 16))
+    k = r.standard_normal((1, 3, 16))
+    for base in (1e4, 5e5):
+        s0 = np.einsum("thd,thd->h", O.rope(q, np.array([9]), base), O.rope(k, np.array([4]), base))
+        for p in (1, 37, 1000):
+            s1 = np.einsum("thd,thd->h", O.rope(q, np.array([9 + p]), base),
+                           O.rope(k, np.array([4 + p]), base))
+            _close(s1, s0, 1e-9, f"shift {p}")
+        # the norm is kept
+        _close(np.linalg.norm(O.rope(q, np.array([123]), base)), np.linalg.norm(q), 1e-12, "norm")
+
+
+# --------------------------------------------------------------------------
+# Convolution, QK-mean, value-shift, projection
+# --------------------------------------------------------------------------
+def pin_seq_conv_closed_forms():
+    r = _rng(7)
+    S, Ch, K = 9, 5, 4
+    z = r.standard_normal((S, Ch))
+    w = np.zeros((Ch, K))
+    w[:, 0] = 1.0
+    _close(O.seq_conv(z, w), z, 0, "identity tap")
+    for j in range(1, K):
+        w = np.zeros((Ch, K))
+        w[:, j] = 1.0
+        exp = np.zeros_like(z)
+        exp[j:] = z[:-j]
+        _close(O.seq_conv(z, w), exp, 0, f"shift by {j}")
+        hist = r.standard_normal((K - 1, Ch))
+        exp_h = exp.copy()
+        exp_h[:j] = hist[K - 1 - j: K - 1]   # rows -j .. -1 come from the history
+        _close(O.seq_conv(z, w, hist), exp_h, 0, f"shift by {j} with history")
+    # per-channel taps: channel c scaled by (c + 1), tap 0 only
+    w = np.zeros((Ch, K))
+    w[:, 0] = np.arange(1, Ch + 1)
+    _close(O.seq_conv(z, w), z * np.arange(1, Ch + 1), 0, "depthwise scale")
+    # sum of all taps = 1 on a constant sequence (away from the start)
+    w = r.random((Ch, K))
+    w /= w.sum(axis=1, keepdims=True)
+    _close(O.seq_conv(np.ones((S, Ch)), w)[K - 1:], np.ones((S - K + 1, Ch)), 1e-14, "partition of unity")
+
+
+def pin_channel_mix_permutation():
+    """A cyclic permutation matrix moves channel i+1 to channel i; a transposed
+    operand would move it the other way."""
+    r = _rng(8)
+    S, H, d = 3, 2, 5
+    u = r.standard_normal((S, H, d))
+    P = np.zeros((H, d, d))
+    for i in range(d):
+        P[:, i, (i + 1) % d] = 1.0
+    _close(O.channel_mix(u, P), np.roll(u, -1, axis=2), 0, "cyclic permutation")
+    D = np.zeros((H, d, d))
+    D[0] = np.eye(d) * 2.0
+    D[1] = np.eye(d) * -1.0
+    exp = u.copy()
+    exp[:, 0] *= 2.0
+    exp[:, 1] *= -1.0
+    _close(O.channel_mix(u, D), exp, 0, "per-head matrices")
+
+
+def pin_qk_mean_closed_form():
+    """Constant heads: q~ head h = h + 1, k~ head g = 10 (g + 1)."""
+    S, Hq, Hkv, d = 2, 4, 2, 3
+    G = Hq // Hkv
+    q = np.zeros((S, Hq, d))
+    k = np.zeros((S, Hkv, d))
+    for h in range(Hq):
+        q[:, h] = h + 1
+    for g in range(Hkv):
+        k[:, g] = 10 * (g + 1)
+    m_q, m_k = O.qk_mean(q, k, G)
+    exp_q = np.array([(1 + 10) / 2, (2 + 10) / 2, (3 + 20) / 2, (4 + 20) / 2])
+    exp_k = np.array([((1 + 2) / 2 + 10) / 2, ((3 + 4) / 2 + 20) / 2])
+    _close(m_q[0, :, 0], exp_q, 0, "m_q")
+    _close(m_k[0, :, 0], exp_k, 0, "m_k")
+    r = _rng(9)
+    q1 = r.standard_normal((4, 3, 6))
+    k1 = r.standard_normal((4, 3, 6))
+    a, b = O.qk_mean(q1, k1, 1)
+    _close(a, b, 0, "G = 1: one shared mean")
+
+
+def pin_value_shift_gather():
+    r = _rng(10)
+    S, Hkv, d = 6, 3, 8
+    v = r.standard_normal((S, Hkv, d))
+    out = O.value_shift(v)
+    assert np.array_equal(out[:, :, : d // 2], v[:, :, : d // 2])
+    assert np.array_equal(out[1:, :, d // 2:], v[:-1, :, d // 2:])
+    assert np.all(out[0, :, d // 2:] == 0)
+    prev = r.standard_normal((Hkv, d))
+    out = O.value_shift(v, prev)
+    assert np.array_equal(out[0, :, d // 2:], prev[:, d // 2:])
+
+
+def pin_down_project_blocks():
+    """With W = I the projection returns the column blocks q | k | v in order."""
+    sh = O.Shape(E=48, C=1, Hq=2, Hkv=1)     # d = 24, n_qkv = 96
+    x = _rng(11).standard_normal((3, sh.n_qkv))
+    q, k, v = O.down_project(x, None, sh)
+    d = sh.d
+    _close(q.reshape(3, -1), x[:, :2 * d], 0, "q block")
+    _close(k.reshape(3, -1), x[:, 2 * d:3 * d], 0, "k block")
+    _close(v.reshape(3, -1), x[:, 3 * d:], 0, "v block")
+    sh2 = O.Shape(E=sh.n_qkv, C=2, Hq=1, Hkv=1)   # E = 96, d = 48, n_qkv = 144
+    x2 = _rng(12).standard_normal((3, sh2.E))
+    W2 = np.zeros((sh2.n_qkv, sh2.E))
+    W2[:96, :96] = np.eye(96)                     # q = x[:, :48], k = x[:, 48:96], v = 0
+    q2, k2, v2 = O.down_project(x2, W2, sh2)
+    _close(q2.reshape(3, -1), x2[:, :48], 0, "q from W rows")
+    _close(k2.reshape(3, -1), x2[:, 48:96], 0, "k from W rows")
+    _close(v2, np.zeros_like(v2), 0, "v rows zero")
+
+
+# --------------------------------------------------------------------------
+# Whole-layer invariants
+# --------------------------------------------------------------------------
+def pin_causality():
+    """Changing tokens after position t leaves outputs up to t unchanged
+    (covers the convolution, the value-shift and the mask)."""
+    lay = _small_layer()
+    r = _rng(13)
+    S = 12
+    x = r.standard_normal((S, lay.sh.E))
+    o1, _ = O.prefill(lay, x)
+    x2 = x.copy()
+    x2[7:] = r.standard_normal((S - 7, lay.sh.E))
+    o2, _ = O.prefill(lay, x2)
+    _close(o2[:7], o1[:7], 1e-13, "prefix unchanged")
+    assert np.max(np.abs(o2[7:] - o1[7:])) > 1e-3, "later rows must change"
+
+
+def pin_decode_matches_prefill():
+    """prefill over S tokens, row S-1 == prefill over S-1 tokens followed by one
+    decode step; the decode state equals the longer prefill's state."""
+    for lay in (_small_layer(), _small_layer(K=2, chan=False, qk=False),
+                _small_layer(K=0, qk=False, vs=False, base=0.0)):
+        r = _rng(14)
+        S = 10
+        x = r.standard_normal((S, lay.sh.E))
+        full, st_full = O.prefill(lay, x)
+        part, st = O.prefill(lay, x[:-1])
+        o, st2 = O.decode_step(lay, st, x[-1])
+        _close(o, full[-1], 1e-12, "decode row")
+        _close(st2.k, st_full.k, 1e-12, "cache k")
+        _close(st2.v, st_full.v, 1e-12, "cache v")
+        _close(st2.hist_q, st_full.hist_q, 1e-13, "hist q")
+        _close(st2.hist_k, st_full.hist_k, 1e-13, "hist k")
+        _close(st2.v_prev, st_full.v_prev, 1e-13, "v_prev")
+        # two more steps from the end of the full prefill stay consistent
+        x3 = r.standard_normal((2, lay.sh.E))
+        ref, _ = O.prefill(lay, np.concatenate([x, x3]))
+        o1, s1 = O.decode_step(lay, st_full, x3[0])
+        o2, _ = O.decode_step(lay, s1, x3[1])
+        _close(np.stack([o1, o2]), ref[-2:], 1e-12, "two steps")
+
+
+def pin_prefill_rows_subset():
+    lay = _small_layer()
+    x = _rng(15).standard_normal((11, lay.sh.E))
+    full, _ = O.prefill(lay, x)
+    rows = np.array([0, 3, 10])
+    part, _ = O.prefill(lay, x, rows=rows)
+    _close(part, full[rows], 0, "sampled rows")
+
+
+def pin_features_off_is_plain_gqa():
+    """With no conv, QK-mean, value-shift or RoPE the layer is plain GQA on the
+    projected heads (library special case: SDPA with grouped heads)."""
+    lay = _small_layer(K=0, qk=False, vs=False, base=0.0, packed=True)
+    sh = lay.sh
+    x = _rng(16).standard_normal((9, sh.n_qkv))
+    o, _ = O.prefill(lay, x)
+    d = sh.d
+    q = torch.from_numpy(x[:, :sh.Hq * d].reshape(9, sh.Hq, d).transpose(1, 0, 2).copy())
+    k = torch.from_numpy(x[:, sh.Hq * d:(sh.Hq + sh.Hkv) * d].reshape(9, sh.Hkv, d).transpose(1, 0, 2).copy())
+    v = torch.from_numpy(x[:, (sh.Hq + sh.Hkv) * d:].reshape(9, sh.Hkv, d).transpose(1, 0, 2).copy())
+    ref = F.scaled_dot_product_attention(q[None], k[None], v[None], is_causal=True, enable_gqa=True)
+    _close(o, ref[0].permute(1, 0, 2).reshape(9, -1).numpy(), 1e-12, "plain GQA")
+
+
+def pin_cache_sizing():
+    """The GQA page's Llama 3.1 8B cache arithmetic."""
+    g = read_golden("gqa_cache_sizing.txt")
+    L, H, d, b, ctx, Hm = (int(g[k]) for k in ("layers", "kv_heads", "head_dim", "bytes_per_value",
+                                               "context_tokens", "mha_kv_heads"))
+    per_tok = L * O.cache_values_per_token(H, d) * b
+    assert per_tok == int(g["kib_per_token_gqa"]) * 1024
+    assert per_tok * ctx == int(g["gib_full_context_gqa"]) * 2 ** 30
+    per_tok_m = L * O.cache_values_per_token(Hm, d) * b
+    assert per_tok_m == int(g["kib_per_token_mha"]) * 1024
+    assert per_tok_m * ctx == int(g["gib_full_context_mha"]) * 2 ** 30
+
+
+def pin_compression_factor():
+    """Attention work and cache shrink by the compression factor C at a fixed
+    head count (CCA page, "Belangrijkste Bijdragen" and "Resultaten" 3)."""
+    E, Hq, S = 4096, 32, 1000
+    for C in (1, 2, 4, 8):
+        sh = O.Shape(E, C, Hq, Hq)
+        mha = O.Shape(E, 1, Hq, Hq)
+        assert O.attention_flops(S, Hq, sh.d) * C == O.attention_flops(S, Hq, mha.d)
+        assert O.cache_values_per_token(Hq, sh.d) * C == O.cache_values_per_token(Hq, mha.d)
+    # counted flops equal the visible score pairs times 4 d
+    assert O.attention_flops(4, 1, 8, causal=False) == 4 * 8 * 16
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

@@ -1,0 +1,151 @@
+"""Planted mistakes in the oracle (CPU only): every plausible slip -- a dropped
+term, a wrong sign or index, a transposed operand -- must make at least one pin
+fail.  Each mutant replaces one oracle function for the duration of the test."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle.ccgqa as O
+import oracle_pins
+
+_orig = {name: getattr(O, name) for name in
+         ("seq_conv", "channel_mix", "qk_mean", "rope", "value_shift", "attention",
+          "down_project", "prefill", "decode_step")}
+
+
+def _seq_conv_drop_last_tap(z, w, history=None):
+    w = w.copy()
+    w[:, -1] = 0
+    return _orig["seq_conv"](z, w, history)
+
+
+def _seq_conv_anticausal(z, w, history=None):
+    return _orig["seq_conv"](z[::-1].copy(), w, None)[::-1].copy()
+
+
+def _seq_conv_history_reversed(z, w, history=None):
+    return _orig["seq_conv"](z, w, None if history is None else history[::-1].copy())
+
+
+def _channel_mix_transposed(u, W):
+    return _orig["channel_mix"](u, np.swapaxes(W, 1, 2))
+
+
+def _qk_mean_self(q, k, G):
+    return 0.5 * (q + q), 0.5 * (k + k)
+
+
+def _qk_mean_no_half(q, k, G):
+    a, b = _orig["qk_mean"](q, k, G)
+    return 2 * a, 2 * b
+
+
+def _qk_mean_head_mod(q, k, G):
+    S, Hq, d = q.shape
+    Hkv = k.shape[1]
+    kk = k[:, np.arange(Hq) % Hkv]
+    return 0.5 * (q + kk), _orig["qk_mean"](q, k, G)[1]
+
+
+def _rope_sign(z, pos, base):
+    return _orig["rope"](z, -np.asarray(pos, dtype=np.float64), base)
+
+
+def _rope_interleaved(z, pos, base):
+    d = z.shape[-1]
+    perm = np.concatenate([np.arange(0, d, 2), np.arange(1, d, 2)])
+    inv = np.argsort(perm)
+    return _orig["rope"](z[..., perm], pos, base)[..., inv]
+
+
+def _rope_theta(z, pos, base):
+    # exponent -i/d instead of -2i/d: same as squaring the base's root
+    return _orig["rope"](z, pos, math.sqrt(base) if base else base)
+
+
+def _value_shift_lower(v, v_prev=None):
+    out = _orig["value_shift"](v[..., ::-1].copy(), None if v_prev is None else v_prev[..., ::-1].copy())
+    return out[..., ::-1].copy()
+
+
+def _value_shift_two(v, v_prev=None):
+    return _orig["value_shift"](_orig["value_shift"](v, v_prev), v_prev)
+
+
+def _attention_no_scale(q, k, v, G, causal, q_pos=None):
+    return _orig["attention"](q * math.sqrt(q.shape[-1]), k, v, G, causal, q_pos)
+
+
+def _attention_strict_mask(q, k, v, G, causal, q_pos=None):
+    T = q.shape[0]
+    pos = np.arange(T) if q_pos is None else np.asarray(q_pos)
+    if not causal:
+        return _orig["attention"](q, k, v, G, causal, q_pos)
+    out = np.zeros_like(q)
+    for i, t in enumerate(pos):
+        if t == 0:
+            out[i] = 0
+        else:
+            out[i] = _orig["attention"](q[i:i + 1], k[:t], v[:t], G, True, np.array([t - 1]))[0]
+    return out
+
+
+def _attention_head_mod(q, k, v, G, causal, q_pos=None):
+    Hq = q.shape[1]
+    Hkv = k.shape[1]
+    idx = np.arange(Hq) % Hkv
+    return _orig["attention"](q, k[:, idx], v[:, idx], 1, causal, q_pos)
+
+
+def _down_project_kv_swapped(x, W, sh):
+    q, k, v = _orig["down_project"](x, W, sh)
+    return q, v, k
+
+
+def _prefill_hist_reversed(layer, x, rows=None):
+    o, st = _orig["prefill"](layer, x, rows)
+    st.hist_q = st.hist_q[::-1].copy()
+    st.hist_k = st.hist_k[::-1].copy()
+    return o, st
+
+
+def _decode_keeps_old_vprev(layer, state, x_t):
+    o, ns = _orig["decode_step"](layer, state, x_t)
+    ns.v_prev = state.v_prev
+    return o, ns
+
+
+MUTANTS = {
+    "seq_conv_drop_last_tap": ("seq_conv", _seq_conv_drop_last_tap),
+    "seq_conv_anticausal": ("seq_conv", _seq_conv_anticausal),
+    "seq_conv_history_reversed": ("seq_conv", _seq_conv_history_reversed),
+    "channel_mix_transposed": ("channel_mix", _channel_mix_transposed),
+    "qk_mean_self": ("qk_mean", _qk_mean_self),
+    "qk_mean_no_half": ("qk_mean", _qk_mean_no_half),
+    "qk_mean_head_mod": ("qk_mean", _qk_mean_head_mod),
+    "rope_sign": ("rope", _rope_sign),
+    "rope_interleaved": ("rope", _rope_interleaved),
+    "rope_theta": ("rope", _rope_theta),
+    "value_shift_lower_half": ("value_shift", _value_shift_lower),
+    "value_shift_two_steps": ("value_shift", _value_shift_two),
+    "attention_no_scale": ("attention", _attention_no_scale),
+    "attention_strict_mask": ("attention", _attention_strict_mask),
+    "attention_head_mod": ("attention", _attention_head_mod),
+    "down_project_kv_swapped": ("down_project", _down_project_kv_swapped),
+    "prefill_hist_reversed": ("prefill", _prefill_hist_reversed),
+    "decode_keeps_old_vprev": ("decode_step", _decode_keeps_old_vprev),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, monkeypatch):
+    fn_name, mutant = MUTANTS[name]
+    monkeypatch.setattr(O, fn_name, mutant)
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin()
+        except (AssertionError, ValueError, IndexError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin catches the planted mistake {name}"
