@@ -1,0 +1,372 @@
+"""Benchmark of the CCGQA hot path on B200.
+
+One step = one pass of the whole path over one batch: bf16 prefill of
+B=4 x S=4096 tokens (latent projection on tcgen05, fused conv / QK-mean / RoPE /
+value-shift, tcgen05 flash attention, cache write) followed by one decode step
+of every sequence against the cache the prefill just wrote (projection, one-token
+pre-step with cache append, split-K attention over S+1 keys).
+
+Prints one JSON line (rank 0).  Timing: W untimed warm-up steps, then K steps,
+each preceded by an untimed write of a buffer larger than L2 and timed with CUDA
+events on the launching stream; the job is bracketed by a barrier and
+torch.cuda.synchronize() on both sides and the time is the max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "bf16_prefill_b4_s4096"
+METRIC = "CCGQA prefill TFLOP/s & tokens/s; decode latent-KV GB/s vs B200 peak"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+ATTN_SRC = os.path.join(ROOT, "compressed_latent_grouped_b200", "csrc", "attn_prefill_tc.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_prefill_tc_traffic.txt")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def attn_traffic_per_launch():
+    """DRAM bytes of one attention launch from the committed ncu capture, or
+    None when the kernel source changed since the capture."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    vals = {}
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#") and "=" in line:
+                k, v = (s.strip() for s in line.split("=", 1))
+                vals[k] = v
+    with open(ATTN_SRC, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()[:16]
+    if vals.get("source_sha256_16") != h or vals.get("workload") != WORKLOAD:
+        return None
+    return float(vals["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x1: "gpu_idle", 0x2: "applications_clocks_setting",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # noqa: BLE001 - report null clocks instead
+            self.max_mhz = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl" if torch.cuda.is_available() else "gloo",
+                                timeout=timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device):
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------- oracle
+def oracle_step_time(w, inp, b: int = 0):
+    """One bounded sample of the workload through the float64 oracle on the
+    host cores: the prefill of sequence b (all S tokens) plus its decode step."""
+    import numpy as np
+    import oracle.ccgqa as O
+    f = lambda t: None if t is None else t.double().numpy()  # noqa: E731
+    lay = O.Layer(sh=O.Shape(w.E, w.C, w.Hq, w.Hkv), W_qkv=f(inp["W_qkv"]),
+                  conv_width=w.conv_width, conv_q_seq=f(inp["conv_q_seq"]),
+                  conv_q_chan=f(inp["conv_q_chan"]), conv_k_seq=f(inp["conv_k_seq"]),
+                  conv_k_chan=f(inp["conv_k_chan"]), qk_mean=w.qk_mean,
+                  value_shift=w.value_shift, rope_base=w.rope_base, causal=w.causal)
+    x = f(inp["x"][b])
+    t0 = time.perf_counter()
+    _, st = O.prefill(lay, x)
+    O.decode_step(lay, st, x[-1])
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def run_reference(args, world, rank):
+    from compressed_latent_grouped_b200.workloads import WORKLOADS, make_inputs
+    if rank != 0:
+        return
+    w = WORKLOADS[WORKLOAD]
+    inp = make_inputs(w, seed=0, batch=1)
+    for _ in range(args.warmup):
+        oracle_step_time(w, inp)
+    times = [oracle_step_time(w, inp) for _ in range(args.steps)]
+    t = sum(times)
+    tokens = (w.S + 1) * args.steps
+    value = tokens / t
+    cores = blas_threads()
+    sample = f"1 of {w.B} sequences per step: prefill of all {w.S} tokens + 1 decode step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded PCG64 normals)",
+        "config": {"workload": WORKLOAD, "B": w.B, "S": w.S, "E": w.E, "C": w.C, "Hq": w.Hq,
+                   "Hkv": w.Hkv, "d": w.d, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------- ours
+def run_ours(args, world, rank, local):
+    import torch
+    from compressed_latent_grouped_b200 import binding as B
+    from compressed_latent_grouped_b200.device import DeviceLayer
+    from compressed_latent_grouped_b200.workloads import WORKLOADS, make_inputs
+    import oracle.ccgqa as O
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = WORKLOADS[WORKLOAD]
+    inp = make_inputs(w, seed=rank)
+    lay = DeviceLayer(w, inp, device=dev, cap=w.S + 1)
+    lay.alloc_cache()
+    x = inp["x"].to(dev)
+    g = torch.Generator().manual_seed(1000 + rank)
+    x_t = torch.randn(w.B, w.E, generator=g).to(w.torch_dtype).to(dev)
+    out = torch.empty(w.B, w.S, w.Hq * w.d, dtype=w.torch_dtype, device=dev)
+    out_t = torch.empty(w.B, w.Hq * w.d, dtype=w.torch_dtype, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        lay.prefill(x, out)
+        lay.decode_step(x_t, out_t)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if lay.error_bits():
+        raise RuntimeError(f"device error bits {lay.error_bits()}")
+
+    K = args.steps
+    mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    st_ev = [(mk(), mk()) for _ in range(K)]
+    pf_ev = [[mk() for _ in range(4)] for _ in range(K)]
+    dc_ev = [[mk() for _ in range(4)] for _ in range(K)]
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    n0 = B.ccgqa_launch_count()
+    with sampler:
+        for i in range(K):
+            flush.zero_()
+            st_ev[i][0].record(stream)
+            B.ccgqa_set_phase_events(pf_ev[i])
+            lay.prefill(x, out)
+            B.ccgqa_set_phase_events(dc_ev[i])
+            lay.decode_step(x_t, out_t)
+            B.ccgqa_set_phase_events(None)
+            st_ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    launches = B.ccgqa_launch_count() - n0
+    barrier(world)
+    if lay.error_bits():
+        raise RuntimeError(f"device error bits {lay.error_bits()}")
+    step_ms = [a.elapsed_time(b) for a, b in st_ev]
+    t_ms = max_over_ranks(sum(step_ms), world, dev)
+    phase = lambda evs, i, j: sum(e[i].elapsed_time(e[j]) for e in evs) / K  # noqa: E731
+    proj_ms, pre_ms, attn_ms = phase(pf_ev, 0, 1), phase(pf_ev, 1, 2), phase(pf_ev, 2, 3)
+    dproj_ms, dpre_ms, dattn_ms = phase(dc_ev, 0, 1), phase(dc_ev, 1, 2), phase(dc_ev, 2, 3)
+    prefill_ms = phase(pf_ev, 0, 3)
+
+    tokens_per_step = w.B * w.S + w.B
+    value = tokens_per_step * K * world / (t_ms / 1e3)
+    attn_flop = w.B * O.attention_flops(w.S, w.Hq, w.d)
+    proj_flop = 2.0 * w.B * w.S * w.E * w.n_qkv
+    kv_bytes = 2 * w.B * w.Hkv * (w.S + 1) * w.d * 2
+    peaks, peak_kind = load_peaks()
+    achieved = attn_flop / (attn_ms / 1e3) / 1e12
+    traffic = attn_traffic_per_launch()
+
+    # end to end through the public API: pinned host buffers in, results out
+    x_h = inp["x"].pin_memory()
+    xt_h = x_t.cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    outt_h = torch.empty(out_t.shape, dtype=out_t.dtype).pin_memory()
+    x_d = torch.empty_like(x)
+    xt_d = torch.empty_like(x_t)
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        xt_d.copy_(xt_h, non_blocking=True)
+        lay.prefill(x_d, out)
+        lay.decode_step(xt_d, out_t)
+        out_h.copy_(out, non_blocking=True)
+        outt_h.copy_(out_t, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = mk(), mk()
+    e0.record(stream)
+    for _ in range(K):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    barrier(world)
+    h2d = x.numel() * x.element_size() + x_t.numel() * x_t.element_size()
+    d2h = out.numel() * out.element_size() + out_t.numel() * out_t.element_size()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        one = make_inputs(w, seed=0, batch=1)
+        t_cpu = oracle_step_time(w, one)
+        cpu = {"value": (w.S + 1) / t_cpu, "unit": "tokens/s", "cores": blas_threads(),
+               "kind": "oracle",
+               "sample": f"1 of {w.B} sequences: float64 prefill of all {w.S} tokens + 1 "
+                         f"decode step ({t_cpu:.1f} s)"}
+
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": max(args.warmup, 3), "ms_per_step": t_ms / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded PCG64 normals, weights N(0, 1/fan_in))",
+        "config": {"workload": f"{WORKLOAD} prefill + 1 decode step", "B": w.B, "S": w.S,
+                   "E": w.E, "C": w.C, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+                   "conv_width": w.conv_width, "rope_base": w.rope_base,
+                   "parallelism": f"replicas x{world} (independent sequences per GPU)",
+                   "l2": "flushed (256 MiB write) before every timed step"},
+        "roofline": {"bound": "tensor", "kernel": "attn_prefill_tc", "achieved": achieved,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                     "peak_kind": f"{peak_kind} bf16 dense burst",
+                     "flop_per_launch": attn_flop, "ms_per_launch": attn_ms},
+        "phases_ms": {"proj_gemm": proj_ms, "pre_attn": pre_ms, "attn_prefill_tc": attn_ms,
+                      "prefill_total": prefill_ms, "decode_proj": dproj_ms,
+                      "decode_pre": dpre_ms, "decode_attn": dattn_ms},
+        "prefill": {"tokens_per_s": w.B * w.S / (prefill_ms / 1e3) * world,
+                    "tflops_attn_plus_proj": (attn_flop + proj_flop) / (prefill_ms / 1e3) / 1e12,
+                    "proj_tflops": proj_flop / (proj_ms / 1e3) / 1e12},
+        "decode": {"kv_bytes": kv_bytes, "attn_gbs": kv_bytes / (dattn_ms / 1e-3) / 1e9 * 1e-6 * 1e6
+                   if dattn_ms > 0 else None,
+                   "step_ms": dproj_ms + dpre_ms + dattn_ms,
+                   "hbm_frac_attn": (kv_bytes / (dattn_ms / 1e3) / 1e9) / peaks["hbm_gbs"]},
+        "clocks": sampler.summary(),
+        "e2e": {"value": tokens_per_step * K * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "cpu_baseline": cpu,
+    }
+    line["decode"]["attn_gbs"] = kv_bytes / (dattn_ms / 1e3) / 1e9 if dattn_ms > 0 else None
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

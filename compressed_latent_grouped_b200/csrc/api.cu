@@ -1,0 +1,365 @@
+// C ABI of the CCGQA hot path: host-side validation, workspace layout and
+// kernel dispatch.  Every entry point validates all arguments before the first
+// launch and returns a status; the kernels themselves never trap.
+#include <atomic>
+#include <cmath>
+
+#include "kernels.h"
+
+namespace ccgqa {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+
+// Optional phase events of the calling thread (ccgqa_set_phase_events).
+static thread_local void* const* t_phase_events = nullptr;
+static void phase_mark(int i, cudaStream_t st) {
+  if (t_phase_events) cudaEventRecord(static_cast<cudaEvent_t>(t_phase_events[i]), st);
+}
+
+namespace {
+
+struct Geo {
+  int E, C, Hq, Hkv, d, G, N, K;
+  int qk_mean, value_shift, causal, rope_on;
+  double rope_log2_base;
+  int dtype;
+  size_t es;  // element size
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+ccgqa_status derive(const ccgqa_config* cfg, Geo* g) {
+  if (!cfg) return CCGQA_ERR_INVALID_ARG;
+  if (cfg->E <= 0 || cfg->C <= 0 || cfg->n_q_heads <= 0 || cfg->n_kv_heads <= 0)
+    return CCGQA_ERR_INVALID_ARG;
+  if (cfg->n_q_heads % cfg->n_kv_heads != 0) return CCGQA_ERR_INVALID_ARG;
+  if (cfg->E % (cfg->C * cfg->n_q_heads) != 0) return CCGQA_ERR_INVALID_ARG;
+  if (cfg->conv_width < 0 || cfg->conv_width > 4) return CCGQA_ERR_INVALID_ARG;
+  if ((cfg->qk_mean | cfg->value_shift | cfg->causal) & ~1) return CCGQA_ERR_INVALID_ARG;
+  if (!(cfg->rope_base >= 0.0) || std::isinf(cfg->rope_base)) return CCGQA_ERR_INVALID_ARG;
+  if (cfg->dtype != CCGQA_F32 && cfg->dtype != CCGQA_BF16) return CCGQA_ERR_INVALID_ARG;
+  g->E = cfg->E;
+  g->C = cfg->C;
+  g->Hq = cfg->n_q_heads;
+  g->Hkv = cfg->n_kv_heads;
+  g->d = cfg->E / (cfg->C * cfg->n_q_heads);
+  g->G = g->Hq / g->Hkv;
+  g->N = (g->Hq + 2 * g->Hkv) * g->d;
+  g->K = cfg->conv_width;
+  g->qk_mean = cfg->qk_mean;
+  g->value_shift = cfg->value_shift;
+  g->causal = cfg->causal;
+  g->rope_on = cfg->rope_base > 0.0;
+  g->rope_log2_base = g->rope_on ? std::log2(cfg->rope_base) : 0.0;
+  g->dtype = cfg->dtype;
+  g->es = cfg->dtype == CCGQA_F32 ? 4 : 2;
+  if (g->d != 16 && g->d != 32 && g->d != 64 && g->d != 128) return CCGQA_ERR_UNSUPPORTED;
+  if (g->dtype == CCGQA_BF16 && (g->d < 32 || !pow2(g->G) || g->G > 128))
+    return CCGQA_ERR_UNSUPPORTED;
+  if (g->G * (g->d * static_cast<int>(g->es) / 16) > 128) return CCGQA_ERR_UNSUPPORTED;
+  return CCGQA_OK;
+}
+
+ccgqa_status check_weights(const Geo& g, const ccgqa_weights* w) {
+  if (!w) return CCGQA_ERR_INVALID_ARG;
+  if (w->W_qkv && !aligned16(w->W_qkv)) return CCGQA_ERR_INVALID_ARG;
+  if (g.K > 0) {
+    if (!w->conv_q_seq || !w->conv_k_seq) return CCGQA_ERR_INVALID_ARG;
+    if (!aligned16(w->conv_q_seq) || !aligned16(w->conv_k_seq)) return CCGQA_ERR_INVALID_ARG;
+    if ((w->conv_q_chan && !aligned16(w->conv_q_chan)) ||
+        (w->conv_k_chan && !aligned16(w->conv_k_chan)))
+      return CCGQA_ERR_INVALID_ARG;
+  }
+  return CCGQA_OK;
+}
+
+ccgqa_status check_cache(const Geo& g, const ccgqa_kvcache* c, bool need_state) {
+  if (!c) return CCGQA_ERR_INVALID_ARG;
+  if (c->batch <= 0 || c->cap <= 0) return CCGQA_ERR_INVALID_ARG;
+  if (!c->k || !c->v || !c->len || !aligned16(c->k) || !aligned16(c->v))
+    return CCGQA_ERR_INVALID_ARG;
+  if (need_state) {
+    if (g.K > 1 && (!c->conv_hist_q || !c->conv_hist_k)) return CCGQA_ERR_INVALID_ARG;
+    if (g.value_shift && !c->v_prev) return CCGQA_ERR_INVALID_ARG;
+  }
+  return CCGQA_OK;
+}
+
+struct PrefillWs {
+  size_t proj, q, k, v, total;
+};
+PrefillWs prefill_ws(const Geo& g, int64_t B, int64_t S) {
+  PrefillWs w;
+  size_t off = 0;
+  w.proj = off;
+  off += up256(static_cast<size_t>(B * S) * g.N * g.es);
+  w.q = off;
+  off += up256(static_cast<size_t>(B * S) * g.Hq * g.d * g.es);
+  w.k = off;
+  off += up256(static_cast<size_t>(B * S) * g.Hkv * g.d * g.es);
+  w.v = off;
+  off += up256(static_cast<size_t>(B * S) * g.Hkv * g.d * g.es);
+  w.total = off;
+  return w;
+}
+
+struct DecodeWs {
+  size_t proj, q, po, pml, tick, total;
+  int e_splits, splits, chunk;
+};
+DecodeWs decode_ws(const Geo& g, int64_t B, int64_t cap, bool has_proj) {
+  DecodeWs w;
+  decode_plan(static_cast<int>(B), g.Hkv, g.E, g.N, cap, has_proj, &w.e_splits, &w.splits,
+              &w.chunk);
+  size_t off = 0;
+  w.tick = off;  // tickets first: the part a fresh zero-fill must cover
+  off += up256(static_cast<size_t>(B * g.Hkv + B) * 4);
+  w.proj = off;
+  off += up256(static_cast<size_t>(w.e_splits) * B * g.N * 4);
+  w.q = off;
+  off += up256(static_cast<size_t>(B) * g.Hq * g.d * 4);
+  w.po = off;
+  off += up256(static_cast<size_t>(B) * g.Hkv * w.splits * g.G * g.d * 4);
+  w.pml = off;
+  off += up256(static_cast<size_t>(B) * g.Hkv * w.splits * g.G * 2 * 4);
+  w.total = off;
+  return w;
+}
+
+template <typename T>
+ccgqa_status run_prefill(const Geo& g, const ccgqa_weights* w, const void* x, int B, int S,
+                         void* out, const ccgqa_kvcache* cache, uint8_t* ws, int32_t* dev_err,
+                         cudaStream_t st) {
+  const PrefillWs L = prefill_ws(g, B, S);
+  const T* src = static_cast<const T*>(x);
+  cudaError_t e = cudaSuccess;
+  phase_mark(0, st);
+  if (w->W_qkv) {
+    T* proj = reinterpret_cast<T*>(ws + L.proj);
+    if constexpr (sizeof(T) == 2)
+      e = launch_proj_gemm_bf16(static_cast<const bf16*>(x), static_cast<const bf16*>(w->W_qkv),
+                                proj, B * S, g.N, g.E, dev_err, st);
+    else
+      e = launch_proj_gemm_f32(static_cast<const float*>(x), static_cast<const float*>(w->W_qkv),
+                               proj, B * S, g.N, g.E, st);
+    if (e != cudaSuccess) return CCGQA_ERR_CUDA;
+    src = proj;
+  }
+  phase_mark(1, st);
+  PreAttnArgs<T> a{};
+  a.src = src;
+  a.src_ld = g.N;
+  a.B = B;
+  a.S = S;
+  a.Hq = g.Hq;
+  a.Hkv = g.Hkv;
+  a.d = g.d;
+  a.G = g.G;
+  a.K = g.K;
+  a.qk_mean = g.qk_mean;
+  a.value_shift = g.value_shift;
+  a.rope_on = g.rope_on;
+  a.rope_log2_base = g.rope_log2_base;
+  a.wq_seq = static_cast<const T*>(w->conv_q_seq);
+  a.wq_chan = static_cast<const T*>(w->conv_q_chan);
+  a.wk_seq = static_cast<const T*>(w->conv_k_seq);
+  a.wk_chan = static_cast<const T*>(w->conv_k_chan);
+  a.q_out = reinterpret_cast<T*>(ws + L.q);
+  if (cache) {
+    a.k_out = static_cast<T*>(cache->k);
+    a.v_out = static_cast<T*>(cache->v);
+    a.kv_cap = cache->cap;
+    a.hist_q = static_cast<T*>(cache->conv_hist_q);
+    a.hist_k = static_cast<T*>(cache->conv_hist_k);
+    a.v_prev = static_cast<T*>(cache->v_prev);
+    a.len = cache->len;
+  } else {
+    a.k_out = reinterpret_cast<T*>(ws + L.k);
+    a.v_out = reinterpret_cast<T*>(ws + L.v);
+    a.kv_cap = S;
+  }
+  a.dev_err = dev_err;
+  if (launch_pre_attn<T>(a, st) != cudaSuccess) return CCGQA_ERR_CUDA;
+  phase_mark(2, st);
+  AttnArgs at{};
+  at.q = a.q_out;
+  at.k = a.k_out;
+  at.v = a.v_out;
+  at.out = out;
+  at.B = B;
+  at.S = S;
+  at.Hq = g.Hq;
+  at.Hkv = g.Hkv;
+  at.d = g.d;
+  at.G = g.G;
+  at.kv_cap = a.kv_cap;
+  at.causal = g.causal;
+  at.dev_err = dev_err;
+  if constexpr (sizeof(T) == 2)
+    e = launch_attn_prefill_tc(at, st);
+  else
+    e = launch_attn_prefill_simt<T>(at, st);
+  phase_mark(3, st);
+  return e == cudaSuccess ? CCGQA_OK : CCGQA_ERR_CUDA;
+}
+
+template <typename T>
+ccgqa_status run_decode(const Geo& g, const ccgqa_weights* w, const void* x_t,
+                        const ccgqa_kvcache* c, void* out, uint8_t* ws, int32_t* dev_err,
+                        cudaStream_t st) {
+  const DecodeWs L = decode_ws(g, c->batch, c->cap, w->W_qkv != nullptr);
+  DecodeArgs<T> a{};
+  a.x_t = static_cast<const T*>(x_t);
+  a.W = static_cast<const T*>(w->W_qkv);
+  a.B = c->batch;
+  a.E = g.E;
+  a.N = g.N;
+  a.Hq = g.Hq;
+  a.Hkv = g.Hkv;
+  a.d = g.d;
+  a.G = g.G;
+  a.K = g.K;
+  a.qk_mean = g.qk_mean;
+  a.value_shift = g.value_shift;
+  a.causal = g.causal;
+  a.rope_on = g.rope_on;
+  a.rope_log2_base = g.rope_log2_base;
+  a.wq_seq = static_cast<const T*>(w->conv_q_seq);
+  a.wq_chan = static_cast<const T*>(w->conv_q_chan);
+  a.wk_seq = static_cast<const T*>(w->conv_k_seq);
+  a.wk_chan = static_cast<const T*>(w->conv_k_chan);
+  a.cache_k = static_cast<T*>(c->k);
+  a.cache_v = static_cast<T*>(c->v);
+  a.len = c->len;
+  a.cap = c->cap;
+  a.hist_q = static_cast<T*>(c->conv_hist_q);
+  a.hist_k = static_cast<T*>(c->conv_hist_k);
+  a.v_prev = static_cast<T*>(c->v_prev);
+  a.out = static_cast<T*>(out);
+  a.proj_part = reinterpret_cast<float*>(ws + L.proj);
+  a.e_splits = L.e_splits;
+  a.q_ws = reinterpret_cast<float*>(ws + L.q);
+  a.part_o = reinterpret_cast<float*>(ws + L.po);
+  a.part_ml = reinterpret_cast<float*>(ws + L.pml);
+  a.tickets = reinterpret_cast<int32_t*>(ws + L.tick);
+  a.splits = L.splits;
+  a.chunk = L.chunk;
+  a.dev_err = dev_err;
+  a.phase_events = t_phase_events;
+  return launch_decode_step<T>(a, st) == cudaSuccess ? CCGQA_OK : CCGQA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace ccgqa
+
+using namespace ccgqa;
+
+extern "C" {
+
+CCGQA_API size_t ccgqa_prefill_workspace_size(const ccgqa_config* cfg, int32_t batch,
+                                              int32_t seq_len) {
+  Geo g;
+  if (derive(cfg, &g) != CCGQA_OK || batch <= 0 || seq_len <= 0) return 0;
+  return prefill_ws(g, batch, seq_len).total;
+}
+
+CCGQA_API size_t ccgqa_decode_workspace_size(const ccgqa_config* cfg, int32_t batch,
+                                             int32_t cap) {
+  Geo g;
+  if (derive(cfg, &g) != CCGQA_OK || batch <= 0 || cap <= 0) return 0;
+  return decode_ws(g, batch, cap, true).total;
+}
+
+CCGQA_API ccgqa_status ccgqa_prefill(const ccgqa_config* cfg, const ccgqa_weights* w,
+                                     const void* x, int32_t batch, int32_t seq_len, void* out,
+                                     const ccgqa_kvcache* cache, void* workspace,
+                                     size_t workspace_bytes, int32_t* dev_err, void* stream) {
+  Geo g;
+  ccgqa_status s = derive(cfg, &g);
+  if (s != CCGQA_OK) return s;
+  if ((s = check_weights(g, w)) != CCGQA_OK) return s;
+  if (batch <= 0 || seq_len <= 0) return CCGQA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(batch) * seq_len > (int64_t(1) << 30)) return CCGQA_ERR_UNSUPPORTED;
+  if (!x || !out || !aligned16(x) || !aligned16(out)) return CCGQA_ERR_INVALID_ARG;
+  if (cache) {
+    if ((s = check_cache(g, cache, true)) != CCGQA_OK) return s;
+    if (cache->batch != batch) return CCGQA_ERR_INVALID_ARG;
+    if (seq_len > cache->cap) return CCGQA_ERR_CAPACITY;
+  }
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) ||
+      workspace_bytes < prefill_ws(g, batch, seq_len).total)
+    return CCGQA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (g.dtype == CCGQA_BF16)
+    return run_prefill<bf16>(g, w, x, batch, seq_len, out, cache, ws, dev_err, st);
+  return run_prefill<float>(g, w, x, batch, seq_len, out, cache, ws, dev_err, st);
+}
+
+CCGQA_API ccgqa_status ccgqa_decode_step(const ccgqa_config* cfg, const ccgqa_weights* w,
+                                         const void* x_t, const ccgqa_kvcache* cache, void* out,
+                                         void* workspace, size_t workspace_bytes,
+                                         int32_t* dev_err, void* stream) {
+  Geo g;
+  ccgqa_status s = derive(cfg, &g);
+  if (s != CCGQA_OK) return s;
+  if ((s = check_weights(g, w)) != CCGQA_OK) return s;
+  if ((s = check_cache(g, cache, true)) != CCGQA_OK) return s;
+  if (!x_t || !out || !aligned16(x_t) || !aligned16(out)) return CCGQA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) ||
+      workspace_bytes < decode_ws(g, cache->batch, cache->cap, w->W_qkv != nullptr).total)
+    return CCGQA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (g.dtype == CCGQA_BF16) return run_decode<bf16>(g, w, x_t, cache, out, ws, dev_err, st);
+  return run_decode<float>(g, w, x_t, cache, out, ws, dev_err, st);
+}
+
+CCGQA_API ccgqa_status ccgqa_kvcache_append(const ccgqa_config* cfg, const ccgqa_kvcache* cache,
+                                            const void* k_new, const void* v_new, int32_t n_new,
+                                            int32_t* dev_err, void* stream) {
+  Geo g;
+  ccgqa_status s = derive(cfg, &g);
+  if (s != CCGQA_OK) return s;
+  if ((s = check_cache(g, cache, false)) != CCGQA_OK) return s;
+  if (n_new < 0) return CCGQA_ERR_INVALID_ARG;
+  if (n_new > cache->cap) return CCGQA_ERR_CAPACITY;
+  if (n_new == 0) return CCGQA_OK;
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return CCGQA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (g.dtype == CCGQA_BF16)
+    e = launch_kv_append<bf16>(static_cast<bf16*>(cache->k), static_cast<bf16*>(cache->v),
+                               cache->len, static_cast<const bf16*>(k_new),
+                               static_cast<const bf16*>(v_new), cache->batch, g.Hkv, g.d,
+                               cache->cap, n_new, dev_err, st);
+  else
+    e = launch_kv_append<float>(static_cast<float*>(cache->k), static_cast<float*>(cache->v),
+                                cache->len, static_cast<const float*>(k_new),
+                                static_cast<const float*>(v_new), cache->batch, g.Hkv, g.d,
+                                cache->cap, n_new, dev_err, st);
+  return e == cudaSuccess ? CCGQA_OK : CCGQA_ERR_CUDA;
+}
+
+CCGQA_API const char* ccgqa_status_string(ccgqa_status s) {
+  switch (s) {
+    case CCGQA_OK: return "ok";
+    case CCGQA_ERR_INVALID_ARG: return "invalid argument";
+    case CCGQA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case CCGQA_ERR_CAPACITY: return "tokens exceed the cache capacity";
+    case CCGQA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case CCGQA_ERR_CUDA: return "CUDA launch or runtime error";
+  }
+  return "unknown status";
+}
+
+CCGQA_API uint64_t ccgqa_launch_count(void) { return g_launches.load(); }
+
+CCGQA_API void ccgqa_set_phase_events(void* const* events, int32_t n) {
+  t_phase_events = (events != nullptr && n >= 4) ? events : nullptr;
+}
+
+}  // extern "C"

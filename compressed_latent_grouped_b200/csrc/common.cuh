@@ -1,0 +1,33 @@
+// Shared device/host helpers for the CCGQA kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/ccgqa.h"
+
+namespace ccgqa {
+
+// Element conversions used by every templated kernel.
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+// OR an error bit into the caller's device status word (nullable).
+__device__ __forceinline__ void raise_dev_err(int32_t* dev_err, int32_t bit) {
+  if (dev_err) atomicOr(dev_err, bit);
+}
+
+// Cycles a bounded in-kernel wait may spin before it gives up (about one
+// second at the B200's clock).  A healthy wait ends in microseconds.
+constexpr long long kWaitLimitCycles = 2000000000LL;
+
+// Host-side launch accounting (ccgqa_launch_count).
+void count_launches(int n);
+
+}  // namespace ccgqa

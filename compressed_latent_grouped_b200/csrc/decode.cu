@@ -1,0 +1,567 @@
+// Decode path: one new token per sequence against the latent KV cache
+// ("Compressed Convolutional Attention", Probleemstelling 2: the KV cache grows
+// with the sequence and decode is bound by reading it; Resultaten 3: the cache
+// shrinks with C.  "Grouped Query Attention (GQA)", "Por qué GQA reduce la
+// caché KV": decode speed is set by memory bandwidth).
+//
+//   kv_append        bit-exact copy of new rows into the cache at len[b]
+//   decode_proj      x_t W^T for all sequences, split over E (fp32 partials)
+//   decode_pre       one-token conv from the stored history, channel mix,
+//                    QK-mean, RoPE at position len[b], value-shift from the
+//                    stored previous row, cache append, state update
+//   decode_attn      split-K attention over len[b] + 1 keys: each CTA streams
+//                    one chunk of K and V of one kv group with bulk copies
+//                    through a shared-memory ring; every K/V row read serves
+//                    all G query heads.  The last CTA of a (sequence, group)
+//                    -- found with an atomic ticket, never by waiting --
+//                    merges the chunks; the last group of a sequence bumps len.
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace ccgqa {
+
+// ----------------------------------------------------------------- split plan
+void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int* e_splits,
+                 int* splits, int* chunk) {
+  const int target = 2 * 148;
+  if (has_proj) {
+    const int tiles = ((N + 127) / 128) * ((B + 63) / 64);
+    int es = target / (tiles > 0 ? tiles : 1);
+    const int max_es = (E + 255) / 256;
+    if (es > max_es) es = max_es;
+    if (es < 1) es = 1;
+    *e_splits = es;
+  } else {
+    *e_splits = 0;
+  }
+  const int64_t bh = static_cast<int64_t>(B) * Hkv;
+  int64_t sp = (cap + 511) / 512;
+  if (bh * sp < target) {
+    const int64_t want = (target + bh - 1) / bh;
+    const int64_t maxsp = (cap + 63) / 64;
+    sp = want < maxsp ? want : maxsp;
+  }
+  if (sp < 1) sp = 1;
+  int64_t ch = (cap + sp - 1) / sp;
+  ch = (ch + 63) / 64 * 64;
+  *chunk = static_cast<int>(ch);
+  *splits = static_cast<int>((cap + ch - 1) / ch);
+}
+
+namespace {
+
+using namespace sm100;
+
+// ----------------------------------------------------------------- kv append
+template <typename T>
+__global__ void kv_append_kernel(T* __restrict__ ck, T* __restrict__ cv, const int32_t* len,
+                                 const T* __restrict__ kn, const T* __restrict__ vn, int Hkv,
+                                 int d, int64_t cap, int n_new, int32_t* dev_err) {
+  constexpr int VEC = 16 / sizeof(T);
+  const int b = blockIdx.y;
+  const int L = len[b];
+  if (L < 0 || static_cast<int64_t>(L) + n_new > cap) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) raise_dev_err(dev_err, CCGQA_DEVERR_CAPACITY);
+    return;
+  }
+  const int nch = d / VEC;
+  const int64_t total = static_cast<int64_t>(n_new) * Hkv * nch;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(idx % nch);
+    const int64_t rg = idx / nch;
+    const int g = static_cast<int>(rg % Hkv);
+    const int64_t i = rg / Hkv;
+    const int64_t src = ((static_cast<int64_t>(b) * n_new + i) * Hkv + g) * d + c * VEC;
+    const int64_t dst = ((static_cast<int64_t>(b) * Hkv + g) * cap + L + i) * d + c * VEC;
+    *reinterpret_cast<uint4*>(ck + dst) = *reinterpret_cast<const uint4*>(kn + src);
+    *reinterpret_cast<uint4*>(cv + dst) = *reinterpret_cast<const uint4*>(vn + src);
+  }
+}
+
+__global__ void len_add_kernel(int32_t* len, int B, int64_t cap, int n_new) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B && len[b] >= 0 && static_cast<int64_t>(len[b]) + n_new <= cap) len[b] += n_new;
+}
+
+// ----------------------------------------------------------------- projection
+constexpr int kPB = 64, kPN = 128, kPE = 32;
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+    decode_proj_kernel(const T* __restrict__ x, const T* __restrict__ W, float* __restrict__ part,
+                       int B, int E, int N, int e_len) {
+  __shared__ __align__(16) float xs[kPE][kPB + 4];
+  __shared__ __align__(16) float wsm[kPE][kPN + 4];
+  const int n0 = blockIdx.x * kPN, sp = blockIdx.y, b0 = blockIdx.z * kPB;
+  const int e_lo = sp * e_len, e_hi = min(E, e_lo + e_len);
+  const int tb = threadIdx.x / 16, tn = threadIdx.x % 16;
+  float acc[4][8] = {};
+  for (int e0 = e_lo; e0 < e_hi; e0 += kPE) {
+    for (int idx = threadIdx.x; idx < kPB * kPE; idx += 256) {
+      const int r = idx / kPE, c = idx % kPE;
+      const int gb = b0 + r, ge = e0 + c;
+      xs[c][r] = (gb < B && ge < e_hi) ? to_f32(x[static_cast<int64_t>(gb) * E + ge]) : 0.f;
+    }
+    for (int idx = threadIdx.x; idx < kPN * kPE; idx += 256) {
+      const int r = idx / kPE, c = idx % kPE;
+      const int gn = n0 + r, ge = e0 + c;
+      wsm[c][r] = (gn < N && ge < e_hi) ? to_f32(W[static_cast<int64_t>(gn) * E + ge]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int e = 0; e < kPE; ++e) {
+      const float4 xv = *reinterpret_cast<const float4*>(&xs[e][tb * 4]);
+      const float4 w0 = *reinterpret_cast<const float4*>(&wsm[e][tn * 8]);
+      const float4 w1 = *reinterpret_cast<const float4*>(&wsm[e][tn * 8 + 4]);
+      const float xr[4] = {xv.x, xv.y, xv.z, xv.w};
+      const float wr[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(xr[i], wr[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int gb = b0 + tb * 4 + i;
+    if (gb >= B) continue;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int gn = n0 + tn * 8 + j;
+      if (gn < N) part[(static_cast<int64_t>(sp) * B + gb) * N + gn] = acc[i][j];
+    }
+  }
+}
+
+// ----------------------------------------------------------------- pre-step
+template <typename T>
+__global__ void __launch_bounds__(128) decode_pre_kernel(const DecodeArgs<T> a) {
+  extern __shared__ float4 dsm_f4[];
+  float* sm = reinterpret_cast<float*>(dsm_f4);
+  const int g = blockIdx.x, b = blockIdx.y;
+  const int d = a.d, G = a.G, K = a.K, half = d / 2;
+  const int KH = K > 0 ? K - 1 : 0;
+  const int QC = G * d, HC = QC + d, AC = HC + d;  // q | k | v channels of the group
+  float* zc = sm;                 // [AC] current pre-conv row
+  float* hz = zc + AC;            // [KH][HC] history
+  float* u = hz + KH * HC;        // [HC]
+  float* y = u + HC;              // [HC]
+  const int tid = threadIdx.x;
+  const int L = __ldcg(a.len + b);
+  if (L < 0 || L >= a.cap) {
+    if (g == 0 && tid == 0) raise_dev_err(a.dev_err, CCGQA_DEVERR_CAPACITY);
+    return;
+  }
+  const int qcol0 = g * G * d, kcol0 = a.Hq * d + g * d, vcol0 = (a.Hq + a.Hkv) * d + g * d;
+  for (int c = tid; c < AC; c += blockDim.x) {
+    const int col = c < QC ? qcol0 + c : (c < HC ? kcol0 + (c - QC) : vcol0 + (c - HC));
+    float val;
+    if (a.W) {
+      val = 0.f;
+      for (int s = 0; s < a.e_splits; ++s)
+        val += a.proj_part[(static_cast<int64_t>(s) * a.B + b) * a.N + col];
+      val = to_f32(from_f32<T>(val));  // the projection output is held in the working dtype
+    } else {
+      val = to_f32(a.x_t[static_cast<int64_t>(b) * a.N + col]);
+    }
+    zc[c] = val;
+  }
+  for (int idx = tid; idx < KH * HC; idx += blockDim.x) {
+    const int r = idx / HC, c = idx - r * HC;
+    hz[idx] = c < QC ? to_f32(a.hist_q[(static_cast<int64_t>(b) * KH + r) * a.Hq * d + qcol0 + c])
+                     : to_f32(a.hist_k[(static_cast<int64_t>(b) * KH + r) * a.Hkv * d + g * d +
+                                       (c - QC)]);
+  }
+  __syncthreads();
+  // causal conv: tap j reads the row j steps back (history row KH - j)
+  for (int c = tid; c < HC; c += blockDim.x) {
+    float acc;
+    if (K > 0) {
+      const bool is_q = c < QC;
+      const T* w = is_q ? a.wq_seq + static_cast<int64_t>(qcol0 + c) * K
+                        : a.wk_seq + static_cast<int64_t>(g * d + (c - QC)) * K;
+      acc = to_f32(w[0]) * zc[c];
+      for (int j = 1; j < K; ++j) acc = fmaf(to_f32(w[j]), hz[(KH - j) * HC + c], acc);
+    } else {
+      acc = zc[c];
+    }
+    u[c] = acc;
+  }
+  __syncthreads();
+  // channel mix + QK-mean
+  for (int c = tid; c < HC; c += blockDim.x) {
+    const bool is_q = c < QC;
+    const int hh = c / d, i = c - hh * d;
+    const T* wch = is_q ? a.wq_chan : a.wk_chan;
+    float acc;
+    if (K > 0 && wch) {
+      const int head = is_q ? g * G + hh : g;
+      const T* wr = wch + (static_cast<int64_t>(head) * d + i) * d;
+      acc = 0.f;
+      for (int j = 0; j < d; ++j) acc = fmaf(to_f32(wr[j]), u[hh * d + j], acc);
+    } else {
+      acc = u[c];
+    }
+    if (a.qk_mean) {
+      float qp;
+      if (is_q) {
+        qp = zc[c];
+      } else {
+        qp = 0.f;
+        for (int hl = 0; hl < G; ++hl) qp += zc[hl * d + i];
+        qp /= static_cast<float>(G);
+      }
+      acc += 0.5f * (qp + zc[QC + i]);
+    }
+    y[c] = acc;
+  }
+  __syncthreads();
+  // RoPE at position L on (i, i + d/2), then q -> workspace, k -> cache row L
+  const int64_t crow = ((static_cast<int64_t>(b) * a.Hkv + g) * a.cap + L) * d;
+  for (int idx = tid; idx < (G + 1) * half; idx += blockDim.x) {
+    const int hh = idx / half, i = idx - hh * half;
+    float ya = y[hh * d + i], yb = y[hh * d + i + half];
+    if (a.rope_on) {
+      const double th = exp2(-(2.0 * i / d) * a.rope_log2_base);
+      double f = static_cast<double>(L) * th * 0.15915494309189533577;
+      f -= rint(f);
+      float s, c;
+      sincospif(static_cast<float>(2.0 * f), &s, &c);
+      const float na = ya * c - yb * s, nb = ya * s + yb * c;
+      ya = na;
+      yb = nb;
+    }
+    if (hh < G) {
+      float* qd = a.q_ws + (static_cast<int64_t>(b) * a.Hq + g * G + hh) * d;
+      qd[i] = ya;
+      qd[i + half] = yb;
+    } else {
+      a.cache_k[crow + i] = from_f32<T>(ya);
+      a.cache_k[crow + i + half] = from_f32<T>(yb);
+    }
+  }
+  for (int i = tid; i < d; i += blockDim.x) {
+    T v = from_f32<T>(zc[HC + i]);
+    if (a.value_shift && i >= half) v = a.v_prev[static_cast<int64_t>(b) * a.Hkv * d + g * d + i];
+    a.cache_v[crow + i] = v;
+  }
+  __syncthreads();
+  // state: histories shift by one row, v_prev = this row's v~
+  for (int idx = tid; idx < KH * HC; idx += blockDim.x) {
+    const int r = idx / HC, c = idx - r * HC;
+    const float val = (r + 1 < KH) ? hz[(r + 1) * HC + c] : zc[c];
+    if (c < QC)
+      a.hist_q[(static_cast<int64_t>(b) * KH + r) * a.Hq * d + qcol0 + c] = from_f32<T>(val);
+    else
+      a.hist_k[(static_cast<int64_t>(b) * KH + r) * a.Hkv * d + g * d + (c - QC)] = from_f32<T>(val);
+  }
+  if (a.v_prev) {
+    for (int i = tid; i < d; i += blockDim.x)
+      a.v_prev[static_cast<int64_t>(b) * a.Hkv * d + g * d + i] = from_f32<T>(zc[HC + i]);
+  }
+}
+
+// ----------------------------------------------------------------- attention
+constexpr int kDecThreads = 128, kDecStages = 4, kPPMax = 4;
+
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <typename T, int D>
+struct DecCfg {
+  static constexpr int CH = 16 / sizeof(T);  // elements per 16-byte chunk
+  static constexpr int NCH = D / CH;         // chunks per row
+  static constexpr int KS_raw = 8192 / (D * static_cast<int>(sizeof(T)));
+  static constexpr int KS = KS_raw > 64 ? 64 : (KS_raw < 16 ? 16 : KS_raw);  // keys per stage
+  static constexpr int KW = KS / 4;          // keys per warp per stage
+  static constexpr uint32_t kStageBytes = 2u * KS * D * sizeof(T);
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kDecThreads)
+    decode_attn_kernel(const DecodeArgs<T> a) {
+  using C = DecCfg<T, D>;
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dsm_raw) + 127) & ~uintptr_t(127));
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + kDecStages * C::kStageBytes);
+  float* wbuf = reinterpret_cast<float*>(full + kDecStages);  // merge scratch
+  __shared__ int abort_flag, last_flag;
+
+  const int sp = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int G = a.G, P = G * C::NCH;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const int L = __ldcg(a.len + b);
+  const bool valid_b = L >= 0 && L < a.cap;
+  const int n_keys = valid_b ? L + 1 : 0;
+  const int k0 = sp * a.chunk;
+  const int k1 = min(k0 + a.chunk, n_keys);
+  const int nk = max(0, k1 - k0);
+  const int n_st = (nk + C::KS - 1) / C::KS;
+  const int64_t kv_base = (static_cast<int64_t>(b) * a.Hkv + g) * a.cap * D;
+
+  if (tid == 0) {
+    for (int s = 0; s < kDecStages; ++s) mbar_init(&full[s], 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  auto issue = [&](int st_idx) {
+    const int s = st_idx % kDecStages;
+    const int key0 = k0 + st_idx * C::KS;
+    const int rows = min(C::KS, k1 - key0);
+    const uint32_t bytes = static_cast<uint32_t>(rows) * D * sizeof(T);
+    uint8_t* dst = ring + s * C::kStageBytes;
+    mbar_arrive_expect_tx(&full[s], 2 * bytes);
+    bulk_load(dst, a.cache_k + kv_base + static_cast<int64_t>(key0) * D, bytes, &full[s]);
+    bulk_load(dst + C::kStageBytes / 2, a.cache_v + kv_base + static_cast<int64_t>(key0) * D, bytes,
+              &full[s]);
+  };
+  if (tid == 0)
+    for (int i = 0; i < kDecStages && i < n_st; ++i) issue(i);
+
+  // per-lane pairs: pair p = lane + 32 kk -> head p / NCH, chunk p % NCH
+  const float scale = 1.4426950408889634f * rsqrtf(static_cast<float>(D));
+  float qr[kPPMax][C::CH], o[kPPMax][C::CH], m[kPPMax], l[kPPMax];
+  const int chunk = lane % C::NCH;
+#pragma unroll
+  for (int kk = 0; kk < kPPMax; ++kk) {
+    const int p = lane + 32 * kk;
+    const int h = p / C::NCH;
+    m[kk] = -INFINITY;
+    l[kk] = 0.f;
+#pragma unroll
+    for (int e = 0; e < C::CH; ++e) {
+      o[kk][e] = 0.f;
+      qr[kk][e] = (p < P) ? a.q_ws[(static_cast<int64_t>(b) * a.Hq + g * G + h) * D +
+                                   chunk * C::CH + e] *
+                                scale
+                          : 0.f;
+    }
+  }
+  const int PP = (P + 31) / 32;
+
+  for (int it = 0; it < n_st; ++it) {
+    const int s = it % kDecStages;
+    if (!mbar_wait(&full[s], (it / kDecStages) & 1, &abort_flag, a.dev_err)) break;
+    const T* Ks = reinterpret_cast<const T*>(ring + s * C::kStageBytes);
+    const T* Vs = reinterpret_cast<const T*>(ring + s * C::kStageBytes + C::kStageBytes / 2);
+    const int key_base = k0 + it * C::KS;
+    const int rows = min(C::KS, k1 - key_base);
+    const int c_lo = warp * C::KW;
+    float sc[kPPMax][C::KW];
+#pragma unroll
+    for (int c = 0; c < C::KW; ++c) {
+      const int kr = c_lo + c;
+      const bool kv = kr < rows;
+      uint4 kraw = kv ? *reinterpret_cast<const uint4*>(Ks + kr * D + chunk * C::CH)
+                      : make_uint4(0, 0, 0, 0);
+      const T* ke = reinterpret_cast<const T*>(&kraw);
+#pragma unroll
+      for (int kk = 0; kk < kPPMax; ++kk) {
+        if (kk >= PP) break;
+        float part = 0.f;
+#pragma unroll
+        for (int e = 0; e < C::CH; ++e) part = fmaf(qr[kk][e], to_f32(ke[e]), part);
+#pragma unroll
+        for (int off = 1; off < C::NCH; off <<= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+        sc[kk][c] = kv ? part : -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int kk = 0; kk < kPPMax; ++kk) {
+      if (kk >= PP) break;
+      float mx = m[kk];
+#pragma unroll
+      for (int c = 0; c < C::KW; ++c) mx = fmaxf(mx, sc[kk][c]);
+      if (mx == -INFINITY) continue;
+      const float corr = ex2f(m[kk] - mx);
+      l[kk] *= corr;
+#pragma unroll
+      for (int e = 0; e < C::CH; ++e) o[kk][e] *= corr;
+      m[kk] = mx;
+#pragma unroll
+      for (int c = 0; c < C::KW; ++c) {
+        const int kr = c_lo + c;
+        if (kr >= rows) break;
+        const float pr = ex2f(sc[kk][c] - mx);
+        l[kk] += pr;
+        const uint4 vraw = *reinterpret_cast<const uint4*>(Vs + kr * D + chunk * C::CH);
+        const T* ve = reinterpret_cast<const T*>(&vraw);
+#pragma unroll
+        for (int e = 0; e < C::CH; ++e) o[kk][e] = fmaf(pr, to_f32(ve[e]), o[kk][e]);
+      }
+    }
+    __syncthreads();  // every warp is done with stage s
+    if (tid == 0 && it + kDecStages < n_st) issue(it + kDecStages);
+  }
+
+  // merge the four warps: wbuf[warp][p] = (m, l), then o
+  float* wm = wbuf;                       // [4][P]
+  float* wl = wm + 4 * P;                 // [4][P]
+  float* wo = wl + 4 * P;                 // [4][P][CH]
+#pragma unroll
+  for (int kk = 0; kk < kPPMax; ++kk) {
+    const int p = lane + 32 * kk;
+    if (kk >= PP || p >= P) break;
+    wm[warp * P + p] = m[kk];
+    wl[warp * P + p] = l[kk];
+#pragma unroll
+    for (int e = 0; e < C::CH; ++e) wo[(warp * P + p) * C::CH + e] = o[kk][e];
+  }
+  __syncthreads();
+  const int64_t pbase = ((static_cast<int64_t>(b) * a.Hkv + g) * a.splits + sp) * G;
+  for (int p = tid; p < P; p += kDecThreads) {
+    float M = -INFINITY;
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, wm[w * P + p]);
+    float lsum = 0.f, oacc[C::CH];
+#pragma unroll
+    for (int e = 0; e < C::CH; ++e) oacc[e] = 0.f;
+    for (int w = 0; w < 4; ++w) {
+      const float f = (M == -INFINITY) ? 0.f : ex2f(wm[w * P + p] - M);
+      lsum += wl[w * P + p] * f;
+#pragma unroll
+      for (int e = 0; e < C::CH; ++e) oacc[e] += wo[(w * P + p) * C::CH + e] * f;
+    }
+    const int h = p / C::NCH, ck = p % C::NCH;
+    if (ck == 0) {
+      a.part_ml[(pbase + h) * 2] = M;
+      a.part_ml[(pbase + h) * 2 + 1] = lsum;
+    }
+#pragma unroll
+    for (int e = 0; e < C::CH; ++e) a.part_o[(pbase + h) * D + ck * C::CH + e] = oacc[e];
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int prev = atomicAdd(a.tickets + b * a.Hkv + g, 1);
+    last_flag = (prev == a.splits - 1);
+  }
+  __syncthreads();
+  if (!last_flag) return;
+  __threadfence();
+  // the last CTA of (b, g) merges every split of its G heads
+  const int64_t gbase = (static_cast<int64_t>(b) * a.Hkv + g) * a.splits * G;
+  for (int idx = tid; idx < G * D; idx += kDecThreads) {
+    const int h = idx / D, i = idx - h * D;
+    float M = -INFINITY;
+    for (int s2 = 0; s2 < a.splits; ++s2)
+      M = fmaxf(M, __ldcg(a.part_ml + (gbase + static_cast<int64_t>(s2) * G + h) * 2));
+    float lsum = 0.f, acc = 0.f;
+    for (int s2 = 0; s2 < a.splits; ++s2) {
+      const int64_t pi = gbase + static_cast<int64_t>(s2) * G + h;
+      const float ms = __ldcg(a.part_ml + pi * 2);
+      if (ms == -INFINITY) continue;
+      const float f = ex2f(ms - M);
+      lsum += __ldcg(a.part_ml + pi * 2 + 1) * f;
+      acc += __ldcg(a.part_o + pi * D + i) * f;
+    }
+    const float val = (valid_b && lsum > 0.f) ? acc / lsum : 0.f;
+    a.out[static_cast<int64_t>(b) * a.Hq * D + (g * G + h) * D + i] = from_f32<T>(val);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    a.tickets[b * a.Hkv + g] = 0;
+    __threadfence();
+    const int prev = atomicAdd(a.tickets + a.B * a.Hkv + b, 1);
+    if (prev == a.Hkv - 1) {
+      a.tickets[a.B * a.Hkv + b] = 0;
+      if (valid_b) a.len[b] = L + 1;
+    }
+  }
+}
+
+template <typename T, int D>
+size_t dec_attn_smem(int G) {
+  using C = DecCfg<T, D>;
+  const int P = G * C::NCH;
+  return 128 + kDecStages * C::kStageBytes + kDecStages * 8 +
+         static_cast<size_t>(4 * P * (2 + C::CH)) * 4 + 16;
+}
+
+template <typename T, int D>
+cudaError_t launch_dec_attn(const DecodeArgs<T>& a, cudaStream_t stream) {
+  using C = DecCfg<T, D>;
+  if (a.G * C::NCH > 32 * kPPMax) return cudaErrorInvalidValue;
+  const size_t smem = dec_attn_smem<T, D>(a.G);
+  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<T, D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.splits, a.Hkv, a.B);
+  decode_attn_kernel<T, D><<<grid, kDecThreads, smem, stream>>>(a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+template <typename T>
+cudaError_t launch_kv_append(T* cache_k, T* cache_v, int32_t* len, const T* k_new,
+                             const T* v_new, int B, int Hkv, int d, int64_t cap, int n_new,
+                             int32_t* dev_err, cudaStream_t stream) {
+  const int64_t chunks = static_cast<int64_t>(n_new) * Hkv * (d * sizeof(T) / 16);
+  int64_t blocks = (chunks + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  if (blocks < 1) blocks = 1;
+  dim3 grid(static_cast<unsigned>(blocks), B);
+  kv_append_kernel<T><<<grid, 256, 0, stream>>>(cache_k, cache_v, len, k_new, v_new, Hkv, d, cap,
+                                                n_new, dev_err);
+  len_add_kernel<<<(B + 127) / 128, 128, 0, stream>>>(len, B, cap, n_new);
+  count_launches(2);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_decode_step(const DecodeArgs<T>& a, cudaStream_t stream) {
+  cudaError_t e;
+  auto mark = [&](int i) {
+    if (a.phase_events) cudaEventRecord(static_cast<cudaEvent_t>(a.phase_events[i]), stream);
+  };
+  mark(0);
+  if (a.W) {
+    const int e_len = ((a.E + a.e_splits - 1) / a.e_splits + kPE - 1) / kPE * kPE;
+    dim3 grid((a.N + kPN - 1) / kPN, a.e_splits, (a.B + kPB - 1) / kPB);
+    decode_proj_kernel<T><<<grid, 256, 0, stream>>>(a.x_t, a.W, a.proj_part, a.B, a.E, a.N, e_len);
+    count_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  mark(1);
+  {
+    const int KH = a.K > 0 ? a.K - 1 : 0;
+    const int HC = (a.G + 1) * a.d, AC = HC + a.d;
+    const size_t smem = static_cast<size_t>(AC + KH * HC + 2 * HC) * 4 + 16;
+    if (smem > 48 * 1024) {
+      e = cudaFuncSetAttribute(decode_pre_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+    }
+    decode_pre_kernel<T><<<dim3(a.Hkv, a.B), 128, smem, stream>>>(a);
+    count_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  mark(2);
+  switch (a.d) {
+    case 16: e = launch_dec_attn<T, 16>(a, stream); break;
+    case 32: e = launch_dec_attn<T, 32>(a, stream); break;
+    case 64: e = launch_dec_attn<T, 64>(a, stream); break;
+    case 128: e = launch_dec_attn<T, 128>(a, stream); break;
+    default: e = cudaErrorInvalidValue;
+  }
+  mark(3);
+  return e;
+}
+
+template cudaError_t launch_kv_append<float>(float*, float*, int32_t*, const float*, const float*,
+                                             int, int, int, int64_t, int, int32_t*, cudaStream_t);
+template cudaError_t launch_kv_append<bf16>(bf16*, bf16*, int32_t*, const bf16*, const bf16*, int,
+                                            int, int, int64_t, int, int32_t*, cudaStream_t);
+template cudaError_t launch_decode_step<float>(const DecodeArgs<float>&, cudaStream_t);
+template cudaError_t launch_decode_step<bf16>(const DecodeArgs<bf16>&, cudaStream_t);
+
+}  // namespace ccgqa

@@ -1,0 +1,111 @@
+// Internal launcher declarations shared by the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace ccgqa {
+
+using bf16 = __nv_bfloat16;
+
+// ----------------------------------------------------------------- tensor maps
+// Encode a tiled TMA descriptor through the driver entry point (no libcuda link).
+// dims / box are innermost-first; strides_bytes has rank-1 entries (dims 1..).
+bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base,
+                       const uint64_t* dims, const uint64_t* strides_bytes,
+                       const uint32_t* box, CUtensorMapSwizzle swizzle);
+
+// ----------------------------------------------------------------- projection
+// C[M, N] = A[M, K] * W[N, K]^T, bf16 in / fp32 accumulate / bf16 out (tcgen05).
+cudaError_t launch_proj_gemm_bf16(const bf16* A, const bf16* W, bf16* C, int M, int N, int K,
+                                  int32_t* dev_err, cudaStream_t stream);
+// Same contraction in fp32 on the CUDA cores.
+cudaError_t launch_proj_gemm_f32(const float* A, const float* W, float* C, int M, int N, int K,
+                                 cudaStream_t stream);
+
+// ----------------------------------------------------------------- pre-attention
+template <typename T>
+struct PreAttnArgs {
+  const T* src;          // [B*S, src_ld] rows: q~ | k~ | v~ columns
+  int64_t src_ld;
+  int B, S, Hq, Hkv, d, G, K;   // K = conv width, 0 = no conv / channel mix
+  int qk_mean, value_shift;
+  int rope_on;
+  double rope_log2_base;
+  const T *wq_seq, *wq_chan, *wk_seq, *wk_chan;  // chan may be null
+  T* q_out;              // [B, S, Hq, d]
+  T* k_out;              // [B, Hkv, kv_cap, d]
+  T* v_out;
+  int64_t kv_cap;
+  T* hist_q;             // nullable decode state
+  T* hist_k;
+  T* v_prev;
+  int32_t* len;
+  int32_t* dev_err;
+};
+template <typename T>
+cudaError_t launch_pre_attn(const PreAttnArgs<T>& a, cudaStream_t stream);
+
+// ----------------------------------------------------------------- attention
+struct AttnArgs {
+  const void* q;         // [B, S, Hq, d]
+  const void* k;         // [B, Hkv, kv_cap, d]
+  const void* v;
+  void* out;             // [B, S, Hq, d]
+  int B, S, Hq, Hkv, d, G;
+  int64_t kv_cap;
+  int causal;
+  int32_t* dev_err;
+};
+// bf16, d in {32, 64, 128}, G a power of two <= 128: tcgen05/TMEM/TMA flash attention.
+cudaError_t launch_attn_prefill_tc(const AttnArgs& a, cudaStream_t stream);
+// CUDA-core flash attention (fp32 path).
+template <typename T>
+cudaError_t launch_attn_prefill_simt(const AttnArgs& a, cudaStream_t stream);
+
+// ----------------------------------------------------------------- cache + decode
+template <typename T>
+cudaError_t launch_kv_append(T* cache_k, T* cache_v, int32_t* len, const T* k_new,
+                             const T* v_new, int B, int Hkv, int d, int64_t cap, int n_new,
+                             int32_t* dev_err, cudaStream_t stream);
+
+template <typename T>
+struct DecodeArgs {
+  const T* x_t;          // [B, E] or packed [B, N] when W is null
+  const T* W;            // [N, E] or null
+  int B, E, N, Hq, Hkv, d, G, K;
+  int qk_mean, value_shift, causal, rope_on;
+  double rope_log2_base;
+  const T *wq_seq, *wq_chan, *wk_seq, *wk_chan;
+  T* cache_k;            // [B, Hkv, cap, d]
+  T* cache_v;
+  int32_t* len;
+  int64_t cap;
+  T* hist_q;             // [B, K-1, Hq d]
+  T* hist_k;             // [B, K-1, Hkv d]
+  T* v_prev;             // [B, Hkv d]
+  T* out;                // [B, Hq d]
+  // workspace pieces
+  float* proj_part;      // [e_splits, B, N]
+  int e_splits;
+  float* q_ws;           // [B, Hq, d]
+  float* part_o;         // [B, Hkv, splits, G, d]
+  float* part_ml;        // [B, Hkv, splits, G, 2]
+  int32_t* tickets;      // [B*Hkv + B], zero before the first step, left zero after
+  int splits;
+  int chunk;             // keys per split
+  int32_t* dev_err;
+  void* const* phase_events;  // optional: 4 cudaEvent_t recorded between the kernels
+};
+template <typename T>
+cudaError_t launch_decode_step(const DecodeArgs<T>& a, cudaStream_t stream);
+
+// Split plan for the decode step, shared by the workspace-size query and the launch.
+void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int* e_splits,
+                 int* splits, int* chunk);
+
+}  // namespace ccgqa

@@ -1,0 +1,275 @@
+// Fused pre-attention kernel: causal sequence conv + per-head channel mix +
+// QK-mean + RoPE on q~ and k~, value-shift on v~
+// ("Compressed Convolutional Attention", Methodologie items 2-4).
+//
+// One CTA owns TT consecutive positions of one kv group (its G query heads, its
+// key head and its value head) of one sequence, so QK-mean, which mixes the
+// group's query heads with its key head, needs no data from other CTAs.
+//   1. the pre-conv q~/k~ rows [t0 - (K-1), t0 + TT) of the group are staged in
+//      shared memory channel-major (the K-1 halo rows come along);
+//   2. per head: the depthwise causal conv over the staged rows, then the
+//      channel mix y = W_h u as a register-tiled (4 positions x 4 channels)
+//      product, QK-mean from the staged pre-conv rows, RoPE from a per-CTA
+//      cos/sin table, one store;
+//   3. value-shift: upper half-channels of each value head come from the
+//      previous position -- a bit-exact copy;
+//   4. the CTA holding the last position writes the decode state.
+// All arithmetic in fp32; inputs and outputs in the working dtype.
+#include "kernels.h"
+
+namespace ccgqa {
+namespace {
+
+constexpr int kPreThreads = 256;
+
+__host__ __device__ inline int round4(int x) { return (x + 3) & ~3; }
+
+struct PreLayout {
+  int TT, KH, ZS, US;
+  int off_z, off_u, off_w, off_cs, off_theta;  // in floats
+  size_t bytes;
+};
+
+__host__ __device__ inline PreLayout pre_layout(int TT, int K, int G, int d) {
+  PreLayout L;
+  L.TT = TT;
+  L.KH = K > 0 ? K - 1 : 0;
+  L.ZS = (TT + L.KH) | 1;  // odd row stride: channel-major writes avoid bank conflicts
+  L.US = TT + 4;           // multiple of 4 for float4 reads
+  const int HC = (G + 1) * d;
+  L.off_z = 0;
+  L.off_u = round4(HC * L.ZS);
+  L.off_w = L.off_u + round4(d * L.US);
+  L.off_cs = L.off_w + round4(d * d);
+  L.off_theta = L.off_cs + round4(TT * d);  // cs holds TT * d/2 float2
+  L.bytes = static_cast<size_t>(L.off_theta) * 4 + static_cast<size_t>(d / 2) * 8 + 16;
+  return L;
+}
+
+template <typename T> struct Vec2;
+template <> struct Vec2<float> {
+  using type = float2;
+  __device__ static type make(float a, float b) { return make_float2(a, b); }
+};
+template <> struct Vec2<bf16> {
+  using type = __nv_bfloat162;
+  __device__ static type make(float a, float b) { return __floats2bfloat162_rn(a, b); }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kPreThreads)
+    pre_attn_kernel(const PreAttnArgs<T> a, const int TT) {
+  extern __shared__ float4 smem_f4[];
+  float* sm = reinterpret_cast<float*>(smem_f4);
+  const int b = blockIdx.z, g = blockIdx.y, t0 = blockIdx.x * TT;
+  const int d = a.d, G = a.G, K = a.K, S = a.S;
+  const int half = d / 2;
+  const PreLayout L = pre_layout(TT, K, G, d);
+  float* zT = sm + L.off_z;
+  float* u = sm + L.off_u;
+  float* Wt = sm + L.off_w;
+  float2* cs = reinterpret_cast<float2*>(sm + L.off_cs);
+  double* theta = reinterpret_cast<double*>(sm + L.off_theta);
+  const int KH = L.KH, ZS = L.ZS, US = L.US;
+  const int HC = (G + 1) * d;
+  const int tid = threadIdx.x;
+  const int64_t ld = a.src_ld;
+  const T* src_b = a.src + static_cast<int64_t>(b) * S * ld;
+  const int qcol0 = g * G * d;
+  const int kcol0 = a.Hq * d + g * d;
+  const int vcol0 = (a.Hq + a.Hkv) * d + g * d;
+
+  // 1. stage pre-conv rows t0-KH .. t0+TT-1 (zero outside [0, S)).
+  const int R = TT + KH;
+  for (int idx = tid; idx < R * HC; idx += kPreThreads) {
+    const int r = idx / HC, c = idx - r * HC;
+    const int t = t0 - KH + r;
+    const int col = c < G * d ? qcol0 + c : kcol0 + (c - G * d);
+    zT[c * ZS + r] = (t >= 0 && t < S) ? to_f32(src_b[static_cast<int64_t>(t) * ld + col]) : 0.f;
+  }
+  // 2. RoPE table: pair i turns by t * base^(-2i/d).  The angle is formed and
+  // reduced modulo one turn in fp64, so long positions keep full precision.
+  if (a.rope_on) {
+    for (int i = tid; i < half; i += kPreThreads)
+      theta[i] = exp2(-(2.0 * i / d) * a.rope_log2_base);
+  }
+  __syncthreads();
+  if (a.rope_on) {
+    const double inv_turn = 0.15915494309189533577;  // 1 / (2 pi)
+    for (int idx = tid; idx < TT * half; idx += kPreThreads) {
+      const int tl = idx / half, i = idx - tl * half;
+      double f = static_cast<double>(t0 + tl) * theta[i] * inv_turn;
+      f -= rint(f);
+      float s, c;
+      sincospif(static_cast<float>(2.0 * f), &s, &c);
+      cs[idx] = make_float2(c, s);
+    }
+  }
+
+  // 3. per head of the group: G query heads, then the key head.
+  for (int hh = 0; hh <= G; ++hh) {
+    const bool is_q = hh < G;
+    const int head = is_q ? g * G + hh : g;
+    const T* wseq = K > 0 ? (is_q ? a.wq_seq : a.wk_seq) + static_cast<int64_t>(head) * d * K
+                          : nullptr;
+    const T* wch_base = is_q ? a.wq_chan : a.wk_chan;
+    const T* wch = (K > 0 && wch_base) ? wch_base + static_cast<int64_t>(head) * d * d : nullptr;
+    const int cb = hh * d;
+    for (int idx = tid; idx < d * TT; idx += kPreThreads) {
+      const int j = idx / TT, tl = idx - j * TT;
+      const float* zr = zT + (cb + j) * ZS + tl + KH;
+      float acc;
+      if (K > 0) {
+        acc = 0.f;
+        for (int jj = 0; jj < K; ++jj) acc = fmaf(to_f32(wseq[j * K + jj]), zr[-jj], acc);
+      } else {
+        acc = zr[0];
+      }
+      u[j * US + tl] = acc;
+    }
+    if (wch) {
+      for (int idx = tid; idx < d * d; idx += kPreThreads) {
+        const int i = idx / d, j = idx - i * d;
+        Wt[j * d + i] = to_f32(wch[idx]);
+      }
+    }
+    __syncthreads();
+
+    const int nI2 = d / 4;  // channel pairs (i0, i0+1) in the lower half
+    const int ntile = (TT / 4) * nI2;
+    for (int idx = tid; idx < ntile; idx += kPreThreads) {
+      const int ip = idx % nI2, tq = idx / nI2;
+      const int tl0 = tq * 4, i0 = ip * 2, i1 = i0 + half;
+      float y[4][4];
+      if (wch) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) y[r][k] = 0.f;
+#pragma unroll 4
+        for (int j = 0; j < d; ++j) {
+          const float4 uu = *reinterpret_cast<const float4*>(u + j * US + tl0);
+          const float2 wl = *reinterpret_cast<const float2*>(Wt + j * d + i0);
+          const float2 wh = *reinterpret_cast<const float2*>(Wt + j * d + i1);
+          const float ur[4] = {uu.x, uu.y, uu.z, uu.w};
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            y[r][0] = fmaf(ur[r], wl.x, y[r][0]);
+            y[r][1] = fmaf(ur[r], wl.y, y[r][1]);
+            y[r][2] = fmaf(ur[r], wh.x, y[r][2]);
+            y[r][3] = fmaf(ur[r], wh.y, y[r][3]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          y[r][0] = u[i0 * US + tl0 + r];
+          y[r][1] = u[(i0 + 1) * US + tl0 + r];
+          y[r][2] = u[i1 * US + tl0 + r];
+          y[r][3] = u[(i1 + 1) * US + tl0 + r];
+        }
+      }
+      const int ch[4] = {i0, i0 + 1, i1, i1 + 1};
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int tl = tl0 + r, t = t0 + tl;
+        if (t >= S) continue;
+        const int zrow = tl + KH;
+        if (a.qk_mean) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float kp = zT[(G * d + ch[k]) * ZS + zrow];
+            float qp;
+            if (is_q) {
+              qp = zT[(hh * d + ch[k]) * ZS + zrow];
+            } else {
+              qp = 0.f;
+              for (int hl = 0; hl < G; ++hl) qp += zT[(hl * d + ch[k]) * ZS + zrow];
+              qp /= static_cast<float>(G);
+            }
+            y[r][k] += 0.5f * (qp + kp);
+          }
+        }
+        if (a.rope_on) {
+          const float2 c0 = cs[tl * half + i0], c1 = cs[tl * half + i0 + 1];
+          const float a0 = y[r][0], b0 = y[r][2], a1 = y[r][1], b1 = y[r][3];
+          y[r][0] = a0 * c0.x - b0 * c0.y;
+          y[r][2] = a0 * c0.y + b0 * c0.x;
+          y[r][1] = a1 * c1.x - b1 * c1.y;
+          y[r][3] = a1 * c1.y + b1 * c1.x;
+        }
+        T* dst = is_q ? a.q_out + ((static_cast<int64_t>(b) * S + t) * a.Hq + head) * d
+                      : a.k_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + t) * d;
+        using V2 = typename Vec2<T>::type;
+        *reinterpret_cast<V2*>(dst + i0) = Vec2<T>::make(y[r][0], y[r][1]);
+        *reinterpret_cast<V2*>(dst + i1) = Vec2<T>::make(y[r][2], y[r][3]);
+      }
+    }
+    __syncthreads();
+  }
+
+  // 4. value-shift: bit-exact gather of the current / previous v~ row.
+  constexpr int VEC = 16 / sizeof(T);
+  const int nchunk = d / VEC;
+  for (int idx = tid; idx < TT * nchunk; idx += kPreThreads) {
+    const int tl = idx / nchunk, i = (idx - tl * nchunk) * VEC;
+    const int t = t0 + tl;
+    if (t >= S) continue;
+    const bool from_prev = a.value_shift && i >= half;
+    uint4 val = make_uint4(0, 0, 0, 0);
+    const int ts = from_prev ? t - 1 : t;
+    if (ts >= 0)
+      val = *reinterpret_cast<const uint4*>(src_b + static_cast<int64_t>(ts) * ld + vcol0 + i);
+    *reinterpret_cast<uint4*>(a.v_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + t) * d +
+                              i) = val;
+  }
+
+  // 5. decode state, written by the CTA that holds position S-1.
+  if (a.len != nullptr && t0 <= S - 1 && S - 1 < t0 + TT) {
+    const int Hq = a.Hq, Hkv = a.Hkv;
+    for (int r = 0; r < KH; ++r) {
+      const int srow = S - KH + r;
+      for (int c = tid; c < G * d + d; c += kPreThreads) {
+        const bool q = c < G * d;
+        const int col = q ? qcol0 + c : kcol0 + (c - G * d);
+        const T val = srow >= 0 ? src_b[static_cast<int64_t>(srow) * ld + col] : from_f32<T>(0.f);
+        if (q)
+          a.hist_q[(static_cast<int64_t>(b) * KH + r) * Hq * d + qcol0 + c] = val;
+        else
+          a.hist_k[(static_cast<int64_t>(b) * KH + r) * Hkv * d + g * d + (c - G * d)] = val;
+      }
+    }
+    if (a.v_prev) {
+      for (int i = tid; i < d; i += kPreThreads)
+        a.v_prev[static_cast<int64_t>(b) * Hkv * d + g * d + i] =
+            src_b[static_cast<int64_t>(S - 1) * ld + vcol0 + i];
+    }
+    if (g == 0 && tid == 0) a.len[b] = S;
+  }
+}
+
+}  // namespace
+
+template <typename T>
+cudaError_t launch_pre_attn(const PreAttnArgs<T>& a, cudaStream_t stream) {
+  // Positions per CTA: TT * d = 4096 gives exactly one 4x4 register tile per
+  // thread in the channel mix; halve TT while the staging does not fit.
+  int TT = 4096 / a.d;
+  if (TT > 256) TT = 256;
+  while (TT > 4 && pre_layout(TT, a.K, a.G, a.d).bytes > 200 * 1024) TT /= 2;
+  const PreLayout L = pre_layout(TT, a.K, a.G, a.d);
+  if (L.bytes > 227 * 1024) return cudaErrorInvalidConfiguration;
+  cudaError_t e = cudaFuncSetAttribute(pre_attn_kernel<T>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(L.bytes));
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.S + TT - 1) / TT, a.Hkv, a.B);
+  pre_attn_kernel<T><<<grid, kPreThreads, L.bytes, stream>>>(a, TT);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_pre_attn<float>(const PreAttnArgs<float>&, cudaStream_t);
+template cudaError_t launch_pre_attn<bf16>(const PreAttnArgs<bf16>&, cudaStream_t);
+
+}  // namespace ccgqa

@@ -1,0 +1,239 @@
+// Latent down-projection x -> [q~ | k~ | v~]
+// ("Compressed Convolutional Attention", Methodologie item 1: tokens are
+// projected straight into the latent space of width E/C).
+//
+// bf16: C[M, N] = A[M, K] * W[N, K]^T on the 5th-generation tensor core.
+//   One CTA computes a 128 x 256 output tile.  Warp 0 streams 128x64 A and
+//   256x64 W tiles with TMA (128B swizzle) through a 4-stage shared-memory ring;
+//   warp 1 allocates 256 TMEM columns and one elected thread issues
+//   tcgen05.mma (M=128, N=256, K=16, fp32 accumulate in TMEM); warps 2-5 read
+//   the accumulator back with tcgen05.ld and store bf16 rows.
+// fp32: a plain shared-memory tiled GEMM on the CUDA cores.
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace ccgqa {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128, kBN = 256, kBK = 64, kStages = 4;
+constexpr int kGemmThreads = 192;
+constexpr uint32_t kATile = kBM * kBK * 2;      // 16 KB
+constexpr uint32_t kBTile = kBN * kBK * 2;      // 32 KB
+constexpr uint32_t kStageBytes = kATile + kBTile;
+constexpr size_t kGemmSmem = size_t(kStages) * kStageBytes + 1024 + 256;
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    proj_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
+                          const __grid_constant__ CUtensorMap tmB, bf16* __restrict__ C, int M,
+                          int N, int K, int32_t* dev_err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * kBM, n0 = blockIdx.x * kBN;
+  const int nkb = (K + kBK - 1) / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kBN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tensormap(&tmA);
+      prefetch_tensormap(&tmB);
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % kStages;
+        const uint32_t ph = (kb / kStages) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, &abort_flag, dev_err)) break;
+        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        uint8_t* sa = smem + s * kStageBytes;
+        tma_load_2d(sa, &tmA, &full[s], kb * kBK, m0);
+        tma_load_2d(sa + kATile, &tmB, &full[s], kb * kBK, n0);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc_bf16(kBM, kBN, false);
+      int kb = 0;
+      for (; kb < nkb; ++kb) {
+        const int s = kb % kStages;
+        const uint32_t ph = (kb / kStages) & 1;
+        if (!mbar_wait(&full[s], ph, &abort_flag, dev_err)) break;
+        tc_fence_after();
+        const uint32_t a_base = smem_addr(smem + s * kStageBytes);
+        const uint32_t b_base = a_base + kATile;
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k) {
+          // K-major, 128B-swizzled tiles: 8-row groups 1024 B apart; a K step of
+          // 16 bf16 advances the start address by 32 B inside the swizzle row.
+          const uint64_t ad = make_smem_desc(a_base + k * 32, 16, 1024, kSwizzle128B);
+          const uint64_t bd = make_smem_desc(b_base + k * 32, 16, 1024, kSwizzle128B);
+          mma_ss(tmem, ad, bd, idesc, (kb | k) != 0);
+        }
+        mma_commit(&empty[s]);
+      }
+      mma_commit(acc_full);
+    }
+  } else {
+    // Epilogue: warp w may only touch TMEM lanes [32 (w % 4), 32 (w % 4) + 32).
+    const int q4 = warp & 3;
+    if (mbar_wait(acc_full, 0, &abort_flag, dev_err)) {
+      tc_fence_after();
+      const int row = m0 + q4 * 32 + lane;
+      const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < kBN / 32; ++c) {
+        const int col0 = n0 + c * 32;
+        if (col0 >= N) break;  // warp-uniform
+        uint32_t r[32];
+        tmem_ld32(trow + c * 32, r);
+        tmem_wait_ld();
+        if (row < M) {
+          bf16* dst = C + static_cast<int64_t>(row) * N + col0;
+          if (col0 + 32 <= N && (N % 8) == 0) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 pk;
+              uint32_t* pw = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[v * 8 + 2 * e]),
+                                                          __uint_as_float(r[v * 8 + 2 * e + 1]));
+                pw[e] = *reinterpret_cast<uint32_t*>(&h2);
+              }
+              *reinterpret_cast<uint4*>(dst + v * 8) = pk;
+            }
+          } else {
+            for (int e = 0; e < 32 && col0 + e < N; ++e)
+              dst[e] = __float2bfloat16_rn(__uint_as_float(r[e]));
+          }
+        }
+      }
+    }
+  }
+
+  if (abort_flag && warp == 1 && lane == 0) {
+    // Do not release TMEM while an MMA might still write it.
+    mma_commit(drain);
+    const long long t0 = clock64();
+    while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitLimitCycles) {
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kBN);
+  }
+}
+
+// ------------------------------------------------------------------ fp32 SIMT
+constexpr int kFBM = 64, kFBN = 64, kFBK = 16;
+
+__global__ void __launch_bounds__(256)
+    proj_gemm_f32_kernel(const float* __restrict__ A, const float* __restrict__ W,
+                         float* __restrict__ C, int M, int N, int K) {
+  __shared__ float As[kFBK][kFBM + 4];
+  __shared__ float Ws[kFBK][kFBN + 4];
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  const int m0 = blockIdx.y * kFBM, n0 = blockIdx.x * kFBN;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += kFBK) {
+    for (int i = threadIdx.x; i < kFBM * kFBK; i += 256) {
+      const int r = i / kFBK, c = i % kFBK;
+      const int gm = m0 + r, gk = k0 + c;
+      As[c][r] = (gm < M && gk < K) ? A[static_cast<int64_t>(gm) * K + gk] : 0.f;
+      const int gn = n0 + r;
+      Ws[c][r] = (gn < N && gk < K) ? W[static_cast<int64_t>(gn) * K + gk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < kFBK; ++k) {
+      float a[4], w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[i] = As[k][ty * 4 + i];
+        w[i] = Ws[k][tx * 4 + i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], w[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int gm = m0 + ty * 4 + i;
+    if (gm >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int gn = n0 + tx * 4 + j;
+      if (gn < N) C[static_cast<int64_t>(gm) * N + gn] = acc[i][j];
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_proj_gemm_bf16(const bf16* A, const bf16* W, bf16* C, int M, int N, int K,
+                                  int32_t* dev_err, cudaStream_t stream) {
+  CUtensorMap tmA, tmB;
+  const uint64_t dA[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+  const uint64_t sA[1] = {static_cast<uint64_t>(K) * 2};
+  const uint32_t bA[2] = {kBK, kBM};
+  const uint64_t dB[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
+  const uint32_t bB[2] = {kBK, kBN};
+  if (!encode_tensor_map(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, dA, sA, bA,
+                         CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tensor_map(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, dB, sA, bB,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(proj_gemm_bf16_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kGemmSmem));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  dim3 grid((N + kBN - 1) / kBN, (M + kBM - 1) / kBM);
+  proj_gemm_bf16_kernel<<<grid, kGemmThreads, kGemmSmem, stream>>>(tmA, tmB, C, M, N, K,
+                                                                    dev_err);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_proj_gemm_f32(const float* A, const float* W, float* C, int M, int N, int K,
+                                 cudaStream_t stream) {
+  dim3 grid((N + kFBN - 1) / kFBN, (M + kFBM - 1) / kFBM);
+  proj_gemm_f32_kernel<<<grid, 256, 0, stream>>>(A, W, C, M, N, K);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace ccgqa

@@ -1,0 +1,105 @@
+"""Device-side plumbing around the C ABI: torch owns the memory (weights, KV
+cache, decode state, workspaces, the device error word) and this module hands
+pointers to the library.  No arithmetic of the method happens here."""
+from __future__ import annotations
+
+import torch
+
+from . import binding as B
+from .workloads import Workload
+
+
+def config_of(w: Workload) -> B.ccgqa_config:
+    return B.make_config(w.E, w.C, w.Hq, w.Hkv, conv_width=w.conv_width, qk_mean=w.qk_mean,
+                         value_shift=w.value_shift, causal=w.causal, rope_base=w.rope_base,
+                         dtype=B.F32 if w.dtype == "f32" else B.BF16)
+
+
+class DeviceLayer:
+    """Weights of one CCGQA layer resident on the GPU plus the buffers the
+    entry points need.  ``inputs`` is the dict produced by
+    ``workloads.make_inputs`` (CPU tensors in the working dtype)."""
+
+    def __init__(self, w: Workload, inputs: dict, device="cuda", batch: int | None = None,
+                 cap: int | None = None):
+        if not torch.cuda.is_available():
+            raise RuntimeError("CCGQA needs a CUDA device")
+        self.w = w
+        self.device = torch.device(device)
+        self.cfg = config_of(w)
+        dev = lambda t: None if t is None else t.to(self.device).contiguous()  # noqa: E731
+        self.W_qkv = dev(inputs.get("W_qkv"))
+        self.conv = {k: dev(inputs.get(k)) for k in ("conv_q_seq", "conv_q_chan", "conv_k_seq",
+                                                    "conv_k_chan")}
+        self.weights = B.make_weights(self.W_qkv, self.conv["conv_q_seq"], self.conv["conv_q_chan"],
+                                      self.conv["conv_k_seq"], self.conv["conv_k_chan"])
+        self.batch = batch if batch is not None else w.B
+        self.cap = cap if cap is not None else w.S
+        self.dev_err = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self.cache_tensors = None
+        self.cache = None
+        self._pf_ws = None
+        self._dec_ws = None
+
+    # -------------------------------------------------------------- buffers
+    def alloc_cache(self, batch: int | None = None, cap: int | None = None):
+        w = self.w
+        batch = self.batch if batch is None else batch
+        cap = self.cap if cap is None else cap
+        dt = w.torch_dtype
+        km1 = max(w.conv_width - 1, 0)
+        t = dict(
+            k=torch.zeros(batch, w.Hkv, cap, w.d, dtype=dt, device=self.device),
+            v=torch.zeros(batch, w.Hkv, cap, w.d, dtype=dt, device=self.device),
+            len=torch.zeros(batch, dtype=torch.int32, device=self.device),
+            hist_q=torch.zeros(batch, max(km1, 1), w.Hq * w.d, dtype=dt, device=self.device),
+            hist_k=torch.zeros(batch, max(km1, 1), w.Hkv * w.d, dtype=dt, device=self.device),
+            v_prev=torch.zeros(batch, w.Hkv * w.d, dtype=dt, device=self.device),
+        )
+        self.cache_tensors = t
+        self.cache = B.make_kvcache(t["k"], t["v"], t["len"], t["hist_q"], t["hist_k"], t["v_prev"])
+        return t
+
+    def prefill_workspace(self, batch: int, seq_len: int):
+        n = B.ccgqa_prefill_workspace_size(self.cfg, batch, seq_len)
+        if n == 0:
+            raise B.CCGQAError(1, "ccgqa_prefill_workspace_size")
+        if self._pf_ws is None or self._pf_ws.numel() < n:
+            self._pf_ws = torch.zeros(n, dtype=torch.uint8, device=self.device)
+        return self._pf_ws
+
+    def decode_workspace(self):
+        t = self.cache_tensors
+        batch, cap = t["k"].shape[0], t["k"].shape[2]
+        n = B.ccgqa_decode_workspace_size(self.cfg, batch, cap)
+        if self._dec_ws is None or self._dec_ws.numel() < n:
+            self._dec_ws = torch.zeros(n, dtype=torch.uint8, device=self.device)
+        return self._dec_ws
+
+    # -------------------------------------------------------------- calls
+    def prefill(self, x: torch.Tensor, out: torch.Tensor | None = None, use_cache: bool = True,
+                stream=None):
+        batch, seq_len = x.shape[0], x.shape[1]
+        w = self.w
+        if out is None:
+            out = torch.empty(batch, seq_len, w.Hq * w.d, dtype=w.torch_dtype, device=self.device)
+        ws = self.prefill_workspace(batch, seq_len)
+        B.ccgqa_prefill(self.cfg, self.weights, x, batch, seq_len, out,
+                        self.cache if use_cache else None, ws, self.dev_err, stream)
+        return out
+
+    def decode_step(self, x_t: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+        w = self.w
+        batch = x_t.shape[0]
+        if out is None:
+            out = torch.empty(batch, w.Hq * w.d, dtype=w.torch_dtype, device=self.device)
+        B.ccgqa_decode_step(self.cfg, self.weights, x_t, self.cache, out, self.decode_workspace(),
+                            self.dev_err, stream)
+        return out
+
+    def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None):
+        B.ccgqa_kvcache_append(self.cfg, self.cache, k_new, v_new, k_new.shape[1], self.dev_err,
+                               stream)
+
+    def error_bits(self) -> int:
+        return int(self.dev_err.item())

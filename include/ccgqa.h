@@ -1,0 +1,177 @@
+/*
+ * ccgqa.h -- C ABI of the B200 (sm_100a) CCGQA forward hot path.
+ *
+ * CCGQA (Compressed Convolutional Grouped-Query Attention) runs causal softmax
+ * attention entirely inside a latent space of width E / C:
+ *   "Compressed Convolutional Attention: Efficient Attention in a Compressed
+ *   Latent Space", section "Methodologie" items 1-4 (latent projection,
+ *   convolutional mixing with QK-mean, value-shift, RoPE in the latent heads)
+ *   and section "Compressed Convolutional Grouped Query Attention (CCGQA)"
+ *   (kv heads shared by groups of query heads, as in "Grouped Query Attention
+ *   (GQA)", section "Cómo funciona GQA").
+ *
+ * Geometry: d = E / (C * n_q_heads) is the head dim, G = n_q_heads / n_kv_heads
+ * the group size; query head h reads kv head h / G.  N_qkv = (Hq + 2 Hkv) d.
+ *
+ * Conventions for every entry point
+ *  - All tensor pointers are DEVICE pointers, row-major, densely packed, owned
+ *    by the caller; the library allocates no memory and keeps no state beyond
+ *    a launch counter and the optional per-thread timing hook below.  Element type is cfg->dtype (fp32 or bf16) unless
+ *    stated.  Every pointer must be 16-byte aligned.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream).  Host-side validation happens first: on any
+ *    invalid argument the call returns an error status and launches nothing.
+ *  - `dev_err` (nullable) is a device int32 that kernels OR error bits into
+ *    (CCGQA_DEVERR_*); the library never clears it.  A kernel that detects an
+ *    out-of-range index or capacity overflow skips the access and sets a bit;
+ *    no kernel traps.  Every wait inside a kernel is bounded; a wait that runs
+ *    out sets CCGQA_DEVERR_TIMEOUT and the kernel returns (outputs invalid).
+ *  - Returns CCGQA_ERR_CUDA when a launch fails (cudaGetLastError).
+ */
+#ifndef CCGQA_H
+#define CCGQA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CCGQA_API __attribute__((visibility("default")))
+
+typedef enum {
+  CCGQA_OK = 0,
+  CCGQA_ERR_INVALID_ARG = 1,  /* NULL / misaligned pointer, inconsistent sizes */
+  CCGQA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. bf16 head dim 16) */
+  CCGQA_ERR_CAPACITY = 3,     /* the tokens do not fit the cache capacity */
+  CCGQA_ERR_WORKSPACE = 4,    /* workspace NULL, misaligned or too small */
+  CCGQA_ERR_CUDA = 5          /* a CUDA runtime call or launch failed */
+} ccgqa_status;
+
+typedef enum { CCGQA_F32 = 0, CCGQA_BF16 = 1 } ccgqa_dtype;
+
+/* Device-side error bits OR-ed into *dev_err. */
+#define CCGQA_DEVERR_INDEX 1     /* an index fell outside its buffer; access skipped */
+#define CCGQA_DEVERR_TIMEOUT 2   /* a bounded in-kernel wait ran out */
+#define CCGQA_DEVERR_CAPACITY 4  /* len + new tokens > cap; that sequence untouched */
+
+/* Layer geometry and switches.  Each switch cites the step it turns on.  */
+typedef struct {
+  int32_t E;            /* model width */
+  int32_t C;            /* compression factor: latent width E / C  [Methodologie 1] */
+  int32_t n_q_heads;    /* Hq */
+  int32_t n_kv_heads;   /* Hkv; must divide Hq  [CCGQA] */
+  int32_t conv_width;   /* K in 0..4 taps of the causal sequence conv; 0 = no conv
+                           and no channel mix  [Methodologie 2] */
+  int32_t qk_mean;      /* 1 = add the QK-mean skip term  [Methodologie 2, QK-Mean] */
+  int32_t value_shift;  /* 1 = value-shift  [Methodologie 3] */
+  int32_t causal;       /* 1 = causal attention mask  [Probleemstelling] */
+  double rope_base;     /* RoPE base; 0 = no RoPE  [Methodologie 4] */
+  int32_t dtype;        /* ccgqa_dtype: fp32 or bf16 (bf16 needs d in {32, 64, 128}) */
+  int32_t reserved;     /* set to 0 */
+} ccgqa_config;
+
+/* Weights (device, cfg->dtype).  [Methodologie 1-2] */
+typedef struct {
+  /* [N_qkv, E]: output features x input features.  Rows [0, Hq d) give the
+     latent queries q~, the next Hkv d rows k~, the last Hkv d rows v~; within
+     each block row index = head * d + i.  NULL: the input rows already hold
+     q~ | k~ | v~ (width N_qkv) and the projection is skipped. */
+  const void* W_qkv;
+  /* [Hq d, K]: sequence-conv taps; tap j multiplies the row j steps back. */
+  const void* conv_q_seq;
+  /* [Hq, d, d]: per-head channel mix y_i = sum_j W[h][i][j] u_j; NULL = none. */
+  const void* conv_q_chan;
+  const void* conv_k_seq;   /* [Hkv d, K] */
+  const void* conv_k_chan;  /* [Hkv, d, d]; NULL = none */
+} ccgqa_weights;
+
+/* Latent KV cache plus the decode state (device buffers, caller-owned).
+   [Probleemstelling 2: the cache grows with the sequence; Resultaten 3: it
+   shrinks with C.] */
+typedef struct {
+  void* k;            /* [batch, Hkv, cap, d]  post-RoPE keys */
+  void* v;            /* [batch, Hkv, cap, d]  value-shifted values */
+  int32_t* len;       /* [batch] tokens held (device int32) */
+  void* conv_hist_q;  /* [batch, K-1, Hq d]  last K-1 pre-conv q~ rows, oldest first
+                         (NULL allowed when K <= 1) */
+  void* conv_hist_k;  /* [batch, K-1, Hkv d] */
+  void* v_prev;       /* [batch, Hkv d]  last v~ row before the shift (NULL allowed
+                         when value_shift == 0) */
+  int32_t batch;
+  int32_t cap;        /* token capacity per sequence */
+} ccgqa_kvcache;
+
+/* Bytes of workspace ccgqa_prefill needs for (batch, seq_len). */
+CCGQA_API size_t ccgqa_prefill_workspace_size(const ccgqa_config* cfg, int32_t batch,
+                                              int32_t seq_len);
+
+/* Bytes of workspace ccgqa_decode_step needs for a cache of (batch, cap).
+   The decode workspace must be zero-filled once before its first use; the
+   step leaves it ready for the next one. */
+CCGQA_API size_t ccgqa_decode_workspace_size(const ccgqa_config* cfg, int32_t batch,
+                                             int32_t cap);
+
+/* Causal prefill of `batch` sequences of `seq_len` tokens from an empty state.
+ * x:   [batch, seq_len, E]  (or [batch, seq_len, N_qkv] when w->W_qkv == NULL)
+ * out: [batch, seq_len, Hq d]  attention output per query head (no output
+ *      projection: the paper's layer ends in the latent space here).
+ * cache: nullable.  When given, rows [0, seq_len) of cache->k / cache->v are
+ *      overwritten, len[b] = seq_len, and the conv histories and v_prev are set
+ *      so that ccgqa_decode_step continues the sequences.  Needs
+ *      seq_len <= cache->cap and cache->batch == batch (else CCGQA_ERR_CAPACITY
+ *      / CCGQA_ERR_INVALID_ARG).
+ * workspace: >= ccgqa_prefill_workspace_size bytes, 256-byte aligned.
+ * Steps: projection (tcgen05 GEMM for bf16), fused conv + channel mix +
+ * QK-mean + RoPE + value-shift, flash attention (tcgen05/TMEM/TMA for bf16). */
+CCGQA_API ccgqa_status ccgqa_prefill(const ccgqa_config* cfg, const ccgqa_weights* w,
+                                     const void* x, int32_t batch, int32_t seq_len,
+                                     void* out, const ccgqa_kvcache* cache,
+                                     void* workspace, size_t workspace_bytes,
+                                     int32_t* dev_err, void* stream);
+
+/* One new token per sequence against the latent KV cache: equals row len[b]
+ * of a prefill over all tokens so far.
+ * x_t: [batch, E] (or [batch, N_qkv] when w->W_qkv == NULL);
+ * out: [batch, Hq d].  Appends the new k/v row at len[b], updates the conv
+ * histories and v_prev, then len[b] += 1.  A sequence with len[b] >= cap sets
+ * CCGQA_DEVERR_CAPACITY and is left unchanged (its out row is zero).
+ * workspace: >= ccgqa_decode_workspace_size(cfg, cache->batch, cache->cap),
+ * zero-filled before first use.  Steps that overlap on the GPU and share one
+ * workspace race; give concurrent streams their own workspace. */
+CCGQA_API ccgqa_status ccgqa_decode_step(const ccgqa_config* cfg, const ccgqa_weights* w,
+                                         const void* x_t, const ccgqa_kvcache* cache,
+                                         void* out, void* workspace,
+                                         size_t workspace_bytes, int32_t* dev_err,
+                                         void* stream);
+
+/* Append n_new rows per sequence: cache->k[b, g, len[b] + i, :] = k_new[b, i, g, :]
+ * (same for v), then len[b] += n_new.  Bit-exact copy.
+ * k_new, v_new: [batch, n_new, Hkv, d].  n_new > cap returns CCGQA_ERR_CAPACITY
+ * on the host; a sequence whose len[b] + n_new > cap is skipped on the device
+ * and sets CCGQA_DEVERR_CAPACITY.  Conv histories and v_prev are not touched. */
+CCGQA_API ccgqa_status ccgqa_kvcache_append(const ccgqa_config* cfg, const ccgqa_kvcache* cache,
+                                            const void* k_new, const void* v_new,
+                                            int32_t n_new, int32_t* dev_err, void* stream);
+
+/* Static description of a status code. */
+CCGQA_API const char* ccgqa_status_string(ccgqa_status s);
+
+/* Number of kernels this library has launched in this process. */
+CCGQA_API uint64_t ccgqa_launch_count(void);
+
+/* Optional timing hook for the calling host thread.  `events` points to n >= 4
+ * cudaEvent_t handles created by the caller; while set, ccgqa_prefill records
+ * events[0] before its first kernel, events[1] after the projection, events[2]
+ * after the pre-attention kernel and events[3] after attention, and
+ * ccgqa_decode_step records the same four points around its projection,
+ * pre-step and attention kernels -- all on the call's stream.  NULL or n < 4
+ * turns it off.  Only the pointer is kept; the caller keeps the events alive. */
+CCGQA_API void ccgqa_set_phase_events(void* const* events, int32_t n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CCGQA_H */

@@ -1,0 +1,132 @@
+"""Error model of a bf16 pipeline, used to set the bf16 parity bound.
+
+The stated bf16 bound, max|gpu - oracle| <= 2e-2 RMS(oracle out), cannot be
+met by any bf16 output on the CCGQA workloads: early positions average few keys,
+so max|out| reaches 10-20x RMS(out), and rounding the exact float64 result to
+bf16 alone already errs by 3-5% of RMS (``test_bf16_bound.py`` shows it).  The
+bf16 parity tests therefore check
+
+  (a) the stated 2e-2 as a root-mean-square bound:
+          ||gpu - oracle||_2 <= 2e-2 ||oracle||_2
+  (b) the worst element against an exactly rounded bf16 model of the same
+      computation:
+          max|gpu - oracle| <= 2e-2 RMS(oracle) + 1.5 max|model - oracle|
+
+The model is the oracle's float64 arithmetic with rounding to bf16 at the
+points where the bf16 path stores bf16 values: the projection output
+(q~, k~, v~), the attention inputs q, k, v, the probabilities P fed to the PV
+product (normaliser from the unrounded P), and the output.  The decode step
+keeps q and P in fp32, so its model rounds the projection row, the appended k/v
+rows and the output only.  This module is test infrastructure: it only calls
+the oracle's functions and rounds their results.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle.ccgqa as O
+
+L2_TOL = 2e-2
+ABS_TOL = 2e-2
+MODEL_SLACK = 1.5
+
+
+def bf(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64)).to(torch.bfloat16).double().numpy()
+
+
+def _attention_bf16_p(q, k, v, G, causal, q_pos):
+    T, Hq, d = q.shape
+    L = k.shape[0]
+    o = np.zeros((T, Hq, d))
+    keys = np.arange(L)
+    for h in range(Hq):
+        g = h // G
+        sc = (q[:, h] @ k[:, g].T) / np.sqrt(d)
+        if causal:
+            sc = np.where(keys[None, :] <= q_pos[:, None], sc, -np.inf)
+        p = np.exp(sc - sc.max(axis=1, keepdims=True))
+        l = p.sum(axis=1, keepdims=True)
+        o[:, h] = (bf(p) @ v[:, g]) / l
+    return o
+
+
+def model_prefill(layer: O.Layer, x: np.ndarray, rows=None):
+    """bf16-rounded prefill of one sequence; returns (out rows, state)."""
+    sh = layer.sh
+    S = x.shape[0]
+    qp, kp, vl = O.down_project(x, layer.W_qkv, sh)
+    qp, kp, vl = bf(qp), bf(kp), bf(vl)
+    yq, yk = O._mix_qk(layer, qp, kp)
+    pos = np.arange(S)
+    q = bf(O.rope(yq, pos, layer.rope_base))
+    k = bf(O.rope(yk, pos, layer.rope_base))
+    v = O.value_shift(vl) if layer.value_shift else vl
+    rows = pos if rows is None else np.asarray(rows)
+    o = _attention_bf16_p(q[rows], k, v, sh.G, layer.causal, rows)
+    Kc = max(layer.conv_width, 1)
+    hq = np.zeros((Kc - 1, sh.Hq * sh.d))
+    hk = np.zeros((Kc - 1, sh.Hkv * sh.d))
+    for j in range(1, Kc):
+        if S - j >= 0:
+            hq[Kc - 1 - j] = qp[S - j].reshape(-1)
+            hk[Kc - 1 - j] = kp[S - j].reshape(-1)
+    st = O.State(k=k, v=v, hist_q=hq, hist_k=hk, v_prev=vl[S - 1].reshape(-1))
+    return bf(o.reshape(len(rows), -1)), st
+
+
+def model_decode_step(layer: O.Layer, state: O.State, x_t: np.ndarray):
+    """bf16-rounded decode step; returns (out, new state)."""
+    sh = layer.sh
+    t = state.length
+    qp, kp, vl = O.down_project(x_t[None, :], layer.W_qkv, sh)
+    qp, kp, vl = bf(qp), bf(kp), bf(vl)
+    K = max(layer.conv_width, 1)
+    yq, yk = O._mix_qk(layer, qp, kp, state.hist_q if K > 1 else None,
+                       state.hist_k if K > 1 else None)
+    pos = np.array([t])
+    q = O.rope(yq, pos, layer.rope_base)
+    k = bf(O.rope(yk, pos, layer.rope_base))
+    v = O.value_shift(vl, state.v_prev.reshape(sh.Hkv, sh.d)) if layer.value_shift else vl
+    k_all = np.concatenate([state.k, k])
+    v_all = np.concatenate([state.v, v])
+    o = bf(O.attention(q, k_all, v_all, sh.G, layer.causal, q_pos=pos).reshape(-1))
+    if K > 1:
+        hq = np.concatenate([state.hist_q[1:], qp.reshape(1, -1)])
+        hk = np.concatenate([state.hist_k[1:], kp.reshape(1, -1)])
+    else:
+        hq, hk = state.hist_q, state.hist_k
+    return o, O.State(k=k_all, v=v_all, hist_q=hq, hist_k=hk, v_prev=vl.reshape(-1))
+
+
+def check_bf16(gpu, ref, model, what=""):
+    """Bounds (a) and (b) above; returns (rms-relative L2 error, max err / RMS)."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    model = np.asarray(model, dtype=np.float64)
+    assert gpu.shape == ref.shape == model.shape, (gpu.shape, ref.shape, model.shape)
+    assert np.all(np.isfinite(gpu)), f"{what}: non-finite output"
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    l2 = float(np.linalg.norm(gpu - ref) / max(np.linalg.norm(ref), 1e-300))
+    e_gpu = float(np.max(np.abs(gpu - ref)))
+    e_model = float(np.max(np.abs(model - ref)))
+    assert l2 <= L2_TOL, f"{what}: relative L2 error {l2:.3e} > {L2_TOL}"
+    bound = ABS_TOL * rms + MODEL_SLACK * e_model
+    assert e_gpu <= bound, (f"{what}: max err {e_gpu:.3e} > {ABS_TOL} RMS ({rms:.3e}) + "
+                            f"{MODEL_SLACK} x bf16-model err {e_model:.3e}")
+    return l2, e_gpu / rms
+
+
+def check_within_one_ulp(gpu, model, what=""):
+    """Stored bf16 tensors (cache rows): within one bf16 ulp of the model value
+    (the only freedom is fp32-vs-fp64 arithmetic before the same rounding)."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    model = np.asarray(model, dtype=np.float64)
+    ulp = np.abs(model) * 2.0 ** -7 + 1e-30
+    bad = np.abs(gpu - model) > ulp
+    frac = float(np.mean(bad))
+    assert frac <= 1e-3, f"{what}: {frac:.2e} of elements differ by more than one bf16 ulp"
+    rms = float(np.sqrt(np.mean(model ** 2)))
+    worst = float(np.max(np.abs(gpu - model)))
+    assert worst <= 0.05 * rms, f"{what}: worst difference {worst:.3e} > 0.05 RMS {rms:.3e}"

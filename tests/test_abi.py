@@ -1,0 +1,160 @@
+"""The C ABI on the host (no GPU needed): the library loads, exports every
+entry point the header declares, its struct layouts match the C compiler's,
+and argument validation rejects bad calls before any launch."""
+import ctypes
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+from compressed_latent_grouped_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(B.LIB_PATH):
+        from compressed_latent_grouped_b200 import build
+        build.build()
+    return B.load()
+
+
+def test_exports_every_header_symbol(lib):
+    names = B.header_symbols()
+    assert set(names) >= {"ccgqa_prefill", "ccgqa_decode_step", "ccgqa_kvcache_append",
+                          "ccgqa_prefill_workspace_size", "ccgqa_decode_workspace_size",
+                          "ccgqa_status_string", "ccgqa_launch_count"}
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ccgqa.h but not exported"
+
+
+def test_struct_layout_matches_c():
+    src = r"""
+#include <stdio.h>
+#include <stddef.h>
+#include "ccgqa.h"
+int main(void) {
+  printf("%zu %zu %zu %zu %zu\n", sizeof(ccgqa_config), offsetof(ccgqa_config, rope_base),
+         offsetof(ccgqa_config, dtype), sizeof(ccgqa_weights), sizeof(ccgqa_kvcache));
+  printf("%zu %zu\n", offsetof(ccgqa_kvcache, batch), offsetof(ccgqa_kvcache, cap));
+  return 0;
+}
+"""
+    with tempfile.TemporaryDirectory() as td:
+        c = os.path.join(td, "l.c")
+        exe = os.path.join(td, "l")
+        open(c, "w").write(src)
+        subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe], check=True)
+        out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split()
+    vals = [int(v) for v in out]
+    assert vals[0] == ctypes.sizeof(B.ccgqa_config)
+    assert vals[1] == B.ccgqa_config.rope_base.offset
+    assert vals[2] == B.ccgqa_config.dtype.offset
+    assert vals[3] == ctypes.sizeof(B.ccgqa_weights)
+    assert vals[4] == ctypes.sizeof(B.ccgqa_kvcache)
+    assert vals[5] == B.ccgqa_kvcache.batch.offset
+    assert vals[6] == B.ccgqa_kvcache.cap.offset
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert B.ccgqa_status_string(s)
+    assert B.ccgqa_status_string(0) == "ok"
+
+
+def _cfg(**kw):
+    base = dict(E=2048, C=4, n_q_heads=16, n_kv_heads=4, conv_width=4, qk_mean=1, value_shift=1,
+                causal=1, rope_base=1e4, dtype=B.BF16)
+    base.update(kw)
+    return B.make_config(**base)
+
+
+def test_workspace_sizes(lib):
+    cfg = _cfg()
+    n = B.ccgqa_prefill_workspace_size(cfg, 4, 4096)
+    d = 32
+    N = (16 + 8) * d
+    expect = 4 * 4096 * (N + 16 * d + 2 * 4 * d) * 2
+    assert expect <= n <= expect + 4 * 256
+    assert B.ccgqa_decode_workspace_size(cfg, 64, 16384) > 0
+    # invalid geometry -> 0
+    assert B.ccgqa_prefill_workspace_size(_cfg(n_kv_heads=3), 1, 16) == 0
+    assert B.ccgqa_prefill_workspace_size(cfg, 0, 16) == 0
+
+
+class _FakeTensor:
+    """Stands in for a device tensor: the calls below are rejected by host
+    validation before anything reaches the GPU."""
+
+    def __init__(self, addr, nbytes=1 << 30):
+        self.addr, self.nbytes = addr, nbytes
+
+    def data_ptr(self):
+        return self.addr
+
+    def numel(self):
+        return self.nbytes
+
+    def element_size(self):
+        return 1
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(n_kv_heads=3), 1),           # Hq % Hkv != 0
+    (dict(E=2050), 1),                 # E % (C Hq) != 0
+    (dict(conv_width=5), 1),
+    (dict(dtype=7), 1),
+    (dict(rope_base=-1.0), 1),
+    (dict(E=1024, C=8), 2),            # d = 8 unsupported
+    (dict(E=256, C=1, n_q_heads=16, n_kv_heads=16), 2),  # bf16 d = 16 unsupported
+])
+def test_invalid_config_rejected(lib, bad, status):
+    cfg = _cfg(**bad)
+    w = B.make_weights()
+    st = lib.ccgqa_prefill(ctypes.byref(cfg), ctypes.byref(w), ctypes.c_void_p(4096), 1, 16,
+                           ctypes.c_void_p(8192), None, ctypes.c_void_p(1 << 20), 1 << 30, None,
+                           None)
+    assert st == status
+
+
+def test_invalid_pointers_and_workspace_rejected(lib):
+    cfg = _cfg(conv_width=0, qk_mean=0, value_shift=0)
+    w = B.make_weights()
+    ok_ws = _FakeTensor(1 << 20)
+    assert B.ccgqa_prefill(cfg, w, _FakeTensor(4096), 1, 16, None, None, ok_ws, stream=0, check=False) == 1
+    assert B.ccgqa_prefill(cfg, w, _FakeTensor(4097), 1, 16, _FakeTensor(8192), None, ok_ws,
+                           stream=0, check=False) == 1                    # misaligned x
+    assert B.ccgqa_prefill(cfg, w, _FakeTensor(4096), 1, 16, _FakeTensor(8192), None,
+                           _FakeTensor(1 << 20, 16), stream=0, check=False) == 4   # workspace too small
+    assert B.ccgqa_prefill(cfg, w, _FakeTensor(4096), 1, 16, _FakeTensor(8192), None,
+                           _FakeTensor((1 << 20) + 16), stream=0, check=False) == 4  # misaligned workspace
+    assert B.ccgqa_prefill(cfg, w, _FakeTensor(4096), 0, 16, _FakeTensor(8192), None, ok_ws,
+                           stream=0, check=False) == 1
+    # conv on but no conv weights
+    cfg2 = _cfg()
+    assert B.ccgqa_prefill(cfg2, w, _FakeTensor(4096), 1, 16, _FakeTensor(8192), None, ok_ws,
+                           stream=0, check=False) == 1
+
+
+def test_capacity_checked_on_host(lib):
+    cfg = _cfg(conv_width=0, qk_mean=0, value_shift=0)
+    cache = B.ccgqa_kvcache(4096, 8192, 12288, None, None, None, 1, 8)
+    w = B.make_weights()
+    st = lib.ccgqa_prefill(ctypes.byref(cfg), ctypes.byref(w), ctypes.c_void_p(4096), 1, 16,
+                           ctypes.c_void_p(8192), ctypes.byref(cache), ctypes.c_void_p(1 << 20),
+                           1 << 30, None, None)
+    assert st == 3   # 16 tokens > cap 8
+    st = lib.ccgqa_kvcache_append(ctypes.byref(cfg), ctypes.byref(cache), ctypes.c_void_p(4096),
+                                  ctypes.c_void_p(8192), 9, None, None)
+    assert st == 3
+    cache.batch = 2
+    st = lib.ccgqa_prefill(ctypes.byref(cfg), ctypes.byref(w), ctypes.c_void_p(4096), 1, 4,
+                           ctypes.c_void_p(8192), ctypes.byref(cache), ctypes.c_void_p(1 << 20),
+                           1 << 30, None, None)
+    assert st == 1   # cache batch mismatch
+
+
+def test_launch_count_starts_at_zero(lib):
+    assert B.ccgqa_launch_count() == 0

@@ -1,0 +1,132 @@
+"""Prefill parity: the CUDA path through the C ABI against the float64 oracle.
+
+Small cases are compared element by element (several 128-row tiles and a
+ragged tail); the full-size workloads are run in the launch configuration the
+benchmark times and compared on sampled query rows."""
+import numpy as np
+import pytest
+import torch
+
+from compressed_latent_grouped_b200 import binding as B
+from compressed_latent_grouped_b200.device import DeviceLayer
+from compressed_latent_grouped_b200.workloads import WORKLOADS, make_inputs, sample_rows
+from gpu_ref import check_prefill
+
+pytestmark = pytest.mark.gpu
+
+W1 = WORKLOADS["f32_s128"]
+W2 = WORKLOADS["bf16_prefill_b4_s4096"]
+W3 = WORKLOADS["bf16_prefill_b1_s32768"]
+W5 = WORKLOADS["bf16_gqa_b2_s8192"]
+
+SMALL = {
+    "f32_s128": W1,
+    "f32_d64_s70": W3.with_(name="f32_d64", dtype="f32", B=2, S=70),
+    "f32_d32_noncausal": W2.with_(name="f32_nc", dtype="f32", B=1, S=45, causal=False),
+    "bf16_d32_s200": W2.with_(name="d32", B=2, S=200),
+    "bf16_d64_s300": W3.with_(name="d64", S=300),
+    "bf16_d128_s260_plain": W5.with_(name="d128", B=1, S=260),
+    "bf16_d32_noncausal": W2.with_(name="d32nc", B=1, S=333, causal=False),
+    "bf16_d64_mha": W3.with_(name="mha", E=1024, C=2, Hq=8, Hkv=8, S=150),
+    "bf16_d64_g8": W3.with_(name="g8", E=2048, C=4, Hq=8, Hkv=1, S=140),
+    "bf16_d128_conv": W5.with_(name="d128conv", B=1, S=190, conv_width=4, qk_mean=True,
+                               value_shift=True, packed_input=False, E=2048, C=1, Hq=16, Hkv=4),
+    "bf16_d64_s1": W3.with_(name="s1", S=1),
+    "bf16_d64_s3": W3.with_(name="s3", S=3),
+    "bf16_d32_conv2_nochan": W2.with_(name="k2", B=1, S=77, conv_width=2),
+    "bf16_d64_norope": W3.with_(name="norope", S=129, rope_base=0.0),
+}
+
+
+def _run(w, inp, use_cache=True, cap=None):
+    lay = DeviceLayer(w, inp, cap=cap)
+    if use_cache:
+        lay.alloc_cache()
+    x = inp["x"].cuda()
+    out = lay.prefill(x, use_cache=use_cache)
+    torch.cuda.synchronize()
+    assert lay.error_bits() == 0
+    return lay, out
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_prefill_small_elementwise(name):
+    w = SMALL[name]
+    inp = make_inputs(w, seed=0)
+    if name == "bf16_d32_conv2_nochan":
+        inp["conv_q_chan"] = inp["conv_k_chan"] = None
+    lay, out = _run(w, inp, use_cache=(name != "bf16_d64_norope"))
+    got = out.float().cpu().numpy()
+    for b in range(w.B):
+        ck = cv = None
+        if lay.cache is not None:
+            ck = lay.cache_tensors["k"][b, :, : w.S].float().cpu().numpy().transpose(1, 0, 2)
+            cv = lay.cache_tensors["v"][b, :, : w.S].float().cpu().numpy().transpose(1, 0, 2)
+            assert int(lay.cache_tensors["len"][b]) == w.S
+        check_prefill(w, inp, b, got[b], cache_k=ck, cache_v=cv, what=f"{name} b={b}")
+
+
+@pytest.mark.parametrize("w", [W2, W3, W5], ids=lambda w: w.name)
+def test_prefill_full_size_sampled_rows(w):
+    inp = make_inputs(w, seed=0)
+    _, out = _run(w, inp, use_cache=True)
+    rows = sample_rows(w.S, 1024)
+    for b in range(w.B):
+        got = out[b, torch.from_numpy(rows).cuda()].float().cpu().numpy()
+        check_prefill(w, inp, b, got, rows=rows, what=f"{w.name} b={b}")
+
+
+def test_prefill_without_cache_matches_with_cache():
+    w = W2.with_(B=1, S=257)
+    inp = make_inputs(w, seed=3)
+    _, a = _run(w, inp, use_cache=True)
+    _, b = _run(w, inp, use_cache=False)
+    assert torch.equal(a, b)
+
+
+def test_prefill_is_deterministic():
+    w = W3.with_(S=520)
+    inp = make_inputs(w, seed=5)
+    _, a = _run(w, inp)
+    _, b = _run(w, inp)
+    assert torch.equal(a, b)
+
+
+def test_value_shift_gather_bit_exact():
+    """With packed input the cache's values are a pure gather of v~ bits:
+    lower half-channels from the same position, upper half from the previous
+    one, zero at position 0."""
+    w = W5.with_(B=2, S=300, value_shift=True)
+    inp = make_inputs(w, seed=1)
+    lay, _ = _run(w, inp)
+    x = inp["x"]
+    d, Hq, Hkv = w.d, w.Hq, w.Hkv
+    vt = x[..., (Hq + Hkv) * d:].reshape(w.B, w.S, Hkv, d)
+    v = lay.cache_tensors["v"][:, :, : w.S].cpu().permute(0, 2, 1, 3)
+    h = d // 2
+    assert torch.equal(v[..., :h].view(torch.int16), vt[..., :h].view(torch.int16))
+    assert torch.equal(v[:, 1:, :, h:].view(torch.int16), vt[:, :-1, :, h:].view(torch.int16))
+    assert torch.all(v[:, 0, :, h:].view(torch.int16) == 0)
+    # decode state: the last v~ row and the last K-1 pre-conv rows, bit for bit
+    assert torch.equal(lay.cache_tensors["v_prev"].cpu().view(torch.int16),
+                       vt[:, -1].reshape(w.B, -1).view(torch.int16))
+
+
+def test_decode_state_after_prefill_bit_exact():
+    w = W2.with_(B=2, S=130, packed_input=True)
+    inp = make_inputs(w, seed=2)
+    lay, _ = _run(w, inp)
+    x = inp["x"]
+    d, Hq, Hkv = w.d, w.Hq, w.Hkv
+    hq = lay.cache_tensors["hist_q"].cpu()
+    hk = lay.cache_tensors["hist_k"].cpu()
+    assert torch.equal(hq.view(torch.int16), x[:, -3:, : Hq * d].view(torch.int16))
+    assert torch.equal(hk.view(torch.int16), x[:, -3:, Hq * d:(Hq + Hkv) * d].view(torch.int16))
+
+
+def test_launches_are_counted():
+    w = W2.with_(B=1, S=64)
+    inp = make_inputs(w, seed=0)
+    n0 = B.ccgqa_launch_count()
+    _run(w, inp)
+    assert B.ccgqa_launch_count() - n0 == 3   # projection, pre-attention, attention
