@@ -119,14 +119,14 @@ def check_bf16(gpu, ref, model, what=""):
 
 
 def check_within_one_ulp(gpu, model, what=""):
-    """Stored bf16 tensors (cache rows): within one bf16 ulp of the model value
-    (the only freedom is fp32-vs-fp64 arithmetic before the same rounding)."""
+    """Stored bf16 tensors (cache rows) against the model: within one bf16 ulp
+    of the element plus one bf16 ulp of the tensor's RMS.  The freedom is
+    fp32-vs-fp64 arithmetic before the same rounding; a one-ulp difference in a
+    rounded input propagates through the convolution in absolute terms, hence
+    the RMS term."""
     gpu = np.asarray(gpu, dtype=np.float64)
     model = np.asarray(model, dtype=np.float64)
-    ulp = np.abs(model) * 2.0 ** -7 + 1e-30
-    bad = np.abs(gpu - model) > ulp
-    frac = float(np.mean(bad))
-    assert frac <= 1e-3, f"{what}: {frac:.2e} of elements differ by more than one bf16 ulp"
     rms = float(np.sqrt(np.mean(model ** 2)))
-    worst = float(np.max(np.abs(gpu - model)))
-    assert worst <= 0.05 * rms, f"{what}: worst difference {worst:.3e} > 0.05 RMS {rms:.3e}"
+    excess = np.abs(gpu - model) - 2.0 ** -7 * (np.abs(model) + rms)
+    worst = float(np.max(excess))
+    assert worst <= 0.0, f"{what}: a stored value is {worst:.3e} beyond one ulp (+ one ulp of RMS)"
