@@ -3,22 +3,25 @@
 // group of query heads inside the latent space; "Grouped Query Attention
 // (GQA)", "Cómo funciona GQA").
 //
-// One CTA = one 128-row query tile of one kv group of one sequence.  The tile
-// packs the group's G query heads: row r is position t0 + r / G, head
-// g*G + r % G.  A 5-D TMA box gathers those rows straight from q[B, S, Hq, d],
-// so one K/V tile load in shared memory serves all G query heads.
+// Query rows are packed per kv group: row r of a tile is position
+// t0 + r / G, head g*G + r % G, so a 5-D TMA box gathers a tile straight from
+// q[B, S, Hq, d] and one K/V tile in shared memory serves all G query heads.
 //
-//   warp 0     TMA producer: Q once, then K/V tiles of 128 keys through a ring
-//   warp 1     TMEM allocator; one elected thread issues every tcgen05.mma:
-//                S_j = Q K_j^T   (SS, M=128 N=128, fp32 into TMEM, 2 buffers)
-//                O  += P_j V_j   (SS, M=128 N=d, V read MN-major)
-//   warps 2-5  softmax: each thread owns one row (TMEM lane), loads S_j with
-//              tcgen05.ld, masks, keeps a running max / sum in registers,
-//              writes bf16 P into a 128B-swizzled shared tile, rescales O in
-//              TMEM when the running max grows by more than 2^8, and at the
-//              end normalises O and stores it.
-// The S double buffer lets the MMA of tile j+1 run under the softmax of tile j.
-// No cluster multicast is used; every wait is bounded.
+// One CTA owns two 128-row query tiles (A and B) of one kv group and streams
+// the K/V tiles both need once:
+//   warp 0      TMA producer: Q_A, Q_B once, then K/V tiles of 128 keys
+//               through a ring of shared-memory stages
+//   warp 1      TMEM allocator; one elected thread issues every tcgen05.mma:
+//                 S_X = Q_X K_j^T  (SS, M=128 N=128, fp32 accumulators in TMEM)
+//                 O_X += P_X V_j   (TS: P read from TMEM, V from shared memory)
+//   warps 2-5   softmax of tile A, warps 6-9 softmax of tile B: one thread per
+//               row (TMEM lane); tcgen05.ld of S, running max / sum in
+//               registers, P written back to TMEM as bf16 pairs in the upper
+//               half of the S columns, O rescaled in TMEM when the running max
+//               grows by more than 2^8, normalised O stored at the end.
+// While one warpgroup exponentiates, the tensor core runs the other tile's
+// MMAs, so the exp unit, the FMA pipe and the tensor pipe overlap.  No cluster
+// multicast is used; every wait is bounded.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -27,9 +30,8 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 320;
 constexpr int kBlockM = 128, kBlockN = 128;
-// exp(x) = exp2(x * log2(e)); scores are kept in the log2 domain.
 constexpr float kLog2e = 1.4426950408889634f;
 // The running max used for exp2 is only raised when it falls behind by more
 // than this many doublings, so P <= 2^8 and O is rescaled rarely.
@@ -43,17 +45,17 @@ struct Cfg {
   static constexpr uint32_t kSwz = (D == 32) ? kSwizzle64B : kSwizzle128B;
   static constexpr uint32_t kSbo = 8 * kRowBytes;             // 8-row group stride
   static constexpr uint32_t kPanelBytes = 128 * kRowBytes;    // one panel of 128 rows
-  static constexpr uint32_t kTileBytes = 128 * D * 2;         // Q / K / V tile
-  static constexpr int kStages = (D == 128) ? 2 : 3;
-  static constexpr uint32_t kPBytes = 128 * 128 * 2;
-  static constexpr uint32_t kOffQ = 0;
-  static constexpr uint32_t kOffK = kOffQ + kTileBytes;
+  static constexpr uint32_t kTileBytes = 128 * D * 2;         // one Q / K / V tile
+  static constexpr int kStages = (D == 128) ? 2 : (D == 64 ? 3 : 4);
+  static constexpr uint32_t kOffQ = 0;                        // Q_A, Q_B
+  static constexpr uint32_t kOffK = 2 * kTileBytes;
   static constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
-  static constexpr uint32_t kOffP = kOffV + kStages * kTileBytes;
-  static constexpr uint32_t kOffBar = kOffP + kPBytes;
+  static constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
   static constexpr size_t kSmem = kOffBar + 256 + 1024;
-  static constexpr uint32_t kTmemCols = 512;                  // S0 | S1 | O
-  static constexpr uint32_t kColO = 256;
+  static constexpr uint32_t kTmemCols = 512;
+  __device__ static constexpr uint32_t col_s(int x) { return x * 128; }       // S_A | S_B
+  __device__ static constexpr uint32_t col_p(int x) { return x * 128 + 64; }  // P in S's upper half
+  __device__ static constexpr uint32_t col_o(int x) { return 256 + x * D; }   // O_A | O_B
 };
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -62,12 +64,37 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe, used for part of the probabilities so the exp unit and
+// the FMA pipe share the work.  Cody-Waite style reduction x = n + f with
+// n = round(x) and f in [-0.5, 0.5] (adding 1.5 * 2^23 leaves round(x) in the
+// low mantissa bits), 2^f from a degree-3 polynomial fitted for this kernel
+// (relative error below 8e-5, well under bf16's 2^-9), and 2^n added to the
+// exponent field.  Inputs are clamped at -126 (the exponent field of p,
+// 126 or 127, must stay positive after adding n), so -inf gives ~1e-38.
+__device__ __forceinline__ float soft_exp2(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  float p = fmaf(0.05521968f, f, 0.24260941f);
+  p = fmaf(p, f, 0.69325167f);
+  p = fmaf(p, f, 0.99992800f);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
+// Pairs (c2 % 4 == 0) of each softmax row use soft_exp2: one element in four.
+constexpr int kSoftExpEvery = 4;
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h2 = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h2);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                            const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, bf16* __restrict__ out,
-                           int B, int S, int Hq, int Hkv, int G_log2, int n_qt, int causal,
+                           int B, int S, int Hq, int Hkv, int G_log2, int n_pairs, int causal,
                            int32_t* dev_err) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -77,22 +104,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;                  // [kStages]
   uint64_t* kv_empty = kv_full + C::kStages;     // [kStages]
-  uint64_t* s_full = kv_empty + C::kStages;      // [2]
-  uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = p_full + 1;
-  uint64_t* drain = pv_done + 1;
+  uint64_t* s_full = kv_empty + C::kStages;      // [2]  S_X ready
+  uint64_t* p_full = s_full + 2;                 // [2]  P_X written (128 arrivals)
+  uint64_t* o_done = p_full + 2;                 // [2]  PV_X complete
+  uint64_t* drain = o_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = 1 << G_log2;
   const int BH = B * Hkv;
-  const int qt = n_qt - 1 - static_cast<int>(blockIdx.x) / BH;  // longest tiles first
+  const int pair = n_pairs - 1 - static_cast<int>(blockIdx.x) / BH;  // longest first
   const int bg = static_cast<int>(blockIdx.x) % BH;
   const int b = bg / Hkv, g = bg % Hkv;
-  const int rows_pos = kBlockM >> G_log2;       // positions per tile
-  const int t0 = qt * rows_pos;
-  const int t_last = min(t0 + rows_pos - 1, S - 1);
+  const int pos_per_tile = kBlockM >> G_log2;
+  const int t0 = pair * 2 * pos_per_tile;
+  const int t_last = min(t0 + 2 * pos_per_tile - 1, S - 1);
   const int n_kv = causal ? (t_last / kBlockN + 1) : (S + kBlockN - 1) / kBlockN;
 
   if (threadIdx.x == 0) {
@@ -101,10 +128,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(p_full, 128);
-    mbar_init(pv_done, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[x], 128);
+      mbar_init(&o_done[x], 1);
+    }
     mbar_init(drain, 1);
     abort_flag = 0;
     fence_barrier_init();
@@ -124,11 +152,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
-      mbar_arrive_expect_tx(q_full, C::kTileBytes);
+      mbar_arrive_expect_tx(q_full, 2 * C::kTileBytes);
 #pragma unroll
-      for (int p = 0; p < C::kPanels; ++p)
-        tma_load_5d(smem + C::kOffQ + p * C::kPanelBytes, &tmQ, q_full, p * C::kPanelCols, 0, g,
-                    t0, b);
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int p = 0; p < C::kPanels; ++p)
+          tma_load_5d(smem + C::kOffQ + x * C::kTileBytes + p * C::kPanelBytes, &tmQ, q_full,
+                      p * C::kPanelCols, 0, g, t0 + x * pos_per_tile, b);
       for (int j = 0; j < n_kv; ++j) {
         const int st = j % C::kStages;
         const uint32_t ph = (j / C::kStages) & 1;
@@ -145,96 +175,106 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Order: S_A(0) S_B(0) | PV_A(j) S_A(j+1) PV_B(j) S_B(j+1) | ...
+    // S_X(j+1) follows PV_X(j) directly, so tile A's next softmax can start
+    // while tile B's softmax is still running (the two warpgroups alternate).
     if (lane == 0) {
       const uint32_t idesc_s = make_idesc_bf16(kBlockM, kBlockN, false);
       const uint32_t idesc_o = make_idesc_bf16(kBlockM, D, true);
       const uint32_t q_base = smem_addr(smem + C::kOffQ);
-      const uint32_t p_base = smem_addr(smem + C::kOffP);
-      auto issue_pv = [&](int jj) {
+      auto issue_s = [&](int x, int jj) {
         const int st = jj % C::kStages;
-        const uint32_t v_base = smem_addr(smem + C::kOffV + st * C::kTileBytes);
-#pragma unroll
-        for (int k = 0; k < kBlockN / 16; ++k) {
-          // P: K-major, two 64-key panels of 128 rows x 128 B.
-          const uint64_t ad = make_smem_desc(p_base + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024,
-                                             kSwizzle128B);
-          // V: MN-major (d contiguous); 16 keys = 16 rows of the swizzle width.
-          const uint64_t bd = make_smem_desc(v_base + k * 16 * C::kRowBytes, C::kPanelBytes,
-                                             C::kSbo, C::kSwz);
-          mma_ss(tmem + C::kColO, ad, bd, idesc_o, (jj > 0 || k > 0) ? 1u : 0u);
-        }
-        mma_commit(pv_done);
-        mma_commit(&kv_empty[st]);
-      };
-      bool ok = mbar_wait(q_full, 0, &abort_flag, dev_err);
-      int j = 0;
-      for (; ok && j < n_kv; ++j) {
-        const int st = j % C::kStages;
-        if (!mbar_wait(&kv_full[st], (j / C::kStages) & 1, &abort_flag, dev_err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
         const uint32_t k_base = smem_addr(smem + C::kOffK + st * C::kTileBytes);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const int p = (k * 16) / C::kPanelCols;
           const uint32_t off = p * C::kPanelBytes + ((k * 16) % C::kPanelCols) * 2;
-          const uint64_t ad = make_smem_desc(q_base + off, 16, C::kSbo, C::kSwz);
+          const uint64_t ad = make_smem_desc(q_base + x * C::kTileBytes + off, 16, C::kSbo, C::kSwz);
           const uint64_t bd = make_smem_desc(k_base + off, 16, C::kSbo, C::kSwz);
-          mma_ss(tmem + (j & 1) * kBlockN, ad, bd, idesc_s, k > 0 ? 1u : 0u);
+          mma_ss(tmem + C::col_s(x), ad, bd, idesc_s, k > 0 ? 1u : 0u);
         }
-        mma_commit(&s_full[j & 1]);
-        if (j > 0) {
-          if (!mbar_wait(p_full, (j - 1) & 1, &abort_flag, dev_err)) {
+        mma_commit(&s_full[x]);
+      };
+      auto issue_pv = [&](int x, int jj) {
+        const int st = jj % C::kStages;
+        const uint32_t v_base = smem_addr(smem + C::kOffV + st * C::kTileBytes);
+#pragma unroll
+        for (int k = 0; k < kBlockN / 16; ++k) {
+          // V: MN-major (d contiguous); 16 keys = 16 rows of the swizzle width.
+          const uint64_t bd = make_smem_desc(v_base + k * 16 * C::kRowBytes, C::kPanelBytes,
+                                             C::kSbo, C::kSwz);
+          // P: 16 keys per K step = 8 TMEM columns of bf16 pairs.
+          mma_ts(tmem + C::col_o(x), tmem + C::col_p(x) + k * 8, bd, idesc_o,
+                 (jj > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(&o_done[x]);
+      };
+      bool ok = mbar_wait(q_full, 0, &abort_flag, dev_err) &&
+                mbar_wait(&kv_full[0], 0, &abort_flag, dev_err);
+      if (ok && n_kv > 0) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+      }
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const bool more = j + 1 < n_kv;
+        const int st_next = (j + 1) % C::kStages;
+        if (more && !mbar_wait(&kv_full[st_next], ((j + 1) / C::kStages) & 1, &abort_flag, dev_err))
+          break;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if (!mbar_wait(&p_full[x], j & 1, &abort_flag, dev_err)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          issue_pv(j - 1);
-        }
-      }
-      if (ok && n_kv > 0) {
-        if (mbar_wait(p_full, (n_kv - 1) & 1, &abort_flag, dev_err)) {
-          tc_fence_after();
-          issue_pv(n_kv - 1);
+          issue_pv(x, j);
+          if (x == 1) mma_commit(&kv_empty[j % C::kStages]);
+          if (more) {
+            // S_X(j+1) overwrites the columns P_X(j) is read from: wait for PV_X(j).
+            if (!mbar_wait(&o_done[x], j & 1, &abort_flag, dev_err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(x, j + 1);
+          }
         }
       }
     }
   } else {
     // ------------------------------------------------------------ softmax
+    const int x = (warp - 2) >> 2;                // tile A (0) or B (1)
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;                 // tile row == TMEM lane
-    const int t = t0 + (r >> G_log2);
+    const int t = t0 + x * pos_per_tile + (r >> G_log2);
     const int hl = r & (G - 1);
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const float scale = kLog2e * rsqrtf(static_cast<float>(D));
     float m_used = -INFINITY, l = 0.f;
-    uint8_t* p_tile = smem + C::kOffP;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
-      if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1, &abort_flag, dev_err)) {
+      if (!mbar_wait(&s_full[x], j & 1, &abort_flag, dev_err)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sr[128];
+      float s[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        tmem_ld32(trow + (j & 1) * kBlockN + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        tmem_ld32(trow + C::col_s(x) + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
       tmem_wait_ld();
-      // keys s = j*128 + c are visible when c <= lim
+      // keys j*128 + c are visible when c <= lim
       int lim = S - 1 - j * kBlockN;
       if (causal) lim = min(lim, t - j * kBlockN);
-      float tmax = -INFINITY;
-      float* sf = reinterpret_cast<float*>(sr);
+      if (!__all_sync(0xffffffffu, lim >= kBlockN - 1)) {
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const float v = (c <= lim) ? sf[c] * scale : -INFINITY;
-        sf[c] = v;
-        tmax = fmaxf(tmax, v);
+        for (int c = 0; c < 128; ++c) s[c] = (c <= lim) ? s[c] : -INFINITY;
       }
-      const float m_new = fmaxf(m_used, tmax);
+      float tmax = s[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) tmax = fmaxf(tmax, s[c]);
+      const float m_new = tmax * scale;
       bool need = false;
       float factor = 1.f;
       if (j == 0) {
@@ -245,47 +285,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         m_used = m_new;
         need = true;
       }
-      const float mu = (m_used == -INFINITY) ? 0.f : m_used;
-      uint32_t pk[64];
+      const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = fast_exp2(sf[2 * c] - mu);
-        const float p1 = fast_exp2(sf[2 * c + 1] - mu);
-        l += p0 + p1;
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-        pk[c] = *reinterpret_cast<uint32_t*>(&h2);
-      }
-      if (j > 0) {
-        // O holds P_0..j-1 V: wait for the last PV before rescaling O or
-        // overwriting the P tile it reads.
-        if (!mbar_wait(pv_done, (j - 1) & 1, &abort_flag, dev_err)) {
-          ok = false;
-          break;
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c2 = 0; c2 < 32; ++c2) {
+          const float a0 = fmaf(s[h * 64 + 2 * c2], scale, neg_m);
+          const float a1 = fmaf(s[h * 64 + 2 * c2 + 1], scale, neg_m);
+          const bool soft = (c2 % kSoftExpEvery) == 0;
+          const float p0 = soft ? soft_exp2(a0) : fast_exp2(a0);
+          const float p1 = soft ? soft_exp2(a1) : fast_exp2(a1);
+          l += p0 + p1;
+          pk[c2] = pack_bf16x2(p0, p1);
         }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, need)) {
+        tmem_st32(trow + C::col_p(x) + h * 32, pk);
+      }
+      if (__any_sync(0xffffffffu, need)) {
+        // O_X holds P_0..j-1 V: its last PV completed before S_X(j) was issued.
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(trow + C::kColO + c * 32, o);
-            tmem_wait_ld();
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(trow + C::col_o(x) + c * 32, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-            tmem_st32(trow + C::kColO + c * 32, o);
-          }
-          tmem_wait_st();
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+          tmem_st32(trow + C::col_o(x) + c * 32, o);
         }
       }
-#pragma unroll
-      for (int cc = 0; cc < 16; ++cc) {
-        uint4 v = make_uint4(pk[cc * 4], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
-        *reinterpret_cast<uint4*>(p_tile + (cc >> 3) * 16384 + sw128_offset(r, cc & 7)) = v;
-      }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[x]);
     }
-    if (ok && n_kv > 0 && mbar_wait(pv_done, (n_kv - 1) & 1, &abort_flag, dev_err)) {
+    if (ok && n_kv > 0 && mbar_wait(&o_done[x], (n_kv - 1) & 1, &abort_flag, dev_err)) {
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool store = t < S;
@@ -293,19 +325,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(trow + C::kColO + c * 32, o);
+        tmem_ld32(trow + C::col_o(x) + c * 32, o);
         tmem_wait_ld();
         if (store) {
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint4 pkd;
-            uint32_t* pw = reinterpret_cast<uint32_t*>(&pkd);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[v * 8 + 2 * e]) * inv_l,
-                                                        __uint_as_float(o[v * 8 + 2 * e + 1]) * inv_l);
-              pw[e] = *reinterpret_cast<uint32_t*>(&h2);
-            }
+            pkd.x = pack_bf16x2(__uint_as_float(o[v * 8 + 0]) * inv_l, __uint_as_float(o[v * 8 + 1]) * inv_l);
+            pkd.y = pack_bf16x2(__uint_as_float(o[v * 8 + 2]) * inv_l, __uint_as_float(o[v * 8 + 3]) * inv_l);
+            pkd.z = pack_bf16x2(__uint_as_float(o[v * 8 + 4]) * inv_l, __uint_as_float(o[v * 8 + 5]) * inv_l);
+            pkd.w = pack_bf16x2(__uint_as_float(o[v * 8 + 6]) * inv_l, __uint_as_float(o[v * 8 + 7]) * inv_l);
             *reinterpret_cast<uint4*>(dst + c * 32 + v * 8) = pkd;
           }
         }
@@ -314,6 +343,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 
   if (abort_flag && warp == 1 && lane == 0) {
+    // Do not release TMEM while an MMA might still write it.
     mma_commit(drain);
     const long long t0c = clock64();
     while (!mbar_try_wait(drain, 0) && clock64() - t0c < kWaitLimitCycles) {
@@ -364,11 +394,11 @@ cudaError_t launch_d(const AttnArgs& a, cudaStream_t stream) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
-  const int n_qt = (a.S * a.G + kBlockM - 1) / kBlockM;
-  const int grid = n_qt * a.B * a.Hkv;
+  const int n_pairs = (a.S * a.G + 2 * kBlockM - 1) / (2 * kBlockM);
+  const int grid = n_pairs * a.B * a.Hkv;
   attn_prefill_tc_kernel<D><<<grid, kAttnThreads, C::kSmem, stream>>>(
-      tmQ, tmK, tmV, static_cast<bf16*>(a.out), a.B, a.S, a.Hq, a.Hkv, G_log2, n_qt, a.causal,
-      a.dev_err);
+      tmQ, tmK, tmV, static_cast<bf16*>(a.out), a.B, a.S, a.Hq, a.Hkv, G_log2, n_pairs,
+      a.causal, a.dev_err);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -27,7 +27,7 @@ void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int* 
   if (has_proj) {
     const int tiles = ((N + 127) / 128) * ((B + 63) / 64);
     int es = target / (tiles > 0 ? tiles : 1);
-    const int max_es = (E + 255) / 256;
+    const int max_es = (E + 63) / 64;
     if (es > max_es) es = max_es;
     if (es < 1) es = 1;
     *e_splits = es;
@@ -160,8 +160,10 @@ __global__ void __launch_bounds__(128) decode_pre_kernel(const DecodeArgs<T> a) 
     float val;
     if (a.W) {
       val = 0.f;
-      for (int s = 0; s < a.e_splits; ++s)
-        val += a.proj_part[(static_cast<int64_t>(s) * a.B + b) * a.N + col];
+      const float* pp = a.proj_part + static_cast<int64_t>(b) * a.N + col;
+      const int64_t pstride = static_cast<int64_t>(a.B) * a.N;
+#pragma unroll 8
+      for (int s = 0; s < a.e_splits; ++s) val += __ldcg(pp + s * pstride);
       val = to_f32(from_f32<T>(val));  // the projection output is held in the working dtype
     } else {
       val = to_f32(a.x_t[static_cast<int64_t>(b) * a.N + col]);
@@ -445,21 +447,27 @@ __global__ void __launch_bounds__(kDecThreads)
   __syncthreads();
   if (!last_flag) return;
   __threadfence();
-  // the last CTA of (b, g) merges every split of its G heads
+  // the last CTA of (b, g) merges every split of its G heads in one pass
   const int64_t gbase = (static_cast<int64_t>(b) * a.Hkv + g) * a.splits * G;
   for (int idx = tid; idx < G * D; idx += kDecThreads) {
     const int h = idx / D, i = idx - h * D;
-    float M = -INFINITY;
-    for (int s2 = 0; s2 < a.splits; ++s2)
-      M = fmaxf(M, __ldcg(a.part_ml + (gbase + static_cast<int64_t>(s2) * G + h) * 2));
-    float lsum = 0.f, acc = 0.f;
+    float M = -INFINITY, lsum = 0.f, acc = 0.f;
+#pragma unroll 4
     for (int s2 = 0; s2 < a.splits; ++s2) {
       const int64_t pi = gbase + static_cast<int64_t>(s2) * G + h;
       const float ms = __ldcg(a.part_ml + pi * 2);
+      const float ls = __ldcg(a.part_ml + pi * 2 + 1);
+      const float os = __ldcg(a.part_o + pi * D + i);
       if (ms == -INFINITY) continue;
+      if (ms > M) {
+        const float corr = ex2f(M - ms);   // 0 when M is still -inf
+        lsum *= corr;
+        acc *= corr;
+        M = ms;
+      }
       const float f = ex2f(ms - M);
-      lsum += __ldcg(a.part_ml + pi * 2 + 1) * f;
-      acc += __ldcg(a.part_o + pi * D + i) * f;
+      lsum = fmaf(ls, f, lsum);
+      acc = fmaf(os, f, acc);
     }
     const float val = (valid_b && lsum > 0.f) ? acc / lsum : 0.f;
     a.out[static_cast<int64_t>(b) * a.Hq * D + (g * G + h) * D + i] = from_f32<T>(val);

@@ -5,14 +5,15 @@
 // One CTA owns TT consecutive positions of one kv group (its G query heads, its
 // key head and its value head) of one sequence, so QK-mean, which mixes the
 // group's query heads with its key head, needs no data from other CTAs.
-//   1. the pre-conv q~/k~ rows [t0 - (K-1), t0 + TT) of the group are staged in
-//      shared memory channel-major (the K-1 halo rows come along);
-//   2. per head: the depthwise causal conv over the staged rows, then the
-//      channel mix y = W_h u as a register-tiled (4 positions x 4 channels)
-//      product, QK-mean from the staged pre-conv rows, RoPE from a per-CTA
-//      cos/sin table, one store;
+//   1. the group's q~ | k~ | v~ rows [t0 - HALO, t0 + TT) are copied into
+//      shared memory with 16-byte cp.async (raw working dtype; the halo rows
+//      feed the causal conv and the value-shift);
+//   2. per head: the depthwise causal conv, one thread per channel sliding a
+//      K-tap register window down its rows, then the channel mix y = W_h u as
+//      a register-tiled (4 positions x 4 channels) product, QK-mean from the
+//      staged pre-conv rows, RoPE from a per-CTA cos/sin table, one store;
 //   3. value-shift: upper half-channels of each value head come from the
-//      previous position -- a bit-exact copy;
+//      previous position -- a bit-exact copy out of shared memory;
 //   4. the CTA holding the last position writes the decode state.
 // All arithmetic in fp32; inputs and outputs in the working dtype.
 #include "kernels.h"
@@ -25,24 +26,25 @@ constexpr int kPreThreads = 256;
 __host__ __device__ inline int round4(int x) { return (x + 3) & ~3; }
 
 struct PreLayout {
-  int TT, KH, ZS, US;
-  int off_z, off_u, off_w, off_cs, off_theta;  // in floats
-  size_t bytes;
+  int TT, KH, HALO, R, ZC, US;
+  int off_u, off_w, off_cs, off_theta;  // in floats, after the z tile
+  size_t z_bytes, bytes;
 };
 
-__host__ __device__ inline PreLayout pre_layout(int TT, int K, int G, int d) {
+__host__ __device__ inline PreLayout pre_layout(int TT, int K, int G, int d, int es) {
   PreLayout L;
   L.TT = TT;
   L.KH = K > 0 ? K - 1 : 0;
-  L.ZS = (TT + L.KH) | 1;  // odd row stride: channel-major writes avoid bank conflicts
-  L.US = TT + 4;           // multiple of 4 for float4 reads
-  const int HC = (G + 1) * d;
-  L.off_z = 0;
-  L.off_u = round4(HC * L.ZS);
+  L.HALO = L.KH > 1 ? L.KH : 1;   // at least one row back for the value-shift
+  L.R = TT + L.HALO;
+  L.ZC = (G + 2) * d + 16 / es;   // q | k | v channels + one 16-byte pad
+  L.US = TT + 4;                  // multiple of 4 for float4 reads
+  L.z_bytes = (static_cast<size_t>(L.R) * L.ZC * es + 15) & ~size_t(15);
+  L.off_u = 0;
   L.off_w = L.off_u + round4(d * L.US);
   L.off_cs = L.off_w + round4(d * d);
-  L.off_theta = L.off_cs + round4(TT * d);  // cs holds TT * d/2 float2
-  L.bytes = static_cast<size_t>(L.off_theta) * 4 + static_cast<size_t>(d / 2) * 8 + 16;
+  L.off_theta = L.off_cs + round4(TT * d);  // cs: TT * d/2 float2
+  L.bytes = L.z_bytes + static_cast<size_t>(L.off_theta) * 4 + static_cast<size_t>(d / 2) * 8 + 16;
   return L;
 }
 
@@ -56,43 +58,75 @@ template <> struct Vec2<bf16> {
   __device__ static type make(float a, float b) { return __floats2bfloat162_rn(a, b); }
 };
 
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kPreThreads)
     pre_attn_kernel(const PreAttnArgs<T> a, const int TT) {
   extern __shared__ float4 smem_f4[];
-  float* sm = reinterpret_cast<float*>(smem_f4);
+  uint8_t* smem = reinterpret_cast<uint8_t*>(smem_f4);
   const int b = blockIdx.z, g = blockIdx.y, t0 = blockIdx.x * TT;
   const int d = a.d, G = a.G, K = a.K, S = a.S;
   const int half = d / 2;
-  const PreLayout L = pre_layout(TT, K, G, d);
-  float* zT = sm + L.off_z;
-  float* u = sm + L.off_u;
-  float* Wt = sm + L.off_w;
-  float2* cs = reinterpret_cast<float2*>(sm + L.off_cs);
-  double* theta = reinterpret_cast<double*>(sm + L.off_theta);
-  const int KH = L.KH, ZS = L.ZS, US = L.US;
-  const int HC = (G + 1) * d;
+  const PreLayout L = pre_layout(TT, K, G, d, sizeof(T));
+  T* z = reinterpret_cast<T*>(smem);                      // [R][ZC]: q | k | v
+  float* fs = reinterpret_cast<float*>(smem + L.z_bytes);
+  float* u = fs + L.off_u;                                // [d][US]
+  float* Wt = fs + L.off_w;                               // [d][d] transposed
+  float2* cs = reinterpret_cast<float2*>(fs + L.off_cs);  // [TT][d/2]
+  double* theta = reinterpret_cast<double*>(fs + L.off_theta);
+  const int HALO = L.HALO, ZC = L.ZC, US = L.US, R = L.R;
   const int tid = threadIdx.x;
   const int64_t ld = a.src_ld;
   const T* src_b = a.src + static_cast<int64_t>(b) * S * ld;
-  const int qcol0 = g * G * d;
+  const int QC = G * d;                   // q channels of the group
+  const int qcol0 = g * QC;
   const int kcol0 = a.Hq * d + g * d;
   const int vcol0 = (a.Hq + a.Hkv) * d + g * d;
 
-  // 1. stage pre-conv rows t0-KH .. t0+TT-1 (zero outside [0, S)).
-  const int R = TT + KH;
-  for (int idx = tid; idx < R * HC; idx += kPreThreads) {
-    const int r = idx / HC, c = idx - r * HC;
-    const int t = t0 - KH + r;
-    const int col = c < G * d ? qcol0 + c : kcol0 + (c - G * d);
-    zT[c * ZS + r] = (t >= 0 && t < S) ? to_f32(src_b[static_cast<int64_t>(t) * ld + col]) : 0.f;
+  // 1. stage rows t0-HALO .. t0+TT-1 of the group's q | k | v channels.
+  {
+    constexpr int VEC = 16 / sizeof(T);
+    const int cq = QC / VEC, ck = d / VEC;            // 16-byte chunks per block
+    const int per_row = cq + 2 * ck;
+    for (int idx = tid; idx < R * per_row; idx += kPreThreads) {
+      const int r = idx / per_row;
+      const int c = idx - r * per_row;
+      const int t = t0 - HALO + r;
+      int col, zc;
+      if (c < cq) {
+        col = qcol0 + c * VEC;
+        zc = c * VEC;
+      } else if (c < cq + ck) {
+        col = kcol0 + (c - cq) * VEC;
+        zc = QC + (c - cq) * VEC;
+      } else {
+        col = vcol0 + (c - cq - ck) * VEC;
+        zc = QC + d + (c - cq - ck) * VEC;
+      }
+      T* dst = z + r * ZC + zc;
+      if (t >= 0 && t < S)
+        cp_async16(dst, src_b + static_cast<int64_t>(t) * ld + col);
+      else
+        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+    }
   }
-  // 2. RoPE table: pair i turns by t * base^(-2i/d).  The angle is formed and
-  // reduced modulo one turn in fp64, so long positions keep full precision.
+  // 2. RoPE table while the copies fly: pair i turns by t * base^(-2i/d).  The
+  // angle is formed and reduced modulo one turn in fp64, so long positions
+  // keep full precision.
   if (a.rope_on) {
     for (int i = tid; i < half; i += kPreThreads)
       theta[i] = exp2(-(2.0 * i / d) * a.rope_log2_base);
   }
+  cp_async_wait_all();
   __syncthreads();
   if (a.rope_on) {
     const double inv_turn = 0.15915494309189533577;  // 1 / (2 pi)
@@ -107,25 +141,43 @@ __global__ void __launch_bounds__(kPreThreads)
   }
 
   // 3. per head of the group: G query heads, then the key head.
+  constexpr int SEG = 8;                 // rows per conv thread
+  const int n_seg = TT / SEG;
   for (int hh = 0; hh <= G; ++hh) {
     const bool is_q = hh < G;
     const int head = is_q ? g * G + hh : g;
-    const T* wseq = K > 0 ? (is_q ? a.wq_seq : a.wk_seq) + static_cast<int64_t>(head) * d * K
-                          : nullptr;
+    const int cb = hh * d;               // channel offset inside the z tile
     const T* wch_base = is_q ? a.wq_chan : a.wk_chan;
     const T* wch = (K > 0 && wch_base) ? wch_base + static_cast<int64_t>(head) * d * d : nullptr;
-    const int cb = hh * d;
-    for (int idx = tid; idx < d * TT; idx += kPreThreads) {
-      const int j = idx / TT, tl = idx - j * TT;
-      const float* zr = zT + (cb + j) * ZS + tl + KH;
-      float acc;
+    // causal depthwise conv: thread = (channel, 8-row segment), taps in registers
+    for (int idx = tid; idx < d * n_seg; idx += kPreThreads) {
+      const int j = idx % d, sg = idx / d;
+      const int tl0 = sg * SEG;
+      const T* zc = z + cb + j;
       if (K > 0) {
-        acc = 0.f;
-        for (int jj = 0; jj < K; ++jj) acc = fmaf(to_f32(wseq[j * K + jj]), zr[-jj], acc);
+        const T* w = (is_q ? a.wq_seq : a.wk_seq) + static_cast<int64_t>(head * d + j) * K;
+        float wr[4] = {0.f, 0.f, 0.f, 0.f};
+        float win[4] = {0.f, 0.f, 0.f, 0.f};   // win[k] = row tl - k
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (k < K) wr[k] = to_f32(w[k]);
+#pragma unroll
+        for (int k = 1; k < 4; ++k)
+          if (k < K) win[k] = to_f32(zc[(tl0 + HALO - k) * ZC]);
+#pragma unroll
+        for (int s = 0; s < SEG; ++s) {
+          win[0] = to_f32(zc[(tl0 + s + HALO) * ZC]);
+          float acc = wr[0] * win[0];
+#pragma unroll
+          for (int k = 1; k < 4; ++k) acc = fmaf(wr[k], win[k], acc);
+          u[j * US + tl0 + s] = acc;
+#pragma unroll
+          for (int k = 3; k > 0; --k) win[k] = win[k - 1];
+        }
       } else {
-        acc = zr[0];
+#pragma unroll
+        for (int s = 0; s < SEG; ++s) u[j * US + tl0 + s] = to_f32(zc[(tl0 + s + HALO) * ZC]);
       }
-      u[j * US + tl] = acc;
     }
     if (wch) {
       for (int idx = tid; idx < d * d; idx += kPreThreads) {
@@ -174,17 +226,17 @@ __global__ void __launch_bounds__(kPreThreads)
       for (int r = 0; r < 4; ++r) {
         const int tl = tl0 + r, t = t0 + tl;
         if (t >= S) continue;
-        const int zrow = tl + KH;
+        const T* zrow = z + (tl + HALO) * ZC;
         if (a.qk_mean) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const float kp = zT[(G * d + ch[k]) * ZS + zrow];
+            const float kp = to_f32(zrow[QC + ch[k]]);
             float qp;
             if (is_q) {
-              qp = zT[(hh * d + ch[k]) * ZS + zrow];
+              qp = to_f32(zrow[hh * d + ch[k]]);
             } else {
               qp = 0.f;
-              for (int hl = 0; hl < G; ++hl) qp += zT[(hl * d + ch[k]) * ZS + zrow];
+              for (int hl = 0; hl < G; ++hl) qp += to_f32(zrow[hl * d + ch[k]]);
               qp /= static_cast<float>(G);
             }
             y[r][k] += 0.5f * (qp + kp);
@@ -215,34 +267,29 @@ __global__ void __launch_bounds__(kPreThreads)
     const int tl = idx / nchunk, i = (idx - tl * nchunk) * VEC;
     const int t = t0 + tl;
     if (t >= S) continue;
-    const bool from_prev = a.value_shift && i >= half;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    const int ts = from_prev ? t - 1 : t;
-    if (ts >= 0)
-      val = *reinterpret_cast<const uint4*>(src_b + static_cast<int64_t>(ts) * ld + vcol0 + i);
+    const int row = (a.value_shift && i >= half) ? tl + HALO - 1 : tl + HALO;
+    const uint4 val = *reinterpret_cast<const uint4*>(z + row * ZC + QC + d + i);
     *reinterpret_cast<uint4*>(a.v_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + t) * d +
                               i) = val;
   }
 
-  // 5. decode state, written by the CTA that holds position S-1.
+  // 5. decode state, written by the CTA that holds position S-1 (its rows
+  // S-KH .. S-1 are all staged; rows before position 0 are zero).
   if (a.len != nullptr && t0 <= S - 1 && S - 1 < t0 + TT) {
-    const int Hq = a.Hq, Hkv = a.Hkv;
+    const int KH = L.KH, Hq = a.Hq, Hkv = a.Hkv;
     for (int r = 0; r < KH; ++r) {
-      const int srow = S - KH + r;
-      for (int c = tid; c < G * d + d; c += kPreThreads) {
-        const bool q = c < G * d;
-        const int col = q ? qcol0 + c : kcol0 + (c - G * d);
-        const T val = srow >= 0 ? src_b[static_cast<int64_t>(srow) * ld + col] : from_f32<T>(0.f);
-        if (q)
-          a.hist_q[(static_cast<int64_t>(b) * KH + r) * Hq * d + qcol0 + c] = val;
+      const T* zrow = z + (S - KH + r - t0 + HALO) * ZC;
+      for (int c = tid; c < QC + d; c += kPreThreads) {
+        if (c < QC)
+          a.hist_q[(static_cast<int64_t>(b) * KH + r) * Hq * d + qcol0 + c] = zrow[c];
         else
-          a.hist_k[(static_cast<int64_t>(b) * KH + r) * Hkv * d + g * d + (c - G * d)] = val;
+          a.hist_k[(static_cast<int64_t>(b) * KH + r) * Hkv * d + g * d + (c - QC)] = zrow[c];
       }
     }
     if (a.v_prev) {
+      const T* zrow = z + (S - 1 - t0 + HALO) * ZC;
       for (int i = tid; i < d; i += kPreThreads)
-        a.v_prev[static_cast<int64_t>(b) * Hkv * d + g * d + i] =
-            src_b[static_cast<int64_t>(S - 1) * ld + vcol0 + i];
+        a.v_prev[static_cast<int64_t>(b) * Hkv * d + g * d + i] = zrow[QC + d + i];
     }
     if (g == 0 && tid == 0) a.len[b] = S;
   }
@@ -256,8 +303,9 @@ cudaError_t launch_pre_attn(const PreAttnArgs<T>& a, cudaStream_t stream) {
   // thread in the channel mix; halve TT while the staging does not fit.
   int TT = 4096 / a.d;
   if (TT > 256) TT = 256;
-  while (TT > 4 && pre_layout(TT, a.K, a.G, a.d).bytes > 200 * 1024) TT /= 2;
-  const PreLayout L = pre_layout(TT, a.K, a.G, a.d);
+  const int es = sizeof(T);
+  while (TT > 8 && pre_layout(TT, a.K, a.G, a.d, es).bytes > 200 * 1024) TT /= 2;
+  const PreLayout L = pre_layout(TT, a.K, a.G, a.d, es);
   if (L.bytes > 227 * 1024) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(pre_attn_kernel<T>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
