@@ -44,7 +44,10 @@ class ccgqa_kvcache(ctypes.Structure):
 class CCGQAError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {STATUS.get(status, status)} ({_status_string(status)})")
+        msg = f"{where}: {STATUS.get(status, status)} ({_status_string(status)})"
+        if status == 5:
+            msg += f" [{ccgqa_last_error_string()}]"
+        super().__init__(msg)
 
 
 _lib = None
@@ -79,6 +82,8 @@ def load() -> ctypes.CDLL:
     lib.ccgqa_status_string.restype = c_char_p
     lib.ccgqa_launch_count.argtypes = []
     lib.ccgqa_launch_count.restype = c_uint64
+    lib.ccgqa_last_error_string.argtypes = []
+    lib.ccgqa_last_error_string.restype = c_char_p
     lib.ccgqa_set_phase_events.argtypes = [c_void_p, c_int32]
     lib.ccgqa_set_phase_events.restype = None
     _lib = lib
@@ -179,6 +184,10 @@ def ccgqa_kvcache_append(cfg, cache, k_new, v_new, n_new, dev_err=None, stream=N
 
 def ccgqa_status_string(status: int) -> str:
     return load().ccgqa_status_string(status).decode()
+
+
+def ccgqa_last_error_string() -> str:
+    return load().ccgqa_last_error_string().decode()
 
 
 def ccgqa_launch_count() -> int:

@@ -3,6 +3,7 @@
 // launch and returns a status; the kernels themselves never trap.
 #include <atomic>
 #include <cmath>
+#include <cstdio>
 
 #include "kernels.h"
 
@@ -10,6 +11,13 @@ namespace ccgqa {
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+
+// Last CUDA error met by an entry point on this thread.
+static thread_local char t_last_error[256] = "no error";
+static ccgqa_status cuda_fail(cudaError_t e) {
+  snprintf(t_last_error, sizeof(t_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+  return CCGQA_ERR_CUDA;
+}
 
 // Optional phase events of the calling thread (ccgqa_set_phase_events).
 static thread_local void* const* t_phase_events = nullptr;
@@ -145,7 +153,7 @@ ccgqa_status run_prefill(const Geo& g, const ccgqa_weights* w, const void* x, in
     else
       e = launch_proj_gemm_f32(static_cast<const float*>(x), static_cast<const float*>(w->W_qkv),
                                proj, B * S, g.N, g.E, st);
-    if (e != cudaSuccess) return CCGQA_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_fail(e);
     src = proj;
   }
   phase_mark(1, st);
@@ -182,7 +190,7 @@ ccgqa_status run_prefill(const Geo& g, const ccgqa_weights* w, const void* x, in
     a.kv_cap = S;
   }
   a.dev_err = dev_err;
-  if (launch_pre_attn<T>(a, st) != cudaSuccess) return CCGQA_ERR_CUDA;
+  if ((e = launch_pre_attn<T>(a, st)) != cudaSuccess) return cuda_fail(e);
   phase_mark(2, st);
   AttnArgs at{};
   at.q = a.q_out;
@@ -203,7 +211,7 @@ ccgqa_status run_prefill(const Geo& g, const ccgqa_weights* w, const void* x, in
   else
     e = launch_attn_prefill_simt<T>(at, st);
   phase_mark(3, st);
-  return e == cudaSuccess ? CCGQA_OK : CCGQA_ERR_CUDA;
+  return e == cudaSuccess ? CCGQA_OK : cuda_fail(e);
 }
 
 template <typename T>
@@ -249,7 +257,8 @@ ccgqa_status run_decode(const Geo& g, const ccgqa_weights* w, const void* x_t,
   a.chunk = L.chunk;
   a.dev_err = dev_err;
   a.phase_events = t_phase_events;
-  return launch_decode_step<T>(a, st) == cudaSuccess ? CCGQA_OK : CCGQA_ERR_CUDA;
+  const cudaError_t e = launch_decode_step<T>(a, st);
+  return e == cudaSuccess ? CCGQA_OK : cuda_fail(e);
 }
 
 }  // namespace
@@ -341,7 +350,7 @@ CCGQA_API ccgqa_status ccgqa_kvcache_append(const ccgqa_config* cfg, const ccgqa
                                 cache->len, static_cast<const float*>(k_new),
                                 static_cast<const float*>(v_new), cache->batch, g.Hkv, g.d,
                                 cache->cap, n_new, dev_err, st);
-  return e == cudaSuccess ? CCGQA_OK : CCGQA_ERR_CUDA;
+  return e == cudaSuccess ? CCGQA_OK : cuda_fail(e);
 }
 
 CCGQA_API const char* ccgqa_status_string(ccgqa_status s) {
@@ -357,6 +366,8 @@ CCGQA_API const char* ccgqa_status_string(ccgqa_status s) {
 }
 
 CCGQA_API uint64_t ccgqa_launch_count(void) { return g_launches.load(); }
+
+CCGQA_API const char* ccgqa_last_error_string(void) { return t_last_error; }
 
 CCGQA_API void ccgqa_set_phase_events(void* const* events, int32_t n) {
   t_phase_events = (events != nullptr && n >= 4) ? events : nullptr;

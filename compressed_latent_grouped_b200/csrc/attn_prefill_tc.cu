@@ -8,20 +8,26 @@
 // q[B, S, Hq, d] and one K/V tile in shared memory serves all G query heads.
 //
 // One CTA owns two 128-row query tiles (A and B) of one kv group and streams
-// the K/V tiles both need once:
+// the K/V tiles both need once, as 128-key tiles split into two 64-key halves:
 //   warp 0      TMA producer: Q_A, Q_B once, then K/V tiles of 128 keys
 //               through a ring of shared-memory stages
-//   warp 1      TMEM allocator; one elected thread issues every tcgen05.mma:
-//                 S_X = Q_X K_j^T  (SS, M=128 N=128, fp32 accumulators in TMEM)
-//                 O_X += P_X V_j   (TS: P read from TMEM, V from shared memory)
-//   warps 2-5   softmax of tile A, warps 6-9 softmax of tile B: one thread per
+//   warps 1, 2  one thread each issues the tcgen05.mma of tile A / tile B
+//               (warp 1 also owns the TMEM allocation):
+//                 S_X = Q_X K_h^T  (SS, M=128 N=64, fp32 accumulators in TMEM)
+//                 O_X += P_X V_h   (TS: P read from TMEM, V from shared memory)
+//               With one issuer per tile, waiting for one tile's PV never
+//               delays the other tile's MMAs.
+//   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: one thread per
 //               row (TMEM lane); tcgen05.ld of S, running max / sum in
 //               registers, P written back to TMEM as bf16 pairs in the upper
-//               half of the S columns, O rescaled in TMEM when the running max
+//               half of its S buffer, O rescaled in TMEM when the running max
 //               grows by more than 2^8, normalised O stored at the end.
-// While one warpgroup exponentiates, the tensor core runs the other tile's
-// MMAs, so the exp unit, the FMA pipe and the tensor pipe overlap.  No cluster
-// multicast is used; every wait is bounded.
+// Each tile has two S buffers (one per 64-key half), so the S of the next half
+// is computed while the softmax works on the current one and a softmax
+// warpgroup never waits for the PV -> S round trip; the two warpgroups keep
+// the exp unit and the FMA pipe busy while the tensor core runs their MMAs.
+// TMEM: S/P of tile X at columns 128 X + {0, 64}, O_X at 256 + X d (d <= 128).
+// No cluster multicast is used; every wait is bounded.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -30,8 +36,8 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kAttnThreads = 320;
-constexpr int kBlockM = 128, kBlockN = 128;
+constexpr int kAttnThreads = 384;
+constexpr int kBlockM = 128, kBlockN = 128, kHalfN = 64;
 constexpr float kLog2e = 1.4426950408889634f;
 // The running max used for exp2 is only raised when it falls behind by more
 // than this many doublings, so P <= 2^8 and O is rescaled rarely.
@@ -53,9 +59,10 @@ struct Cfg {
   static constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
   static constexpr size_t kSmem = kOffBar + 256 + 1024;
   static constexpr uint32_t kTmemCols = 512;
-  __device__ static constexpr uint32_t col_s(int x) { return x * 128; }       // S_A | S_B
-  __device__ static constexpr uint32_t col_p(int x) { return x * 128 + 64; }  // P in S's upper half
-  __device__ static constexpr uint32_t col_o(int x) { return 256 + x * D; }   // O_A | O_B
+  // S buffer h of tile x, its P (upper 32 columns: 64 keys as bf16 pairs), O_x
+  __device__ static constexpr uint32_t col_s(int x, int h) { return x * 128 + h * 64; }
+  __device__ static constexpr uint32_t col_p(int x, int h) { return x * 128 + h * 64 + 32; }
+  __device__ static constexpr uint32_t col_o(int x) { return 256 + x * D; }
 };
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -81,8 +88,45 @@ __device__ __forceinline__ float soft_exp2(float x) {
   return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
-// Pairs (c2 % 4 == 0) of each softmax row use soft_exp2: one element in four.
-constexpr int kSoftExpEvery = 4;
+// Packed fp32 pairs (one instruction for two lanes' worth of FMA-pipe work).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)),
+        "l"(*reinterpret_cast<const uint64_t*>(&c)));
+  return *reinterpret_cast<float2*>(&d);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)));
+  return *reinterpret_cast<float2*>(&d);
+}
+
+// soft_exp2 on a pair, with the FMA-pipe steps packed.
+__device__ __forceinline__ float2 soft_exp2x2(float2 x) {
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 big = make_float2(12582912.0f, 12582912.0f);
+  const float2 t = fadd2(x, big);
+  const float2 n = fadd2(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = ffma2(n, make_float2(-1.0f, -1.0f), x);
+  float2 p = ffma2(make_float2(0.05521968f, 0.05521968f), f, make_float2(0.24260941f, 0.24260941f));
+  p = ffma2(p, f, make_float2(0.69325167f, 0.69325167f));
+  p = ffma2(p, f, make_float2(0.99992800f, 0.99992800f));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// Pairs (c2 % kSoftExpEvery == 0) of each softmax row use the software exp2.
+// Measured on B200: while the softmax is latency-bound the extra instructions
+// cost more than the exp unit time they save, so it is off by default.
+#ifndef CCGQA_SOFT_EXP_EVERY
+#define CCGQA_SOFT_EXP_EVERY 1000000
+#endif
+constexpr int kSoftExpEvery = CCGQA_SOFT_EXP_EVERY;
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h2 = __floats2bfloat162_rn(lo, hi);
@@ -104,10 +148,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;                  // [kStages]
   uint64_t* kv_empty = kv_full + C::kStages;     // [kStages]
-  uint64_t* s_full = kv_empty + C::kStages;      // [2]  S_X ready
-  uint64_t* p_full = s_full + 2;                 // [2]  P_X written (128 arrivals)
-  uint64_t* o_done = p_full + 2;                 // [2]  PV_X complete
-  uint64_t* drain = o_done + 2;
+  uint64_t* s_full = kv_empty + C::kStages;      // [2 tiles][2 halves]  S ready
+  uint64_t* p_full = s_full + 4;                 // [2][2]  P written (128 arrivals)
+  uint64_t* o_done = p_full + 4;                 // [2][2]  PV of that half complete
+  uint64_t* drain = o_done + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   __shared__ int abort_flag;
 
@@ -126,14 +170,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(q_full, 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], 2);   // released by both tiles' last PV of the stage
     }
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(&s_full[x], 1);
-      mbar_init(&p_full[x], 128);
-      mbar_init(&o_done[x], 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&o_done[i], 1);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, 2);   // one commit from each MMA issuer
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -173,151 +217,178 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    // Order: S_A(0) S_B(0) | PV_A(j) S_A(j+1) PV_B(j) S_B(j+1) | ...
-    // S_X(j+1) follows PV_X(j) directly, so tile A's next softmax can start
-    // while tile B's softmax is still running (the two warpgroups alternate).
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
+    // Tile x = warp - 1.  Per K/V tile j and half h: PV_x(j,h), then
+    // S_x(j+1,h) into the buffer P_x(j,h) was read from (after that PV
+    // completes); the softmax is meanwhile busy with the other half.
     if (lane == 0) {
-      const uint32_t idesc_s = make_idesc_bf16(kBlockM, kBlockN, false);
+      const int x = warp - 1;
+      const uint32_t idesc_s = make_idesc_bf16(kBlockM, kHalfN, false);
       const uint32_t idesc_o = make_idesc_bf16(kBlockM, D, true);
-      const uint32_t q_base = smem_addr(smem + C::kOffQ);
-      auto issue_s = [&](int x, int jj) {
+      const uint32_t q_base = smem_addr(smem + C::kOffQ) + x * C::kTileBytes;
+      auto issue_s = [&](int jj, int h) {
         const int st = jj % C::kStages;
-        const uint32_t k_base = smem_addr(smem + C::kOffK + st * C::kTileBytes);
+        const uint32_t k_base =
+            smem_addr(smem + C::kOffK + st * C::kTileBytes) + h * kHalfN * C::kRowBytes;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const int p = (k * 16) / C::kPanelCols;
           const uint32_t off = p * C::kPanelBytes + ((k * 16) % C::kPanelCols) * 2;
-          const uint64_t ad = make_smem_desc(q_base + x * C::kTileBytes + off, 16, C::kSbo, C::kSwz);
+          const uint64_t ad = make_smem_desc(q_base + off, 16, C::kSbo, C::kSwz);
           const uint64_t bd = make_smem_desc(k_base + off, 16, C::kSbo, C::kSwz);
-          mma_ss(tmem + C::col_s(x), ad, bd, idesc_s, k > 0 ? 1u : 0u);
+          mma_ss(tmem + C::col_s(x, h), ad, bd, idesc_s, k > 0 ? 1u : 0u);
         }
-        mma_commit(&s_full[x]);
+        mma_commit(&s_full[x * 2 + h]);
       };
-      auto issue_pv = [&](int x, int jj) {
+      auto issue_pv = [&](int jj, int h) {
         const int st = jj % C::kStages;
-        const uint32_t v_base = smem_addr(smem + C::kOffV + st * C::kTileBytes);
+        const uint32_t v_base =
+            smem_addr(smem + C::kOffV + st * C::kTileBytes) + h * kHalfN * C::kRowBytes;
 #pragma unroll
-        for (int k = 0; k < kBlockN / 16; ++k) {
+        for (int k = 0; k < kHalfN / 16; ++k) {
           // V: MN-major (d contiguous); 16 keys = 16 rows of the swizzle width.
           const uint64_t bd = make_smem_desc(v_base + k * 16 * C::kRowBytes, C::kPanelBytes,
                                              C::kSbo, C::kSwz);
           // P: 16 keys per K step = 8 TMEM columns of bf16 pairs.
-          mma_ts(tmem + C::col_o(x), tmem + C::col_p(x) + k * 8, bd, idesc_o,
-                 (jj > 0 || k > 0) ? 1u : 0u);
+          mma_ts(tmem + C::col_o(x), tmem + C::col_p(x, h) + k * 8, bd, idesc_o,
+                 (jj > 0 || h > 0 || k > 0) ? 1u : 0u);
         }
-        mma_commit(&o_done[x]);
+        mma_commit(&o_done[x * 2 + h]);
       };
       bool ok = mbar_wait(q_full, 0, &abort_flag, dev_err) &&
                 mbar_wait(&kv_full[0], 0, &abort_flag, dev_err);
       if (ok && n_kv > 0) {
         tc_fence_after();
         issue_s(0, 0);
-        issue_s(1, 0);
+        issue_s(0, 1);
       }
       for (int j = 0; ok && j < n_kv; ++j) {
         const bool more = j + 1 < n_kv;
-        const int st_next = (j + 1) % C::kStages;
-        if (more && !mbar_wait(&kv_full[st_next], ((j + 1) / C::kStages) & 1, &abort_flag, dev_err))
-          break;
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          if (!mbar_wait(&p_full[x], j & 1, &abort_flag, dev_err)) {
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait(&p_full[x * 2 + h], j & 1, &abort_flag, dev_err)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          issue_pv(x, j);
-          if (x == 1) mma_commit(&kv_empty[j % C::kStages]);
+          issue_pv(j, h);
+          if (h == 1) mma_commit(&kv_empty[j % C::kStages]);
           if (more) {
-            // S_X(j+1) overwrites the columns P_X(j) is read from: wait for PV_X(j).
-            if (!mbar_wait(&o_done[x], j & 1, &abort_flag, dev_err)) {
+            if (h == 0 && !mbar_wait(&kv_full[(j + 1) % C::kStages], ((j + 1) / C::kStages) & 1,
+                                     &abort_flag, dev_err)) {
+              ok = false;
+              break;
+            }
+            if (!mbar_wait(&o_done[x * 2 + h], j & 1, &abort_flag, dev_err)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            issue_s(x, j + 1);
+            issue_s(j + 1, h);
           }
         }
       }
     }
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
-    const int x = (warp - 2) >> 2;                // tile A (0) or B (1)
+    const int x = (warp - 4) >> 2;                // tile A (0) or B (1)
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;                 // tile row == TMEM lane
     const int t = t0 + x * pos_per_tile + (r >> G_log2);
     const int hl = r & (G - 1);
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const float scale = kLog2e * rsqrtf(static_cast<float>(D));
+    const float2 scale2 = make_float2(scale, scale);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      if (!mbar_wait(&s_full[x], j & 1, &abort_flag, dev_err)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float s[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld32(trow + C::col_s(x) + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
-      tmem_wait_ld();
-      // keys j*128 + c are visible when c <= lim
-      int lim = S - 1 - j * kBlockN;
-      if (causal) lim = min(lim, t - j * kBlockN);
-      if (!__all_sync(0xffffffffu, lim >= kBlockN - 1)) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = (c <= lim) ? s[c] : -INFINITY;
-      }
-      float tmax = s[0];
-#pragma unroll
-      for (int c = 1; c < 128; ++c) tmax = fmaxf(tmax, s[c]);
-      const float m_new = tmax * scale;
-      bool need = false;
-      float factor = 1.f;
-      if (j == 0) {
-        m_used = m_new;
-      } else if (m_new > m_used + kRescaleThreshold) {
-        factor = fast_exp2(m_used - m_new);
-        l *= factor;
-        m_used = m_new;
-        need = true;
-      }
-      const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
-#pragma unroll
+    for (int j = 0; ok && j < n_kv; ++j) {
       for (int h = 0; h < 2; ++h) {
+        const int sb = x * 2 + h;
+        if (!mbar_wait(&s_full[sb], j & 1, &abort_flag, dev_err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float s[64];
+        tmem_ld32(trow + C::col_s(x, h), *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        tmem_ld32(trow + C::col_s(x, h) + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+        tmem_wait_ld();
+        // keys j*128 + h*64 + c are visible when c <= lim
+        const int kb = j * kBlockN + h * kHalfN;
+        int lim = S - 1 - kb;
+        if (causal) lim = min(lim, t - kb);
+        if (!__all_sync(0xffffffffu, lim >= kHalfN - 1)) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s[c] = (c <= lim) ? s[c] : -INFINITY;
+        }
+        float mx[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = s[k];
+#pragma unroll
+        for (int c = 8; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) mx[k] = fmaxf(mx[k], mx[k + 4]);
+        const float m_new = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * scale;
+        bool need = false;
+        float factor = 1.f;
+        if (j == 0 && h == 0) {
+          m_used = m_new;
+        } else if (m_new > m_used + kRescaleThreshold) {
+          factor = fast_exp2(m_used - m_new);
+          l *= factor;
+          m_used = m_new;
+          need = true;
+        }
+        const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
+        const float2 negm2 = make_float2(neg_m, neg_m);
+        float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                          make_float2(0.f, 0.f)};
+        const float2* s2 = reinterpret_cast<const float2*>(s);
         uint32_t pk[32];
 #pragma unroll
         for (int c2 = 0; c2 < 32; ++c2) {
-          const float a0 = fmaf(s[h * 64 + 2 * c2], scale, neg_m);
-          const float a1 = fmaf(s[h * 64 + 2 * c2 + 1], scale, neg_m);
-          const bool soft = (c2 % kSoftExpEvery) == 0;
-          const float p0 = soft ? soft_exp2(a0) : fast_exp2(a0);
-          const float p1 = soft ? soft_exp2(a1) : fast_exp2(a1);
-          l += p0 + p1;
-          pk[c2] = pack_bf16x2(p0, p1);
+          const float2 arg = ffma2(s2[c2], scale2, negm2);
+          float2 p;
+          if ((c2 % kSoftExpEvery) == 0) {
+            p = soft_exp2x2(arg);
+          } else {
+            p.x = fast_exp2(arg.x);
+            p.y = fast_exp2(arg.y);
+          }
+          lsum[c2 & 3] = fadd2(lsum[c2 & 3], p);
+          pk[c2] = pack_bf16x2(p.x, p.y);
         }
-        tmem_st32(trow + C::col_p(x) + h * 32, pk);
-      }
-      if (__any_sync(0xffffffffu, need)) {
-        // O_X holds P_0..j-1 V: its last PV completed before S_X(j) was issued.
+        {
+          const float2 a2 = fadd2(fadd2(lsum[0], lsum[1]), fadd2(lsum[2], lsum[3]));
+          l += a2.x + a2.y;
+        }
+        if (__any_sync(0xffffffffu, need)) {
+          // O must hold every earlier half: wait for the previous PV of this tile.
+          const int pb = x * 2 + (1 - h);
+          const uint32_t pph = (h == 1 ? j : j - 1) & 1;
+          if (!mbar_wait(&o_done[pb], pph, &abort_flag, dev_err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(trow + C::col_o(x) + c * 32, o);
-          tmem_wait_ld();
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(trow + C::col_o(x) + c * 32, o);
+            tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-          tmem_st32(trow + C::col_o(x) + c * 32, o);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+            tmem_st32(trow + C::col_o(x) + c * 32, o);
+          }
         }
+        tmem_st32(trow + C::col_p(x, h), pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[sb]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&p_full[x]);
     }
-    if (ok && n_kv > 0 && mbar_wait(&o_done[x], (n_kv - 1) & 1, &abort_flag, dev_err)) {
+    // the last PV of this tile (half 1 of tile n_kv-1) completes after all others
+    if (ok && n_kv > 0 && mbar_wait(&o_done[x * 2 + 1], (n_kv - 1) & 1, &abort_flag, dev_err)) {
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool store = t < S;
@@ -342,8 +413,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   }
 
-  if (abort_flag && warp == 1 && lane == 0) {
-    // Do not release TMEM while an MMA might still write it.
+  if (abort_flag && (warp == 1 || warp == 2) && lane == 0) {
+    // Do not release TMEM while an MMA of either issuer might still write it.
     mma_commit(drain);
     const long long t0c = clock64();
     while (!mbar_try_wait(drain, 0) && clock64() - t0c < kWaitLimitCycles) {
@@ -390,12 +461,12 @@ cudaError_t launch_d(const AttnArgs& a, cudaStream_t stream) {
         !encode_tensor_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.v, dims, st, box, swz))
       return cudaErrorInvalidValue;
   }
+  const int n_pairs = (a.S * a.G + 2 * kBlockM - 1) / (2 * kBlockM);
+  const int grid = n_pairs * a.B * a.Hkv;
   cudaError_t e = cudaFuncSetAttribute(attn_prefill_tc_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
-  const int n_pairs = (a.S * a.G + 2 * kBlockM - 1) / (2 * kBlockM);
-  const int grid = n_pairs * a.B * a.Hkv;
   attn_prefill_tc_kernel<D><<<grid, kAttnThreads, C::kSmem, stream>>>(
       tmQ, tmK, tmV, static_cast<bf16*>(a.out), a.B, a.S, a.Hq, a.Hkv, G_log2, n_pairs,
       a.causal, a.dev_err);

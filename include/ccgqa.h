@@ -16,8 +16,9 @@
  * Conventions for every entry point
  *  - All tensor pointers are DEVICE pointers, row-major, densely packed, owned
  *    by the caller; the library allocates no memory and keeps no state beyond
- *    a launch counter and the optional per-thread timing hook below.  Element type is cfg->dtype (fp32 or bf16) unless
- *    stated.  Every pointer must be 16-byte aligned.
+ *    a launch counter, the last CUDA error of each thread and the optional
+ *    per-thread timing hook below.  Element type is cfg->dtype (fp32 or bf16)
+ *    unless stated.  Every pointer must be 16-byte aligned.
  *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the
  *    legacy default stream).  Host-side validation happens first: on any
  *    invalid argument the call returns an error status and launches nothing.
@@ -157,6 +158,10 @@ CCGQA_API ccgqa_status ccgqa_kvcache_append(const ccgqa_config* cfg, const ccgqa
 
 /* Static description of a status code. */
 CCGQA_API const char* ccgqa_status_string(ccgqa_status s);
+
+/* Name and description of the last CUDA error an entry point met on the
+ * calling thread (after it returned CCGQA_ERR_CUDA); "no error" otherwise. */
+CCGQA_API const char* ccgqa_last_error_string(void);
 
 /* Number of kernels this library has launched in this process. */
 CCGQA_API uint64_t ccgqa_launch_count(void);
