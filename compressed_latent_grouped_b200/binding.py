@@ -75,6 +75,11 @@ def load() -> ctypes.CDLL:
                                       P(ccgqa_kvcache), c_void_p, c_void_p, c_size_t, c_void_p,
                                       c_void_p]
     lib.ccgqa_decode_step.restype = c_int
+    lib.ccgqa_decode_step_noalloc.argtypes = [P(ccgqa_config), P(ccgqa_weights), c_void_p,
+                                              P(ccgqa_kvcache), c_void_p, c_void_p, c_void_p]
+    lib.ccgqa_decode_step_noalloc.restype = c_int
+    lib.ccgqa_decode_noalloc_max_bytes.argtypes = []
+    lib.ccgqa_decode_noalloc_max_bytes.restype = c_size_t
     lib.ccgqa_kvcache_append.argtypes = [P(ccgqa_config), P(ccgqa_kvcache), c_void_p, c_void_p,
                                          c_int32, c_void_p, c_void_p]
     lib.ccgqa_kvcache_append.restype = c_int
@@ -170,6 +175,21 @@ def ccgqa_decode_step(cfg, weights, x_t, cache, out, workspace, dev_err=None, st
     if check and st != 0:
         raise CCGQAError(st, "ccgqa_decode_step")
     return st
+
+
+def ccgqa_decode_step_noalloc(cfg, weights, x_t, cache, out, dev_err=None, stream=None,
+                              check=True) -> int:
+    lib = load()
+    st = lib.ccgqa_decode_step_noalloc(ctypes.byref(cfg), ctypes.byref(weights), _ptr(x_t),
+                                       ctypes.byref(cache), _ptr(out), _ptr(dev_err),
+                                       _stream(stream))
+    if check and st != 0:
+        raise CCGQAError(st, "ccgqa_decode_step_noalloc")
+    return st
+
+
+def ccgqa_decode_noalloc_max_bytes() -> int:
+    return int(load().ccgqa_decode_noalloc_max_bytes())
 
 
 def ccgqa_kvcache_append(cfg, cache, k_new, v_new, n_new, dev_err=None, stream=None,

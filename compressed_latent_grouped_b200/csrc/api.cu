@@ -4,6 +4,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdio>
+#include <mutex>
 
 #include "kernels.h"
 
@@ -262,6 +263,37 @@ ccgqa_status run_decode(const Geo& g, const ccgqa_weights* w, const void* x_t,
 }
 
 }  // namespace
+
+// ----------------------------------------------------------------------------
+// Scratch of ccgqa_decode_step_noalloc: a fixed array in device global memory
+// that exists on every GPU that loads the library, from load until exit.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+struct ScratchSlot {
+  std::once_flag once;
+  void* ptr = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+ScratchSlot g_scratch_slots[kMaxDevices];
+
+// In host code g_noalloc_scratch only names a host-side stand-in, so the device
+// address is looked up once per device, with that device current.
+cudaError_t noalloc_scratch(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  ScratchSlot& slot = g_scratch_slots[dev];
+  std::call_once(slot.once, [&] {
+    slot.err = cudaGetSymbolAddress(&slot.ptr, g_noalloc_scratch);
+  });
+  *ptr = slot.ptr;
+  return slot.err;
+}
+}  // namespace
 }  // namespace ccgqa
 
 using namespace ccgqa;
@@ -326,6 +358,35 @@ CCGQA_API ccgqa_status ccgqa_decode_step(const ccgqa_config* cfg, const ccgqa_we
   if (g.dtype == CCGQA_BF16) return run_decode<bf16>(g, w, x_t, cache, out, ws, dev_err, st);
   return run_decode<float>(g, w, x_t, cache, out, ws, dev_err, st);
 }
+
+CCGQA_API ccgqa_status ccgqa_decode_step_noalloc(const ccgqa_config* cfg,
+                                                 const ccgqa_weights* w, const void* x_t,
+                                                 const ccgqa_kvcache* cache, void* out,
+                                                 int32_t* dev_err, void* stream) {
+  Geo g;
+  ccgqa_status s = derive(cfg, &g);
+  if (s != CCGQA_OK) return s;
+  if ((s = check_weights(g, w)) != CCGQA_OK) return s;
+  if ((s = check_cache(g, cache, true)) != CCGQA_OK) return s;
+  if (!x_t || !out || !aligned16(x_t) || !aligned16(out)) return CCGQA_ERR_INVALID_ARG;
+  const DecodeWs L = decode_ws(g, cache->batch, cache->cap, w->W_qkv != nullptr);
+  if (L.total > kNoAllocScratchBytes) return CCGQA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The merge tickets must start at zero; the array keeps whatever the last
+  // call left, so clear them on every call (the other regions are written
+  // before they are read).
+  e = cudaMemsetAsync(static_cast<uint8_t*>(scratch) + L.tick, 0,
+                      static_cast<size_t>(cache->batch) * (g.Hkv + 1) * sizeof(int32_t), st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  if (g.dtype == CCGQA_BF16) return run_decode<bf16>(g, w, x_t, cache, out, ws, dev_err, st);
+  return run_decode<float>(g, w, x_t, cache, out, ws, dev_err, st);
+}
+
+CCGQA_API size_t ccgqa_decode_noalloc_max_bytes(void) { return kNoAllocScratchBytes; }
 
 CCGQA_API ccgqa_status ccgqa_kvcache_append(const ccgqa_config* cfg, const ccgqa_kvcache* cache,
                                             const void* k_new, const void* v_new, int32_t n_new,

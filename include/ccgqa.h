@@ -147,6 +147,32 @@ CCGQA_API ccgqa_status ccgqa_decode_step(const ccgqa_config* cfg, const ccgqa_we
                                          size_t workspace_bytes, int32_t* dev_err,
                                          void* stream);
 
+/* ccgqa_decode_step without a caller-provided workspace.  The paper has no
+ * counterpart: this is a deployment convenience.  Some callers cannot
+ * allocate device memory -- for example a serving runtime whose memory plan is
+ * fixed up front and owned entirely by its own allocator, or a host that only
+ * lends this library existing buffers and has no way to hand it a new one.
+ * This entry point takes the same inputs and outputs as ccgqa_decode_step
+ * (no workspace arguments) and uses instead a scratch array compiled into the
+ * library: ccgqa_decode_noalloc_max_bytes() bytes (16 MiB) of device global
+ * memory that every GPU loading the library holds until the process exits.
+ *  - Returns CCGQA_ERR_WORKSPACE when the decode needs more scratch than that
+ *    (see ccgqa_decode_workspace_size); it never allocates, frees or calls an
+ *    allocating library routine.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ *  - All calls share the one array and it keeps the last call's contents: the
+ *    call clears the parts that must start at zero itself, but calls whose work
+ *    overlaps on the GPU (other streams, other host threads) race on it --
+ *    order them, or use ccgqa_decode_step with separate workspaces. */
+CCGQA_API ccgqa_status ccgqa_decode_step_noalloc(const ccgqa_config* cfg, const ccgqa_weights* w,
+                                                 const void* x_t, const ccgqa_kvcache* cache,
+                                                 void* out, int32_t* dev_err, void* stream);
+
+/* Scratch bytes available to ccgqa_decode_step_noalloc. */
+CCGQA_API size_t ccgqa_decode_noalloc_max_bytes(void);
+
 /* Append n_new rows per sequence: cache->k[b, g, len[b] + i, :] = k_new[b, i, g, :]
  * (same for v), then len[b] += n_new.  Bit-exact copy.
  * k_new, v_new: [batch, n_new, Hkv, d].  n_new > cap returns CCGQA_ERR_CAPACITY
