@@ -31,7 +31,10 @@ struct PreLayout {
   size_t z_bytes, bytes;
 };
 
-__host__ __device__ inline PreLayout pre_layout(int TT, int K, int G, int d, int es) {
+// has_mix: a channel-mix weight is present (else no transposed-weight buffer);
+// K == 0: no conv output buffer either.
+__host__ __device__ inline PreLayout pre_layout(int TT, int K, int G, int d, int es,
+                                                bool has_mix) {
   PreLayout L;
   L.TT = TT;
   L.KH = K > 0 ? K - 1 : 0;
@@ -41,8 +44,8 @@ __host__ __device__ inline PreLayout pre_layout(int TT, int K, int G, int d, int
   L.US = TT + 4;                  // multiple of 4 for float4 reads
   L.z_bytes = (static_cast<size_t>(L.R) * L.ZC * es + 15) & ~size_t(15);
   L.off_u = 0;
-  L.off_w = L.off_u + round4(d * L.US);
-  L.off_cs = L.off_w + round4(d * d);
+  L.off_w = L.off_u + (K > 0 ? round4(d * L.US) : 0);
+  L.off_cs = L.off_w + (K > 0 && has_mix ? round4(d * (d + 2)) : 0);
   L.off_theta = L.off_cs + round4(TT * d);  // cs: TT * d/2 float2
   L.bytes = L.z_bytes + static_cast<size_t>(L.off_theta) * 4 + static_cast<size_t>(d / 2) * 8 + 16;
   return L;
@@ -68,15 +71,16 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
-template <typename T>
+template <typename T, int D>
 __global__ void __launch_bounds__(kPreThreads)
     pre_attn_kernel(const PreAttnArgs<T> a, const int TT) {
   extern __shared__ float4 smem_f4[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(smem_f4);
   const int b = blockIdx.z, g = blockIdx.y, t0 = blockIdx.x * TT;
-  const int d = a.d, G = a.G, K = a.K, S = a.S;
-  const int half = d / 2;
-  const PreLayout L = pre_layout(TT, K, G, d, sizeof(T));
+  constexpr int d = D, half = D / 2;
+  constexpr int WS = D + 2;        // padded row of the transposed channel-mix weight
+  const int G = a.G, K = a.K, S = a.S;
+  const PreLayout L = pre_layout(TT, K, G, d, sizeof(T), a.wq_chan != nullptr || a.wk_chan != nullptr);
   T* z = reinterpret_cast<T*>(smem);                      // [R][ZC]: q | k | v
   float* fs = reinterpret_cast<float*>(smem + L.z_bytes);
   float* u = fs + L.off_u;                                // [d][US]
@@ -139,6 +143,7 @@ __global__ void __launch_bounds__(kPreThreads)
       cs[idx] = make_float2(c, s);
     }
   }
+  __syncthreads();   // the table is read by every head's epilogue
 
   // 3. per head of the group: G query heads, then the key head.
   constexpr int SEG = 8;                 // rows per conv thread
@@ -150,7 +155,8 @@ __global__ void __launch_bounds__(kPreThreads)
     const T* wch_base = is_q ? a.wq_chan : a.wk_chan;
     const T* wch = (K > 0 && wch_base) ? wch_base + static_cast<int64_t>(head) * d * d : nullptr;
     // causal depthwise conv: thread = (channel, 8-row segment), taps in registers
-    for (int idx = tid; idx < d * n_seg; idx += kPreThreads) {
+    // (no conv: the epilogue reads q~ / k~ straight from the staged rows)
+    for (int idx = tid; K > 0 && idx < d * n_seg; idx += kPreThreads) {
       const int j = idx % d, sg = idx / d;
       const int tl0 = sg * SEG;
       const T* zc = z + cb + j;
@@ -182,10 +188,10 @@ __global__ void __launch_bounds__(kPreThreads)
     if (wch) {
       for (int idx = tid; idx < d * d; idx += kPreThreads) {
         const int i = idx / d, j = idx - i * d;
-        Wt[j * d + i] = to_f32(wch[idx]);
+        Wt[j * WS + i] = to_f32(wch[idx]);
       }
     }
-    __syncthreads();
+    if (K > 0) __syncthreads();
 
     const int nI2 = d / 4;  // channel pairs (i0, i0+1) in the lower half
     const int ntile = (TT / 4) * nI2;
@@ -198,11 +204,11 @@ __global__ void __launch_bounds__(kPreThreads)
         for (int r = 0; r < 4; ++r)
 #pragma unroll
           for (int k = 0; k < 4; ++k) y[r][k] = 0.f;
-#pragma unroll 4
+#pragma unroll 8
         for (int j = 0; j < d; ++j) {
           const float4 uu = *reinterpret_cast<const float4*>(u + j * US + tl0);
-          const float2 wl = *reinterpret_cast<const float2*>(Wt + j * d + i0);
-          const float2 wh = *reinterpret_cast<const float2*>(Wt + j * d + i1);
+          const float2 wl = *reinterpret_cast<const float2*>(Wt + j * WS + i0);
+          const float2 wh = *reinterpret_cast<const float2*>(Wt + j * WS + i1);
           const float ur[4] = {uu.x, uu.y, uu.z, uu.w};
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
@@ -212,13 +218,22 @@ __global__ void __launch_bounds__(kPreThreads)
             y[r][3] = fmaf(ur[r], wh.y, y[r][3]);
           }
         }
-      } else {
+      } else if (K > 0) {
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           y[r][0] = u[i0 * US + tl0 + r];
           y[r][1] = u[(i0 + 1) * US + tl0 + r];
           y[r][2] = u[i1 * US + tl0 + r];
           y[r][3] = u[(i1 + 1) * US + tl0 + r];
+        }
+      } else {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const T* zr = z + (tl0 + r + HALO) * ZC + cb;
+          y[r][0] = to_f32(zr[i0]);
+          y[r][1] = to_f32(zr[i0 + 1]);
+          y[r][2] = to_f32(zr[i1]);
+          y[r][3] = to_f32(zr[i1 + 1]);
         }
       }
       const int ch[4] = {i0, i0 + 1, i1, i1 + 1};
@@ -257,7 +272,7 @@ __global__ void __launch_bounds__(kPreThreads)
         *reinterpret_cast<V2*>(dst + i1) = Vec2<T>::make(y[r][2], y[r][3]);
       }
     }
-    __syncthreads();
+    if (K > 0) __syncthreads();
   }
 
   // 4. value-shift: bit-exact gather of the current / previous v~ row.
@@ -304,15 +319,20 @@ cudaError_t launch_pre_attn(const PreAttnArgs<T>& a, cudaStream_t stream) {
   int TT = 4096 / a.d;
   if (TT > 256) TT = 256;
   const int es = sizeof(T);
-  while (TT > 8 && pre_layout(TT, a.K, a.G, a.d, es).bytes > 200 * 1024) TT /= 2;
-  const PreLayout L = pre_layout(TT, a.K, a.G, a.d, es);
+  const bool has_mix = a.wq_chan != nullptr || a.wk_chan != nullptr;
+  while (TT > 8 && pre_layout(TT, a.K, a.G, a.d, es, has_mix).bytes > 200 * 1024) TT /= 2;
+  const PreLayout L = pre_layout(TT, a.K, a.G, a.d, es, has_mix);
   if (L.bytes > 227 * 1024) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaFuncSetAttribute(pre_attn_kernel<T>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kernel = a.d == 16 ? pre_attn_kernel<T, 16>
+              : a.d == 32 ? pre_attn_kernel<T, 32>
+              : a.d == 64 ? pre_attn_kernel<T, 64>
+                          : pre_attn_kernel<T, 128>;
+  if (a.d != 16 && a.d != 32 && a.d != 64 && a.d != 128) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(L.bytes));
   if (e != cudaSuccess) return e;
   dim3 grid((a.S + TT - 1) / TT, a.Hkv, a.B);
-  pre_attn_kernel<T><<<grid, kPreThreads, L.bytes, stream>>>(a, TT);
+  kernel<<<grid, kPreThreads, L.bytes, stream>>>(a, TT);
   count_launches(1);
   return cudaGetLastError();
 }
