@@ -34,16 +34,18 @@ void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int* 
   } else {
     *e_splits = 0;
   }
+  // splits of whole 128-key chunks, up to 2048 keys each, and at least
+  // ~2 CTAs per SM when the cache is long enough
   const int64_t bh = static_cast<int64_t>(B) * Hkv;
-  int64_t sp = (cap + 511) / 512;
+  int64_t sp = (cap + 2047) / 2048;
   if (bh * sp < target) {
     const int64_t want = (target + bh - 1) / bh;
-    const int64_t maxsp = (cap + 63) / 64;
+    const int64_t maxsp = (cap + 127) / 128;
     sp = want < maxsp ? want : maxsp;
   }
   if (sp < 1) sp = 1;
   int64_t ch = (cap + sp - 1) / sp;
-  ch = (ch + 63) / 64 * 64;
+  ch = (ch + 127) / 128 * 128;
   *chunk = static_cast<int>(ch);
   *splits = static_cast<int>((cap + ch - 1) / ch);
 }
@@ -554,6 +556,13 @@ cudaError_t launch_decode_step(const DecodeArgs<T>& a, cudaStream_t stream) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   mark(2);
+  if constexpr (sizeof(T) == 2) {
+    if (a.G <= 16 && a.d >= 32) {
+      e = launch_decode_attn_tc(a, stream);
+      mark(3);
+      return e;
+    }
+  }
   switch (a.d) {
     case 16: e = launch_dec_attn<T, 16>(a, stream); break;
     case 32: e = launch_dec_attn<T, 32>(a, stream); break;

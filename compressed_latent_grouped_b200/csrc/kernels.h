@@ -103,6 +103,8 @@ struct DecodeArgs {
 };
 template <typename T>
 cudaError_t launch_decode_step(const DecodeArgs<T>& a, cudaStream_t stream);
+// bf16 decode attention on the tensor core (d in {32, 64, 128}, G <= 16).
+cudaError_t launch_decode_attn_tc(const DecodeArgs<bf16>& a, cudaStream_t stream);
 
 // Split plan for the decode step, shared by the workspace-size query and the launch.
 void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int* e_splits,

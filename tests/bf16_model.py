@@ -16,8 +16,7 @@ The model is the oracle's float64 arithmetic with rounding to bf16 at the
 points where the bf16 path stores bf16 values: the projection output
 (q~, k~, v~), the attention inputs q, k, v, the probabilities P fed to the PV
 product (normaliser from the unrounded P), and the output.  The decode step
-keeps q and P in fp32, so its model rounds the projection row, the appended k/v
-rows and the output only.  This module is test infrastructure: it only calls
+rounds the same points (its query and P feed the tensor core as bf16).  This module is test infrastructure: it only calls
 the oracle's functions and rounds their results.
 """
 from __future__ import annotations
@@ -86,12 +85,12 @@ def model_decode_step(layer: O.Layer, state: O.State, x_t: np.ndarray):
     yq, yk = O._mix_qk(layer, qp, kp, state.hist_q if K > 1 else None,
                        state.hist_k if K > 1 else None)
     pos = np.array([t])
-    q = O.rope(yq, pos, layer.rope_base)
+    q = bf(O.rope(yq, pos, layer.rope_base))
     k = bf(O.rope(yk, pos, layer.rope_base))
     v = O.value_shift(vl, state.v_prev.reshape(sh.Hkv, sh.d)) if layer.value_shift else vl
     k_all = np.concatenate([state.k, k])
     v_all = np.concatenate([state.v, v])
-    o = bf(O.attention(q, k_all, v_all, sh.G, layer.causal, q_pos=pos).reshape(-1))
+    o = bf(_attention_bf16_p(q, k_all, v_all, sh.G, layer.causal, pos).reshape(-1))
     if K > 1:
         hq = np.concatenate([state.hist_q[1:], qp.reshape(1, -1)])
         hk = np.concatenate([state.hist_k[1:], kp.reshape(1, -1)])
