@@ -199,6 +199,96 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+
+# ----------------------------------------------------------------------- per-workload kernels
+def measure_prefill_workload(w, steps, dev):
+    """Attention / projection / pre-attention device times of one prefill
+    workload (events around each kernel; L2 flushed before every step)."""
+    import torch
+    from compressed_latent_grouped_b200 import binding as B
+    from compressed_latent_grouped_b200.device import DeviceLayer
+    from compressed_latent_grouped_b200.workloads import make_inputs
+    import oracle.ccgqa as O
+    inp = make_inputs(w, seed=0)
+    lay = DeviceLayer(w, inp, device=dev, cap=w.S)
+    lay.alloc_cache()
+    x = inp["x"].to(dev)
+    out = torch.empty(w.B, w.S, w.Hq * w.d, dtype=w.torch_dtype, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        lay.prefill(x, out)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for e in evs:
+        flush.zero_()
+        B.ccgqa_set_phase_events(e)
+        lay.prefill(x, out)
+        B.ccgqa_set_phase_events(None)
+    torch.cuda.synchronize()
+    if lay.error_bits():
+        raise RuntimeError(f"device error bits {lay.error_bits()}")
+    ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps for i in range(3)]
+    fl = w.B * O.attention_flops(w.S, w.Hq, w.d)
+    res = {"attn_ms": ms[2], "attn_tflops": fl / (ms[2] / 1e3) / 1e12,
+           "pre_attn_ms": ms[1], "prefill_ms": sum(ms),
+           "tokens_per_s": w.B * w.S / (sum(ms) / 1e3)}
+    if not w.packed_input:
+        res["proj_ms"] = ms[0]
+        res["proj_tflops"] = 2.0 * w.B * w.S * w.E * w.n_qkv / (ms[0] / 1e3) / 1e12
+    return res
+
+
+def measure_decode_workload(w, steps, dev):
+    """Decode step on a full latent cache: device times of the projection,
+    the one-token pre-step and the split-K attention over len + 1 keys."""
+    import torch
+    from compressed_latent_grouped_b200 import binding as B
+    from compressed_latent_grouped_b200.device import DeviceLayer
+    from compressed_latent_grouped_b200.workloads import make_inputs
+    inp = make_inputs(w, seed=0)
+    lay = DeviceLayer(w, inp, device=dev, cap=w.S + 64)
+    t = lay.alloc_cache()
+    lay.append(inp["cache_k"].to(dev), inp["cache_v"].to(dev))
+    t["hist_q"].copy_(inp["hist_q"])
+    t["hist_k"].copy_(inp["hist_k"])
+    t["v_prev"].copy_(inp["v_prev"])
+    x_t = inp["x_t"].to(dev)
+    out = torch.empty(w.B, w.Hq * w.d, dtype=w.torch_dtype, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        t["len"].fill_(w.S)
+        lay.decode_step(x_t, out)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for e in evs:
+        t["len"].fill_(w.S)
+        flush.zero_()
+        B.ccgqa_set_phase_events(e)
+        lay.decode_step(x_t, out)
+        B.ccgqa_set_phase_events(None)
+    torch.cuda.synchronize()
+    if lay.error_bits():
+        raise RuntimeError(f"device error bits {lay.error_bits()}")
+    ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps for i in range(3)]
+    kv = 2 * w.B * w.Hkv * (w.S + 1) * w.d * 2
+    return {"attn_ms": ms[2], "kv_bytes": kv, "attn_gbs": kv / (ms[2] / 1e3) / 1e9,
+            "proj_ms": ms[0], "pre_ms": ms[1], "step_ms": sum(ms),
+            "tokens_per_s": w.B / (sum(ms) / 1e3)}
+
+
+def run_workload_only(args, local):
+    """--workload: time one named workload's kernels (profiling runs)."""
+    import torch
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from compressed_latent_grouped_b200.workloads import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if args.batch:
+        w = w.with_(B=args.batch)
+    if args.seq:
+        w = w.with_(S=args.seq)
+    res = (measure_decode_workload if w.decode else measure_prefill_workload)(
+        w, args.steps, dev)
+    print(json.dumps({"workload": args.workload, "B": w.B, "S": w.S, **res}), flush=True)
+
 # ----------------------------------------------------------------------- ours
 def run_ours(args, world, rank, local):
     import torch
@@ -311,6 +401,15 @@ def run_ours(args, world, rank, local):
                "sample": f"1 of {w.B} sequences: float64 prefill of all {w.S} tokens + 1 "
                          f"decode step ({t_cpu:.1f} s)"}
 
+    by_workload = None
+    if rank == 0 and not args.no_extra:
+        by_workload = {}
+        for name in ("bf16_prefill_b1_s32768", "bf16_gqa_b2_s8192"):
+            by_workload[name] = measure_prefill_workload(WORKLOADS[name], 10, dev)
+        by_workload["bf16_decode_b64_l16384"] = measure_decode_workload(
+            WORKLOADS["bf16_decode_b64_l16384"], 20, dev)
+        torch.cuda.empty_cache()
+
     if rank != 0:
         return
     line = {
@@ -334,8 +433,7 @@ def run_ours(args, world, rank, local):
         "prefill": {"tokens_per_s": w.B * w.S / (prefill_ms / 1e3) * world,
                     "tflops_attn_plus_proj": (attn_flop + proj_flop) / (prefill_ms / 1e3) / 1e12,
                     "proj_tflops": proj_flop / (proj_ms / 1e3) / 1e12},
-        "decode": {"kv_bytes": kv_bytes, "attn_gbs": kv_bytes / (dattn_ms / 1e-3) / 1e9 * 1e-6 * 1e6
-                   if dattn_ms > 0 else None,
+        "decode": {"kv_bytes": kv_bytes, "attn_gbs": None,
                    "step_ms": dproj_ms + dpre_ms + dattn_ms,
                    "hbm_frac_attn": (kv_bytes / (dattn_ms / 1e3) / 1e9) / peaks["hbm_gbs"]},
         "clocks": sampler.summary(),
@@ -343,6 +441,7 @@ def run_ours(args, world, rank, local):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "cpu_baseline": cpu,
+        "by_workload": by_workload,
     }
     line["decode"]["attn_gbs"] = kv_bytes / (dattn_ms / 1e3) / 1e9 if dattn_ms > 0 else None
     print(json.dumps(line), flush=True)
@@ -355,11 +454,19 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other workloads' kernel measurements")
+    ap.add_argument("--workload", default=None,
+                    help="time only this workload's kernels (profiling)")
+    ap.add_argument("--batch", type=int, default=0, help="with --workload: override B")
+    ap.add_argument("--seq", type=int, default=0, help="with --workload: override S (or L)")
     args = ap.parse_args()
     world, rank, local = dist_setup(args.gpus)
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.workload:
+            run_workload_only(args, local)
         else:
             run_ours(args, world, rank, local)
     finally:

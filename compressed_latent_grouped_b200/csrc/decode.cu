@@ -15,6 +15,8 @@
 //                    all G query heads.  The last CTA of a (sequence, group)
 //                    -- found with an atomic ticket, never by waiting --
 //                    merges the chunks; the last group of a sequence bumps len.
+#include <cmath>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -34,16 +36,27 @@ void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int* 
   } else {
     *e_splits = 0;
   }
-  // splits of whole 128-key chunks, up to 2048 keys each, and at least
-  // ~2 CTAs per SM when the cache is long enough
+  // Splits of whole 128-key chunks.  The CTAs of one launch should fill a whole
+  // number of waves of the resident slots (148 SMs x 2 CTAs), each CTA
+  // streaming at least ~1024 keys so its start-up cost stays small.
   const int64_t bh = static_cast<int64_t>(B) * Hkv;
-  int64_t sp = (cap + 2047) / 2048;
-  if (bh * sp < target) {
-    const int64_t want = (target + bh - 1) / bh;
-    const int64_t maxsp = (cap + 127) / 128;
-    sp = want < maxsp ? want : maxsp;
+  const int64_t slots = 148 * 2;
+  const int64_t max_sp = (cap + 127) / 128;
+  int64_t best_sp = 1;
+  double best = -1.0;
+  for (int64_t spc = 1; spc <= max_sp && spc <= 64; ++spc) {
+    const int64_t chk = ((cap + spc - 1) / spc + 127) / 128 * 128;
+    const int64_t real_sp = (cap + chk - 1) / chk;
+    const int64_t ctas = bh * real_sp;
+    const double waves = static_cast<double>(ctas) / slots;
+    double eff = waves / std::ceil(waves);
+    if (chk < 1024 && spc > 1) eff -= 0.25 * (1024 - chk) / 1024.0;
+    if (eff > best + 1e-9) {
+      best = eff;
+      best_sp = real_sp;
+    }
   }
-  if (sp < 1) sp = 1;
+  int64_t sp = best_sp;
   int64_t ch = (cap + sp - 1) / sp;
   ch = (ch + 127) / 128 * 128;
   *chunk = static_cast<int>(ch);

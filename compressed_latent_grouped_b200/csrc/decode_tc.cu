@@ -47,14 +47,15 @@ struct DCfg {
   static constexpr uint32_t kSbo = 8 * kRowBytes;
   static constexpr uint32_t kPanelBytes = kChunk * kRowBytes;   // one panel of 128 keys
   static constexpr uint32_t kTileBytes = kChunk * D * 2;        // K or V chunk
-  static constexpr int kStages = (D == 128) ? 2 : 3;
+  static constexpr int kStages = (D == 128) ? 2 : 3;   // d = 64: ~104 KB, two CTAs per SM
   static constexpr uint32_t kQPanelBytes = kQRows * kRowBytes;
   // d >= 64: O^T = V^T P^T with P^T [16 heads][128 keys]; d = 32: O = P V with
   // P [128 rows][128 keys] (M must be 64 or 128).
   static constexpr bool kT = D >= 64;
   static constexpr uint32_t kPRows = kT ? kQRows : 128;
   static constexpr uint32_t kPPanelBytes = kPRows * 128;       // 64 keys x 2 B per row
-  static constexpr uint32_t kPBytes = 2 * kPPanelBytes;
+  static constexpr uint32_t kPBufBytes = 2 * kPPanelBytes;     // one P tile (two key panels)
+  static constexpr uint32_t kPBytes = 2 * kPBufBytes;          // double-buffered across chunks
   static constexpr uint32_t kOffK = 0;
   static constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
   static constexpr uint32_t kOffP = kOffV + kStages * kTileBytes;
@@ -91,8 +92,8 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
   uint64_t* q_ready = kv_empty + C::kStages; // 128 arrivals: Q^T and zeroed P built
   uint64_t* s_full = q_ready + 1;            // [2] S^T buffers
   uint64_t* p_full = s_full + 2;             // 128 arrivals
-  uint64_t* o_done = p_full + 1;
-  uint64_t* drain = o_done + 1;
+  uint64_t* o_done = p_full + 1;             // [2] PV of chunks using P buffer 0 / 1
+  uint64_t* drain = o_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffBar + 256);
   float* red = reinterpret_cast<float*>(smem + C::kOffBar + 512);   // [2][4 warps][kQRows]
   __shared__ int abort_flag, last_flag;
@@ -117,7 +118,8 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
     mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
+    mbar_init(&o_done[0], 1);
+    mbar_init(&o_done[1], 1);
     mbar_init(drain, 1);
     abort_flag = 0;
     fence_barrier_init();
@@ -188,14 +190,15 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
           const uint64_t vd = make_smem_desc(v_base + k * 16 * C::kRowBytes, C::kPanelBytes,
                                              C::kSbo, C::kSwz);
           // P (or P^T): K-major over keys, two 64-key panels, 128B swizzle
-          const uint64_t pd = make_smem_desc(p_base + (k >> 2) * C::kPPanelBytes + (k & 3) * 32, 16,
-                                             1024, kSwizzle128B);
+          const uint64_t pd = make_smem_desc(p_base + (c & 1) * C::kPBufBytes +
+                                                 (k >> 2) * C::kPPanelBytes + (k & 3) * 32,
+                                             16, 1024, kSwizzle128B);
           if constexpr (C::kT)
             mma_ss(tmem + C::kColO, vd, pd, idesc_o, (c > 0 || k > 0) ? 1u : 0u);
           else
             mma_ss(tmem + C::kColO, pd, vd, idesc_o, (c > 0 || k > 0) ? 1u : 0u);
         }
-        mma_commit(o_done);
+        mma_commit(&o_done[c & 1]);
         mma_commit(&kv_empty[st]);
       };
       bool ok = mbar_wait(q_ready, 0, &abort_flag, a.dev_err);
@@ -290,14 +293,20 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
         p[h] = (m_run[h] == -INFINITY) ? 0.f : ex2(sv[h] - m_run[h]);
         l_part[h] += p[h];
       }
-      // P(c) may overwrite P(c-1) once PV(c-1) is done; O must hold it before a rescale
-      if (c > 0) {
-        if (!mbar_wait(o_done, (c - 1) & 1, &abort_flag, a.dev_err)) {
+      // P buffer c&1 was last read by PV(c-2); a rescale needs O to hold PV(c-1)
+      if (c >= 2) {
+        if (!mbar_wait(&o_done[c & 1], ((c - 2) >> 1) & 1, &abort_flag, a.dev_err)) {
           ok = false;
           break;
         }
-        tc_fence_after();
       }
+      if (need_any && c >= 1) {
+        if (!mbar_wait(&o_done[(c - 1) & 1], ((c - 1) >> 1) & 1, &abort_flag, a.dev_err)) {
+          ok = false;
+          break;
+        }
+      }
+      tc_fence_after();
       if (need_any) {
         if constexpr (C::kT) {
           // O^T: TMEM lane = output channel, column h = head h
@@ -330,7 +339,7 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
 #pragma unroll
       for (int h = 0; h < kQRows; ++h) {
         if (h >= G) break;
-        *reinterpret_cast<bf16*>(ptile + (key >> 6) * C::kPPanelBytes +
+        *reinterpret_cast<bf16*>(ptile + (c & 1) * C::kPBufBytes + (key >> 6) * C::kPPanelBytes +
                                  swz_offset(h, (key & 63) * 2, 128)) = __float2bfloat16_rn(p[h]);
       }
       if (!kv) {
@@ -348,8 +357,9 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
       mbar_arrive(p_full);
     }
     // ---- split partials: max and sum per head, unnormalised O rows
+    // the last PV completes after every earlier one
     const bool have = ok && n_ch > 0 && !abort_flag &&
-                      mbar_wait(o_done, (n_ch - 1) & 1, &abort_flag, a.dev_err);
+                      mbar_wait(&o_done[(n_ch - 1) & 1], ((n_ch - 1) >> 1) & 1, &abort_flag, a.dev_err);
     tc_fence_after();
     named_barrier_sync(1, 128);   // everyone is done reading red[] of the last chunk
 #pragma unroll
