@@ -7,26 +7,28 @@
 // t0 + r / G, head g*G + r % G, so a 5-D TMA box gathers a tile straight from
 // q[B, S, Hq, d] and one K/V tile in shared memory serves all G query heads.
 //
-// One CTA owns two 128-row query tiles (A and B) of one kv group and streams
-// the K/V tiles both need once, as 128-key tiles split into two 64-key halves:
-//   warp 0      TMA producer: Q_A, Q_B once, then K/V tiles of 128 keys
-//               through a ring of shared-memory stages
-//   warps 1, 2  one thread each issues the tcgen05.mma of tile A / tile B
+// One CTA owns T consecutive 128-row query tiles of one kv group (T = 3 at
+// d = 32, else 2) and streams the K/V tiles they need once, as 128-key tiles
+// split into two 64-key halves:
+//   warp 0      TMA producer: the T query tiles once, then K/V tiles of 128
+//               keys through a ring of shared-memory stages
+//   warps 1..T  one thread each issues the tcgen05.mma of one query tile
 //               (warp 1 also owns the TMEM allocation):
 //                 S_X = Q_X K_h^T  (SS, M=128 N=64, fp32 accumulators in TMEM)
 //                 O_X += P_X V_h   (TS: P read from TMEM, V from shared memory)
 //               With one issuer per tile, waiting for one tile's PV never
 //               delays the other tile's MMAs.
-//   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: one thread per
+//   warps 4+4x..7+4x  softmax of tile x: one thread per
 //               row (TMEM lane); tcgen05.ld of S, running max / sum in
 //               registers, P written back to TMEM as bf16 pairs in the upper
-//               half of its S buffer, O rescaled in TMEM when the running max
-//               grows by more than 2^8, normalised O stored at the end.
+//               half of its S buffer, O rescaled in TMEM on the rare half whose
+//               partial sum shows the running max fell behind, normalised O
+//               stored at the end.
 // Each tile has two S buffers (one per 64-key half), so the S of the next half
 // is computed while the softmax works on the current one and a softmax
 // warpgroup never waits for the PV -> S round trip; the two warpgroups keep
 // the exp unit and the FMA pipe busy while the tensor core runs their MMAs.
-// TMEM: S/P of tile X at columns 128 X + {0, 64}, O_X at 256 + X d (d <= 128).
+// TMEM: S/P of tile x at columns 128 x + {0, 64}, O_x at 128 T + x d.
 // No cluster multicast is used; every wait is bounded.
 #include "kernels.h"
 #include "sm100.cuh"
@@ -36,12 +38,12 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kAttnThreads = 384;
 constexpr int kBlockM = 128, kBlockN = 128, kHalfN = 64;
 constexpr float kLog2e = 1.4426950408889634f;
-// The running max used for exp2 is only raised when it falls behind by more
-// than this many doublings, so P <= 2^8 and O is rescaled rarely.
-constexpr float kRescaleThreshold = 8.0f;
+// The running max used for exp2 is only raised when a row's partial sum over
+// a 64-key half exceeds this, so every P stays below 2^10 and O is rescaled
+// rarely.
+constexpr float kSumLimit = 1024.0f;
 
 template <int D>
 struct Cfg {
@@ -53,8 +55,12 @@ struct Cfg {
   static constexpr uint32_t kPanelBytes = 128 * kRowBytes;    // one panel of 128 rows
   static constexpr uint32_t kTileBytes = 128 * D * 2;         // one Q / K / V tile
   static constexpr int kStages = (D == 128) ? 2 : (D == 64 ? 3 : 4);
+  // Query tiles per CTA: three where their S buffers and accumulators fit
+  // in TMEM (3 x 128 + 3 x 32 columns at d = 32), else two.
+  static constexpr int kTiles = (D == 32) ? 3 : 2;
+  static constexpr int kThreads = 128 + 128 * kTiles;   // 4 control warps + softmax
   static constexpr uint32_t kOffQ = 0;                        // Q_A, Q_B
-  static constexpr uint32_t kOffK = 2 * kTileBytes;
+  static constexpr uint32_t kOffK = kTiles * kTileBytes;
   static constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
   static constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
   static constexpr size_t kSmem = kOffBar + 256 + 1024;
@@ -62,7 +68,7 @@ struct Cfg {
   // S buffer h of tile x, its P (upper 32 columns: 64 keys as bf16 pairs), O_x
   __device__ static constexpr uint32_t col_s(int x, int h) { return x * 128 + h * 64; }
   __device__ static constexpr uint32_t col_p(int x, int h) { return x * 128 + h * 64 + 32; }
-  __device__ static constexpr uint32_t col_o(int x) { return 256 + x * D; }
+  __device__ static constexpr uint32_t col_o(int x) { return kTiles * 128 + x * D; }
 };
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -120,11 +126,12 @@ __device__ __forceinline__ float2 soft_exp2x2(float2 x) {
                      __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
-// Pairs (c2 % kSoftExpEvery == 0) of each softmax row use the software exp2.
-// Measured on B200: while the softmax is latency-bound the extra instructions
-// cost more than the exp unit time they save, so it is off by default.
+// Pairs (c2 % kSoftExpEvery == 0) of each softmax row use the software exp2,
+// so the FMA pipe takes a quarter of the exponentials off the exp unit
+// (measured on B200: 1 in 4 is the best split at d = 64 and d = 128, neutral
+// at d = 32).
 #ifndef CCGQA_SOFT_EXP_EVERY
-#define CCGQA_SOFT_EXP_EVERY 1000000
+#define CCGQA_SOFT_EXP_EVERY 4
 #endif
 constexpr int kSoftExpEvery = CCGQA_SOFT_EXP_EVERY;
 
@@ -134,11 +141,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                            const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, bf16* __restrict__ out,
-                           int B, int S, int Hq, int Hkv, int G_log2, int n_pairs, int causal,
+                           int B, int S, int Hq, int Hkv, int G_log2, int n_groups, int causal,
                            int32_t* dev_err) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -148,36 +155,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;                  // [kStages]
   uint64_t* kv_empty = kv_full + C::kStages;     // [kStages]
-  uint64_t* s_full = kv_empty + C::kStages;      // [2 tiles][2 halves]  S ready
-  uint64_t* p_full = s_full + 4;                 // [2][2]  P written (128 arrivals)
-  uint64_t* o_done = p_full + 4;                 // [2][2]  PV of that half complete
-  uint64_t* drain = o_done + 4;
+  uint64_t* s_full = kv_empty + C::kStages;      // [tile][half]  S ready
+  uint64_t* p_full = s_full + 2 * C::kTiles;     // [tile][half]  P written (128 arrivals)
+  uint64_t* o_done = p_full + 2 * C::kTiles;     // [tile][half]  PV of that half complete
+  uint64_t* drain = o_done + 2 * C::kTiles;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = 1 << G_log2;
   const int BH = B * Hkv;
-  const int pair = n_pairs - 1 - static_cast<int>(blockIdx.x) / BH;  // longest first
+  const int grp = n_groups - 1 - static_cast<int>(blockIdx.x) / BH;  // longest first
   const int bg = static_cast<int>(blockIdx.x) % BH;
   const int b = bg / Hkv, g = bg % Hkv;
   const int pos_per_tile = kBlockM >> G_log2;
-  const int t0 = pair * 2 * pos_per_tile;
-  const int t_last = min(t0 + 2 * pos_per_tile - 1, S - 1);
+  const int t0 = grp * C::kTiles * pos_per_tile;
+  const int t_last = min(t0 + C::kTiles * pos_per_tile - 1, S - 1);
   const int n_kv = causal ? (t_last / kBlockN + 1) : (S + kBlockN - 1) / kBlockN;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 2);   // released by both tiles' last PV of the stage
+      mbar_init(&kv_empty[s], C::kTiles);   // released by every tile's last PV of the stage
     }
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2 * C::kTiles; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
       mbar_init(&o_done[i], 1);
     }
-    mbar_init(drain, 2);   // one commit from each MMA issuer
+    mbar_init(drain, C::kTiles);   // one commit from each MMA issuer
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -196,9 +203,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
-      mbar_arrive_expect_tx(q_full, 2 * C::kTileBytes);
+      mbar_arrive_expect_tx(q_full, C::kTiles * C::kTileBytes);
 #pragma unroll
-      for (int x = 0; x < 2; ++x)
+      for (int x = 0; x < C::kTiles; ++x)
 #pragma unroll
         for (int p = 0; p < C::kPanels; ++p)
           tma_load_5d(smem + C::kOffQ + x * C::kTileBytes + p * C::kPanelBytes, &tmQ, q_full,
@@ -217,7 +224,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
     }
-  } else if (warp == 1 || warp == 2) {
+  } else if (warp >= 1 && warp <= C::kTiles) {
     // ------------------------------------------------------------ MMA issuers
     // Tile x = warp - 1.  Per K/V tile j and half h: PV_x(j,h), then
     // S_x(j+1,h) into the buffer P_x(j,h) was read from (after that PV
@@ -291,7 +298,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
-    const int x = (warp - 4) >> 2;                // tile A (0) or B (1)
+    const int x = (warp - 4) >> 2;                // query tile of this warpgroup
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;                 // tile row == TMEM lane
     const int t = t0 + x * pos_per_tile + (r >> G_log2);
@@ -309,59 +316,84 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           break;
         }
         tc_fence_after();
-        float s[64];
-        tmem_ld32(trow + C::col_s(x, h), *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-        tmem_ld32(trow + C::col_s(x, h) + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-        tmem_wait_ld();
         // keys j*128 + h*64 + c are visible when c <= lim
         const int kb = j * kBlockN + h * kHalfN;
         int lim = S - 1 - kb;
         if (causal) lim = min(lim, t - kb);
-        if (!__all_sync(0xffffffffu, lim >= kHalfN - 1)) {
+        const bool full_half = __all_sync(0xffffffffu, lim >= kHalfN - 1);
+        auto load_s = [&](float (&sv)[64]) {
+          tmem_ld32(trow + C::col_s(x, h), *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+          tmem_ld32(trow + C::col_s(x, h) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+          tmem_wait_ld();
+          if (!full_half) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) s[c] = (c <= lim) ? s[c] : -INFINITY;
+            for (int c = 0; c < 64; ++c) sv[c] = (c <= lim) ? sv[c] : -INFINITY;
+          }
+        };
+        auto row_max = [&](const float (&sv)[64]) {
+          float mx[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx[k] = sv[k];
+#pragma unroll
+          for (int c = 8; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], sv[c]);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) mx[k] = fmaxf(mx[k], mx[k + 4]);
+          return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * scale;
+        };
+        uint32_t pk[32];
+        // p = 2^(s * scale - m_used) as bf16 pairs; returns the row's sum of p
+        auto exp_pass = [&](const float (&sv)[64]) {
+          const float2 negm2 = make_float2(-m_used, -m_used);
+          const float2* s2 = reinterpret_cast<const float2*>(sv);
+          float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                            make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+          for (int c2 = 0; c2 < 32; ++c2) {
+            const float2 arg = ffma2(s2[c2], scale2, negm2);
+            float2 p;
+            if ((c2 % kSoftExpEvery) == 0) {
+              p = soft_exp2x2(arg);
+            } else {
+              p.x = fast_exp2(arg.x);
+              p.y = fast_exp2(arg.y);
+            }
+            lsum[c2 & 3] = fadd2(lsum[c2 & 3], p);
+            pk[c2] = pack_bf16x2(p.x, p.y);
+          }
+          const float2 a2 = fadd2(fadd2(lsum[0], lsum[1]), fadd2(lsum[2], lsum[3]));
+          return a2.x + a2.y;
+        };
+        // The first half sets the running max (key 0 is visible to every
+        // row, so it is finite).  Later halves exponentiate against the
+        // running max as it stands and look only at the row's partial sum:
+        // while it stays within kSumLimit every p is below it.  A row whose
+        // sum overshoots (some p > kSumLimit / 64, so its max lies above the
+        // running max by more than log2(kSumLimit / 64)) reloads S from TMEM,
+        // which still holds it, raises the running max to the half's max and
+        // redoes the half.
+        float part;
+        {
+          float sv[64];
+          load_s(sv);
+          if (j == 0 && h == 0) m_used = row_max(sv);
+          part = exp_pass(sv);
         }
-        float mx[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = s[k];
-#pragma unroll
-        for (int c = 8; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) mx[k] = fmaxf(mx[k], mx[k + 4]);
-        const float m_new = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * scale;
+        const bool redo = !(part <= kSumLimit);
         bool need = false;
         float factor = 1.f;
-        if (j == 0 && h == 0) {
-          m_used = m_new;
-        } else if (m_new > m_used + kRescaleThreshold) {
-          factor = fast_exp2(m_used - m_new);
-          l *= factor;
-          m_used = m_new;
-          need = true;
-        }
-        const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
-        const float2 negm2 = make_float2(neg_m, neg_m);
-        float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                          make_float2(0.f, 0.f)};
-        const float2* s2 = reinterpret_cast<const float2*>(s);
-        uint32_t pk[32];
-#pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) {
-          const float2 arg = ffma2(s2[c2], scale2, negm2);
-          float2 p;
-          if ((c2 % kSoftExpEvery) == 0) {
-            p = soft_exp2x2(arg);
-          } else {
-            p.x = fast_exp2(arg.x);
-            p.y = fast_exp2(arg.y);
+        if (__any_sync(0xffffffffu, redo)) {
+          float sv[64];
+          load_s(sv);   // warp-wide
+          if (redo) {
+            const float m_new = row_max(sv);
+            factor = fast_exp2(m_used - m_new);
+            l *= factor;
+            m_used = m_new;
+            need = true;
+            part = exp_pass(sv);
           }
-          lsum[c2 & 3] = fadd2(lsum[c2 & 3], p);
-          pk[c2] = pack_bf16x2(p.x, p.y);
         }
-        {
-          const float2 a2 = fadd2(fadd2(lsum[0], lsum[1]), fadd2(lsum[2], lsum[3]));
-          l += a2.x + a2.y;
-        }
+        l += part;
         if (__any_sync(0xffffffffu, need)) {
           // O must hold every earlier half: wait for the previous PV of this tile.
           const int pb = x * 2 + (1 - h);
@@ -413,7 +445,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   }
 
-  if (abort_flag && (warp == 1 || warp == 2) && lane == 0) {
+  if (abort_flag && warp >= 1 && warp <= C::kTiles && lane == 0) {
     // Do not release TMEM while an MMA of either issuer might still write it.
     mma_commit(drain);
     const long long t0c = clock64();
@@ -461,14 +493,15 @@ cudaError_t launch_d(const AttnArgs& a, cudaStream_t stream) {
         !encode_tensor_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.v, dims, st, box, swz))
       return cudaErrorInvalidValue;
   }
-  const int n_pairs = (a.S * a.G + 2 * kBlockM - 1) / (2 * kBlockM);
-  const int grid = n_pairs * a.B * a.Hkv;
+  const int rows_per_cta = C::kTiles * kBlockM;
+  const int n_groups = (a.S * a.G + rows_per_cta - 1) / rows_per_cta;
+  const int grid = n_groups * a.B * a.Hkv;
   cudaError_t e = cudaFuncSetAttribute(attn_prefill_tc_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
-  attn_prefill_tc_kernel<D><<<grid, kAttnThreads, C::kSmem, stream>>>(
-      tmQ, tmK, tmV, static_cast<bf16*>(a.out), a.B, a.S, a.Hq, a.Hkv, G_log2, n_pairs,
+  attn_prefill_tc_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(
+      tmQ, tmK, tmV, static_cast<bf16*>(a.out), a.B, a.S, a.Hq, a.Hkv, G_log2, n_groups,
       a.causal, a.dev_err);
   count_launches(1);
   return cudaGetLastError();
