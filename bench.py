@@ -200,6 +200,21 @@ def run_reference(args, world, rank):
 
 
 
+def exp_roofline(w, attn_ms, peaks):
+    """The softmax's exponentials against the exp unit: 16 ex2 per clock per SM
+    (the B200 SFU rate, measured 15.8 on this part) x 148 SMs x the maximum SM
+    clock.  Causal scores: B Hq S (S + 1) / 2 exponentials per launch.  One in
+    four runs on the FMA pipe instead, so frac can pass 0.75 of the exp-unit
+    time only by that offload."""
+    n_exp = w.B * w.Hq * w.S * (w.S + 1) / 2 if w.causal else w.B * w.Hq * w.S * w.S
+    mhz = peaks.get("sm_max_mhz", 1965.0)
+    peak = 16 * 148 * mhz * 1e6 / 1e12
+    achieved = n_exp / (attn_ms / 1e3) / 1e12
+    return {"bound": "alu", "unit": "Texp/s", "achieved": achieved, "peak": peak,
+            "frac": achieved / peak, "exp_per_launch": n_exp,
+            "peak_kind": f"16 ex2/clk/SM x 148 SMs x {mhz:.0f} MHz"}
+
+
 # ----------------------------------------------------------------------- per-workload kernels
 def measure_prefill_workload(w, steps, dev):
     """Attention / projection / pre-attention device times of one prefill
@@ -228,7 +243,10 @@ def measure_prefill_workload(w, steps, dev):
         raise RuntimeError(f"device error bits {lay.error_bits()}")
     ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps for i in range(3)]
     fl = w.B * O.attention_flops(w.S, w.Hq, w.d)
+    peaks, _ = load_peaks()
     res = {"attn_ms": ms[2], "attn_tflops": fl / (ms[2] / 1e3) / 1e12,
+           "attn_tensor_frac": fl / (ms[2] / 1e3) / 1e12 / peaks["bf16_tflops"],
+           "attn_exp_frac": exp_roofline(w, ms[2], peaks)["frac"],
            "pre_attn_ms": ms[1], "prefill_ms": sum(ms),
            "tokens_per_s": w.B * w.S / (sum(ms) / 1e3)}
     if not w.packed_input:
@@ -269,7 +287,9 @@ def measure_decode_workload(w, steps, dev):
         raise RuntimeError(f"device error bits {lay.error_bits()}")
     ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps for i in range(3)]
     kv = 2 * w.B * w.Hkv * (w.S + 1) * w.d * 2
+    peaks, _ = load_peaks()
     return {"attn_ms": ms[2], "kv_bytes": kv, "attn_gbs": kv / (ms[2] / 1e3) / 1e9,
+            "attn_hbm_frac": kv / (ms[2] / 1e3) / 1e9 / peaks["hbm_gbs"],
             "proj_ms": ms[0], "pre_ms": ms[1], "step_ms": sum(ms),
             "tokens_per_s": w.B / (sum(ms) / 1e3)}
 
@@ -357,6 +377,8 @@ def run_ours(args, world, rank, local):
     attn_flop = w.B * O.attention_flops(w.S, w.Hq, w.d)
     proj_flop = 2.0 * w.B * w.S * w.E * w.n_qkv
     kv_bytes = 2 * w.B * w.Hkv * (w.S + 1) * w.d * 2
+    # pre-attention: q~|k~|v~ read once, q, k, v written once (bf16)
+    pre_bytes = 2 * w.B * w.S * w.n_qkv * 2
     peaks, peak_kind = load_peaks()
     achieved = attn_flop / (attn_ms / 1e3) / 1e12
     traffic = attn_traffic_per_launch()
@@ -427,6 +449,16 @@ def run_ours(args, world, rank, local):
                      "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
                      "peak_kind": f"{peak_kind} bf16 dense burst",
                      "flop_per_launch": attn_flop, "ms_per_launch": attn_ms},
+        "roofline_exp": exp_roofline(w, attn_ms, peaks),
+        "kernels": {
+            "proj_gemm": {"ms": proj_ms, "tflops": proj_flop / (proj_ms / 1e3) / 1e12,
+                          "tensor_frac": proj_flop / (proj_ms / 1e3) / 1e12 / peaks["bf16_tflops"]},
+            "pre_attn": {"ms": pre_ms, "bytes": pre_bytes,
+                         "gbs": pre_bytes / (pre_ms / 1e3) / 1e9,
+                         "hbm_frac": pre_bytes / (pre_ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
+            "attn_prefill_tc": {"ms": attn_ms, "tflops": achieved,
+                                "tensor_frac": achieved / peaks["bf16_tflops"]},
+        },
         "phases_ms": {"proj_gemm": proj_ms, "pre_attn": pre_ms, "attn_prefill_tc": attn_ms,
                       "prefill_total": prefill_ms, "decode_proj": dproj_ms,
                       "decode_pre": dpre_ms, "decode_attn": dattn_ms},

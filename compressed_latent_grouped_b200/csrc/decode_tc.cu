@@ -65,13 +65,6 @@ struct DCfg {
   static constexpr uint32_t kColS = 0, kColO = 32, kTmemCols = 64;   // S^T x2 | O^T or O
 };
 
-// Byte offset of element (row, col) in a K-major tile whose rows are `row_bytes`
-// wide (64 or 128), with the matching TMA / UMMA swizzle.
-__device__ __forceinline__ uint32_t swz_offset(uint32_t row, uint32_t col_byte, uint32_t row_bytes) {
-  const uint32_t off = row * row_bytes + col_byte;
-  return row_bytes == 128 ? (off ^ (((off >> 7) & 7u) << 4)) : (off ^ (((off >> 7) & 3u) << 4));
-}
-
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -16,6 +16,8 @@
 //      previous position -- a bit-exact copy out of shared memory;
 //   4. the CTA holding the last position writes the decode state.
 // All arithmetic in fp32; inputs and outputs in the working dtype.
+#include <type_traits>
+
 #include "kernels.h"
 
 namespace ccgqa {
@@ -314,6 +316,9 @@ __global__ void __launch_bounds__(kPreThreads)
 
 template <typename T>
 cudaError_t launch_pre_attn(const PreAttnArgs<T>& a, cudaStream_t stream) {
+  if constexpr (std::is_same<T, bf16>::value) {
+    if (pre_attn_tc_supported(a)) return launch_pre_attn_tc(a, stream);
+  }
   // Positions per CTA: TT * d = 4096 gives exactly one 4x4 register tile per
   // thread in the channel mix; halve TT while the staging does not fit.
   int TT = 4096 / a.d;

@@ -1,0 +1,415 @@
+// Fused pre-attention with the per-head channel mix on the 5th-generation
+// tensor core (bf16 heads of dim 32 or 64): causal sequence conv, channel mix,
+// QK-mean, RoPE and value-shift ("Compressed Convolutional Attention",
+// Methodologie items 2-4; the mix is a d x d product per position and head,
+// i.e. a [positions x d] by [d x d] contraction).
+//
+// One CTA owns 128 consecutive positions of one kv group (its G query heads,
+// its key head and its value head) of one sequence:
+//   1. the group's q~ | k~ rows [t0 - 3, t0 + 128) are copied into shared
+//      memory with 16-byte cp.async, the G + 1 mix weights W_h [d_out, d_in]
+//      straight into the swizzled K-major layout of a UMMA B operand, the conv
+//      taps as fp32, and a cos/sin table per (pair, position) is formed (angle
+//      reduced modulo one turn in fp64);
+//   2. per head h (G query heads, then the key head):
+//        conv   one thread per (position, 16-byte channel chunk): u = sum_k
+//               w[c, k] z[t - k, c] in fp32, split as u = hi + lo with hi, lo
+//               bf16 and both written as the A operands [128 x d] of the MMA;
+//        mix    one thread issues Y_h = U_hi W_h^T + U_lo W_h^T (M = 128, N = d,
+//               fp32 accumulators in TMEM, two buffers), so the product keeps
+//               fp32 accuracy (u - hi - lo is below 2^-16 |u|);
+//        epilogue  thread = (position row = TMEM lane, half of the rotary pairs):
+//               tcgen05.ld of Y_h, QK-mean from the staged pre-conv rows, RoPE on
+//               the pairs (i, i + d/2) it holds, bf16 store.
+//      The epilogue of head h - 1 runs while the tensor core computes head h.
+//   3. value-shift: each v row is gathered from rows t and t - 1 of v~, a
+//      bit-exact copy.
+//   4. the CTA holding the last position writes the decode state.
+// Every wait is bounded; no cluster multicast is used.
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace ccgqa {
+namespace {
+
+using namespace sm100;
+
+constexpr int kPtThreads = 256;
+constexpr int kPtTT = 128;     // positions per CTA == MMA M == TMEM lanes
+constexpr int kPtHalo = 3;     // the conv reaches back K - 1 <= 3 rows
+
+struct PtLayout {
+  int ZC;                      // staged row width in elements: (G + 1) d + 8
+  uint32_t u_bytes, w_bytes;   // one A tile (hi or lo), one head's B tile
+  uint32_t off_u, off_w, off_z, off_cs, off_ws, off_theta, off_bar, bytes;
+};
+
+// Byte layout of the dynamic shared memory (from a 1024-byte aligned base).
+__host__ __device__ inline PtLayout pt_layout(int d, int G) {
+  PtLayout L;
+  const uint32_t row = static_cast<uint32_t>(d) * 2;
+  L.ZC = (G + 1) * d + 8;      // + 16 bytes: an odd number of 16-byte units per row
+  L.u_bytes = kPtTT * row;
+  L.w_bytes = static_cast<uint32_t>(d) * row;
+  L.off_u = 0;                                      // U_hi, U_lo
+  L.off_w = 2 * L.u_bytes;                          // W_h, h = 0..G
+  L.off_z = L.off_w + (G + 1) * L.w_bytes;          // [131][ZC] bf16
+  L.off_cs = L.off_z + ((static_cast<uint32_t>(kPtTT + kPtHalo) * L.ZC * 2 + 15u) & ~15u);
+  L.off_ws = L.off_cs + static_cast<uint32_t>(d / 2) * kPtTT * 8;   // [d/2][128] float2
+  L.off_theta = L.off_ws + static_cast<uint32_t>(G + 1) * d * 16;  // [(G+1) d][4] float
+  L.off_bar = L.off_theta + static_cast<uint32_t>(d / 2) * 8;      // [d/2] double
+  L.bytes = L.off_bar + 64 + 1024;                  // barriers + alignment slack
+  return L;
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 p = __bfloat1622float2(h[i]);
+    f[2 * i] = p.x;
+    f[2 * i + 1] = p.y;
+  }
+}
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPtThreads)
+    pre_attn_tc_kernel(const PreAttnArgs<bf16> a) {
+  constexpr uint32_t kRowBytes = D * 2;                 // 64: 64B swizzle, 128: 128B swizzle
+  constexpr uint32_t kSwz = (D == 32) ? kSwizzle64B : kSwizzle128B;
+  constexpr uint32_t kSbo = 8 * kRowBytes;
+  constexpr int NCH = D / 8;                            // 16-byte chunks per row
+  constexpr int Q4 = D / 4;                             // rotary pairs per epilogue thread
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int G = a.G, S = a.S, K = a.K;
+  const PtLayout L = pt_layout(D, G);
+  const int ZC = L.ZC, NH = G + 1, QC = G * D;
+  const int b = blockIdx.z, g = blockIdx.y, t0 = blockIdx.x * kPtTT;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  bf16* z = reinterpret_cast<bf16*>(smem + L.off_z);
+  float2* cs = reinterpret_cast<float2*>(smem + L.off_cs);
+  float* ws = reinterpret_cast<float*>(smem + L.off_ws);
+  double* theta = reinterpret_cast<double*>(smem + L.off_theta);
+  uint64_t* mma_done = reinterpret_cast<uint64_t*>(smem + L.off_bar);   // [2]
+  uint64_t* drain = mma_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  __shared__ int abort_flag;
+
+  const int64_t ld = a.src_ld;
+  const bf16* src_b = a.src + static_cast<int64_t>(b) * S * ld;
+  const int qcol0 = g * QC;
+  const int kcol0 = a.Hq * D + g * D;
+  const int vcol0 = (a.Hq + a.Hkv) * D + g * D;
+
+  if (tid == 0) {
+    mbar_init(&mma_done[0], 1);
+    mbar_init(&mma_done[1], 1);
+    mbar_init(drain, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 2 * D);
+    tmem_relinquish();
+  }
+
+  // 1. staging
+  {
+    const int cq = QC / 8, per_row = cq + NCH;
+    for (int idx = tid; idx < (kPtTT + kPtHalo) * per_row; idx += kPtThreads) {
+      const int r = idx / per_row, c = idx - r * per_row;
+      const int t = t0 - kPtHalo + r;
+      const int col = c < cq ? qcol0 + c * 8 : kcol0 + (c - cq) * 8;
+      bf16* dst = z + r * ZC + c * 8;               // q channels, then the key head's
+      if (t >= 0 && t < S)
+        cp_async16(dst, src_b + static_cast<int64_t>(t) * ld + col);
+      else
+        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+    }
+    // W_h row n (output channel), chunk j of the input channels -> B operand
+    for (int idx = tid; idx < NH * D * NCH; idx += kPtThreads) {
+      const int hh = idx / (D * NCH), rem = idx - hh * (D * NCH);
+      const int n = rem / NCH, j = rem - n * NCH;
+      const bf16* w = hh < G ? a.wq_chan + (static_cast<int64_t>(g * G + hh) * D + n) * D
+                             : a.wk_chan + (static_cast<int64_t>(g) * D + n) * D;
+      cp_async16(smem + L.off_w + hh * L.w_bytes + swz_offset(n, j * 16, kRowBytes), w + j * 8);
+    }
+    // conv taps w[c][k] as fp32, zero past K
+    for (int idx = tid; idx < NH * D * 4; idx += kPtThreads) {
+      const int hc = idx >> 2, k = idx & 3;
+      const int hh = hc / D, c = hc - hh * D;
+      const bf16* w = hh < G ? a.wq_seq + (static_cast<int64_t>(g * G + hh) * D + c) * K
+                             : a.wk_seq + (static_cast<int64_t>(g) * D + c) * K;
+      ws[idx] = k < K ? __bfloat162float(w[k]) : 0.f;
+    }
+    if (a.rope_on)
+      for (int i = tid; i < D / 2; i += kPtThreads)
+        theta[i] = exp2(-(2.0 * i / D) * a.rope_log2_base);
+  }
+  // value-shift while the copies fly: v[t, :d/2] = v~[t, :d/2], v[t, d/2:] = v~[t-1, d/2:]
+  for (int idx = tid; idx < kPtTT * NCH; idx += kPtThreads) {
+    const int tl = idx / NCH, i = (idx - tl * NCH) * 8;
+    const int t = t0 + tl;
+    if (t >= S) continue;
+    const int row = (a.value_shift && i >= D / 2) ? t - 1 : t;
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (row >= 0) val = *reinterpret_cast<const uint4*>(src_b + static_cast<int64_t>(row) * ld + vcol0 + i);
+    *reinterpret_cast<uint4*>(a.v_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + t) * D +
+                              i) = val;
+  }
+  cp_async_wait_all();
+  fence_proxy_async_smem();    // W tiles (and later U) are read by the tensor core
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (a.rope_on) {
+    const double inv_turn = 0.15915494309189533577;  // 1 / (2 pi)
+    for (int idx = tid; idx < (D / 2) * kPtTT; idx += kPtThreads) {
+      const int i = idx / kPtTT, tl = idx - i * kPtTT;
+      double f = static_cast<double>(t0 + tl) * theta[i] * inv_turn;
+      f -= rint(f);
+      float s, c;
+      sincospif(static_cast<float>(2.0 * f), &s, &c);
+      cs[idx] = make_float2(c, s);
+    }
+  }
+  __syncthreads();
+
+  // 2. per head
+  const int r = tid & (kPtTT - 1);         // position row == TMEM lane
+  const int part = tid >> 7;               // conv chunks j = part (mod 2); pairs of half `part`
+  const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+  const uint32_t u_hi = smem_addr(smem + L.off_u);
+  const uint32_t u_lo = u_hi + L.u_bytes;
+  const uint32_t w_base = smem_addr(smem + L.off_w);
+  const uint32_t idesc = make_idesc_bf16(kPtTT, D, false);
+  const bf16* zrow = z + (r + kPtHalo) * ZC;
+  const int t = t0 + r;
+  bool ok = true;
+
+  auto conv = [&](int hh) {
+#pragma unroll
+    for (int j = part; j < NCH; j += 2) {
+      float acc[8];
+      const float4* w4 = reinterpret_cast<const float4*>(ws) + hh * D + j * 8;   // taps of 8 channels
+      float4 w[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w[e] = w4[e];
+      {
+        float v[8];
+        unpack8(*reinterpret_cast<const uint4*>(z + (r + kPtHalo) * ZC + hh * D + j * 8), v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = w[e].x * v[e];
+      }
+#pragma unroll
+      for (int k = 1; k < 4; ++k) {
+        float v[8];
+        unpack8(*reinterpret_cast<const uint4*>(z + (r + kPtHalo - k) * ZC + hh * D + j * 8), v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float wk = k == 1 ? w[e].y : (k == 2 ? w[e].z : w[e].w);
+          acc[e] = fmaf(wk, v[e], acc[e]);
+        }
+      }
+      uint4 hi, lo;
+      uint32_t* hp = reinterpret_cast<uint32_t*>(&hi);
+      uint32_t* lp = reinterpret_cast<uint32_t*>(&lo);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
+        const float2 hf = __bfloat1622float2(h2);
+        hp[e] = *reinterpret_cast<const uint32_t*>(&h2);
+        lp[e] = pack2(acc[2 * e] - hf.x, acc[2 * e + 1] - hf.y);
+      }
+      const uint32_t off = swz_offset(r, j * 16, kRowBytes);
+      *reinterpret_cast<uint4*>(smem + L.off_u + off) = hi;
+      *reinterpret_cast<uint4*>(smem + L.off_u + L.u_bytes + off) = lo;
+    }
+  };
+
+  auto issue_mma = [&](int hh) {
+    const uint32_t dt = tmem + (hh & 1) * D;
+    const uint32_t wb = w_base + hh * L.w_bytes;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk)
+      mma_ss(dt, make_smem_desc(u_hi + kk * 32, 16, kSbo, kSwz),
+             make_smem_desc(wb + kk * 32, 16, kSbo, kSwz), idesc, kk > 0 ? 1u : 0u);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk)
+      mma_ss(dt, make_smem_desc(u_lo + kk * 32, 16, kSbo, kSwz),
+             make_smem_desc(wb + kk * 32, 16, kSbo, kSwz), idesc, 1u);
+    mma_commit(&mma_done[hh & 1]);
+  };
+
+  auto epilogue = [&](int hh) {
+    const uint32_t col = (hh & 1) * D + part * Q4;
+    uint32_t ya[Q4], yb[Q4];                 // channels part*Q4 + e and D/2 + part*Q4 + e
+    if constexpr (Q4 == 8) {
+      tmem_ld8(trow + col, ya);
+      tmem_ld8(trow + col + D / 2, yb);
+    } else {
+      tmem_ld16(trow + col, ya);
+      tmem_ld16(trow + col + D / 2, yb);
+    }
+    tmem_wait_ld();
+    if (t >= S) return;
+    const int i0 = part * Q4;
+    float lo[Q4], hi[Q4];
+#pragma unroll
+    for (int e = 0; e < Q4; ++e) {
+      lo[e] = __uint_as_float(ya[e]);
+      hi[e] = __uint_as_float(yb[e]);
+    }
+    if (a.qk_mean) {
+      const bool is_q = hh < G;
+      // y[e] += (q~ + k~) / 2 over channels c0 + e (q~: this head, or the
+      // mean of the group's query heads for the key head)
+      auto add_mean = [&](float (&y)[Q4], int c0) {
+#pragma unroll
+        for (int q8 = 0; q8 < Q4 / 8; ++q8) {
+          float kp[8], qp[8];
+          unpack8(*reinterpret_cast<const uint4*>(zrow + QC + c0 + q8 * 8), kp);
+          if (is_q) {
+            unpack8(*reinterpret_cast<const uint4*>(zrow + hh * D + c0 + q8 * 8), qp);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) qp[e] = 0.f;
+            for (int hl = 0; hl < G; ++hl) {
+              float v[8];
+              unpack8(*reinterpret_cast<const uint4*>(zrow + hl * D + c0 + q8 * 8), v);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) qp[e] += v[e];
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) qp[e] /= static_cast<float>(G);
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) y[q8 * 8 + e] += 0.5f * (qp[e] + kp[e]);
+        }
+      };
+      add_mean(lo, i0);
+      add_mean(hi, i0 + D / 2);
+    }
+    if (a.rope_on) {
+#pragma unroll
+      for (int e = 0; e < Q4; ++e) {
+        const float2 c = cs[(i0 + e) * kPtTT + r];
+        const float x0 = lo[e], x1 = hi[e];
+        lo[e] = x0 * c.x - x1 * c.y;
+        hi[e] = x0 * c.y + x1 * c.x;
+      }
+    }
+    bf16* dst = hh < G ? a.q_out + ((static_cast<int64_t>(b) * S + t) * a.Hq + g * G + hh) * D
+                       : a.k_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + t) * D;
+#pragma unroll
+    for (int q8 = 0; q8 < Q4 / 8; ++q8) {
+      uint4 pl, ph;
+      pl.x = pack2(lo[q8 * 8 + 0], lo[q8 * 8 + 1]);
+      pl.y = pack2(lo[q8 * 8 + 2], lo[q8 * 8 + 3]);
+      pl.z = pack2(lo[q8 * 8 + 4], lo[q8 * 8 + 5]);
+      pl.w = pack2(lo[q8 * 8 + 6], lo[q8 * 8 + 7]);
+      ph.x = pack2(hi[q8 * 8 + 0], hi[q8 * 8 + 1]);
+      ph.y = pack2(hi[q8 * 8 + 2], hi[q8 * 8 + 3]);
+      ph.z = pack2(hi[q8 * 8 + 4], hi[q8 * 8 + 5]);
+      ph.w = pack2(hi[q8 * 8 + 6], hi[q8 * 8 + 7]);
+      *reinterpret_cast<uint4*>(dst + i0 + q8 * 8) = pl;
+      *reinterpret_cast<uint4*>(dst + D / 2 + i0 + q8 * 8) = ph;
+    }
+  };
+
+  for (int hh = 0; hh < NH; ++hh) {
+    if (hh > 0) {
+      // MMA(hh - 1) complete: U may be overwritten, accumulator (hh - 1) & 1 is final
+      ok = ok && mbar_wait(&mma_done[(hh - 1) & 1], ((hh - 1) >> 1) & 1, &abort_flag, a.dev_err);
+      tc_fence_after();
+    }
+    if (ok) conv(hh);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    ok = ok && !abort_flag;
+    if (ok && tid == 0) issue_mma(hh);
+    if (ok && hh > 0) epilogue(hh - 1);
+  }
+  ok = ok && mbar_wait(&mma_done[(NH - 1) & 1], ((NH - 1) >> 1) & 1, &abort_flag, a.dev_err);
+  tc_fence_after();
+  if (ok) epilogue(NH - 1);
+
+  // 4. decode state, written by the CTA that holds position S-1 (rows S-KH .. S-1
+  // are staged; rows before position 0 are zero).
+  if (a.len != nullptr && t0 <= S - 1 && S - 1 < t0 + kPtTT) {
+    const int KH = K - 1, Hq = a.Hq, Hkv = a.Hkv;
+    for (int rr = 0; rr < KH; ++rr) {
+      const bf16* zr = z + (S - KH + rr - t0 + kPtHalo) * ZC;
+      for (int c = tid; c < QC + D; c += kPtThreads) {
+        if (c < QC)
+          a.hist_q[(static_cast<int64_t>(b) * KH + rr) * Hq * D + qcol0 + c] = zr[c];
+        else
+          a.hist_k[(static_cast<int64_t>(b) * KH + rr) * Hkv * D + g * D + (c - QC)] = zr[c];
+      }
+    }
+    if (a.v_prev)
+      for (int i = tid; i < D; i += kPtThreads)
+        a.v_prev[static_cast<int64_t>(b) * Hkv * D + g * D + i] =
+            src_b[static_cast<int64_t>(S - 1) * ld + vcol0 + i];
+    if (g == 0 && tid == 0) a.len[b] = S;
+  }
+
+  if (abort_flag && tid == 0) {
+    // Do not release TMEM while an MMA might still write it.
+    mma_commit(drain);
+    const long long c0 = clock64();
+    while (!mbar_try_wait(drain, 0) && clock64() - c0 < kWaitLimitCycles) {
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 2 * D);
+  }
+}
+
+template <int D>
+cudaError_t launch_d(const PreAttnArgs<bf16>& a, cudaStream_t stream) {
+  const PtLayout L = pt_layout(D, a.G);
+  cudaError_t e = cudaFuncSetAttribute(pre_attn_tc_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(L.bytes));
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.S + kPtTT - 1) / kPtTT, a.Hkv, a.B);
+  pre_attn_tc_kernel<D><<<grid, kPtThreads, L.bytes, stream>>>(a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool pre_attn_tc_supported(const PreAttnArgs<bf16>& a) {
+  if (a.d != 32 && a.d != 64) return false;
+  if (a.K < 1 || a.K > 4 || a.wq_chan == nullptr || a.wk_chan == nullptr) return false;
+  if (a.wq_seq == nullptr || a.wk_seq == nullptr) return false;
+  return pt_layout(a.d, a.G).bytes <= 227 * 1024;
+}
+
+cudaError_t launch_pre_attn_tc(const PreAttnArgs<bf16>& a, cudaStream_t stream) {
+  return a.d == 32 ? launch_d<32>(a, stream) : launch_d<64>(a, stream);
+}
+
+}  // namespace ccgqa

@@ -223,6 +223,12 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[15])
       : "memory");
 }
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -269,6 +275,15 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool b_mn_m
 // tile written with the 128B swizzle (the layout TMA SWIZZLE_128B produces).
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
   return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+// Byte offset of element (row, col) in a K-major tile whose rows are `row_bytes`
+// wide (64 or 128), with the matching TMA / UMMA swizzle (64B: address bits
+// [4,6) ^= bits [7,9); 128B: bits [4,7) ^= bits [7,10)).  The tile must start
+// on a 512-byte (64B swizzle) or 1024-byte (128B swizzle) boundary.
+__device__ __forceinline__ uint32_t swz_offset(uint32_t row, uint32_t col_byte, uint32_t row_bytes) {
+  const uint32_t off = row * row_bytes + col_byte;
+  return row_bytes == 128 ? (off ^ (((off >> 7) & 7u) << 4)) : (off ^ (((off >> 7) & 3u) << 4));
 }
 
 __device__ __forceinline__ uint32_t elect_one_lane() {

@@ -130,3 +130,40 @@ def test_launches_are_counted():
     n0 = B.ccgqa_launch_count()
     _run(w, inp)
     assert B.ccgqa_launch_count() - n0 == 3   # projection, pre-attention, attention
+
+
+def _growing_score_inputs(w, slope, seed=0):
+    """Packed q|k|v with q along e_0 and key t along e_0 scaled by slope * t,
+    so q.k / sqrt(d) = slope * t: every later 64-key half holds scores far
+    above the running max, and the softmax must raise it (and rescale O)
+    over and over.  Values are whole numbers, exact in bf16."""
+    inp = make_inputs(w, seed=seed)
+    d, Hq, Hkv = w.d, w.Hq, w.Hkv
+    x = inp["x"].float()
+    x[..., : (Hq + Hkv) * d] = 0.0
+    q = x[..., : Hq * d].view(w.B, w.S, Hq, d)
+    k = x[..., Hq * d: (Hq + Hkv) * d].view(w.B, w.S, Hkv, d)
+    q[..., 0] = float(d) ** 0.5 if d in (64,) else 1.0
+    scale_k = slope * float(d) ** 0.5 / float(q[0, 0, 0, 0])
+    t = torch.arange(w.S, dtype=torch.float32)
+    k[..., 0] = torch.round(scale_k * t)[None, :, None]
+    inp["x"] = x.to(w.torch_dtype)
+    return inp
+
+
+@pytest.mark.parametrize("slope", [0.125, 2.0])
+@pytest.mark.parametrize("w", [
+    W2.with_(name="grow_d32", B=1, S=700, E=512, C=1, Hq=16, Hkv=4, conv_width=0, qk_mean=False,
+             value_shift=False, rope_base=0.0, packed_input=True),
+    W3.with_(name="grow_d64", B=1, S=520, E=512, C=1, Hq=8, Hkv=2, conv_width=0, qk_mean=False,
+             value_shift=False, rope_base=0.0, packed_input=True),
+    W5.with_(name="grow_d128", B=1, S=390, rope_base=0.0),
+], ids=lambda w: w.name)
+def test_prefill_growing_scores_raise_running_max(w, slope):
+    # slope 1/8 nat per key: each half's sum overshoots (p up to 2^11);
+    # slope 2: the first pass overflows to inf before the running max is raised
+    inp = _growing_score_inputs(w, slope)
+    lay, out = _run(w, inp, use_cache=False)
+    got = out.float().cpu().numpy()
+    assert np.all(np.isfinite(got))
+    check_prefill(w, inp, 0, got[0], what=f"{w.name} slope={slope}")
