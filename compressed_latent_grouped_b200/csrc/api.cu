@@ -37,6 +37,15 @@ struct Geo {
 };
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// theta_i / (2 pi) * 2^64 with theta_i = base^(-2i/d) (RoPE, "Compressed
+// Convolutional Attention", Methodologie item 4), rounded to an integer in
+// extended precision; below 2^62 since theta_i <= 1.
+uint64_t rope_turn_fraction(double log2_base, int i, int d) {
+  const long double th = exp2l(-(2.0L * i / d) * static_cast<long double>(log2_base));
+  const long double two_pi = 6.283185307179586476925286766559005768L;
+  return static_cast<uint64_t>(llroundl(th / two_pi * 18446744073709551616.0L));
+}
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
@@ -172,6 +181,8 @@ ccgqa_status run_prefill(const Geo& g, const ccgqa_weights* w, const void* x, in
   a.value_shift = g.value_shift;
   a.rope_on = g.rope_on;
   a.rope_log2_base = g.rope_log2_base;
+  if (g.rope_on)
+    for (int i = 0; i < g.d / 2; ++i) a.rope_frac[i] = rope_turn_fraction(g.rope_log2_base, i, g.d);
   a.wq_seq = static_cast<const T*>(w->conv_q_seq);
   a.wq_chan = static_cast<const T*>(w->conv_q_chan);
   a.wk_seq = static_cast<const T*>(w->conv_k_seq);

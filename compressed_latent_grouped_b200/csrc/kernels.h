@@ -36,6 +36,10 @@ struct PreAttnArgs {
   int qk_mean, value_shift;
   int rope_on;
   double rope_log2_base;
+  // theta_i / (2 pi) as a 0.64 fixed-point fraction of a turn, i < d/2: the
+  // product t * rope_frac[i] modulo 2^64 is the angle t * theta_i reduced
+  // modulo one turn, exactly (used by the tensor-core pre-attention kernel)
+  uint64_t rope_frac[64];
   const T *wq_seq, *wq_chan, *wk_seq, *wk_chan;  // chan may be null
   T* q_out;              // [B, S, Hq, d]
   T* k_out;              // [B, Hkv, kv_cap, d]

@@ -6,11 +6,11 @@
 //
 // One CTA owns 128 consecutive positions of one kv group (its G query heads,
 // its key head and its value head) of one sequence:
-//   1. the group's q~ | k~ rows [t0 - 3, t0 + 128) are copied into shared
-//      memory with 16-byte cp.async, the G + 1 mix weights W_h [d_out, d_in]
-//      straight into the swizzled K-major layout of a UMMA B operand, the conv
-//      taps as fp32, and a cos/sin table per (pair, position) is formed (angle
-//      reduced modulo one turn in fp64);
+//   1. the group's q~ | k~ | v~ rows [t0 - 3, t0 + 128), the G + 1 mix weights
+//      W_h [d_out, d_in] (straight into the swizzled K-major layout of a UMMA
+//      B operand) and the conv taps are copied into shared memory with 16-byte
+//      cp.async; meanwhile a cos/sin table per (pair, position) is formed, the
+//      angle t theta_i reduced modulo one turn exactly in 64-bit fixed point;
 //   2. per head h (G query heads, then the key head):
 //        conv   one thread per (position, 16-byte channel chunk): u = sum_k
 //               w[c, k] z[t - k, c] in fp32, split as u = hi + lo with hi, lo
@@ -22,10 +22,12 @@
 //               tcgen05.ld of Y_h, QK-mean from the staged pre-conv rows, RoPE on
 //               the pairs (i, i + d/2) it holds, bf16 store.
 //      The epilogue of head h - 1 runs while the tensor core computes head h.
-//   3. value-shift: each v row is gathered from rows t and t - 1 of v~, a
-//      bit-exact copy.
+//   3. value-shift: each v row is gathered from staged rows t and t - 1 of
+//      v~, a bit-exact copy.
 //   4. the CTA holding the last position writes the decode state.
 // Every wait is bounded; no cluster multicast is used.
+#include <type_traits>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -39,16 +41,16 @@ constexpr int kPtTT = 128;     // positions per CTA == MMA M == TMEM lanes
 constexpr int kPtHalo = 3;     // the conv reaches back K - 1 <= 3 rows
 
 struct PtLayout {
-  int ZC;                      // staged row width in elements: (G + 1) d + 8
+  int ZC;                      // staged row width in elements: (G + 2) d + 8
   uint32_t u_bytes, w_bytes;   // one A tile (hi or lo), one head's B tile
-  uint32_t off_u, off_w, off_z, off_cs, off_ws, off_theta, off_bar, bytes;
+  uint32_t off_u, off_w, off_z, off_cs, off_ws, off_tr, off_bar, bytes;
 };
 
 // Byte layout of the dynamic shared memory (from a 1024-byte aligned base).
 __host__ __device__ inline PtLayout pt_layout(int d, int G) {
   PtLayout L;
   const uint32_t row = static_cast<uint32_t>(d) * 2;
-  L.ZC = (G + 1) * d + 8;      // + 16 bytes: an odd number of 16-byte units per row
+  L.ZC = (G + 2) * d + 8;      // q | k | v, + 16 bytes: an odd number of 16-byte units per row
   L.u_bytes = kPtTT * row;
   L.w_bytes = static_cast<uint32_t>(d) * row;
   L.off_u = 0;                                      // U_hi, U_lo
@@ -56,8 +58,8 @@ __host__ __device__ inline PtLayout pt_layout(int d, int G) {
   L.off_z = L.off_w + (G + 1) * L.w_bytes;          // [131][ZC] bf16
   L.off_cs = L.off_z + ((static_cast<uint32_t>(kPtTT + kPtHalo) * L.ZC * 2 + 15u) & ~15u);
   L.off_ws = L.off_cs + static_cast<uint32_t>(d / 2) * kPtTT * 8;   // [d/2][128] float2
-  L.off_theta = L.off_ws + static_cast<uint32_t>(G + 1) * d * 16;  // [(G+1) d][4] float
-  L.off_bar = L.off_theta + static_cast<uint32_t>(d / 2) * 8;      // [d/2] double
+  L.off_tr = L.off_ws + static_cast<uint32_t>(G + 1) * d * 16;     // [(G+1) d][4] float
+  L.off_bar = L.off_tr + static_cast<uint32_t>(G + 1) * d * 4 * 2;  // raw taps, <= 4 per channel
   L.bytes = L.off_bar + 64 + 1024;                  // barriers + alignment slack
   return L;
 }
@@ -79,6 +81,15 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
     f[2 * i + 1] = p.y;
   }
 }
+// d = a * b + c on a pair (one packed fp32x2 instruction), rounded like fmaf
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)),
+        "l"(*reinterpret_cast<const uint64_t*>(&c)));
+  return *reinterpret_cast<float2*>(&d);
+}
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -86,7 +97,7 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 
 template <int D>
 __global__ void __launch_bounds__(kPtThreads)
-    pre_attn_tc_kernel(const PreAttnArgs<bf16> a) {
+    pre_attn_tc_kernel(const __grid_constant__ PreAttnArgs<bf16> a) {
   constexpr uint32_t kRowBytes = D * 2;                 // 64: 64B swizzle, 128: 128B swizzle
   constexpr uint32_t kSwz = (D == 32) ? kSwizzle64B : kSwizzle128B;
   constexpr uint32_t kSbo = 8 * kRowBytes;
@@ -103,7 +114,7 @@ __global__ void __launch_bounds__(kPtThreads)
   bf16* z = reinterpret_cast<bf16*>(smem + L.off_z);
   float2* cs = reinterpret_cast<float2*>(smem + L.off_cs);
   float* ws = reinterpret_cast<float*>(smem + L.off_ws);
-  double* theta = reinterpret_cast<double*>(smem + L.off_theta);
+  bf16* tr = reinterpret_cast<bf16*>(smem + L.off_tr);
   uint64_t* mma_done = reinterpret_cast<uint64_t*>(smem + L.off_bar);   // [2]
   uint64_t* drain = mma_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -127,49 +138,53 @@ __global__ void __launch_bounds__(kPtThreads)
     tmem_relinquish();
   }
 
-  // 1. staging
+  // 1. staging, all by cp.async: the q~ | k~ | v~ rows, the mix weights and
+  // the raw conv taps
   {
-    const int cq = QC / 8, per_row = cq + NCH;
-    for (int idx = tid; idx < (kPtTT + kPtHalo) * per_row; idx += kPtThreads) {
-      const int r = idx / per_row, c = idx - r * per_row;
+    // a warp per staged row, lanes over its 16-byte chunks
+    const int cq = QC / 8, per_row = cq + 2 * NCH;
+    const int lane = tid & 31;
+    for (int r = warp; r < kPtTT + kPtHalo; r += kPtThreads / 32) {
       const int t = t0 - kPtHalo + r;
-      const int col = c < cq ? qcol0 + c * 8 : kcol0 + (c - cq) * 8;
-      bf16* dst = z + r * ZC + c * 8;               // q channels, then the key head's
-      if (t >= 0 && t < S)
-        cp_async16(dst, src_b + static_cast<int64_t>(t) * ld + col);
-      else
-        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+      const bool in = t >= 0 && t < S;
+      const bf16* srow = src_b + static_cast<int64_t>(in ? t : 0) * ld;
+      for (int c = lane; c < per_row; c += 32) {
+        const int col = c < cq ? qcol0 + c * 8
+                               : (c < cq + NCH ? kcol0 + (c - cq) * 8 : vcol0 + (c - cq - NCH) * 8);
+        bf16* dst = z + r * ZC + c * 8;
+        if (in)
+          cp_async16(dst, srow + col);
+        else
+          *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+      }
     }
     // W_h row n (output channel), chunk j of the input channels -> B operand
     for (int idx = tid; idx < NH * D * NCH; idx += kPtThreads) {
-      const int hh = idx / (D * NCH), rem = idx - hh * (D * NCH);
-      const int n = rem / NCH, j = rem - n * NCH;
+      const int hh = idx / (D * NCH), rem = idx % (D * NCH);   // D * NCH: a power of two
+      const int n = rem / NCH, j = rem % NCH;
       const bf16* w = hh < G ? a.wq_chan + (static_cast<int64_t>(g * G + hh) * D + n) * D
                              : a.wk_chan + (static_cast<int64_t>(g) * D + n) * D;
       cp_async16(smem + L.off_w + hh * L.w_bytes + swz_offset(n, j * 16, kRowBytes), w + j * 8);
     }
-    // conv taps w[c][k] as fp32, zero past K
-    for (int idx = tid; idx < NH * D * 4; idx += kPtThreads) {
-      const int hc = idx >> 2, k = idx & 3;
-      const int hh = hc / D, c = hc - hh * D;
-      const bf16* w = hh < G ? a.wq_seq + (static_cast<int64_t>(g * G + hh) * D + c) * K
-                             : a.wk_seq + (static_cast<int64_t>(g) * D + c) * K;
-      ws[idx] = k < K ? __bfloat162float(w[k]) : 0.f;
+    // taps [channel][K]: the group's G d query channels, then its d key channels
+    const int nq = G * D * K / 8, nk = D * K / 8;
+    for (int idx = tid; idx < nq + nk; idx += kPtThreads) {
+      const bf16* w = idx < nq ? a.wq_seq + static_cast<int64_t>(g) * G * D * K + idx * 8
+                               : a.wk_seq + static_cast<int64_t>(g) * D * K + (idx - nq) * 8;
+      cp_async16(tr + idx * 8, w);
     }
-    if (a.rope_on)
-      for (int i = tid; i < D / 2; i += kPtThreads)
-        theta[i] = exp2(-(2.0 * i / D) * a.rope_log2_base);
   }
-  // value-shift while the copies fly: v[t, :d/2] = v~[t, :d/2], v[t, d/2:] = v~[t-1, d/2:]
-  for (int idx = tid; idx < kPtTT * NCH; idx += kPtThreads) {
-    const int tl = idx / NCH, i = (idx - tl * NCH) * 8;
-    const int t = t0 + tl;
-    if (t >= S) continue;
-    const int row = (a.value_shift && i >= D / 2) ? t - 1 : t;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (row >= 0) val = *reinterpret_cast<const uint4*>(src_b + static_cast<int64_t>(row) * ld + vcol0 + i);
-    *reinterpret_cast<uint4*>(a.v_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + t) * D +
-                              i) = val;
+  // RoPE table while the copies fly: (cos, sin) of t * theta_i, the angle taken
+  // modulo one turn exactly in 64-bit fixed point, then |2 pi f| <= pi.
+  if (a.rope_on) {
+    for (int idx = tid; idx < (D / 2) * kPtTT; idx += kPtThreads) {
+      const int i = idx / kPtTT, tl = idx - i * kPtTT;
+      const uint64_t ph = static_cast<uint64_t>(t0 + tl) * a.rope_frac[i];
+      const float f = static_cast<float>(static_cast<int64_t>(ph)) * 5.42101086242752217e-20f;
+      float sn, cn;
+      __sincosf(6.28318530717958648f * f, &sn, &cn);
+      cs[idx] = make_float2(cn, sn);
+    }
   }
   cp_async_wait_all();
   fence_proxy_async_smem();    // W tiles (and later U) are read by the tensor core
@@ -177,16 +192,20 @@ __global__ void __launch_bounds__(kPtThreads)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (a.rope_on) {
-    const double inv_turn = 0.15915494309189533577;  // 1 / (2 pi)
-    for (int idx = tid; idx < (D / 2) * kPtTT; idx += kPtThreads) {
-      const int i = idx / kPtTT, tl = idx - i * kPtTT;
-      double f = static_cast<double>(t0 + tl) * theta[i] * inv_turn;
-      f -= rint(f);
-      float s, c;
-      sincospif(static_cast<float>(2.0 * f), &s, &c);
-      cs[idx] = make_float2(c, s);
-    }
+  // conv taps as fp32 [channel][4], zero past K
+  for (int idx = tid; idx < NH * D * 4; idx += kPtThreads) {
+    const int hc = idx >> 2, k = idx & 3;
+    ws[idx] = k < K ? __bfloat162float(tr[hc * K + k]) : 0.f;
+  }
+  // 3. value-shift out of the staged rows: v[t, :d/2] = v~[t, :d/2] and
+  // v[t, d/2:] = v~[t-1, d/2:] (the staged row before position 0 is zero)
+  for (int idx = tid; idx < kPtTT * NCH; idx += kPtThreads) {
+    const int tl = idx / NCH, i = (idx - tl * NCH) * 8;
+    const int t = t0 + tl;
+    if (t >= S) continue;
+    const int row = (a.value_shift && i >= D / 2) ? tl + kPtHalo - 1 : tl + kPtHalo;
+    *reinterpret_cast<uint4*>(a.v_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + t) * D +
+                              i) = *reinterpret_cast<const uint4*>(z + row * ZC + QC + D + i);
   }
   __syncthreads();
 
@@ -202,28 +221,29 @@ __global__ void __launch_bounds__(kPtThreads)
   const int t = t0 + r;
   bool ok = true;
 
-  auto conv = [&](int hh) {
+  // conv of head hh for chunks j = P, P + 2, ... of row r (P: compile-time part)
+  auto conv_part = [&](int hh, auto part_c) {
+    constexpr int P = decltype(part_c)::value;
 #pragma unroll
-    for (int j = part; j < NCH; j += 2) {
-      float acc[8];
+    for (int j = P; j < NCH; j += 2) {
       const float4* w4 = reinterpret_cast<const float4*>(ws) + hh * D + j * 8;   // taps of 8 channels
+      const bf16* zc = z + (r + kPtHalo) * ZC + hh * D + j * 8;
       float4 w[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) w[e] = w4[e];
-      {
-        float v[8];
-        unpack8(*reinterpret_cast<const uint4*>(z + (r + kPtHalo) * ZC + hh * D + j * 8), v);
+      float2 acc[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = w[e].x * v[e];
-      }
+      for (int k = 0; k < 4; ++k) {
+        const uint4 zz = *reinterpret_cast<const uint4*>(zc - k * ZC);
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&zz);
 #pragma unroll
-      for (int k = 1; k < 4; ++k) {
-        float v[8];
-        unpack8(*reinterpret_cast<const uint4*>(z + (r + kPtHalo - k) * ZC + hh * D + j * 8), v);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float wk = k == 1 ? w[e].y : (k == 2 ? w[e].z : w[e].w);
-          acc[e] = fmaf(wk, v[e], acc[e]);
+        for (int e = 0; e < 4; ++e) {
+          const float2 v = __bfloat1622float2(h2[e]);
+          const float2 wk = k == 0 ? make_float2(w[2 * e].x, w[2 * e + 1].x)
+                          : k == 1 ? make_float2(w[2 * e].y, w[2 * e + 1].y)
+                          : k == 2 ? make_float2(w[2 * e].z, w[2 * e + 1].z)
+                                   : make_float2(w[2 * e].w, w[2 * e + 1].w);
+          acc[e] = k == 0 ? make_float2(wk.x * v.x, wk.y * v.y) : ffma2(wk, v, acc[e]);
         }
       }
       uint4 hi, lo;
@@ -231,15 +251,21 @@ __global__ void __launch_bounds__(kPtThreads)
       uint32_t* lp = reinterpret_cast<uint32_t*>(&lo);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[e].x, acc[e].y);
         const float2 hf = __bfloat1622float2(h2);
         hp[e] = *reinterpret_cast<const uint32_t*>(&h2);
-        lp[e] = pack2(acc[2 * e] - hf.x, acc[2 * e + 1] - hf.y);
+        lp[e] = pack2(acc[e].x - hf.x, acc[e].y - hf.y);
       }
       const uint32_t off = swz_offset(r, j * 16, kRowBytes);
       *reinterpret_cast<uint4*>(smem + L.off_u + off) = hi;
       *reinterpret_cast<uint4*>(smem + L.off_u + L.u_bytes + off) = lo;
     }
+  };
+  auto conv = [&](int hh) {
+    if (part == 0)
+      conv_part(hh, std::integral_constant<int, 0>{});
+    else
+      conv_part(hh, std::integral_constant<int, 1>{});
   };
 
   auto issue_mma = [&](int hh) {
@@ -364,10 +390,11 @@ __global__ void __launch_bounds__(kPtThreads)
           a.hist_k[(static_cast<int64_t>(b) * KH + rr) * Hkv * D + g * D + (c - QC)] = zr[c];
       }
     }
-    if (a.v_prev)
+    if (a.v_prev) {
+      const bf16* zr = z + (S - 1 - t0 + kPtHalo) * ZC + QC + D;
       for (int i = tid; i < D; i += kPtThreads)
-        a.v_prev[static_cast<int64_t>(b) * Hkv * D + g * D + i] =
-            src_b[static_cast<int64_t>(S - 1) * ld + vcol0 + i];
+        a.v_prev[static_cast<int64_t>(b) * Hkv * D + g * D + i] = zr[i];
+    }
     if (g == 0 && tid == 0) a.len[b] = S;
   }
 
