@@ -15,9 +15,10 @@
 //                                   P^T a 16 x 128 tile)
 //                O  += P_c V_c     (d = 32: M = 128, P rows 0..G-1 are the
 //                                   heads, the other rows stay zero; N = d)
-//   warps 2-5  softmax: thread k owns key k of the chunk and its G scores; the
-//              chunk max per head is reduced with shuffles and a named barrier,
-//              exp2 once per (key, head), P written to shared memory.  Keys at
+//   warps 2-5  softmax: thread k owns key k of the chunk and its G scores; one
+//              barrier-OR tells whether any score passed the running max by
+//              more than 2^8 (only then is the chunk max reduced and O
+//              rescaled), exp2 once per (key, head), P written to shared memory.  Keys at
 //              or past len + 1 are masked and their V rows zeroed (a stale cache
 //              row may hold anything, and 0 * NaN is NaN in the MMA).
 // Each split writes (max, sum, unnormalised output) per head; the last CTA of a
@@ -80,12 +81,14 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* kv_full = bars;                  // [kStages]
-  uint64_t* kv_empty = kv_full + C::kStages; // [kStages]
-  uint64_t* q_ready = kv_empty + C::kStages; // 128 arrivals: Q^T and zeroed P built
+  uint64_t* k_full = bars;                   // [kStages] K ring
+  uint64_t* k_empty = k_full + C::kStages;   // [kStages] released when S of that chunk is done
+  uint64_t* v_full = k_empty + C::kStages;   // [kStages] V ring
+  uint64_t* v_empty = v_full + C::kStages;   // [kStages] released when PV of that chunk is done
+  uint64_t* q_ready = v_empty + C::kStages;  // 128 arrivals: Q^T and zeroed P built
   uint64_t* s_full = q_ready + 1;            // [2] S^T buffers
-  uint64_t* p_full = s_full + 2;             // 128 arrivals
-  uint64_t* o_done = p_full + 1;             // [2] PV of chunks using P buffer 0 / 1
+  uint64_t* p_full = s_full + 2;             // [2] 128 arrivals: P of chunks using buffer 0 / 1
+  uint64_t* o_done = p_full + 2;             // [2] PV of chunks using P buffer 0 / 1
   uint64_t* drain = o_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffBar + 256);
   float* red = reinterpret_cast<float*>(smem + C::kOffBar + 512);   // [2][4 warps][kQRows]
@@ -104,13 +107,16 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
 
   if (tid == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     mbar_init(q_ready, 128);
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
-    mbar_init(p_full, 128);
+    mbar_init(&p_full[0], 128);
+    mbar_init(&p_full[1], 128);
     mbar_init(&o_done[0], 1);
     mbar_init(&o_done[1], 1);
     mbar_init(drain, 1);
@@ -135,19 +141,46 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // One thread streams K and V through two rings, polling both without
+    // blocking on either: a K slot frees as soon as the S of its chunk is
+    // computed, well before the PV that frees the V slot, so the K loads run
+    // ahead of the V loads.
     if (lane == 0) {
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
-      for (int c = 0; c < n_ch; ++c) {
-        const int st = c % C::kStages;
-        if (!mbar_wait(&kv_empty[st], ((c / C::kStages) & 1) ^ 1, &abort_flag, a.dev_err)) break;
-        mbar_arrive_expect_tx(&kv_full[st], 2 * C::kTileBytes);
+      volatile int* abort_v = &abort_flag;
+      int ck = 0, cv = 0;
+      long long t_last = clock64();
+      while (ck < n_ch || cv < n_ch) {
+        bool progress = false;
+        if (ck < n_ch && mbar_test(&k_empty[ck % C::kStages], ((ck / C::kStages) & 1) ^ 1)) {
+          const int st = ck % C::kStages;
+          mbar_arrive_expect_tx(&k_full[st], C::kTileBytes);
 #pragma unroll
-        for (int p = 0; p < C::kPanels; ++p) {
-          tma_load_3d(smem + C::kOffK + st * C::kTileBytes + p * C::kPanelBytes, &tmK, &kv_full[st],
-                      p * C::kPanelCols, k0 + c * kChunk, bg);
-          tma_load_3d(smem + C::kOffV + st * C::kTileBytes + p * C::kPanelBytes, &tmV, &kv_full[st],
-                      p * C::kPanelCols, k0 + c * kChunk, bg);
+          for (int p = 0; p < C::kPanels; ++p)
+            tma_load_3d(smem + C::kOffK + st * C::kTileBytes + p * C::kPanelBytes, &tmK, &k_full[st],
+                        p * C::kPanelCols, k0 + ck * kChunk, bg);
+          ++ck;
+          progress = true;
+        }
+        if (cv < n_ch && mbar_test(&v_empty[cv % C::kStages], ((cv / C::kStages) & 1) ^ 1)) {
+          const int st = cv % C::kStages;
+          mbar_arrive_expect_tx(&v_full[st], C::kTileBytes);
+#pragma unroll
+          for (int p = 0; p < C::kPanels; ++p)
+            tma_load_3d(smem + C::kOffV + st * C::kTileBytes + p * C::kPanelBytes, &tmV, &v_full[st],
+                        p * C::kPanelCols, k0 + cv * kChunk, bg);
+          ++cv;
+          progress = true;
+        }
+        if (progress) {
+          t_last = clock64();
+        } else if (*abort_v || clock64() - t_last > kWaitLimitCycles) {
+          if (!*abort_v) {
+            *abort_v = 1;
+            raise_dev_err(a.dev_err, CCGQA_DEVERR_TIMEOUT);
+          }
+          break;
         }
       }
     }
@@ -173,6 +206,7 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
           mma_ss(tmem + C::kColS + (c & 1) * 16, ad, bd, idesc_s, k > 0 ? 1u : 0u);
         }
         mma_commit(&s_full[c & 1]);
+        mma_commit(&k_empty[st]);   // K slot free once this S is computed
       };
       auto issue_pv = [&](int c) {
         const int st = c % C::kStages;
@@ -192,27 +226,44 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
             mma_ss(tmem + C::kColO, pd, vd, idesc_o, (c > 0 || k > 0) ? 1u : 0u);
         }
         mma_commit(&o_done[c & 1]);
-        mma_commit(&kv_empty[st]);
+        mma_commit(&v_empty[st]);
       };
       bool ok = mbar_wait(q_ready, 0, &abort_flag, a.dev_err);
       for (int c = 0; ok && c < 2 && c < n_ch; ++c) {
-        if (!mbar_wait(&kv_full[c % C::kStages], (c / C::kStages) & 1, &abort_flag, a.dev_err)) {
+        if (!mbar_wait(&k_full[c % C::kStages], (c / C::kStages) & 1, &abort_flag, a.dev_err)) {
           ok = false;
           break;
         }
         tc_fence_after();
         issue_s(c);
       }
+      volatile int* abort_v = &abort_flag;
       for (int c = 0; ok && c < n_ch; ++c) {
-        if (!mbar_wait(p_full, c & 1, &abort_flag, a.dev_err)) break;
-        tc_fence_after();
-        issue_pv(c);
-        if (c + 2 < n_ch) {
-          if (!mbar_wait(&kv_full[(c + 2) % C::kStages], ((c + 2) / C::kStages) & 1, &abort_flag,
-                         a.dev_err))
+        if (!mbar_wait(&p_full[c & 1], (c >> 1) & 1, &abort_flag, a.dev_err)) break;
+        // PV(c) needs V(c); S(c+2) reuses the S buffer the softmax has just
+        // released and needs K(c+2): issue whichever is ready first.
+        bool pv_left = true, s_left = c + 2 < n_ch;
+        const uint32_t vpar = (c / C::kStages) & 1, kpar = ((c + 2) / C::kStages) & 1;
+        const long long t0c = clock64();
+        while (pv_left || s_left) {
+          if (pv_left && mbar_test(&v_full[c % C::kStages], vpar)) {
+            tc_fence_after();
+            issue_pv(c);
+            pv_left = false;
+          }
+          if (s_left && mbar_test(&k_full[(c + 2) % C::kStages], kpar)) {
+            tc_fence_after();
+            issue_s(c + 2);
+            s_left = false;
+          }
+          if ((pv_left || s_left) && (*abort_v || clock64() - t0c > kWaitLimitCycles)) {
+            if (!*abort_v) {
+              *abort_v = 1;
+              raise_dev_err(a.dev_err, CCGQA_DEVERR_TIMEOUT);
+            }
+            ok = false;
             break;
-          tc_fence_after();
-          issue_s(c + 2);
+          }
         }
       }
     }
@@ -228,13 +279,23 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
     // P / P^T tile: all zero (rows >= G stay zero for the whole CTA).
     for (int i = t128; i < static_cast<int>(C::kPBytes / 16); i += 128)
       reinterpret_cast<uint4*>(ptile)[i] = make_uint4(0, 0, 0, 0);
-    const float* qsrc = a.q_ws + (static_cast<int64_t>(b) * a.Hq + g * G) * D;
-    for (int i = t128; i < kQRows * D; i += 128) {
-      const int h = i / D, e = i - h * D;
-      const float v = h < G ? qsrc[h * D + e] : 0.f;
-      const int p = e / C::kPanelCols, ec = e % C::kPanelCols;
-      *reinterpret_cast<bf16*>(smem + C::kOffQ + p * C::kQPanelBytes +
-                               swz_offset(h, ec * 2, C::kRowBytes)) = __float2bfloat16_rn(v);
+    {
+      // all loads first, then the stores (one memory latency, not one per element)
+      const float* qsrc = a.q_ws + (static_cast<int64_t>(b) * a.Hq + g * G) * D;
+      constexpr int kPer = kQRows * D / 128;
+      float qv[kPer];
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int i = t128 + u * 128, h = i / D;
+        qv[u] = h < G ? __ldcg(qsrc + i) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int i = t128 + u * 128, h = i / D, e = i - h * D;
+        const int p = e / C::kPanelCols, ec = e % C::kPanelCols;
+        *reinterpret_cast<bf16*>(smem + C::kOffQ + p * C::kQPanelBytes +
+                                 swz_offset(h, ec * 2, C::kRowBytes)) = __float2bfloat16_rn(qv[u]);
+      }
     }
     fence_proxy_async_smem();
     mbar_arrive(q_ready);
@@ -254,29 +315,41 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
       float sv[kQRows];
 #pragma unroll
       for (int h = 0; h < kQRows; ++h) sv[h] = (kv && h < G) ? __uint_as_float(sr[h]) * scale : -INFINITY;
-      // chunk max per head over the 128 keys
-      float* rb = red + (c & 1) * 4 * kQRows;   // double-buffered across chunks
+      // The running max per head only moves when some key of the chunk lies
+      // more than kRescale above it; one barrier-OR over the 128 softmax
+      // threads answers that, and only then is the chunk max formed (warp
+      // shuffles, then the four warps' maxima through shared memory).
+      bool over = false;
 #pragma unroll
       for (int h = 0; h < kQRows; ++h) {
         if (h >= G) break;
-        float m = sv[h];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-        if (lane == 0) rb[sw * kQRows + h] = m;
+        over |= sv[h] > m_run[h] + kRescale;   // also when m_run is still -inf
       }
-      named_barrier_sync(1, 128);
       bool need_any = false;
       float factor[kQRows];
 #pragma unroll
-      for (int h = 0; h < kQRows; ++h) {
-        factor[h] = 1.f;
-        if (h >= G) break;
-        const float cm = fmaxf(fmaxf(rb[h], rb[kQRows + h]), fmaxf(rb[2 * kQRows + h], rb[3 * kQRows + h]));
-        if (cm > m_run[h] + kRescale) {        // also when m_run is still -inf
-          factor[h] = (m_run[h] == -INFINITY) ? 0.f : ex2(m_run[h] - cm);
-          m_run[h] = cm;
-          need_any = true;
-          l_part[h] *= factor[h];
+      for (int h = 0; h < kQRows; ++h) factor[h] = 1.f;
+      if (named_barrier_or(1, 128, over)) {
+        float* rb = red + (c & 1) * 4 * kQRows;   // double-buffered across chunks
+#pragma unroll
+        for (int h = 0; h < kQRows; ++h) {
+          if (h >= G) break;
+          float m = sv[h];
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+          if (lane == 0) rb[sw * kQRows + h] = m;
+        }
+        named_barrier_sync(1, 128);
+#pragma unroll
+        for (int h = 0; h < kQRows; ++h) {
+          if (h >= G) break;
+          const float cm = fmaxf(fmaxf(rb[h], rb[kQRows + h]), fmaxf(rb[2 * kQRows + h], rb[3 * kQRows + h]));
+          if (cm > m_run[h] + kRescale) {
+            factor[h] = (m_run[h] == -INFINITY) ? 0.f : ex2(m_run[h] - cm);
+            m_run[h] = cm;
+            need_any = true;
+            l_part[h] *= factor[h];
+          }
         }
       }
       float p[kQRows];
@@ -335,8 +408,9 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
         *reinterpret_cast<bf16*>(ptile + (c & 1) * C::kPBufBytes + (key >> 6) * C::kPPanelBytes +
                                  swz_offset(h, (key & 63) * 2, 128)) = __float2bfloat16_rn(p[h]);
       }
-      if (!kv) {
-        // zero the V row of a key past the sequence (its P is zero, but 0 * NaN is not)
+      if (!kv && mbar_wait(&v_full[c % C::kStages], (c / C::kStages) & 1, &abort_flag, a.dev_err)) {
+        // zero the V row of a key past the sequence (its P is zero, but 0 * NaN
+        // is not) once the V chunk has landed
         uint8_t* vt = smem + C::kOffV + (c % C::kStages) * C::kTileBytes;
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn)
@@ -347,7 +421,7 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[c & 1]);
     }
     // ---- split partials: max and sum per head, unnormalised O rows
     // the last PV completes after every earlier one
