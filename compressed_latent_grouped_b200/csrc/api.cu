@@ -4,7 +4,9 @@
 #include <atomic>
 #include <cmath>
 #include <cstdio>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "kernels.h"
 
@@ -12,6 +14,20 @@ namespace ccgqa {
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+
+cudaError_t allow_smem(const void* func, int bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<int, const void*>, int> allowed;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  int& have = allowed[{dev, func}];
+  if (have >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) have = bytes;
+  return e;
+}
 
 // Last CUDA error met by an entry point on this thread.
 static thread_local char t_last_error[256] = "no error";
@@ -247,6 +263,8 @@ ccgqa_status run_decode(const Geo& g, const ccgqa_weights* w, const void* x_t,
   a.causal = g.causal;
   a.rope_on = g.rope_on;
   a.rope_log2_base = g.rope_log2_base;
+  if (g.rope_on)
+    for (int i = 0; i < g.d / 2; ++i) a.rope_frac[i] = rope_turn_fraction(g.rope_log2_base, i, g.d);
   a.wq_seq = static_cast<const T*>(w->conv_q_seq);
   a.wq_chan = static_cast<const T*>(w->conv_q_chan);
   a.wk_seq = static_cast<const T*>(w->conv_k_seq);

@@ -496,8 +496,7 @@ cudaError_t launch_d(const AttnArgs& a, cudaStream_t stream) {
   const int rows_per_cta = C::kTiles * kBlockM;
   const int n_groups = (a.S * a.G + rows_per_cta - 1) / rows_per_cta;
   const int grid = n_groups * a.B * a.Hkv;
-  cudaError_t e = cudaFuncSetAttribute(attn_prefill_tc_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = allow_smem(reinterpret_cast<const void*>(attn_prefill_tc_kernel<D>),
                                        static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
   attn_prefill_tc_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(

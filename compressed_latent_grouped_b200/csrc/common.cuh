@@ -30,4 +30,9 @@ constexpr long long kWaitLimitCycles = 2000000000LL;
 // Host-side launch accounting (ccgqa_launch_count).
 void count_launches(int n);
 
+// cudaFuncSetAttribute(func, MaxDynamicSharedMemorySize, bytes) on the current
+// device, skipped when an earlier call already allowed at least `bytes`
+// (the attribute is per device, the check costs a lock and a map lookup).
+cudaError_t allow_smem(const void* func, int bytes);
+
 }  // namespace ccgqa

@@ -23,16 +23,22 @@
 namespace ccgqa {
 
 // ----------------------------------------------------------------- split plan
+// E range of one projection split: E / e_splits rounded up to whole 64-wide steps.
+static int decode_proj_e_len(int E, int e_splits) {
+  const int per = (E + e_splits - 1) / e_splits;
+  return (per + 63) / 64 * 64;
+}
+
 void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int* e_splits,
                  int* splits, int* chunk) {
   const int target = 2 * 148;
   if (has_proj) {
-    const int tiles = ((N + 127) / 128) * ((B + 63) / 64);
+    // projection CTAs: 64 columns x 64 sequences x one E-split of whole 64-wide steps
+    const int tiles = ((N + 63) / 64) * ((B + 63) / 64);
     int es = target / (tiles > 0 ? tiles : 1);
-    const int max_es = (E + 63) / 64;
-    if (es > max_es) es = max_es;
     if (es < 1) es = 1;
-    *e_splits = es;
+    const int e_len = decode_proj_e_len(E, es);
+    *e_splits = (E + e_len - 1) / e_len;
   } else {
     *e_splits = 0;
   }
@@ -100,41 +106,82 @@ __global__ void len_add_kernel(int32_t* len, int B, int64_t cap, int n_new) {
 }
 
 // ----------------------------------------------------------------- projection
-constexpr int kPB = 64, kPN = 128, kPE = 32;
+// part[s][b][n] = sum over k in split s of x[b][k] W[n][k]: one CTA per (64
+// columns, E-split, 64 sequences); both operands staged through shared memory
+// with 16-byte loads, a 4 x 4 register tile per thread, float4 partial stores.
+constexpr int kPB = 64, kPN = 64, kPK = 64;
+
+template <typename T>
+__device__ __forceinline__ void load16(const T* p, float (&v)[16 / sizeof(T)]) {
+  if constexpr (sizeof(T) == 2) {
+    const uint4 r = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
+  } else {
+    const float4 r = *reinterpret_cast<const float4*>(p);
+    v[0] = r.x;
+    v[1] = r.y;
+    v[2] = r.z;
+    v[3] = r.w;
+  }
+}
 
 template <typename T>
 __global__ void __launch_bounds__(256)
     decode_proj_kernel(const T* __restrict__ x, const T* __restrict__ W, float* __restrict__ part,
                        int B, int E, int N, int e_len) {
-  __shared__ __align__(16) float xs[kPE][kPB + 4];
-  __shared__ __align__(16) float wsm[kPE][kPN + 4];
+  constexpr int VEC = 16 / sizeof(T);
+  constexpr int CPR = kPK / VEC;          // 16-byte chunks per staged row
+  __shared__ __align__(16) float xs[kPK][kPB + 4];   // [k][sequence]
+  __shared__ __align__(16) float wsm[kPK][kPN + 4];  // [k][column]
   const int n0 = blockIdx.x * kPN, sp = blockIdx.y, b0 = blockIdx.z * kPB;
   const int e_lo = sp * e_len, e_hi = min(E, e_lo + e_len);
   const int tb = threadIdx.x / 16, tn = threadIdx.x % 16;
-  float acc[4][8] = {};
-  for (int e0 = e_lo; e0 < e_hi; e0 += kPE) {
-    for (int idx = threadIdx.x; idx < kPB * kPE; idx += 256) {
-      const int r = idx / kPE, c = idx % kPE;
-      const int gb = b0 + r, ge = e0 + c;
-      xs[c][r] = (gb < B && ge < e_hi) ? to_f32(x[static_cast<int64_t>(gb) * E + ge]) : 0.f;
+  float acc[4][4] = {};
+  for (int e0 = e_lo; e0 < e_hi; e0 += kPK) {
+    // lanes run over rows, so the transposed shared-memory stores do not conflict
+    for (int idx = threadIdx.x; idx < kPB * CPR; idx += 256) {
+      const int r = idx % kPB, c = idx / kPB;
+      const int gb = b0 + r, ge = e0 + c * VEC;
+      float v[VEC];
+      if (gb < B && ge < e_hi) {
+        load16(x + static_cast<int64_t>(gb) * E + ge, v);
+      } else {
+#pragma unroll
+        for (int u = 0; u < VEC; ++u) v[u] = 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < VEC; ++u) xs[c * VEC + u][r] = v[u];
     }
-    for (int idx = threadIdx.x; idx < kPN * kPE; idx += 256) {
-      const int r = idx / kPE, c = idx % kPE;
-      const int gn = n0 + r, ge = e0 + c;
-      wsm[c][r] = (gn < N && ge < e_hi) ? to_f32(W[static_cast<int64_t>(gn) * E + ge]) : 0.f;
+    for (int idx = threadIdx.x; idx < kPN * CPR; idx += 256) {
+      const int r = idx % kPN, c = idx / kPN;
+      const int gn = n0 + r, ge = e0 + c * VEC;
+      float v[VEC];
+      if (gn < N && ge < e_hi) {
+        load16(W + static_cast<int64_t>(gn) * E + ge, v);
+      } else {
+#pragma unroll
+        for (int u = 0; u < VEC; ++u) v[u] = 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < VEC; ++u) wsm[c * VEC + u][r] = v[u];
     }
     __syncthreads();
-#pragma unroll 8
-    for (int e = 0; e < kPE; ++e) {
-      const float4 xv = *reinterpret_cast<const float4*>(&xs[e][tb * 4]);
-      const float4 w0 = *reinterpret_cast<const float4*>(&wsm[e][tn * 8]);
-      const float4 w1 = *reinterpret_cast<const float4*>(&wsm[e][tn * 8 + 4]);
+#pragma unroll 16
+    for (int k = 0; k < kPK; ++k) {
+      const float4 xv = *reinterpret_cast<const float4*>(&xs[k][tb * 4]);
+      const float4 wv = *reinterpret_cast<const float4*>(&wsm[k][tn * 4]);
       const float xr[4] = {xv.x, xv.y, xv.z, xv.w};
-      const float wr[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      const float wr[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(xr[i], wr[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xr[i], wr[j], acc[i][j]);
     }
     __syncthreads();
   }
@@ -142,17 +189,40 @@ __global__ void __launch_bounds__(256)
   for (int i = 0; i < 4; ++i) {
     const int gb = b0 + tb * 4 + i;
     if (gb >= B) continue;
+    const int gn = n0 + tn * 4;
+    float* dst = part + (static_cast<int64_t>(sp) * B + gb) * N + gn;
+    if (gn + 3 < N && (N & 3) == 0) {
+      *reinterpret_cast<float4*>(dst) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    } else {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int gn = n0 + tn * 8 + j;
-      if (gn < N) part[(static_cast<int64_t>(sp) * B + gb) * N + gn] = acc[i][j];
+      for (int j = 0; j < 4; ++j)
+        if (gn + j < N) dst[j] = acc[i][j];
     }
   }
 }
 
 // ----------------------------------------------------------------- pre-step
+// Shared-memory bytes of the pre-step: fp32 rows (current, history, conv out,
+// mix out) plus, when it fits, the group's G + 1 channel-mix weights staged
+// transposed in the working dtype.
 template <typename T>
-__global__ void __launch_bounds__(128) decode_pre_kernel(const DecodeArgs<T> a) {
+__host__ __device__ inline size_t decode_pre_floats(int G, int d, int K) {
+  const int KH = K > 0 ? K - 1 : 0, HC = (G + 1) * d, AC = HC + d;
+  return (static_cast<size_t>(AC + KH * HC + 2 * HC) + 3) & ~size_t(3);
+}
+template <typename T>
+__host__ __device__ inline size_t decode_pre_wt_bytes(int G, int d) {
+  return static_cast<size_t>(G + 1) * d * d * sizeof(T);
+}
+constexpr size_t kPreWtMax = 160 * 1024;
+// One CTA per (sequence, kv group); its work is a handful of dependent phases,
+// each limited by one round of global loads, so every loop below is unrolled
+// to keep several independent loads in flight per thread.
+constexpr int kPreThreads = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_constant__ DecodeArgs<T> a,
+                                                         int stage_wt) {
   extern __shared__ float4 dsm_f4[];
   float* sm = reinterpret_cast<float*>(dsm_f4);
   const int g = blockIdx.x, b = blockIdx.y;
@@ -170,6 +240,26 @@ __global__ void __launch_bounds__(128) decode_pre_kernel(const DecodeArgs<T> a) 
     return;
   }
   const int qcol0 = g * G * d, kcol0 = a.Hq * d + g * d, vcol0 = (a.Hq + a.Hkv) * d + g * d;
+  // channel-mix weights of the group, transposed: wt[hh][j][i] = W_hh[i][j]
+  T* wt = reinterpret_cast<T*>(sm + decode_pre_floats<T>(G, d, K));
+  const bool have_mix = K > 0 && a.wq_chan != nullptr && a.wk_chan != nullptr;
+  if (stage_wt && have_mix) {
+    constexpr int VEC = 16 / sizeof(T);
+    const int per_head = d * d / VEC;
+#pragma unroll 4
+    for (int idx = tid; idx < (G + 1) * per_head; idx += blockDim.x) {
+      // lanes run over rows i, so the transposed stores hit consecutive addresses
+      const int hh = idx / per_head, rem = idx - hh * per_head;
+      const int i = rem % d, j0 = (rem / d) * VEC;
+      const T* src = hh < G ? a.wq_chan + (static_cast<int64_t>(g * G + hh) * d + i) * d + j0
+                            : a.wk_chan + (static_cast<int64_t>(g) * d + i) * d + j0;
+      T v[VEC];
+      *reinterpret_cast<uint4*>(v) = *reinterpret_cast<const uint4*>(src);
+#pragma unroll
+      for (int u = 0; u < VEC; ++u) wt[(static_cast<int64_t>(hh) * d + j0 + u) * d + i] = v[u];
+    }
+  }
+#pragma unroll 2
   for (int c = tid; c < AC; c += blockDim.x) {
     const int col = c < QC ? qcol0 + c : (c < HC ? kcol0 + (c - QC) : vcol0 + (c - HC));
     float val;
@@ -177,14 +267,23 @@ __global__ void __launch_bounds__(128) decode_pre_kernel(const DecodeArgs<T> a) 
       val = 0.f;
       const float* pp = a.proj_part + static_cast<int64_t>(b) * a.N + col;
       const int64_t pstride = static_cast<int64_t>(a.B) * a.N;
-#pragma unroll 8
-      for (int s = 0; s < a.e_splits; ++s) val += __ldcg(pp + s * pstride);
+      // all partials loaded first, then summed in split order (deterministic)
+      float pv[8];
+      int s = 0;
+      for (; s + 8 <= a.e_splits; s += 8) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) pv[u] = __ldcg(pp + (s + u) * pstride);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) val += pv[u];
+      }
+      for (; s < a.e_splits; ++s) val += __ldcg(pp + s * pstride);
       val = to_f32(from_f32<T>(val));  // the projection output is held in the working dtype
     } else {
       val = to_f32(a.x_t[static_cast<int64_t>(b) * a.N + col]);
     }
     zc[c] = val;
   }
+#pragma unroll 4
   for (int idx = tid; idx < KH * HC; idx += blockDim.x) {
     const int r = idx / HC, c = idx - r * HC;
     hz[idx] = c < QC ? to_f32(a.hist_q[(static_cast<int64_t>(b) * KH + r) * a.Hq * d + qcol0 + c])
@@ -213,7 +312,12 @@ __global__ void __launch_bounds__(128) decode_pre_kernel(const DecodeArgs<T> a) 
     const int hh = c / d, i = c - hh * d;
     const T* wch = is_q ? a.wq_chan : a.wk_chan;
     float acc;
-    if (K > 0 && wch) {
+    if (K > 0 && wch && stage_wt && have_mix) {
+      const T* wc = wt + static_cast<int64_t>(hh) * d * d + i;   // column i of W_hh^T
+      acc = 0.f;
+#pragma unroll 8
+      for (int j = 0; j < d; ++j) acc = fmaf(to_f32(wc[j * d]), u[hh * d + j], acc);
+    } else if (K > 0 && wch) {
       const int head = is_q ? g * G + hh : g;
       const T* wr = wch + (static_cast<int64_t>(head) * d + i) * d;
       acc = 0.f;
@@ -241,11 +345,11 @@ __global__ void __launch_bounds__(128) decode_pre_kernel(const DecodeArgs<T> a) 
     const int hh = idx / half, i = idx - hh * half;
     float ya = y[hh * d + i], yb = y[hh * d + i + half];
     if (a.rope_on) {
-      const double th = exp2(-(2.0 * i / d) * a.rope_log2_base);
-      double f = static_cast<double>(L) * th * 0.15915494309189533577;
-      f -= rint(f);
+      // angle L * theta_i reduced modulo one turn exactly in 64-bit fixed point
+      const uint64_t ph = static_cast<uint64_t>(L) * a.rope_frac[i];
+      const float f = static_cast<float>(static_cast<int64_t>(ph)) * 5.42101086242752217e-20f;
       float s, c;
-      sincospif(static_cast<float>(2.0 * f), &s, &c);
+      sincospif(2.0f * f, &s, &c);
       const float na = ya * c - yb * s, nb = ya * s + yb * c;
       ya = na;
       yb = nb;
@@ -512,8 +616,7 @@ cudaError_t launch_dec_attn(const DecodeArgs<T>& a, cudaStream_t stream) {
   using C = DecCfg<T, D>;
   if (a.G * C::NCH > 32 * kPPMax) return cudaErrorInvalidValue;
   const size_t smem = dec_attn_smem<T, D>(a.G);
-  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<T, D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = allow_smem(reinterpret_cast<const void*>(decode_attn_kernel<T, D>),
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(a.splits, a.Hkv, a.B);
@@ -548,7 +651,7 @@ cudaError_t launch_decode_step(const DecodeArgs<T>& a, cudaStream_t stream) {
   };
   mark(0);
   if (a.W) {
-    const int e_len = ((a.E + a.e_splits - 1) / a.e_splits + kPE - 1) / kPE * kPE;
+    const int e_len = decode_proj_e_len(a.E, a.e_splits);
     dim3 grid((a.N + kPN - 1) / kPN, a.e_splits, (a.B + kPB - 1) / kPB);
     decode_proj_kernel<T><<<grid, 256, 0, stream>>>(a.x_t, a.W, a.proj_part, a.B, a.E, a.N, e_len);
     count_launches(1);
@@ -556,15 +659,15 @@ cudaError_t launch_decode_step(const DecodeArgs<T>& a, cudaStream_t stream) {
   }
   mark(1);
   {
-    const int KH = a.K > 0 ? a.K - 1 : 0;
-    const int HC = (a.G + 1) * a.d, AC = HC + a.d;
-    const size_t smem = static_cast<size_t>(AC + KH * HC + 2 * HC) * 4 + 16;
+    const size_t wt = decode_pre_wt_bytes<T>(a.G, a.d);
+    const int stage_wt = wt <= kPreWtMax;
+    const size_t smem = decode_pre_floats<T>(a.G, a.d, a.K) * 4 + (stage_wt ? wt : 0) + 16;
     if (smem > 48 * 1024) {
-      e = cudaFuncSetAttribute(decode_pre_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      e = allow_smem(reinterpret_cast<const void*>(decode_pre_kernel<T>),
                                static_cast<int>(smem));
       if (e != cudaSuccess) return e;
     }
-    decode_pre_kernel<T><<<dim3(a.Hkv, a.B), 128, smem, stream>>>(a);
+    decode_pre_kernel<T><<<dim3(a.Hkv, a.B), kPreThreads, smem, stream>>>(a, stage_wt);
     count_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

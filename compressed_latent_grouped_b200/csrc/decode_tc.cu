@@ -547,8 +547,7 @@ cudaError_t launch_tc(const DecodeArgs<bf16>& a, cudaStream_t stream) {
   if (!encode_tensor_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.cache_k, dims, st, box, swz) ||
       !encode_tensor_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.cache_v, dims, st, box, swz))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(decode_attn_tc_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = allow_smem(reinterpret_cast<const void*>(decode_attn_tc_kernel<D>),
                                        static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
   dim3 grid(a.splits, a.Hkv, a.B);

@@ -88,6 +88,7 @@ struct DecodeArgs {
   int B, E, N, Hq, Hkv, d, G, K;
   int qk_mean, value_shift, causal, rope_on;
   double rope_log2_base;
+  uint64_t rope_frac[64];  // theta_i / (2 pi) in 0.64 fixed point, i < d/2 (see PreAttnArgs)
   const T *wq_seq, *wq_chan, *wk_seq, *wk_chan;
   T* cache_k;            // [B, Hkv, cap, d]
   T* cache_v;

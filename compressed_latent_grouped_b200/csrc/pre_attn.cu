@@ -333,7 +333,7 @@ cudaError_t launch_pre_attn(const PreAttnArgs<T>& a, cudaStream_t stream) {
               : a.d == 64 ? pre_attn_kernel<T, 64>
                           : pre_attn_kernel<T, 128>;
   if (a.d != 16 && a.d != 32 && a.d != 64 && a.d != 128) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = allow_smem(reinterpret_cast<const void*>(kernel),
                                        static_cast<int>(L.bytes));
   if (e != cudaSuccess) return e;
   dim3 grid((a.S + TT - 1) / TT, a.Hkv, a.B);

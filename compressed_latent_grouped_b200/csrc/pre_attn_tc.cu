@@ -416,8 +416,7 @@ __global__ void __launch_bounds__(kPtThreads)
 template <int D>
 cudaError_t launch_d(const PreAttnArgs<bf16>& a, cudaStream_t stream) {
   const PtLayout L = pt_layout(D, a.G);
-  cudaError_t e = cudaFuncSetAttribute(pre_attn_tc_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = allow_smem(reinterpret_cast<const void*>(pre_attn_tc_kernel<D>),
                                        static_cast<int>(L.bytes));
   if (e != cudaSuccess) return e;
   dim3 grid((a.S + kPtTT - 1) / kPtTT, a.Hkv, a.B);

@@ -215,8 +215,7 @@ cudaError_t launch_proj_gemm_bf16(const bf16* A, const bf16* W, bf16* C, int M, 
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(proj_gemm_bf16_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = allow_smem(reinterpret_cast<const void*>(proj_gemm_bf16_kernel),
                                          static_cast<int>(kGemmSmem));
     if (e != cudaSuccess) return e;
     attr_set = true;
