@@ -499,29 +499,39 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
   __syncthreads();
   if (!last_flag) return;
   __threadfence();
+  // Two passes, each with its loads in flight together: per head, the max over
+  // the splits, then each split's weight 2^(m_s - M) and the total sum (one
+  // thread per head, weights kept in the now idle K ring); then every output
+  // element sums its splits' unnormalised rows with those weights.
   const int64_t gbase = static_cast<int64_t>(bg) * a.splits * G;
-  for (int idx = tid; idx < G * D; idx += kDecTcThreads) {
-    const int h = idx / D, i = idx - h * D;
-    float M = -INFINITY, lsum = 0.f, acc = 0.f;
-#pragma unroll 4
+  float* wts = reinterpret_cast<float*>(smem + C::kOffK);   // [splits][G], then inv_l[G]
+  float* inv_l = wts + a.splits * G;
+  if (tid < G) {
+    const int h = tid;
+    float M = -INFINITY;
+#pragma unroll 16
+    for (int s2 = 0; s2 < a.splits; ++s2)
+      M = fmaxf(M, __ldcg(a.part_ml + (gbase + static_cast<int64_t>(s2) * G + h) * 2));
+    float lsum = 0.f;
+#pragma unroll 16
     for (int s2 = 0; s2 < a.splits; ++s2) {
       const int64_t pi = gbase + static_cast<int64_t>(s2) * G + h;
       const float ms = __ldcg(a.part_ml + pi * 2);
-      const float ls = __ldcg(a.part_ml + pi * 2 + 1);
-      const float os = __ldcg(a.part_o + pi * D + i);
-      if (ms == -INFINITY) continue;
-      if (ms > M) {
-        const float corr = ex2(M - ms);
-        lsum *= corr;
-        acc *= corr;
-        M = ms;
-      }
-      const float f = ex2(ms - M);
-      lsum = fmaf(ls, f, lsum);
-      acc = fmaf(os, f, acc);
+      const float wgt = (ms == -INFINITY) ? 0.f : ex2(ms - M);
+      lsum = fmaf(__ldcg(a.part_ml + pi * 2 + 1), wgt, lsum);
+      wts[s2 * G + h] = wgt;
     }
-    const float val = (valid_b && lsum > 0.f) ? acc / lsum : 0.f;
-    a.out[static_cast<int64_t>(b) * a.Hq * D + (g * G + h) * D + i] = __float2bfloat16_rn(val);
+    inv_l[h] = (valid_b && lsum > 0.f) ? 1.f / lsum : 0.f;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < G * D; idx += kDecTcThreads) {
+    const int h = idx / D, i = idx - h * D;
+    float acc = 0.f;
+#pragma unroll 16
+    for (int s2 = 0; s2 < a.splits; ++s2)
+      acc = fmaf(__ldcg(a.part_o + (gbase + static_cast<int64_t>(s2) * G + h) * D + i),
+                 wts[s2 * G + h], acc);
+    a.out[static_cast<int64_t>(b) * a.Hq * D + (g * G + h) * D + i] = __float2bfloat16_rn(acc * inv_l[h]);
   }
   __syncthreads();
   if (tid == 0) {
