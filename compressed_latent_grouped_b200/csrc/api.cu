@@ -146,7 +146,7 @@ struct DecodeWs {
 };
 DecodeWs decode_ws(const Geo& g, int64_t B, int64_t cap, bool has_proj) {
   DecodeWs w;
-  decode_plan(static_cast<int>(B), g.Hkv, g.E, g.N, cap, has_proj, &w.e_splits, &w.splits,
+  decode_plan(static_cast<int>(B), g.Hkv, g.E, g.N, cap, has_proj, g.es, &w.e_splits, &w.splits,
               &w.chunk);
   size_t off = 0;
   w.tick = off;  // tickets first: the part a fresh zero-fill must cover

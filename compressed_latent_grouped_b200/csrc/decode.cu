@@ -23,16 +23,25 @@
 namespace ccgqa {
 
 // ----------------------------------------------------------------- split plan
+// Few sequences: the projection streams W once, one warp per output column,
+// with x (B x E, working dtype) held in shared memory.
+constexpr int kGvMaxB = 16;
+constexpr size_t kGvMaxX = 64 * 1024;
+static bool decode_use_gemv(int B, int E, int es) {
+  return B <= kGvMaxB && static_cast<size_t>(B) * E * es <= kGvMaxX;
+}
 // E range of one projection split: E / e_splits rounded up to whole 64-wide steps.
 static int decode_proj_e_len(int E, int e_splits) {
   const int per = (E + e_splits - 1) / e_splits;
   return (per + 63) / 64 * 64;
 }
 
-void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int* e_splits,
-                 int* splits, int* chunk) {
+void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int es,
+                 int* e_splits, int* splits, int* chunk) {
   const int target = 2 * 148;
-  if (has_proj) {
+  if (has_proj && decode_use_gemv(B, E, es)) {
+    *e_splits = 1;   // one weight-streaming pass, no partials to sum
+  } else if (has_proj) {
     // projection CTAs: 64 columns x 64 sequences x one E-split of whole 64-wide steps
     const int tiles = ((N + 63) / 64) * ((B + 63) / 64);
     int es = target / (tiles > 0 ? tiles : 1);
@@ -197,6 +206,53 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
       for (int j = 0; j < 4; ++j)
         if (gn + j < N) dst[j] = acc[i][j];
+    }
+  }
+}
+
+// out[b][n] = sum_k x[b][k] W[n][k] for B <= 16: x staged once per CTA in shared
+// memory, each warp owns output columns and streams their W rows with 16-byte
+// loads (all of a row's loads in flight), then reduces across its lanes.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    decode_gemv_kernel(const T* __restrict__ x, const T* __restrict__ W, float* __restrict__ out,
+                       int B, int E, int N) {
+  constexpr int VEC = 16 / sizeof(T);
+  extern __shared__ float4 gv_f4[];
+  T* xs = reinterpret_cast<T*>(gv_f4);             // [B][E]
+#pragma unroll 4
+  for (int idx = threadIdx.x; idx < B * E / VEC; idx += blockDim.x)
+    reinterpret_cast<uint4*>(xs)[idx] = reinterpret_cast<const uint4*>(x)[idx];
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  for (int n = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); n < N; n += warps) {
+    float acc[kGvMaxB];
+#pragma unroll
+    for (int b = 0; b < kGvMaxB; ++b) acc[b] = 0.f;
+    const T* wr = W + static_cast<int64_t>(n) * E;
+#pragma unroll 4
+    for (int k0 = lane * VEC; k0 < E; k0 += 32 * VEC) {
+      float wv[VEC];
+      load16(wr + k0, wv);
+#pragma unroll
+      for (int b = 0; b < kGvMaxB; ++b) {
+        if (b < B) {
+          float xv[VEC];
+          load16(xs + static_cast<int64_t>(b) * E + k0, xv);
+#pragma unroll
+          for (int u = 0; u < VEC; ++u) acc[b] = fmaf(wv[u], xv[u], acc[b]);
+        }
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < kGvMaxB; ++b) {
+      if (b < B) {
+        float v = acc[b];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == 0) out[static_cast<int64_t>(b) * N + n] = v;
+      }
     }
   }
 }
@@ -651,9 +707,19 @@ cudaError_t launch_decode_step(const DecodeArgs<T>& a, cudaStream_t stream) {
   };
   mark(0);
   if (a.W) {
-    const int e_len = decode_proj_e_len(a.E, a.e_splits);
-    dim3 grid((a.N + kPN - 1) / kPN, a.e_splits, (a.B + kPB - 1) / kPB);
-    decode_proj_kernel<T><<<grid, 256, 0, stream>>>(a.x_t, a.W, a.proj_part, a.B, a.E, a.N, e_len);
+    if (decode_use_gemv(a.B, a.E, sizeof(T)) && a.e_splits == 1) {
+      const size_t xb = static_cast<size_t>(a.B) * a.E * sizeof(T);
+      if (xb > 48 * 1024 &&
+          (e = allow_smem(reinterpret_cast<const void*>(decode_gemv_kernel<T>), static_cast<int>(xb))) !=
+              cudaSuccess)
+        return e;
+      const int blocks = (a.N + 7) / 8;   // one warp per column
+      decode_gemv_kernel<T><<<blocks, 256, xb, stream>>>(a.x_t, a.W, a.proj_part, a.B, a.E, a.N);
+    } else {
+      const int e_len = decode_proj_e_len(a.E, a.e_splits);
+      dim3 grid((a.N + kPN - 1) / kPN, a.e_splits, (a.B + kPB - 1) / kPB);
+      decode_proj_kernel<T><<<grid, 256, 0, stream>>>(a.x_t, a.W, a.proj_part, a.B, a.E, a.N, e_len);
+    }
     count_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

@@ -506,20 +506,37 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
   const int64_t gbase = static_cast<int64_t>(bg) * a.splits * G;
   float* wts = reinterpret_cast<float*>(smem + C::kOffK);   // [splits][G], then inv_l[G]
   float* inv_l = wts + a.splits * G;
+  // (loops over splits run in blocks of 8 with the block's loads issued first,
+  // so a block costs one memory latency)
+  constexpr int kBlk = 8;
   if (tid < G) {
     const int h = tid;
     float M = -INFINITY;
-#pragma unroll 16
-    for (int s2 = 0; s2 < a.splits; ++s2)
-      M = fmaxf(M, __ldcg(a.part_ml + (gbase + static_cast<int64_t>(s2) * G + h) * 2));
+    for (int s0 = 0; s0 < a.splits; s0 += kBlk) {
+      float mv[kBlk];
+#pragma unroll
+      for (int u = 0; u < kBlk; ++u)
+        mv[u] = s0 + u < a.splits
+                    ? __ldcg(a.part_ml + (gbase + static_cast<int64_t>(s0 + u) * G + h) * 2)
+                    : -INFINITY;
+#pragma unroll
+      for (int u = 0; u < kBlk; ++u) M = fmaxf(M, mv[u]);
+    }
     float lsum = 0.f;
-#pragma unroll 16
-    for (int s2 = 0; s2 < a.splits; ++s2) {
-      const int64_t pi = gbase + static_cast<int64_t>(s2) * G + h;
-      const float ms = __ldcg(a.part_ml + pi * 2);
-      const float wgt = (ms == -INFINITY) ? 0.f : ex2(ms - M);
-      lsum = fmaf(__ldcg(a.part_ml + pi * 2 + 1), wgt, lsum);
-      wts[s2 * G + h] = wgt;
+    for (int s0 = 0; s0 < a.splits; s0 += kBlk) {
+      float mv[kBlk], lv[kBlk];
+#pragma unroll
+      for (int u = 0; u < kBlk; ++u) {
+        const int64_t pi = gbase + static_cast<int64_t>(s0 + u) * G + h;
+        mv[u] = s0 + u < a.splits ? __ldcg(a.part_ml + pi * 2) : -INFINITY;
+        lv[u] = s0 + u < a.splits ? __ldcg(a.part_ml + pi * 2 + 1) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kBlk; ++u) {
+        const float wgt = (mv[u] == -INFINITY) ? 0.f : ex2(mv[u] - M);
+        lsum = fmaf(lv[u], wgt, lsum);
+        if (s0 + u < a.splits) wts[(s0 + u) * G + h] = wgt;
+      }
     }
     inv_l[h] = (valid_b && lsum > 0.f) ? 1.f / lsum : 0.f;
   }
@@ -527,10 +544,17 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
   for (int idx = tid; idx < G * D; idx += kDecTcThreads) {
     const int h = idx / D, i = idx - h * D;
     float acc = 0.f;
-#pragma unroll 16
-    for (int s2 = 0; s2 < a.splits; ++s2)
-      acc = fmaf(__ldcg(a.part_o + (gbase + static_cast<int64_t>(s2) * G + h) * D + i),
-                 wts[s2 * G + h], acc);
+    for (int s0 = 0; s0 < a.splits; s0 += kBlk) {
+      float ov[kBlk];
+#pragma unroll
+      for (int u = 0; u < kBlk; ++u)
+        ov[u] = s0 + u < a.splits
+                    ? __ldcg(a.part_o + (gbase + static_cast<int64_t>(s0 + u) * G + h) * D + i)
+                    : 0.f;
+#pragma unroll
+      for (int u = 0; u < kBlk; ++u)
+        if (s0 + u < a.splits) acc = fmaf(ov[u], wts[(s0 + u) * G + h], acc);
+    }
     a.out[static_cast<int64_t>(b) * a.Hq * D + (g * G + h) * D + i] = __float2bfloat16_rn(acc * inv_l[h]);
   }
   __syncthreads();

@@ -116,7 +116,7 @@ cudaError_t launch_decode_step(const DecodeArgs<T>& a, cudaStream_t stream);
 cudaError_t launch_decode_attn_tc(const DecodeArgs<bf16>& a, cudaStream_t stream);
 
 // Split plan for the decode step, shared by the workspace-size query and the launch.
-void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int* e_splits,
-                 int* splits, int* chunk);
+void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int es,
+                 int* e_splits, int* splits, int* chunk);
 
 }  // namespace ccgqa
