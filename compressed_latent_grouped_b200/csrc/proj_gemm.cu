@@ -3,11 +3,12 @@
 // projected straight into the latent space of width E/C).
 //
 // bf16: C[M, N] = A[M, K] * W[N, K]^T on the 5th-generation tensor core.
-//   One CTA computes a 128 x 256 output tile.  Warp 0 streams 128x64 A and
-//   256x64 W tiles with TMA (128B swizzle) through a 4-stage shared-memory ring;
-//   warp 1 allocates 256 TMEM columns and one elected thread issues
-//   tcgen05.mma (M=128, N=256, K=16, fp32 accumulate in TMEM); warps 2-5 read
-//   the accumulator back with tcgen05.ld and store bf16 rows.
+//   One persistent CTA per SM walks 128 x 256 output tiles.  Warp 0 streams
+//   128x64 A and 256x64 W tiles with TMA (128B swizzle) through a 4-stage
+//   shared-memory ring; warp 1 allocates 2 x 256 TMEM columns and one thread
+//   issues tcgen05.mma (M=128, N=256, K=16, fp32 accumulate) into them in turn;
+//   warps 2-5 read a finished accumulator back with tcgen05.ld and store bf16
+//   rows while the next tile accumulates into the other.
 // fp32: a plain shared-memory tiled GEMM on the CUDA cores.
 #include "kernels.h"
 #include "sm100.cuh"
@@ -24,6 +25,11 @@ constexpr uint32_t kBTile = kBN * kBK * 2;      // 32 KB
 constexpr uint32_t kStageBytes = kATile + kBTile;
 constexpr size_t kGemmSmem = size_t(kStages) * kStageBytes + 1024 + 256;
 
+// Persistent: CTA c computes tiles c, c + gridDim.x, ... (tile t = row block
+// t / n_tiles, column block t % n_tiles, so CTAs running together share A rows
+// through L2).  The TMA ring and the k-block counter run on across tiles, and
+// the accumulator alternates between two 256-column TMEM buffers, so the
+// epilogue of one tile overlaps the main loop of the next.
 __global__ void __launch_bounds__(kGemmThreads, 1)
     proj_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
                           const __grid_constant__ CUtensorMap tmB, bf16* __restrict__ C, int M,
@@ -33,27 +39,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
   uint64_t* empty = full + kStages;
-  uint64_t* acc_full = empty + kStages;
-  uint64_t* drain = acc_full + 1;
+  uint64_t* acc_full = empty + kStages;   // [2] accumulator b complete
+  uint64_t* acc_empty = acc_full + 2;     // [2] accumulator b read back (128 arrivals)
+  uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * kBM, n0 = blockIdx.x * kBN;
   const int nkb = (K + kBK - 1) / kBK;
+  const int n_tiles = (N + kBN - 1) / kBN;
+  const int tiles = n_tiles * ((M + kBM - 1) / kBM);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
     mbar_init(drain, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kBN);
+    tmem_alloc(tmem_slot, 2 * kBN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -65,52 +76,73 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       prefetch_tensormap(&tmA);
       prefetch_tensormap(&tmB);
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % kStages;
-        const uint32_t ph = (kb / kStages) & 1;
-        if (!mbar_wait(&empty[s], ph ^ 1, &abort_flag, dev_err)) break;
-        mbar_arrive_expect_tx(&full[s], kStageBytes);
-        uint8_t* sa = smem + s * kStageBytes;
-        tma_load_2d(sa, &tmA, &full[s], kb * kBK, m0);
-        tma_load_2d(sa + kATile, &tmB, &full[s], kb * kBK, n0);
+      int g = 0;   // k-blocks issued by this CTA so far
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+        const int m0 = (t / n_tiles) * kBM, n0 = (t % n_tiles) * kBN;
+        for (int kb = 0; kb < nkb; ++kb, ++g) {
+          const int s = g % kStages;
+          if (!mbar_wait(&empty[s], ((g / kStages) & 1) ^ 1, &abort_flag, dev_err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], kStageBytes);
+          uint8_t* sa = smem + s * kStageBytes;
+          tma_load_2d(sa, &tmA, &full[s], kb * kBK, m0);
+          tma_load_2d(sa + kATile, &tmB, &full[s], kb * kBK, n0);
+        }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = make_idesc_bf16(kBM, kBN, false);
-      int kb = 0;
-      for (; kb < nkb; ++kb) {
-        const int s = kb % kStages;
-        const uint32_t ph = (kb / kStages) & 1;
-        if (!mbar_wait(&full[s], ph, &abort_flag, dev_err)) break;
+      int g = 0, i = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++i) {
+        const int bsel = i & 1;
+        // the epilogue has read this accumulator's previous tile back
+        if (!mbar_wait(&acc_empty[bsel], ((i >> 1) & 1) ^ 1, &abort_flag, dev_err)) break;
         tc_fence_after();
-        const uint32_t a_base = smem_addr(smem + s * kStageBytes);
-        const uint32_t b_base = a_base + kATile;
+        const uint32_t acc = tmem + bsel * kBN;
+        for (int kb = 0; kb < nkb; ++kb, ++g) {
+          const int s = g % kStages;
+          if (!mbar_wait(&full[s], (g / kStages) & 1, &abort_flag, dev_err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_addr(smem + s * kStageBytes);
+          const uint32_t b_base = a_base + kATile;
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k) {
-          // K-major, 128B-swizzled tiles: 8-row groups 1024 B apart; a K step of
-          // 16 bf16 advances the start address by 32 B inside the swizzle row.
-          const uint64_t ad = make_smem_desc(a_base + k * 32, 16, 1024, kSwizzle128B);
-          const uint64_t bd = make_smem_desc(b_base + k * 32, 16, 1024, kSwizzle128B);
-          mma_ss(tmem, ad, bd, idesc, (kb | k) != 0);
+          for (int k = 0; k < kBK / 16; ++k) {
+            // K-major, 128B-swizzled tiles: 8-row groups 1024 B apart; a K step of
+            // 16 bf16 advances the start address by 32 B inside the swizzle row.
+            const uint64_t ad = make_smem_desc(a_base + k * 32, 16, 1024, kSwizzle128B);
+            const uint64_t bd = make_smem_desc(b_base + k * 32, 16, 1024, kSwizzle128B);
+            mma_ss(acc, ad, bd, idesc, (kb | k) != 0);
+          }
+          mma_commit(&empty[s]);
         }
-        mma_commit(&empty[s]);
+        if (ok) mma_commit(&acc_full[bsel]);
       }
-      mma_commit(acc_full);
     }
   } else {
     // Epilogue: warp w may only touch TMEM lanes [32 (w % 4), 32 (w % 4) + 32).
     const int q4 = warp & 3;
-    if (mbar_wait(acc_full, 0, &abort_flag, dev_err)) {
+    const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    int i = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+      const int bsel = i & 1;
+      if (!mbar_wait(&acc_full[bsel], (i >> 1) & 1, &abort_flag, dev_err)) break;
       tc_fence_after();
+      const int m0 = (t / n_tiles) * kBM, n0 = (t % n_tiles) * kBN;
       const int row = m0 + q4 * 32 + lane;
-      const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
 #pragma unroll 1
       for (int c = 0; c < kBN / 32; ++c) {
         const int col0 = n0 + c * 32;
         if (col0 >= N) break;  // warp-uniform
         uint32_t r[32];
-        tmem_ld32(trow + c * 32, r);
+        tmem_ld32(trow + bsel * kBN + c * 32, r);
         tmem_wait_ld();
         if (row < M) {
           bf16* dst = C + static_cast<int64_t>(row) * N + col0;
@@ -133,6 +165,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[bsel]);
     }
   }
 
@@ -147,7 +181,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kBN);
+    tmem_dealloc(tmem, 2 * kBN);
   }
 }
 
@@ -213,14 +247,14 @@ cudaError_t launch_proj_gemm_bf16(const bf16* A, const bf16* W, bf16* C, int M, 
       !encode_tensor_map(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, dB, sA, bB,
                          CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = allow_smem(reinterpret_cast<const void*>(proj_gemm_bf16_kernel),
-                                         static_cast<int>(kGemmSmem));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  dim3 grid((N + kBN - 1) / kBN, (M + kBM - 1) / kBM);
+  cudaError_t e = allow_smem(reinterpret_cast<const void*>(proj_gemm_bf16_kernel),
+                             static_cast<int>(kGemmSmem));
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int tiles = ((N + kBN - 1) / kBN) * ((M + kBM - 1) / kBM);
+  const int grid = tiles < sms ? tiles : sms;   // one persistent CTA per SM
   proj_gemm_bf16_kernel<<<grid, kGemmThreads, kGemmSmem, stream>>>(tmA, tmB, C, M, N, K,
                                                                     dev_err);
   count_launches(1);
