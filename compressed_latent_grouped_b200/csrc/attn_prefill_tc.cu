@@ -58,6 +58,7 @@ struct Cfg {
   // Query tiles per CTA: three where their S buffers and accumulators fit
   // in TMEM (3 x 128 + 3 x 32 columns at d = 32), else two.
   static constexpr int kTiles = (D == 32) ? 3 : 2;
+  static constexpr int kSoftEvery = (D == 64) ? 3 : 4;
   static constexpr int kThreads = 128 + 128 * kTiles;   // 4 control warps + softmax
   static constexpr uint32_t kOffQ = 0;                        // Q_A, Q_B
   static constexpr uint32_t kOffK = kTiles * kTileBytes;
@@ -126,14 +127,10 @@ __device__ __forceinline__ float2 soft_exp2x2(float2 x) {
                      __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
-// Pairs (c2 % kSoftExpEvery == 0) of each softmax row use the software exp2,
-// so the FMA pipe takes a quarter of the exponentials off the exp unit
-// (measured on B200: 1 in 4 is the best split at d = 64 and d = 128, neutral
-// at d = 32).
-#ifndef CCGQA_SOFT_EXP_EVERY
-#define CCGQA_SOFT_EXP_EVERY 4
-#endif
-constexpr int kSoftExpEvery = CCGQA_SOFT_EXP_EVERY;
+// Pairs (c2 % Cfg<D>::kSoftEvery == 0) of each softmax row use the software
+// exp2, so the FMA pipe takes part of the exponentials off the exp unit.
+// Measured on B200: one pair in 3 is best at d = 64 (1.445 ms against 1.514 ms
+// for 1 in 4 on S = 32768), one in 4 at d = 32 and d = 128.
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h2 = __floats2bfloat162_rn(lo, hi);
@@ -286,6 +283,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
               ok = false;
               break;
             }
+            // S(j+1,h) overwrites the S buffer that holds P(j,h): PV(j,h) first
             if (!mbar_wait(&o_done[x * 2 + h], j & 1, &abort_flag, dev_err)) {
               ok = false;
               break;
@@ -351,7 +349,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
           for (int c2 = 0; c2 < 32; ++c2) {
             const float2 arg = ffma2(s2[c2], scale2, negm2);
             float2 p;
-            if ((c2 % kSoftExpEvery) == 0) {
+            if ((c2 % C::kSoftEvery) == 0) {
               p = soft_exp2x2(arg);
             } else {
               p.x = fast_exp2(arg.x);
