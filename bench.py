@@ -143,9 +143,10 @@ def barrier(world):
 
 
 # ----------------------------------------------------------------------- oracle
-def oracle_step_time(w, inp, b: int = 0):
+def oracle_step_time(w, inp, b: int = 0, s_len: int | None = None):
     """One bounded sample of the workload through the float64 oracle on the
-    host cores: the prefill of sequence b (all S tokens) plus its decode step."""
+    host cores: the prefill of the first s_len tokens (default all S) of
+    sequence b plus its decode step."""
     import numpy as np
     import oracle.ccgqa as O
     f = lambda t: None if t is None else t.double().numpy()  # noqa: E731
@@ -155,6 +156,8 @@ def oracle_step_time(w, inp, b: int = 0):
                   conv_k_chan=f(inp["conv_k_chan"]), qk_mean=w.qk_mean,
                   value_shift=w.value_shift, rope_base=w.rope_base, causal=w.causal)
     x = f(inp["x"][b])
+    if s_len is not None:
+        x = x[:s_len]
     t0 = time.perf_counter()
     _, st = O.prefill(lay, x)
     O.decode_step(lay, st, x[-1])
@@ -170,20 +173,35 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
+def reference_sample_len(w, inp, n_calls, budget_s):
+    """Prefix length S' (a multiple of 128, at most S) whose oracle step fits
+    budget_s / n_calls, from a 512-token probe scaled by (S'/512)^2 (the
+    attention's share grows quadratically, so the estimate errs long)."""
+    probe = min(512, w.S)
+    t_probe = oracle_step_time(w, inp, s_len=probe)
+    per_call = budget_s / max(n_calls, 1)
+    s_len = int(probe * (per_call / max(t_probe, 1e-6)) ** 0.5) // 128 * 128
+    return max(128, min(w.S, s_len))
+
+
 def run_reference(args, world, rank):
     from compressed_latent_grouped_b200.workloads import WORKLOADS, make_inputs
     if rank != 0:
         return
     w = WORKLOADS[WORKLOAD]
     inp = make_inputs(w, seed=0, batch=1)
+    # each step: one sequence's prefill over a prefix sized so that the whole
+    # run (warm-up included) stays within --ref-seconds
+    s_len = reference_sample_len(w, inp, args.steps + args.warmup, args.ref_seconds)
     for _ in range(args.warmup):
-        oracle_step_time(w, inp)
-    times = [oracle_step_time(w, inp) for _ in range(args.steps)]
+        oracle_step_time(w, inp, s_len=s_len)
+    times = [oracle_step_time(w, inp, s_len=s_len) for _ in range(args.steps)]
     t = sum(times)
-    tokens = (w.S + 1) * args.steps
+    tokens = (s_len + 1) * args.steps
     value = tokens / t
     cores = blas_threads()
-    sample = f"1 of {w.B} sequences per step: prefill of all {w.S} tokens + 1 decode step"
+    sample = (f"1 of {w.B} sequences per step: float64 prefill of its first {s_len} of {w.S} "
+              f"tokens + 1 decode step")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -444,11 +462,14 @@ def run_ours(args, world, rank, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         one = make_inputs(w, seed=0, batch=1)
-        t_cpu = oracle_step_time(w, one)
-        cpu = {"value": (w.S + 1) / t_cpu, "unit": "tokens/s", "cores": blas_threads(),
+        t_cpu, reps = 0.0, 0
+        while t_cpu < 10.0 and reps < 8:   # about 10-30 s of host work
+            t_cpu += oracle_step_time(w, one)
+            reps += 1
+        cpu = {"value": reps * (w.S + 1) / t_cpu, "unit": "tokens/s", "cores": blas_threads(),
                "kind": "oracle",
-               "sample": f"1 of {w.B} sequences: float64 prefill of all {w.S} tokens + 1 "
-                         f"decode step ({t_cpu:.1f} s)"}
+               "sample": f"1 of {w.B} sequences, {reps} times: float64 prefill of all {w.S} "
+                         f"tokens + 1 decode step ({t_cpu:.1f} s)"}
 
     by_workload = None
     if rank == 0 and not args.no_extra:
@@ -513,6 +534,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=150.0,
+                    help="--impl reference: host-time budget of the whole run")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the other workloads' kernel measurements")
     ap.add_argument("--workload", default=None,
