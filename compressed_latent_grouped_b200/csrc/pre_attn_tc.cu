@@ -68,8 +68,24 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
                : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Wait until at most n of this thread's committed cp.async groups are pending
+// (n < 10; the instruction takes an immediate).
+__device__ __forceinline__ void cp_async_wait_pending(int n) {
+  switch (n) {
+    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+    case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+    case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+    case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
+    case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
+    case 7: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
+    case 8: asm volatile("cp.async.wait_group 8;" ::: "memory"); break;
+    default: asm volatile("cp.async.wait_group 9;" ::: "memory"); break;
+  }
 }
 
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
@@ -138,26 +154,25 @@ __global__ void __launch_bounds__(kPtThreads)
     tmem_relinquish();
   }
 
-  // 1. staging, all by cp.async: the q~ | k~ | v~ rows, the mix weights and
-  // the raw conv taps
-  {
-    // a warp per staged row, lanes over its 16-byte chunks
-    const int cq = QC / 8, per_row = cq + 2 * NCH;
-    const int lane = tid & 31;
-    for (int r = warp; r < kPtTT + kPtHalo; r += kPtThreads / 32) {
+  // 1. staging, all by cp.async, in commit groups in the order the head loop
+  // needs them: A = taps, every W_h, the key head's and query head 0's rows;
+  // then query head 1, ..., query head G-1; last the value head's rows.  The
+  // loop waits for one more group per head, so copies overlap the first heads.
+  const int cq = QC / 8;
+  // one head's NCH 16-byte chunks of every staged row, starting at chunk c_lo
+  // (threads run over (row, chunk) pairs, NCH a power of two)
+  auto stage_head = [&](int c_lo, int col0) {
+    for (int idx = tid; idx < (kPtTT + kPtHalo) * NCH; idx += kPtThreads) {
+      const int r = idx / NCH, c = idx % NCH;
       const int t = t0 - kPtHalo + r;
-      const bool in = t >= 0 && t < S;
-      const bf16* srow = src_b + static_cast<int64_t>(in ? t : 0) * ld;
-      for (int c = lane; c < per_row; c += 32) {
-        const int col = c < cq ? qcol0 + c * 8
-                               : (c < cq + NCH ? kcol0 + (c - cq) * 8 : vcol0 + (c - cq - NCH) * 8);
-        bf16* dst = z + r * ZC + c * 8;
-        if (in)
-          cp_async16(dst, srow + col);
-        else
-          *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-      }
+      bf16* dst = z + r * ZC + (c_lo + c) * 8;
+      if (t >= 0 && t < S)
+        cp_async16(dst, src_b + static_cast<int64_t>(t) * ld + col0 + c * 8);
+      else
+        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
     }
+  };
+  {
     // W_h row n (output channel), chunk j of the input channels -> B operand
     for (int idx = tid; idx < NH * D * NCH; idx += kPtThreads) {
       const int hh = idx / (D * NCH), rem = idx % (D * NCH);   // D * NCH: a power of two
@@ -173,6 +188,15 @@ __global__ void __launch_bounds__(kPtThreads)
                                : a.wk_seq + static_cast<int64_t>(g) * D * K + (idx - nq) * 8;
       cp_async16(tr + idx * 8, w);
     }
+    stage_head(cq, kcol0);   // key head
+    stage_head(0, qcol0);    // query head 0
+    cp_async_commit();
+    for (int hh = 1; hh < G; ++hh) {
+      stage_head(hh * NCH, qcol0 + hh * D);
+      cp_async_commit();
+    }
+    stage_head(cq + NCH, vcol0);   // value head
+    cp_async_commit();
   }
   // RoPE table while the copies fly: (cos, sin) of t * theta_i, the angle taken
   // modulo one turn exactly in 64-bit fixed point, then |2 pi f| <= pi.
@@ -186,7 +210,7 @@ __global__ void __launch_bounds__(kPtThreads)
       cs[idx] = make_float2(cn, sn);
     }
   }
-  cp_async_wait_all();
+  cp_async_wait_pending(G);    // group A: taps, W, key head, query head 0
   fence_proxy_async_smem();    // W tiles (and later U) are read by the tensor core
   tc_fence_before();
   __syncthreads();
@@ -197,17 +221,7 @@ __global__ void __launch_bounds__(kPtThreads)
     const int hc = idx >> 2, k = idx & 3;
     ws[idx] = k < K ? __bfloat162float(tr[hc * K + k]) : 0.f;
   }
-  // 3. value-shift out of the staged rows: v[t, :d/2] = v~[t, :d/2] and
-  // v[t, d/2:] = v~[t-1, d/2:] (the staged row before position 0 is zero)
-  for (int idx = tid; idx < kPtTT * NCH; idx += kPtThreads) {
-    const int tl = idx / NCH, i = (idx - tl * NCH) * 8;
-    const int t = t0 + tl;
-    if (t >= S) continue;
-    const int row = (a.value_shift && i >= D / 2) ? tl + kPtHalo - 1 : tl + kPtHalo;
-    *reinterpret_cast<uint4*>(a.v_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + t) * D +
-                              i) = *reinterpret_cast<const uint4*>(z + row * ZC + QC + D + i);
-  }
-  __syncthreads();
+  __syncthreads();   // fp32 taps ready
 
   // 2. per head
   const int r = tid & (kPtTT - 1);         // position row == TMEM lane
@@ -365,6 +379,9 @@ __global__ void __launch_bounds__(kPtThreads)
       tc_fence_after();
     }
     if (ok) conv(hh);
+    // the next head's rows (the key head needs every query head's): at most
+    // G - hh - 1 groups may still be pending, or just the value head's
+    if (hh + 1 < NH) cp_async_wait_pending(hh + 1 < G ? G - hh - 1 : 1);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -376,6 +393,20 @@ __global__ void __launch_bounds__(kPtThreads)
   ok = ok && mbar_wait(&mma_done[(NH - 1) & 1], ((NH - 1) >> 1) & 1, &abort_flag, a.dev_err);
   tc_fence_after();
   if (ok) epilogue(NH - 1);
+  cp_async_wait_pending(0);   // the value head's rows
+  __syncthreads();
+
+  // 3. value-shift out of the staged rows: v[t, :d/2] = v~[t, :d/2] and
+  // v[t, d/2:] = v~[t-1, d/2:] (the staged row before position 0 is zero)
+  for (int idx = tid; idx < kPtTT * NCH; idx += kPtThreads) {
+    const int tl = idx / NCH, i = (idx - tl * NCH) * 8;
+    const int t = t0 + tl;
+    if (t >= S) continue;
+    const int row = (a.value_shift && i >= D / 2) ? tl + kPtHalo - 1 : tl + kPtHalo;
+    *reinterpret_cast<uint4*>(a.v_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + t) * D +
+                              i) = *reinterpret_cast<const uint4*>(z + row * ZC + QC + D + i);
+  }
+
 
   // 4. decode state, written by the CTA that holds position S-1 (rows S-KH .. S-1
   // are staged; rows before position 0 are zero).
