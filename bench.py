@@ -323,6 +323,8 @@ def run_workload_only(args, local):
         w = w.with_(B=args.batch)
     if args.seq:
         w = w.with_(S=args.seq)
+    if args.decode:
+        w = w.with_(decode=True)
     res = (measure_decode_workload if w.decode else measure_prefill_workload)(
         w, args.steps, dev)
     print(json.dumps({"workload": args.workload, "B": w.B, "S": w.S, **res}), flush=True)
@@ -542,6 +544,8 @@ def main():
                     help="time only this workload's kernels (profiling)")
     ap.add_argument("--batch", type=int, default=0, help="with --workload: override B")
     ap.add_argument("--seq", type=int, default=0, help="with --workload: override S (or L)")
+    ap.add_argument("--decode", action="store_true",
+                    help="with --workload: time a decode step against a cache of S tokens")
     args = ap.parse_args()
     world, rank, local = dist_setup(args.gpus)
     try:

@@ -28,7 +28,11 @@ namespace ccgqa {
 constexpr int kGvMaxB = 16;
 constexpr size_t kGvMaxX = 64 * 1024;
 static bool decode_use_gemv(int B, int E, int es) {
-  return B <= kGvMaxB && static_cast<size_t>(B) * E * es <= kGvMaxX;
+  // x fits in shared memory, and a W row is a whole number of 512-byte steps
+  // (32 lanes x 16 bytes), at most 16 of them (held in registers)
+  const size_t row = static_cast<size_t>(E) * es;
+  return B <= kGvMaxB && static_cast<size_t>(B) * row <= kGvMaxX && row % 512 == 0 &&
+         row <= 512 * 16;
 }
 // E range of one projection split: E / e_splits rounded up to whole 64-wide steps.
 static int decode_proj_e_len(int E, int e_splits) {
@@ -210,51 +214,96 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// out[b][n] = sum_k x[b][k] W[n][k] for B <= 16: x staged once per CTA in shared
-// memory, each warp owns output columns and streams their W rows with 16-byte
-// loads (all of a row's loads in flight), then reduces across its lanes.
-template <typename T>
+// out[b][n] = sum_k x[b][k] W[n][k] for B <= BB (<= 16): one warp per output
+// column.  A warp first issues every 16-byte load of its W row (the row stays
+// in registers as raw 16-byte words), then the CTA stages x in shared memory,
+// so the two memory latencies overlap; the products are reduced across lanes.
+constexpr int kGvMaxIt = 16;   // 16-byte words per lane: E <= 32 * kGvMaxIt * (16 / sizeof(T))
+
+template <typename T, int BB>
 __global__ void __launch_bounds__(256)
     decode_gemv_kernel(const T* __restrict__ x, const T* __restrict__ W, float* __restrict__ out,
                        int B, int E, int N) {
   constexpr int VEC = 16 / sizeof(T);
   extern __shared__ float4 gv_f4[];
   T* xs = reinterpret_cast<T*>(gv_f4);             // [B][E]
+  const int lane = threadIdx.x & 31;
+  const int n = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int nit = E / (32 * VEC);
+  uint4 wraw[kGvMaxIt];
+  if (n < N) {
+    const uint4* wr = reinterpret_cast<const uint4*>(W + static_cast<int64_t>(n) * E) + lane;
+#pragma unroll
+    for (int it = 0; it < kGvMaxIt; ++it)
+      if (it < nit) wraw[it] = __ldg(wr + it * 32);
+  }
 #pragma unroll 4
   for (int idx = threadIdx.x; idx < B * E / VEC; idx += blockDim.x)
     reinterpret_cast<uint4*>(xs)[idx] = reinterpret_cast<const uint4*>(x)[idx];
   __syncthreads();
-  const int lane = threadIdx.x & 31;
-  const int warps = gridDim.x * (blockDim.x >> 5);
-  for (int n = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); n < N; n += warps) {
-    float acc[kGvMaxB];
+  if (n >= N) return;
+  float acc[BB];
 #pragma unroll
-    for (int b = 0; b < kGvMaxB; ++b) acc[b] = 0.f;
-    const T* wr = W + static_cast<int64_t>(n) * E;
-#pragma unroll 4
-    for (int k0 = lane * VEC; k0 < E; k0 += 32 * VEC) {
-      float wv[VEC];
-      load16(wr + k0, wv);
+  for (int b = 0; b < BB; ++b) acc[b] = 0.f;
 #pragma unroll
-      for (int b = 0; b < kGvMaxB; ++b) {
-        if (b < B) {
-          float xv[VEC];
-          load16(xs + static_cast<int64_t>(b) * E + k0, xv);
+  for (int it = 0; it < kGvMaxIt; ++it) {
+    if (it >= nit) break;
+    float wv[VEC];
+    if constexpr (sizeof(T) == 2) {
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&wraw[it]);
 #pragma unroll
-          for (int u = 0; u < VEC; ++u) acc[b] = fmaf(wv[u], xv[u], acc[b]);
-        }
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h[i]);
+        wv[2 * i] = f.x;
+        wv[2 * i + 1] = f.y;
       }
+    } else {
+      const float4 f = *reinterpret_cast<const float4*>(&wraw[it]);
+      wv[0] = f.x;
+      wv[1] = f.y;
+      wv[2] = f.z;
+      wv[3] = f.w;
     }
+    const int k0 = (it * 32 + lane) * VEC;
 #pragma unroll
-    for (int b = 0; b < kGvMaxB; ++b) {
+    for (int b = 0; b < BB; ++b) {
       if (b < B) {
-        float v = acc[b];
+        float xv[VEC];
+        load16(xs + b * E + k0, xv);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        if (lane == 0) out[static_cast<int64_t>(b) * N + n] = v;
+        for (int u = 0; u < VEC; ++u) acc[b] = fmaf(wv[u], xv[u], acc[b]);
       }
     }
   }
+#pragma unroll
+  for (int b = 0; b < BB; ++b) {
+    if (b < B) {
+      float v = acc[b];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      if (lane == 0) out[static_cast<int64_t>(b) * N + n] = v;
+    }
+  }
+}
+
+template <typename T>
+cudaError_t launch_gemv(const T* x, const T* W, float* out, int B, int E, int N,
+                        cudaStream_t stream) {
+  const size_t xb = static_cast<size_t>(B) * E * sizeof(T);
+  const int blocks = (N + 7) / 8;   // one warp per column
+  auto go = [&](auto kernel) -> cudaError_t {
+    if (xb > 48 * 1024) {
+      cudaError_t e = allow_smem(reinterpret_cast<const void*>(kernel), static_cast<int>(xb));
+      if (e != cudaSuccess) return e;
+    }
+    kernel<<<blocks, 256, xb, stream>>>(x, W, out, B, E, N);
+    return cudaSuccess;
+  };
+  if (B <= 1) return go(decode_gemv_kernel<T, 1>);
+  if (B <= 2) return go(decode_gemv_kernel<T, 2>);
+  if (B <= 4) return go(decode_gemv_kernel<T, 4>);
+  if (B <= 8) return go(decode_gemv_kernel<T, 8>);
+  return go(decode_gemv_kernel<T, 16>);
 }
 
 // ----------------------------------------------------------------- pre-step
@@ -264,7 +313,7 @@ __global__ void __launch_bounds__(256)
 template <typename T>
 __host__ __device__ inline size_t decode_pre_floats(int G, int d, int K) {
   const int KH = K > 0 ? K - 1 : 0, HC = (G + 1) * d, AC = HC + d;
-  return (static_cast<size_t>(AC + KH * HC + 2 * HC) + 3) & ~size_t(3);
+  return (static_cast<size_t>(AC + KH * HC + 2 * HC + 4 * HC) + 3) & ~size_t(3);
 }
 template <typename T>
 __host__ __device__ inline size_t decode_pre_wt_bytes(int G, int d) {
@@ -289,6 +338,7 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
   float* hz = zc + AC;            // [KH][HC] history
   float* u = hz + KH * HC;        // [HC]
   float* y = u + HC;              // [HC]
+  float* tp = y + HC;             // [HC][4] conv taps, zero past K
   const int tid = threadIdx.x;
   const int L = __ldcg(a.len + b);
   if (L < 0 || L >= a.cap) {
@@ -340,6 +390,15 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
     zc[c] = val;
   }
 #pragma unroll 4
+  for (int idx = tid; idx < HC * 4; idx += blockDim.x) {
+    const int c = idx >> 2, j = idx & 3;
+    float v = 0.f;
+    if (j < K)
+      v = to_f32(c < QC ? a.wq_seq[static_cast<int64_t>(qcol0 + c) * K + j]
+                        : a.wk_seq[static_cast<int64_t>(g * d + (c - QC)) * K + j]);
+    tp[idx] = v;
+  }
+#pragma unroll 4
   for (int idx = tid; idx < KH * HC; idx += blockDim.x) {
     const int r = idx / HC, c = idx - r * HC;
     hz[idx] = c < QC ? to_f32(a.hist_q[(static_cast<int64_t>(b) * KH + r) * a.Hq * d + qcol0 + c])
@@ -351,11 +410,9 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
   for (int c = tid; c < HC; c += blockDim.x) {
     float acc;
     if (K > 0) {
-      const bool is_q = c < QC;
-      const T* w = is_q ? a.wq_seq + static_cast<int64_t>(qcol0 + c) * K
-                        : a.wk_seq + static_cast<int64_t>(g * d + (c - QC)) * K;
-      acc = to_f32(w[0]) * zc[c];
-      for (int j = 1; j < K; ++j) acc = fmaf(to_f32(w[j]), hz[(KH - j) * HC + c], acc);
+      const float* w = tp + c * 4;
+      acc = w[0] * zc[c];
+      for (int j = 1; j < K; ++j) acc = fmaf(w[j], hz[(KH - j) * HC + c], acc);
     } else {
       acc = zc[c];
     }
@@ -708,13 +765,8 @@ cudaError_t launch_decode_step(const DecodeArgs<T>& a, cudaStream_t stream) {
   mark(0);
   if (a.W) {
     if (decode_use_gemv(a.B, a.E, sizeof(T)) && a.e_splits == 1) {
-      const size_t xb = static_cast<size_t>(a.B) * a.E * sizeof(T);
-      if (xb > 48 * 1024 &&
-          (e = allow_smem(reinterpret_cast<const void*>(decode_gemv_kernel<T>), static_cast<int>(xb))) !=
-              cudaSuccess)
+      if ((e = launch_gemv<T>(a.x_t, a.W, a.proj_part, a.B, a.E, a.N, stream)) != cudaSuccess)
         return e;
-      const int blocks = (a.N + 7) / 8;   // one warp per column
-      decode_gemv_kernel<T><<<blocks, 256, xb, stream>>>(a.x_t, a.W, a.proj_part, a.B, a.E, a.N);
     } else {
       const int e_len = decode_proj_e_len(a.E, a.e_splits);
       dim3 grid((a.N + kPN - 1) / kPN, a.e_splits, (a.B + kPB - 1) / kPB);
