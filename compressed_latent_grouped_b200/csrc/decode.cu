@@ -307,19 +307,46 @@ cudaError_t launch_gemv(const T* x, const T* W, float* out, int B, int E, int N,
 }
 
 // ----------------------------------------------------------------- pre-step
-// Shared-memory bytes of the pre-step: fp32 rows (current, history, conv out,
-// mix out) plus, when it fits, the group's G + 1 channel-mix weights staged
-// transposed in the working dtype.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_group() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all_groups() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// Shared memory of the pre-step (byte offsets, each 16-byte aligned): fp32
+// rows (current pre-conv row zc[AC], conv out u[HC], mix out y[HC], taps
+// tp[HC][4]), the history rows hz[KH][HC] and the raw taps in the working
+// dtype, and -- when they fit -- the group's G + 1 channel-mix weights, raw
+// (as copied) and transposed.
+struct PreSmem {
+  size_t zc, u, y, tp, hz, tr, wt, wraw, bytes_no_w, bytes;
+};
 template <typename T>
-__host__ __device__ inline size_t decode_pre_floats(int G, int d, int K) {
+__host__ __device__ inline PreSmem pre_smem(int G, int d, int K) {
   const int KH = K > 0 ? K - 1 : 0, HC = (G + 1) * d, AC = HC + d;
-  return (static_cast<size_t>(AC + KH * HC + 2 * HC + 4 * HC) + 3) & ~size_t(3);
+  auto up = [](size_t x) { return (x + 15) & ~size_t(15); };
+  PreSmem L;
+  L.zc = 0;
+  L.u = up(L.zc + AC * 4);
+  L.y = up(L.u + HC * 4);
+  L.tp = up(L.y + HC * 4);
+  L.hz = up(L.tp + HC * 16);
+  L.tr = up(L.hz + static_cast<size_t>(KH) * HC * sizeof(T));
+  L.wt = up(L.tr + static_cast<size_t>(HC) * (K > 0 ? K : 1) * sizeof(T));
+  L.bytes_no_w = L.wt;
+  const size_t wb = static_cast<size_t>(G + 1) * d * d * sizeof(T);
+  L.wraw = up(L.wt + wb);
+  L.bytes = up(L.wraw + wb);
+  return L;
 }
-template <typename T>
-__host__ __device__ inline size_t decode_pre_wt_bytes(int G, int d) {
-  return static_cast<size_t>(G + 1) * d * d * sizeof(T);
-}
-constexpr size_t kPreWtMax = 160 * 1024;
+constexpr size_t kPreSmemMax = 200 * 1024;
 // One CTA per (sequence, kv group); its work is a handful of dependent phases,
 // each limited by one round of global loads, so every loop below is unrolled
 // to keep several independent loads in flight per thread.
@@ -329,16 +356,20 @@ template <typename T>
 __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_constant__ DecodeArgs<T> a,
                                                          int stage_wt) {
   extern __shared__ float4 dsm_f4[];
-  float* sm = reinterpret_cast<float*>(dsm_f4);
+  uint8_t* sm = reinterpret_cast<uint8_t*>(dsm_f4);
   const int g = blockIdx.x, b = blockIdx.y;
   const int d = a.d, G = a.G, K = a.K, half = d / 2;
   const int KH = K > 0 ? K - 1 : 0;
   const int QC = G * d, HC = QC + d, AC = HC + d;  // q | k | v channels of the group
-  float* zc = sm;                 // [AC] current pre-conv row
-  float* hz = zc + AC;            // [KH][HC] history
-  float* u = hz + KH * HC;        // [HC]
-  float* y = u + HC;              // [HC]
-  float* tp = y + HC;             // [HC][4] conv taps, zero past K
+  const PreSmem Ls = pre_smem<T>(G, d, K);
+  float* zc = reinterpret_cast<float*>(sm + Ls.zc);   // [AC] current pre-conv row
+  float* u = reinterpret_cast<float*>(sm + Ls.u);     // [HC]
+  float* y = reinterpret_cast<float*>(sm + Ls.y);     // [HC]
+  float* tp = reinterpret_cast<float*>(sm + Ls.tp);   // [HC][4] conv taps, zero past K
+  T* hz = reinterpret_cast<T*>(sm + Ls.hz);           // [KH][HC] history rows
+  T* tr = reinterpret_cast<T*>(sm + Ls.tr);           // [HC][K] taps as stored
+  T* wt = reinterpret_cast<T*>(sm + Ls.wt);           // [G+1][d][d] mix weights, transposed
+  T* wraw = reinterpret_cast<T*>(sm + Ls.wraw);       // [G+1][d][d] mix weights, as stored
   const int tid = threadIdx.x;
   const int L = __ldcg(a.len + b);
   if (L < 0 || L >= a.cap) {
@@ -346,24 +377,28 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
     return;
   }
   const int qcol0 = g * G * d, kcol0 = a.Hq * d + g * d, vcol0 = (a.Hq + a.Hkv) * d + g * d;
-  // channel-mix weights of the group, transposed: wt[hh][j][i] = W_hh[i][j]
-  T* wt = reinterpret_cast<T*>(sm + decode_pre_floats<T>(G, d, K));
   const bool have_mix = K > 0 && a.wq_chan != nullptr && a.wk_chan != nullptr;
-  if (stage_wt && have_mix) {
+  // 1. every input in one round of memory latency: the weights, taps and
+  // history rows by 16-byte cp.async (contiguous per group), the projection
+  // partials summed meanwhile
+  {
     constexpr int VEC = 16 / sizeof(T);
-    const int per_head = d * d / VEC;
-#pragma unroll 4
-    for (int idx = tid; idx < (G + 1) * per_head; idx += blockDim.x) {
-      // lanes run over rows i, so the transposed stores hit consecutive addresses
-      const int hh = idx / per_head, rem = idx - hh * per_head;
-      const int i = rem % d, j0 = (rem / d) * VEC;
-      const T* src = hh < G ? a.wq_chan + (static_cast<int64_t>(g * G + hh) * d + i) * d + j0
-                            : a.wk_chan + (static_cast<int64_t>(g) * d + i) * d + j0;
-      T v[VEC];
-      *reinterpret_cast<uint4*>(v) = *reinterpret_cast<const uint4*>(src);
-#pragma unroll
-      for (int u = 0; u < VEC; ++u) wt[(static_cast<int64_t>(hh) * d + j0 + u) * d + i] = v[u];
+    auto copy = [&](T* dst, const T* src, int n) {   // n elements, a multiple of VEC
+      for (int i = tid * VEC; i < n; i += blockDim.x * VEC) cp_async16(dst + i, src + i);
+    };
+    if (stage_wt && have_mix) {
+      copy(wraw, a.wq_chan + static_cast<int64_t>(g) * G * d * d, G * d * d);
+      copy(wraw + G * d * d, a.wk_chan + static_cast<int64_t>(g) * d * d, d * d);
     }
+    if (K > 0) {
+      copy(tr, a.wq_seq + static_cast<int64_t>(g) * G * d * K, G * d * K);
+      copy(tr + G * d * K, a.wk_seq + static_cast<int64_t>(g) * d * K, d * K);
+    }
+    for (int r = 0; r < KH; ++r) {
+      copy(hz + r * HC, a.hist_q + (static_cast<int64_t>(b) * KH + r) * a.Hq * d + qcol0, QC);
+      copy(hz + r * HC + QC, a.hist_k + (static_cast<int64_t>(b) * KH + r) * a.Hkv * d + g * d, d);
+    }
+    cp_async_commit_group();
   }
 #pragma unroll 2
   for (int c = tid; c < AC; c += blockDim.x) {
@@ -378,9 +413,9 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
       int s = 0;
       for (; s + 8 <= a.e_splits; s += 8) {
 #pragma unroll
-        for (int u = 0; u < 8; ++u) pv[u] = __ldcg(pp + (s + u) * pstride);
+        for (int q = 0; q < 8; ++q) pv[q] = __ldcg(pp + (s + q) * pstride);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) val += pv[u];
+        for (int q = 0; q < 8; ++q) val += pv[q];
       }
       for (; s < a.e_splits; ++s) val += __ldcg(pp + s * pstride);
       val = to_f32(from_f32<T>(val));  // the projection output is held in the working dtype
@@ -389,21 +424,20 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
     }
     zc[c] = val;
   }
-#pragma unroll 4
+  cp_async_wait_all_groups();
+  __syncthreads();
+  // 2. shared-memory reshuffles: taps to fp32 [HC][4]; mix weights transposed,
+  // wt[hh][j][i] = W_hh[i][j] (lanes run over rows i: consecutive stores)
   for (int idx = tid; idx < HC * 4; idx += blockDim.x) {
     const int c = idx >> 2, j = idx & 3;
-    float v = 0.f;
-    if (j < K)
-      v = to_f32(c < QC ? a.wq_seq[static_cast<int64_t>(qcol0 + c) * K + j]
-                        : a.wk_seq[static_cast<int64_t>(g * d + (c - QC)) * K + j]);
-    tp[idx] = v;
+    tp[idx] = j < K ? to_f32(tr[c * K + j]) : 0.f;
   }
-#pragma unroll 4
-  for (int idx = tid; idx < KH * HC; idx += blockDim.x) {
-    const int r = idx / HC, c = idx - r * HC;
-    hz[idx] = c < QC ? to_f32(a.hist_q[(static_cast<int64_t>(b) * KH + r) * a.Hq * d + qcol0 + c])
-                     : to_f32(a.hist_k[(static_cast<int64_t>(b) * KH + r) * a.Hkv * d + g * d +
-                                       (c - QC)]);
+  if (stage_wt && have_mix) {
+    for (int idx = tid; idx < (G + 1) * d * d; idx += blockDim.x) {
+      const int hh = idx / (d * d), rem = idx - hh * d * d;
+      const int i = rem % d, j = rem / d;
+      wt[(hh * d + j) * d + i] = wraw[(hh * d + i) * d + j];
+    }
   }
   __syncthreads();
   // causal conv: tap j reads the row j steps back (history row KH - j)
@@ -412,7 +446,7 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
     if (K > 0) {
       const float* w = tp + c * 4;
       acc = w[0] * zc[c];
-      for (int j = 1; j < K; ++j) acc = fmaf(w[j], hz[(KH - j) * HC + c], acc);
+      for (int j = 1; j < K; ++j) acc = fmaf(w[j], to_f32(hz[(KH - j) * HC + c]), acc);
     } else {
       acc = zc[c];
     }
@@ -485,7 +519,7 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
   // state: histories shift by one row, v_prev = this row's v~
   for (int idx = tid; idx < KH * HC; idx += blockDim.x) {
     const int r = idx / HC, c = idx - r * HC;
-    const float val = (r + 1 < KH) ? hz[(r + 1) * HC + c] : zc[c];
+    const float val = (r + 1 < KH) ? to_f32(hz[(r + 1) * HC + c]) : zc[c];
     if (c < QC)
       a.hist_q[(static_cast<int64_t>(b) * KH + r) * a.Hq * d + qcol0 + c] = from_f32<T>(val);
     else
@@ -777,9 +811,9 @@ cudaError_t launch_decode_step(const DecodeArgs<T>& a, cudaStream_t stream) {
   }
   mark(1);
   {
-    const size_t wt = decode_pre_wt_bytes<T>(a.G, a.d);
-    const int stage_wt = wt <= kPreWtMax;
-    const size_t smem = decode_pre_floats<T>(a.G, a.d, a.K) * 4 + (stage_wt ? wt : 0) + 16;
+    const PreSmem Ls = pre_smem<T>(a.G, a.d, a.K);
+    const int stage_wt = Ls.bytes <= kPreSmemMax;
+    const size_t smem = stage_wt ? Ls.bytes : Ls.bytes_no_w;
     if (smem > 48 * 1024) {
       e = allow_smem(reinterpret_cast<const void*>(decode_pre_kernel<T>),
                                static_cast<int>(smem));
