@@ -6,11 +6,13 @@
 //
 // One CTA owns 128 consecutive positions of one kv group (its G query heads,
 // its key head and its value head) of one sequence:
-//   1. the group's q~ | k~ | v~ rows [t0 - 3, t0 + 128), the G + 1 mix weights
+//   1. the group's q~ | k~ rows [t0 - 3, t0 + 128), the G + 1 mix weights
 //      W_h [d_out, d_in] (straight into the swizzled K-major layout of a UMMA
 //      B operand) and the conv taps are copied into shared memory with 16-byte
-//      cp.async; meanwhile a cos/sin table per (pair, position) is formed, the
-//      angle t theta_i reduced modulo one turn exactly in 64-bit fixed point;
+//      cp.async, in commit groups in the order the heads use them; each thread
+//      loads its value-shift rows into registers and forms the cos/sin of its
+//      own rotary pairs (angle t theta_i reduced modulo one turn exactly in
+//      64-bit fixed point) while the copies land;
 //   2. per head h (G query heads, then the key head):
 //        conv   one thread per (position, 16-byte channel chunk): u = sum_k
 //               w[c, k] z[t - k, c] in fp32, split as u = hi + lo with hi, lo
@@ -22,9 +24,9 @@
 //               tcgen05.ld of Y_h, QK-mean from the staged pre-conv rows, RoPE on
 //               the pairs (i, i + d/2) it holds, bf16 store.
 //      The epilogue of head h - 1 runs while the tensor core computes head h.
-//   3. value-shift: each v row is gathered from staged rows t and t - 1 of
-//      v~, a bit-exact copy.
+//   3. value-shift: the rows loaded in step 1 are stored (bit-exact copies).
 //   4. the CTA holding the last position writes the decode state.
+// At d = 32 three CTAs fit on an SM (about 74 KB of shared memory each).
 // Every wait is bounded; no cluster multicast is used.
 #include <type_traits>
 
@@ -41,25 +43,25 @@ constexpr int kPtTT = 128;     // positions per CTA == MMA M == TMEM lanes
 constexpr int kPtHalo = 3;     // the conv reaches back K - 1 <= 3 rows
 
 struct PtLayout {
-  int ZC;                      // staged row width in elements: (G + 2) d + 8
+  int ZC;                      // staged row width in elements: (G + 1) d + 8
   uint32_t u_bytes, w_bytes;   // one A tile (hi or lo), one head's B tile
-  uint32_t off_u, off_w, off_z, off_cs, off_ws, off_tr, off_bar, bytes;
+  uint32_t off_u, off_w, off_z, off_ws, off_bar, bytes;
 };
 
 // Byte layout of the dynamic shared memory (from a 1024-byte aligned base).
 __host__ __device__ inline PtLayout pt_layout(int d, int G) {
   PtLayout L;
   const uint32_t row = static_cast<uint32_t>(d) * 2;
-  L.ZC = (G + 2) * d + 8;      // q | k | v, + 16 bytes: an odd number of 16-byte units per row
+  L.ZC = (G + 1) * d + 8;      // q | k, + 16 bytes: an odd number of 16-byte units per row
   L.u_bytes = kPtTT * row;
   L.w_bytes = static_cast<uint32_t>(d) * row;
-  L.off_u = 0;                                      // U_hi, U_lo
-  L.off_w = 2 * L.u_bytes;                          // W_h, h = 0..G
+  // U_hi | U_lo; before the first conv the same bytes hold the raw conv taps
+  const uint32_t tr_bytes = (static_cast<uint32_t>(G + 1) * d * 4 * 2 + 15u) & ~15u;
+  L.off_u = 0;
+  L.off_w = 2 * L.u_bytes > tr_bytes ? 2 * L.u_bytes : tr_bytes;   // W_h, h = 0..G
   L.off_z = L.off_w + (G + 1) * L.w_bytes;          // [131][ZC] bf16
-  L.off_cs = L.off_z + ((static_cast<uint32_t>(kPtTT + kPtHalo) * L.ZC * 2 + 15u) & ~15u);
-  L.off_ws = L.off_cs + static_cast<uint32_t>(d / 2) * kPtTT * 8;   // [d/2][128] float2
-  L.off_tr = L.off_ws + static_cast<uint32_t>(G + 1) * d * 16;     // [(G+1) d][4] float
-  L.off_bar = L.off_tr + static_cast<uint32_t>(G + 1) * d * 4 * 2;  // raw taps, <= 4 per channel
+  L.off_ws = L.off_z + ((static_cast<uint32_t>(kPtTT + kPtHalo) * L.ZC * 2 + 15u) & ~15u);
+  L.off_bar = L.off_ws + static_cast<uint32_t>(G + 1) * d * 16;     // [(G+1) d][4] float
   L.bytes = L.off_bar + 64 + 1024;                  // barriers + alignment slack
   return L;
 }
@@ -111,8 +113,10 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// d = 32: three CTAs per SM (about 74 KB of shared memory and at most 85
+// registers a thread each); d = 64: one.
 template <int D>
-__global__ void __launch_bounds__(kPtThreads)
+__global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
     pre_attn_tc_kernel(const __grid_constant__ PreAttnArgs<bf16> a) {
   constexpr uint32_t kRowBytes = D * 2;                 // 64: 64B swizzle, 128: 128B swizzle
   constexpr uint32_t kSwz = (D == 32) ? kSwizzle64B : kSwizzle128B;
@@ -128,9 +132,8 @@ __global__ void __launch_bounds__(kPtThreads)
   const int b = blockIdx.z, g = blockIdx.y, t0 = blockIdx.x * kPtTT;
   const int tid = threadIdx.x, warp = tid >> 5;
   bf16* z = reinterpret_cast<bf16*>(smem + L.off_z);
-  float2* cs = reinterpret_cast<float2*>(smem + L.off_cs);
   float* ws = reinterpret_cast<float*>(smem + L.off_ws);
-  bf16* tr = reinterpret_cast<bf16*>(smem + L.off_tr);
+  bf16* tr = reinterpret_cast<bf16*>(smem + L.off_u);   // raw taps, until the first conv
   uint64_t* mma_done = reinterpret_cast<uint64_t*>(smem + L.off_bar);   // [2]
   uint64_t* drain = mma_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -195,22 +198,39 @@ __global__ void __launch_bounds__(kPtThreads)
       stage_head(hh * NCH, qcol0 + hh * D);
       cp_async_commit();
     }
-    stage_head(cq + NCH, vcol0);   // value head
-    cp_async_commit();
   }
-  // RoPE table while the copies fly: (cos, sin) of t * theta_i, the angle taken
-  // modulo one turn exactly in 64-bit fixed point, then |2 pi f| <= pi.
-  if (a.rope_on) {
-    for (int idx = tid; idx < (D / 2) * kPtTT; idx += kPtThreads) {
-      const int i = idx / kPtTT, tl = idx - i * kPtTT;
-      const uint64_t ph = static_cast<uint64_t>(t0 + tl) * a.rope_frac[i];
-      const float f = static_cast<float>(static_cast<int64_t>(ph)) * 5.42101086242752217e-20f;
-      float sn, cn;
-      __sincosf(6.28318530717958648f * f, &sn, &cn);
-      cs[idx] = make_float2(cn, sn);
+  // value-shift rows straight into registers (stored at the end of the kernel):
+  // v[t, :d/2] = v~[t, :d/2], v[t, d/2:] = v~[t-1, d/2:], zero before position 0
+  constexpr int kVPer = kPtTT * NCH / kPtThreads;
+  uint4 vreg[kVPer];
+#pragma unroll
+  for (int q = 0; q < kVPer; ++q) {
+    const int idx = tid + q * kPtThreads;
+    const int tl = idx / NCH, i = (idx % NCH) * 8;
+    const int tv = t0 + tl;
+    const int row = (a.value_shift && i >= D / 2) ? tv - 1 : tv;
+    vreg[q] = make_uint4(0, 0, 0, 0);
+    if (tv < S && row >= 0)
+      vreg[q] = *reinterpret_cast<const uint4*>(src_b + static_cast<int64_t>(row) * ld + vcol0 + i);
+  }
+  // RoPE of this thread's epilogue pairs (row tid % 128, pairs of half tid / 128)
+  // while the copies fly: (cos, sin) of t * theta_i, the angle taken modulo one
+  // turn exactly in 64-bit fixed point, then |2 pi f| <= pi.
+  float rc[Q4], rs[Q4];
+  {
+    const int tp = t0 + (tid & (kPtTT - 1)), ip = (tid >> 7) * Q4;
+#pragma unroll
+    for (int e = 0; e < Q4; ++e) {
+      rc[e] = 1.f;
+      rs[e] = 0.f;
+      if (a.rope_on) {
+        const uint64_t ph = static_cast<uint64_t>(tp) * a.rope_frac[ip + e];
+        const float f = static_cast<float>(static_cast<int64_t>(ph)) * 5.42101086242752217e-20f;
+        __sincosf(6.28318530717958648f * f, &rs[e], &rc[e]);
+      }
     }
   }
-  cp_async_wait_pending(G);    // group A: taps, W, key head, query head 0
+  cp_async_wait_pending(G - 1);   // group A: taps, W, key head, query head 0
   fence_proxy_async_smem();    // W tiles (and later U) are read by the tensor core
   tc_fence_before();
   __syncthreads();
@@ -348,10 +368,9 @@ __global__ void __launch_bounds__(kPtThreads)
     if (a.rope_on) {
 #pragma unroll
       for (int e = 0; e < Q4; ++e) {
-        const float2 c = cs[(i0 + e) * kPtTT + r];
         const float x0 = lo[e], x1 = hi[e];
-        lo[e] = x0 * c.x - x1 * c.y;
-        hi[e] = x0 * c.y + x1 * c.x;
+        lo[e] = x0 * rc[e] - x1 * rs[e];
+        hi[e] = x0 * rs[e] + x1 * rc[e];
       }
     }
     bf16* dst = hh < G ? a.q_out + ((static_cast<int64_t>(b) * S + t) * a.Hq + g * G + hh) * D
@@ -380,8 +399,8 @@ __global__ void __launch_bounds__(kPtThreads)
     }
     if (ok) conv(hh);
     // the next head's rows (the key head needs every query head's): at most
-    // G - hh - 1 groups may still be pending, or just the value head's
-    if (hh + 1 < NH) cp_async_wait_pending(hh + 1 < G ? G - hh - 1 : 1);
+    // G - hh - 2 groups may still be pending, none before the key head
+    if (hh + 1 < NH) cp_async_wait_pending(hh + 1 < G ? G - hh - 2 : 0);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -393,20 +412,16 @@ __global__ void __launch_bounds__(kPtThreads)
   ok = ok && mbar_wait(&mma_done[(NH - 1) & 1], ((NH - 1) >> 1) & 1, &abort_flag, a.dev_err);
   tc_fence_after();
   if (ok) epilogue(NH - 1);
-  cp_async_wait_pending(0);   // the value head's rows
-  __syncthreads();
-
-  // 3. value-shift out of the staged rows: v[t, :d/2] = v~[t, :d/2] and
-  // v[t, d/2:] = v~[t-1, d/2:] (the staged row before position 0 is zero)
-  for (int idx = tid; idx < kPtTT * NCH; idx += kPtThreads) {
-    const int tl = idx / NCH, i = (idx - tl * NCH) * 8;
-    const int t = t0 + tl;
-    if (t >= S) continue;
-    const int row = (a.value_shift && i >= D / 2) ? tl + kPtHalo - 1 : tl + kPtHalo;
-    *reinterpret_cast<uint4*>(a.v_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + t) * D +
-                              i) = *reinterpret_cast<const uint4*>(z + row * ZC + QC + D + i);
+  // 3. value-shift rows loaded at the start
+#pragma unroll
+  for (int q = 0; q < kVPer; ++q) {
+    const int idx = tid + q * kPtThreads;
+    const int tl = idx / NCH, i = (idx % NCH) * 8;
+    const int tv = t0 + tl;
+    if (tv < S)
+      *reinterpret_cast<uint4*>(a.v_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + tv) * D +
+                                i) = vreg[q];
   }
-
 
   // 4. decode state, written by the CTA that holds position S-1 (rows S-KH .. S-1
   // are staged; rows before position 0 are zero).
@@ -421,11 +436,10 @@ __global__ void __launch_bounds__(kPtThreads)
           a.hist_k[(static_cast<int64_t>(b) * KH + rr) * Hkv * D + g * D + (c - QC)] = zr[c];
       }
     }
-    if (a.v_prev) {
-      const bf16* zr = z + (S - 1 - t0 + kPtHalo) * ZC + QC + D;
+    if (a.v_prev)
       for (int i = tid; i < D; i += kPtThreads)
-        a.v_prev[static_cast<int64_t>(b) * Hkv * D + g * D + i] = zr[i];
-    }
+        a.v_prev[static_cast<int64_t>(b) * Hkv * D + g * D + i] =
+            src_b[static_cast<int64_t>(S - 1) * ld + vcol0 + i];
     if (g == 0 && tid == 0) a.len[b] = S;
   }
 
