@@ -433,10 +433,16 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
     tp[idx] = j < K ? to_f32(tr[c * K + j]) : 0.f;
   }
   if (stage_wt && have_mix) {
-    for (int idx = tid; idx < (G + 1) * d * d; idx += blockDim.x) {
-      const int hh = idx / (d * d), rem = idx - hh * d * d;
-      const int i = rem % d, j = rem / d;
-      wt[(hh * d + j) * d + i] = wraw[(hh * d + i) * d + j];
+    // 16-byte words of W rows out, scattered into columns (lanes over rows i)
+    constexpr int VEC = 16 / sizeof(T);
+    const int per_head = d * d / VEC;
+    for (int idx = tid; idx < (G + 1) * per_head; idx += blockDim.x) {
+      const int hh = idx / per_head, rem = idx - hh * per_head;
+      const int i = rem % d, j0 = (rem / d) * VEC;
+      T v[VEC];
+      *reinterpret_cast<uint4*>(v) = *reinterpret_cast<const uint4*>(wraw + (hh * d + i) * d + j0);
+#pragma unroll
+      for (int q = 0; q < VEC; ++q) wt[(hh * d + j0 + q) * d + i] = v[q];
     }
   }
   __syncthreads();
