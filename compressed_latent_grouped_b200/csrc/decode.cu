@@ -34,6 +34,11 @@ static bool decode_use_gemv(int B, int E, int es) {
   return B <= kGvMaxB && static_cast<size_t>(B) * row <= kGvMaxX && row % 512 == 0 &&
          row <= 512 * 16;
 }
+// More sequences, bf16: the projection on the tensor core, swapped (W rows as M),
+// one CTA per (128 W rows, 64 sequences, 128 of E).
+constexpr int kDpN = 128, kDpB = 64, kDpK = 128;
+static bool decode_use_proj_tc(int E, int es) { return es == 2 && E % kDpK == 0; }
+
 // E range of one projection split: E / e_splits rounded up to whole 64-wide steps.
 static int decode_proj_e_len(int E, int e_splits) {
   const int per = (E + e_splits - 1) / e_splits;
@@ -45,12 +50,14 @@ void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int e
   const int target = 2 * 148;
   if (has_proj && decode_use_gemv(B, E, es)) {
     *e_splits = 1;   // one weight-streaming pass, no partials to sum
+  } else if (has_proj && decode_use_proj_tc(E, es)) {
+    *e_splits = E / kDpK;   // tensor-core tiles of 128 columns x 64 sequences x 128 of E
   } else if (has_proj) {
     // projection CTAs: 64 columns x 64 sequences x one E-split of whole 64-wide steps
     const int tiles = ((N + 63) / 64) * ((B + 63) / 64);
-    int es = target / (tiles > 0 ? tiles : 1);
-    if (es < 1) es = 1;
-    const int e_len = decode_proj_e_len(E, es);
+    int nsp = target / (tiles > 0 ? tiles : 1);
+    if (nsp < 1) nsp = 1;
+    const int e_len = decode_proj_e_len(E, nsp);
     *e_splits = (E + e_len - 1) / e_len;
   } else {
     *e_splits = 0;
@@ -304,6 +311,123 @@ cudaError_t launch_gemv(const T* x, const T* W, float* out, int B, int E, int N,
   if (B <= 4) return go(decode_gemv_kernel<T, 4>);
   if (B <= 8) return go(decode_gemv_kernel<T, 8>);
   return go(decode_gemv_kernel<T, 16>);
+}
+
+// part[s][b][n] = sum over k in [128 s, 128 s + 128) of W[n][k] x[b][k] on the
+// tensor core: D^T = W_tile x_tile^T with M = 128 W rows, N = 64 sequences
+// (rows past B read as zero), K = 128 in 8 steps.  Both tiles arrive by TMA in
+// one round (128B swizzle); one thread issues the MMAs; four warps read the
+// accumulator back (lane = W row) and store fp32 partials, lanes over columns.
+constexpr uint32_t kDpATile = kDpN * 64 * 2, kDpBTile = kDpB * 64 * 2;
+constexpr size_t kDpSmem = 2 * (kDpATile + kDpBTile) + 64 + 1024;
+
+__global__ void __launch_bounds__(128)
+    decode_proj_tc_kernel(const __grid_constant__ CUtensorMap tmW,
+                          const __grid_constant__ CUtensorMap tmX, float* __restrict__ part, int B,
+                          int N, int32_t* dev_err) {
+  extern __shared__ uint8_t dp_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dp_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sa = smem;                          // [2][128 x 64] W blocks
+  uint8_t* sb = smem + 2 * kDpATile;           // [2][64 x 64] x blocks
+  uint64_t* full = reinterpret_cast<uint64_t*>(sb + 2 * kDpBTile);
+  uint64_t* done = full + 1;
+  uint64_t* drain = done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n0 = blockIdx.x * kDpN, sp = blockIdx.y, b0 = blockIdx.z * kDpB;
+  const int e0 = sp * kDpK;
+  if (tid == 0) {
+    mbar_init(full, 1);
+    mbar_init(done, 1);
+    mbar_init(drain, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kDpB);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (tid == 0) {
+    prefetch_tensormap(&tmW);
+    prefetch_tensormap(&tmX);
+    mbar_arrive_expect_tx(full, 2 * (kDpATile + kDpBTile));
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb) {
+      tma_load_2d(sa + kb * kDpATile, &tmW, full, e0 + kb * 64, n0);
+      tma_load_2d(sb + kb * kDpBTile, &tmX, full, e0 + kb * 64, b0);
+    }
+    if (mbar_wait(full, 0, &abort_flag, dev_err)) {
+      tc_fence_after();
+      const uint32_t idesc = make_idesc_bf16(kDpN, kDpB, false);
+#pragma unroll
+      for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t ad = make_smem_desc(smem_addr(sa + kb * kDpATile) + k * 32, 16, 1024,
+                                             kSwizzle128B);
+          const uint64_t bd = make_smem_desc(smem_addr(sb + kb * kDpBTile) + k * 32, 16, 1024,
+                                             kSwizzle128B);
+          mma_ss(tmem, ad, bd, idesc, (kb | k) != 0);
+        }
+      mma_commit(done);
+    }
+  }
+  if (mbar_wait(done, 0, &abort_flag, dev_err)) {
+    tc_fence_after();
+    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    uint32_t v0[32], v1[32];
+    tmem_ld32(trow, v0);
+    tmem_ld32(trow + 32, v1);
+    tmem_wait_ld();
+    const int n = n0 + warp * 32 + lane;
+    if (n < N) {
+#pragma unroll
+      for (int c = 0; c < kDpB; ++c) {
+        const int b = b0 + c;
+        if (b < B)
+          part[(static_cast<int64_t>(sp) * B + b) * N + n] = __uint_as_float(c < 32 ? v0[c] : v1[c - 32]);
+      }
+    }
+  }
+  if (abort_flag && tid == 0) {
+    // Do not release TMEM while an MMA might still write it.
+    mma_commit(drain);
+    const long long c0 = clock64();
+    while (!mbar_try_wait(drain, 0) && clock64() - c0 < kWaitLimitCycles) {
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kDpB);
+  }
+}
+
+cudaError_t launch_decode_proj_tc(const bf16* x, const bf16* W, float* part, int B, int E, int N,
+                                  int32_t* dev_err, cudaStream_t stream) {
+  CUtensorMap tmW, tmX;
+  const uint64_t dW[2] = {static_cast<uint64_t>(E), static_cast<uint64_t>(N)};
+  const uint64_t dX[2] = {static_cast<uint64_t>(E), static_cast<uint64_t>(B)};
+  const uint64_t st[1] = {static_cast<uint64_t>(E) * 2};
+  const uint32_t bW[2] = {64, kDpN}, bX[2] = {64, kDpB};
+  if (!encode_tensor_map(&tmW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, dW, st, bW,
+                         CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tensor_map(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, dX, st, bX,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  cudaError_t e = allow_smem(reinterpret_cast<const void*>(decode_proj_tc_kernel),
+                             static_cast<int>(kDpSmem));
+  if (e != cudaSuccess) return e;
+  dim3 grid((N + kDpN - 1) / kDpN, E / kDpK, (B + kDpB - 1) / kDpB);
+  decode_proj_tc_kernel<<<grid, 128, kDpSmem, stream>>>(tmW, tmX, part, B, N, dev_err);
+  return cudaSuccess;
 }
 
 // ----------------------------------------------------------------- pre-step
@@ -807,6 +931,12 @@ cudaError_t launch_decode_step(const DecodeArgs<T>& a, cudaStream_t stream) {
     if (decode_use_gemv(a.B, a.E, sizeof(T)) && a.e_splits == 1) {
       if ((e = launch_gemv<T>(a.x_t, a.W, a.proj_part, a.B, a.E, a.N, stream)) != cudaSuccess)
         return e;
+    } else if (decode_use_proj_tc(a.E, sizeof(T)) && a.e_splits == a.E / kDpK) {
+      if constexpr (sizeof(T) == 2) {
+        if ((e = launch_decode_proj_tc(a.x_t, a.W, a.proj_part, a.B, a.E, a.N, a.dev_err,
+                                       stream)) != cudaSuccess)
+          return e;
+      }
     } else {
       const int e_len = decode_proj_e_len(a.E, a.e_splits);
       dim3 grid((a.N + kPN - 1) / kPN, a.e_splits, (a.B + kPB - 1) / kPB);
