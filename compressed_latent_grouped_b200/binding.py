@@ -91,6 +91,8 @@ def load() -> ctypes.CDLL:
     lib.ccgqa_last_error_string.restype = c_char_p
     lib.ccgqa_set_phase_events.argtypes = [c_void_p, c_int32]
     lib.ccgqa_set_phase_events.restype = None
+    lib.ccgqa_selftest_wait_timeout.argtypes = [ctypes.c_int64, c_void_p, c_void_p]
+    lib.ccgqa_selftest_wait_timeout.restype = c_int
     _lib = lib
     return lib
 
@@ -212,6 +214,13 @@ def ccgqa_last_error_string() -> str:
 
 def ccgqa_launch_count() -> int:
     return int(load().ccgqa_launch_count())
+
+
+def ccgqa_selftest_wait_timeout(limit_cycles: int, dev_err=None, stream=None, check=True) -> int:
+    st = load().ccgqa_selftest_wait_timeout(int(limit_cycles), _ptr(dev_err), _stream(stream))
+    if check and st != 0:
+        raise CCGQAError(st, "ccgqa_selftest_wait_timeout")
+    return st
 
 
 _phase_keep = None

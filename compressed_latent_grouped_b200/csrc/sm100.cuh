@@ -81,16 +81,17 @@ __device__ __forceinline__ bool named_barrier_or(uint32_t id, uint32_t count, bo
 
 // Bounded wait for the phase with the given parity to complete.  Gives up when
 // another thread of the CTA has already given up (*abort != 0) or after
-// kWaitLimitCycles; on a time-out it sets *abort and the caller's error bit.
-// Returns true when the phase completed.
+// `limit` cycles (kWaitLimitCycles, about one second, unless a caller such as
+// the wait self-test asks for less); on a time-out it sets *abort and the
+// caller's error bit.  Returns true when the phase completed.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int32_t* dev_err) {
+                                          int32_t* dev_err, long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       *abort = 1;
       raise_dev_err(dev_err, CCGQA_DEVERR_TIMEOUT);
       return false;

@@ -201,6 +201,18 @@ CCGQA_API uint64_t ccgqa_launch_count(void);
  * turns it off.  Only the pointer is kept; the caller keeps the events alive. */
 CCGQA_API void ccgqa_set_phase_events(void* const* events, int32_t n);
 
+/* Self-test of the device-side failure reporting (no counterpart in the
+ * papers; it exercises the bounded wait every kernel of this library uses).
+ * Launches one small kernel on `stream` whose threads wait on an mbarrier that
+ * nothing ever arrives on; each wait gives up after about `limit_cycles` SM
+ * clock cycles (1 <= limit_cycles <= 2e9), and the kernel then ORs
+ * CCGQA_DEVERR_TIMEOUT into *dev_err (device, nullable) and returns, leaving
+ * the CUDA context usable.  Returns CCGQA_ERR_INVALID_ARG for a limit out of
+ * range, CCGQA_ERR_CUDA if the launch fails, else CCGQA_OK (asynchronous: read
+ * *dev_err after synchronising the stream). */
+CCGQA_API ccgqa_status ccgqa_selftest_wait_timeout(int64_t limit_cycles, int32_t* dev_err,
+                                                   void* stream);
+
 #ifdef __cplusplus
 }
 #endif

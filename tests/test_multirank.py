@@ -56,13 +56,15 @@ def test_rank_helpers_two_ranks_gloo(tmp_path):
         mine = torch.tensor([float(x.double().sum())])
         every = [torch.zeros(1) for _ in range(world)]
         dist.all_gather(every, mine)
-        print(json.dumps({{"rank": rank, "world": world, "local": local, "t": t,
-                          "sums": [float(v) for v in every]}}), flush=True)
+        # one file per rank: the ranks' stdout lines may interleave
+        with open(sys.argv[1] + f"/rank{{rank}}.json", "w") as f:
+            json.dump({{"rank": rank, "world": world, "local": local, "t": t,
+                       "sums": [float(v) for v in every]}}, f)
         dist.destroy_process_group()
     """))
-    r = _torchrun([str(script)])
+    r = _torchrun([str(script), str(tmp_path)])
     assert r.returncode == 0, r.stderr[-2000:]
-    lines = _json_lines(r.stdout)
+    lines = [json.loads((tmp_path / f"rank{k}.json").read_text()) for k in range(2)]
     assert sorted(d["rank"] for d in lines) == [0, 1]
     for d in lines:
         assert d["world"] == 2 and d["local"] == d["rank"]
