@@ -64,7 +64,10 @@ void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int e
   }
   // Splits of whole 128-key chunks.  The CTAs of one launch should fill a whole
   // number of waves of the resident slots (148 SMs x 2 CTAs), each CTA
-  // streaming at least ~1024 keys so its start-up cost stays small.
+  // streaming at least ~1024 keys so its start-up cost stays small, and never
+  // fewer than 4 chunks (512 keys) when the cache has that many: measured on
+  // B200, a launch of a few hundred 2-chunk CTAs spends longer starting them
+  // (about 37 per microsecond) and merging their partials than streaming keys.
   const int64_t bh = static_cast<int64_t>(B) * Hkv;
   const int64_t slots = 148 * 2;
   const int64_t max_sp = (cap + 127) / 128;
@@ -72,6 +75,7 @@ void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int e
   double best = -1.0;
   for (int64_t spc = 1; spc <= max_sp && spc <= 64; ++spc) {
     const int64_t chk = ((cap + spc - 1) / spc + 127) / 128 * 128;
+    if (spc > 1 && chk < 512) break;   // fewer splits only from here on
     const int64_t real_sp = (cap + chk - 1) / chk;
     const int64_t ctas = bh * real_sp;
     const double waves = static_cast<double>(ctas) / slots;
