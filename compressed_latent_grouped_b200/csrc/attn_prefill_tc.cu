@@ -78,23 +78,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, used for part of the probabilities so the exp unit and
-// the FMA pipe share the work.  Cody-Waite style reduction x = n + f with
-// n = round(x) and f in [-0.5, 0.5] (adding 1.5 * 2^23 leaves round(x) in the
-// low mantissa bits), 2^f from a degree-3 polynomial fitted for this kernel
-// (relative error below 8e-5, well under bf16's 2^-9), and 2^n added to the
-// exponent field.  Inputs are clamped at -126 (the exponent field of p,
-// 126 or 127, must stay positive after adding n), so -inf gives ~1e-38.
-__device__ __forceinline__ float soft_exp2(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  float p = fmaf(0.05521968f, f, 0.24260941f);
-  p = fmaf(p, f, 0.69325167f);
-  p = fmaf(p, f, 0.99992800f);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
-
 // Packed fp32 pairs (one instruction for two lanes' worth of FMA-pipe work).
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   uint64_t d;
@@ -112,7 +95,14 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return *reinterpret_cast<float2*>(&d);
 }
 
-// soft_exp2 on a pair, with the FMA-pipe steps packed.
+// 2^x on a pair, on the FMA pipe (packed fp32x2 steps), used for part of the
+// probabilities so the exp unit and the FMA pipe share the work.  Cody-Waite
+// style reduction x = n + f with
+// n = round(x) and f in [-0.5, 0.5] (adding 1.5 * 2^23 leaves round(x) in the
+// low mantissa bits), 2^f from a degree-3 polynomial fitted for this kernel
+// (relative error below 8e-5, well under bf16's 2^-9), and 2^n added to the
+// exponent field.  Inputs are clamped at -126 (the exponent field of p,
+// 126 or 127, must stay positive after adding n), so -inf gives ~1e-38.
 __device__ __forceinline__ float2 soft_exp2x2(float2 x) {
   x.x = fmaxf(x.x, -126.0f);
   x.y = fmaxf(x.y, -126.0f);
