@@ -286,12 +286,6 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool b_mn_m
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// Byte offset of the 16-byte chunk `chunk` of row `row` inside a 128-byte-row
-// tile written with the 128B swizzle (the layout TMA SWIZZLE_128B produces).
-__device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
-  return row * 128u + ((chunk ^ (row & 7u)) << 4);
-}
-
 // Byte offset of element (row, col) in a K-major tile whose rows are `row_bytes`
 // wide (64 or 128), with the matching TMA / UMMA swizzle (64B: address bits
 // [4,6) ^= bits [7,9); 128B: bits [4,7) ^= bits [7,10)).  The tile must start
@@ -299,16 +293,6 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
 __device__ __forceinline__ uint32_t swz_offset(uint32_t row, uint32_t col_byte, uint32_t row_bytes) {
   const uint32_t off = row * row_bytes + col_byte;
   return row_bytes == 128 ? (off ^ (((off >> 7) & 7u) << 4)) : (off ^ (((off >> 7) & 3u) << 4));
-}
-
-__device__ __forceinline__ uint32_t elect_one_lane() {
-  uint32_t pred = 0;
-  asm volatile(
-      "{\n\t.reg .pred P;\n\t"
-      "elect.sync _|P, 0xffffffff;\n\t"
-      "selp.u32 %0, 1, 0, P;\n\t}"
-      : "=r"(pred));
-  return pred;
 }
 
 }  // namespace sm100
