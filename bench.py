@@ -333,7 +333,7 @@ def run_workload_only(args, local):
 def run_ours(args, world, rank, local):
     import torch
     from compressed_latent_grouped_b200 import binding as B
-    from compressed_latent_grouped_b200.device import DeviceLayer
+    from compressed_latent_grouped_b200.device import DeviceLayer, Graph
     from compressed_latent_grouped_b200.workloads import WORKLOADS, make_inputs
     import oracle.ccgqa as O
 
@@ -349,7 +349,10 @@ def run_ours(args, world, rank, local):
     out = torch.empty(w.B, w.S, w.Hq * w.d, dtype=w.torch_dtype, device=dev)
     out_t = torch.empty(w.B, w.Hq * w.d, dtype=w.torch_dtype, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
+    # a created stream (graphs cannot record the legacy default stream), made
+    # current so the flush and the events go on it too
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(stream)
 
     def step():
         lay.prefill(x, out)
@@ -366,27 +369,52 @@ def run_ours(args, world, rank, local):
     st_ev = [(mk(), mk()) for _ in range(K)]
     pf_ev = [[mk() for _ in range(4)] for _ in range(K)]
     dc_ev = [[mk() for _ in range(4)] for _ in range(K)]
+    for e_ in [e_ for l_ in pf_ev + dc_ev for e_ in l_]:
+        e_.record(stream)          # create the CUDA events outside the timed passes
     sampler = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize()
-    n0 = B.ccgqa_launch_count()
+    # the step recorded once as a CUDA graph of library calls (ccgqa_graph_*):
+    # each timed step is one graph launch, the serving loop's form
+    graph = Graph(step, stream)
+    for _ in range(3):
+        graph.launch()
+    torch.cuda.synchronize()
+    eager_ev = [(mk(), mk()) for _ in range(K)]
     with sampler:
+        # pass 1, the step time: events only around whole steps.  An event
+        # recorded between two kernels serialises them (about 3 us a record on
+        # B200), so the per-kernel events live in pass 3.
+        n0 = B.ccgqa_launch_count()
         for i in range(K):
             flush.zero_()
             st_ev[i][0].record(stream)
+            graph.launch()
+            st_ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        launches = B.ccgqa_launch_count() - n0
+        # pass 2, the same K steps as eager library calls (no graph)
+        for i in range(K):
+            flush.zero_()
+            eager_ev[i][0].record(stream)
+            step()
+            eager_ev[i][1].record(stream)
+        # pass 3, the same K steps with events between the kernels (phase times)
+        for i in range(K):
+            flush.zero_()
             B.ccgqa_set_phase_events(pf_ev[i])
             lay.prefill(x, out)
             B.ccgqa_set_phase_events(dc_ev[i])
             lay.decode_step(x_t, out_t)
             B.ccgqa_set_phase_events(None)
-            st_ev[i][1].record(stream)
         torch.cuda.synchronize()
-    launches = B.ccgqa_launch_count() - n0
     barrier(world)
     if lay.error_bits():
         raise RuntimeError(f"device error bits {lay.error_bits()}")
     step_ms = [a.elapsed_time(b) for a, b in st_ev]
     t_ms = max_over_ranks(sum(step_ms), world, dev)
+    eager_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eager_ev), world, dev) / K
+    graph.close()
     phase = lambda evs, i, j: sum(e[i].elapsed_time(e[j]) for e in evs) / K  # noqa: E731
     proj_ms, pre_ms, attn_ms = phase(pf_ev, 0, 1), phase(pf_ev, 1, 2), phase(pf_ev, 2, 3)
     dproj_ms, dpre_ms, dattn_ms = phase(dc_ev, 0, 1), phase(dc_ev, 1, 2), phase(dc_ev, 2, 3)
@@ -435,8 +463,7 @@ def run_ours(args, world, rank, local):
             in_ready[k].record(s_in)
             s_cmp.wait_event(in_ready[k])
             s_cmp.wait_event(out_free[k])
-            lay.prefill(x_d[k], o_d[k], stream=s_cmp)
-            lay.decode_step(xt_d[k], ot_d[k], stream=s_cmp)
+            graphs[k].launch()
             in_free[k].record(s_cmp)
             out_ready[k].record(s_cmp)
             s_out.wait_event(out_ready[k])
@@ -445,6 +472,9 @@ def run_ours(args, world, rank, local):
                 outt_h.copy_(ot_d[k], non_blocking=True)
             out_free[k].record(s_out)
 
+    graphs = [Graph(lambda k=k: (lay.prefill(x_d[k], o_d[k], stream=s_cmp),
+                                 lay.decode_step(xt_d[k], ot_d[k], stream=s_cmp)), s_cmp)
+              for k in range(2)]
     e2e_steps(2)
     torch.cuda.synchronize()
     barrier(world)
@@ -455,6 +485,8 @@ def run_ours(args, world, rank, local):
     e1.record(s_out)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    for g_ in graphs:
+        g_.close()
     barrier(world)
     if lay.error_bits():
         raise RuntimeError(f"device error bits {lay.error_bits()}")
@@ -487,18 +519,23 @@ def run_ours(args, world, rank, local):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": max(args.warmup, 3), "ms_per_step": t_ms / K,
+        "eager_ms_per_step": eager_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded PCG64 normals, weights N(0, 1/fan_in))",
         "config": {"workload": f"{WORKLOAD} prefill + 1 decode step", "B": w.B, "S": w.S,
                    "E": w.E, "C": w.C, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
                    "conv_width": w.conv_width, "rope_base": w.rope_base,
                    "parallelism": f"replicas x{world} (independent sequences per GPU)",
-                   "l2": "flushed (256 MiB write) before every timed step"},
+                   "l2": "flushed (256 MiB write) before every timed step",
+                   "launch": "each step one CUDA graph launch of the recorded library calls "
+                             "(ccgqa_graph_launch); eager_ms_per_step: the same calls made "
+                             "one by one"},
         "roofline": {"bound": "tensor", "kernel": "attn_prefill_tc", "achieved": achieved,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
                      "peak_kind": f"{peak_kind} bf16 dense burst",
-                     "flop_per_launch": attn_flop, "ms_per_launch": attn_ms},
+                     "flop_per_launch": attn_flop, "ms_per_launch": attn_ms,
+                     "timing": "CUDA events around each launch, second pass of the K steps"},
         "roofline_exp": exp_roofline(w, attn_ms, peaks),
         "kernels": {
             "proj_gemm": {"ms": proj_ms, "tflops": proj_flop / (proj_ms / 1e3) / 1e12,

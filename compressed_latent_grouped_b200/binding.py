@@ -93,6 +93,16 @@ def load() -> ctypes.CDLL:
     lib.ccgqa_set_phase_events.restype = None
     lib.ccgqa_selftest_wait_timeout.argtypes = [ctypes.c_int64, c_void_p, c_void_p]
     lib.ccgqa_selftest_wait_timeout.restype = c_int
+    lib.ccgqa_graph_begin.argtypes = [c_void_p]
+    lib.ccgqa_graph_begin.restype = c_int
+    lib.ccgqa_graph_end.argtypes = [c_void_p, POINTER(c_void_p)]
+    lib.ccgqa_graph_end.restype = c_int
+    lib.ccgqa_graph_launch.argtypes = [c_void_p, c_void_p]
+    lib.ccgqa_graph_launch.restype = c_int
+    lib.ccgqa_graph_kernel_count.argtypes = [c_void_p]
+    lib.ccgqa_graph_kernel_count.restype = ctypes.c_int64
+    lib.ccgqa_graph_destroy.argtypes = [c_void_p]
+    lib.ccgqa_graph_destroy.restype = c_int
     _lib = lib
     return lib
 
@@ -221,6 +231,39 @@ def ccgqa_selftest_wait_timeout(limit_cycles: int, dev_err=None, stream=None, ch
     if check and st != 0:
         raise CCGQAError(st, "ccgqa_selftest_wait_timeout")
     return st
+
+
+def ccgqa_graph_begin(stream=None, check=True) -> int:
+    st = load().ccgqa_graph_begin(_stream(stream))
+    if check and st != 0:
+        raise CCGQAError(st, "ccgqa_graph_begin")
+    return st
+
+
+def ccgqa_graph_end(stream=None) -> int:
+    """Stop recording on `stream`; returns the graph handle (an integer)."""
+    h = c_void_p()
+    st = load().ccgqa_graph_end(_stream(stream), ctypes.byref(h))
+    if st != 0:
+        raise CCGQAError(st, "ccgqa_graph_end")
+    return h.value
+
+
+def ccgqa_graph_launch(graph: int, stream=None, check=True) -> int:
+    st = load().ccgqa_graph_launch(c_void_p(graph), _stream(stream))
+    if check and st != 0:
+        raise CCGQAError(st, "ccgqa_graph_launch")
+    return st
+
+
+def ccgqa_graph_kernel_count(graph) -> int:
+    return int(load().ccgqa_graph_kernel_count(c_void_p(graph)))
+
+
+def ccgqa_graph_destroy(graph) -> None:
+    st = load().ccgqa_graph_destroy(c_void_p(graph))
+    if st != 0:
+        raise CCGQAError(st, "ccgqa_graph_destroy")
 
 
 _phase_keep = None

@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <map>
 #include <mutex>
+#include <new>
 #include <utility>
 
 #include "kernels.h"
@@ -13,7 +14,25 @@
 namespace ccgqa {
 
 static std::atomic<uint64_t> g_launches{0};
-void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+
+// Graph capture of the calling thread (ccgqa_graph_begin .. ccgqa_graph_end):
+// the stream being captured and the library kernels recorded so far.  Kernels
+// recorded into a graph count when a launch of the graph runs them.
+struct Capture {
+  cudaStream_t stream = nullptr;
+  int64_t kernels = 0;
+  bool active = false;
+};
+static thread_local Capture t_capture;
+
+void count_launches(int n) {
+  if (t_capture.active)
+    t_capture.kernels += n;
+  else
+    g_launches.fetch_add(static_cast<uint64_t>(n));
+}
+// While this thread captures, every launching call must use the captured stream.
+bool stream_allowed(cudaStream_t st) { return !t_capture.active || st == t_capture.stream; }
 
 cudaError_t allow_smem(const void* func, int bytes) {
   static std::mutex mu;
@@ -39,7 +58,8 @@ static ccgqa_status cuda_fail(cudaError_t e) {
 // Optional phase events of the calling thread (ccgqa_set_phase_events).
 static thread_local void* const* t_phase_events = nullptr;
 static void phase_mark(int i, cudaStream_t st) {
-  if (t_phase_events) cudaEventRecord(static_cast<cudaEvent_t>(t_phase_events[i]), st);
+  if (t_phase_events && !t_capture.active)
+    cudaEventRecord(static_cast<cudaEvent_t>(t_phase_events[i]), st);
 }
 
 namespace {
@@ -286,7 +306,7 @@ ccgqa_status run_decode(const Geo& g, const ccgqa_weights* w, const void* x_t,
   a.splits = L.splits;
   a.chunk = L.chunk;
   a.dev_err = dev_err;
-  a.phase_events = t_phase_events;
+  a.phase_events = t_capture.active ? nullptr : t_phase_events;
   const cudaError_t e = launch_decode_step<T>(a, st);
   return e == cudaSuccess ? CCGQA_OK : cuda_fail(e);
 }
@@ -363,6 +383,7 @@ CCGQA_API ccgqa_status ccgqa_prefill(const ccgqa_config* cfg, const ccgqa_weight
       workspace_bytes < prefill_ws(g, batch, seq_len).total)
     return CCGQA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!stream_allowed(st)) return CCGQA_ERR_INVALID_ARG;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   if (g.dtype == CCGQA_BF16)
     return run_prefill<bf16>(g, w, x, batch, seq_len, out, cache, ws, dev_err, st);
@@ -383,6 +404,7 @@ CCGQA_API ccgqa_status ccgqa_decode_step(const ccgqa_config* cfg, const ccgqa_we
       workspace_bytes < decode_ws(g, cache->batch, cache->cap, w->W_qkv != nullptr).total)
     return CCGQA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!stream_allowed(st)) return CCGQA_ERR_INVALID_ARG;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   if (g.dtype == CCGQA_BF16) return run_decode<bf16>(g, w, x_t, cache, out, ws, dev_err, st);
   return run_decode<float>(g, w, x_t, cache, out, ws, dev_err, st);
@@ -400,6 +422,7 @@ CCGQA_API ccgqa_status ccgqa_decode_step_noalloc(const ccgqa_config* cfg,
   if (!x_t || !out || !aligned16(x_t) || !aligned16(out)) return CCGQA_ERR_INVALID_ARG;
   const DecodeWs L = decode_ws(g, cache->batch, cache->cap, w->W_qkv != nullptr);
   if (L.total > kNoAllocScratchBytes) return CCGQA_ERR_WORKSPACE;
+  if (!stream_allowed(static_cast<cudaStream_t>(stream))) return CCGQA_ERR_INVALID_ARG;
   void* scratch = nullptr;
   cudaError_t e = noalloc_scratch(&scratch);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -429,6 +452,7 @@ CCGQA_API ccgqa_status ccgqa_kvcache_append(const ccgqa_config* cfg, const ccgqa
   if (n_new == 0) return CCGQA_OK;
   if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return CCGQA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!stream_allowed(st)) return CCGQA_ERR_INVALID_ARG;
   cudaError_t e;
   if (g.dtype == CCGQA_BF16)
     e = launch_kv_append<bf16>(static_cast<bf16*>(cache->k), static_cast<bf16*>(cache->v),
@@ -461,6 +485,88 @@ CCGQA_API const char* ccgqa_last_error_string(void) { return t_last_error; }
 
 CCGQA_API void ccgqa_set_phase_events(void* const* events, int32_t n) {
   t_phase_events = (events != nullptr && n >= 4) ? events : nullptr;
+}
+
+// ----------------------------------------------------------------------------
+// CUDA graphs of library calls: the calls a thread makes on one stream between
+// ccgqa_graph_begin and ccgqa_graph_end are recorded (not run) and become one
+// executable graph, replayed with all its arguments fixed.
+}  // extern "C"
+
+struct ccgqa_graph {
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  int64_t kernels = 0;     // library kernels one launch runs
+};
+
+extern "C" {
+
+CCGQA_API ccgqa_status ccgqa_graph_begin(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the legacy default stream cannot be captured
+  if (st == nullptr || st == cudaStreamLegacy || st == cudaStreamPerThread)
+    return CCGQA_ERR_INVALID_ARG;
+  if (t_capture.active) return CCGQA_ERR_INVALID_ARG;
+  const cudaError_t e = cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal);
+  if (e != cudaSuccess) return cuda_fail(e);
+  t_capture.stream = st;
+  t_capture.kernels = 0;
+  t_capture.active = true;
+  return CCGQA_OK;
+}
+
+CCGQA_API ccgqa_status ccgqa_graph_end(void* stream, ccgqa_graph** graph) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (graph == nullptr || !t_capture.active || st != t_capture.stream)
+    return CCGQA_ERR_INVALID_ARG;
+  *graph = nullptr;
+  t_capture.active = false;
+  cudaGraph_t g = nullptr;
+  cudaError_t e = cudaStreamEndCapture(st, &g);
+  if (e != cudaSuccess) {
+    if (g) cudaGraphDestroy(g);
+    return cuda_fail(e);
+  }
+  cudaGraphExec_t exec = nullptr;
+  e = cudaGraphInstantiate(&exec, g, 0);
+  if (e != cudaSuccess) {
+    cudaGraphDestroy(g);
+    return cuda_fail(e);
+  }
+  ccgqa_graph* h = new (std::nothrow) ccgqa_graph;
+  if (h == nullptr) {
+    cudaGraphExecDestroy(exec);
+    cudaGraphDestroy(g);
+    return CCGQA_ERR_WORKSPACE;
+  }
+  h->graph = g;
+  h->exec = exec;
+  h->kernels = t_capture.kernels;
+  *graph = h;
+  return CCGQA_OK;
+}
+
+CCGQA_API ccgqa_status ccgqa_graph_launch(const ccgqa_graph* graph, void* stream) {
+  if (graph == nullptr) return CCGQA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!stream_allowed(st)) return CCGQA_ERR_INVALID_ARG;
+  const cudaError_t e = cudaGraphLaunch(graph->exec, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  count_launches(static_cast<int>(graph->kernels));
+  return CCGQA_OK;
+}
+
+CCGQA_API int64_t ccgqa_graph_kernel_count(const ccgqa_graph* graph) {
+  return graph == nullptr ? -1 : graph->kernels;
+}
+
+CCGQA_API ccgqa_status ccgqa_graph_destroy(ccgqa_graph* graph) {
+  if (graph == nullptr) return CCGQA_OK;
+  cudaError_t e = cudaGraphExecDestroy(graph->exec);
+  const cudaError_t e2 = cudaGraphDestroy(graph->graph);
+  delete graph;
+  if (e == cudaSuccess) e = e2;
+  return e == cudaSuccess ? CCGQA_OK : cuda_fail(e);
 }
 
 }  // extern "C"

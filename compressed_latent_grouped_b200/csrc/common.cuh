@@ -27,8 +27,11 @@ __device__ __forceinline__ void raise_dev_err(int32_t* dev_err, int32_t bit) {
 // second at the B200's clock).  A healthy wait ends in microseconds.
 constexpr long long kWaitLimitCycles = 2000000000LL;
 
-// Host-side launch accounting (ccgqa_launch_count).
+// Host-side launch accounting (ccgqa_launch_count); while the calling thread
+// records a graph the kernels count towards the graph instead.
 void count_launches(int n);
+// False while the calling thread records a graph on a stream other than st.
+bool stream_allowed(cudaStream_t st);
 
 // cudaFuncSetAttribute(func, MaxDynamicSharedMemorySize, bytes) on the current
 // device, skipped when an earlier call already allowed at least `bytes`

@@ -31,6 +31,7 @@ __global__ void wait_timeout_kernel(int32_t* dev_err, long long limit) {
 extern "C" __attribute__((visibility("default"))) ccgqa_status ccgqa_selftest_wait_timeout(
     int64_t limit_cycles, int32_t* dev_err, void* stream) {
   if (limit_cycles < 1 || limit_cycles > ccgqa::kWaitLimitCycles) return CCGQA_ERR_INVALID_ARG;
+  if (!ccgqa::stream_allowed(static_cast<cudaStream_t>(stream))) return CCGQA_ERR_INVALID_ARG;
   ccgqa::wait_timeout_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(
       dev_err, static_cast<long long>(limit_cycles));
   ccgqa::count_launches(1);

@@ -103,3 +103,34 @@ class DeviceLayer:
 
     def error_bits(self) -> int:
         return int(self.dev_err.item())
+
+
+class Graph:
+    """Library calls recorded once into a CUDA graph (ccgqa_graph_*) and
+    launched again with the same arguments: ``Graph(fn, stream)`` records what
+    ``fn()`` enqueues on ``stream`` (a created torch stream, not the default
+    stream); ``launch()`` replays it on that stream; ``close()`` frees it."""
+
+    def __init__(self, fn, stream):
+        self.stream = stream
+        self.handle = None
+        B.ccgqa_graph_begin(stream)
+        try:
+            with torch.cuda.stream(stream):
+                fn()
+        except BaseException:
+            try:
+                B.ccgqa_graph_destroy(B.ccgqa_graph_end(stream))
+            except B.CCGQAError:
+                pass
+            raise
+        self.handle = B.ccgqa_graph_end(stream)
+        self.kernels = B.ccgqa_graph_kernel_count(self.handle)
+
+    def launch(self):
+        B.ccgqa_graph_launch(self.handle, self.stream)
+
+    def close(self):
+        if self.handle is not None:
+            B.ccgqa_graph_destroy(self.handle)
+            self.handle = None

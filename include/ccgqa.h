@@ -213,6 +213,45 @@ CCGQA_API void ccgqa_set_phase_events(void* const* events, int32_t n);
 CCGQA_API ccgqa_status ccgqa_selftest_wait_timeout(int64_t limit_cycles, int32_t* dev_err,
                                                    void* stream);
 
+/* CUDA graphs of library calls (no counterpart in the papers: a launch-cost
+ * device for fixed-shape serving loops, where one graph launch replaces the
+ * per-kernel launches of a prefill and a decode step).
+ *
+ * ccgqa_graph_begin starts recording on `stream` (a created stream: NULL, the
+ * legacy and the per-thread default streams return CCGQA_ERR_INVALID_ARG) in
+ * thread-local capture mode.  Until ccgqa_graph_end, the calling thread's
+ * ccgqa_prefill / ccgqa_decode_step / ccgqa_decode_step_noalloc /
+ * ccgqa_kvcache_append / ccgqa_selftest_wait_timeout calls validate their
+ * arguments as usual but only RECORD their kernels, which do not run; a call
+ * that names another stream returns CCGQA_ERR_INVALID_ARG, and phase events
+ * (ccgqa_set_phase_events) are not recorded.  Other work the caller puts on the
+ * stream meanwhile (copies, its own kernels) is recorded too.  A second begin
+ * on the same thread before end returns CCGQA_ERR_INVALID_ARG.
+ *
+ * ccgqa_graph_end(stream, &graph) stops recording and instantiates the graph;
+ * *graph receives a handle the caller owns (free it with ccgqa_graph_destroy).
+ * Errors: CCGQA_ERR_INVALID_ARG if this thread is not recording on `stream` or
+ * graph is NULL; CCGQA_ERR_CUDA if the capture was invalidated or
+ * instantiation failed (*graph = NULL, recording has stopped either way).
+ *
+ * ccgqa_graph_launch(graph, stream) runs the recorded work once on `stream`
+ * (any stream of the graph's device), with every pointer and size exactly as
+ * recorded: to run on new inputs, write them into the recorded buffers
+ * first.  The device error word and the cache are updated as by the recorded
+ * calls.  Launch order on a stream is the only ordering; two launches of one
+ * graph must not overlap in time.  Each launch adds the graph's kernel count to
+ * ccgqa_launch_count (recording adds nothing).
+ *
+ * ccgqa_graph_kernel_count: library kernels one launch runs (-1 for NULL).
+ * ccgqa_graph_destroy: frees the graph (NULL is a no-op); the caller makes sure
+ * no launch of it is still running. */
+typedef struct ccgqa_graph ccgqa_graph;
+CCGQA_API ccgqa_status ccgqa_graph_begin(void* stream);
+CCGQA_API ccgqa_status ccgqa_graph_end(void* stream, ccgqa_graph** graph);
+CCGQA_API ccgqa_status ccgqa_graph_launch(const ccgqa_graph* graph, void* stream);
+CCGQA_API int64_t ccgqa_graph_kernel_count(const ccgqa_graph* graph);
+CCGQA_API ccgqa_status ccgqa_graph_destroy(ccgqa_graph* graph);
+
 #ifdef __cplusplus
 }
 #endif

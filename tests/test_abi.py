@@ -158,3 +158,16 @@ def test_capacity_checked_on_host(lib):
 
 def test_launch_count_starts_at_zero(lib):
     assert B.ccgqa_launch_count() == 0
+
+
+def test_graph_calls_checked_on_host(lib):
+    # the legacy default stream cannot be recorded; end/launch need a recording
+    # or a graph; no CUDA call is reached by any of these
+    assert lib.ccgqa_graph_begin(None) == 1
+    h = ctypes.c_void_p()
+    assert lib.ccgqa_graph_end(None, ctypes.byref(h)) == 1
+    assert lib.ccgqa_graph_end(ctypes.c_void_p(4096), None) == 1
+    assert lib.ccgqa_graph_launch(None, None) == 1
+    assert lib.ccgqa_graph_kernel_count(None) == -1
+    assert lib.ccgqa_graph_destroy(None) == 0
+    assert B.ccgqa_launch_count() == 0
