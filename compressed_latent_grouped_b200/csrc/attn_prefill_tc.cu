@@ -134,6 +134,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
                            const __grid_constant__ CUtensorMap tmV, bf16* __restrict__ out,
                            int B, int S, int Hq, int Hkv, int G_log2, int n_groups, int causal,
                            int32_t* dev_err) {
+  pdl_enter();
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -487,11 +488,11 @@ cudaError_t launch_d(const AttnArgs& a, cudaStream_t stream) {
   cudaError_t e = allow_smem(reinterpret_cast<const void*>(attn_prefill_tc_kernel<D>),
                                        static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
-  attn_prefill_tc_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(
-      tmQ, tmK, tmV, static_cast<bf16*>(a.out), a.B, a.S, a.Hq, a.Hkv, G_log2, n_groups,
-      a.causal, a.dev_err);
+  const cudaError_t el = launch_pdl(attn_prefill_tc_kernel<D>, dim3(grid), dim3(C::kThreads),
+                                    C::kSmem, stream, tmQ, tmK, tmV, static_cast<bf16*>(a.out),
+                                    a.B, a.S, a.Hq, a.Hkv, G_log2, n_groups, a.causal, a.dev_err);
   count_launches(1);
-  return cudaGetLastError();
+  return el != cudaSuccess ? el : cudaGetLastError();
 }
 
 }  // namespace

@@ -38,4 +38,38 @@ bool stream_allowed(cudaStream_t st);
 // (the attribute is per device, the check costs a lock and a map lookup).
 cudaError_t allow_smem(const void* func, int bytes);
 
+// Programmatic dependent launch.  A kernel launched by launch_pdl may be
+// scheduled while the kernel before it on the stream is still finishing (once
+// every CTA of that kernel has run pdl_trigger() or exited).  Every such kernel
+// runs pdl_wait() in all its threads as its first statement: the wait returns
+// when the previous kernel has completed and its memory writes are visible, so
+// nothing (global memory, TMEM) is touched before it.  The overlap gained is
+// the launch and CTA scheduling of this kernel during the previous one's tail.
+// Kernels launched without the attribute see pdl_wait() return at once.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Both in one call: the first statement of every kernel launched by launch_pdl.
+__device__ __forceinline__ void pdl_enter() {
+  pdl_wait();
+  pdl_trigger();
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 }  // namespace ccgqa

@@ -235,6 +235,7 @@ template <typename T, int BB>
 __global__ void __launch_bounds__(256)
     decode_gemv_kernel(const T* __restrict__ x, const T* __restrict__ W, float* __restrict__ out,
                        int B, int E, int N) {
+  pdl_enter();
   constexpr int VEC = 16 / sizeof(T);
   extern __shared__ float4 gv_f4[];
   T* xs = reinterpret_cast<T*>(gv_f4);             // [B][E]
@@ -307,8 +308,7 @@ cudaError_t launch_gemv(const T* x, const T* W, float* out, int B, int E, int N,
       cudaError_t e = allow_smem(reinterpret_cast<const void*>(kernel), static_cast<int>(xb));
       if (e != cudaSuccess) return e;
     }
-    kernel<<<blocks, 256, xb, stream>>>(x, W, out, B, E, N);
-    return cudaSuccess;
+    return launch_pdl(kernel, dim3(blocks), dim3(256), xb, stream, x, W, out, B, E, N);
   };
   if (B <= 1) return go(decode_gemv_kernel<T, 1>);
   if (B <= 2) return go(decode_gemv_kernel<T, 2>);
@@ -329,6 +329,7 @@ __global__ void __launch_bounds__(128)
     decode_proj_tc_kernel(const __grid_constant__ CUtensorMap tmW,
                           const __grid_constant__ CUtensorMap tmX, float* __restrict__ part, int B,
                           int N, int32_t* dev_err) {
+  pdl_enter();
   extern __shared__ uint8_t dp_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dp_raw) + 1023) & ~uintptr_t(1023));
@@ -430,8 +431,8 @@ cudaError_t launch_decode_proj_tc(const bf16* x, const bf16* W, float* part, int
                              static_cast<int>(kDpSmem));
   if (e != cudaSuccess) return e;
   dim3 grid((N + kDpN - 1) / kDpN, E / kDpK, (B + kDpB - 1) / kDpB);
-  decode_proj_tc_kernel<<<grid, 128, kDpSmem, stream>>>(tmW, tmX, part, B, N, dev_err);
-  return cudaSuccess;
+  return launch_pdl(decode_proj_tc_kernel, grid, dim3(128), kDpSmem, stream, tmW, tmX, part, B,
+                    N, dev_err);
 }
 
 // ----------------------------------------------------------------- pre-step
@@ -483,6 +484,7 @@ constexpr int kPreThreads = 256;
 template <typename T>
 __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_constant__ DecodeArgs<T> a,
                                                          int stage_wt) {
+  pdl_enter();
   extern __shared__ float4 dsm_f4[];
   uint8_t* sm = reinterpret_cast<uint8_t*>(dsm_f4);
   const int g = blockIdx.x, b = blockIdx.y;
@@ -959,9 +961,10 @@ cudaError_t launch_decode_step(const DecodeArgs<T>& a, cudaStream_t stream) {
                                static_cast<int>(smem));
       if (e != cudaSuccess) return e;
     }
-    decode_pre_kernel<T><<<dim3(a.Hkv, a.B), kPreThreads, smem, stream>>>(a, stage_wt);
+    e = launch_pdl(decode_pre_kernel<T>, dim3(a.Hkv, a.B), dim3(kPreThreads), smem, stream, a,
+                   stage_wt);
     count_launches(1);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (e != cudaSuccess || (e = cudaGetLastError()) != cudaSuccess) return e;
   }
   mark(2);
   if constexpr (sizeof(T) == 2) {

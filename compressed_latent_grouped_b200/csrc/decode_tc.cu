@@ -76,6 +76,7 @@ template <int D>
 __global__ void __launch_bounds__(kDecTcThreads, 1)
     decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const DecodeArgs<bf16> a) {
+  pdl_enter();
   using C = DCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -585,9 +586,10 @@ cudaError_t launch_tc(const DecodeArgs<bf16>& a, cudaStream_t stream) {
                                        static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
   dim3 grid(a.splits, a.Hkv, a.B);
-  decode_attn_tc_kernel<D><<<grid, kDecTcThreads, C::kSmem, stream>>>(tmK, tmV, a);
+  const cudaError_t el = launch_pdl(decode_attn_tc_kernel<D>, grid, dim3(kDecTcThreads),
+                                    C::kSmem, stream, tmK, tmV, a);
   count_launches(1);
-  return cudaGetLastError();
+  return el != cudaSuccess ? el : cudaGetLastError();
 }
 
 }  // namespace

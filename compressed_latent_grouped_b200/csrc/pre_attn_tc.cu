@@ -118,6 +118,7 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 template <int D>
 __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
     pre_attn_tc_kernel(const __grid_constant__ PreAttnArgs<bf16> a) {
+  pdl_enter();
   constexpr uint32_t kRowBytes = D * 2;                 // 64: 64B swizzle, 128: 128B swizzle
   constexpr uint32_t kSwz = (D == 32) ? kSwizzle64B : kSwizzle128B;
   constexpr uint32_t kSbo = 8 * kRowBytes;
@@ -465,9 +466,10 @@ cudaError_t launch_d(const PreAttnArgs<bf16>& a, cudaStream_t stream) {
                                        static_cast<int>(L.bytes));
   if (e != cudaSuccess) return e;
   dim3 grid((a.S + kPtTT - 1) / kPtTT, a.Hkv, a.B);
-  pre_attn_tc_kernel<D><<<grid, kPtThreads, L.bytes, stream>>>(a);
+  const cudaError_t el =
+      launch_pdl(pre_attn_tc_kernel<D>, grid, dim3(kPtThreads), L.bytes, stream, a);
   count_launches(1);
-  return cudaGetLastError();
+  return el != cudaSuccess ? el : cudaGetLastError();
 }
 
 }  // namespace

@@ -34,6 +34,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     proj_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
                           const __grid_constant__ CUtensorMap tmB, bf16* __restrict__ C, int M,
                           int N, int K, int32_t* dev_err) {
+  pdl_enter();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -255,10 +256,10 @@ cudaError_t launch_proj_gemm_bf16(const bf16* A, const bf16* W, bf16* C, int M, 
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int tiles = ((N + kBN - 1) / kBN) * ((M + kBM - 1) / kBM);
   const int grid = tiles < sms ? tiles : sms;   // one persistent CTA per SM
-  proj_gemm_bf16_kernel<<<grid, kGemmThreads, kGemmSmem, stream>>>(tmA, tmB, C, M, N, K,
-                                                                    dev_err);
+  const cudaError_t el = launch_pdl(proj_gemm_bf16_kernel, dim3(grid), dim3(kGemmThreads),
+                                    kGemmSmem, stream, tmA, tmB, C, M, N, K, dev_err);
   count_launches(1);
-  return cudaGetLastError();
+  return el != cudaSuccess ? el : cudaGetLastError();
 }
 
 cudaError_t launch_proj_gemm_f32(const float* A, const float* W, float* C, int M, int N, int K,
