@@ -61,7 +61,7 @@ __host__ __device__ inline PtLayout pt_layout(int d, int G) {
   L.off_w = 2 * L.u_bytes > tr_bytes ? 2 * L.u_bytes : tr_bytes;   // W_h, h = 0..G
   L.off_z = L.off_w + (G + 1) * L.w_bytes;          // [131][ZC] bf16
   L.off_ws = L.off_z + ((static_cast<uint32_t>(kPtTT + kPtHalo) * L.ZC * 2 + 15u) & ~15u);
-  L.off_bar = L.off_ws + static_cast<uint32_t>(G + 1) * d * 16;     // [(G+1) d][4] float
+  L.off_bar = L.off_ws + static_cast<uint32_t>(G + 1) * d * 8;      // [(G+1) d][4] bf16
   L.bytes = L.off_bar + 64 + 1024;                  // barriers + alignment slack
   return L;
 }
@@ -90,24 +90,26 @@ __device__ __forceinline__ void cp_async_wait_pending(int n) {
   }
 }
 
-__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 p = __bfloat1622float2(h[i]);
-    f[2 * i] = p.x;
-    f[2 * i + 1] = p.y;
-  }
+// d = a * b + c for bf16 a, b and fp32 c, d in one instruction: the product
+// of two bf16 values is exact in fp32, so this equals fmaf(float(a), float(b), c)
+// and needs no conversion of a and b.
+__device__ __forceinline__ float fma_bf16(uint16_t a, uint16_t b, float c) {
+  float d;
+  asm("fma.rn.f32.bf16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(c));
+  return d;
 }
-// d = a * b + c on a pair (one packed fp32x2 instruction), rounded like fmaf
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;"
-      : "=l"(d)
-      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)),
-        "l"(*reinterpret_cast<const uint64_t*>(&c)));
-  return *reinterpret_cast<float2*>(&d);
+// d = a + c for bf16 a and fp32 c, d
+__device__ __forceinline__ float add_bf16(uint16_t a, float c) {
+  float d;
+  asm("add.rn.f32.bf16 %0, %1, %2;" : "=f"(d) : "h"(a), "f"(c));
+  return d;
 }
+// the two bf16 halves of a 32-bit word (low half = lower channel)
+__device__ __forceinline__ void halves(uint32_t v, uint16_t& lo, uint16_t& hi) {
+  asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(v));
+}
+constexpr uint16_t kBf16MinusOne = 0xBF80, kBf16Half = 0x3F00;
+
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -133,7 +135,7 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
   const int b = blockIdx.z, g = blockIdx.y, t0 = blockIdx.x * kPtTT;
   const int tid = threadIdx.x, warp = tid >> 5;
   bf16* z = reinterpret_cast<bf16*>(smem + L.off_z);
-  float* ws = reinterpret_cast<float*>(smem + L.off_ws);
+  uint2* ws = reinterpret_cast<uint2*>(smem + L.off_ws);   // taps of a channel: 4 bf16
   bf16* tr = reinterpret_cast<bf16*>(smem + L.off_u);   // raw taps, until the first conv
   uint64_t* mma_done = reinterpret_cast<uint64_t*>(smem + L.off_bar);   // [2]
   uint64_t* drain = mma_done + 2;
@@ -237,12 +239,16 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // conv taps as fp32 [channel][4], zero past K
-  for (int idx = tid; idx < NH * D * 4; idx += kPtThreads) {
-    const int hc = idx >> 2, k = idx & 3;
-    ws[idx] = k < K ? __bfloat162float(tr[hc * K + k]) : 0.f;
+  // conv taps as bf16 [channel][4], zero past K
+  for (int hc = tid; hc < NH * D; hc += kPtThreads) {
+    uint16_t w4[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      w4[k] = k < K ? __bfloat16_as_ushort(tr[hc * K + k]) : static_cast<uint16_t>(0);
+    ws[hc] = make_uint2(w4[0] | (static_cast<uint32_t>(w4[1]) << 16),
+                        w4[2] | (static_cast<uint32_t>(w4[3]) << 16));
   }
-  __syncthreads();   // fp32 taps ready
+  __syncthreads();   // padded taps ready
 
   // 2. per head
   const int r = tid & (kPtTT - 1);         // position row == TMEM lane
@@ -256,44 +262,54 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
   const int t = t0 + r;
   bool ok = true;
 
-  // conv of head hh for chunks j = P, P + 2, ... of row r (P: compile-time part)
+  // conv of head hh for chunks j = P, P + 2, ... of row r (P: compile-time part):
+  // u = sum_k w[c, k] z[t - k, c] by fp32 FMAs straight from the bf16 operands
+  // (taps in order k = 0..3, as exact products), then u = hi + lo in bf16
   auto conv_part = [&](int hh, auto part_c) {
     constexpr int P = decltype(part_c)::value;
 #pragma unroll
     for (int j = P; j < NCH; j += 2) {
-      const float4* w4 = reinterpret_cast<const float4*>(ws) + hh * D + j * 8;   // taps of 8 channels
+      const uint4* tw = reinterpret_cast<const uint4*>(ws + hh * D + j * 8);   // 2 channels each
       const bf16* zc = z + (r + kPtHalo) * ZC + hh * D + j * 8;
-      float4 w[8];
+      uint4 t4[4], zz[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) w[e] = w4[e];
-      float2 acc[4];
+      for (int q = 0; q < 4; ++q) t4[q] = tw[q];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint4 zz = *reinterpret_cast<const uint4*>(zc - k * ZC);
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&zz);
+      for (int k = 0; k < 4; ++k) zz[k] = *reinterpret_cast<const uint4*>(zc - k * ZC);
+      float acc[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 v = __bfloat1622float2(h2[e]);
-          const float2 wk = k == 0 ? make_float2(w[2 * e].x, w[2 * e + 1].x)
-                          : k == 1 ? make_float2(w[2 * e].y, w[2 * e + 1].y)
-                          : k == 2 ? make_float2(w[2 * e].z, w[2 * e + 1].z)
-                                   : make_float2(w[2 * e].w, w[2 * e + 1].w);
-          acc[e] = k == 0 ? make_float2(wk.x * v.x, wk.y * v.y) : ffma2(wk, v, acc[e]);
+      for (int e = 0; e < 8; ++e) {
+        const uint4& tq = t4[e >> 1];
+        uint16_t w[4], zv[4];
+        halves((e & 1) ? tq.z : tq.x, w[0], w[1]);
+        halves((e & 1) ? tq.w : tq.y, w[2], w[3]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t* zw = reinterpret_cast<const uint32_t*>(&zz[k]);
+          uint16_t lo, hi;
+          halves(zw[e >> 1], lo, hi);
+          zv[k] = (e & 1) ? hi : lo;
         }
+        float a = fma_bf16(zv[0], w[0], 0.f);
+#pragma unroll
+        for (int k = 1; k < 4; ++k) a = fma_bf16(zv[k], w[k], a);
+        acc[e] = a;
       }
-      uint4 hi, lo;
-      uint32_t* hp = reinterpret_cast<uint32_t*>(&hi);
-      uint32_t* lp = reinterpret_cast<uint32_t*>(&lo);
+      uint4 hi4, lo4;
+      uint32_t* hp = reinterpret_cast<uint32_t*>(&hi4);
+      uint32_t* lp = reinterpret_cast<uint32_t*>(&lo4);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[e].x, acc[e].y);
-        const float2 hf = __bfloat1622float2(h2);
-        hp[e] = *reinterpret_cast<const uint32_t*>(&h2);
-        lp[e] = pack2(acc[e].x - hf.x, acc[e].y - hf.y);
+        hp[e] = pack2(acc[2 * e], acc[2 * e + 1]);
+        uint16_t h0, h1;
+        halves(hp[e], h0, h1);
+        // u - hi is exact in fp32
+        lp[e] = pack2(fma_bf16(h0, kBf16MinusOne, acc[2 * e]),
+                      fma_bf16(h1, kBf16MinusOne, acc[2 * e + 1]));
       }
       const uint32_t off = swz_offset(r, j * 16, kRowBytes);
-      *reinterpret_cast<uint4*>(smem + L.off_u + off) = hi;
-      *reinterpret_cast<uint4*>(smem + L.off_u + L.u_bytes + off) = lo;
+      *reinterpret_cast<uint4*>(smem + L.off_u + off) = hi4;
+      *reinterpret_cast<uint4*>(smem + L.off_u + L.u_bytes + off) = lo4;
     }
   };
   auto conv = [&](int hh) {
@@ -339,28 +355,50 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
     if (a.qk_mean) {
       const bool is_q = hh < G;
       // y[e] += (q~ + k~) / 2 over channels c0 + e (q~: this head, or the
-      // mean of the group's query heads for the key head)
+      // mean of the group's query heads for the key head), as fp32 FMAs on the
+      // staged bf16 values
       auto add_mean = [&](float (&y)[Q4], int c0) {
 #pragma unroll
         for (int q8 = 0; q8 < Q4 / 8; ++q8) {
-          float kp[8], qp[8];
-          unpack8(*reinterpret_cast<const uint4*>(zrow + QC + c0 + q8 * 8), kp);
+          const uint4 kw = *reinterpret_cast<const uint4*>(zrow + QC + c0 + q8 * 8);
+          const uint32_t* kp = reinterpret_cast<const uint32_t*>(&kw);
           if (is_q) {
-            unpack8(*reinterpret_cast<const uint4*>(zrow + hh * D + c0 + q8 * 8), qp);
-          } else {
+            const uint4 qw = *reinterpret_cast<const uint4*>(zrow + hh * D + c0 + q8 * 8);
+            const uint32_t* qp = reinterpret_cast<const uint32_t*>(&qw);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) qp[e] = 0.f;
-            for (int hl = 0; hl < G; ++hl) {
-              float v[8];
-              unpack8(*reinterpret_cast<const uint4*>(zrow + hl * D + c0 + q8 * 8), v);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) qp[e] += v[e];
+            for (int e = 0; e < 4; ++e) {
+              uint16_t q0, q1, k0, k1;
+              halves(qp[e], q0, q1);
+              halves(kp[e], k0, k1);
+              y[q8 * 8 + 2 * e] = fma_bf16(k0, kBf16Half, fma_bf16(q0, kBf16Half, y[q8 * 8 + 2 * e]));
+              y[q8 * 8 + 2 * e + 1] =
+                  fma_bf16(k1, kBf16Half, fma_bf16(q1, kBf16Half, y[q8 * 8 + 2 * e + 1]));
             }
+          } else {
+            float sq[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) qp[e] /= static_cast<float>(G);
+            for (int e = 0; e < 8; ++e) sq[e] = 0.f;
+            for (int hl = 0; hl < G; ++hl) {
+              const uint4 qw = *reinterpret_cast<const uint4*>(zrow + hl * D + c0 + q8 * 8);
+              const uint32_t* qp = reinterpret_cast<const uint32_t*>(&qw);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                uint16_t q0, q1;
+                halves(qp[e], q0, q1);
+                sq[2 * e] = add_bf16(q0, sq[2 * e]);
+                sq[2 * e + 1] = add_bf16(q1, sq[2 * e + 1]);
+              }
+            }
+            const float hg = 0.5f / static_cast<float>(G);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              uint16_t k0, k1;
+              halves(kp[e], k0, k1);
+              y[q8 * 8 + 2 * e] = fma_bf16(k0, kBf16Half, fmaf(sq[2 * e], hg, y[q8 * 8 + 2 * e]));
+              y[q8 * 8 + 2 * e + 1] =
+                  fma_bf16(k1, kBf16Half, fmaf(sq[2 * e + 1], hg, y[q8 * 8 + 2 * e + 1]));
+            }
           }
-#pragma unroll
-          for (int e = 0; e < 8; ++e) y[q8 * 8 + e] += 0.5f * (qp[e] + kp[e]);
         }
       };
       add_mean(lo, i0);
