@@ -6,13 +6,15 @@
 //
 // One CTA owns 128 consecutive positions of one kv group (its G query heads,
 // its key head and its value head) of one sequence:
-//   1. the group's q~ | k~ rows [t0 - 3, t0 + 128), the G + 1 mix weights
-//      W_h [d_out, d_in] (straight into the swizzled K-major layout of a UMMA
-//      B operand) and the conv taps are copied into shared memory with 16-byte
-//      cp.async, in commit groups in the order the heads use them; each thread
-//      loads its value-shift rows into registers and forms the cos/sin of its
-//      own rotary pairs (angle t theta_i reduced modulo one turn exactly in
-//      64-bit fixed point) while the copies land;
+//   1. one thread issues the copies into shared memory: per head a TMA box of
+//      the rows [t0 - 3, t0 + 128) of its d columns of q~ | k~ (rows outside
+//      the sequence arrive as zeros; 64B / 128B swizzled rows), the G + 1 mix
+//      weights W_h [d_out, d_in] as TMA tiles (straight into the swizzled
+//      K-major layout of a UMMA B operand) and the conv taps as two bulk
+//      copies, completing on one mbarrier per head in the order the heads use
+//      them; meanwhile each thread loads its value-shift rows into registers
+//      and forms the cos/sin of its own rotary pairs (angle t theta_i reduced
+//      modulo one turn exactly in 64-bit fixed point);
 //   2. per head h (G query heads, then the key head):
 //        conv   one thread per (position, 16-byte channel chunk): u = sum_k
 //               w[c, k] z[t - k, c] in fp32, split as u = hi + lo with hi, lo
@@ -43,8 +45,8 @@ constexpr int kPtTT = 128;     // positions per CTA == MMA M == TMEM lanes
 constexpr int kPtHalo = 3;     // the conv reaches back K - 1 <= 3 rows
 
 struct PtLayout {
-  int ZC;                      // staged row width in elements: (G + 1) d + 8
   uint32_t u_bytes, w_bytes;   // one A tile (hi or lo), one head's B tile
+  uint32_t zh_bytes;           // one head's staged rows (131 of d columns), 1024-aligned
   uint32_t off_u, off_w, off_z, off_ws, off_bar, bytes;
 };
 
@@ -52,42 +54,18 @@ struct PtLayout {
 __host__ __device__ inline PtLayout pt_layout(int d, int G) {
   PtLayout L;
   const uint32_t row = static_cast<uint32_t>(d) * 2;
-  L.ZC = (G + 1) * d + 8;      // q | k, + 16 bytes: an odd number of 16-byte units per row
   L.u_bytes = kPtTT * row;
   L.w_bytes = static_cast<uint32_t>(d) * row;
+  L.zh_bytes = ((kPtTT + kPtHalo) * row + 1023u) & ~1023u;
   // U_hi | U_lo; before the first conv the same bytes hold the raw conv taps
   const uint32_t tr_bytes = (static_cast<uint32_t>(G + 1) * d * 4 * 2 + 15u) & ~15u;
   L.off_u = 0;
   L.off_w = 2 * L.u_bytes > tr_bytes ? 2 * L.u_bytes : tr_bytes;   // W_h, h = 0..G
-  L.off_z = L.off_w + (G + 1) * L.w_bytes;          // [131][ZC] bf16
-  L.off_ws = L.off_z + ((static_cast<uint32_t>(kPtTT + kPtHalo) * L.ZC * 2 + 15u) & ~15u);
+  L.off_z = L.off_w + (G + 1) * L.w_bytes;          // head h's rows: off_z + h zh_bytes
+  L.off_ws = L.off_z + (G + 1) * L.zh_bytes;
   L.off_bar = L.off_ws + static_cast<uint32_t>(G + 1) * d * 8;      // [(G+1) d][4] bf16
-  L.bytes = L.off_bar + 64 + 1024;                  // barriers + alignment slack
+  L.bytes = L.off_bar + 8 * (G + 4) + 16 + 1024;    // barriers, TMEM slot, alignment slack
   return L;
-}
-
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-// Wait until at most n of this thread's committed cp.async groups are pending
-// (n < 10; the instruction takes an immediate).
-__device__ __forceinline__ void cp_async_wait_pending(int n) {
-  switch (n) {
-    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
-    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
-    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
-    case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
-    case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
-    case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
-    case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
-    case 7: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
-    case 8: asm volatile("cp.async.wait_group 8;" ::: "memory"); break;
-    default: asm volatile("cp.async.wait_group 9;" ::: "memory"); break;
-  }
 }
 
 // d = a * b + c for bf16 a, b and fp32 c, d in one instruction: the product
@@ -119,7 +97,10 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 // registers a thread each); d = 64: one.
 template <int D>
 __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
-    pre_attn_tc_kernel(const __grid_constant__ PreAttnArgs<bf16> a) {
+    pre_attn_tc_kernel(const __grid_constant__ CUtensorMap tmZ,
+                       const __grid_constant__ CUtensorMap tmWq,
+                       const __grid_constant__ CUtensorMap tmWk,
+                       const __grid_constant__ PreAttnArgs<bf16> a) {
   pdl_enter();
   constexpr uint32_t kRowBytes = D * 2;                 // 64: 64B swizzle, 128: 128B swizzle
   constexpr uint32_t kSwz = (D == 32) ? kSwizzle64B : kSwizzle128B;
@@ -131,15 +112,16 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int G = a.G, S = a.S, K = a.K;
   const PtLayout L = pt_layout(D, G);
-  const int ZC = L.ZC, NH = G + 1, QC = G * D;
+  const int NH = G + 1, QC = G * D;
   const int b = blockIdx.z, g = blockIdx.y, t0 = blockIdx.x * kPtTT;
   const int tid = threadIdx.x, warp = tid >> 5;
-  bf16* z = reinterpret_cast<bf16*>(smem + L.off_z);
+  uint8_t* z = smem + L.off_z;                           // head h: z + h zh_bytes
   uint2* ws = reinterpret_cast<uint2*>(smem + L.off_ws);   // taps of a channel: 4 bf16
   bf16* tr = reinterpret_cast<bf16*>(smem + L.off_u);   // raw taps, until the first conv
   uint64_t* mma_done = reinterpret_cast<uint64_t*>(smem + L.off_bar);   // [2]
   uint64_t* drain = mma_done + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* ld_bar = drain + 1;       // [G]: 0 = taps, W, key head, query head 0; h = query head h
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ld_bar + G);
   __shared__ int abort_flag;
 
   const int64_t ld = a.src_ld;
@@ -152,6 +134,7 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
     mbar_init(&mma_done[0], 1);
     mbar_init(&mma_done[1], 1);
     mbar_init(drain, 1);
+    for (int h = 0; h < G; ++h) mbar_init(&ld_bar[h], 1);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -160,46 +143,27 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
     tmem_relinquish();
   }
 
-  // 1. staging, all by cp.async, in commit groups in the order the head loop
-  // needs them: A = taps, every W_h, the key head's and query head 0's rows;
-  // then query head 1, ..., query head G-1; last the value head's rows.  The
-  // loop waits for one more group per head, so copies overlap the first heads.
-  const int cq = QC / 8;
-  // one head's NCH 16-byte chunks of every staged row, starting at chunk c_lo
-  // (threads run over (row, chunk) pairs, NCH a power of two)
-  auto stage_head = [&](int c_lo, int col0) {
-    for (int idx = tid; idx < (kPtTT + kPtHalo) * NCH; idx += kPtThreads) {
-      const int r = idx / NCH, c = idx % NCH;
-      const int t = t0 - kPtHalo + r;
-      bf16* dst = z + r * ZC + (c_lo + c) * 8;
-      if (t >= 0 && t < S)
-        cp_async16(dst, src_b + static_cast<int64_t>(t) * ld + col0 + c * 8);
-      else
-        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-    }
-  };
-  {
-    // W_h row n (output channel), chunk j of the input channels -> B operand
-    for (int idx = tid; idx < NH * D * NCH; idx += kPtThreads) {
-      const int hh = idx / (D * NCH), rem = idx % (D * NCH);   // D * NCH: a power of two
-      const int n = rem / NCH, j = rem % NCH;
-      const bf16* w = hh < G ? a.wq_chan + (static_cast<int64_t>(g * G + hh) * D + n) * D
-                             : a.wk_chan + (static_cast<int64_t>(g) * D + n) * D;
-      cp_async16(smem + L.off_w + hh * L.w_bytes + swz_offset(n, j * 16, kRowBytes), w + j * 8);
-    }
-    // taps [channel][K]: the group's G d query channels, then its d key channels
-    const int nq = G * D * K / 8, nk = D * K / 8;
-    for (int idx = tid; idx < nq + nk; idx += kPtThreads) {
-      const bf16* w = idx < nq ? a.wq_seq + static_cast<int64_t>(g) * G * D * K + idx * 8
-                               : a.wk_seq + static_cast<int64_t>(g) * D * K + (idx - nq) * 8;
-      cp_async16(tr + idx * 8, w);
-    }
-    stage_head(cq, kcol0);   // key head
-    stage_head(0, qcol0);    // query head 0
-    cp_async_commit();
-    for (int hh = 1; hh < G; ++hh) {
-      stage_head(hh * NCH, qcol0 + hh * D);
-      cp_async_commit();
+  // 1. staging: one thread issues every copy (z boxes are 131 rows x d columns
+  // of the [B][S][cols] tensor; head slot h < G is query head h, slot G the key
+  // head; rows before position 0 and past S are zero-filled by the TMA unit)
+  if (tid == 0) {
+    prefetch_tensormap(&tmZ);
+    prefetch_tensormap(&tmWq);
+    prefetch_tensormap(&tmWk);
+    const uint32_t zbox = (kPtTT + kPtHalo) * kRowBytes;
+    const uint32_t tq = static_cast<uint32_t>(G) * D * K * 2, tk = static_cast<uint32_t>(D) * K * 2;
+    mbar_arrive_expect_tx(&ld_bar[0], tq + tk + NH * L.w_bytes + 2 * zbox);
+    bulk_load(tr, a.wq_seq + static_cast<int64_t>(g) * G * D * K, tq, &ld_bar[0]);
+    bulk_load(reinterpret_cast<uint8_t*>(tr) + tq, a.wk_seq + static_cast<int64_t>(g) * D * K, tk,
+              &ld_bar[0]);
+    for (int h = 0; h < G; ++h)
+      tma_load_2d(smem + L.off_w + h * L.w_bytes, &tmWq, &ld_bar[0], 0, (g * G + h) * D);
+    tma_load_2d(smem + L.off_w + G * L.w_bytes, &tmWk, &ld_bar[0], 0, g * D);
+    tma_load_3d(z + G * L.zh_bytes, &tmZ, &ld_bar[0], kcol0, t0 - kPtHalo, b);
+    tma_load_3d(z, &tmZ, &ld_bar[0], qcol0, t0 - kPtHalo, b);
+    for (int h = 1; h < G; ++h) {
+      mbar_arrive_expect_tx(&ld_bar[h], zbox);
+      tma_load_3d(z + h * L.zh_bytes, &tmZ, &ld_bar[h], qcol0 + h * D, t0 - kPtHalo, b);
     }
   }
   // value-shift rows straight into registers (stored at the end of the kernel):
@@ -233,8 +197,7 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
       }
     }
   }
-  cp_async_wait_pending(G - 1);   // group A: taps, W, key head, query head 0
-  fence_proxy_async_smem();    // W tiles (and later U) are read by the tensor core
+  bool ok = mbar_wait(&ld_bar[0], 0, &abort_flag, a.dev_err);   // taps, W, key head, query head 0
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -258,9 +221,11 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
   const uint32_t u_lo = u_hi + L.u_bytes;
   const uint32_t w_base = smem_addr(smem + L.off_w);
   const uint32_t idesc = make_idesc_bf16(kPtTT, D, false);
-  const bf16* zrow = z + (r + kPtHalo) * ZC;
   const int t = t0 + r;
-  bool ok = true;
+  // 16 bytes at channel chunk c of head slot h, staged row rr (swizzled rows)
+  auto zchunk = [&](int h, int rr, int c) -> const uint4* {
+    return reinterpret_cast<const uint4*>(z + h * L.zh_bytes + swz_offset(rr, c * 16, kRowBytes));
+  };
 
   // conv of head hh for chunks j = P, P + 2, ... of row r (P: compile-time part):
   // u = sum_k w[c, k] z[t - k, c] by fp32 FMAs straight from the bf16 operands
@@ -270,12 +235,11 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
 #pragma unroll
     for (int j = P; j < NCH; j += 2) {
       const uint4* tw = reinterpret_cast<const uint4*>(ws + hh * D + j * 8);   // 2 channels each
-      const bf16* zc = z + (r + kPtHalo) * ZC + hh * D + j * 8;
       uint4 t4[4], zz[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) t4[q] = tw[q];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) zz[k] = *reinterpret_cast<const uint4*>(zc - k * ZC);
+      for (int k = 0; k < 4; ++k) zz[k] = *zchunk(hh, r + kPtHalo - k, j);
       float acc[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -360,10 +324,10 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
       auto add_mean = [&](float (&y)[Q4], int c0) {
 #pragma unroll
         for (int q8 = 0; q8 < Q4 / 8; ++q8) {
-          const uint4 kw = *reinterpret_cast<const uint4*>(zrow + QC + c0 + q8 * 8);
+          const uint4 kw = *zchunk(G, r + kPtHalo, c0 / 8 + q8);
           const uint32_t* kp = reinterpret_cast<const uint32_t*>(&kw);
           if (is_q) {
-            const uint4 qw = *reinterpret_cast<const uint4*>(zrow + hh * D + c0 + q8 * 8);
+            const uint4 qw = *zchunk(hh, r + kPtHalo, c0 / 8 + q8);
             const uint32_t* qp = reinterpret_cast<const uint32_t*>(&qw);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -379,7 +343,7 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) sq[e] = 0.f;
             for (int hl = 0; hl < G; ++hl) {
-              const uint4 qw = *reinterpret_cast<const uint4*>(zrow + hl * D + c0 + q8 * 8);
+              const uint4 qw = *zchunk(hl, r + kPtHalo, c0 / 8 + q8);
               const uint32_t* qp = reinterpret_cast<const uint32_t*>(&qw);
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
@@ -436,11 +400,10 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
       ok = ok && mbar_wait(&mma_done[(hh - 1) & 1], ((hh - 1) >> 1) & 1, &abort_flag, a.dev_err);
       tc_fence_after();
     }
+    // query head hh's rows (head 0's and the key head's came with the first barrier)
+    if (hh > 0 && hh < G) ok = ok && mbar_wait(&ld_bar[hh], 0, &abort_flag, a.dev_err);
     if (ok) conv(hh);
-    // the next head's rows (the key head needs every query head's): at most
-    // G - hh - 2 groups may still be pending, none before the key head
-    if (hh + 1 < NH) cp_async_wait_pending(hh + 1 < G ? G - hh - 2 : 0);
-    fence_proxy_async_smem();
+    fence_proxy_async_smem();   // U is read by the tensor core
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -467,12 +430,14 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
   if (a.len != nullptr && t0 <= S - 1 && S - 1 < t0 + kPtTT) {
     const int KH = K - 1, Hq = a.Hq, Hkv = a.Hkv;
     for (int rr = 0; rr < KH; ++rr) {
-      const bf16* zr = z + (S - KH + rr - t0 + kPtHalo) * ZC;
+      const int srow = S - KH + rr - t0 + kPtHalo;
       for (int c = tid; c < QC + D; c += kPtThreads) {
+        const int h = c / D, ch = c % D;   // slot G: the key head
+        const bf16 v = reinterpret_cast<const bf16*>(zchunk(h, srow, ch / 8))[ch % 8];
         if (c < QC)
-          a.hist_q[(static_cast<int64_t>(b) * KH + rr) * Hq * D + qcol0 + c] = zr[c];
+          a.hist_q[(static_cast<int64_t>(b) * KH + rr) * Hq * D + qcol0 + c] = v;
         else
-          a.hist_k[(static_cast<int64_t>(b) * KH + rr) * Hkv * D + g * D + (c - QC)] = zr[c];
+          a.hist_k[(static_cast<int64_t>(b) * KH + rr) * Hkv * D + g * D + (c - QC)] = v;
       }
     }
     if (a.v_prev)
@@ -483,10 +448,16 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
   }
 
   if (abort_flag && tid == 0) {
-    // Do not release TMEM while an MMA might still write it.
+    // Do not release TMEM while an MMA might still write it, nor leave while
+    // copies into this CTA's shared memory are in flight (bounded waits).
     mma_commit(drain);
     const long long c0 = clock64();
     while (!mbar_try_wait(drain, 0) && clock64() - c0 < kWaitLimitCycles) {
+    }
+    for (int h = 0; h < G; ++h) {
+      const long long c1 = clock64();
+      while (!mbar_try_wait(&ld_bar[h], 0) && clock64() - c1 < kWaitLimitCycles) {
+      }
     }
   }
   tc_fence_before();
@@ -500,12 +471,34 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
 template <int D>
 cudaError_t launch_d(const PreAttnArgs<bf16>& a, cudaStream_t stream) {
   const PtLayout L = pt_layout(D, a.G);
+  const CUtensorMapSwizzle swz = (D == 32) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  CUtensorMap tmZ, tmWq, tmWk;
+  {
+    // q~ | k~ | v~ as [B][S][src_ld]: boxes of 131 rows x D columns
+    const uint64_t dims[3] = {static_cast<uint64_t>(a.src_ld), static_cast<uint64_t>(a.S),
+                              static_cast<uint64_t>(a.B)};
+    const uint64_t st[2] = {static_cast<uint64_t>(a.src_ld) * 2,
+                            static_cast<uint64_t>(a.S) * a.src_ld * 2};
+    const uint32_t box[3] = {static_cast<uint32_t>(D), kPtTT + kPtHalo, 1};
+    if (!encode_tensor_map(&tmZ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.src, dims, st, box, swz))
+      return cudaErrorInvalidValue;
+  }
+  {
+    // channel-mix weights [heads * D][D]: one D x D tile per head
+    const uint64_t dq[2] = {static_cast<uint64_t>(D), static_cast<uint64_t>(a.Hq) * D};
+    const uint64_t dk[2] = {static_cast<uint64_t>(D), static_cast<uint64_t>(a.Hkv) * D};
+    const uint64_t st[1] = {static_cast<uint64_t>(D) * 2};
+    const uint32_t box[2] = {static_cast<uint32_t>(D), static_cast<uint32_t>(D)};
+    if (!encode_tensor_map(&tmWq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.wq_chan, dq, st, box, swz) ||
+        !encode_tensor_map(&tmWk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.wk_chan, dk, st, box, swz))
+      return cudaErrorInvalidValue;
+  }
   cudaError_t e = allow_smem(reinterpret_cast<const void*>(pre_attn_tc_kernel<D>),
                                        static_cast<int>(L.bytes));
   if (e != cudaSuccess) return e;
   dim3 grid((a.S + kPtTT - 1) / kPtTT, a.Hkv, a.B);
-  const cudaError_t el =
-      launch_pdl(pre_attn_tc_kernel<D>, grid, dim3(kPtThreads), L.bytes, stream, a);
+  const cudaError_t el = launch_pdl(pre_attn_tc_kernel<D>, grid, dim3(kPtThreads), L.bytes,
+                                    stream, tmZ, tmWq, tmWk, a);
   count_launches(1);
   return el != cudaSuccess ? el : cudaGetLastError();
 }
@@ -516,6 +509,11 @@ bool pre_attn_tc_supported(const PreAttnArgs<bf16>& a) {
   if (a.d != 32 && a.d != 64) return false;
   if (a.K < 1 || a.K > 4 || a.wq_chan == nullptr || a.wk_chan == nullptr) return false;
   if (a.wq_seq == nullptr || a.wk_seq == nullptr) return false;
+  // TMA and bulk copies: 16-byte aligned bases and row pitches
+  auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  if (!al16(a.src) || !al16(a.wq_chan) || !al16(a.wk_chan) || !al16(a.wq_seq) || !al16(a.wk_seq))
+    return false;
+  if ((a.src_ld * 2) % 16 != 0 || a.S > (1 << 30)) return false;
   return pt_layout(a.d, a.G).bytes <= 227 * 1024;
 }
 
