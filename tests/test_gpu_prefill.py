@@ -35,6 +35,11 @@ SMALL = {
     "bf16_d64_s3": W3.with_(name="s3", S=3),
     "bf16_d32_conv2_nochan": W2.with_(name="k2", B=1, S=77, conv_width=2),
     "bf16_d64_norope": W3.with_(name="norope", S=129, rope_base=0.0),
+    # tensor-core pre-attention: 3 and 1 conv taps (other bulk-copy sizes), and a
+    # group of 16 query heads (17 staged heads, about 213 KB of shared memory)
+    "bf16_d32_conv3": W2.with_(name="k3", B=1, S=259, conv_width=3),
+    "bf16_d64_conv1": W3.with_(name="k1", S=131, conv_width=1),
+    "bf16_d32_g16": W2.with_(name="g16", B=1, S=200, Hkv=1),
 }
 
 
