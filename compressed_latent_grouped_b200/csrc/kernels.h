@@ -53,8 +53,9 @@ struct PreAttnArgs {
 };
 template <typename T>
 cudaError_t launch_pre_attn(const PreAttnArgs<T>& a, cudaStream_t stream);
-// bf16, d in {32, 64}, conv 1..4 taps with both channel-mix weights: the mix on
-// tcgen05 (launch_pre_attn dispatches there when this holds).
+// bf16, d in {32, 64}, conv 1..4 taps with both channel-mix weights, 16-byte
+// aligned inputs and weights, the layout within 227 KB of shared memory: the mix
+// on tcgen05, staging by TMA (launch_pre_attn dispatches there when this holds).
 bool pre_attn_tc_supported(const PreAttnArgs<bf16>& a);
 cudaError_t launch_pre_attn_tc(const PreAttnArgs<bf16>& a, cudaStream_t stream);
 
