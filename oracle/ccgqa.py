@@ -41,7 +41,7 @@ import numpy as np
 __all__ = [
     "Shape", "down_project", "seq_conv", "channel_mix", "qk_mean", "rope",
     "value_shift", "attention", "prefill", "decode_step", "kvcache_append",
-    "cache_values_per_token", "attention_flops",
+    "output_projection", "cache_values_per_token", "attention_flops",
 ]
 
 
@@ -361,6 +361,23 @@ def kvcache_append(cache_k: np.ndarray, cache_v: np.ndarray, length: int,
     cache_k[length:length + n] = k_new
     cache_v[length:length + n] = v_new
     return length + n
+
+
+# --------------------------------------------------------------------------
+# Output up-projection  [CCA Methodologie 1 "Compressie in Latente Ruimte"]
+# --------------------------------------------------------------------------
+def output_projection(o: np.ndarray, W_o: np.ndarray):
+    """Map the latent attention output back to the model width.
+
+    The page runs the whole attention inside the latent space of width E/C and
+    says nothing of how its result returns to width E.  Reading: one bias-free
+    linear map W_o [E, Hq d] (output-feature major, like W_qkv) applied to the
+    concatenated head outputs, y[m, e] = sum_j o[m, j] W_o[e, j].
+
+    o: [M, Hq d] (rows of one or more prefill outputs, or decode outputs).
+    Returns y: [M, E].
+    """
+    return o @ W_o.T
 
 
 # --------------------------------------------------------------------------

@@ -318,6 +318,44 @@ def pin_down_project_blocks():
     _close(v2, np.zeros_like(v2), 0, "v rows zero")
 
 
+def pin_output_projection():
+    """The up-projection against explicit loops, a permutation and linearity."""
+    rng = _rng(21)
+    M, J, E = 3, 5, 4                       # rectangular: a transposed W_o cannot apply
+    o = rng.standard_normal((M, J))
+    W = rng.standard_normal((E, J))
+    y = O.output_projection(o, W)
+    assert y.shape == (M, E)
+    ref = np.zeros((M, E))
+    for m in range(M):
+        for e in range(E):
+            acc = 0.0
+            for j in range(J):
+                acc += o[m, j] * W[e, j]
+            ref[m, e] = acc
+    _close(y, ref, 1e-12, "explicit loops")
+    # W_o = a permutation matrix P (row e picks latent feature p[e]): y[:, e] = o[:, p[e]]
+    p = np.array([2, 0, 3, 1])
+    P = np.zeros((4, 4))
+    P[np.arange(4), p] = 1.0
+    o4 = rng.standard_normal((2, 4))
+    _close(O.output_projection(o4, P), o4[:, p], 0, "permutation")
+    # linear in o
+    o2 = rng.standard_normal((M, J))
+    _close(O.output_projection(2.5 * o + o2, W), 2.5 * y + O.output_projection(o2, W), 1e-12,
+           "linearity")
+    # after a prefill: the layer output of a tiny layer equals the loops on its rows
+    sh = O.Shape(E=8, C=2, Hq=2, Hkv=1)     # latent width Hq d = 4
+    layer = O.Layer(sh, rng.standard_normal((sh.n_qkv, sh.E)) / 3, conv_width=0,
+                    qk_mean=False, value_shift=False)
+    out, _ = O.prefill(layer, rng.standard_normal((3, sh.E)))
+    Wo = rng.standard_normal((sh.E, sh.Hq * sh.d))
+    y3 = O.output_projection(out, Wo)
+    for m in range(3):
+        for e in range(sh.E):
+            assert abs(y3[m, e] - sum(out[m, j] * Wo[e, j] for j in range(4))) < 1e-12
+
+
 # --------------------------------------------------------------------------
 # Whole-layer invariants
 # --------------------------------------------------------------------------

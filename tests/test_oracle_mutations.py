@@ -116,6 +116,14 @@ def _decode_keeps_old_vprev(layer, state, x_t):
     return o, ns
 
 
+def _output_projection_transposed(o, W_o):
+    return o @ W_o
+
+
+def _output_projection_drop_last(o, W_o):
+    return o[:, :-1] @ W_o[:, :-1].T
+
+
 MUTANTS = {
     "seq_conv_drop_last_tap": ("seq_conv", _seq_conv_drop_last_tap),
     "seq_conv_anticausal": ("seq_conv", _seq_conv_anticausal),
@@ -135,6 +143,8 @@ MUTANTS = {
     "down_project_kv_swapped": ("down_project", _down_project_kv_swapped),
     "prefill_hist_reversed": ("prefill", _prefill_hist_reversed),
     "decode_keeps_old_vprev": ("decode_step", _decode_keeps_old_vprev),
+    "output_projection_transposed": ("output_projection", _output_projection_transposed),
+    "output_projection_drop_last": ("output_projection", _output_projection_drop_last),
 }
 
 
