@@ -334,7 +334,7 @@ def run_ours(args, world, rank, local):
     import torch
     from compressed_latent_grouped_b200 import binding as B
     from compressed_latent_grouped_b200.device import DeviceLayer, Graph
-    from compressed_latent_grouped_b200.workloads import WORKLOADS, make_inputs
+    from compressed_latent_grouped_b200.workloads import WORKLOADS, make_inputs, make_output_weights
     import oracle.ccgqa as O
 
     torch.cuda.set_device(local)
@@ -411,6 +411,23 @@ def run_ours(args, world, rank, local):
     barrier(world)
     if lay.error_bits():
         raise RuntimeError(f"device error bits {lay.error_bits()}")
+    # the output up-projection of the prefill output (a row beyond the step's
+    # path, timed on its own): y [B S, E] = out [B S, Hq d] W_o^T
+    W_o = make_output_weights(w, seed=rank).to(dev)
+    y_o = torch.empty(w.B * w.S, w.E, dtype=w.torch_dtype, device=dev)
+    o2 = out.view(w.B * w.S, -1)
+    for _ in range(3):
+        lay.output_projection(o2, W_o, y_o)
+    op_ev = [(mk(), mk()) for _ in range(K)]
+    for a_, b_ in op_ev:
+        flush.zero_()
+        a_.record(stream)
+        lay.output_projection(o2, W_o, y_o)
+        b_.record(stream)
+    torch.cuda.synchronize()
+    oproj_ms = sum(a_.elapsed_time(b_) for a_, b_ in op_ev) / K
+    oproj_flop = 2.0 * w.B * w.S * w.E * w.Hq * w.d
+
     step_ms = [a.elapsed_time(b) for a, b in st_ev]
     t_ms = max_over_ranks(sum(step_ms), world, dev)
     eager_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eager_ev), world, dev) / K
@@ -545,6 +562,10 @@ def run_ours(args, world, rank, local):
                          "hbm_frac": pre_bytes / (pre_ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
             "attn_prefill_tc": {"ms": attn_ms, "tflops": achieved,
                                 "tensor_frac": achieved / peaks["bf16_tflops"]},
+            "output_projection": {
+                "ms": oproj_ms, "tflops": oproj_flop / (oproj_ms / 1e3) / 1e12,
+                "tensor_frac": oproj_flop / (oproj_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                "note": "not part of the step: y = out W_o^T, timed on its own"},
         },
         "phases_ms": {"proj_gemm": proj_ms, "pre_attn": pre_ms, "attn_prefill_tc": attn_ms,
                       "prefill_total": prefill_ms, "decode_proj": dproj_ms,

@@ -83,6 +83,9 @@ def load() -> ctypes.CDLL:
     lib.ccgqa_kvcache_append.argtypes = [P(ccgqa_config), P(ccgqa_kvcache), c_void_p, c_void_p,
                                          c_int32, c_void_p, c_void_p]
     lib.ccgqa_kvcache_append.restype = c_int
+    lib.ccgqa_output_projection.argtypes = [P(ccgqa_config), c_void_p, c_void_p, ctypes.c_int64,
+                                            c_void_p, c_void_p, c_void_p]
+    lib.ccgqa_output_projection.restype = c_int
     lib.ccgqa_status_string.argtypes = [c_int]
     lib.ccgqa_status_string.restype = c_char_p
     lib.ccgqa_launch_count.argtypes = []
@@ -211,6 +214,14 @@ def ccgqa_kvcache_append(cfg, cache, k_new, v_new, n_new, dev_err=None, stream=N
                                   _ptr(v_new), n_new, _ptr(dev_err), _stream(stream))
     if check and st != 0:
         raise CCGQAError(st, "ccgqa_kvcache_append")
+    return st
+
+
+def ccgqa_output_projection(cfg, W_o, o, M, y, dev_err=None, stream=None, check=True) -> int:
+    st = load().ccgqa_output_projection(ctypes.byref(cfg), _ptr(W_o), _ptr(o), int(M), _ptr(y),
+                                        _ptr(dev_err), _stream(stream))
+    if check and st != 0:
+        raise CCGQAError(st, "ccgqa_output_projection")
     return st
 
 

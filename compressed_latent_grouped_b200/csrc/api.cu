@@ -467,6 +467,30 @@ CCGQA_API ccgqa_status ccgqa_kvcache_append(const ccgqa_config* cfg, const ccgqa
   return e == cudaSuccess ? CCGQA_OK : cuda_fail(e);
 }
 
+CCGQA_API ccgqa_status ccgqa_output_projection(const ccgqa_config* cfg, const void* W_o,
+                                               const void* o, int64_t M, void* y,
+                                               int32_t* dev_err, void* stream) {
+  Geo g;
+  ccgqa_status s = derive(cfg, &g);
+  if (s != CCGQA_OK) return s;
+  if (M <= 0 || !W_o || !o || !y) return CCGQA_ERR_INVALID_ARG;
+  if (!aligned16(W_o) || !aligned16(o) || !aligned16(y)) return CCGQA_ERR_INVALID_ARG;
+  if (M > (int64_t(1) << 30)) return CCGQA_ERR_UNSUPPORTED;
+  const int K = g.Hq * g.d, N = g.E;   // y [M, E] = o [M, Hq d] W_o^T
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!stream_allowed(st)) return CCGQA_ERR_INVALID_ARG;
+  cudaError_t e;
+  if (g.dtype == CCGQA_BF16) {
+    if (K % 8 != 0) return CCGQA_ERR_UNSUPPORTED;   // 16-byte TMA row pitch
+    e = launch_proj_gemm_bf16(static_cast<const bf16*>(o), static_cast<const bf16*>(W_o),
+                              static_cast<bf16*>(y), static_cast<int>(M), N, K, dev_err, st);
+  } else {
+    e = launch_proj_gemm_f32(static_cast<const float*>(o), static_cast<const float*>(W_o),
+                             static_cast<float*>(y), static_cast<int>(M), N, K, st);
+  }
+  return e == cudaSuccess ? CCGQA_OK : cuda_fail(e);
+}
+
 CCGQA_API const char* ccgqa_status_string(ccgqa_status s) {
   switch (s) {
     case CCGQA_OK: return "ok";

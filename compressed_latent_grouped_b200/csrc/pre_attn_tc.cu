@@ -142,6 +142,11 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
     tmem_alloc(tmem_slot, 2 * D);
     tmem_relinquish();
   }
+  // barriers, abort flag and TMEM address visible before any thread uses them
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
 
   // 1. staging: one thread issues every copy (z boxes are 131 rows x d columns
   // of the [B][S][cols] tensor; head slot h < G is query head h, slot G the key
@@ -198,10 +203,6 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
     }
   }
   bool ok = mbar_wait(&ld_bar[0], 0, &abort_flag, a.dev_err);   // taps, W, key head, query head 0
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
   // conv taps as bf16 [channel][4], zero past K
   for (int hc = tid; hc < NH * D; hc += kPtThreads) {
     uint16_t w4[4];

@@ -101,6 +101,16 @@ class DeviceLayer:
         B.ccgqa_kvcache_append(self.cfg, self.cache, k_new, v_new, k_new.shape[1], self.dev_err,
                                stream)
 
+    def output_projection(self, o: torch.Tensor, W_o: torch.Tensor,
+                          y: torch.Tensor | None = None, stream=None):
+        """y [M, E] = o [M, Hq d] W_o^T (W_o [E, Hq d] on this device)."""
+        w = self.w
+        M = o.numel() // (w.Hq * w.d)
+        if y is None:
+            y = torch.empty(M, w.E, dtype=w.torch_dtype, device=self.device)
+        B.ccgqa_output_projection(self.cfg, W_o, o, M, y, self.dev_err, stream)
+        return y
+
     def error_bits(self) -> int:
         return int(self.dev_err.item())
 

@@ -130,6 +130,13 @@ def make_inputs(w: Workload, seed: int = 0, batch: int | None = None) -> dict:
     return out
 
 
+def make_output_weights(w: Workload, seed: int = 0) -> torch.Tensor:
+    """W_o [E, Hq d] of the output up-projection, N(0, 1 / (Hq d)) in the working
+    dtype, from a generator of its own (the draws of make_inputs are unchanged)."""
+    rng = np.random.default_rng(seed + 7919)
+    return _normal(rng, (w.E, w.Hq * w.d), (1.0 / (w.Hq * w.d)) ** 0.5, w.dtype)
+
+
 def sample_rows(S: int, n: int = 1024, tile: int = 128, seed: int = 1) -> np.ndarray:
     """Query positions checked one by one on full-size workloads: the first and
     last ``tile`` positions, positions on both sides of every ``tile`` boundary

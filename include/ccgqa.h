@@ -182,6 +182,28 @@ CCGQA_API ccgqa_status ccgqa_kvcache_append(const ccgqa_config* cfg, const ccgqa
                                             const void* k_new, const void* v_new,
                                             int32_t n_new, int32_t* dev_err, void* stream);
 
+/* Output up-projection: the latent attention output mapped back to the model
+ * width E.  The CCA page ("Compressed Convolutional Attention", Methodologie
+ * item 1) runs the whole attention inside the latent space and leaves the way
+ * back to width E unstated; the reading here is one bias-free linear map:
+ *   y[m, e] = sum_j o[m, j] * W_o[e, j],   m < M, j < Hq*d, e < E.
+ *  - o:   [M, Hq*d] device, e.g. ccgqa_prefill's out viewed as [batch*seq_len,
+ *         Hq*d] or ccgqa_decode_step's out ([batch, Hq*d]);
+ *  - W_o: [E, Hq*d] device, output-feature major (like W_qkv);
+ *  - y:   [M, E] device, written; must not overlap o or W_o.
+ * All three in cfg->dtype and 16-byte aligned, caller-owned.  bf16: tcgen05
+ * GEMM with fp32 accumulation, y rounded to bf16 once; f32: fp32 GEMM on the
+ * CUDA cores.  Only E, C, n_q_heads and dtype of cfg are used (validated as
+ * for every call).  Returns CCGQA_ERR_INVALID_ARG for M <= 0, a NULL or
+ * misaligned pointer, or another stream while this thread records a graph;
+ * CCGQA_ERR_UNSUPPORTED for M > 2^30 or (bf16) Hq*d not a multiple of 8;
+ * CCGQA_ERR_CUDA on a launch failure; else CCGQA_OK (asynchronous on
+ * `stream`; a bounded wait that runs out sets CCGQA_DEVERR_TIMEOUT in
+ * *dev_err, nullable). */
+CCGQA_API ccgqa_status ccgqa_output_projection(const ccgqa_config* cfg, const void* W_o,
+                                               const void* o, int64_t M, void* y,
+                                               int32_t* dev_err, void* stream);
+
 /* Static description of a status code. */
 CCGQA_API const char* ccgqa_status_string(ccgqa_status s);
 

@@ -171,3 +171,18 @@ def test_graph_calls_checked_on_host(lib):
     assert lib.ccgqa_graph_kernel_count(None) == -1
     assert lib.ccgqa_graph_destroy(None) == 0
     assert B.ccgqa_launch_count() == 0
+
+
+def test_output_projection_checked_on_host(lib):
+    cfg = B.make_config(E=512, C=4, n_q_heads=4, n_kv_heads=2)      # d = 32
+    fake = ctypes.c_void_p(4096)          # aligned, never dereferenced on these paths
+    f = lib.ccgqa_output_projection
+    assert f(ctypes.byref(cfg), fake, fake, 0, fake, None, None) == 1          # M <= 0
+    assert f(ctypes.byref(cfg), None, fake, 4, fake, None, None) == 1          # NULL W_o
+    assert f(ctypes.byref(cfg), fake, ctypes.c_void_p(4098), 4, fake, None, None) == 1
+    assert f(ctypes.byref(cfg), fake, fake, (1 << 30) + 1, fake, None, None) == 2
+    odd = B.make_config(E=20, C=1, n_q_heads=4, n_kv_heads=2)   # head dim 5: unsupported
+    assert f(ctypes.byref(odd), fake, fake, 4, fake, None, None) == 2
+    bad = B.make_config(E=500, C=4, n_q_heads=4, n_kv_heads=2)  # E not a multiple of C Hq
+    assert f(ctypes.byref(bad), fake, fake, 4, fake, None, None) == 1
+    assert B.ccgqa_launch_count() == 0
