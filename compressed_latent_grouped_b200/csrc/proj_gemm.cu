@@ -7,8 +7,10 @@
 //   128x64 A and 256x64 W tiles with TMA (128B swizzle) through a 4-stage
 //   shared-memory ring; warp 1 allocates 2 x 256 TMEM columns and one thread
 //   issues tcgen05.mma (M=128, N=256, K=16, fp32 accumulate) into them in turn;
-//   warps 2-5 read a finished accumulator back with tcgen05.ld and store bf16
-//   rows while the next tile accumulates into the other.
+//   warps 2-5 read a finished accumulator back with tcgen05.ld, 32 x 32 at a
+//   time, into a 64B-swizzled bf16 staging buffer (two per warp, alternating)
+//   that a TMA tile store writes out as whole output rows (clipped at M and N),
+//   while the next tile accumulates into the other.
 // fp32: a plain shared-memory tiled GEMM on the CUDA cores.
 #include "kernels.h"
 #include "sm100.cuh"
@@ -23,7 +25,28 @@ constexpr int kGemmThreads = 192;
 constexpr uint32_t kATile = kBM * kBK * 2;      // 16 KB
 constexpr uint32_t kBTile = kBN * kBK * 2;      // 32 KB
 constexpr uint32_t kStageBytes = kATile + kBTile;
-constexpr size_t kGemmSmem = size_t(kStages) * kStageBytes + 1024 + 256;
+constexpr uint32_t kOffBar = kStages * kStageBytes;          // barriers, TMEM slot (< 1 KB)
+constexpr uint32_t kOffOut = kOffBar + 1024;                  // output staging, 1024-aligned
+constexpr uint32_t kOutBuf = 32 * 32 * 2;                     // one 32 x 32 bf16 chunk
+constexpr size_t kGemmSmem = size_t(kOffOut) + 4 * 2 * kOutBuf + 1024;   // + alignment slack
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int c0,
+                                             int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::
+                   "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_addr(src)), "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// at most one of this thread's bulk groups still reading shared memory
+__device__ __forceinline__ void bulk_wait_read_1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+// every bulk group of this thread complete
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
 
 // Persistent: CTA c computes tiles c, c + gridDim.x, ... (tile t = row block
 // t / n_tiles, column block t % n_tiles, so CTAs running together share A rows
@@ -32,13 +55,14 @@ constexpr size_t kGemmSmem = size_t(kStages) * kStageBytes + 1024 + 256;
 // epilogue of one tile overlaps the main loop of the next.
 __global__ void __launch_bounds__(kGemmThreads, 1)
     proj_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
-                          const __grid_constant__ CUtensorMap tmB, bf16* __restrict__ C, int M,
-                          int N, int K, int32_t* dev_err) {
+                          const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ CUtensorMap tmC, int M, int N, int K,
+                          int32_t* dev_err) {
   pdl_enter();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;   // [2] accumulator b complete
   uint64_t* acc_empty = acc_full + 2;     // [2] accumulator b read back (128 arrivals)
@@ -131,13 +155,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // Epilogue: warp w may only touch TMEM lanes [32 (w % 4), 32 (w % 4) + 32).
     const int q4 = warp & 3;
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-    int i = 0;
+    uint8_t* stage = smem + kOffOut + (warp - 2) * 2 * kOutBuf;
+    int i = 0, nst = 0;   // tiles read back, chunks stored by this warp
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
       const int bsel = i & 1;
       if (!mbar_wait(&acc_full[bsel], (i >> 1) & 1, &abort_flag, dev_err)) break;
       tc_fence_after();
       const int m0 = (t / n_tiles) * kBM, n0 = (t % n_tiles) * kBN;
-      const int row = m0 + q4 * 32 + lane;
+      const int r0 = m0 + q4 * 32;   // this warp's 32 output rows
 #pragma unroll 1
       for (int c = 0; c < kBN / 32; ++c) {
         const int col0 = n0 + c * 32;
@@ -145,30 +170,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t r[32];
         tmem_ld32(trow + bsel * kBN + c * 32, r);
         tmem_wait_ld();
-        if (row < M) {
-          bf16* dst = C + static_cast<int64_t>(row) * N + col0;
-          if (col0 + 32 <= N && (N % 8) == 0) {
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 pk;
-              uint32_t* pw = reinterpret_cast<uint32_t*>(&pk);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[v * 8 + 2 * e]),
-                                                          __uint_as_float(r[v * 8 + 2 * e + 1]));
-                pw[e] = *reinterpret_cast<uint32_t*>(&h2);
-              }
-              *reinterpret_cast<uint4*>(dst + v * 8) = pk;
-            }
-          } else {
-            for (int e = 0; e < 32 && col0 + e < N; ++e)
-              dst[e] = __float2bfloat16_rn(__uint_as_float(r[e]));
-          }
+        if (r0 >= M) continue;   // rows past M: nothing to store (warp-uniform)
+        uint8_t* buf = stage + (nst & 1) * kOutBuf;
+        if (nst >= 2) {
+          // the store issued from this buffer two chunks ago has read it
+          if (lane == 0) bulk_wait_read_1();
+          __syncwarp();
         }
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint4 pk;
+          uint32_t* pw = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[v * 8 + 2 * e]),
+                                                      __uint_as_float(r[v * 8 + 2 * e + 1]));
+            pw[e] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+          *reinterpret_cast<uint4*>(buf + swz_offset(lane, v * 16, 64)) = pk;
+        }
+        fence_proxy_async_smem();   // the TMA unit reads what the threads wrote
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmC, buf, col0, r0);
+          bulk_commit();
+        }
+        ++nst;
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[bsel]);
     }
+    if (lane == 0) bulk_wait_all();   // no store may still read this CTA's shared memory
   }
 
   if (abort_flag && warp == 1 && lane == 0) {
@@ -237,16 +269,22 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_proj_gemm_bf16(const bf16* A, const bf16* W, bf16* C, int M, int N, int K,
                                   int32_t* dev_err, cudaStream_t stream) {
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmB, tmC;
   const uint64_t dA[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
   const uint64_t sA[1] = {static_cast<uint64_t>(K) * 2};
   const uint32_t bA[2] = {kBK, kBM};
   const uint64_t dB[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
   const uint32_t bB[2] = {kBK, kBN};
+  if (N % 8 != 0) return cudaErrorInvalidValue;   // 16-byte output row pitch for the TMA store
+  const uint64_t dC[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(M)};
+  const uint64_t sC[1] = {static_cast<uint64_t>(N) * 2};
+  const uint32_t bC[2] = {32, 32};
   if (!encode_tensor_map(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, dA, sA, bA,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tensor_map(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, dB, sA, bB,
-                         CU_TENSOR_MAP_SWIZZLE_128B))
+                         CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tensor_map(&tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, dC, sC, bC,
+                         CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   cudaError_t e = allow_smem(reinterpret_cast<const void*>(proj_gemm_bf16_kernel),
                              static_cast<int>(kGemmSmem));
@@ -257,7 +295,7 @@ cudaError_t launch_proj_gemm_bf16(const bf16* A, const bf16* W, bf16* C, int M, 
   const int tiles = ((N + kBN - 1) / kBN) * ((M + kBM - 1) / kBM);
   const int grid = tiles < sms ? tiles : sms;   // one persistent CTA per SM
   const cudaError_t el = launch_pdl(proj_gemm_bf16_kernel, dim3(grid), dim3(kGemmThreads),
-                                    kGemmSmem, stream, tmA, tmB, C, M, N, K, dev_err);
+                                    kGemmSmem, stream, tmA, tmB, tmC, M, N, K, dev_err);
   count_launches(1);
   return el != cudaSuccess ? el : cudaGetLastError();
 }
