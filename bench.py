@@ -313,6 +313,34 @@ def measure_decode_workload(w, steps, dev):
             "tokens_per_s": w.B / (sum(ms) / 1e3)}
 
 
+def measure_output_projection(w, steps, dev):
+    """The output up-projection alone on the workload's B S rows of latent
+    output (y [B S, E] = o W_o^T): 4 warm-up launches, then ``steps`` timed back
+    to back with CUDA events."""
+    import torch
+    from compressed_latent_grouped_b200.device import DeviceLayer
+    from compressed_latent_grouped_b200.workloads import make_inputs, make_output_weights
+    lay = DeviceLayer(w, make_inputs(w.with_(B=1, S=8), seed=0), device=dev)
+    g = torch.Generator().manual_seed(0)
+    o = torch.randn(w.B * w.S, w.Hq * w.d, generator=g).to(w.torch_dtype).to(dev)
+    W_o = make_output_weights(w).to(dev)
+    y = torch.empty(w.B * w.S, w.E, dtype=w.torch_dtype, device=dev)
+    for _ in range(4):
+        lay.output_projection(o, W_o, y)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        lay.output_projection(o, W_o, y)
+    e1.record()
+    torch.cuda.synchronize()
+    if lay.error_bits():
+        raise RuntimeError(f"device error bits {lay.error_bits()}")
+    ms = e0.elapsed_time(e1) / steps
+    flop = 2.0 * w.B * w.S * w.E * w.Hq * w.d
+    return {"output_projection_ms": ms, "tflops": flop / (ms / 1e3) / 1e12}
+
+
 def run_workload_only(args, local):
     """--workload: time one named workload's kernels (profiling runs)."""
     import torch
@@ -326,8 +354,11 @@ def run_workload_only(args, local):
         w = w.with_(S=args.seq)
     if args.decode:
         w = w.with_(decode=True)
-    res = (measure_decode_workload if w.decode else measure_prefill_workload)(
-        w, args.steps, dev)
+    if args.output_projection:
+        res = measure_output_projection(w, args.steps, dev)
+    else:
+        res = (measure_decode_workload if w.decode else measure_prefill_workload)(
+            w, args.steps, dev)
     print(json.dumps({"workload": args.workload, "B": w.B, "S": w.S, **res}), flush=True)
 
 # ----------------------------------------------------------------------- ours
@@ -618,6 +649,8 @@ def main():
     ap.add_argument("--seq", type=int, default=0, help="with --workload: override S (or L)")
     ap.add_argument("--decode", action="store_true",
                     help="with --workload: time a decode step against a cache of S tokens")
+    ap.add_argument("--output-projection", action="store_true",
+                    help="with --workload: time the output up-projection of its B S rows")
     args = ap.parse_args()
     world, rank, local = dist_setup(args.gpus)
     try:
