@@ -21,6 +21,8 @@ bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, co
 
 // ----------------------------------------------------------------- projection
 // C[M, N] = A[M, K] * W[N, K]^T, bf16 in / fp32 accumulate / bf16 out (tcgen05).
+// A, W, C 16-byte aligned, K and N multiples of 8 (TMA row pitches; N % 8 != 0
+// returns cudaErrorInvalidValue).
 cudaError_t launch_proj_gemm_bf16(const bf16* A, const bf16* W, bf16* C, int M, int N, int K,
                                   int32_t* dev_err, cudaStream_t stream);
 // Same contraction in fp32 on the CUDA cores.
