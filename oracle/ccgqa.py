@@ -29,7 +29,9 @@ checks it against something other than itself (closed forms, a library special
 case, brute force, invariants).  The semantics of the convolution, QK-mean and
 value-shift readings themselves cannot be pinned against the pages (the pages
 print no example): for those three readings the parity is "parity unpinned"
-with respect to the paper, while the arithmetic of each reading is pinned.
+with respect to the paper, while the arithmetic of each reading is pinned, and
+so is the order in which ``_mix_qk``, ``prefill`` and ``decode_step`` compose
+them (a whole-layer case written out by hand).
 """
 from __future__ import annotations
 

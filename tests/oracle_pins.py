@@ -359,6 +359,95 @@ def pin_output_projection():
 # --------------------------------------------------------------------------
 # Whole-layer invariants
 # --------------------------------------------------------------------------
+def _composition_layer(d, rope_base):
+    """A packed-input layer (x rows are q~ | k~ | v~) with Hq = 2, Hkv = 1,
+    conv width 2 and per-channel taps: even channels keep the current row
+    (tap 0), odd channels take the previous row (tap 1).  The channel mix is
+    the cyclic permutation y[i] = u[(i + 1) mod d] in both heads.  With lags
+    that differ between neighbouring channels the conv and the mix do not
+    commute, so their order is visible."""
+    sh = O.Shape(E=2 * d, C=1, Hq=2, Hkv=1)
+    P = np.zeros((d, d))
+    for i in range(d):
+        P[i, (i + 1) % d] = 1.0
+
+    def taps(ch):
+        w = np.zeros((ch, 2))
+        w[np.arange(ch) % 2 == 0, 0] = 1.0
+        w[np.arange(ch) % 2 == 1, 1] = 1.0
+        return w
+
+    return O.Layer(sh=sh, W_qkv=None, conv_width=2,
+                   conv_q_seq=taps(2 * d), conv_q_chan=np.stack([P, P]),
+                   conv_k_seq=taps(d), conv_k_chan=P[None].copy(),
+                   qk_mean=True, value_shift=True, rope_base=rope_base, causal=True)
+
+
+def _composition_by_hand(qt, kt, vt, d, rope_on):
+    """q, k, v of the composition layer written out index by index from the
+    spec's steps: sequence conv, then channel mix, then the QK-mean of the
+    PRE-conv values added, then RoPE (d = 2: the pair turns by t radians),
+    and the value-shift of the upper half-channels."""
+    S = qt.shape[0]
+
+    def pre(z, t, h, c):             # z[t - lag(c)], lag 0 on even and 1 on odd channels
+        s = t - c % 2
+        return z[s, h, c] if s >= 0 else 0.0
+
+    q = np.zeros((S, 2, d))
+    k = np.zeros((S, 1, d))
+    v = np.zeros((S, 1, d))
+    for t in range(S):
+        for i in range(d):
+            j = (i + 1) % d          # the mix reads conv channel i + 1
+            for h in range(2):
+                m_q = 0.5 * (qt[t, h, i] + kt[t, 0, i])
+                q[t, h, i] = pre(qt, t, h, j) + m_q
+            m_k = 0.5 * (0.5 * (qt[t, 0, i] + qt[t, 1, i]) + kt[t, 0, i])
+            k[t, 0, i] = pre(kt, t, 0, j) + m_k
+            if i < d // 2:
+                v[t, 0, i] = vt[t, 0, i]
+            else:
+                v[t, 0, i] = vt[t - 1, 0, i] if t > 0 else 0.0
+        if rope_on:                  # d = 2: (a, b) -> (a cos t - b sin t, a sin t + b cos t)
+            c, s = math.cos(t), math.sin(t)
+            for z in (q[t], k[t]):
+                for h in range(z.shape[0]):
+                    a, b = z[h, 0], z[h, 1]
+                    z[h, 0], z[h, 1] = a * c - b * s, a * s + b * c
+    return q, k, v
+
+
+def pin_layer_composition():
+    """The whole layer on a tiny case against values written out by hand:
+    which tensors feed QK-mean (the pre-conv q~ and k~), the order of the
+    sequence conv and the channel mix, and RoPE after the QK-mean add (CCA
+    page, Methodologie items 2-4).  Checks the prefill's q, its cache k and v,
+    every output row (brute-force attention on the hand values), and a decode
+    step from the prefix state."""
+    r = _rng(22)
+    for d, base in ((4, 0.0), (2, 777.0)):
+        lay = _composition_layer(d, base)
+        S = 6
+        x = r.standard_normal((S, 4 * d))
+        qt = x[:, :2 * d].reshape(S, 2, d)
+        kt = x[:, 2 * d:3 * d].reshape(S, 1, d)
+        vt = x[:, 3 * d:].reshape(S, 1, d)
+        q, k, v = _composition_by_hand(qt, kt, vt, d, base != 0.0)
+        out, st = O.prefill(lay, x)
+        _close(st.extra["q"], q, 1e-13, f"d={d} q")
+        _close(st.k, k, 1e-13, f"d={d} cache k")
+        _close(st.v, v, 0, f"d={d} cache v")
+        o = brute_force_attention(q, k, v, 2, True, np.arange(S))
+        _close(out, o.reshape(S, -1), 1e-12, f"d={d} output rows")
+        # decode of the last token from the state after S - 1 tokens
+        _, st5 = O.prefill(lay, x[:-1])
+        od, nst = O.decode_step(lay, st5, x[-1])
+        _close(nst.extra["q"][0], q[-1], 1e-13, f"d={d} decode q")
+        _close(nst.k[-1], k[-1], 1e-13, f"d={d} decode k")
+        _close(od, o[-1].reshape(-1), 1e-12, f"d={d} decode output")
+
+
 def pin_causality():
     """Changing tokens after position t leaves outputs up to t unchanged
     (covers the convolution, the value-shift and the mask)."""

@@ -1,6 +1,7 @@
 """Planted mistakes in the oracle (CPU only): every plausible slip -- a dropped
 term, a wrong sign or index, a transposed operand -- must make at least one pin
 fail.  Each mutant replaces one oracle function for the duration of the test."""
+import dataclasses
 import math
 
 import numpy as np
@@ -11,7 +12,7 @@ import oracle_pins
 
 _orig = {name: getattr(O, name) for name in
          ("seq_conv", "channel_mix", "qk_mean", "rope", "value_shift", "attention",
-          "down_project", "prefill", "decode_step")}
+          "down_project", "prefill", "decode_step", "_mix_qk")}
 
 
 def _seq_conv_drop_last_tap(z, w, history=None):
@@ -124,6 +125,53 @@ def _output_projection_drop_last(o, W_o):
     return o[:, :-1] @ W_o[:, :-1].T
 
 
+def _mix_qk_mean_of_post_conv(layer, q_pre, k_pre, hq=None, hk=None):
+    # QK-mean fed the conv output instead of the pre-conv q~ and k~
+    y_q, y_k = _orig["_mix_qk"](dataclasses.replace(layer, qk_mean=False), q_pre, k_pre, hq, hk)
+    if layer.qk_mean:
+        m_q, m_k = O.qk_mean(y_q, y_k, layer.sh.G)
+        y_q, y_k = y_q + m_q, y_k + m_k
+    return y_q, y_k
+
+
+def _mix_qk_mix_before_conv(layer, q_pre, k_pre, hq=None, hk=None):
+    # channel mix applied to the pre-conv rows (and history), then the conv
+    if layer.conv_width == 0 or layer.conv_q_chan is None:
+        return _orig["_mix_qk"](layer, q_pre, k_pre, hq, hk)
+    sh = layer.sh
+
+    def mixed(z, W, hist):
+        zm = O.channel_mix(z, W)
+        hm = None if hist is None else O.channel_mix(
+            hist.reshape(hist.shape[0], -1, sh.d), W).reshape(hist.shape[0], -1)
+        return zm, hm
+
+    qm, hqm = mixed(q_pre, layer.conv_q_chan, hq)
+    km, hkm = mixed(k_pre, layer.conv_k_chan, hk)
+    nochan = dataclasses.replace(layer, conv_q_chan=None, conv_k_chan=None, qk_mean=False)
+    y_q, y_k = _orig["_mix_qk"](nochan, qm, km, hqm, hkm)
+    if layer.qk_mean:
+        m_q, m_k = O.qk_mean(q_pre, k_pre, sh.G)
+        y_q, y_k = y_q + m_q, y_k + m_k
+    return y_q, y_k
+
+
+def _prefill_rope_before_mean(layer, x, rows=None):
+    # RoPE turns the conv output, and the QK-mean term is added unrotated
+    o, st = _orig["prefill"](dataclasses.replace(layer, qk_mean=False), x, None)
+    if not layer.qk_mean:
+        return _orig["prefill"](layer, x, rows)
+    sh = layer.sh
+    m_q, m_k = O.qk_mean(st.extra["q_pre"], st.extra["k_pre"], sh.G)
+    q = st.extra["q"] + m_q
+    st.k = st.k + m_k
+    st.extra["q"] = q
+    pos = np.arange(x.shape[0])
+    rows = pos if rows is None else np.asarray(rows)
+    o = O.attention(q[rows], st.k, st.v, sh.G, layer.causal, q_pos=rows)
+    return o.reshape(len(rows), -1), st
+
+
 MUTANTS = {
     "seq_conv_drop_last_tap": ("seq_conv", _seq_conv_drop_last_tap),
     "seq_conv_anticausal": ("seq_conv", _seq_conv_anticausal),
@@ -145,6 +193,9 @@ MUTANTS = {
     "decode_keeps_old_vprev": ("decode_step", _decode_keeps_old_vprev),
     "output_projection_transposed": ("output_projection", _output_projection_transposed),
     "output_projection_drop_last": ("output_projection", _output_projection_drop_last),
+    "qk_mean_of_post_conv": ("_mix_qk", _mix_qk_mean_of_post_conv),
+    "channel_mix_before_conv": ("_mix_qk", _mix_qk_mix_before_conv),
+    "rope_before_qk_mean": ("prefill", _prefill_rope_before_mean),
 }
 
 
