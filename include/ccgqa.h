@@ -155,13 +155,21 @@ CCGQA_API ccgqa_status ccgqa_decode_step(const ccgqa_config* cfg, const ccgqa_we
  * This entry point takes the same inputs and outputs as ccgqa_decode_step
  * (no workspace arguments) and uses instead a scratch array compiled into the
  * library: ccgqa_decode_noalloc_max_bytes() bytes (16 MiB) of device global
- * memory that every GPU loading the library holds until the process exits.
+ * memory, held by each GPU from the moment the library's module is loaded on
+ * it until the process exits.
+ *  - When the module loads: CUDA loads modules lazily by default (since
+ *    CUDA 12.2, CUDA_MODULE_LOADING=LAZY), so the array is placed on a device
+ *    by the first call of this entry point there, not when the library is
+ *    opened.  That first call therefore takes 16 MiB from the device; with an
+ *    eager module-loading setting the array is placed at context creation.
+ *    Callers with a fixed memory plan should make one warm-up call on each
+ *    device at initialisation, before their plan is fixed and before any
+ *    stream capture; later calls take no device memory.
  *  - Returns CCGQA_ERR_WORKSPACE when the decode needs more scratch than that
  *    (see ccgqa_decode_workspace_size); it never allocates, frees or calls an
  *    allocating library routine.
- *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current); make that first call
- *    before any stream capture.
+ *  - The first call on each device also looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current).
  *  - All calls share the one array and it keeps the last call's contents: the
  *    call clears the parts that must start at zero itself, but calls whose work
  *    overlaps on the GPU (other streams, other host threads) race on it --
