@@ -1,15 +1,17 @@
 """Benchmark of the CCGQA hot path on B200.
 
-One step = one pass of the whole path over one batch: bf16 prefill of
-B=4 x S=4096 tokens (latent projection on tcgen05, fused conv / QK-mean / RoPE /
+One step = one pass of the whole path on the largest single-GPU workloads: the
+bf16 prefill of one S=32768 sequence (E=4096, C=8, 8 query / 2 kv heads of dim
+64, RoPE base 5e5: latent projection on tcgen05, fused conv / QK-mean / RoPE /
 value-shift, tcgen05 flash attention, cache write) followed by one decode step
-of every sequence against the cache the prefill just wrote (projection, one-token
-pre-step with cache append, split-K attention over S+1 keys).
+of 64 sequences against latent caches of 16384 tokens each (projection,
+one-token pre-step with cache append, split-K attention over 16385 keys).
 
 Prints one JSON line (rank 0).  Timing: W untimed warm-up steps, then K steps,
-each preceded by an untimed write of a buffer larger than L2 and timed with CUDA
-events on the launching stream; the job is bracketed by a barrier and
-torch.cuda.synchronize() on both sides and the time is the max over ranks.
+each preceded by an untimed write of a buffer larger than L2 (and a reset of the
+decode caches' lengths to 16384) and timed with CUDA events on the launching
+stream; the job is bracketed by a barrier and torch.cuda.synchronize() on both
+sides and the time is the max over ranks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """
@@ -27,11 +29,23 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = "bf16_prefill_b4_s4096"
+PREFILL_WL = "bf16_prefill_b1_s32768"
+DECODE_WL = "bf16_decode_b64_l16384"
+WORKLOAD = f"{PREFILL_WL} prefill + {DECODE_WL} decode step"
 METRIC = "CCGQA prefill TFLOP/s & tokens/s; decode latent-KV GB/s vs B200 peak"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ATTN_SRC = os.path.join(ROOT, "compressed_latent_grouped_b200", "csrc", "attn_prefill_tc.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_prefill_tc_traffic.txt")
+# one exponential pair in SOFT_EVERY[d] of each softmax row runs on the FMA pipe
+# (a polynomial) in attn_prefill_tc, the rest on the exp unit
+SOFT_EVERY = {32: 4, 64: 3, 128: 4}
+
+
+def attention_flops(B: int, S: int, Hq: int, d: int, causal: bool = True) -> float:
+    """Algorithmic FLOPs of one prefill attention launch: 2 d for QK^T plus 2 d
+    for PV per visible (query, key) pair; causal counts S^2/2 pairs."""
+    pairs = S * S / 2 if causal else S * S
+    return 4.0 * d * Hq * pairs * B
 
 
 def load_peaks():
@@ -57,7 +71,7 @@ def attn_traffic_per_launch():
                 vals[k] = v
     with open(ATTN_SRC, "rb") as f:
         h = hashlib.sha256(f.read()).hexdigest()[:16]
-    if vals.get("source_sha256_16") != h or vals.get("workload") != WORKLOAD:
+    if vals.get("source_sha256_16") != h or vals.get("workload") != PREFILL_WL:
         return None
     return float(vals["dram_bytes_per_launch"])
 
@@ -143,25 +157,49 @@ def barrier(world):
 
 
 # ----------------------------------------------------------------------- oracle
-def oracle_step_time(w, inp, b: int = 0, s_len: int | None = None):
-    """One bounded sample of the workload through the float64 oracle on the
-    host cores: the prefill of the first s_len tokens (default all S) of
-    sequence b plus its decode step."""
-    import numpy as np
+def _oracle_layer(w, inp):
     import oracle.ccgqa as O
     f = lambda t: None if t is None else t.double().numpy()  # noqa: E731
-    lay = O.Layer(sh=O.Shape(w.E, w.C, w.Hq, w.Hkv), W_qkv=f(inp["W_qkv"]),
-                  conv_width=w.conv_width, conv_q_seq=f(inp["conv_q_seq"]),
-                  conv_q_chan=f(inp["conv_q_chan"]), conv_k_seq=f(inp["conv_k_seq"]),
-                  conv_k_chan=f(inp["conv_k_chan"]), qk_mean=w.qk_mean,
-                  value_shift=w.value_shift, rope_base=w.rope_base, causal=w.causal)
-    x = f(inp["x"][b])
-    if s_len is not None:
-        x = x[:s_len]
+    return O.Layer(sh=O.Shape(w.E, w.C, w.Hq, w.Hkv), W_qkv=f(inp["W_qkv"]),
+                   conv_width=w.conv_width, conv_q_seq=f(inp["conv_q_seq"]),
+                   conv_q_chan=f(inp["conv_q_chan"]), conv_k_seq=f(inp["conv_k_seq"]),
+                   conv_k_chan=f(inp["conv_k_chan"]), qk_mean=w.qk_mean,
+                   value_shift=w.value_shift, rope_base=w.rope_base, causal=w.causal)
+
+
+def oracle_prefill_time(w, inp, lay, b: int = 0, s_len: int | None = None, rows=None):
+    """Host seconds of the float64 oracle's prefill of sequence b (its first
+    s_len tokens, default all S; query rows ``rows``, default all)."""
+    import oracle.ccgqa as O
+    x = (inp["x"][b] if s_len is None else inp["x"][b, :s_len]).double().numpy()
     t0 = time.perf_counter()
-    _, st = O.prefill(lay, x)
-    O.decode_step(lay, st, x[-1])
+    O.prefill(lay, x, rows=rows)
     return time.perf_counter() - t0
+
+
+class OracleDecode:
+    """Decode steps of the float64 oracle against the decode workload's caches
+    (one sequence at a time; the state is built outside the timed call)."""
+
+    def __init__(self, w, inp):
+        self.w, self.inp = w, inp
+        self.lay = _oracle_layer(w, inp)
+
+    def state(self, b):
+        import oracle.ccgqa as O
+        inp = self.inp
+        return O.State(k=inp["cache_k"][b].double().numpy(), v=inp["cache_v"][b].double().numpy(),
+                       hist_q=inp["hist_q"][b].double().numpy(),
+                       hist_k=inp["hist_k"][b].double().numpy(),
+                       v_prev=inp["v_prev"][b].double().numpy())
+
+    def time(self, b):
+        import oracle.ccgqa as O
+        st = self.state(b)
+        x_t = self.inp["x_t"][b].double().numpy()
+        t0 = time.perf_counter()
+        O.decode_step(self.lay, st, x_t)
+        return time.perf_counter() - t0
 
 
 def blas_threads():
@@ -173,63 +211,100 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def reference_sample_len(w, inp, n_calls, budget_s):
-    """Prefix length S' (a multiple of 128, at most S) whose oracle step fits
+def cpu_baseline_headline(wp, inp_p, wd, inp_d):
+    """The float64 oracle on the headline step, on a bounded sample.
+
+    Prefill: the oracle's prefill of the S-token sequence with n query rows
+    evaluated (keys and values always built for all S positions), timed at two
+    row counts; a straight line through the two times extrapolates to all S rows
+    (the oracle computes every score row in full, so its cost per row does not
+    depend on the position).  Decode: the oracle's decode step of each of the
+    B sequences against its full cache, timed one by one."""
+    from compressed_latent_grouped_b200.workloads import sample_rows
+    lay = _oracle_layer(wp, inp_p)
+    n1, n2 = 64, 576
+    rows = sample_rows(wp.S, n=n2, seed=11)
+    t1 = oracle_prefill_time(wp, inp_p, lay, rows=rows[:: n2 // n1][:n1])
+    t2 = oracle_prefill_time(wp, inp_p, lay, rows=rows)
+    per_row = max(t2 - t1, 0.0) / (n2 - n1)
+    t_prefill = t1 - per_row * n1 + per_row * wp.S
+    dec = OracleDecode(wd, inp_d)
+    t_dec = sum(dec.time(b) for b in range(wd.B))
+    tokens = wp.B * wp.S + wd.B
+    return {"value": tokens / (t_prefill + t_dec), "unit": "tokens/s", "cores": blas_threads(),
+            "nproc": os.cpu_count(), "kind": "oracle",
+            "sample": (f"prefill: float64 oracle over all {wp.S} tokens with {n1} and {n2} query "
+                       f"rows evaluated ({t1:.1f} s, {t2:.1f} s), extrapolated linearly to "
+                       f"{wp.S} rows = {t_prefill:.1f} s; decode: all {wd.B} sequences against "
+                       f"their {wd.S}-token caches, timed ({t_dec:.1f} s); cores = BLAS "
+                       f"threads (the rest of the oracle runs on one thread)"),
+            "extrapolated": True, "host_seconds": t1 + t2 + t_dec}
+
+
+def reference_sample_len(wp, inp_p, lay, n_calls, budget_s):
+    """Prefix length S' (a multiple of 128, at most S) whose oracle prefill fits
     budget_s / n_calls, from a 512-token probe scaled by (S'/512)^2 (the
     attention's share grows quadratically, so the estimate errs long)."""
-    probe = min(512, w.S)
-    t_probe = oracle_step_time(w, inp, s_len=probe)
+    probe = min(512, wp.S)
+    t_probe = oracle_prefill_time(wp, inp_p, lay, s_len=probe)
     per_call = budget_s / max(n_calls, 1)
     s_len = int(probe * (per_call / max(t_probe, 1e-6)) ** 0.5) // 128 * 128
-    return max(128, min(w.S, s_len))
+    return max(128, min(wp.S, s_len))
 
 
 def run_reference(args, world, rank):
+    """The reference arm: the float64 oracle on the host cores, on this arm's
+    workload, each step a bounded sample of it."""
     from compressed_latent_grouped_b200.workloads import WORKLOADS, make_inputs
     if rank != 0:
         return
-    w = WORKLOADS[WORKLOAD]
-    inp = make_inputs(w, seed=0, batch=1)
-    # each step: one sequence's prefill over a prefix sized so that the whole
-    # run (warm-up included) stays within --ref-seconds
-    s_len = reference_sample_len(w, inp, args.steps + args.warmup, args.ref_seconds)
-    for _ in range(args.warmup):
-        oracle_step_time(w, inp, s_len=s_len)
-    times = [oracle_step_time(w, inp, s_len=s_len) for _ in range(args.steps)]
-    t = sum(times)
-    tokens = (s_len + 1) * args.steps
-    value = tokens / t
-    cores = blas_threads()
-    sample = (f"1 of {w.B} sequences per step: float64 prefill of its first {s_len} of {w.S} "
-              f"tokens + 1 decode step")
+    wp, wd = WORKLOADS[PREFILL_WL], WORKLOADS[DECODE_WL]
+    inp_p = make_inputs(wp, seed=0)
+    inp_d = make_inputs(wd, seed=0, batch=8)
+    lay = _oracle_layer(wp, inp_p)
+    dec = OracleDecode(wd, inp_d)
+    n = args.steps + args.warmup
+    s_len = reference_sample_len(wp, inp_p, lay, n, 0.8 * args.ref_seconds)
+
+    def one(i):
+        return oracle_prefill_time(wp, inp_p, lay, s_len=s_len) + dec.time(i % 8)
+
+    for i in range(args.warmup):
+        one(i)
+    t = sum(one(i) for i in range(args.steps))
+    value = (s_len + 1) * args.steps / t
+    sample = (f"per step: float64 prefill of the first {s_len} of {wp.S} tokens of the "
+              f"{PREFILL_WL} sequence + 1 decode step of one of the {wd.B} sequences against "
+              f"its {wd.S}-token cache")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded PCG64 normals)",
-        "config": {"workload": WORKLOAD, "B": w.B, "S": w.S, "E": w.E, "C": w.C, "Hq": w.Hq,
-                   "Hkv": w.Hkv, "d": w.d, "sample": sample},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": sample},
+        "config": {"workload": WORKLOAD, "S": wp.S, "E": wp.E, "C": wp.C, "Hq": wp.Hq,
+                   "Hkv": wp.Hkv, "d": wp.d, "decode_B": wd.B, "decode_L": wd.S,
+                   "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+                         "nproc": os.cpu_count(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-
 def exp_roofline(w, attn_ms, peaks):
-    """The softmax's exponentials against the exp unit: 16 ex2 per clock per SM
-    (the B200 SFU rate, measured 15.8 on this part) x 148 SMs x the maximum SM
-    clock.  Causal scores: B Hq S (S + 1) / 2 exponentials per launch.  One in
-    four runs on the FMA pipe instead, so frac can pass 0.75 of the exp-unit
-    time only by that offload."""
+    """The exponentials the exp unit executes against its peak: 16 ex2 per
+    clock per SM (the B200 SFU rate, measured 15.8 on this part) x 148 SMs x the
+    maximum SM clock.  A causal launch has B Hq S (S + 1) / 2 exponentials; one
+    pair in SOFT_EVERY[d] runs on the FMA pipe instead, so the exp unit's share
+    is the rest, and frac is that share's rate over the unit's peak."""
     n_exp = w.B * w.Hq * w.S * (w.S + 1) / 2 if w.causal else w.B * w.Hq * w.S * w.S
+    mufu_share = 1.0 - 1.0 / SOFT_EVERY.get(w.d, 4)
     mhz = peaks.get("sm_max_mhz", 1965.0)
     peak = 16 * 148 * mhz * 1e6 / 1e12
-    achieved = n_exp / (attn_ms / 1e3) / 1e12
+    achieved = n_exp * mufu_share / (attn_ms / 1e3) / 1e12
     return {"bound": "alu", "unit": "Texp/s", "achieved": achieved, "peak": peak,
-            "frac": achieved / peak, "exp_per_launch": n_exp,
+            "frac": achieved / peak, "exp_per_launch": n_exp, "exp_unit_share": mufu_share,
             "peak_kind": f"exp unit (ex2): 16/clk/SM x 148 SMs x {mhz:.0f} MHz, derived "
                          f"(15.8/clk/SM measured with a throughput probe)"}
 
@@ -242,7 +317,6 @@ def measure_prefill_workload(w, steps, dev):
     from compressed_latent_grouped_b200 import binding as B
     from compressed_latent_grouped_b200.device import DeviceLayer
     from compressed_latent_grouped_b200.workloads import make_inputs
-    import oracle.ccgqa as O
     inp = make_inputs(w, seed=0)
     lay = DeviceLayer(w, inp, device=dev, cap=w.S)
     lay.alloc_cache()
@@ -261,17 +335,47 @@ def measure_prefill_workload(w, steps, dev):
     if lay.error_bits():
         raise RuntimeError(f"device error bits {lay.error_bits()}")
     ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps for i in range(3)]
-    fl = w.B * O.attention_flops(w.S, w.Hq, w.d)
+    fl = attention_flops(w.B, w.S, w.Hq, w.d, w.causal)
     peaks, _ = load_peaks()
     res = {"attn_ms": ms[2], "attn_tflops": fl / (ms[2] / 1e3) / 1e12,
            "attn_tensor_frac": fl / (ms[2] / 1e3) / 1e12 / peaks["bf16_tflops"],
-           "attn_exp_frac": exp_roofline(w, ms[2], peaks)["frac"],
+           "attn_exp_unit_frac": exp_roofline(w, ms[2], peaks)["frac"],
            "pre_attn_ms": ms[1], "prefill_ms": sum(ms),
            "tokens_per_s": w.B * w.S / (sum(ms) / 1e3)}
     if not w.packed_input:
         res["proj_ms"] = ms[0]
         res["proj_tflops"] = 2.0 * w.B * w.S * w.E * w.n_qkv / (ms[0] / 1e3) / 1e12
+        pre_bytes = 2 * w.B * w.S * w.n_qkv * 2
+        res["pre_attn_hbm_frac"] = pre_bytes / (ms[1] / 1e3) / 1e9 / peaks["hbm_gbs"]
     return res
+
+
+def setup_decode(w, dev, seed=0, extra_cap=64):
+    """A decode layer whose caches hold w.S tokens per sequence, plus the
+    device tensor that resets the lengths to w.S between timed steps."""
+    import torch
+    from compressed_latent_grouped_b200.device import DeviceLayer
+    from compressed_latent_grouped_b200.workloads import make_inputs
+    inp = make_inputs(w, seed=seed)
+    lay = DeviceLayer(w, inp, device=dev, cap=w.S + extra_cap)
+    t = lay.alloc_cache()
+    lay.append(inp["cache_k"].to(dev), inp["cache_v"].to(dev))
+    t["hist_q"].copy_(inp["hist_q"])
+    t["hist_k"].copy_(inp["hist_k"])
+    t["v_prev"].copy_(inp["v_prev"])
+    len0 = torch.full((w.B,), w.S, dtype=torch.int32, device=dev)
+    return lay, inp, len0
+
+
+def decode_numbers(w, proj_ms, pre_ms, attn_ms, peaks):
+    kv = 2 * w.B * w.Hkv * (w.S + 1) * w.d * 2
+    step = proj_ms + pre_ms + attn_ms
+    return {"kv_bytes": kv, "proj_ms": proj_ms, "pre_ms": pre_ms, "attn_ms": attn_ms,
+            "step_ms": step, "attn_gbs": kv / (attn_ms / 1e3) / 1e9,
+            "attn_hbm_frac": kv / (attn_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "step_gbs": kv / (step / 1e3) / 1e9,
+            "step_hbm_frac": kv / (step / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "tokens_per_s": w.B / (step / 1e3)}
 
 
 def measure_decode_workload(w, steps, dev):
@@ -279,24 +383,17 @@ def measure_decode_workload(w, steps, dev):
     the one-token pre-step and the split-K attention over len + 1 keys."""
     import torch
     from compressed_latent_grouped_b200 import binding as B
-    from compressed_latent_grouped_b200.device import DeviceLayer
-    from compressed_latent_grouped_b200.workloads import make_inputs
-    inp = make_inputs(w, seed=0)
-    lay = DeviceLayer(w, inp, device=dev, cap=w.S + 64)
-    t = lay.alloc_cache()
-    lay.append(inp["cache_k"].to(dev), inp["cache_v"].to(dev))
-    t["hist_q"].copy_(inp["hist_q"])
-    t["hist_k"].copy_(inp["hist_k"])
-    t["v_prev"].copy_(inp["v_prev"])
+    lay, inp, len0 = setup_decode(w, dev)
     x_t = inp["x_t"].to(dev)
     out = torch.empty(w.B, w.Hq * w.d, dtype=w.torch_dtype, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    lens = lay.cache_tensors["len"]
     for _ in range(3):
-        t["len"].fill_(w.S)
+        lens.copy_(len0)
         lay.decode_step(x_t, out)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     for e in evs:
-        t["len"].fill_(w.S)
+        lens.copy_(len0)
         flush.zero_()
         B.ccgqa_set_phase_events(e)
         lay.decode_step(x_t, out)
@@ -305,18 +402,14 @@ def measure_decode_workload(w, steps, dev):
     if lay.error_bits():
         raise RuntimeError(f"device error bits {lay.error_bits()}")
     ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps for i in range(3)]
-    kv = 2 * w.B * w.Hkv * (w.S + 1) * w.d * 2
     peaks, _ = load_peaks()
-    return {"attn_ms": ms[2], "kv_bytes": kv, "attn_gbs": kv / (ms[2] / 1e3) / 1e9,
-            "attn_hbm_frac": kv / (ms[2] / 1e3) / 1e9 / peaks["hbm_gbs"],
-            "proj_ms": ms[0], "pre_ms": ms[1], "step_ms": sum(ms),
-            "tokens_per_s": w.B / (sum(ms) / 1e3)}
+    return decode_numbers(w, ms[0], ms[1], ms[2], peaks)
 
 
 def measure_output_projection(w, steps, dev):
     """The output up-projection alone on the workload's B S rows of latent
-    output (y [B S, E] = o W_o^T): 4 warm-up launches, then ``steps`` timed back
-    to back with CUDA events."""
+    output (y [B S, E] = o W_o^T): 4 warm-up launches, then ``steps`` timed one
+    by one with CUDA events, L2 flushed before each."""
     import torch
     from compressed_latent_grouped_b200.device import DeviceLayer
     from compressed_latent_grouped_b200.workloads import make_inputs, make_output_weights
@@ -325,20 +418,24 @@ def measure_output_projection(w, steps, dev):
     o = torch.randn(w.B * w.S, w.Hq * w.d, generator=g).to(w.torch_dtype).to(dev)
     W_o = make_output_weights(w).to(dev)
     y = torch.empty(w.B * w.S, w.E, dtype=w.torch_dtype, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     for _ in range(4):
         lay.output_projection(o, W_o, y)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for a, b in evs:
+        flush.zero_()
+        a.record()
         lay.output_projection(o, W_o, y)
-    e1.record()
+        b.record()
     torch.cuda.synchronize()
     if lay.error_bits():
         raise RuntimeError(f"device error bits {lay.error_bits()}")
-    ms = e0.elapsed_time(e1) / steps
+    ms = sum(a.elapsed_time(b) for a, b in evs) / steps
     flop = 2.0 * w.B * w.S * w.E * w.Hq * w.d
-    return {"output_projection_ms": ms, "tflops": flop / (ms / 1e3) / 1e12}
+    peaks, _ = load_peaks()
+    return {"ms": ms, "tflops": flop / (ms / 1e3) / 1e12,
+            "tensor_frac": flop / (ms / 1e3) / 1e12 / peaks["bf16_tflops"]}
 
 
 def run_workload_only(args, local):
@@ -361,40 +458,47 @@ def run_workload_only(args, local):
             w, args.steps, dev)
     print(json.dumps({"workload": args.workload, "B": w.B, "S": w.S, **res}), flush=True)
 
+
 # ----------------------------------------------------------------------- ours
 def run_ours(args, world, rank, local):
     import torch
     from compressed_latent_grouped_b200 import binding as B
     from compressed_latent_grouped_b200.device import DeviceLayer, Graph
-    from compressed_latent_grouped_b200.workloads import WORKLOADS, make_inputs, make_output_weights
-    import oracle.ccgqa as O
+    from compressed_latent_grouped_b200.workloads import WORKLOADS, make_inputs
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    w = WORKLOADS[WORKLOAD]
-    inp = make_inputs(w, seed=rank)
-    lay = DeviceLayer(w, inp, device=dev, cap=w.S + 1)
-    lay.alloc_cache()
-    x = inp["x"].to(dev)
-    g = torch.Generator().manual_seed(1000 + rank)
-    x_t = torch.randn(w.B, w.E, generator=g).to(w.torch_dtype).to(dev)
-    out = torch.empty(w.B, w.S, w.Hq * w.d, dtype=w.torch_dtype, device=dev)
-    out_t = torch.empty(w.B, w.Hq * w.d, dtype=w.torch_dtype, device=dev)
+    wp, wd = WORKLOADS[PREFILL_WL], WORKLOADS[DECODE_WL]
+    inp_p = make_inputs(wp, seed=rank)
+    pf = DeviceLayer(wp, inp_p, device=dev, cap=wp.S)
+    pf.alloc_cache()
+    x = inp_p["x"].to(dev)
+    out = torch.empty(wp.B, wp.S, wp.Hq * wp.d, dtype=wp.torch_dtype, device=dev)
+    dc, inp_d, len0 = setup_decode(wd, dev, seed=1000 + rank)
+    x_t = inp_d["x_t"].to(dev)
+    out_t = torch.empty(wd.B, wd.Hq * wd.d, dtype=wd.torch_dtype, device=dev)
+    lens = dc.cache_tensors["len"]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     # a created stream (graphs cannot record the legacy default stream), made
-    # current so the flush and the events go on it too
+    # current so the flush, the length reset and the events go on it too
     stream = torch.cuda.Stream(dev)
     torch.cuda.set_stream(stream)
 
     def step():
-        lay.prefill(x, out)
-        lay.decode_step(x_t, out_t)
+        pf.prefill(x, out)
+        dc.decode_step(x_t, out_t)
+
+    def between_steps():
+        # untimed: evict L2 and put the decode caches back at wd.S tokens
+        flush.zero_()
+        lens.copy_(len0)
 
     for _ in range(max(args.warmup, 3)):
+        between_steps()
         step()
     torch.cuda.synchronize()
-    if lay.error_bits():
-        raise RuntimeError(f"device error bits {lay.error_bits()}")
+    if pf.error_bits() or dc.error_bits():
+        raise RuntimeError(f"device error bits {pf.error_bits()} {dc.error_bits()}")
 
     K = args.steps
     mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
@@ -410,6 +514,7 @@ def run_ours(args, world, rank, local):
     # each timed step is one graph launch, the serving loop's form
     graph = Graph(step, stream)
     for _ in range(3):
+        between_steps()
         graph.launch()
     torch.cuda.synchronize()
     eager_ev = [(mk(), mk()) for _ in range(K)]
@@ -419,7 +524,7 @@ def run_ours(args, world, rank, local):
         # B200), so the per-kernel events live in pass 3.
         n0 = B.ccgqa_launch_count()
         for i in range(K):
-            flush.zero_()
+            between_steps()
             st_ev[i][0].record(stream)
             graph.launch()
             st_ev[i][1].record(stream)
@@ -427,38 +532,22 @@ def run_ours(args, world, rank, local):
         launches = B.ccgqa_launch_count() - n0
         # pass 2, the same K steps as eager library calls (no graph)
         for i in range(K):
-            flush.zero_()
+            between_steps()
             eager_ev[i][0].record(stream)
             step()
             eager_ev[i][1].record(stream)
         # pass 3, the same K steps with events between the kernels (phase times)
         for i in range(K):
-            flush.zero_()
+            between_steps()
             B.ccgqa_set_phase_events(pf_ev[i])
-            lay.prefill(x, out)
+            pf.prefill(x, out)
             B.ccgqa_set_phase_events(dc_ev[i])
-            lay.decode_step(x_t, out_t)
+            dc.decode_step(x_t, out_t)
             B.ccgqa_set_phase_events(None)
         torch.cuda.synchronize()
     barrier(world)
-    if lay.error_bits():
-        raise RuntimeError(f"device error bits {lay.error_bits()}")
-    # the output up-projection of the prefill output (a row beyond the step's
-    # path, timed on its own): y [B S, E] = out [B S, Hq d] W_o^T
-    W_o = make_output_weights(w, seed=rank).to(dev)
-    y_o = torch.empty(w.B * w.S, w.E, dtype=w.torch_dtype, device=dev)
-    o2 = out.view(w.B * w.S, -1)
-    for _ in range(3):
-        lay.output_projection(o2, W_o, y_o)
-    op_ev = [(mk(), mk()) for _ in range(K)]
-    for a_, b_ in op_ev:
-        flush.zero_()
-        a_.record(stream)
-        lay.output_projection(o2, W_o, y_o)
-        b_.record(stream)
-    torch.cuda.synchronize()
-    oproj_ms = sum(a_.elapsed_time(b_) for a_, b_ in op_ev) / K
-    oproj_flop = 2.0 * w.B * w.S * w.E * w.Hq * w.d
+    if pf.error_bits() or dc.error_bits():
+        raise RuntimeError(f"device error bits {pf.error_bits()} {dc.error_bits()}")
 
     step_ms = [a.elapsed_time(b) for a, b in st_ev]
     t_ms = max_over_ranks(sum(step_ms), world, dev)
@@ -469,23 +558,23 @@ def run_ours(args, world, rank, local):
     dproj_ms, dpre_ms, dattn_ms = phase(dc_ev, 0, 1), phase(dc_ev, 1, 2), phase(dc_ev, 2, 3)
     prefill_ms = phase(pf_ev, 0, 3)
 
-    tokens_per_step = w.B * w.S + w.B
+    tokens_per_step = wp.B * wp.S + wd.B
     value = tokens_per_step * K * world / (t_ms / 1e3)
-    attn_flop = w.B * O.attention_flops(w.S, w.Hq, w.d)
-    proj_flop = 2.0 * w.B * w.S * w.E * w.n_qkv
-    kv_bytes = 2 * w.B * w.Hkv * (w.S + 1) * w.d * 2
+    attn_flop = attention_flops(wp.B, wp.S, wp.Hq, wp.d, wp.causal)
+    proj_flop = 2.0 * wp.B * wp.S * wp.E * wp.n_qkv
     # pre-attention: q~|k~|v~ read once, q, k, v written once (bf16)
-    pre_bytes = 2 * w.B * w.S * w.n_qkv * 2
+    pre_bytes = 2 * wp.B * wp.S * wp.n_qkv * 2
     peaks, peak_kind = load_peaks()
     achieved = attn_flop / (attn_ms / 1e3) / 1e12
     traffic = attn_traffic_per_launch()
+    dec = decode_numbers(wd, dproj_ms, dpre_ms, dattn_ms, peaks)
 
     # end to end through the public API: pinned host buffers in, results out.
     # Three streams, as a serving loop would run it: step i+1's inputs are copied
     # in and step i-1's results copied out while step i computes; device inputs
     # and outputs are double-buffered, and events order each buffer's reuse.
-    x_h = inp["x"].pin_memory()
-    xt_h = x_t.cpu().pin_memory()
+    x_h = inp_p["x"].pin_memory()
+    xt_h = inp_d["x_t"].pin_memory()
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     outt_h = torch.empty(out_t.shape, dtype=out_t.dtype).pin_memory()
     x_d = [torch.empty_like(x) for _ in range(2)]
@@ -512,6 +601,8 @@ def run_ours(args, world, rank, local):
             in_ready[k].record(s_in)
             s_cmp.wait_event(in_ready[k])
             s_cmp.wait_event(out_free[k])
+            with torch.cuda.stream(s_cmp):
+                lens.copy_(len0)       # device-to-device, 256 bytes
             graphs[k].launch()
             in_free[k].record(s_cmp)
             out_ready[k].record(s_cmp)
@@ -521,8 +612,8 @@ def run_ours(args, world, rank, local):
                 outt_h.copy_(ot_d[k], non_blocking=True)
             out_free[k].record(s_out)
 
-    graphs = [Graph(lambda k=k: (lay.prefill(x_d[k], o_d[k], stream=s_cmp),
-                                 lay.decode_step(xt_d[k], ot_d[k], stream=s_cmp)), s_cmp)
+    graphs = [Graph(lambda k=k: (pf.prefill(x_d[k], o_d[k], stream=s_cmp),
+                                 dc.decode_step(xt_d[k], ot_d[k], stream=s_cmp)), s_cmp)
               for k in range(2)]
     e2e_steps(2)
     torch.cuda.synchronize()
@@ -537,68 +628,61 @@ def run_ours(args, world, rank, local):
     for g_ in graphs:
         g_.close()
     barrier(world)
-    if lay.error_bits():
-        raise RuntimeError(f"device error bits {lay.error_bits()}")
+    if pf.error_bits() or dc.error_bits():
+        raise RuntimeError(f"device error bits {pf.error_bits()} {dc.error_bits()}")
     h2d = x.numel() * x.element_size() + x_t.numel() * x_t.element_size()
     d2h = out.numel() * out.element_size() + out_t.numel() * out_t.element_size()
+    del x_d, o_d, x_h, out_h
+    torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        one = make_inputs(w, seed=0, batch=1)
-        t_cpu, reps = 0.0, 0
-        while t_cpu < 10.0 and reps < 8:   # about 10-30 s of host work
-            t_cpu += oracle_step_time(w, one)
-            reps += 1
-        cpu = {"value": reps * (w.S + 1) / t_cpu, "unit": "tokens/s", "cores": blas_threads(),
-               "kind": "oracle",
-               "sample": f"1 of {w.B} sequences, {reps} times: float64 prefill of all {w.S} "
-                         f"tokens + 1 decode step ({t_cpu:.1f} s)"}
+        cpu = cpu_baseline_headline(wp, make_inputs(wp, seed=0), wd, make_inputs(wd, seed=1000))
 
-    by_workload = None
+    by_workload, oproj = None, None
     if rank == 0 and not args.no_extra:
+        # the output up-projection of the prefill's rows (outside the step)
+        oproj = measure_output_projection(wp, 20, dev)
+        oproj["note"] = "not part of the step: y = out W_o^T, timed on its own"
         by_workload = {}
-        for name in ("bf16_prefill_b1_s32768", "bf16_gqa_b2_s8192"):
-            by_workload[name] = measure_prefill_workload(WORKLOADS[name], 10, dev)
-        by_workload["bf16_decode_b64_l16384"] = measure_decode_workload(
-            WORKLOADS["bf16_decode_b64_l16384"], 20, dev)
+        for name in ("bf16_prefill_b4_s4096", "bf16_gqa_b2_s8192"):
+            by_workload[name] = measure_prefill_workload(WORKLOADS[name], 20, dev)
+        by_workload["bf16_prefill_b4_s4096"]["decode_b4_l4096"] = measure_decode_workload(
+            WORKLOADS["bf16_prefill_b4_s4096"].with_(decode=True), 20, dev)
         torch.cuda.empty_cache()
 
     if rank != 0:
         return
-    # The attention kernel's roofline is that of its binding unit: the tensor
-    # core (4 d FLOP per visible score) or the exp unit (one exponential per
-    # visible score), whichever needs more time at its peak (at d <= 64 the exp
-    # unit).  Both fractions are reported.
     timing = "CUDA events around each launch, third pass of the K steps"
-    roof_tensor = {"bound": "tensor", "kernel": "attn_prefill_tc", "achieved": achieved,
-                   "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+    roof_tensor = {"bound": "tensor", "kernel": f"attn_prefill_tc (d = {wp.d})",
+                   "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                    "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
                    "peak_kind": f"{peak_kind} bf16 dense burst",
+                   "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained",
+                                                             peaks["bf16_tflops"]),
                    "flop_per_launch": attn_flop, "ms_per_launch": attn_ms, "timing": timing}
-    roof_exp = {**exp_roofline(w, attn_ms, peaks), "kernel": "attn_prefill_tc",
-                "traffic": traffic, "ms_per_launch": attn_ms, "timing": timing}
-    t_tensor_ms = attn_flop / (peaks["bf16_tflops"] * 1e12) * 1e3
-    t_exp_ms = roof_exp["exp_per_launch"] / (roof_exp["peak"] * 1e12) * 1e3
-    roof = dict(roof_exp if t_exp_ms > t_tensor_ms else roof_tensor)
-    roof["binding"] = (f"time at peak: exp unit {t_exp_ms * 1e3:.0f} us, tensor core "
-                       f"{t_tensor_ms * 1e3:.0f} us")
+    roof_exp = {**exp_roofline(wp, attn_ms, peaks), "kernel": "attn_prefill_tc",
+                "ms_per_launch": attn_ms, "timing": timing}
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": max(args.warmup, 3), "ms_per_step": t_ms / K,
         "eager_ms_per_step": eager_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded PCG64 normals, weights N(0, 1/fan_in))",
-        "config": {"workload": f"{WORKLOAD} prefill + 1 decode step", "B": w.B, "S": w.S,
-                   "E": w.E, "C": w.C, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
-                   "conv_width": w.conv_width, "rope_base": w.rope_base,
+        "config": {"workload": WORKLOAD,
+                   "prefill": {"B": wp.B, "S": wp.S, "E": wp.E, "C": wp.C, "Hq": wp.Hq,
+                               "Hkv": wp.Hkv, "d": wp.d, "conv_width": wp.conv_width,
+                               "rope_base": wp.rope_base},
+                   "decode": {"B": wd.B, "L": wd.S, "E": wd.E, "C": wd.C, "Hq": wd.Hq,
+                              "Hkv": wd.Hkv, "d": wd.d},
                    "parallelism": f"replicas x{world} (independent sequences per GPU)",
-                   "l2": "flushed (256 MiB write) before every timed step",
+                   "l2": "flushed (256 MiB write) before every timed step; inputs larger "
+                         "than L2 as well",
                    "launch": "each step one CUDA graph launch of the recorded library calls "
                              "(ccgqa_graph_launch); eager_ms_per_step: the same calls made "
                              "one by one"},
-        "roofline": roof,
-        "roofline_tensor": roof_tensor,
-        "roofline_exp": roof_exp,
+        "roofline": roof_tensor,
+        "roofline_exp_unit": roof_exp,
         "kernels": {
             "proj_gemm": {"ms": proj_ms, "tflops": proj_flop / (proj_ms / 1e3) / 1e12,
                           "tensor_frac": proj_flop / (proj_ms / 1e3) / 1e12 / peaks["bf16_tflops"]},
@@ -607,20 +691,18 @@ def run_ours(args, world, rank, local):
                          "hbm_frac": pre_bytes / (pre_ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
             "attn_prefill_tc": {"ms": attn_ms, "tflops": achieved,
                                 "tensor_frac": achieved / peaks["bf16_tflops"]},
-            "output_projection": {
-                "ms": oproj_ms, "tflops": oproj_flop / (oproj_ms / 1e3) / 1e12,
-                "tensor_frac": oproj_flop / (oproj_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
-                "note": "not part of the step: y = out W_o^T, timed on its own"},
+            "decode_attn": {"ms": dattn_ms, "gbs": dec["attn_gbs"],
+                            "hbm_frac": dec["attn_hbm_frac"]},
+            "output_projection": oproj,
         },
         "phases_ms": {"proj_gemm": proj_ms, "pre_attn": pre_ms, "attn_prefill_tc": attn_ms,
                       "prefill_total": prefill_ms, "decode_proj": dproj_ms,
                       "decode_pre": dpre_ms, "decode_attn": dattn_ms},
-        "prefill": {"tokens_per_s": w.B * w.S / (prefill_ms / 1e3) * world,
+        "prefill": {"tokens_per_s": wp.B * wp.S / (prefill_ms / 1e3) * world,
                     "tflops_attn_plus_proj": (attn_flop + proj_flop) / (prefill_ms / 1e3) / 1e12,
-                    "proj_tflops": proj_flop / (proj_ms / 1e3) / 1e12},
-        "decode": {"kv_bytes": kv_bytes, "attn_gbs": None,
-                   "step_ms": dproj_ms + dpre_ms + dattn_ms,
-                   "hbm_frac_attn": (kv_bytes / (dattn_ms / 1e3) / 1e9) / peaks["hbm_gbs"]},
+                    "tensor_frac_attn_plus_proj": (attn_flop + proj_flop) / (prefill_ms / 1e3)
+                    / 1e12 / peaks["bf16_tflops"]},
+        "decode": dec,
         "clocks": sampler.summary(),
         "e2e": {"value": tokens_per_step * K * world / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -628,7 +710,6 @@ def run_ours(args, world, rank, local):
         "cpu_baseline": cpu,
         "by_workload": by_workload,
     }
-    line["decode"]["attn_gbs"] = kv_bytes / (dattn_ms / 1e3) / 1e9 if dattn_ms > 0 else None
     print(json.dumps(line), flush=True)
 
 

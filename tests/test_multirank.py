@@ -83,4 +83,4 @@ def test_reference_arm_runs_on_rank_zero_only():
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["unit"] == "tokens/s"
     assert d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
-    assert "prefill of its first" in d["config"]["sample"]
+    assert "float64 prefill of the first" in d["config"]["sample"]
