@@ -41,10 +41,17 @@ from dataclasses import dataclass, field
 import numpy as np
 
 __all__ = [
-    "Shape", "down_project", "seq_conv", "channel_mix", "qk_mean", "rope",
-    "value_shift", "attention", "prefill", "decode_step", "kvcache_append",
-    "output_projection", "cache_values_per_token", "attention_flops",
+    "Shape", "down_project", "seq_conv", "channel_mix", "channel_conv", "qk_mean",
+    "qk_mean_self", "rope", "value_shift", "value_shift_heads", "attention", "prefill",
+    "decode_step", "kvcache_append", "output_projection", "cache_values_per_token",
+    "attention_flops", "QK_OFF", "QK_CROSS", "QK_SELF", "VS_OFF", "VS_HALF_CHANNELS",
+    "VS_WHOLE_HEADS",
 ]
+
+# Switches of the readings a layer can take (the CCA page's wording admits
+# more than one; see the functions below).
+QK_OFF, QK_CROSS, QK_SELF = 0, 1, 2
+VS_OFF, VS_HALF_CHANNELS, VS_WHOLE_HEADS = 0, 1, 2
 
 
 @dataclass(frozen=True)
@@ -128,6 +135,28 @@ def channel_mix(u: np.ndarray, W_chan: np.ndarray):
     return np.einsum("hij,thj->thi", W_chan, u)
 
 
+def channel_conv(z: np.ndarray, W: np.ndarray, history: np.ndarray | None = None):
+    """Temporal channel convolution inside each head (a reading variant of
+    [CCA Methodologie 2]: the conv mixes the channels of a head with its own
+    d x d matrix at every tap, instead of a depthwise sequence conv followed
+    by one per-position mix):
+        y[t, h, :] = sum_{j=0}^{K-1} W[h, j] @ z[t - j, h, :].
+
+    z: [S, H, d] pre-convolution rows; W: [H, K, d, d]; history: [K-1, H d]
+    (oldest first, as for seq_conv) or None for zeros before the start.  The
+    depthwise-plus-mix reading is the special case W[h, j] = W_c[h] diag(w_seq[h, :, j]).
+    """
+    S, H, d = z.shape
+    K = W.shape[1]
+    hist = np.zeros((K - 1, H, d)) if history is None else history.reshape(K - 1, H, d)
+    full = np.concatenate([hist, z], axis=0)      # row t of z is row t+K-1 here
+    y = np.zeros((S, H, d))
+    for t in range(S):
+        for j in range(K):
+            y[t] += np.einsum("hij,hj->hi", W[:, j], full[t + K - 1 - j])
+    return y
+
+
 # --------------------------------------------------------------------------
 # a4: QK-mean  [CCA Methodologie 2 "QK-Mean"]
 # --------------------------------------------------------------------------
@@ -147,6 +176,14 @@ def qk_mean(q_pre: np.ndarray, k_pre: np.ndarray, G: int):
     q_grp = q_pre.reshape(S, Hkv, G, d).mean(axis=2)
     m_k = 0.5 * (q_grp + k_pre)
     return m_q, m_k
+
+
+def qk_mean_self(q_pre, y_q, k_pre, y_k):
+    """Reading variant "self" of [CCA Methodologie 2 "QK-Mean"]: each head's
+    output is the mean of its own pre- and post-convolution values,
+        q = (q_pre + y_q) / 2,   k = (k_pre + y_k) / 2,
+    the literal reading of the garbled sentence (no mixing between q and k)."""
+    return 0.5 * (q_pre + y_q), 0.5 * (k_pre + y_k)
 
 
 # --------------------------------------------------------------------------
@@ -189,6 +226,21 @@ def value_shift(v_lat: np.ndarray, v_prev: np.ndarray | None = None):
     shifted = np.concatenate([prev, v_lat[:-1]], axis=0)
     out = v_lat.copy()
     out[..., d // 2:] = shifted[..., d // 2:]
+    return out
+
+
+def value_shift_heads(v_lat: np.ndarray, v_prev: np.ndarray | None = None):
+    """Whole-head reading variant of [CCA Methodologie 3 "Value-Shift"]: half
+    of the kv heads take the previous token's values.  The last floor(Hkv/2)
+    heads are shifted (heads g >= Hkv - floor(Hkv/2)), the others keep the
+    current row; the row before the first is ``v_prev`` ([Hkv, d]) or zero.
+    With one kv head nothing is shifted."""
+    S, Hkv, d = v_lat.shape
+    prev = np.zeros((1, Hkv, d)) if v_prev is None else v_prev[None]
+    shifted = np.concatenate([prev, v_lat[:-1]], axis=0)
+    out = v_lat.copy()
+    g0 = Hkv - Hkv // 2
+    out[:, g0:] = shifted[:, g0:]
     return out
 
 
@@ -238,10 +290,13 @@ class Layer:
     conv_q_chan: np.ndarray | None = None    # [Hq, d, d] or None = no channel mix
     conv_k_seq: np.ndarray | None = None     # [Hkv d, K]
     conv_k_chan: np.ndarray | None = None    # [Hkv, d, d]
-    qk_mean: bool = True
-    value_shift: bool = True
+    qk_mean: int = QK_CROSS                  # QK_OFF / QK_CROSS / QK_SELF (bools: off / cross)
+    value_shift: int = VS_HALF_CHANNELS      # VS_OFF / VS_HALF_CHANNELS / VS_WHOLE_HEADS
     rope_base: float = 10000.0
     causal: bool = True
+    # True: the temporal channel conv (channel_conv); conv_*_chan are then
+    # [H, K, d, d] per-tap matrices and conv_*_seq are unused
+    channel_conv: bool = False
 
 
 @dataclass
@@ -266,18 +321,33 @@ def _mix_qk(layer: Layer, q_pre, k_pre, hq=None, hk=None):
     sh = layer.sh
     T = q_pre.shape[0]
     d = sh.d
-    if layer.conv_width > 0:
+    if layer.conv_width > 0 and layer.channel_conv:
+        y_q = channel_conv(q_pre, layer.conv_q_chan, hq)
+        y_k = channel_conv(k_pre, layer.conv_k_chan, hk)
+    elif layer.conv_width > 0:
         u_q = seq_conv(q_pre.reshape(T, -1), layer.conv_q_seq, hq).reshape(T, sh.Hq, d)
         u_k = seq_conv(k_pre.reshape(T, -1), layer.conv_k_seq, hk).reshape(T, sh.Hkv, d)
         y_q = u_q if layer.conv_q_chan is None else channel_mix(u_q, layer.conv_q_chan)
         y_k = u_k if layer.conv_k_chan is None else channel_mix(u_k, layer.conv_k_chan)
     else:
         y_q, y_k = q_pre.copy(), k_pre.copy()
-    if layer.qk_mean:
+    if int(layer.qk_mean) == QK_SELF:
+        y_q, y_k = qk_mean_self(q_pre, y_q, k_pre, y_k)
+    elif layer.qk_mean:
         m_q, m_k = qk_mean(q_pre, k_pre, sh.G)
         y_q = y_q + m_q
         y_k = y_k + m_k
     return y_q, y_k
+
+
+def _shift_values(layer: Layer, v_lat, v_prev=None):
+    """Step a6 under the layer's value-shift reading."""
+    mode = int(layer.value_shift)
+    if mode == VS_WHOLE_HEADS:
+        return value_shift_heads(v_lat, v_prev)
+    if mode:
+        return value_shift(v_lat, v_prev)
+    return v_lat.copy()
 
 
 def prefill(layer: Layer, x: np.ndarray, rows: np.ndarray | None = None):
@@ -297,7 +367,7 @@ def prefill(layer: Layer, x: np.ndarray, rows: np.ndarray | None = None):
     pos = np.arange(S)
     q = rope(y_q, pos, layer.rope_base)
     k = rope(y_k, pos, layer.rope_base)
-    v = value_shift(v_lat) if layer.value_shift else v_lat.copy()
+    v = _shift_values(layer, v_lat)
     if rows is None:
         rows = pos
     rows = np.asarray(rows)
@@ -334,10 +404,7 @@ def decode_step(layer: Layer, state: State, x_t: np.ndarray):
     pos = np.array([t])
     q = rope(y_q, pos, layer.rope_base)
     k = rope(y_k, pos, layer.rope_base)
-    if layer.value_shift:
-        v = value_shift(v_lat, state.v_prev.reshape(sh.Hkv, sh.d))
-    else:
-        v = v_lat.copy()
+    v = _shift_values(layer, v_lat, state.v_prev.reshape(sh.Hkv, sh.d))
     k_all = np.concatenate([state.k, k], axis=0)
     v_all = np.concatenate([state.v, v], axis=0)
     o = attention(q, k_all, v_all, sh.G, layer.causal, q_pos=pos)

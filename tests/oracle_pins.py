@@ -448,26 +448,132 @@ def pin_layer_composition():
         _close(od, o[-1].reshape(-1), 1e-12, f"d={d} decode output")
 
 
+def pin_qk_mean_self_composition():
+    """The "self" QK-mean reading on the composition layer, written out by
+    hand: each head's output is the mean of its own pre-conv value and its
+    conv output, with no k term in q and no q term in k (CCA page,
+    Methodologie item 2, the literal reading)."""
+    r = _rng(23)
+    d, S = 4, 6
+    lay = _composition_layer(d, 0.0)
+    lay.qk_mean = O.QK_SELF
+    x = r.standard_normal((S, 4 * d))
+    qt = x[:, :2 * d].reshape(S, 2, d)
+    kt = x[:, 2 * d:3 * d].reshape(S, 1, d)
+
+    def conv_mix(z, t, h, i):          # lag 0 on even, 1 on odd channels, then y[i] = u[i+1]
+        j = (i + 1) % d
+        s_ = t - j % 2
+        return z[s_, h, j] if s_ >= 0 else 0.0
+
+    q = np.zeros((S, 2, d))
+    k = np.zeros((S, 1, d))
+    for t in range(S):
+        for i in range(d):
+            for h in range(2):
+                q[t, h, i] = 0.5 * (qt[t, h, i] + conv_mix(qt, t, h, i))
+            k[t, 0, i] = 0.5 * (kt[t, 0, i] + conv_mix(kt, t, 0, i))
+    _, st = O.prefill(lay, x)
+    _close(st.extra["q"], q, 1e-14, "self q")
+    _close(st.k, k, 1e-14, "self k")
+    _, st5 = O.prefill(lay, x[:-1])
+    _, nst = O.decode_step(lay, st5, x[-1])
+    _close(nst.extra["q"][0], q[-1], 1e-14, "self decode q")
+    _close(nst.k[-1], k[-1], 1e-14, "self decode k")
+
+
+def pin_value_shift_heads_gather():
+    """Whole-head value-shift: the last floor(Hkv/2) kv heads carry the
+    previous token's values, bit for bit (CCA page, Methodologie item 3, read
+    per head)."""
+    r = _rng(24)
+    for Hkv, shifted in ((4, {2, 3}), (3, {2}), (2, {1}), (1, set())):
+        S, d = 5, 6
+        v = r.standard_normal((S, Hkv, d))
+        prev = r.standard_normal((Hkv, d))
+        for vp in (None, prev):
+            out = O.value_shift_heads(v, vp)
+            for g in range(Hkv):
+                for t in range(S):
+                    if g in shifted:
+                        want = (prev[g] if vp is not None else np.zeros(d)) if t == 0 else v[t - 1, g]
+                    else:
+                        want = v[t, g]
+                    assert np.array_equal(out[t, g], want), (Hkv, g, t)
+
+
+def pin_channel_conv_closed_forms():
+    """The temporal channel conv: identity at tap 0, a cyclic channel
+    permutation at tap 1 (which a transposed matrix or reversed taps would
+    turn the other way), history rows, and a random two-tap case against
+    explicit loops."""
+    r = _rng(25)
+    S, H, d, K = 5, 2, 4, 3
+    z = r.standard_normal((S, H, d))
+    W = np.zeros((H, K, d, d))
+    W[:, 0] = np.eye(d)
+    _close(O.channel_conv(z, W), z, 0, "identity tap")
+    W = np.zeros((H, K, d, d))
+    for i in range(d):
+        W[:, 1, i, (i + 1) % d] = 1.0            # y[t, i] = z[t - 1, i + 1]
+    exp = np.zeros_like(z)
+    exp[1:] = np.roll(z[:-1], -1, axis=2)
+    _close(O.channel_conv(z, W), exp, 0, "shifted permutation")
+    hist = r.standard_normal((K - 1, H * d))
+    exp_h = exp.copy()
+    exp_h[0] = np.roll(hist[K - 2].reshape(H, d), -1, axis=1)   # row -1 is the newest history row
+    _close(O.channel_conv(z, W, hist), exp_h, 0, "history")
+    W = r.standard_normal((H, 2, d, d))
+    y = O.channel_conv(z, W)
+    for t in range(S):
+        for h in range(H):
+            for i in range(d):
+                acc = 0.0
+                for j in range(2):
+                    if t - j >= 0:
+                        for c in range(d):
+                            acc += W[h, j, i, c] * z[t - j, h, c]
+                assert abs(y[t, h, i] - acc) < 1e-12
+
+
+def _variant_layers():
+    """The reading variants: QK-mean "self", whole-head value-shift, and the
+    temporal channel conv (per-tap d x d matrices)."""
+    a = _small_layer()
+    a.qk_mean = O.QK_SELF
+    b = _small_layer(Hkv=2)
+    b.value_shift = O.VS_WHOLE_HEADS
+    c = _small_layer(seed=5)
+    r = _rng(26)
+    sh = c.sh
+    c.channel_conv = True
+    c.conv_q_chan = r.standard_normal((sh.Hq, 4, sh.d, sh.d)) / (2 * math.sqrt(sh.d))
+    c.conv_k_chan = r.standard_normal((sh.Hkv, 4, sh.d, sh.d)) / (2 * math.sqrt(sh.d))
+    c.conv_q_seq = c.conv_k_seq = None
+    return a, b, c
+
+
 def pin_causality():
     """Changing tokens after position t leaves outputs up to t unchanged
-    (covers the convolution, the value-shift and the mask)."""
-    lay = _small_layer()
-    r = _rng(13)
-    S = 12
-    x = r.standard_normal((S, lay.sh.E))
-    o1, _ = O.prefill(lay, x)
-    x2 = x.copy()
-    x2[7:] = r.standard_normal((S - 7, lay.sh.E))
-    o2, _ = O.prefill(lay, x2)
-    _close(o2[:7], o1[:7], 1e-13, "prefix unchanged")
-    assert np.max(np.abs(o2[7:] - o1[7:])) > 1e-3, "later rows must change"
+    (covers the convolution, the value-shift and the mask), for the default
+    readings and the variants."""
+    for lay in (_small_layer(), *_variant_layers()):
+        r = _rng(13)
+        S = 12
+        x = r.standard_normal((S, lay.sh.E))
+        o1, _ = O.prefill(lay, x)
+        x2 = x.copy()
+        x2[7:] = r.standard_normal((S - 7, lay.sh.E))
+        o2, _ = O.prefill(lay, x2)
+        _close(o2[:7], o1[:7], 1e-13, "prefix unchanged")
+        assert np.max(np.abs(o2[7:] - o1[7:])) > 1e-3, "later rows must change"
 
 
 def pin_decode_matches_prefill():
     """prefill over S tokens, row S-1 == prefill over S-1 tokens followed by one
     decode step; the decode state equals the longer prefill's state."""
     for lay in (_small_layer(), _small_layer(K=2, chan=False, qk=False),
-                _small_layer(K=0, qk=False, vs=False, base=0.0)):
+                _small_layer(K=0, qk=False, vs=False, base=0.0), *_variant_layers()):
         r = _rng(14)
         S = 10
         x = r.standard_normal((S, lay.sh.E))

@@ -12,7 +12,8 @@ import oracle_pins
 
 _orig = {name: getattr(O, name) for name in
          ("seq_conv", "channel_mix", "qk_mean", "rope", "value_shift", "attention",
-          "down_project", "prefill", "decode_step", "_mix_qk")}
+          "down_project", "prefill", "decode_step", "_mix_qk", "qk_mean_self",
+          "value_shift_heads", "channel_conv")}
 
 
 def _seq_conv_drop_last_tap(z, w, history=None):
@@ -172,6 +173,37 @@ def _prefill_rope_before_mean(layer, x, rows=None):
     return o.reshape(len(rows), -1), st
 
 
+def _qk_mean_self_no_half(q_pre, y_q, k_pre, y_k):
+    return q_pre + y_q, k_pre + y_k
+
+
+def _qk_mean_self_k_unchanged(q_pre, y_q, k_pre, y_k):
+    return 0.5 * (q_pre + y_q), y_k
+
+
+def _value_shift_heads_first(v, v_prev=None):
+    out = _orig["value_shift_heads"](v[:, ::-1].copy(), None if v_prev is None else v_prev[::-1].copy())
+    return out[:, ::-1].copy()
+
+
+def _value_shift_heads_ceil(v, v_prev=None):
+    S, Hkv, d = v.shape
+    prev = np.zeros((1, Hkv, d)) if v_prev is None else v_prev[None]
+    sh = np.concatenate([prev, v[:-1]], axis=0)
+    out = v.copy()
+    g0 = Hkv // 2
+    out[:, g0:] = sh[:, g0:]
+    return out
+
+
+def _channel_conv_transposed(z, W, history=None):
+    return _orig["channel_conv"](z, np.swapaxes(W, 2, 3), history)
+
+
+def _channel_conv_taps_reversed(z, W, history=None):
+    return _orig["channel_conv"](z, W[:, ::-1].copy(), history)
+
+
 MUTANTS = {
     "seq_conv_drop_last_tap": ("seq_conv", _seq_conv_drop_last_tap),
     "seq_conv_anticausal": ("seq_conv", _seq_conv_anticausal),
@@ -196,6 +228,12 @@ MUTANTS = {
     "qk_mean_of_post_conv": ("_mix_qk", _mix_qk_mean_of_post_conv),
     "channel_mix_before_conv": ("_mix_qk", _mix_qk_mix_before_conv),
     "rope_before_qk_mean": ("prefill", _prefill_rope_before_mean),
+    "qk_mean_self_no_half": ("qk_mean_self", _qk_mean_self_no_half),
+    "qk_mean_self_k_unchanged": ("qk_mean_self", _qk_mean_self_k_unchanged),
+    "value_shift_heads_first": ("value_shift_heads", _value_shift_heads_first),
+    "value_shift_heads_ceil": ("value_shift_heads", _value_shift_heads_ceil),
+    "channel_conv_transposed": ("channel_conv", _channel_conv_transposed),
+    "channel_conv_taps_reversed": ("channel_conv", _channel_conv_taps_reversed),
 }
 
 
