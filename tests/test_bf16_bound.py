@@ -40,6 +40,27 @@ def test_model_meets_the_bound_it_sets(name):
     lay = oracle_layer(w, inp)
     x = f64(inp["x"][0])
     ref, _ = O.prefill(lay, x)
-    model, _ = model_prefill(lay, x)
-    l2, _ = check_bf16(model, ref, model, name)
+    model, mst = model_prefill(lay, x)
+    l2, _ = check_bf16(model, ref, model, mst.extra["spread"], name)
     assert l2 < 1e-2
+
+
+def test_elementwise_bound_catches_a_localised_error():
+    """A kernel error confined to a few elements (one head at a run of
+    positions, say a wrong diagonal tile) hides inside the global bounds (a)
+    and (b) but not inside the per-element bound (c)."""
+    import bf16_model as M
+    w = CASES["d64"]
+    inp = make_inputs(w, seed=0)
+    lay = oracle_layer(w, inp)
+    x = f64(inp["x"][0])
+    ref, _ = O.prefill(lay, x)
+    model, mst = model_prefill(lay, x)
+    rms = np.sqrt(np.mean(ref ** 2))
+    bad = model.copy()
+    bad[300:310, 64:128] += 3e-2 * rms        # head 1, ten positions
+    d = np.abs(bad - ref)
+    assert np.linalg.norm(bad - ref) / np.linalg.norm(ref) <= M.L2_TOL                 # (a) passes
+    assert d.max() <= M.ABS_TOL * rms + M.MODEL_SLACK * np.abs(model - ref).max()  # (b) passes
+    with pytest.raises(AssertionError, match="element"):
+        check_bf16(bad, ref, model, mst.extra["spread"], "planted")
