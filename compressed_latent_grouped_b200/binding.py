@@ -27,7 +27,7 @@ class ccgqa_config(ctypes.Structure):
     _fields_ = [("E", c_int32), ("C", c_int32), ("n_q_heads", c_int32), ("n_kv_heads", c_int32),
                 ("conv_width", c_int32), ("qk_mean", c_int32), ("value_shift", c_int32),
                 ("causal", c_int32), ("rope_base", c_double), ("dtype", c_int32),
-                ("reserved", c_int32)]
+                ("channel_conv", c_int32)]
 
 
 class ccgqa_weights(ctypes.Structure):
@@ -140,9 +140,11 @@ def _stream(stream=None):
 
 
 def make_config(E, C, n_q_heads, n_kv_heads, conv_width=4, qk_mean=1, value_shift=1, causal=1,
-                rope_base=10000.0, dtype=BF16) -> ccgqa_config:
+                rope_base=10000.0, dtype=BF16, channel_conv=0) -> ccgqa_config:
+    """qk_mean: 0 off, 1 cross, 2 self; value_shift: 0 off, 1 half channels,
+    2 whole heads; channel_conv: 1 for per-tap d x d matrices."""
     return ccgqa_config(E, C, n_q_heads, n_kv_heads, conv_width, int(qk_mean), int(value_shift),
-                        int(causal), float(rope_base), dtype, 0)
+                        int(causal), float(rope_base), dtype, int(channel_conv))
 
 
 def make_weights(W_qkv=None, conv_q_seq=None, conv_q_chan=None, conv_k_seq=None,

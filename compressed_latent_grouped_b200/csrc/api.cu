@@ -66,7 +66,7 @@ namespace {
 
 struct Geo {
   int E, C, Hq, Hkv, d, G, N, K;
-  int qk_mean, value_shift, causal, rope_on;
+  int qk_mean, value_shift, causal, rope_on, channel_conv;
   double rope_log2_base;
   int dtype;
   size_t es;  // element size
@@ -83,7 +83,6 @@ uint64_t rope_turn_fraction(double log2_base, int i, int d) {
   return static_cast<uint64_t>(llroundl(th / two_pi * 18446744073709551616.0L));
 }
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
-bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
 ccgqa_status derive(const ccgqa_config* cfg, Geo* g) {
   if (!cfg) return CCGQA_ERR_INVALID_ARG;
@@ -92,7 +91,10 @@ ccgqa_status derive(const ccgqa_config* cfg, Geo* g) {
   if (cfg->n_q_heads % cfg->n_kv_heads != 0) return CCGQA_ERR_INVALID_ARG;
   if (cfg->E % (cfg->C * cfg->n_q_heads) != 0) return CCGQA_ERR_INVALID_ARG;
   if (cfg->conv_width < 0 || cfg->conv_width > 4) return CCGQA_ERR_INVALID_ARG;
-  if ((cfg->qk_mean | cfg->value_shift | cfg->causal) & ~1) return CCGQA_ERR_INVALID_ARG;
+  if (cfg->qk_mean < 0 || cfg->qk_mean > 2 || cfg->value_shift < 0 || cfg->value_shift > 2 ||
+      (cfg->causal & ~1) || (cfg->channel_conv & ~1))
+    return CCGQA_ERR_INVALID_ARG;
+  if (cfg->channel_conv && cfg->conv_width == 0) return CCGQA_ERR_INVALID_ARG;
   if (!(cfg->rope_base >= 0.0) || std::isinf(cfg->rope_base)) return CCGQA_ERR_INVALID_ARG;
   if (cfg->dtype != CCGQA_F32 && cfg->dtype != CCGQA_BF16) return CCGQA_ERR_INVALID_ARG;
   g->E = cfg->E;
@@ -106,21 +108,25 @@ ccgqa_status derive(const ccgqa_config* cfg, Geo* g) {
   g->qk_mean = cfg->qk_mean;
   g->value_shift = cfg->value_shift;
   g->causal = cfg->causal;
+  g->channel_conv = cfg->channel_conv;
   g->rope_on = cfg->rope_base > 0.0;
   g->rope_log2_base = g->rope_on ? std::log2(cfg->rope_base) : 0.0;
   g->dtype = cfg->dtype;
   g->es = cfg->dtype == CCGQA_F32 ? 4 : 2;
   if (g->d != 16 && g->d != 32 && g->d != 64 && g->d != 128) return CCGQA_ERR_UNSUPPORTED;
-  if (g->dtype == CCGQA_BF16 && (g->d < 32 || !pow2(g->G) || g->G > 128))
-    return CCGQA_ERR_UNSUPPORTED;
-  if (g->G * (g->d * static_cast<int>(g->es) / 16) > 128) return CCGQA_ERR_UNSUPPORTED;
+  // the per-sequence decode pre-step stages (G + 2) d channels in shared memory
+  if (!decode_pre_fits(g->G, g->d, g->K, static_cast<int>(g->es))) return CCGQA_ERR_UNSUPPORTED;
   return CCGQA_OK;
 }
 
 ccgqa_status check_weights(const Geo& g, const ccgqa_weights* w) {
   if (!w) return CCGQA_ERR_INVALID_ARG;
   if (w->W_qkv && !aligned16(w->W_qkv)) return CCGQA_ERR_INVALID_ARG;
-  if (g.K > 0) {
+  if (g.K > 0 && g.channel_conv) {
+    // per-tap matrices only: [Hq, K, d, d] and [Hkv, K, d, d]
+    if (!w->conv_q_chan || !w->conv_k_chan) return CCGQA_ERR_INVALID_ARG;
+    if (!aligned16(w->conv_q_chan) || !aligned16(w->conv_k_chan)) return CCGQA_ERR_INVALID_ARG;
+  } else if (g.K > 0) {
     if (!w->conv_q_seq || !w->conv_k_seq) return CCGQA_ERR_INVALID_ARG;
     if (!aligned16(w->conv_q_seq) || !aligned16(w->conv_k_seq)) return CCGQA_ERR_INVALID_ARG;
     if ((w->conv_q_chan && !aligned16(w->conv_q_chan)) ||
@@ -183,6 +189,11 @@ DecodeWs decode_ws(const Geo& g, int64_t B, int64_t cap, bool has_proj) {
   return w;
 }
 
+// The tensor-core attention covers d >= 32 and groups of at most 128 heads (a
+// query tile packs floor(128 / G) positions of the G heads); d = 16 and larger
+// groups run on the CUDA-core kernel.
+bool attn_tc_applies(const Geo& g) { return g.d >= 32 && g.G <= 128; }
+
 template <typename T>
 ccgqa_status run_prefill(const Geo& g, const ccgqa_weights* w, const void* x, int B, int S,
                          void* out, const ccgqa_kvcache* cache, uint8_t* ws, int32_t* dev_err,
@@ -215,6 +226,7 @@ ccgqa_status run_prefill(const Geo& g, const ccgqa_weights* w, const void* x, in
   a.K = g.K;
   a.qk_mean = g.qk_mean;
   a.value_shift = g.value_shift;
+  a.channel_conv = g.channel_conv;
   a.rope_on = g.rope_on;
   a.rope_log2_base = g.rope_log2_base;
   if (g.rope_on)
@@ -254,10 +266,14 @@ ccgqa_status run_prefill(const Geo& g, const ccgqa_weights* w, const void* x, in
   at.kv_cap = a.kv_cap;
   at.causal = g.causal;
   at.dev_err = dev_err;
-  if constexpr (sizeof(T) == 2)
-    e = launch_attn_prefill_tc(at, st);
-  else
+  if constexpr (sizeof(T) == 2) {
+    if (attn_tc_applies(g))
+      e = launch_attn_prefill_tc(at, st);
+    else
+      e = launch_attn_prefill_simt<T>(at, st);
+  } else {
     e = launch_attn_prefill_simt<T>(at, st);
+  }
   phase_mark(3, st);
   return e == cudaSuccess ? CCGQA_OK : cuda_fail(e);
 }
@@ -280,6 +296,7 @@ ccgqa_status run_decode(const Geo& g, const ccgqa_weights* w, const void* x_t,
   a.K = g.K;
   a.qk_mean = g.qk_mean;
   a.value_shift = g.value_shift;
+  a.channel_conv = g.channel_conv;
   a.causal = g.causal;
   a.rope_on = g.rope_on;
   a.rope_log2_base = g.rope_log2_base;
@@ -379,6 +396,11 @@ CCGQA_API ccgqa_status ccgqa_prefill(const ccgqa_config* cfg, const ccgqa_weight
     if (cache->batch != batch) return CCGQA_ERR_INVALID_ARG;
     if (seq_len > cache->cap) return CCGQA_ERR_CAPACITY;
   }
+  // the CUDA-core pre-attention kernel must fit its smallest staging layout
+  // (the tensor-core one checks its own layout and otherwise falls back here)
+  if (!pre_attn_fits(g.K, g.G, g.d, static_cast<int>(g.es),
+                     g.K > 0 && !g.channel_conv && (w->conv_q_chan || w->conv_k_chan)))
+    return CCGQA_ERR_UNSUPPORTED;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) ||
       workspace_bytes < prefill_ws(g, batch, seq_len).total)
     return CCGQA_ERR_WORKSPACE;

@@ -6,6 +6,9 @@
 // Query rows are packed per kv group: row r of a tile is position
 // t0 + r / G, head g*G + r % G, so a 5-D TMA box gathers a tile straight from
 // q[B, S, Hq, d] and one K/V tile in shared memory serves all G query heads.
+// A tile holds floor(128 / G) positions; when G does not divide 128 (the
+// kPow2 = false instantiation) the last 128 mod G rows are zeroed once and
+// never stored.
 //
 // One CTA owns T consecutive 128-row query tiles of one kv group (T = 3 at
 // d = 32, else 2) and streams the K/V tiles they need once, as 128-key tiles
@@ -29,6 +32,7 @@
 // warpgroup never waits for the PV -> S round trip; the two warpgroups keep
 // the exp unit and the FMA pipe busy while the tensor core runs their MMAs.
 // TMEM: S/P of tile x at columns 128 x + {0, 64}, O_x at 128 T + x d.
+
 // No cluster multicast is used; every wait is bounded.
 #include "kernels.h"
 #include "sm100.cuh"
@@ -58,7 +62,7 @@ struct Cfg {
   // Query tiles per CTA: three where their S buffers and accumulators fit
   // in TMEM (3 x 128 + 3 x 32 columns at d = 32), else two.
   static constexpr int kTiles = (D == 32) ? 3 : 2;
-  static constexpr int kSoftEvery = (D == 64) ? 3 : 4;
+  static constexpr int kSoftEvery = (D == 64) ? 3 : (D == 32 ? 5 : 4);
   static constexpr int kThreads = 128 + 128 * kTiles;   // 4 control warps + softmax
   static constexpr uint32_t kOffQ = 0;                        // Q_A, Q_B
   static constexpr uint32_t kOffK = kTiles * kTileBytes;
@@ -66,6 +70,7 @@ struct Cfg {
   static constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
   static constexpr size_t kSmem = kOffBar + 256 + 1024;
   static constexpr uint32_t kTmemCols = 512;
+  static_assert(kTiles * 128 + kTiles * D <= 512, "S buffers and accumulators exceed TMEM");
   // S buffer h of tile x, its P (upper 32 columns: 64 keys as bf16 pairs), O_x
   __device__ static constexpr uint32_t col_s(int x, int h) { return x * 128 + h * 64; }
   __device__ static constexpr uint32_t col_p(int x, int h) { return x * 128 + h * 64 + 32; }
@@ -102,7 +107,11 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
 // low mantissa bits), 2^f from a degree-3 polynomial fitted for this kernel
 // (relative error below 8e-5, well under bf16's 2^-9), and 2^n added to the
 // exponent field.  Inputs are clamped at -126 (the exponent field of p,
-// 126 or 127, must stay positive after adding n), so -inf gives ~1e-38.
+// 126 or 127, must stay positive after adding n), so -inf gives ~1e-38.  An
+// input of kSoftArgMax or more would carry the exponent field past its top, so
+// the caller tracks the largest input (one 3-input max per pair) and redoes
+// the half against a raised running max when it gets there.
+constexpr float kSoftArgMax = 127.0f;
 __device__ __forceinline__ float2 soft_exp2x2(float2 x) {
   x.x = fmaxf(x.x, -126.0f);
   x.y = fmaxf(x.y, -126.0f);
@@ -117,23 +126,31 @@ __device__ __forceinline__ float2 soft_exp2x2(float2 x) {
                      __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Pairs (c2 % Cfg<D>::kSoftEvery == 0) of each softmax row use the software
 // exp2, so the FMA pipe takes part of the exponentials off the exp unit.
-// Measured on B200: one pair in 3 is best at d = 64 (1.445 ms against 1.514 ms
-// for 1 in 4 on S = 32768), one in 4 at d = 32 and d = 128.
+// Measured on B200: one pair in 3 is best at d = 64 (1.47 ms against 1.50 ms
+// for 1 in 4 and 1.56 ms for 1 in 2 on S = 32768), one in 5 at d = 32 (174 us
+// against 180 us for 1 in 4 and 177 us for 1 in 6 on 4 x 4096), one in 4 at
+// d = 128.
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h2 = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h2);
 }
 
-template <int D>
+template <int D, bool kPow2>
 __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                            const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, bf16* __restrict__ out,
-                           int B, int S, int Hq, int Hkv, int G_log2, int n_groups, int causal,
-                           int32_t* dev_err) {
+                           int B, int S, int Hq, int Hkv, int G, int G_log2, int n_groups,
+                           int causal, int32_t* dev_err) {
   pdl_enter();
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -151,12 +168,12 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int G = 1 << G_log2;
   const int BH = B * Hkv;
   const int grp = n_groups - 1 - static_cast<int>(blockIdx.x) / BH;  // longest first
   const int bg = static_cast<int>(blockIdx.x) % BH;
   const int b = bg / Hkv, g = bg % Hkv;
-  const int pos_per_tile = kBlockM >> G_log2;
+  const int pos_per_tile = kPow2 ? (kBlockM >> G_log2) : kBlockM / G;
+  const int rows_used = pos_per_tile * G;     // rows of a tile the Q box fills
   const int t0 = grp * C::kTiles * pos_per_tile;
   const int t_last = min(t0 + C::kTiles * pos_per_tile - 1, S - 1);
   const int n_kv = causal ? (t_last / kBlockN + 1) : (S + kBlockN - 1) / kBlockN;
@@ -176,6 +193,17 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     abort_flag = 0;
     fence_barrier_init();
   }
+  if (!kPow2 && rows_used < kBlockM) {
+    // Rows the Q box does not fill (G does not divide 128): zero them so their
+    // scores are finite; the MMA reads them through the async proxy.
+    const int n16 = (kBlockM - rows_used) * C::kRowBytes / 16;
+    for (int i = threadIdx.x; i < C::kTiles * C::kPanels * n16; i += blockDim.x) {
+      const int tp = i / n16, w = i % n16;
+      *reinterpret_cast<uint4*>(smem + C::kOffQ + tp * C::kPanelBytes + rows_used * C::kRowBytes +
+                                w * 16) = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
@@ -191,7 +219,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
-      mbar_arrive_expect_tx(q_full, C::kTiles * C::kTileBytes);
+      mbar_arrive_expect_tx(q_full, C::kTiles * rows_used * D * 2);
 #pragma unroll
       for (int x = 0; x < C::kTiles; ++x)
 #pragma unroll
@@ -290,8 +318,9 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     const int x = (warp - 4) >> 2;                // query tile of this warpgroup
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;                 // tile row == TMEM lane
-    const int t = t0 + x * pos_per_tile + (r >> G_log2);
-    const int hl = r & (G - 1);
+    const int t = t0 + x * pos_per_tile + (kPow2 ? (r >> G_log2) : r / G);
+    const int hl = kPow2 ? (r & (G - 1)) : r % G;
+    const bool row_ok = kPow2 || r < rows_used;   // a row the Q box filled
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const float scale = kLog2e * rsqrtf(static_cast<float>(D));
     const float2 scale2 = make_float2(scale, scale);
@@ -330,17 +359,21 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
           return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * scale;
         };
         uint32_t pk[32];
-        // p = 2^(s * scale - m_used) as bf16 pairs; returns the row's sum of p
+        // p = 2^(s * scale - m_used) as bf16 pairs; returns the row's sum of p,
+        // or +inf when an argument of the software exp2 passed its range (the
+        // overflow the exp unit shows as inf): either way the half is redone
         auto exp_pass = [&](const float (&sv)[64]) {
           const float2 negm2 = make_float2(-m_used, -m_used);
           const float2* s2 = reinterpret_cast<const float2*>(sv);
           float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                             make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+          float soft_max = -INFINITY;
 #pragma unroll
           for (int c2 = 0; c2 < 32; ++c2) {
             const float2 arg = ffma2(s2[c2], scale2, negm2);
             float2 p;
             if ((c2 % C::kSoftEvery) == 0) {
+              soft_max = fmax3(soft_max, arg.x, arg.y);
               p = soft_exp2x2(arg);
             } else {
               p.x = fast_exp2(arg.x);
@@ -350,7 +383,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
             pk[c2] = pack_bf16x2(p.x, p.y);
           }
           const float2 a2 = fadd2(fadd2(lsum[0], lsum[1]), fadd2(lsum[2], lsum[3]));
-          return a2.x + a2.y;
+          return soft_max < kSoftArgMax ? a2.x + a2.y : INFINITY;
         };
         // The first half sets the running max (key 0 is visible to every
         // row, so it is finite).  Later halves exponentiate against the
@@ -412,7 +445,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     if (ok && n_kv > 0 && mbar_wait(&o_done[x * 2 + 1], (n_kv - 1) & 1, &abort_flag, dev_err)) {
       tc_fence_after();
       const float inv_l = 1.f / l;
-      const bool store = t < S;
+      const bool store = row_ok && t < S;
       bf16* dst = out + ((static_cast<int64_t>(b) * S + t) * Hq + g * G + hl) * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
@@ -454,8 +487,6 @@ cudaError_t launch_d(const AttnArgs& a, cudaStream_t stream) {
   using C = Cfg<D>;
   const CUtensorMapSwizzle swz =
       (D == 32) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
-  int G_log2 = 0;
-  while ((1 << G_log2) < a.G) ++G_log2;
   CUtensorMap tmQ, tmK, tmV;
   {
     // q[B, S, Hq, d] viewed as (d, G, Hkv, S, B): a box (panel, G, 1, 128/G, 1)
@@ -482,15 +513,19 @@ cudaError_t launch_d(const AttnArgs& a, cudaStream_t stream) {
         !encode_tensor_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.v, dims, st, box, swz))
       return cudaErrorInvalidValue;
   }
-  const int rows_per_cta = C::kTiles * kBlockM;
-  const int n_groups = (a.S * a.G + rows_per_cta - 1) / rows_per_cta;
+  if (a.G < 1 || a.G > kBlockM) return cudaErrorInvalidValue;
+  const int pos_per_cta = C::kTiles * (kBlockM / a.G);
+  const int n_groups = (a.S + pos_per_cta - 1) / pos_per_cta;
   const int grid = n_groups * a.B * a.Hkv;
-  cudaError_t e = allow_smem(reinterpret_cast<const void*>(attn_prefill_tc_kernel<D>),
-                                       static_cast<int>(C::kSmem));
+  int G_log2 = 0;
+  while ((1 << G_log2) < a.G) ++G_log2;
+  const bool pow2 = (1 << G_log2) == a.G;
+  auto kernel = pow2 ? attn_prefill_tc_kernel<D, true> : attn_prefill_tc_kernel<D, false>;
+  cudaError_t e = allow_smem(reinterpret_cast<const void*>(kernel), static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
-  const cudaError_t el = launch_pdl(attn_prefill_tc_kernel<D>, dim3(grid), dim3(C::kThreads),
-                                    C::kSmem, stream, tmQ, tmK, tmV, static_cast<bf16*>(a.out),
-                                    a.B, a.S, a.Hq, a.Hkv, G_log2, n_groups, a.causal, a.dev_err);
+  const cudaError_t el = launch_pdl(kernel, dim3(grid), dim3(C::kThreads), C::kSmem, stream, tmQ,
+                                    tmK, tmV, static_cast<bf16*>(a.out), a.B, a.S, a.Hq, a.Hkv,
+                                    a.G, G_log2, n_groups, a.causal, a.dev_err);
   count_launches(1);
   return el != cudaSuccess ? el : cudaGetLastError();
 }

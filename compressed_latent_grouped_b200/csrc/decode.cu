@@ -36,7 +36,11 @@ static bool decode_use_gemv(int B, int E, int es) {
 }
 // More sequences, bf16: the projection on the tensor core, swapped (W rows as M),
 // one CTA per (128 W rows, 64 sequences, 128 of E).
-constexpr int kDpN = 128, kDpB = 64, kDpK = 128;
+// Tensor-core decode projection tiles: 128 W rows x 64 sequences x 128 of E
+// (2 blocks of 64, both staged in one round of TMA).  Measured at 64 sequences,
+// E = 4096: 512 of E per CTA (48 CTAs, a quarter of the partials) took 13.6 us
+// against 12.8 us; the pre-step summing fewer partials gained under 1 us.
+constexpr int kDpN = 128, kDpB = 64, kDpK = 128, kDpKB = kDpK / 64;
 static bool decode_use_proj_tc(int E, int es) { return es == 2 && E % kDpK == 0; }
 
 // E range of one projection split: E / e_splits rounded up to whole 64-wide steps.
@@ -51,7 +55,7 @@ void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int e
   if (has_proj && decode_use_gemv(B, E, es)) {
     *e_splits = 1;   // one weight-streaming pass, no partials to sum
   } else if (has_proj && decode_use_proj_tc(E, es)) {
-    *e_splits = E / kDpK;   // tensor-core tiles of 128 columns x 64 sequences x 128 of E
+    *e_splits = E / kDpK;   // tensor-core tiles of 128 columns x 64 sequences x kDpK of E
   } else if (has_proj) {
     // projection CTAs: 64 columns x 64 sequences x one E-split of whole 64-wide steps
     const int tiles = ((N + 63) / 64) * ((B + 63) / 64);
@@ -317,13 +321,14 @@ cudaError_t launch_gemv(const T* x, const T* W, float* out, int B, int E, int N,
   return go(decode_gemv_kernel<T, 16>);
 }
 
-// part[s][b][n] = sum over k in [128 s, 128 s + 128) of W[n][k] x[b][k] on the
-// tensor core: D^T = W_tile x_tile^T with M = 128 W rows, N = 64 sequences
-// (rows past B read as zero), K = 128 in 8 steps.  Both tiles arrive by TMA in
-// one round (128B swizzle); one thread issues the MMAs; four warps read the
-// accumulator back (lane = W row) and store fp32 partials, lanes over columns.
+// part[s][b][n] = sum over k in [kDpK s, kDpK (s + 1)) of W[n][k] x[b][k] on
+// the tensor core: D^T = W_tile x_tile^T with M = 128 W rows, N = 64 sequences
+// (rows past B read as zero), K = kDpK in steps of 16.  All 64-wide blocks of
+// both tiles arrive by TMA in one round (128B swizzle), so a CTA costs one
+// memory latency; one thread issues the MMAs; four warps read the accumulator
+// back (lane = W row) and store fp32 partials, lanes over columns.
 constexpr uint32_t kDpATile = kDpN * 64 * 2, kDpBTile = kDpB * 64 * 2;
-constexpr size_t kDpSmem = 2 * (kDpATile + kDpBTile) + 64 + 1024;
+constexpr size_t kDpSmem = kDpKB * (kDpATile + kDpBTile) + 64 + 1024;
 
 __global__ void __launch_bounds__(128)
     decode_proj_tc_kernel(const __grid_constant__ CUtensorMap tmW,
@@ -333,9 +338,9 @@ __global__ void __launch_bounds__(128)
   extern __shared__ uint8_t dp_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dp_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sa = smem;                          // [2][128 x 64] W blocks
-  uint8_t* sb = smem + 2 * kDpATile;           // [2][64 x 64] x blocks
-  uint64_t* full = reinterpret_cast<uint64_t*>(sb + 2 * kDpBTile);
+  uint8_t* sa = smem;                          // [kDpKB][128 x 64] W blocks
+  uint8_t* sb = smem + kDpKB * kDpATile;       // [kDpKB][64 x 64] x blocks
+  uint64_t* full = reinterpret_cast<uint64_t*>(sb + kDpKB * kDpBTile);
   uint64_t* done = full + 1;
   uint64_t* drain = done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -361,9 +366,9 @@ __global__ void __launch_bounds__(128)
   if (tid == 0) {
     prefetch_tensormap(&tmW);
     prefetch_tensormap(&tmX);
-    mbar_arrive_expect_tx(full, 2 * (kDpATile + kDpBTile));
+    mbar_arrive_expect_tx(full, kDpKB * (kDpATile + kDpBTile));
 #pragma unroll
-    for (int kb = 0; kb < 2; ++kb) {
+    for (int kb = 0; kb < kDpKB; ++kb) {
       tma_load_2d(sa + kb * kDpATile, &tmW, full, e0 + kb * 64, n0);
       tma_load_2d(sb + kb * kDpBTile, &tmX, full, e0 + kb * 64, b0);
     }
@@ -371,7 +376,7 @@ __global__ void __launch_bounds__(128)
       tc_fence_after();
       const uint32_t idesc = make_idesc_bf16(kDpN, kDpB, false);
 #pragma unroll
-      for (int kb = 0; kb < 2; ++kb)
+      for (int kb = 0; kb < kDpKB; ++kb)
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const uint64_t ad = make_smem_desc(smem_addr(sa + kb * kDpATile) + k * 32, 16, 1024,
@@ -507,7 +512,9 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
     return;
   }
   const int qcol0 = g * G * d, kcol0 = a.Hq * d + g * d, vcol0 = (a.Hq + a.Hkv) * d + g * d;
-  const bool have_mix = K > 0 && a.wq_chan != nullptr && a.wk_chan != nullptr;
+  // temporal channel conv: per-tap d x d matrices (wq_chan [Hq, K, d, d]), no depthwise taps
+  const bool full = a.channel_conv && K > 0;
+  const bool have_mix = K > 0 && !full && a.wq_chan != nullptr && a.wk_chan != nullptr;
   // 1. every input in one round of memory latency: the weights, taps and
   // history rows by 16-byte cp.async (contiguous per group), the projection
   // partials summed meanwhile
@@ -520,7 +527,7 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
       copy(wraw, a.wq_chan + static_cast<int64_t>(g) * G * d * d, G * d * d);
       copy(wraw + G * d * d, a.wk_chan + static_cast<int64_t>(g) * d * d, d * d);
     }
-    if (K > 0) {
+    if (K > 0 && !full) {
       copy(tr, a.wq_seq + static_cast<int64_t>(g) * G * d * K, G * d * K);
       copy(tr + G * d * K, a.wk_seq + static_cast<int64_t>(g) * d * K, d * K);
     }
@@ -558,7 +565,7 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
   __syncthreads();
   // 2. shared-memory reshuffles: taps to fp32 [HC][4]; mix weights transposed,
   // wt[hh][j][i] = W_hh[i][j] (lanes run over rows i: consecutive stores)
-  for (int idx = tid; idx < HC * 4; idx += blockDim.x) {
+  for (int idx = tid; !full && idx < HC * 4; idx += blockDim.x) {
     const int c = idx >> 2, j = idx & 3;
     tp[idx] = j < K ? to_f32(tr[c * K + j]) : 0.f;
   }
@@ -579,7 +586,7 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
   // causal conv: tap j reads the row j steps back (history row KH - j)
   for (int c = tid; c < HC; c += blockDim.x) {
     float acc;
-    if (K > 0) {
+    if (K > 0 && !full) {
       const float* w = tp + c * 4;
       acc = w[0] * zc[c];
       for (int j = 1; j < K; ++j) acc = fmaf(w[j], to_f32(hz[(KH - j) * HC + c]), acc);
@@ -595,7 +602,23 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
     const int hh = c / d, i = c - hh * d;
     const T* wch = is_q ? a.wq_chan : a.wk_chan;
     float acc;
-    if (K > 0 && wch && stage_wt && have_mix) {
+    if (full) {
+      // y[i] = sum_k sum_j W_k[i][j] z[t - k, j]; row t - k is history row KH - k
+      const int head = is_q ? g * G + hh : g;
+      const T* wh = wch + static_cast<int64_t>(head) * K * d * d + static_cast<int64_t>(i) * d;
+      acc = 0.f;
+      for (int k = 0; k < K; ++k) {
+        const T* wr = wh + static_cast<int64_t>(k) * d * d;
+        if (k == 0) {
+#pragma unroll 8
+          for (int j = 0; j < d; ++j) acc = fmaf(to_f32(wr[j]), zc[hh * d + j], acc);
+        } else {
+          const T* zr = hz + (KH - k) * HC + hh * d;
+#pragma unroll 8
+          for (int j = 0; j < d; ++j) acc = fmaf(to_f32(wr[j]), to_f32(zr[j]), acc);
+        }
+      }
+    } else if (K > 0 && wch && stage_wt && have_mix) {
       const T* wc = wt + static_cast<int64_t>(hh) * d * d + i;   // column i of W_hh^T
       acc = 0.f;
 #pragma unroll 8
@@ -608,7 +631,9 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
     } else {
       acc = u[c];
     }
-    if (a.qk_mean) {
+    if (a.qk_mean == 2) {
+      acc = 0.5f * (acc + zc[c]);   // "self": the head's own pre-conv value
+    } else if (a.qk_mean) {
       float qp;
       if (is_q) {
         qp = zc[c];
@@ -646,9 +671,11 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
       a.cache_k[crow + i + half] = from_f32<T>(yb);
     }
   }
+  const bool shift_head = a.value_shift == 2 && g >= a.Hkv - a.Hkv / 2;
   for (int i = tid; i < d; i += blockDim.x) {
     T v = from_f32<T>(zc[HC + i]);
-    if (a.value_shift && i >= half) v = a.v_prev[static_cast<int64_t>(b) * a.Hkv * d + g * d + i];
+    if ((a.value_shift == 1 && i >= half) || shift_head)
+      v = a.v_prev[static_cast<int64_t>(b) * a.Hkv * d + g * d + i];
     a.cache_v[crow + i] = v;
   }
   __syncthreads();
@@ -686,6 +713,13 @@ struct DecCfg {
   static constexpr uint32_t kStageBytes = 2u * KS * D * sizeof(T);
 };
 
+// CTAs per (split, kv group): each takes at most 32 kPPMax (head, chunk) pairs.
+template <typename T, int D>
+__host__ __device__ inline int dec_head_chunks(int G) {
+  constexpr int per = 32 * kPPMax / DecCfg<T, D>::NCH;   // heads per CTA
+  return (G + per - 1) / per;
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kDecThreads)
     decode_attn_kernel(const DecodeArgs<T> a) {
@@ -697,8 +731,12 @@ __global__ void __launch_bounds__(kDecThreads)
   float* wbuf = reinterpret_cast<float*>(full + kDecStages);  // merge scratch
   __shared__ int abort_flag, last_flag;
 
-  const int sp = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int G = a.G, P = G * C::NCH;
+  // blockIdx.y = kv group x head chunk: a CTA serves at most 32 kPPMax / NCH
+  // of the group's G query heads (heads hc0 .. hc0 + Gc - 1)
+  const int n_hc = dec_head_chunks<T, D>(a.G);
+  const int sp = blockIdx.x, g = blockIdx.y / n_hc, hc = blockIdx.y % n_hc, b = blockIdx.z;
+  const int G = a.G, Gmax = (G + n_hc - 1) / n_hc, hc0 = hc * Gmax;
+  const int Gc = min(Gmax, G - hc0), P = Gc * C::NCH;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
   const int L = __ldcg(a.len + b);
   const bool valid_b = L >= 0 && L < a.cap;
@@ -742,7 +780,7 @@ __global__ void __launch_bounds__(kDecThreads)
 #pragma unroll
     for (int e = 0; e < C::CH; ++e) {
       o[kk][e] = 0.f;
-      qr[kk][e] = (p < P) ? a.q_ws[(static_cast<int64_t>(b) * a.Hq + g * G + h) * D +
+      qr[kk][e] = (p < P) ? a.q_ws[(static_cast<int64_t>(b) * a.Hq + g * G + hc0 + h) * D +
                                    chunk * C::CH + e] *
                                 scale
                           : 0.f;
@@ -819,7 +857,7 @@ __global__ void __launch_bounds__(kDecThreads)
     for (int e = 0; e < C::CH; ++e) wo[(warp * P + p) * C::CH + e] = o[kk][e];
   }
   __syncthreads();
-  const int64_t pbase = ((static_cast<int64_t>(b) * a.Hkv + g) * a.splits + sp) * G;
+  const int64_t pbase = ((static_cast<int64_t>(b) * a.Hkv + g) * a.splits + sp) * G + hc0;
   for (int p = tid; p < P; p += kDecThreads) {
     float M = -INFINITY;
     for (int w = 0; w < 4; ++w) M = fmaxf(M, wm[w * P + p]);
@@ -844,7 +882,7 @@ __global__ void __launch_bounds__(kDecThreads)
   __syncthreads();
   if (tid == 0) {
     const int prev = atomicAdd(a.tickets + b * a.Hkv + g, 1);
-    last_flag = (prev == a.splits - 1);
+    last_flag = (prev == a.splits * n_hc - 1);
   }
   __syncthreads();
   if (!last_flag) return;
@@ -889,20 +927,19 @@ __global__ void __launch_bounds__(kDecThreads)
 template <typename T, int D>
 size_t dec_attn_smem(int G) {
   using C = DecCfg<T, D>;
-  const int P = G * C::NCH;
+  const int n_hc = dec_head_chunks<T, D>(G);
+  const int P = (G + n_hc - 1) / n_hc * C::NCH;
   return 128 + kDecStages * C::kStageBytes + kDecStages * 8 +
          static_cast<size_t>(4 * P * (2 + C::CH)) * 4 + 16;
 }
 
 template <typename T, int D>
 cudaError_t launch_dec_attn(const DecodeArgs<T>& a, cudaStream_t stream) {
-  using C = DecCfg<T, D>;
-  if (a.G * C::NCH > 32 * kPPMax) return cudaErrorInvalidValue;
   const size_t smem = dec_attn_smem<T, D>(a.G);
   cudaError_t e = allow_smem(reinterpret_cast<const void*>(decode_attn_kernel<T, D>),
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid(a.splits, a.Hkv, a.B);
+  dim3 grid(a.splits, a.Hkv * dec_head_chunks<T, D>(a.G), a.B);
   decode_attn_kernel<T, D><<<grid, kDecThreads, smem, stream>>>(a);
   count_launches(1);
   return cudaGetLastError();
@@ -924,6 +961,12 @@ cudaError_t launch_kv_append(T* cache_k, T* cache_v, int32_t* len, const T* k_ne
   len_add_kernel<<<(B + 127) / 128, 128, 0, stream>>>(len, B, cap, n_new);
   count_launches(2);
   return cudaGetLastError();
+}
+
+bool decode_pre_fits(int G, int d, int K, int es) {
+  const size_t bytes = es == 2 ? pre_smem<bf16>(G, d, K).bytes_no_w
+                               : pre_smem<float>(G, d, K).bytes_no_w;
+  return bytes <= 227 * 1024;
 }
 
 template <typename T>

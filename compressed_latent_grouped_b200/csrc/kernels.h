@@ -35,7 +35,9 @@ struct PreAttnArgs {
   const T* src;          // [B*S, src_ld] rows: q~ | k~ | v~ columns
   int64_t src_ld;
   int B, S, Hq, Hkv, d, G, K;   // K = conv width, 0 = no conv / channel mix
-  int qk_mean, value_shift;
+  int qk_mean;           // 0 off, 1 cross (q~ + k~) / 2 added, 2 self (y + own pre) / 2
+  int value_shift;       // 0 off, 1 upper half-channels, 2 last floor(Hkv / 2) kv heads
+  int channel_conv;      // 1: per-tap d x d matrices (wq_chan [Hq, K, d, d]), no depthwise taps
   int rope_on;
   double rope_log2_base;
   // theta_i / (2 pi) as a 0.64 fixed-point fraction of a turn, i < d/2: the
@@ -55,6 +57,9 @@ struct PreAttnArgs {
 };
 template <typename T>
 cudaError_t launch_pre_attn(const PreAttnArgs<T>& a, cudaStream_t stream);
+// Whether the CUDA-core pre-attention kernel's smallest staging layout (8
+// positions per CTA) fits in shared memory for this group size and head dim.
+bool pre_attn_fits(int K, int G, int d, int es, bool has_mix);
 // bf16, d in {32, 64}, conv 1..4 taps with both channel-mix weights, 16-byte
 // aligned inputs and weights, the layout within 227 KB of shared memory: the mix
 // on tcgen05, staging by TMA (launch_pre_attn dispatches there when this holds).
@@ -72,9 +77,11 @@ struct AttnArgs {
   int causal;
   int32_t* dev_err;
 };
-// bf16, d in {32, 64, 128}, G a power of two <= 128: tcgen05/TMEM/TMA flash attention.
+// bf16, d in {32, 64, 128}, any G <= 128 (a tile holds floor(128 / G)
+// positions of the group's G heads): tcgen05/TMEM/TMA flash attention.
 cudaError_t launch_attn_prefill_tc(const AttnArgs& a, cudaStream_t stream);
-// CUDA-core flash attention (fp32 path).
+// CUDA-core flash attention (the fp32 path; bf16 where the tensor-core kernel
+// does not apply: d = 16 or G > 128).
 template <typename T>
 cudaError_t launch_attn_prefill_simt(const AttnArgs& a, cudaStream_t stream);
 
@@ -89,7 +96,8 @@ struct DecodeArgs {
   const T* x_t;          // [B, E] or packed [B, N] when W is null
   const T* W;            // [N, E] or null
   int B, E, N, Hq, Hkv, d, G, K;
-  int qk_mean, value_shift, causal, rope_on;
+  int qk_mean, value_shift, causal, rope_on;   // modes as in PreAttnArgs
+  int channel_conv;
   double rope_log2_base;
   uint64_t rope_frac[64];  // theta_i / (2 pi) in 0.64 fixed point, i < d/2 (see PreAttnArgs)
   const T *wq_seq, *wq_chan, *wk_seq, *wk_chan;
@@ -117,6 +125,10 @@ template <typename T>
 cudaError_t launch_decode_step(const DecodeArgs<T>& a, cudaStream_t stream);
 // bf16 decode attention on the tensor core (d in {32, 64, 128}, G <= 16).
 cudaError_t launch_decode_attn_tc(const DecodeArgs<bf16>& a, cudaStream_t stream);
+
+// Whether the one-token pre-step's shared memory (without staged mix weights)
+// fits for this group size and head dim.
+bool decode_pre_fits(int G, int d, int K, int es);
 
 // Split plan for the decode step, shared by the workspace-size query and the launch.
 void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int es,

@@ -82,7 +82,9 @@ __global__ void __launch_bounds__(kPreThreads)
   constexpr int d = D, half = D / 2;
   constexpr int WS = D + 2;        // padded row of the transposed channel-mix weight
   const int G = a.G, K = a.K, S = a.S;
-  const PreLayout L = pre_layout(TT, K, G, d, sizeof(T), a.wq_chan != nullptr || a.wk_chan != nullptr);
+  const bool full = a.channel_conv && K > 0;   // per-tap d x d matrices, weights read from L1/L2
+  const PreLayout L = pre_layout(TT, K, G, d, sizeof(T),
+                                 !full && (a.wq_chan != nullptr || a.wk_chan != nullptr));
   T* z = reinterpret_cast<T*>(smem);                      // [R][ZC]: q | k | v
   float* fs = reinterpret_cast<float*>(smem + L.z_bytes);
   float* u = fs + L.off_u;                                // [d][US]
@@ -155,10 +157,13 @@ __global__ void __launch_bounds__(kPreThreads)
     const int head = is_q ? g * G + hh : g;
     const int cb = hh * d;               // channel offset inside the z tile
     const T* wch_base = is_q ? a.wq_chan : a.wk_chan;
-    const T* wch = (K > 0 && wch_base) ? wch_base + static_cast<int64_t>(head) * d * d : nullptr;
+    const T* wch = (K > 0 && wch_base && !full) ? wch_base + static_cast<int64_t>(head) * d * d
+                                                : nullptr;
+    // the head's per-tap matrices W[head][k] (temporal channel conv)
+    const T* wfull = full ? wch_base + static_cast<int64_t>(head) * K * d * d : nullptr;
     // causal depthwise conv: thread = (channel, 8-row segment), taps in registers
     // (no conv: the epilogue reads q~ / k~ straight from the staged rows)
-    for (int idx = tid; K > 0 && idx < d * n_seg; idx += kPreThreads) {
+    for (int idx = tid; K > 0 && !full && idx < d * n_seg; idx += kPreThreads) {
       const int j = idx % d, sg = idx / d;
       const int tl0 = sg * SEG;
       const T* zc = z + cb + j;
@@ -201,7 +206,29 @@ __global__ void __launch_bounds__(kPreThreads)
       const int ip = idx % nI2, tq = idx / nI2;
       const int tl0 = tq * 4, i0 = ip * 2, i1 = i0 + half;
       float y[4][4];
-      if (wch) {
+      if (full) {
+        // y[t, i] = sum_k sum_j W_k[i][j] z[t - k, j]: the halo rows hold t - k
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) y[r][k] = 0.f;
+        const int chs[4] = {i0, i0 + 1, i1, i1 + 1};
+        for (int k = 0; k < K; ++k) {
+          const T* wk = wfull + static_cast<int64_t>(k) * d * d;
+#pragma unroll 4
+          for (int j = 0; j < d; ++j) {
+            float zr[4], wv[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) zr[r] = to_f32(z[(tl0 + r + HALO - k) * ZC + cb + j]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) wv[c] = to_f32(__ldg(wk + chs[c] * d + j));
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+              for (int c = 0; c < 4; ++c) y[r][c] = fmaf(zr[r], wv[c], y[r][c]);
+          }
+        }
+      } else if (wch) {
 #pragma unroll
         for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -244,7 +271,11 @@ __global__ void __launch_bounds__(kPreThreads)
         const int tl = tl0 + r, t = t0 + tl;
         if (t >= S) continue;
         const T* zrow = z + (tl + HALO) * ZC;
-        if (a.qk_mean) {
+        if (a.qk_mean == 2) {
+          // "self" reading: the mean of the head's own pre-conv value and y
+#pragma unroll
+          for (int k = 0; k < 4; ++k) y[r][k] = 0.5f * (y[r][k] + to_f32(zrow[cb + ch[k]]));
+        } else if (a.qk_mean) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const float kp = to_f32(zrow[QC + ch[k]]);
@@ -277,14 +308,16 @@ __global__ void __launch_bounds__(kPreThreads)
     if (K > 0) __syncthreads();
   }
 
-  // 4. value-shift: bit-exact gather of the current / previous v~ row.
+  // 4. value-shift: bit-exact gather of the current / previous v~ row (upper
+  // half-channels, or the whole head when it is one of the last floor(Hkv / 2)).
+  const bool shift_head = a.value_shift == 2 && g >= a.Hkv - a.Hkv / 2;
   constexpr int VEC = 16 / sizeof(T);
   const int nchunk = d / VEC;
   for (int idx = tid; idx < TT * nchunk; idx += kPreThreads) {
     const int tl = idx / nchunk, i = (idx - tl * nchunk) * VEC;
     const int t = t0 + tl;
     if (t >= S) continue;
-    const int row = (a.value_shift && i >= half) ? tl + HALO - 1 : tl + HALO;
+    const int row = ((a.value_shift == 1 && i >= half) || shift_head) ? tl + HALO - 1 : tl + HALO;
     const uint4 val = *reinterpret_cast<const uint4*>(z + row * ZC + QC + d + i);
     *reinterpret_cast<uint4*>(a.v_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + t) * d +
                               i) = val;
@@ -314,6 +347,10 @@ __global__ void __launch_bounds__(kPreThreads)
 
 }  // namespace
 
+bool pre_attn_fits(int K, int G, int d, int es, bool has_mix) {
+  return pre_layout(8, K, G, d, es, has_mix).bytes <= 227 * 1024;
+}
+
 template <typename T>
 cudaError_t launch_pre_attn(const PreAttnArgs<T>& a, cudaStream_t stream) {
   if constexpr (std::is_same<T, bf16>::value) {
@@ -324,7 +361,7 @@ cudaError_t launch_pre_attn(const PreAttnArgs<T>& a, cudaStream_t stream) {
   int TT = 4096 / a.d;
   if (TT > 256) TT = 256;
   const int es = sizeof(T);
-  const bool has_mix = a.wq_chan != nullptr || a.wk_chan != nullptr;
+  const bool has_mix = !a.channel_conv && (a.wq_chan != nullptr || a.wk_chan != nullptr);
   while (TT > 8 && pre_layout(TT, a.K, a.G, a.d, es, has_mix).bytes > 200 * 1024) TT /= 2;
   const PreLayout L = pre_layout(TT, a.K, a.G, a.d, es, has_mix);
   if (L.bytes > 227 * 1024) return cudaErrorInvalidConfiguration;

@@ -173,6 +173,9 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
   }
   // value-shift rows straight into registers (stored at the end of the kernel):
   // v[t, :d/2] = v~[t, :d/2], v[t, d/2:] = v~[t-1, d/2:], zero before position 0
+  // (whole-head reading: every channel of the group's kv head from t-1 when
+  // the head is one of the last floor(Hkv/2))
+  const bool shift_head = a.value_shift == 2 && g >= a.Hkv - a.Hkv / 2;
   constexpr int kVPer = kPtTT * NCH / kPtThreads;
   uint4 vreg[kVPer];
 #pragma unroll
@@ -180,7 +183,7 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
     const int idx = tid + q * kPtThreads;
     const int tl = idx / NCH, i = (idx % NCH) * 8;
     const int tv = t0 + tl;
-    const int row = (a.value_shift && i >= D / 2) ? tv - 1 : tv;
+    const int row = ((a.value_shift == 1 && i >= D / 2) || shift_head) ? tv - 1 : tv;
     vreg[q] = make_uint4(0, 0, 0, 0);
     if (tv < S && row >= 0)
       vreg[q] = *reinterpret_cast<const uint4*>(src_b + static_cast<int64_t>(row) * ld + vcol0 + i);
@@ -317,7 +320,26 @@ __global__ void __launch_bounds__(kPtThreads, (D == 32) ? 3 : 1)
       lo[e] = __uint_as_float(ya[e]);
       hi[e] = __uint_as_float(yb[e]);
     }
-    if (a.qk_mean) {
+    if (a.qk_mean == 2) {
+      // "self" reading: y = (y + own pre-conv value) / 2 over channels c0 + e
+      // (slot hh holds this head's q~, or k~ for the key head)
+      auto self_mean = [&](float (&y)[Q4], int c0) {
+#pragma unroll
+        for (int q8 = 0; q8 < Q4 / 8; ++q8) {
+          const uint4 ow = *zchunk(hh, r + kPtHalo, c0 / 8 + q8);
+          const uint32_t* op = reinterpret_cast<const uint32_t*>(&ow);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint16_t o0, o1;
+            halves(op[e], o0, o1);
+            y[q8 * 8 + 2 * e] = fma_bf16(o0, kBf16Half, 0.5f * y[q8 * 8 + 2 * e]);
+            y[q8 * 8 + 2 * e + 1] = fma_bf16(o1, kBf16Half, 0.5f * y[q8 * 8 + 2 * e + 1]);
+          }
+        }
+      };
+      self_mean(lo, i0);
+      self_mean(hi, i0 + D / 2);
+    } else if (a.qk_mean) {
       const bool is_q = hh < G;
       // y[e] += (q~ + k~) / 2 over channels c0 + e (q~: this head, or the
       // mean of the group's query heads for the key head), as fp32 FMAs on the
@@ -508,6 +530,7 @@ cudaError_t launch_d(const PreAttnArgs<bf16>& a, cudaStream_t stream) {
 
 bool pre_attn_tc_supported(const PreAttnArgs<bf16>& a) {
   if (a.d != 32 && a.d != 64) return false;
+  if (a.channel_conv) return false;   // per-tap matrices: the CUDA-core kernel
   if (a.K < 1 || a.K > 4 || a.wq_chan == nullptr || a.wk_chan == nullptr) return false;
   if (a.wq_seq == nullptr || a.wk_seq == nullptr) return false;
   // TMA and bulk copies: 16-byte aligned bases and row pitches

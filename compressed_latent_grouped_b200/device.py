@@ -12,7 +12,8 @@ from .workloads import Workload
 def config_of(w: Workload) -> B.ccgqa_config:
     return B.make_config(w.E, w.C, w.Hq, w.Hkv, conv_width=w.conv_width, qk_mean=w.qk_mean,
                          value_shift=w.value_shift, causal=w.causal, rope_base=w.rope_base,
-                         dtype=B.F32 if w.dtype == "f32" else B.BF16)
+                         dtype=B.F32 if w.dtype == "f32" else B.BF16,
+                         channel_conv=w.channel_conv)
 
 
 class DeviceLayer:

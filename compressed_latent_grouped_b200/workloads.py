@@ -10,7 +10,9 @@ then rounded to the workload's dtype with round-to-nearest-even.  Draw order is
 fixed: x, W_qkv, conv_q_seq, conv_q_chan, conv_k_seq, conv_k_chan, then the
 decode extras (cache k, cache v, hist_q, hist_k, v_prev, x_t).
 Weights follow N(0, 1/fan_in): W_qkv fan_in = E, sequence-conv taps fan_in = K,
-channel mix fan_in = d.
+channel mix fan_in = d.  With the temporal channel conv (``channel_conv``) the
+channel weights are per-tap matrices [H, K, d, d] with fan_in = K d, drawn in
+the slots of the channel mix, and no sequence-conv taps are drawn.
 """
 from __future__ import annotations
 
@@ -31,12 +33,13 @@ class Workload:
     Hq: int
     Hkv: int
     conv_width: int = 4
-    qk_mean: bool = True
-    value_shift: bool = True
+    qk_mean: int = 1             # 0 off, 1 cross, 2 self
+    value_shift: int = 1         # 0 off, 1 half channels, 2 whole kv heads
     rope_base: float = 10000.0
     causal: bool = True
     packed_input: bool = False   # x already holds q~|k~|v~ (no projection)
     decode: bool = False
+    channel_conv: bool = False   # per-tap d x d channel matrices instead of taps + mix
 
     @property
     def d(self) -> int:
@@ -111,7 +114,11 @@ def make_inputs(w: Workload, seed: int = 0, batch: int | None = None) -> dict:
     else:
         out["x"] = _normal(rng, (B, w.S, w.E), 1.0, dt)
     out["W_qkv"] = None if w.packed_input else _normal(rng, (w.n_qkv, w.E), (1.0 / w.E) ** 0.5, dt)
-    if K > 0:
+    if K > 0 and w.channel_conv:
+        out["conv_q_seq"] = out["conv_k_seq"] = None
+        out["conv_q_chan"] = _normal(rng, (w.Hq, K, d, d), (1.0 / (K * d)) ** 0.5, dt)
+        out["conv_k_chan"] = _normal(rng, (w.Hkv, K, d, d), (1.0 / (K * d)) ** 0.5, dt)
+    elif K > 0:
         out["conv_q_seq"] = _normal(rng, (w.Hq * d, K), (1.0 / K) ** 0.5, dt)
         out["conv_q_chan"] = _normal(rng, (w.Hq, d, d), (1.0 / d) ** 0.5, dt)
         out["conv_k_seq"] = _normal(rng, (w.Hkv * d, K), (1.0 / K) ** 0.5, dt)

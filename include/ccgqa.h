@@ -44,7 +44,10 @@ extern "C" {
 typedef enum {
   CCGQA_OK = 0,
   CCGQA_ERR_INVALID_ARG = 1,  /* NULL / misaligned pointer, inconsistent sizes */
-  CCGQA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. bf16 head dim 16) */
+  CCGQA_ERR_UNSUPPORTED = 2,  /* valid but not implemented: d outside {16, 32, 64,
+                                 128}, or a group so large that (G + 2) d channels of
+                                 one sequence do not fit the decode pre-step's
+                                 shared memory */
   CCGQA_ERR_CAPACITY = 3,     /* the tokens do not fit the cache capacity */
   CCGQA_ERR_WORKSPACE = 4,    /* workspace NULL, misaligned or too small */
   CCGQA_ERR_CUDA = 5          /* a CUDA runtime call or launch failed */
@@ -62,15 +65,32 @@ typedef struct {
   int32_t E;            /* model width */
   int32_t C;            /* compression factor: latent width E / C  [Methodologie 1] */
   int32_t n_q_heads;    /* Hq */
-  int32_t n_kv_heads;   /* Hkv; must divide Hq  [CCGQA] */
+  int32_t n_kv_heads;   /* Hkv; must divide Hq; any group size G = Hq / Hkv
+                           (MQA at Hkv = 1, MHA at Hkv = Hq)  [CCGQA; GQA page,
+                           "Como funciona GQA"] */
   int32_t conv_width;   /* K in 0..4 taps of the causal sequence conv; 0 = no conv
                            and no channel mix  [Methodologie 2] */
-  int32_t qk_mean;      /* 1 = add the QK-mean skip term  [Methodologie 2, QK-Mean] */
-  int32_t value_shift;  /* 1 = value-shift  [Methodologie 3] */
+  int32_t qk_mean;      /* QK-mean skip term  [Methodologie 2, QK-Mean]:
+                           0 off; 1 "cross": (q~ + k~)/2 of the same position added
+                           to q and k (k~ and the mean of the group's q~ for k);
+                           2 "self": each head becomes (own pre-conv + conv
+                           output) / 2 (the literal reading of the page) */
+  int32_t value_shift;  /* value-shift  [Methodologie 3]: 0 off; 1 channels
+                           [d/2, d) of every kv head from the previous token;
+                           2 whole kv heads: the last floor(Hkv/2) heads from the
+                           previous token, the others current */
   int32_t causal;       /* 1 = causal attention mask  [Probleemstelling] */
   double rope_base;     /* RoPE base; 0 = no RoPE  [Methodologie 4] */
-  int32_t dtype;        /* ccgqa_dtype: fp32 or bf16 (bf16 needs d in {32, 64, 128}) */
-  int32_t reserved;     /* set to 0 */
+  int32_t dtype;        /* ccgqa_dtype: fp32 or bf16; head dim d = E / (C Hq) in
+                           {16, 32, 64, 128} for both (bf16 attention runs on the
+                           tensor core for d >= 32 and G <= 128, on the CUDA
+                           cores otherwise) */
+  int32_t channel_conv; /* channel convolution  [Methodologie 2]: 0 = depthwise
+                           sequence taps conv_*_seq then one d x d mix per head
+                           and position (conv_*_chan [H, d, d], or none); 1 =
+                           temporal channel conv with a d x d matrix per tap,
+                           y[t] = sum_j W[h, j] z[t - j]: conv_*_chan [H, K, d, d]
+                           required, conv_*_seq unused (needs conv_width >= 1) */
 } ccgqa_config;
 
 /* Weights (device, cfg->dtype).  [Methodologie 1-2] */
@@ -82,10 +102,12 @@ typedef struct {
   const void* W_qkv;
   /* [Hq d, K]: sequence-conv taps; tap j multiplies the row j steps back. */
   const void* conv_q_seq;
-  /* [Hq, d, d]: per-head channel mix y_i = sum_j W[h][i][j] u_j; NULL = none. */
+  /* [Hq, d, d]: per-head channel mix y_i = sum_j W[h][i][j] u_j; NULL = none.
+     With channel_conv = 1: [Hq, K, d, d], tap j's matrix at [h][j]:
+     y[t]_i = sum_j sum_c W[h][j][i][c] z[t-j]_c (conv_q_seq unused). */
   const void* conv_q_chan;
   const void* conv_k_seq;   /* [Hkv d, K] */
-  const void* conv_k_chan;  /* [Hkv, d, d]; NULL = none */
+  const void* conv_k_chan;  /* [Hkv, d, d]; NULL = none ([Hkv, K, d, d] with channel_conv = 1) */
 } ccgqa_weights;
 
 /* Latent KV cache plus the decode state (device buffers, caller-owned).

@@ -22,8 +22,9 @@ def oracle_layer(w: Workload, inp: dict) -> O.Layer:
         sh=O.Shape(w.E, w.C, w.Hq, w.Hkv), W_qkv=f64(inp.get("W_qkv")),
         conv_width=w.conv_width, conv_q_seq=f64(inp.get("conv_q_seq")),
         conv_q_chan=f64(inp.get("conv_q_chan")), conv_k_seq=f64(inp.get("conv_k_seq")),
-        conv_k_chan=f64(inp.get("conv_k_chan")), qk_mean=bool(w.qk_mean),
-        value_shift=bool(w.value_shift), rope_base=w.rope_base, causal=bool(w.causal))
+        conv_k_chan=f64(inp.get("conv_k_chan")), qk_mean=int(w.qk_mean),
+        value_shift=int(w.value_shift), rope_base=w.rope_base, causal=bool(w.causal),
+        channel_conv=bool(w.channel_conv))
 
 
 def assert_close_f32(gpu, ref, what=""):
@@ -50,7 +51,7 @@ def check_prefill(w: Workload, inp: dict, b: int, got, rows=None, cache_k=None, 
             assert_close_f32(cache_v, st.v, what + " cache v")
         return
     model, mst = model_prefill(lay, x, rows=rows)
-    check_bf16(got, ref, model, what)
+    check_bf16(got, ref, model, mst.extra["spread"], what)
     if cache_k is not None:
         check_within_one_ulp(cache_k, mst.k, what + " cache k")
         check_within_one_ulp(cache_v, mst.v, what + " cache v")
@@ -58,7 +59,8 @@ def check_prefill(w: Workload, inp: dict, b: int, got, rows=None, cache_k=None, 
 
 def decode_references(w: Workload, inp: dict, b: int, xs):
     """Oracle and bf16-model outputs of consecutive decode steps from the
-    workload's synthetic state (xs: list of x_t rows as float64)."""
+    workload's synthetic state (xs: list of x_t rows as float64).  Each model
+    entry is (output, a), a being the bound's weighted absolute value."""
     lay = oracle_layer(w, inp)
     st = O.State(k=f64(inp["cache_k"][b]), v=f64(inp["cache_v"][b]),
                  hist_q=f64(inp["hist_q"][b]), hist_k=f64(inp["hist_k"][b]),
@@ -70,11 +72,12 @@ def decode_references(w: Workload, inp: dict, b: int, xs):
         r, st = O.decode_step(lay, st, x)
         m, mst = model_decode_step(lay, mst, x)
         refs.append(r)
-        models.append(m)
+        models.append((m, mst.extra["spread"]))
     return refs, models, st, mst
 
 
 def check_rows(dtype, got, ref, model, what=""):
+    """model: (bf16-model output, a) from decode_references (unused for f32)."""
     if dtype == "f32":
         return assert_close_f32(got, ref, what)
-    return check_bf16(got, ref, model, what)
+    return check_bf16(got, ref, model[0], model[1], what)

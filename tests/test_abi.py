@@ -108,7 +108,9 @@ class _FakeTensor:
     (dict(dtype=7), 1),
     (dict(rope_base=-1.0), 1),
     (dict(E=1024, C=8), 2),            # d = 8 unsupported
-    (dict(E=256, C=1, n_q_heads=16, n_kv_heads=16), 2),  # bf16 d = 16 unsupported
+    # a group so large that the decode pre-step's (G + 2) d staged channels do
+    # not fit in shared memory
+    (dict(E=131072, C=1, n_q_heads=1024, n_kv_heads=1), 2),
 ])
 def test_invalid_config_rejected(lib, bad, status):
     cfg = _cfg(**bad)
@@ -117,6 +119,22 @@ def test_invalid_config_rejected(lib, bad, status):
                            ctypes.c_void_p(8192), None, ctypes.c_void_p(1 << 20), 1 << 30, None,
                            None)
     assert st == status
+
+
+@pytest.mark.parametrize("geo", [
+    dict(E=256, C=1, n_q_heads=16, n_kv_heads=16),       # bf16 d = 16
+    dict(E=1536, C=2, n_q_heads=12, n_kv_heads=4),       # G = 3
+    dict(E=1536, C=4, n_q_heads=12, n_kv_heads=2),       # G = 6
+    dict(E=3072, C=1, n_q_heads=24, n_kv_heads=2),       # G = 12, d = 128
+    dict(E=1536, C=1, n_q_heads=24, n_kv_heads=1),       # G = 24
+    dict(E=2560, C=1, n_q_heads=160, n_kv_heads=1),      # G = 160, d = 16
+])
+def test_whole_domain_accepted(lib, geo):
+    """Every d in {16, 32, 64, 128} and every Hq % Hkv == 0 is a valid layer
+    (the GQA page's grouping, with MQA and MHA as its ends)."""
+    cfg = _cfg(**geo)
+    assert B.ccgqa_prefill_workspace_size(cfg, 1, 64) > 0
+    assert B.ccgqa_decode_workspace_size(cfg, 2, 64) > 0
 
 
 def test_invalid_pointers_and_workspace_rejected(lib):

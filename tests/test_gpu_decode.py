@@ -70,6 +70,20 @@ def _decode_setup(w, cap_extra=8, seed=0):
     W4.with_(name="dec_d32", B=3, S=333, E=2048, C=4, Hq=16, Hkv=4, rope_base=1e4),
     W4.with_(name="dec_d128_plain", B=2, S=300, E=4096, C=1, Hq=32, Hkv=8, conv_width=0,
              qk_mean=False, value_shift=False, packed_input=True),
+    # d = 16 and group sizes beyond the tensor-core decode (G <= 16) or not
+    # powers of two; G = 24, 40 and 160 take several CTAs per kv group (head chunks)
+    W4.with_(name="dec_bf16_d16", B=3, S=300, E=256, C=4, Hq=4, Hkv=2, rope_base=1e4),
+    W4.with_(name="dec_g3", B=3, S=400, E=1536, C=2, Hq=12, Hkv=4),
+    W4.with_(name="dec_g24", B=2, S=260, E=1536, C=1, Hq=24, Hkv=1),
+    W4.with_(name="dec_f32_g40", B=2, S=150, E=2560, C=1, Hq=40, Hkv=1, dtype="f32"),
+    W4.with_(name="dec_d16_g160", B=2, S=90, E=2560, C=1, Hq=160, Hkv=1),
+    # the readings' variants
+    W4.with_(name="dec_qk_self", B=3, S=300, qk_mean=2),
+    W4.with_(name="dec_vs_heads", B=3, S=250, E=2048, C=4, Hq=16, Hkv=4, value_shift=2,
+             rope_base=1e4),
+    W4.with_(name="dec_chanconv", B=3, S=200, channel_conv=True),
+    W4.with_(name="dec_f32_all_variants", B=2, S=120, channel_conv=True, qk_mean=2,
+             value_shift=2, dtype="f32"),
 ], ids=lambda w: w.name)
 def test_decode_steps_match_oracle(w):
     inp, lay = _decode_setup(w)
@@ -126,7 +140,9 @@ def test_decode_value_shift_bits():
 
 @pytest.mark.parametrize("w", [W2.with_(name="pd_d32", B=2, S=257),
                                W3.with_(name="pd_d64", S=200),
-                               W5.with_(name="pd_d128", B=1, S=130)], ids=lambda w: w.name)
+                               W5.with_(name="pd_d128", B=1, S=130),
+                               W3.with_(name="pd_variants", S=150, qk_mean=2, value_shift=2,
+                                        channel_conv=True)], ids=lambda w: w.name)
 def test_prefill_then_decode_equals_longer_prefill(w):
     """prefill(S) row S-1 == prefill(S-1) followed by one decode step."""
     inp = make_inputs(w, seed=4)
@@ -146,10 +162,12 @@ def test_prefill_then_decode_equals_longer_prefill(w):
         ref, _ = O.prefill(lo, xb, rows=np.array([w.S - 1]))
         # decode path: prefill model over S-1 tokens, then the decode-step model
         _, mst = model_prefill(lo, xb[:-1])
-        m_dec, _ = model_decode_step(lo, mst, xb[-1])
-        check_bf16(o[b].float().cpu().numpy(), ref[0], m_dec, f"{w.name} decode b={b}")
-        m_pf, _ = model_prefill(lo, xb, rows=np.array([w.S - 1]))
-        check_bf16(full_out[b, -1].float().cpu().numpy(), ref[0], m_pf[0], f"{w.name} prefill b={b}")
+        m_dec, dst = model_decode_step(lo, mst, xb[-1])
+        check_bf16(o[b].float().cpu().numpy(), ref[0], m_dec, dst.extra["spread"],
+                   f"{w.name} decode b={b}")
+        m_pf, pst = model_prefill(lo, xb, rows=np.array([w.S - 1]))
+        check_bf16(full_out[b, -1].float().cpu().numpy(), ref[0], m_pf[0], pst.extra["spread"][0],
+                   f"{w.name} prefill b={b}")
     # the caches agree except for the last row's bf16 rounding path
     for key in ("k", "v"):
         a = part.cache_tensors[key][:, :, : w.S - 1].float().cpu().numpy()

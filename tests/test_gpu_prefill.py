@@ -40,6 +40,29 @@ SMALL = {
     "bf16_d32_conv3": W2.with_(name="k3", B=1, S=259, conv_width=3),
     "bf16_d64_conv1": W3.with_(name="k1", S=131, conv_width=1),
     "bf16_d32_g16": W2.with_(name="g16", B=1, S=200, Hkv=1),
+    # the whole C-ABI domain (any Hq % Hkv == 0; bf16 d = 16): d = 16 runs on the
+    # CUDA-core attention, group sizes that do not divide 128 leave 128 mod G
+    # rows of every query tile empty, and G > 128 runs on the CUDA cores
+    "bf16_d16": W1.with_(name="bf16d16", dtype="bf16", B=2, S=200),
+    "bf16_d64_g3": W3.with_(name="g3", E=1536, C=2, Hq=12, Hkv=4, S=300),
+    "bf16_d32_g6": W2.with_(name="g6", B=1, E=1536, C=4, Hq=12, Hkv=2, S=250),
+    "bf16_d128_g12": W5.with_(name="g12", B=1, S=200, E=3072, C=1, Hq=24, Hkv=2, conv_width=4,
+                              qk_mean=True, value_shift=True, packed_input=False),
+    "bf16_d64_g24_noncausal": W3.with_(name="g24", E=1536, C=1, Hq=24, Hkv=1, S=150,
+                                       causal=False),
+    "bf16_d16_g160": W1.with_(name="g160", dtype="bf16", E=2560, C=1, Hq=160, Hkv=1, S=40),
+    "f32_d32_g3": W1.with_(name="f32g3", E=768, C=4, Hq=6, Hkv=2, S=100),
+    # the readings' variants: QK-mean "self" and whole-head value-shift on the
+    # tensor-core pre-attention, the temporal channel conv (per-tap matrices) on
+    # the CUDA-core kernel, all three together in fp32
+    "bf16_d32_qk_self": W2.with_(name="qkself", B=1, S=200, qk_mean=2),
+    "bf16_d64_vs_heads": W3.with_(name="vsheads", S=150, value_shift=2),
+    "bf16_d64_chanconv": W3.with_(name="chanconv", S=180, channel_conv=True),
+    "bf16_d128_all_variants": W5.with_(name="allvar", B=1, S=140, conv_width=3, qk_mean=2,
+                                       value_shift=2, packed_input=False, E=2048, C=1, Hq=16,
+                                       Hkv=4, channel_conv=True),
+    "f32_all_variants": W1.with_(name="f32allvar", S=100, channel_conv=True, qk_mean=2,
+                                 value_shift=2),
 }
 
 
@@ -115,6 +138,22 @@ def test_value_shift_gather_bit_exact():
     # decode state: the last v~ row and the last K-1 pre-conv rows, bit for bit
     assert torch.equal(lay.cache_tensors["v_prev"].cpu().view(torch.int16),
                        vt[:, -1].reshape(w.B, -1).view(torch.int16))
+
+
+def test_whole_head_value_shift_gather_bit_exact():
+    """Whole-head reading: the last floor(Hkv / 2) kv heads hold the previous
+    position's v~ row bit for bit (zero at position 0), the others the
+    current one."""
+    w = W5.with_(B=1, S=200, value_shift=2)
+    inp = make_inputs(w, seed=6)
+    lay, _ = _run(w, inp)
+    d, Hq, Hkv = w.d, w.Hq, w.Hkv
+    vt = inp["x"][..., (Hq + Hkv) * d:].reshape(w.B, w.S, Hkv, d)
+    v = lay.cache_tensors["v"][:, :, : w.S].cpu().permute(0, 2, 1, 3)
+    g0 = Hkv - Hkv // 2
+    assert torch.equal(v[:, :, :g0].view(torch.int16), vt[:, :, :g0].view(torch.int16))
+    assert torch.equal(v[:, 1:, g0:].view(torch.int16), vt[:, :-1, g0:].view(torch.int16))
+    assert torch.all(v[:, 0, g0:].view(torch.int16) == 0)
 
 
 def test_decode_state_after_prefill_bit_exact():

@@ -1,12 +1,13 @@
 """The attention kernel's software exp2 (Cody-Waite reduction + fitted cubic),
 replayed in float32 on the host: relative error, the exponent-field add and
-the clamp that keeps very negative inputs (masked scores) finite."""
+the clamps that keep very negative inputs (masked scores) tiny and very large
+ones (a score far above the running max) finite and huge."""
 import numpy as np
 
 
 def soft_exp2_f32(x):
     f32 = np.float32
-    x = np.maximum(x.astype(f32), f32(-126.0))
+    x = np.minimum(np.maximum(x.astype(f32), f32(-126.0)), f32(127.0))
     t = (x + f32(12582912.0)).astype(f32)
     f = (x - (t - f32(12582912.0))).astype(f32)
     p = (f32(0.05521968) * f + f32(0.24260941)).astype(f32)
@@ -27,3 +28,13 @@ def test_masked_and_tiny_inputs_stay_finite_and_tiny():
     x = np.array([-np.inf, -1e30, -300.0, -127.5, -126.0], dtype=np.float32)
     y = soft_exp2_f32(x)
     assert np.all(np.isfinite(y)) and np.all(y >= 0) and np.all(y < 1e-37)
+
+
+def test_large_inputs_stay_finite_and_huge():
+    """An argument far above the running max must not wrap the exponent field:
+    the result stays finite and above the softmax's partial-sum limit (1024),
+    so the half is redone against a raised running max."""
+    x = np.array([10.5, 127.0, 128.0, 200.0, 369.0, 1e30, np.inf], dtype=np.float32)
+    y = soft_exp2_f32(x)
+    assert np.all(np.isfinite(y)) and np.all(y > 1024.0)
+    assert np.all(y[1:] >= np.float32(2.0 ** 126))
