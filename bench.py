@@ -36,9 +36,10 @@ METRIC = "CCGQA prefill TFLOP/s & tokens/s; decode latent-KV GB/s vs B200 peak"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ATTN_SRC = os.path.join(ROOT, "compressed_latent_grouped_b200", "csrc", "attn_prefill_tc.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_prefill_tc_traffic.txt")
-# one exponential pair in SOFT_EVERY[d] of each softmax row runs on the FMA pipe
-# (a polynomial) in attn_prefill_tc, the rest on the exp unit
-SOFT_EVERY = {32: 4, 64: 3, 128: 4}
+# pairs c2 = 0, k, 2k, ... (k = SOFT_EVERY[d]) of the 32 exponential pairs in a
+# 64-key half run on the FMA pipe (a polynomial) in attn_prefill_tc, the rest
+# on the exp unit
+SOFT_EVERY = {32: 5, 64: 3, 128: 4}
 
 
 def attention_flops(B: int, S: int, Hq: int, d: int, causal: bool = True) -> float:
@@ -295,11 +296,12 @@ def run_reference(args, world, rank):
 def exp_roofline(w, attn_ms, peaks):
     """The exponentials the exp unit executes against its peak: 16 ex2 per
     clock per SM (the B200 SFU rate, measured 15.8 on this part) x 148 SMs x the
-    maximum SM clock.  A causal launch has B Hq S (S + 1) / 2 exponentials; one
-    pair in SOFT_EVERY[d] runs on the FMA pipe instead, so the exp unit's share
-    is the rest, and frac is that share's rate over the unit's peak."""
+    maximum SM clock.  A causal launch has B Hq S (S + 1) / 2 exponentials; the
+    pairs SOFT_EVERY[d] apart run on the FMA pipe instead, so the exp unit's
+    share is the rest, and frac is that share's rate over the unit's peak."""
     n_exp = w.B * w.Hq * w.S * (w.S + 1) / 2 if w.causal else w.B * w.Hq * w.S * w.S
-    mufu_share = 1.0 - 1.0 / SOFT_EVERY.get(w.d, 4)
+    k = SOFT_EVERY.get(w.d, 4)
+    mufu_share = 1.0 - ((32 + k - 1) // k) / 32.0
     mhz = peaks.get("sm_max_mhz", 1965.0)
     peak = 16 * 148 * mhz * 1e6 / 1e12
     achieved = n_exp * mufu_share / (attn_ms / 1e3) / 1e12
@@ -367,11 +369,15 @@ def setup_decode(w, dev, seed=0, extra_cap=64):
     return lay, inp, len0
 
 
-def decode_numbers(w, proj_ms, pre_ms, attn_ms, peaks):
+def decode_numbers(w, proj_ms, pre_ms, attn_ms, step_ms, peaks):
+    """Decode-step figures: the kernels' times from events between them, the
+    step's from events around the whole step only (an event between two
+    kernels serialises them, so the kernel times add up to more than the step)."""
     kv = 2 * w.B * w.Hkv * (w.S + 1) * w.d * 2
-    step = proj_ms + pre_ms + attn_ms
+    step = step_ms
     return {"kv_bytes": kv, "proj_ms": proj_ms, "pre_ms": pre_ms, "attn_ms": attn_ms,
-            "step_ms": step, "attn_gbs": kv / (attn_ms / 1e3) / 1e9,
+            "step_ms": step, "sum_of_kernels_ms": proj_ms + pre_ms + attn_ms,
+            "attn_gbs": kv / (attn_ms / 1e3) / 1e9,
             "attn_hbm_frac": kv / (attn_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
             "step_gbs": kv / (step / 1e3) / 1e9,
             "step_hbm_frac": kv / (step / 1e3) / 1e9 / peaks["hbm_gbs"],
@@ -391,6 +397,15 @@ def measure_decode_workload(w, steps, dev):
     for _ in range(3):
         lens.copy_(len0)
         lay.decode_step(x_t, out)
+    # the whole step: events only around it
+    whole = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(steps)]
+    for e0, e1 in whole:
+        lens.copy_(len0)
+        flush.zero_()
+        e0.record()
+        lay.decode_step(x_t, out)
+        e1.record()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     for e in evs:
         lens.copy_(len0)
@@ -402,8 +417,9 @@ def measure_decode_workload(w, steps, dev):
     if lay.error_bits():
         raise RuntimeError(f"device error bits {lay.error_bits()}")
     ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps for i in range(3)]
+    step_ms = sum(e0.elapsed_time(e1) for e0, e1 in whole) / steps
     peaks, _ = load_peaks()
-    return decode_numbers(w, ms[0], ms[1], ms[2], peaks)
+    return decode_numbers(w, ms[0], ms[1], ms[2], step_ms, peaks)
 
 
 def measure_output_projection(w, steps, dev):
@@ -518,6 +534,7 @@ def run_ours(args, world, rank, local):
         graph.launch()
     torch.cuda.synchronize()
     eager_ev = [(mk(), mk()) for _ in range(K)]
+    dstep_ev = [(mk(), mk()) for _ in range(K)]
     with sampler:
         # pass 1, the step time: events only around whole steps.  An event
         # recorded between two kernels serialises them (about 3 us a record on
@@ -544,6 +561,12 @@ def run_ours(args, world, rank, local):
             B.ccgqa_set_phase_events(dc_ev[i])
             dc.decode_step(x_t, out_t)
             B.ccgqa_set_phase_events(None)
+        # pass 4, the decode step alone with events only around it
+        for i in range(K):
+            between_steps()
+            dstep_ev[i][0].record(stream)
+            dc.decode_step(x_t, out_t)
+            dstep_ev[i][1].record(stream)
         torch.cuda.synchronize()
     barrier(world)
     if pf.error_bits() or dc.error_bits():
@@ -567,7 +590,8 @@ def run_ours(args, world, rank, local):
     peaks, peak_kind = load_peaks()
     achieved = attn_flop / (attn_ms / 1e3) / 1e12
     traffic = attn_traffic_per_launch()
-    dec = decode_numbers(wd, dproj_ms, dpre_ms, dattn_ms, peaks)
+    dstep_ms = sum(a.elapsed_time(b) for a, b in dstep_ev) / K
+    dec = decode_numbers(wd, dproj_ms, dpre_ms, dattn_ms, dstep_ms, peaks)
 
     # end to end through the public API: pinned host buffers in, results out.
     # Three streams, as a serving loop would run it: step i+1's inputs are copied
@@ -654,12 +678,17 @@ def run_ours(args, world, rank, local):
     if rank != 0:
         return
     timing = "CUDA events around each launch, third pass of the K steps"
+    # The kernel is timed inside the step loop (K steps back to back, seconds of
+    # load under the 1 kW cap; the clock record shows sw_power_cap): its peak is
+    # the sustained cuBLAS figure, with the burst fraction beside it.
+    sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     roof_tensor = {"bound": "tensor", "kernel": f"attn_prefill_tc (d = {wp.d})",
-                   "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                   "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
-                   "peak_kind": f"{peak_kind} bf16 dense burst",
-                   "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained",
-                                                             peaks["bf16_tflops"]),
+                   "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
+                   "frac": achieved / sustained, "traffic": traffic,
+                   "peak_kind": f"{peak_kind} bf16 dense sustained (the kernel is timed inside "
+                                f"the step loop)",
+                   "frac_of_burst": achieved / peaks["bf16_tflops"],
+                   "burst_peak": peaks["bf16_tflops"],
                    "flop_per_launch": attn_flop, "ms_per_launch": attn_ms, "timing": timing}
     roof_exp = {**exp_roofline(wp, attn_ms, peaks), "kernel": "attn_prefill_tc",
                 "ms_per_launch": attn_ms, "timing": timing}
