@@ -169,10 +169,11 @@ def check_bf16(gpu, ref, model, spread, what=""):
     assert spread.shape == gpu.shape, (spread.shape, gpu.shape)
     allow = (ELEM_ULPS * bf16_ulp(np.maximum(np.abs(gpu), np.abs(model))) +
              ELEM_SPREAD * spread + ELEM_RMS * rms)
-    worst = int(np.argmax(d - allow))
+    share = d / allow
+    worst = int(np.argmax(share))
     print(f"[bf16 parity] {what}: L2 {l2:.2e}, max|gpu-oracle|/RMS {e_gpu / rms:.2e}, "
           f"max|gpu-model|/RMS {float(d.max()) / rms:.2e}, "
-          f"worst element uses {float(d.flat[worst] / allow.flat[worst]):.2f} of its bound (c)")
+          f"worst element uses {float(share.flat[worst]):.2f} of its bound (c)")
     assert np.all(d <= allow), (
         f"{what}: element {np.unravel_index(worst, d.shape)}: |gpu - model| "
         f"{float(d.flat[worst]):.3e} > ulp + 2^-7 a + 2^-9 RMS = {float(allow.flat[worst]):.3e} "
