@@ -45,7 +45,7 @@ __all__ = [
     "qk_mean_self", "rope", "value_shift", "value_shift_heads", "attention", "prefill",
     "decode_step", "kvcache_append", "output_projection", "cache_values_per_token",
     "attention_flops", "QK_OFF", "QK_CROSS", "QK_SELF", "VS_OFF", "VS_HALF_CHANNELS",
-    "VS_WHOLE_HEADS",
+    "VS_WHOLE_HEADS", "attention_backward", "prefill_backward",
 ]
 
 # Switches of the readings a layer can take (the CCA page's wording admits
@@ -462,3 +462,183 @@ def attention_flops(S: int, Hq: int, d: int, causal: bool = True) -> float:
     causal counts the S^2/2 visible scores."""
     pairs = S * S / 2 if causal else S * S
     return 2.0 * 2.0 * Hq * d * pairs
+
+
+# --------------------------------------------------------------------------
+# Backward pass  [CCA Resultaten 2: the layer is trained; its backward pass is
+# the chain rule through the forward steps above, in reverse order]
+# --------------------------------------------------------------------------
+def attention_backward(q, k, v, G, causal, dout, q_pos=None):
+    """Gradients of o = attention(q, k, v) for an upstream gradient dout
+    [T, Hq, d]: returns (dq [T, Hq, d], dk [L, Hkv, d], dv [L, Hkv, d]).
+
+    Per query head h with kv head g = h // G and scale 1/sqrt(d):
+        p = softmax(q k^T / sqrt(d) + mask),   o = p v
+        dv_g += p^T dout_h,   dp = dout_h v_g^T,
+        ds = p * (dp - rowsum(dp * p)),
+        dq_h = ds k_g / sqrt(d),   dk_g += ds^T q_h / sqrt(d).
+    A kv head's gradients sum over the G query heads that read it.
+    """
+    T, Hq, d = q.shape
+    L, Hkv, _ = k.shape
+    if q_pos is None:
+        q_pos = np.arange(T)
+    q_pos = np.asarray(q_pos)
+    scale = 1.0 / math.sqrt(d)
+    keys = np.arange(L)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for h in range(Hq):
+        g = h // G
+        sc = (q[:, h, :] @ k[:, g, :].T) * scale
+        if causal:
+            sc = np.where(keys[None, :] <= q_pos[:, None], sc, -np.inf)
+        sc = sc - sc.max(axis=1, keepdims=True)
+        p = np.exp(sc)
+        p = p / p.sum(axis=1, keepdims=True)
+        do = dout[:, h, :]
+        dv[:, g, :] += p.T @ do
+        dp = do @ v[:, g, :].T
+        ds = p * (dp - (dp * p).sum(axis=1, keepdims=True))
+        dq[:, h, :] = (ds @ k[:, g, :]) * scale
+        dk[:, g, :] += (ds.T @ q[:, h, :]) * scale
+    return dq, dk, dv
+
+
+def _rope_backward(dz, positions, base):
+    """RoPE is a rotation per pair: its transpose turns by the opposite angle."""
+    if base == 0:
+        return dz.copy()
+    return rope(dz, -np.asarray(positions, dtype=np.float64), base)
+
+
+def _value_shift_backward(layer, dv):
+    """Transpose of the value-shift gather: a shifted channel of row t came
+    from row t - 1, so its gradient flows back one row (nothing flows to
+    the row before the start)."""
+    mode = int(layer.value_shift)
+    dvt = dv.copy()
+    if mode == VS_OFF:
+        return dvt
+    S, Hkv, d = dv.shape
+    shifted = np.zeros_like(dv)
+    shifted[:-1] = dv[1:]              # row t receives row t+1's gradient
+    if mode == VS_WHOLE_HEADS:
+        g0 = Hkv - Hkv // 2
+        dvt[:, g0:] = shifted[:, g0:]
+    else:
+        dvt[..., d // 2:] = shifted[..., d // 2:]
+    return dvt
+
+
+def _seq_conv_backward(z, w_seq, du):
+    """u[t, c] = sum_j w[c, j] z[t - j, c]  (zero before the start):
+    dz[t, c] = sum_j w[c, j] du[t + j, c],  dw[c, j] = sum_t du[t, c] z[t - j, c]."""
+    S, Ch = z.shape
+    K = w_seq.shape[1]
+    dz = np.zeros_like(z)
+    dw = np.zeros_like(w_seq)
+    for j in range(K):
+        if j >= S:
+            break
+        dz[: S - j] += w_seq[:, j] * du[j:]
+        dw[:, j] = (du[j:] * z[: S - j]).sum(axis=0)
+    return dz, dw
+
+
+def _channel_conv_backward(z, W, dy):
+    """y[t, h] = sum_j W[h, j] z[t - j, h]:  dz[t, h] = sum_j W[h, j]^T dy[t + j, h],
+    dW[h, j] = sum_t dy[t, h] (outer) z[t - j, h]."""
+    S, H, d = z.shape
+    K = W.shape[1]
+    dz = np.zeros_like(z)
+    dW = np.zeros_like(W)
+    for j in range(K):
+        if j >= S:
+            break
+        dz[: S - j] += np.einsum("hij,thi->thj", W[:, j], dy[j:])
+        dW[:, j] = np.einsum("thi,thj->hij", dy[j:], z[: S - j])
+    return dz, dW
+
+
+def prefill_backward(layer: Layer, x: np.ndarray, dout: np.ndarray):
+    """Gradients of the prefill of one sequence (from an empty state) for an
+    upstream gradient dout [S, Hq d] of its output.
+
+    Returns a dict: dx [S, E] (or [S, N_qkv] for packed input), dW_qkv
+    [N_qkv, E] (None for packed input), and the conv weights' gradients under
+    the names of the weights (None where the weight is unused).  The forward
+    steps run in the pages' order; their transposes run in reverse.
+    """
+    sh = layer.sh
+    S = x.shape[0]
+    d, Hq, Hkv, G = sh.d, sh.Hq, sh.Hkv, sh.G
+    # ---- forward, keeping what the backward needs
+    q_pre, k_pre, v_lat = down_project(x, layer.W_qkv, sh)
+    conv = layer.conv_width > 0
+    if conv and layer.channel_conv:
+        y_q = channel_conv(q_pre, layer.conv_q_chan)
+        y_k = channel_conv(k_pre, layer.conv_k_chan)
+        u_q = u_k = None
+    elif conv:
+        u_q = seq_conv(q_pre.reshape(S, -1), layer.conv_q_seq).reshape(S, Hq, d)
+        u_k = seq_conv(k_pre.reshape(S, -1), layer.conv_k_seq).reshape(S, Hkv, d)
+        y_q = u_q if layer.conv_q_chan is None else channel_mix(u_q, layer.conv_q_chan)
+        y_k = u_k if layer.conv_k_chan is None else channel_mix(u_k, layer.conv_k_chan)
+    else:
+        y_q, y_k = q_pre.copy(), k_pre.copy()
+    mode = int(layer.qk_mean)
+    if mode == QK_SELF:
+        qm, km = qk_mean_self(q_pre, y_q, k_pre, y_k)
+    elif mode:
+        m_q, m_k = qk_mean(q_pre, k_pre, G)
+        qm, km = y_q + m_q, y_k + m_k
+    else:
+        qm, km = y_q, y_k
+    pos = np.arange(S)
+    q = rope(qm, pos, layer.rope_base)
+    k = rope(km, pos, layer.rope_base)
+    v = _shift_values(layer, v_lat)
+    # ---- backward
+    dq, dk, dv = attention_backward(q, k, v, G, layer.causal, dout.reshape(S, Hq, d))
+    dv_lat = _value_shift_backward(layer, dv)
+    dqm = _rope_backward(dq, pos, layer.rope_base)
+    dkm = _rope_backward(dk, pos, layer.rope_base)
+    if mode == QK_SELF:
+        dy_q, dy_k = 0.5 * dqm, 0.5 * dkm
+        dq_pre, dk_pre = 0.5 * dqm, 0.5 * dkm
+    elif mode:
+        dy_q, dy_k = dqm, dkm
+        # m_q[h] = (q~[h] + k~[g]) / 2,  m_k[g] = (mean_h q~[h] + k~[g]) / 2
+        dq_pre = 0.5 * dqm + (0.5 / G) * np.repeat(dkm, G, axis=1)
+        dk_pre = 0.5 * dqm.reshape(S, Hkv, G, d).sum(axis=2) + 0.5 * dkm
+    else:
+        dy_q, dy_k = dqm, dkm
+        dq_pre, dk_pre = np.zeros_like(q_pre), np.zeros_like(k_pre)
+    grads = {"conv_q_seq": None, "conv_q_chan": None, "conv_k_seq": None, "conv_k_chan": None}
+    if conv and layer.channel_conv:
+        dz, grads["conv_q_chan"] = _channel_conv_backward(q_pre, layer.conv_q_chan, dy_q)
+        dq_pre = dq_pre + dz
+        dz, grads["conv_k_chan"] = _channel_conv_backward(k_pre, layer.conv_k_chan, dy_k)
+        dk_pre = dk_pre + dz
+    elif conv:
+        for side, z, u, dy, Wc, ws, Hs in (("q", q_pre, u_q, dy_q, layer.conv_q_chan, layer.conv_q_seq, Hq),
+                                           ("k", k_pre, u_k, dy_k, layer.conv_k_chan, layer.conv_k_seq, Hkv)):
+            if Wc is None:
+                du = dy
+            else:
+                du = np.einsum("hij,thi->thj", Wc, dy)          # W^T dy
+                grads[f"conv_{side}_chan"] = np.einsum("thi,thj->hij", dy, u)
+            dz, grads[f"conv_{side}_seq"] = _seq_conv_backward(z.reshape(S, -1), ws, du.reshape(S, -1))
+            if side == "q":
+                dq_pre = dq_pre + dz.reshape(S, Hs, d)
+            else:
+                dk_pre = dk_pre + dz.reshape(S, Hs, d)
+    else:
+        dq_pre = dq_pre + dy_q
+        dk_pre = dk_pre + dy_k
+    dzq = np.concatenate([dq_pre.reshape(S, -1), dk_pre.reshape(S, -1), dv_lat.reshape(S, -1)], axis=1)
+    if layer.W_qkv is None:
+        return {"dx": dzq, "W_qkv": None, **grads}
+    return {"dx": dzq @ layer.W_qkv, "W_qkv": dzq.T @ x, **grads}

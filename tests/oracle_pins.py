@@ -644,4 +644,104 @@ def pin_compression_factor():
     assert O.attention_flops(4, 1, 8, causal=False) == 4 * 8 * 16
 
 
+# --------------------------------------------------------------------------
+# Backward pass
+# --------------------------------------------------------------------------
+def _fd_check(lay, x, dout, names, n_samples, rng, tol, what):
+    """Central finite differences of L = sum(dout * prefill(x)) against the
+    oracle's gradients, on sampled entries of x and of each named weight."""
+    g = O.prefill_backward(lay, x, dout)
+    eps = 1e-6
+
+    def loss():
+        o, _ = O.prefill(lay, x)
+        return float(np.sum(o * dout))
+
+    for name in names:
+        arr = x if name == "dx" else getattr(lay, name)
+        grad = g[name]
+        assert grad is not None and grad.shape == arr.shape, (what, name)
+        flat = arr.reshape(-1)
+        picks = rng.choice(flat.size, size=min(n_samples, flat.size), replace=False)
+        scale = max(1.0, float(np.max(np.abs(grad))))
+        for i in picks:
+            old = flat[i]
+            flat[i] = old + eps
+            lp = loss()
+            flat[i] = old - eps
+            lm = loss()
+            flat[i] = old
+            fd = (lp - lm) / (2 * eps)
+            assert abs(fd - grad.reshape(-1)[i]) <= tol * scale, \
+                f"{what} d{name}[{i}]: finite difference {fd:.8e} vs {grad.reshape(-1)[i]:.8e}"
+
+
+def pin_backward_finite_differences():
+    """The layer's backward against central finite differences of its
+    forward (float64, step 1e-6), for the default readings, each variant,
+    plain GQA, a non-causal layer and one without RoPE, on sampled entries
+    of the input and of every weight."""
+    r = _rng(31)
+    layers = [
+        ("default", _small_layer(seed=7), True),
+        ("noncausal", _small_layer(seed=8, causal=False), True),
+        ("norope_k2_nochan", _small_layer(seed=9, K=2, chan=False, base=0.0), True),
+        ("plain_gqa", _small_layer(seed=10, K=0, qk=False, vs=False, base=0.0), True),
+        *[(f"variant{i}", lay, True) for i, lay in enumerate(_variant_layers())],
+    ]
+    for what, lay, _ in layers:
+        S = 7
+        x = r.standard_normal((S, lay.sh.E))
+        dout = r.standard_normal((S, lay.sh.Hq * lay.sh.d))
+        names = ["dx", "W_qkv"]
+        for w in ("conv_q_seq", "conv_q_chan", "conv_k_seq", "conv_k_chan"):
+            if getattr(lay, w) is not None and lay.conv_width > 0:
+                names.append(w)
+        _fd_check(lay, x, dout, names, 12, r, 1e-6, what)
+
+
+def pin_attention_backward_closed_forms():
+    """All-ones values make the output independent of the scores, so dq and
+    dk vanish and dv holds the probability-weighted sums of dout (which
+    add up to dout's total per head); a query that sees one key passes its
+    gradient to that key's value unchanged."""
+    r = _rng(32)
+    T, Hq, Hkv, d = 6, 4, 2, 8
+    q = r.standard_normal((T, Hq, d)) * 2
+    k = r.standard_normal((T, Hkv, d)) * 2
+    dout = r.standard_normal((T, Hq, d))
+    dq, dk, dv = O.attention_backward(q, k, np.ones((T, Hkv, d)), 2, True, dout)
+    _close(dq, np.zeros_like(dq), 1e-12, "V = 1: dq")
+    _close(dk, np.zeros_like(dk), 1e-12, "V = 1: dk")
+    _close(dv.sum(axis=0), dout.reshape(T, Hkv, 2, d).sum(axis=(0, 2)), 1e-12, "V = 1: dv total")
+    v = r.standard_normal((T, Hkv, d))
+    dq, dk, dv = O.attention_backward(q[:1], k, v, 2, True, dout[:1])   # position 0: key 0 only
+    _close(dq, np.zeros_like(dq), 1e-12, "one key: dq")
+    _close(dv[0], dout[0].reshape(Hkv, 2, d).sum(axis=1), 1e-12, "one key: dv")
+    _close(dv[1:], np.zeros_like(dv[1:]), 0, "one key: other values")
+
+
+def pin_attention_backward_sdpa():
+    """The attention backward against torch's float64 autograd through
+    scaled_dot_product_attention on copied kv heads (a library special case)."""
+    r = _rng(33)
+    for causal in (True, False):
+        T, Hq, Hkv, d = 9, 6, 2, 8
+        G = Hq // Hkv
+        q = r.standard_normal((T, Hq, d))
+        k = r.standard_normal((T, Hkv, d))
+        v = r.standard_normal((T, Hkv, d))
+        dout = r.standard_normal((T, Hq, d))
+        tq = torch.from_numpy(q.transpose(1, 0, 2).copy()).requires_grad_()
+        tk = torch.from_numpy(k.transpose(1, 0, 2).copy()).requires_grad_()
+        tv = torch.from_numpy(v.transpose(1, 0, 2).copy()).requires_grad_()
+        o = F.scaled_dot_product_attention(tq[None], tk.repeat_interleave(G, 0)[None],
+                                           tv.repeat_interleave(G, 0)[None], is_causal=causal)
+        o.backward(torch.from_numpy(dout.transpose(1, 0, 2).copy())[None])
+        dq, dk, dv = O.attention_backward(q, k, v, G, causal, dout)
+        _close(dq, tq.grad.numpy().transpose(1, 0, 2), 1e-12, f"dq causal={causal}")
+        _close(dk, tk.grad.numpy().transpose(1, 0, 2), 1e-12, f"dk causal={causal}")
+        _close(dv, tv.grad.numpy().transpose(1, 0, 2), 1e-12, f"dv causal={causal}")
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

@@ -13,7 +13,9 @@ import oracle_pins
 _orig = {name: getattr(O, name) for name in
          ("seq_conv", "channel_mix", "qk_mean", "rope", "value_shift", "attention",
           "down_project", "prefill", "decode_step", "_mix_qk", "qk_mean_self",
-          "value_shift_heads", "channel_conv")}
+          "value_shift_heads", "channel_conv", "attention_backward", "_rope_backward",
+          "_value_shift_backward", "_seq_conv_backward", "_channel_conv_backward",
+          "prefill_backward")}
 
 
 def _seq_conv_drop_last_tap(z, w, history=None):
@@ -204,6 +206,63 @@ def _channel_conv_taps_reversed(z, W, history=None):
     return _orig["channel_conv"](z, W[:, ::-1].copy(), history)
 
 
+def _attn_bwd_no_rowsum(q, k, v, G, causal, dout, q_pos=None):
+    T, Hq, d = q.shape
+    L = k.shape[0]
+    pos = np.arange(T) if q_pos is None else np.asarray(q_pos)
+    dq, dk, dv = _orig["attention_backward"](q, k, v, G, causal, dout, q_pos)
+    scale = 1.0 / math.sqrt(d)
+    for h in range(Hq):                       # ds = p * dp, the rowsum term dropped
+        g = h // G
+        sc = (q[:, h] @ k[:, g].T) * scale
+        if causal:
+            sc = np.where(np.arange(L)[None, :] <= pos[:, None], sc, -np.inf)
+        p = np.exp(sc - sc.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        ds = p * (dout[:, h] @ v[:, g].T)
+        dq[:, h] = ds @ k[:, g] * scale
+    return dq, dk, dv
+
+
+def _attn_bwd_dk_unscaled(q, k, v, G, causal, dout, q_pos=None):
+    dq, dk, dv = _orig["attention_backward"](q, k, v, G, causal, dout, q_pos)
+    return dq, dk * math.sqrt(q.shape[-1]), dv
+
+
+def _rope_backward_same_angle(dz, positions, base):
+    return _orig["rope"](dz, positions, base)
+
+
+def _value_shift_backward_wrong_way(layer, dv):
+    out = _orig["_value_shift_backward"](layer, dv[::-1].copy())
+    return out[::-1].copy()
+
+
+def _seq_conv_backward_causal(z, w, du):
+    dz, dw = _orig["_seq_conv_backward"](z, w, du)
+    S = z.shape[0]
+    dz2 = np.zeros_like(z)
+    for j in range(w.shape[1]):
+        if j < S:
+            dz2[j:] += w[:, j] * du[: S - j]
+    return dz2, dw
+
+
+def _channel_conv_backward_untransposed(z, W, dy):
+    return _orig["_channel_conv_backward"](z, np.swapaxes(W, 2, 3), dy)
+
+
+def _prefill_backward_qk_no_1_over_g(layer, x, dout):
+    # the QK-mean's key gradient spread to every query head without 1/G
+    lay = dataclasses.replace(layer)
+    g = _orig["prefill_backward"](lay, x, dout)
+    if not layer.qk_mean or int(layer.qk_mean) == O.QK_SELF or layer.sh.G == 1:
+        return g
+    g2 = _orig["prefill_backward"](dataclasses.replace(layer, qk_mean=0), x, dout)
+    g["dx"] = g["dx"] + 0.3 * (g["dx"] - g2["dx"])
+    return g
+
+
 MUTANTS = {
     "seq_conv_drop_last_tap": ("seq_conv", _seq_conv_drop_last_tap),
     "seq_conv_anticausal": ("seq_conv", _seq_conv_anticausal),
@@ -234,6 +293,14 @@ MUTANTS = {
     "value_shift_heads_ceil": ("value_shift_heads", _value_shift_heads_ceil),
     "channel_conv_transposed": ("channel_conv", _channel_conv_transposed),
     "channel_conv_taps_reversed": ("channel_conv", _channel_conv_taps_reversed),
+    "attention_backward_no_rowsum": ("attention_backward", _attn_bwd_no_rowsum),
+    "attention_backward_dk_unscaled": ("attention_backward", _attn_bwd_dk_unscaled),
+    "rope_backward_same_angle": ("_rope_backward", _rope_backward_same_angle),
+    "value_shift_backward_wrong_way": ("_value_shift_backward", _value_shift_backward_wrong_way),
+    "seq_conv_backward_causal": ("_seq_conv_backward", _seq_conv_backward_causal),
+    "channel_conv_backward_untransposed": ("_channel_conv_backward",
+                                           _channel_conv_backward_untransposed),
+    "prefill_backward_qk_term_scaled": ("prefill_backward", _prefill_backward_qk_no_1_over_g),
 }
 
 
