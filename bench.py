@@ -454,6 +454,42 @@ def measure_output_projection(w, steps, dev):
             "tensor_frac": flop / (ms / 1e3) / 1e12 / peaks["bf16_tflops"]}
 
 
+def measure_backward(w, steps, dev):
+    """The backward pass of one prefill workload (ccgqa_prefill_backward: the
+    forward recompute, attention backward, pre-attention transposes, weight
+    gradients and dx), timed with events around each call."""
+    import torch
+    from compressed_latent_grouped_b200.device import DeviceLayer
+    from compressed_latent_grouped_b200.workloads import make_inputs
+    inp = make_inputs(w, seed=0)
+    lay = DeviceLayer(w, inp, device=dev)
+    x = inp["x"].to(dev)
+    dout = torch.randn(w.B, w.S, w.Hq * w.d, generator=torch.Generator().manual_seed(3)
+                       ).to(w.torch_dtype).to(dev)
+    for _ in range(2):
+        lay.prefill_backward(x, dout)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for a, b in evs:
+        a.record()
+        lay.prefill_backward(x, dout)
+        b.record()
+    torch.cuda.synchronize()
+    if lay.error_bits():
+        raise RuntimeError(f"device error bits {lay.error_bits()}")
+    ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+    # attention backward: 2 d FLOP per visible pair for each of QK^T (recomputed
+    # twice), PV (recomputed), dO V^T (twice), dV, dK and dQ
+    pairs = w.B * w.Hq * (w.S * w.S / 2 if w.causal else w.S * w.S)
+    attn_flop = 2.0 * w.d * pairs * 9
+    gemm_flop = 0 if w.packed_input else 2 * 2.0 * w.B * w.S * w.E * w.n_qkv
+    peaks, _ = load_peaks()
+    return {"backward_ms": ms, "tokens_per_s": w.B * w.S / (ms / 1e3),
+            "flop": attn_flop + gemm_flop,
+            "tflops": (attn_flop + gemm_flop) / (ms / 1e3) / 1e12,
+            "tensor_frac": (attn_flop + gemm_flop) / (ms / 1e3) / 1e12 / peaks["bf16_tflops"]}
+
+
 def run_workload_only(args, local):
     """--workload: time one named workload's kernels (profiling runs)."""
     import torch
@@ -469,6 +505,8 @@ def run_workload_only(args, local):
         w = w.with_(decode=True)
     if args.output_projection:
         res = measure_output_projection(w, args.steps, dev)
+    elif args.backward:
+        res = measure_backward(w, args.steps, dev)
     else:
         res = (measure_decode_workload if w.decode else measure_prefill_workload)(
             w, args.steps, dev)
@@ -761,6 +799,8 @@ def main():
                     help="with --workload: time a decode step against a cache of S tokens")
     ap.add_argument("--output-projection", action="store_true",
                     help="with --workload: time the output up-projection of its B S rows")
+    ap.add_argument("--backward", action="store_true",
+                    help="with --workload: time the backward pass of its prefill")
     args = ap.parse_args()
     world, rank, local = dist_setup(args.gpus)
     try:

@@ -35,6 +35,11 @@ class ccgqa_weights(ctypes.Structure):
                 ("conv_k_seq", c_void_p), ("conv_k_chan", c_void_p)]
 
 
+class ccgqa_weight_grads(ctypes.Structure):
+    _fields_ = [("W_qkv", c_void_p), ("conv_q_seq", c_void_p), ("conv_q_chan", c_void_p),
+                ("conv_k_seq", c_void_p), ("conv_k_chan", c_void_p)]
+
+
 class ccgqa_kvcache(ctypes.Structure):
     _fields_ = [("k", c_void_p), ("v", c_void_p), ("len", c_void_p), ("conv_hist_q", c_void_p),
                 ("conv_hist_k", c_void_p), ("v_prev", c_void_p), ("batch", c_int32),
@@ -86,6 +91,12 @@ def load() -> ctypes.CDLL:
     lib.ccgqa_output_projection.argtypes = [P(ccgqa_config), c_void_p, c_void_p, ctypes.c_int64,
                                             c_void_p, c_void_p, c_void_p]
     lib.ccgqa_output_projection.restype = c_int
+    lib.ccgqa_prefill_backward_workspace_size.argtypes = [P(ccgqa_config), c_int32, c_int32]
+    lib.ccgqa_prefill_backward_workspace_size.restype = c_size_t
+    lib.ccgqa_prefill_backward.argtypes = [P(ccgqa_config), P(ccgqa_weights), c_void_p, c_int32,
+                                           c_int32, c_void_p, c_void_p, P(ccgqa_weight_grads),
+                                           c_void_p, c_size_t, c_void_p, c_void_p]
+    lib.ccgqa_prefill_backward.restype = c_int
     lib.ccgqa_status_string.argtypes = [c_int]
     lib.ccgqa_status_string.restype = c_char_p
     lib.ccgqa_launch_count.argtypes = []
@@ -224,6 +235,30 @@ def ccgqa_output_projection(cfg, W_o, o, M, y, dev_err=None, stream=None, check=
                                         _ptr(dev_err), _stream(stream))
     if check and st != 0:
         raise CCGQAError(st, "ccgqa_output_projection")
+    return st
+
+
+def make_weight_grads(W_qkv=None, conv_q_seq=None, conv_q_chan=None, conv_k_seq=None,
+                      conv_k_chan=None) -> ccgqa_weight_grads:
+    return ccgqa_weight_grads(*(None if t is None else t.data_ptr()
+                                for t in (W_qkv, conv_q_seq, conv_q_chan, conv_k_seq, conv_k_chan)))
+
+
+def ccgqa_prefill_backward_workspace_size(cfg: ccgqa_config, batch: int, seq_len: int) -> int:
+    return load().ccgqa_prefill_backward_workspace_size(ctypes.byref(cfg), batch, seq_len)
+
+
+def ccgqa_prefill_backward(cfg, weights, x, batch, seq_len, dout, dx, grads, workspace,
+                           dev_err=None, stream=None, check=True) -> int:
+    lib = load()
+    st = lib.ccgqa_prefill_backward(ctypes.byref(cfg), ctypes.byref(weights), _ptr(x), batch,
+                                    seq_len, _ptr(dout), _ptr(dx),
+                                    None if grads is None else ctypes.byref(grads),
+                                    _ptr(workspace),
+                                    0 if workspace is None else workspace.numel(),
+                                    _ptr(dev_err), _stream(stream))
+    if check and st != 0:
+        raise CCGQAError(st, "ccgqa_prefill_backward")
     return st
 
 

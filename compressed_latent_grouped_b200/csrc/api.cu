@@ -278,6 +278,151 @@ ccgqa_status run_prefill(const Geo& g, const ccgqa_weights* w, const void* x, in
   return e == cudaSuccess ? CCGQA_OK : cuda_fail(e);
 }
 
+struct BwdWs {
+  size_t z, q, k, v, dq, dk, dv, lse, dsum, dy, dzm, du, u, dz, total;
+};
+BwdWs backward_ws(const Geo& g, int64_t B, int64_t S, bool has_proj) {
+  BwdWs w;
+  const size_t rows = static_cast<size_t>(B * S);
+  const size_t qn = rows * g.Hq * g.d, kvn = rows * g.Hkv * g.d;
+  const size_t cqk = rows * (g.Hq + g.Hkv) * g.d;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += up256(bytes);
+    return at;
+  };
+  w.z = take(has_proj ? rows * g.N * g.es : 0);
+  w.q = take(qn * g.es);
+  w.k = take(kvn * g.es);
+  w.v = take(kvn * g.es);
+  w.dq = take(qn * 4);
+  w.dk = take(kvn * 4);
+  w.dv = take(kvn * 4);
+  w.lse = take(static_cast<size_t>(B) * g.Hq * S * 4);
+  w.dsum = take(static_cast<size_t>(B) * g.Hq * S * 4);
+  w.dy = take(cqk * 4);
+  w.dzm = take(cqk * 4);
+  w.du = take(cqk * 4);
+  w.u = take(cqk * 4);
+  w.dz = take(rows * g.N * 4);
+  w.total = off;
+  return w;
+}
+
+// Elements of each weight gradient (the shapes of the weights).
+size_t grad_elems(const Geo& g, int which) {
+  const size_t d = g.d, K = g.K;
+  switch (which) {
+    case 0: return static_cast<size_t>(g.N) * g.E;                       // W_qkv
+    case 1: return g.channel_conv ? 0 : static_cast<size_t>(g.Hq) * d * K;   // conv_q_seq
+    case 2: return static_cast<size_t>(g.Hq) * d * d * (g.channel_conv ? K : 1);
+    case 3: return g.channel_conv ? 0 : static_cast<size_t>(g.Hkv) * d * K;
+    default: return static_cast<size_t>(g.Hkv) * d * d * (g.channel_conv ? K : 1);
+  }
+}
+
+template <typename T>
+ccgqa_status run_backward(const Geo& g, const ccgqa_weights* w, const void* x, int B, int S,
+                          const void* dout, void* dx, const ccgqa_weight_grads* dw, uint8_t* ws,
+                          int32_t* dev_err, cudaStream_t st) {
+  const BwdWs L = backward_ws(g, B, S, w->W_qkv != nullptr);
+  cudaError_t e = cudaSuccess;
+  // forward values the backward needs: z = q~ | k~ | v~, then q, k, v
+  const T* z = static_cast<const T*>(x);
+  if (w->W_qkv) {
+    T* zw = reinterpret_cast<T*>(ws + L.z);
+    if constexpr (sizeof(T) == 2)
+      e = launch_proj_gemm_bf16(static_cast<const bf16*>(x), static_cast<const bf16*>(w->W_qkv),
+                                zw, B * S, g.N, g.E, dev_err, st);
+    else
+      e = launch_proj_gemm_f32(static_cast<const float*>(x), static_cast<const float*>(w->W_qkv),
+                               zw, B * S, g.N, g.E, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    z = zw;
+  }
+  PreAttnArgs<T> p{};
+  p.src = z;
+  p.src_ld = g.N;
+  p.B = B;
+  p.S = S;
+  p.Hq = g.Hq;
+  p.Hkv = g.Hkv;
+  p.d = g.d;
+  p.G = g.G;
+  p.K = g.K;
+  p.qk_mean = g.qk_mean;
+  p.value_shift = g.value_shift;
+  p.channel_conv = g.channel_conv;
+  p.rope_on = g.rope_on;
+  p.rope_log2_base = g.rope_log2_base;
+  if (g.rope_on)
+    for (int i = 0; i < g.d / 2; ++i) p.rope_frac[i] = rope_turn_fraction(g.rope_log2_base, i, g.d);
+  p.wq_seq = static_cast<const T*>(w->conv_q_seq);
+  p.wq_chan = static_cast<const T*>(w->conv_q_chan);
+  p.wk_seq = static_cast<const T*>(w->conv_k_seq);
+  p.wk_chan = static_cast<const T*>(w->conv_k_chan);
+  p.q_out = reinterpret_cast<T*>(ws + L.q);
+  p.k_out = reinterpret_cast<T*>(ws + L.k);
+  p.v_out = reinterpret_cast<T*>(ws + L.v);
+  p.kv_cap = S;
+  p.dev_err = dev_err;
+  if ((e = launch_pre_attn<T>(p, st)) != cudaSuccess) return cuda_fail(e);
+  BwdArgs<T> a{};
+  a.B = B;
+  a.S = S;
+  a.E = g.E;
+  a.N = g.N;
+  a.Hq = g.Hq;
+  a.Hkv = g.Hkv;
+  a.d = g.d;
+  a.G = g.G;
+  a.K = g.K;
+  a.qk_mean = g.qk_mean;
+  a.value_shift = g.value_shift;
+  a.causal = g.causal;
+  a.rope_on = g.rope_on;
+  a.channel_conv = g.channel_conv;
+  for (int i = 0; i < 64; ++i) a.rope_frac[i] = p.rope_frac[i];
+  a.x = static_cast<const T*>(x);
+  a.W = static_cast<const T*>(w->W_qkv);
+  a.wq_seq = p.wq_seq;
+  a.wq_chan = p.wq_chan;
+  a.wk_seq = p.wk_seq;
+  a.wk_chan = p.wk_chan;
+  a.z = z;
+  a.q = p.q_out;
+  a.k = p.k_out;
+  a.v = p.v_out;
+  a.dout = static_cast<const T*>(dout);
+  a.dq = reinterpret_cast<float*>(ws + L.dq);
+  a.dk = reinterpret_cast<float*>(ws + L.dk);
+  a.dv = reinterpret_cast<float*>(ws + L.dv);
+  a.lse = reinterpret_cast<float*>(ws + L.lse);
+  a.dsum = reinterpret_cast<float*>(ws + L.dsum);
+  a.dy = reinterpret_cast<float*>(ws + L.dy);
+  a.dzm = reinterpret_cast<float*>(ws + L.dzm);
+  a.du = reinterpret_cast<float*>(ws + L.du);
+  a.u = reinterpret_cast<float*>(ws + L.u);
+  a.dz = reinterpret_cast<float*>(ws + L.dz);
+  a.dx = static_cast<T*>(dx);
+  if (dw) {
+    float* outs[5] = {dw->W_qkv, dw->conv_q_seq, dw->conv_q_chan, dw->conv_k_seq, dw->conv_k_chan};
+    for (int i = 0; i < 5; ++i) {
+      const size_t n = grad_elems(g, i);
+      if (outs[i] && n > 0 && (e = cudaMemsetAsync(outs[i], 0, n * 4, st)) != cudaSuccess)
+        return cuda_fail(e);
+    }
+    a.g_W = dw->W_qkv;
+    a.g_q_seq = dw->conv_q_seq;
+    a.g_q_chan = dw->conv_q_chan;
+    a.g_k_seq = dw->conv_k_seq;
+    a.g_k_chan = dw->conv_k_chan;
+  }
+  e = launch_backward<T>(a, st);
+  return e == cudaSuccess ? CCGQA_OK : cuda_fail(e);
+}
+
 template <typename T>
 ccgqa_status run_decode(const Geo& g, const ccgqa_weights* w, const void* x_t,
                         const ccgqa_kvcache* c, void* out, uint8_t* ws, int32_t* dev_err,
@@ -511,6 +656,41 @@ CCGQA_API ccgqa_status ccgqa_output_projection(const ccgqa_config* cfg, const vo
                              static_cast<float*>(y), static_cast<int>(M), N, K, st);
   }
   return e == cudaSuccess ? CCGQA_OK : cuda_fail(e);
+}
+
+CCGQA_API size_t ccgqa_prefill_backward_workspace_size(const ccgqa_config* cfg, int32_t batch,
+                                                       int32_t seq_len) {
+  Geo g;
+  if (derive(cfg, &g) != CCGQA_OK || batch <= 0 || seq_len <= 0) return 0;
+  return backward_ws(g, batch, seq_len, true).total;
+}
+
+CCGQA_API ccgqa_status ccgqa_prefill_backward(const ccgqa_config* cfg, const ccgqa_weights* w,
+                                              const void* x, int32_t batch, int32_t seq_len,
+                                              const void* dout, void* dx,
+                                              const ccgqa_weight_grads* dw, void* workspace,
+                                              size_t workspace_bytes, int32_t* dev_err,
+                                              void* stream) {
+  Geo g;
+  ccgqa_status s = derive(cfg, &g);
+  if (s != CCGQA_OK) return s;
+  if ((s = check_weights(g, w)) != CCGQA_OK) return s;
+  if (batch <= 0 || seq_len <= 0) return CCGQA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(batch) * seq_len > (int64_t(1) << 30)) return CCGQA_ERR_UNSUPPORTED;
+  if (!x || !dout || !dx || !aligned16(x) || !aligned16(dout) || !aligned16(dx))
+    return CCGQA_ERR_INVALID_ARG;
+  if (!pre_attn_fits(g.K, g.G, g.d, static_cast<int>(g.es),
+                     g.K > 0 && !g.channel_conv && (w->conv_q_chan || w->conv_k_chan)))
+    return CCGQA_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) ||
+      workspace_bytes < backward_ws(g, batch, seq_len, w->W_qkv != nullptr).total)
+    return CCGQA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!stream_allowed(st)) return CCGQA_ERR_INVALID_ARG;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (g.dtype == CCGQA_BF16)
+    return run_backward<bf16>(g, w, x, batch, seq_len, dout, dx, dw, ws, dev_err, st);
+  return run_backward<float>(g, w, x, batch, seq_len, dout, dx, dw, ws, dev_err, st);
 }
 
 CCGQA_API const char* ccgqa_status_string(ccgqa_status s) {

@@ -130,6 +130,30 @@ cudaError_t launch_decode_attn_tc(const DecodeArgs<bf16>& a, cudaStream_t stream
 // fits for this group size and head dim.
 bool decode_pre_fits(int G, int d, int K, int es);
 
+// ----------------------------------------------------------------- backward
+// Backward pass of a prefill (ccgqa_prefill_backward).  Forward values z, q,
+// k, v were recomputed into the workspace; every gradient buffer is fp32.
+template <typename T>
+struct BwdArgs {
+  int B, S, E, N, Hq, Hkv, d, G, K;
+  int qk_mean, value_shift, causal, rope_on, channel_conv;
+  uint64_t rope_frac[64];      // as in PreAttnArgs
+  const T* x;                  // [B S, E] (or the packed rows when W is null)
+  const T* W;                  // [N, E] or null
+  const T *wq_seq, *wq_chan, *wk_seq, *wk_chan;
+  const T* z;                  // [B S, N] q~ | k~ | v~ (the projection output, or x)
+  const T *q, *k, *v;          // [B, S, Hq, d], [B, Hkv, S, d] x 2
+  const T* dout;               // [B, S, Hq, d]
+  float *dq, *dk, *dv;         // like q, k, v
+  float *lse, *dsum;           // [B, Hq, S]: log-sum-exp and rowsum(dO * O)
+  float *dy, *dzm, *du, *u;    // [B S, (Hq + Hkv) d]
+  float* dz;                   // [B S, N]
+  T* dx;                       // [B S, E] (or [B S, N] for packed input)
+  float *g_W, *g_q_seq, *g_q_chan, *g_k_seq, *g_k_chan;   // nullable, zeroed first
+};
+template <typename T>
+cudaError_t launch_backward(const BwdArgs<T>& a, cudaStream_t stream);
+
 // Split plan for the decode step, shared by the workspace-size query and the launch.
 void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int es,
                  int* e_splits, int* splits, int* chunk);

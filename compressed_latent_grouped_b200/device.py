@@ -112,6 +112,27 @@ class DeviceLayer:
         B.ccgqa_output_projection(self.cfg, W_o, o, M, y, self.dev_err, stream)
         return y
 
+    def prefill_backward(self, x: torch.Tensor, dout: torch.Tensor, with_weights: bool = True,
+                         stream=None):
+        """Gradients of a prefill (from an empty state) for the output gradient
+        dout [B, S, Hq d]: returns (dx, {weight name: fp32 gradient or None})."""
+        batch, seq_len = x.shape[0], x.shape[1]
+        n = B.ccgqa_prefill_backward_workspace_size(self.cfg, batch, seq_len)
+        if n == 0:
+            raise B.CCGQAError(1, "ccgqa_prefill_backward_workspace_size")
+        ws = torch.empty(n, dtype=torch.uint8, device=self.device)
+        dx = torch.empty_like(x)
+        grads = {"W_qkv": self.W_qkv, **self.conv}
+        g = {k: (torch.empty(v.shape, dtype=torch.float32, device=self.device)
+                 if (with_weights and v is not None) else None) for k, v in grads.items()}
+        if self.w.channel_conv:
+            g["conv_q_seq"] = g["conv_k_seq"] = None
+        wg = B.make_weight_grads(g["W_qkv"], g["conv_q_seq"], g["conv_q_chan"], g["conv_k_seq"],
+                                 g["conv_k_chan"])
+        B.ccgqa_prefill_backward(self.cfg, self.weights, x, batch, seq_len, dout, dx, wg, ws,
+                                 self.dev_err, stream)
+        return dx, g
+
     def error_bits(self) -> int:
         return int(self.dev_err.item())
 

@@ -212,6 +212,53 @@ CCGQA_API ccgqa_status ccgqa_kvcache_append(const ccgqa_config* cfg, const ccgqa
                                             const void* k_new, const void* v_new,
                                             int32_t n_new, int32_t* dev_err, void* stream);
 
+/* Gradient buffers of the layer's weights for ccgqa_prefill_backward: fp32,
+ * device, caller-owned, each with the shape of its weight (conv_*_chan of the
+ * temporal channel conv included).  Any entry may be NULL (that gradient is
+ * not computed); the call zero-fills the others and then writes them. */
+typedef struct {
+  float* W_qkv;         /* [N_qkv, E] */
+  float* conv_q_seq;    /* [Hq d, K] (depthwise taps) */
+  float* conv_q_chan;   /* [Hq, d, d], or [Hq, K, d, d] with channel_conv = 1 */
+  float* conv_k_seq;    /* [Hkv d, K] */
+  float* conv_k_chan;   /* [Hkv, d, d], or [Hkv, K, d, d] with channel_conv = 1 */
+} ccgqa_weight_grads;
+
+/* Workspace bytes of ccgqa_prefill_backward for `batch` sequences of
+ * `seq_len` tokens (0 on an invalid configuration). */
+CCGQA_API size_t ccgqa_prefill_backward_workspace_size(const ccgqa_config* cfg, int32_t batch,
+                                                       int32_t seq_len);
+
+/* Backward pass of ccgqa_prefill (from an empty state, no cache): given the
+ * gradient dout of the prefill's output, the gradient of the input and of the
+ * weights.  The CCA page ("Compressed Convolutional Attention", Resultaten 2)
+ * trains the layer and reports its backward pass; its steps are the
+ * transposes of the forward steps in reverse order: attention (dQ, dK, dV,
+ * with a kv head's gradients summed over its G query heads), value-shift,
+ * RoPE, QK-mean, channel mix or temporal channel conv, sequence conv,
+ * projection.
+ *  - x:    [batch, seq_len, E] (or the packed q~|k~|v~ rows when W_qkv is NULL),
+ *          the same input the forward was given;
+ *  - dout: [batch, seq_len, Hq*d], gradient of the prefill output;
+ *  - dx:   [batch, seq_len, E] (or [batch, seq_len, N_qkv]) written, cfg->dtype;
+ *  - dw:   weight gradients (fp32), nullable.
+ * x, dout and dx in cfg->dtype, 16-byte aligned, device, caller-owned; dx must
+ * not overlap x or dout.  The forward values the backward needs (projection
+ * output, q, k, v) are recomputed into the workspace (>= the size above,
+ * 256-byte aligned).  Every gradient is accumulated in fp32 on the CUDA cores;
+ * the bf16 path uses the same bf16-rounded q, k and v the forward uses.
+ * Returns the same host-side statuses as ccgqa_prefill (INVALID_ARG,
+ * UNSUPPORTED, WORKSPACE), CCGQA_ERR_CUDA on a launch failure, else CCGQA_OK
+ * (asynchronous on `stream`).  The weight gradients are sums over positions
+ * with atomic adds for the sequence-conv taps, so those bits may differ
+ * between runs; everything else is deterministic. */
+CCGQA_API ccgqa_status ccgqa_prefill_backward(const ccgqa_config* cfg, const ccgqa_weights* w,
+                                              const void* x, int32_t batch, int32_t seq_len,
+                                              const void* dout, void* dx,
+                                              const ccgqa_weight_grads* dw, void* workspace,
+                                              size_t workspace_bytes, int32_t* dev_err,
+                                              void* stream);
+
 /* Output up-projection: the latent attention output mapped back to the model
  * width E.  The CCA page ("Compressed Convolutional Attention", Methodologie
  * item 1) runs the whole attention inside the latent space and leaves the way

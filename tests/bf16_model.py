@@ -193,3 +193,79 @@ def check_within_one_ulp(gpu, model, what=""):
     excess = np.abs(gpu - model) - 2.0 ** -7 * (np.abs(model) + rms)
     worst = float(np.max(excess))
     assert worst <= 0.0, f"{what}: a stored value is {worst:.3e} beyond one ulp (+ one ulp of RMS)"
+
+
+def model_prefill_backward(layer: O.Layer, x: np.ndarray, dout: np.ndarray):
+    """The oracle's backward with the forward values it uses rounded to bf16
+    where the bf16 path rounds them (q~, k~, v~ and q, k, v), and dx rounded
+    to bf16 as the bf16 path stores it; the gradients themselves in float64
+    (the weight gradients stay unrounded: the kernel writes them in fp32).
+    Returns the same dict as O.prefill_backward."""
+    sh = layer.sh
+    S = x.shape[0]
+    d, Hq, Hkv, G = sh.d, sh.Hq, sh.Hkv, sh.G
+    q_pre, k_pre, v_lat = (bf(t) for t in O.down_project(x, layer.W_qkv, sh))
+    conv = layer.conv_width > 0
+    u_q = u_k = None
+    if conv and layer.channel_conv:
+        y_q = O.channel_conv(q_pre, layer.conv_q_chan)
+        y_k = O.channel_conv(k_pre, layer.conv_k_chan)
+    elif conv:
+        u_q = O.seq_conv(q_pre.reshape(S, -1), layer.conv_q_seq).reshape(S, Hq, d)
+        u_k = O.seq_conv(k_pre.reshape(S, -1), layer.conv_k_seq).reshape(S, Hkv, d)
+        y_q = u_q if layer.conv_q_chan is None else O.channel_mix(u_q, layer.conv_q_chan)
+        y_k = u_k if layer.conv_k_chan is None else O.channel_mix(u_k, layer.conv_k_chan)
+    else:
+        y_q, y_k = q_pre.copy(), k_pre.copy()
+    mode = int(layer.qk_mean)
+    if mode == O.QK_SELF:
+        qm, km = O.qk_mean_self(q_pre, y_q, k_pre, y_k)
+    elif mode:
+        m_q, m_k = O.qk_mean(q_pre, k_pre, G)
+        qm, km = y_q + m_q, y_k + m_k
+    else:
+        qm, km = y_q, y_k
+    pos = np.arange(S)
+    q = bf(O.rope(qm, pos, layer.rope_base))
+    k = bf(O.rope(km, pos, layer.rope_base))
+    v = O._shift_values(layer, v_lat)
+    dq, dk, dv = O.attention_backward(q, k, v, G, layer.causal, dout.reshape(S, Hq, d))
+    dv_lat = O._value_shift_backward(layer, dv)
+    dqm = O._rope_backward(dq, pos, layer.rope_base)
+    dkm = O._rope_backward(dk, pos, layer.rope_base)
+    if mode == O.QK_SELF:
+        dy_q, dy_k, dq_pre, dk_pre = 0.5 * dqm, 0.5 * dkm, 0.5 * dqm, 0.5 * dkm
+    elif mode:
+        dy_q, dy_k = dqm, dkm
+        dq_pre = 0.5 * dqm + (0.5 / G) * np.repeat(dkm, G, axis=1)
+        dk_pre = 0.5 * dqm.reshape(S, Hkv, G, d).sum(axis=2) + 0.5 * dkm
+    else:
+        dy_q, dy_k = dqm, dkm
+        dq_pre, dk_pre = np.zeros_like(q_pre), np.zeros_like(k_pre)
+    grads = {"conv_q_seq": None, "conv_q_chan": None, "conv_k_seq": None, "conv_k_chan": None}
+    if conv and layer.channel_conv:
+        dz, grads["conv_q_chan"] = O._channel_conv_backward(q_pre, layer.conv_q_chan, dy_q)
+        dq_pre = dq_pre + dz
+        dz, grads["conv_k_chan"] = O._channel_conv_backward(k_pre, layer.conv_k_chan, dy_k)
+        dk_pre = dk_pre + dz
+    elif conv:
+        for side, z, u, dy, Wc, ws in (("q", q_pre, u_q, dy_q, layer.conv_q_chan, layer.conv_q_seq),
+                                       ("k", k_pre, u_k, dy_k, layer.conv_k_chan, layer.conv_k_seq)):
+            if Wc is None:
+                du = dy
+            else:
+                du = np.einsum("hij,thi->thj", Wc, dy)
+                grads[f"conv_{side}_chan"] = np.einsum("thi,thj->hij", dy, u)
+            dz, grads[f"conv_{side}_seq"] = O._seq_conv_backward(z.reshape(S, -1), ws,
+                                                                 du.reshape(S, -1))
+            if side == "q":
+                dq_pre = dq_pre + dz.reshape(dq_pre.shape)
+            else:
+                dk_pre = dk_pre + dz.reshape(dk_pre.shape)
+    else:
+        dq_pre = dq_pre + dy_q
+        dk_pre = dk_pre + dy_k
+    dzq = np.concatenate([dq_pre.reshape(S, -1), dk_pre.reshape(S, -1), dv_lat.reshape(S, -1)], axis=1)
+    if layer.W_qkv is None:
+        return {"dx": bf(dzq), "W_qkv": None, **grads}
+    return {"dx": bf(dzq @ layer.W_qkv), "W_qkv": dzq.T @ x, **grads}

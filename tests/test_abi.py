@@ -204,3 +204,23 @@ def test_output_projection_checked_on_host(lib):
     bad = B.make_config(E=500, C=4, n_q_heads=4, n_kv_heads=2)  # E not a multiple of C Hq
     assert f(ctypes.byref(bad), fake, fake, 4, fake, None, None) == 1
     assert B.ccgqa_launch_count() == 0
+
+
+def test_backward_checked_on_host(lib):
+    """ccgqa_prefill_backward validates before any launch (no GPU needed)."""
+    cfg = _cfg()
+    assert B.ccgqa_prefill_backward_workspace_size(cfg, 2, 128) > 0
+    assert B.ccgqa_prefill_backward_workspace_size(_cfg(n_kv_heads=3), 2, 128) == 0
+    w = B.make_weights()           # conv taps missing for conv_width 4
+    fake = ctypes.c_void_p(1 << 20)
+    f = lib.ccgqa_prefill_backward
+    assert f(ctypes.byref(cfg), ctypes.byref(w), fake, 1, 16, fake, fake, None, fake,
+             1 << 30, None, None) == 1
+    w0 = B.make_weights()
+    cfg0 = _cfg(conv_width=0, qk_mean=0, value_shift=0)
+    assert f(ctypes.byref(cfg0), ctypes.byref(w0), None, 1, 16, fake, fake, None, fake,
+             1 << 30, None, None) == 1                                   # no input
+    assert f(ctypes.byref(cfg0), ctypes.byref(w0), fake, 0, 16, fake, fake, None, fake,
+             1 << 30, None, None) == 1                                   # empty batch
+    assert f(ctypes.byref(cfg0), ctypes.byref(w0), fake, 1, 16, fake, fake, None, None,
+             0, None, None) == 4                                         # no workspace
