@@ -352,15 +352,26 @@ def measure_prefill_workload(w, steps, dev):
     return res
 
 
-def setup_decode(w, dev, seed=0, extra_cap=64):
+def setup_decode(w, dev, seed=0, extra_cap=64, page=0):
     """A decode layer whose caches hold w.S tokens per sequence, plus the
-    device tensor that resets the lengths to w.S between timed steps."""
+    device tensor that resets the lengths to w.S between timed steps.  With
+    ``page`` > 0 the cache is a pool of pages of that many tokens named by a
+    seeded block table (a sequence's pages scattered over the pool)."""
     import torch
     from compressed_latent_grouped_b200.device import DeviceLayer
-    from compressed_latent_grouped_b200.workloads import make_inputs
+    from compressed_latent_grouped_b200.workloads import make_block_table, make_inputs
     inp = make_inputs(w, seed=seed)
-    lay = DeviceLayer(w, inp, device=dev, cap=w.S + extra_cap)
-    t = lay.alloc_cache()
+    cap = w.S + extra_cap
+    lay = DeviceLayer(w, inp, device=dev, cap=cap)
+    if page > 0:
+        cap = (cap + page - 1) // page * page
+        per_seq = cap // page
+        n_pages = w.B * per_seq + 16
+        lay.cap = cap
+        t = lay.alloc_cache(cap=cap, block_table=make_block_table(w.B, per_seq, n_pages, seed),
+                            page_size=page, n_pages=n_pages)
+    else:
+        t = lay.alloc_cache()
     lay.append(inp["cache_k"].to(dev), inp["cache_v"].to(dev))
     t["hist_q"].copy_(inp["hist_q"])
     t["hist_k"].copy_(inp["hist_k"])
@@ -384,12 +395,13 @@ def decode_numbers(w, proj_ms, pre_ms, attn_ms, step_ms, peaks):
             "tokens_per_s": w.B / (step / 1e3)}
 
 
-def measure_decode_workload(w, steps, dev):
-    """Decode step on a full latent cache: device times of the projection,
-    the one-token pre-step and the split-K attention over len + 1 keys."""
+def measure_decode_workload(w, steps, dev, page=0):
+    """Decode step on a full latent cache (contiguous, or paged with ``page``
+    tokens per page): device times of the projection, the one-token pre-step
+    and the split-K attention over len + 1 keys."""
     import torch
     from compressed_latent_grouped_b200 import binding as B
-    lay, inp, len0 = setup_decode(w, dev)
+    lay, inp, len0 = setup_decode(w, dev, page=page)
     x_t = inp["x_t"].to(dev)
     out = torch.empty(w.B, w.Hq * w.d, dtype=w.torch_dtype, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -507,9 +519,10 @@ def run_workload_only(args, local):
         res = measure_output_projection(w, args.steps, dev)
     elif args.backward:
         res = measure_backward(w, args.steps, dev)
+    elif w.decode:
+        res = measure_decode_workload(w, args.steps, dev, page=args.paged)
     else:
-        res = (measure_decode_workload if w.decode else measure_prefill_workload)(
-            w, args.steps, dev)
+        res = measure_prefill_workload(w, args.steps, dev)
     print(json.dumps({"workload": args.workload, "B": w.B, "S": w.S, **res}), flush=True)
 
 
@@ -711,6 +724,11 @@ def run_ours(args, world, rank, local):
             by_workload[name] = measure_prefill_workload(WORKLOADS[name], 20, dev)
         by_workload["bf16_prefill_b4_s4096"]["decode_b4_l4096"] = measure_decode_workload(
             WORKLOADS["bf16_prefill_b4_s4096"].with_(decode=True), 20, dev)
+        # the headline decode step against a paged cache (pages of 64 and 16
+        # tokens, scattered over the pool by a seeded block table)
+        for page in (64, 16):
+            by_workload[f"{DECODE_WL}_paged{page}"] = measure_decode_workload(wd, 20, dev,
+                                                                              page=page)
         torch.cuda.empty_cache()
 
     if rank != 0:
@@ -797,6 +815,8 @@ def main():
     ap.add_argument("--seq", type=int, default=0, help="with --workload: override S (or L)")
     ap.add_argument("--decode", action="store_true",
                     help="with --workload: time a decode step against a cache of S tokens")
+    ap.add_argument("--paged", type=int, default=0,
+                    help="with --workload and a decode: a paged cache of this many tokens per page")
     ap.add_argument("--output-projection", action="store_true",
                     help="with --workload: time the output up-projection of its B S rows")
     ap.add_argument("--backward", action="store_true",

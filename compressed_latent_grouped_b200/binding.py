@@ -43,7 +43,8 @@ class ccgqa_weight_grads(ctypes.Structure):
 class ccgqa_kvcache(ctypes.Structure):
     _fields_ = [("k", c_void_p), ("v", c_void_p), ("len", c_void_p), ("conv_hist_q", c_void_p),
                 ("conv_hist_k", c_void_p), ("v_prev", c_void_p), ("batch", c_int32),
-                ("cap", c_int32)]
+                ("cap", c_int32), ("block_table", c_void_p), ("page_size", c_int32),
+                ("n_pages", c_int32)]
 
 
 class CCGQAError(RuntimeError):
@@ -164,12 +165,21 @@ def make_weights(W_qkv=None, conv_q_seq=None, conv_q_chan=None, conv_k_seq=None,
                            for t in (W_qkv, conv_q_seq, conv_q_chan, conv_k_seq, conv_k_chan)))
 
 
-def make_kvcache(k, v, len_, conv_hist_q=None, conv_hist_k=None, v_prev=None) -> ccgqa_kvcache:
-    batch, _, cap, _ = k.shape
-    return ccgqa_kvcache(k.data_ptr(), v.data_ptr(), len_.data_ptr(),
-                         None if conv_hist_q is None else conv_hist_q.data_ptr(),
-                         None if conv_hist_k is None else conv_hist_k.data_ptr(),
-                         None if v_prev is None else v_prev.data_ptr(), batch, cap)
+def make_kvcache(k, v, len_, conv_hist_q=None, conv_hist_k=None, v_prev=None,
+                 block_table=None) -> ccgqa_kvcache:
+    """Contiguous cache: k, v [batch, Hkv, cap, d].  Paged cache: k, v are the
+    pool [n_pages, Hkv, page_size, d] and block_table [batch, cap / page_size]
+    (int32) names each sequence's pages."""
+    ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+    if block_table is None:
+        batch, _, cap, _ = k.shape
+        return ccgqa_kvcache(k.data_ptr(), v.data_ptr(), len_.data_ptr(), ptr(conv_hist_q),
+                             ptr(conv_hist_k), ptr(v_prev), batch, cap, None, 0, 0)
+    n_pages, _, page_size, _ = k.shape
+    batch, per_seq = block_table.shape
+    return ccgqa_kvcache(k.data_ptr(), v.data_ptr(), len_.data_ptr(), ptr(conv_hist_q),
+                         ptr(conv_hist_k), ptr(v_prev), batch, per_seq * page_size,
+                         block_table.data_ptr(), page_size, n_pages)
 
 
 # ------------------------------------------------------------------ entry points

@@ -145,7 +145,29 @@ ccgqa_status check_cache(const Geo& g, const ccgqa_kvcache* c, bool need_state) 
     if (g.K > 1 && (!c->conv_hist_q || !c->conv_hist_k)) return CCGQA_ERR_INVALID_ARG;
     if (g.value_shift && !c->v_prev) return CCGQA_ERR_INVALID_ARG;
   }
+  if (c->block_table) {
+    // pages of a power-of-two size from 16 to 4096 tokens that divides cap;
+    // the pool's page planes (n_pages * Hkv) index a TMA coordinate (int32)
+    const int ps = c->page_size;
+    if (ps < 16 || ps > 4096 || (ps & (ps - 1)) || c->cap % ps) return CCGQA_ERR_INVALID_ARG;
+    if (c->n_pages <= 0 || static_cast<int64_t>(c->n_pages) * g.Hkv >= (int64_t(1) << 31))
+      return CCGQA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(c->block_table) & 3) return CCGQA_ERR_INVALID_ARG;
+  }
   return CCGQA_OK;
+}
+
+PageMap page_map(const ccgqa_kvcache* c) {
+  PageMap pm{};
+  if (c && c->block_table) {
+    pm.table = c->block_table;
+    int sh = 0;
+    while ((1 << sh) < c->page_size) ++sh;
+    pm.shift = sh;
+    pm.per_seq = c->cap >> sh;
+    pm.n_pages = c->n_pages;
+  }
+  return pm;
 }
 
 struct PrefillWs {
@@ -236,18 +258,22 @@ ccgqa_status run_prefill(const Geo& g, const ccgqa_weights* w, const void* x, in
   a.wk_seq = static_cast<const T*>(w->conv_k_seq);
   a.wk_chan = static_cast<const T*>(w->conv_k_chan);
   a.q_out = reinterpret_cast<T*>(ws + L.q);
-  if (cache) {
+  // a paged cache takes k / v from the workspace after the attention
+  const bool paged = cache && cache->block_table;
+  if (cache && !paged) {
     a.k_out = static_cast<T*>(cache->k);
     a.v_out = static_cast<T*>(cache->v);
     a.kv_cap = cache->cap;
-    a.hist_q = static_cast<T*>(cache->conv_hist_q);
-    a.hist_k = static_cast<T*>(cache->conv_hist_k);
-    a.v_prev = static_cast<T*>(cache->v_prev);
-    a.len = cache->len;
   } else {
     a.k_out = reinterpret_cast<T*>(ws + L.k);
     a.v_out = reinterpret_cast<T*>(ws + L.v);
     a.kv_cap = S;
+  }
+  if (cache) {
+    a.hist_q = static_cast<T*>(cache->conv_hist_q);
+    a.hist_k = static_cast<T*>(cache->conv_hist_k);
+    a.v_prev = static_cast<T*>(cache->v_prev);
+    a.len = cache->len;
   }
   a.dev_err = dev_err;
   if ((e = launch_pre_attn<T>(a, st)) != cudaSuccess) return cuda_fail(e);
@@ -274,6 +300,10 @@ ccgqa_status run_prefill(const Geo& g, const ccgqa_weights* w, const void* x, in
   } else {
     e = launch_attn_prefill_simt<T>(at, st);
   }
+  if (e == cudaSuccess && paged)
+    e = launch_kv_scatter<T>(static_cast<T*>(cache->k), static_cast<T*>(cache->v),
+                             page_map(cache), a.k_out, a.v_out, B, g.Hkv, g.d, cache->cap, S,
+                             dev_err, st);
   phase_mark(3, st);
   return e == cudaSuccess ? CCGQA_OK : cuda_fail(e);
 }
@@ -453,6 +483,7 @@ ccgqa_status run_decode(const Geo& g, const ccgqa_weights* w, const void* x_t,
   a.wk_chan = static_cast<const T*>(w->conv_k_chan);
   a.cache_k = static_cast<T*>(c->k);
   a.cache_v = static_cast<T*>(c->v);
+  a.pages = page_map(c);
   a.len = c->len;
   a.cap = c->cap;
   a.hist_q = static_cast<T*>(c->conv_hist_q);
@@ -623,12 +654,12 @@ CCGQA_API ccgqa_status ccgqa_kvcache_append(const ccgqa_config* cfg, const ccgqa
   cudaError_t e;
   if (g.dtype == CCGQA_BF16)
     e = launch_kv_append<bf16>(static_cast<bf16*>(cache->k), static_cast<bf16*>(cache->v),
-                               cache->len, static_cast<const bf16*>(k_new),
+                               page_map(cache), cache->len, static_cast<const bf16*>(k_new),
                                static_cast<const bf16*>(v_new), cache->batch, g.Hkv, g.d,
                                cache->cap, n_new, dev_err, st);
   else
     e = launch_kv_append<float>(static_cast<float*>(cache->k), static_cast<float*>(cache->v),
-                                cache->len, static_cast<const float*>(k_new),
+                                page_map(cache), cache->len, static_cast<const float*>(k_new),
                                 static_cast<const float*>(v_new), cache->batch, g.Hkv, g.d,
                                 cache->cap, n_new, dev_err, st);
   return e == cudaSuccess ? CCGQA_OK : cuda_fail(e);

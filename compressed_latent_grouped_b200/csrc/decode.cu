@@ -102,13 +102,16 @@ namespace {
 using namespace sm100;
 
 // ----------------------------------------------------------------- kv append
+// Rows i in [0, n) of sequence b go to token t0 + i, t0 = len[b] (append) or
+// 0 (scatter); the source row of (b, i, g) is b sb + i si + g sg.
 template <typename T>
-__global__ void kv_append_kernel(T* __restrict__ ck, T* __restrict__ cv, const int32_t* len,
-                                 const T* __restrict__ kn, const T* __restrict__ vn, int Hkv,
-                                 int d, int64_t cap, int n_new, int32_t* dev_err) {
+__global__ void kv_append_kernel(T* __restrict__ ck, T* __restrict__ cv, const PageMap pm,
+                                 const int32_t* len, const T* __restrict__ kn,
+                                 const T* __restrict__ vn, int64_t sb, int64_t si, int64_t sg,
+                                 int Hkv, int d, int64_t cap, int n_new, int32_t* dev_err) {
   constexpr int VEC = 16 / sizeof(T);
   const int b = blockIdx.y;
-  const int L = len[b];
+  const int L = len ? len[b] : 0;
   if (L < 0 || static_cast<int64_t>(L) + n_new > cap) {
     if (blockIdx.x == 0 && threadIdx.x == 0) raise_dev_err(dev_err, CCGQA_DEVERR_CAPACITY);
     return;
@@ -121,8 +124,13 @@ __global__ void kv_append_kernel(T* __restrict__ ck, T* __restrict__ cv, const i
     const int64_t rg = idx / nch;
     const int g = static_cast<int>(rg % Hkv);
     const int64_t i = rg / Hkv;
-    const int64_t src = ((static_cast<int64_t>(b) * n_new + i) * Hkv + g) * d + c * VEC;
-    const int64_t dst = ((static_cast<int64_t>(b) * Hkv + g) * cap + L + i) * d + c * VEC;
+    const int64_t src = (b * sb + i * si + g * sg) * d + c * VEC;
+    const int64_t row = kv_row(pm, b, g, Hkv, cap, L + i);
+    if (row < 0) {
+      raise_dev_err(dev_err, CCGQA_DEVERR_INDEX);
+      continue;
+    }
+    const int64_t dst = row * d + c * VEC;
     *reinterpret_cast<uint4*>(ck + dst) = *reinterpret_cast<const uint4*>(kn + src);
     *reinterpret_cast<uint4*>(cv + dst) = *reinterpret_cast<const uint4*>(vn + src);
   }
@@ -511,6 +519,14 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
     if (g == 0 && tid == 0) raise_dev_err(a.dev_err, CCGQA_DEVERR_CAPACITY);
     return;
   }
+  // Paged cache: bring the sequence's block-table entries for tokens 0..L into
+  // L2, so that the attention's CTAs find their page ids there when they start.
+  if (a.pages.table != nullptr && g == 0) {
+    const int32_t* row = a.pages.table + static_cast<int64_t>(b) * a.pages.per_seq;
+    const int last = L >> a.pages.shift;
+    for (int i = tid * 32; i <= last; i += blockDim.x * 32) prefetch_l2(row + i);
+    if (tid == 0) prefetch_l2(row + last);   // the row need not start on a line
+  }
   const int qcol0 = g * G * d, kcol0 = a.Hq * d + g * d, vcol0 = (a.Hq + a.Hkv) * d + g * d;
   // temporal channel conv: per-tap d x d matrices (wq_chan [Hq, K, d, d]), no depthwise taps
   const bool full = a.channel_conv && K > 0;
@@ -648,7 +664,10 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
   }
   __syncthreads();
   // RoPE at position L on (i, i + d/2), then q -> workspace, k -> cache row L
-  const int64_t crow = ((static_cast<int64_t>(b) * a.Hkv + g) * a.cap + L) * d;
+  // (a page id outside the pool: the cache row is not written)
+  const int64_t crow_i = kv_row(a.pages, b, g, a.Hkv, a.cap, L);
+  const int64_t crow = crow_i * d;
+  if (crow_i < 0 && tid == 0) raise_dev_err(a.dev_err, CCGQA_DEVERR_INDEX);
   for (int idx = tid; idx < (G + 1) * half; idx += blockDim.x) {
     const int hh = idx / half, i = idx - hh * half;
     float ya = y[hh * d + i], yb = y[hh * d + i + half];
@@ -666,7 +685,7 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
       float* qd = a.q_ws + (static_cast<int64_t>(b) * a.Hq + g * G + hh) * d;
       qd[i] = ya;
       qd[i + half] = yb;
-    } else {
+    } else if (crow_i >= 0) {
       a.cache_k[crow + i] = from_f32<T>(ya);
       a.cache_k[crow + i + half] = from_f32<T>(yb);
     }
@@ -676,7 +695,7 @@ __global__ void __launch_bounds__(kPreThreads) decode_pre_kernel(const __grid_co
     T v = from_f32<T>(zc[HC + i]);
     if ((a.value_shift == 1 && i >= half) || shift_head)
       v = a.v_prev[static_cast<int64_t>(b) * a.Hkv * d + g * d + i];
-    a.cache_v[crow + i] = v;
+    if (crow_i >= 0) a.cache_v[crow + i] = v;
   }
   __syncthreads();
   // state: histories shift by one row, v_prev = this row's v~
@@ -720,6 +739,40 @@ __host__ __device__ inline int dec_head_chunks(int G) {
   return (G + per - 1) / per;
 }
 
+// One stage of a paged cache: one bulk copy per run of rows within a page (the
+// bytes are counted in a first pass); a page id outside the pool is not loaded
+// (its rows keep what the stage held) and raises the index bit.  Kept out of
+// line: only the issuing thread runs it.
+template <typename T, int D>
+__device__ __noinline__ void issue_paged_rows(const PageMap pm, const T* ck, const T* cv, int Hkv,
+                                              int64_t cap, int32_t* dev_err, int b, int g,
+                                              int key0, int rows, uint8_t* dst_k, uint8_t* dst_v,
+                                              uint64_t* bar) {
+  const int psz = 1 << pm.shift;
+  uint32_t tx = 0;
+  for (int r = 0; r < rows;) {
+    const int t = key0 + r;
+    const int run = min(rows - r, psz - (t & (psz - 1)));
+    if (kv_row(pm, b, g, Hkv, cap, t) >= 0)
+      tx += 2u * static_cast<uint32_t>(run) * D * sizeof(T);
+    else
+      raise_dev_err(dev_err, CCGQA_DEVERR_INDEX);
+    r += run;
+  }
+  mbar_arrive_expect_tx(bar, tx);
+  for (int r = 0; r < rows;) {
+    const int t = key0 + r;
+    const int run = min(rows - r, psz - (t & (psz - 1)));
+    const int64_t row = kv_row(pm, b, g, Hkv, cap, t);
+    if (row >= 0) {
+      const uint32_t nb = static_cast<uint32_t>(run) * D * sizeof(T);
+      bulk_load(dst_k + r * D * sizeof(T), ck + row * D, nb, bar);
+      bulk_load(dst_v + r * D * sizeof(T), cv + row * D, nb, bar);
+    }
+    r += run;
+  }
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kDecThreads)
     decode_attn_kernel(const DecodeArgs<T> a) {
@@ -745,7 +798,6 @@ __global__ void __launch_bounds__(kDecThreads)
   const int k1 = min(k0 + a.chunk, n_keys);
   const int nk = max(0, k1 - k0);
   const int n_st = (nk + C::KS - 1) / C::KS;
-  const int64_t kv_base = (static_cast<int64_t>(b) * a.Hkv + g) * a.cap * D;
 
   if (tid == 0) {
     for (int s = 0; s < kDecStages; ++s) mbar_init(&full[s], 1);
@@ -759,10 +811,15 @@ __global__ void __launch_bounds__(kDecThreads)
     const int rows = min(C::KS, k1 - key0);
     const uint32_t bytes = static_cast<uint32_t>(rows) * D * sizeof(T);
     uint8_t* dst = ring + s * C::kStageBytes;
-    mbar_arrive_expect_tx(&full[s], 2 * bytes);
-    bulk_load(dst, a.cache_k + kv_base + static_cast<int64_t>(key0) * D, bytes, &full[s]);
-    bulk_load(dst + C::kStageBytes / 2, a.cache_v + kv_base + static_cast<int64_t>(key0) * D, bytes,
-              &full[s]);
+    if (a.pages.table == nullptr) {
+      const int64_t row0 = (static_cast<int64_t>(b) * a.Hkv + g) * a.cap + key0;
+      mbar_arrive_expect_tx(&full[s], 2 * bytes);
+      bulk_load(dst, a.cache_k + row0 * D, bytes, &full[s]);
+      bulk_load(dst + C::kStageBytes / 2, a.cache_v + row0 * D, bytes, &full[s]);
+      return;
+    }
+    issue_paged_rows<T, D>(a.pages, a.cache_k, a.cache_v, a.Hkv, a.cap, a.dev_err, b, g, key0,
+                           rows, dst, dst + C::kStageBytes / 2, &full[s]);
   };
   if (tid == 0)
     for (int i = 0; i < kDecStages && i < n_st; ++i) issue(i);
@@ -947,20 +1004,43 @@ cudaError_t launch_dec_attn(const DecodeArgs<T>& a, cudaStream_t stream) {
 
 }  // namespace
 
+namespace {
 template <typename T>
-cudaError_t launch_kv_append(T* cache_k, T* cache_v, int32_t* len, const T* k_new,
-                             const T* v_new, int B, int Hkv, int d, int64_t cap, int n_new,
-                             int32_t* dev_err, cudaStream_t stream) {
-  const int64_t chunks = static_cast<int64_t>(n_new) * Hkv * (d * sizeof(T) / 16);
+cudaError_t launch_rows_copy(T* ck, T* cv, const PageMap& pm, const int32_t* len, const T* kn,
+                             const T* vn, int64_t sb, int64_t si, int64_t sg, int B, int Hkv,
+                             int d, int64_t cap, int n, int32_t* dev_err, cudaStream_t stream) {
+  const int64_t chunks = static_cast<int64_t>(n) * Hkv * (d * sizeof(T) / 16);
   int64_t blocks = (chunks + 255) / 256;
   if (blocks > 4096) blocks = 4096;
   if (blocks < 1) blocks = 1;
   dim3 grid(static_cast<unsigned>(blocks), B);
-  kv_append_kernel<T><<<grid, 256, 0, stream>>>(cache_k, cache_v, len, k_new, v_new, Hkv, d, cap,
-                                                n_new, dev_err);
-  len_add_kernel<<<(B + 127) / 128, 128, 0, stream>>>(len, B, cap, n_new);
-  count_launches(2);
+  kv_append_kernel<T><<<grid, 256, 0, stream>>>(ck, cv, pm, len, kn, vn, sb, si, sg, Hkv, d, cap,
+                                                n, dev_err);
+  count_launches(1);
   return cudaGetLastError();
+}
+}  // namespace
+
+template <typename T>
+cudaError_t launch_kv_append(T* cache_k, T* cache_v, const PageMap& pm, int32_t* len,
+                             const T* k_new, const T* v_new, int B, int Hkv, int d, int64_t cap,
+                             int n_new, int32_t* dev_err, cudaStream_t stream) {
+  const cudaError_t e = launch_rows_copy<T>(cache_k, cache_v, pm, len, k_new, v_new,
+                                            static_cast<int64_t>(n_new) * Hkv, Hkv, 1, B, Hkv, d,
+                                            cap, n_new, dev_err, stream);
+  if (e != cudaSuccess) return e;
+  len_add_kernel<<<(B + 127) / 128, 128, 0, stream>>>(len, B, cap, n_new);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_kv_scatter(T* cache_k, T* cache_v, const PageMap& pm, const T* k_src,
+                              const T* v_src, int B, int Hkv, int d, int64_t cap, int S,
+                              int32_t* dev_err, cudaStream_t stream) {
+  return launch_rows_copy<T>(cache_k, cache_v, pm, nullptr, k_src, v_src,
+                             static_cast<int64_t>(Hkv) * S, 1, S, B, Hkv, d, cap, S, dev_err,
+                             stream);
 }
 
 bool decode_pre_fits(int G, int d, int K, int es) {
@@ -1028,10 +1108,18 @@ cudaError_t launch_decode_step(const DecodeArgs<T>& a, cudaStream_t stream) {
   return e;
 }
 
-template cudaError_t launch_kv_append<float>(float*, float*, int32_t*, const float*, const float*,
-                                             int, int, int, int64_t, int, int32_t*, cudaStream_t);
-template cudaError_t launch_kv_append<bf16>(bf16*, bf16*, int32_t*, const bf16*, const bf16*, int,
-                                            int, int, int64_t, int, int32_t*, cudaStream_t);
+template cudaError_t launch_kv_append<float>(float*, float*, const PageMap&, int32_t*,
+                                             const float*, const float*, int, int, int, int64_t,
+                                             int, int32_t*, cudaStream_t);
+template cudaError_t launch_kv_append<bf16>(bf16*, bf16*, const PageMap&, int32_t*, const bf16*,
+                                            const bf16*, int, int, int, int64_t, int, int32_t*,
+                                            cudaStream_t);
+template cudaError_t launch_kv_scatter<float>(float*, float*, const PageMap&, const float*,
+                                              const float*, int, int, int, int64_t, int, int32_t*,
+                                              cudaStream_t);
+template cudaError_t launch_kv_scatter<bf16>(bf16*, bf16*, const PageMap&, const bf16*,
+                                             const bf16*, int, int, int, int64_t, int, int32_t*,
+                                             cudaStream_t);
 template cudaError_t launch_decode_step<float>(const DecodeArgs<float>&, cudaStream_t);
 template cudaError_t launch_decode_step<bf16>(const DecodeArgs<bf16>&, cudaStream_t);
 

@@ -62,7 +62,9 @@ struct DCfg {
   static constexpr uint32_t kOffP = kOffV + kStages * kTileBytes;
   static constexpr uint32_t kOffQ = kOffP + kPBytes;
   static constexpr uint32_t kOffBar = kOffQ + ((kPanels * kQPanelBytes + 1023) & ~1023u);
-  static constexpr size_t kSmem = kOffBar + 1024 + 1024;   // barriers | TMEM slot | red[2][4][16]
+  static constexpr int kMaxIds = 512;                        // page ids staged per split
+  static constexpr uint32_t kOffIds = kOffBar + 1024;        // after barriers | TMEM slot | red[2][4][16]
+  static constexpr size_t kSmem = kOffIds + kMaxIds * 4 + 1024;
   static constexpr uint32_t kColS = 0, kColO = 32, kTmemCols = 64;   // S^T x2 | O^T or O
 };
 
@@ -146,42 +148,110 @@ __global__ void __launch_bounds__(kDecTcThreads, 1)
     // blocking on either: a K slot frees as soon as the S of its chunk is
     // computed, well before the PV that frees the V slot, so the K loads run
     // ahead of the V loads.
-    if (lane == 0) {
-      prefetch_tensormap(&tmK);
-      prefetch_tensormap(&tmV);
-      volatile int* abort_v = &abort_flag;
-      int ck = 0, cv = 0;
-      long long t_last = clock64();
-      while (ck < n_ch || cv < n_ch) {
-        bool progress = false;
-        if (ck < n_ch && mbar_test(&k_empty[ck % C::kStages], ((ck / C::kStages) & 1) ^ 1)) {
-          const int st = ck % C::kStages;
-          mbar_arrive_expect_tx(&k_full[st], C::kTileBytes);
+    volatile int* abort_v = &abort_flag;
+    if (a.pages.table == nullptr) {
+      if (lane == 0) {
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+        int ck = 0, cv = 0;
+        long long t_last = clock64();
+        while (ck < n_ch || cv < n_ch) {
+          bool progress = false;
+          if (ck < n_ch && mbar_test(&k_empty[ck % C::kStages], ((ck / C::kStages) & 1) ^ 1)) {
+            const int st = ck % C::kStages;
+            mbar_arrive_expect_tx(&k_full[st], C::kTileBytes);
 #pragma unroll
-          for (int p = 0; p < C::kPanels; ++p)
-            tma_load_3d(smem + C::kOffK + st * C::kTileBytes + p * C::kPanelBytes, &tmK, &k_full[st],
-                        p * C::kPanelCols, k0 + ck * kChunk, bg);
-          ++ck;
-          progress = true;
-        }
-        if (cv < n_ch && mbar_test(&v_empty[cv % C::kStages], ((cv / C::kStages) & 1) ^ 1)) {
-          const int st = cv % C::kStages;
-          mbar_arrive_expect_tx(&v_full[st], C::kTileBytes);
-#pragma unroll
-          for (int p = 0; p < C::kPanels; ++p)
-            tma_load_3d(smem + C::kOffV + st * C::kTileBytes + p * C::kPanelBytes, &tmV, &v_full[st],
-                        p * C::kPanelCols, k0 + cv * kChunk, bg);
-          ++cv;
-          progress = true;
-        }
-        if (progress) {
-          t_last = clock64();
-        } else if (*abort_v || clock64() - t_last > kWaitLimitCycles) {
-          if (!*abort_v) {
-            *abort_v = 1;
-            raise_dev_err(a.dev_err, CCGQA_DEVERR_TIMEOUT);
+            for (int p = 0; p < C::kPanels; ++p)
+              tma_load_3d(smem + C::kOffK + st * C::kTileBytes + p * C::kPanelBytes, &tmK,
+                          &k_full[st], p * C::kPanelCols, k0 + ck * kChunk, bg);
+            ++ck;
+            progress = true;
           }
-          break;
+          if (cv < n_ch && mbar_test(&v_empty[cv % C::kStages], ((cv / C::kStages) & 1) ^ 1)) {
+            const int st = cv % C::kStages;
+            mbar_arrive_expect_tx(&v_full[st], C::kTileBytes);
+#pragma unroll
+            for (int p = 0; p < C::kPanels; ++p)
+              tma_load_3d(smem + C::kOffV + st * C::kTileBytes + p * C::kPanelBytes, &tmV,
+                          &v_full[st], p * C::kPanelCols, k0 + cv * kChunk, bg);
+            ++cv;
+            progress = true;
+          }
+          if (progress) {
+            t_last = clock64();
+          } else if (*abort_v || clock64() - t_last > kWaitLimitCycles) {
+            if (!*abort_v) {
+              *abort_v = 1;
+              raise_dev_err(a.dev_err, CCGQA_DEVERR_TIMEOUT);
+            }
+            break;
+          }
+        }
+      }
+    } else {
+      // Paged cache: a chunk is nb = 128 / bx boxes of bx = min(page, 128) rows,
+      // each at (row in page, page * Hkv + g) of the pool.  The warp first
+      // stages the split's page ids (box i of the split at ids[i]) in shared
+      // memory, then lane 0 alone polls and issues as for a contiguous cache
+      // (ids past the staged ones are read from global memory).  Boxes wholly
+      // past the sequence are not loaded (their keys are masked and V rows
+      // zeroed); a page id outside the pool becomes a coordinate past the
+      // pool, which TMA fills with zeros.
+      const int shift = a.pages.shift;
+      const int bx = min(1 << shift, kChunk);
+      const int nb = kChunk / bx;
+      const int pool_z = a.pages.n_pages * a.Hkv;
+      const int32_t* ptab = a.pages.table + static_cast<int64_t>(b) * a.pages.per_seq;
+      int* ids = reinterpret_cast<int*>(smem + C::kOffIds);
+      if (n_ch > 0) {
+        const int n_ids = min((k1 - k0 + bx - 1) / bx, C::kMaxIds);
+        for (int i = lane; i < n_ids; i += 32) ids[i] = __ldg(ptab + ((k0 + i * bx) >> shift));
+      }
+      __syncwarp();
+      if (lane == 0) {
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+        auto load_chunk = [&](uint8_t* dst, const CUtensorMap* tm, uint64_t* bar, int c) {
+          const int t0 = k0 + c * kChunk;
+          const int nbox = min(nb, (k1 - t0 + bx - 1) / bx);
+          mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nbox * bx) * C::kRowBytes * C::kPanels);
+          for (int j = 0; j < nbox; ++j) {
+            const int i = c * nb + j;
+            const int pg = i < C::kMaxIds ? ids[i] : __ldg(ptab + ((k0 + i * bx) >> shift));
+            const bool ok_pg = pg >= 0 && pg < a.pages.n_pages;
+            if (!ok_pg) raise_dev_err(a.dev_err, CCGQA_DEVERR_INDEX);
+            const int row = (t0 + j * bx) & ((1 << shift) - 1);
+#pragma unroll
+            for (int p = 0; p < C::kPanels; ++p)
+              tma_load_3d(dst + p * C::kPanelBytes + j * bx * C::kRowBytes, tm, bar,
+                          p * C::kPanelCols, row, ok_pg ? pg * a.Hkv + g : pool_z);
+          }
+        };
+        int ck = 0, cv = 0;
+        long long t_last = clock64();
+        while (ck < n_ch || cv < n_ch) {
+          bool progress = false;
+          if (ck < n_ch && mbar_test(&k_empty[ck % C::kStages], ((ck / C::kStages) & 1) ^ 1)) {
+            const int st = ck % C::kStages;
+            load_chunk(smem + C::kOffK + st * C::kTileBytes, &tmK, &k_full[st], ck);
+            ++ck;
+            progress = true;
+          }
+          if (cv < n_ch && mbar_test(&v_empty[cv % C::kStages], ((cv / C::kStages) & 1) ^ 1)) {
+            const int st = cv % C::kStages;
+            load_chunk(smem + C::kOffV + st * C::kTileBytes, &tmV, &v_full[st], cv);
+            ++cv;
+            progress = true;
+          }
+          if (progress) {
+            t_last = clock64();
+          } else if (*abort_v || clock64() - t_last > kWaitLimitCycles) {
+            if (!*abort_v) {
+              *abort_v = 1;
+              raise_dev_err(a.dev_err, CCGQA_DEVERR_TIMEOUT);
+            }
+            break;
+          }
         }
       }
     }
@@ -575,10 +645,16 @@ cudaError_t launch_tc(const DecodeArgs<bf16>& a, cudaStream_t stream) {
   using C = DCfg<D>;
   const CUtensorMapSwizzle swz = (D == 32) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   CUtensorMap tmK, tmV;
-  const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(a.cap),
-                            static_cast<uint64_t>(a.B) * a.Hkv};
-  const uint64_t st[2] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(a.cap) * D * 2};
-  const uint32_t box[3] = {static_cast<uint32_t>(C::kPanelCols), kChunk, 1};
+  // contiguous: [B Hkv][cap][d]; paged: [n_pages Hkv][page][d] with boxes of
+  // min(page, 128) rows
+  const bool paged = a.pages.table != nullptr;
+  const uint64_t rows = paged ? (uint64_t{1} << a.pages.shift) : static_cast<uint64_t>(a.cap);
+  const uint64_t planes = paged ? static_cast<uint64_t>(a.pages.n_pages) * a.Hkv
+                                : static_cast<uint64_t>(a.B) * a.Hkv;
+  const uint32_t box_rows = paged ? static_cast<uint32_t>(rows < kChunk ? rows : kChunk) : kChunk;
+  const uint64_t dims[3] = {static_cast<uint64_t>(D), rows, planes};
+  const uint64_t st[2] = {static_cast<uint64_t>(D) * 2, rows * D * 2};
+  const uint32_t box[3] = {static_cast<uint32_t>(C::kPanelCols), box_rows, 1};
   if (!encode_tensor_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.cache_k, dims, st, box, swz) ||
       !encode_tensor_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.cache_v, dims, st, box, swz))
     return cudaErrorInvalidValue;

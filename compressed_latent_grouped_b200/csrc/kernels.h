@@ -86,10 +86,37 @@ template <typename T>
 cudaError_t launch_attn_prefill_simt(const AttnArgs& a, cudaStream_t stream);
 
 // ----------------------------------------------------------------- cache + decode
+// Where token t of (sequence b, kv head g) sits in the cache's k / v buffers.
+// Contiguous (table == null): [B, Hkv, cap, d].  Paged: a pool [n_pages, Hkv,
+// 2^shift, d] and a block table [B, per_seq] naming the page of every
+// 2^shift consecutive tokens of a sequence.
+struct PageMap {
+  const int32_t* table;
+  int per_seq;           // table entries per sequence (cap >> shift)
+  int shift;             // log2(page size)
+  int n_pages;
+};
+// Row (in units of d elements) of token t of (b, g), or -1 when the page id the
+// table gives is outside the pool.
+__device__ __forceinline__ int64_t kv_row(const PageMap& pm, int b, int g, int Hkv, int64_t cap,
+                                          int64_t t) {
+  if (pm.table == nullptr) return (static_cast<int64_t>(b) * Hkv + g) * cap + t;
+  const int pg = __ldg(pm.table + static_cast<int64_t>(b) * pm.per_seq + (t >> pm.shift));
+  if (pg < 0 || pg >= pm.n_pages) return -1;
+  return ((static_cast<int64_t>(pg) * Hkv + g) << pm.shift) + (t & ((int64_t{1} << pm.shift) - 1));
+}
+
+// Append n_new rows per sequence at len[b] (then len[b] += n_new): k_new, v_new
+// [B, n_new, Hkv, d].
 template <typename T>
-cudaError_t launch_kv_append(T* cache_k, T* cache_v, int32_t* len, const T* k_new,
-                             const T* v_new, int B, int Hkv, int d, int64_t cap, int n_new,
-                             int32_t* dev_err, cudaStream_t stream);
+cudaError_t launch_kv_append(T* cache_k, T* cache_v, const PageMap& pm, int32_t* len,
+                             const T* k_new, const T* v_new, int B, int Hkv, int d, int64_t cap,
+                             int n_new, int32_t* dev_err, cudaStream_t stream);
+// Copy rows [0, S) of k_src, v_src [B, Hkv, S, d] into a paged cache (len untouched).
+template <typename T>
+cudaError_t launch_kv_scatter(T* cache_k, T* cache_v, const PageMap& pm, const T* k_src,
+                              const T* v_src, int B, int Hkv, int d, int64_t cap, int S,
+                              int32_t* dev_err, cudaStream_t stream);
 
 template <typename T>
 struct DecodeArgs {
@@ -101,8 +128,9 @@ struct DecodeArgs {
   double rope_log2_base;
   uint64_t rope_frac[64];  // theta_i / (2 pi) in 0.64 fixed point, i < d/2 (see PreAttnArgs)
   const T *wq_seq, *wq_chan, *wk_seq, *wk_chan;
-  T* cache_k;            // [B, Hkv, cap, d]
+  T* cache_k;            // [B, Hkv, cap, d], or a page pool (see PageMap)
   T* cache_v;
+  PageMap pages;
   int32_t* len;
   int64_t cap;
   T* hist_q;             // [B, K-1, Hq d]

@@ -43,22 +43,36 @@ class DeviceLayer:
         self._dec_ws = None
 
     # -------------------------------------------------------------- buffers
-    def alloc_cache(self, batch: int | None = None, cap: int | None = None):
+    def alloc_cache(self, batch: int | None = None, cap: int | None = None,
+                    block_table: torch.Tensor | None = None, page_size: int = 0,
+                    n_pages: int = 0):
+        """Contiguous cache [batch, Hkv, cap, d], or with ``block_table``
+        ([batch, cap / page_size] int32) a pool of ``n_pages`` pages
+        [n_pages, Hkv, page_size, d]."""
         w = self.w
         batch = self.batch if batch is None else batch
         cap = self.cap if cap is None else cap
         dt = w.torch_dtype
         km1 = max(w.conv_width - 1, 0)
+        if block_table is not None:
+            assert block_table.shape == (batch, cap // page_size) and cap % page_size == 0
+            kv_shape = (n_pages, w.Hkv, page_size, w.d)
+        else:
+            kv_shape = (batch, w.Hkv, cap, w.d)
         t = dict(
-            k=torch.zeros(batch, w.Hkv, cap, w.d, dtype=dt, device=self.device),
-            v=torch.zeros(batch, w.Hkv, cap, w.d, dtype=dt, device=self.device),
+            k=torch.zeros(kv_shape, dtype=dt, device=self.device),
+            v=torch.zeros(kv_shape, dtype=dt, device=self.device),
             len=torch.zeros(batch, dtype=torch.int32, device=self.device),
             hist_q=torch.zeros(batch, max(km1, 1), w.Hq * w.d, dtype=dt, device=self.device),
             hist_k=torch.zeros(batch, max(km1, 1), w.Hkv * w.d, dtype=dt, device=self.device),
             v_prev=torch.zeros(batch, w.Hkv * w.d, dtype=dt, device=self.device),
         )
+        if block_table is not None:
+            t["block_table"] = block_table.to(self.device, torch.int32).contiguous()
         self.cache_tensors = t
-        self.cache = B.make_kvcache(t["k"], t["v"], t["len"], t["hist_q"], t["hist_k"], t["v_prev"])
+        self.cache = B.make_kvcache(t["k"], t["v"], t["len"], t["hist_q"], t["hist_k"], t["v_prev"],
+                                    t.get("block_table"))
+        self.cache_batch, self.cache_cap = batch, cap
         return t
 
     def prefill_workspace(self, batch: int, seq_len: int):
@@ -70,9 +84,7 @@ class DeviceLayer:
         return self._pf_ws
 
     def decode_workspace(self):
-        t = self.cache_tensors
-        batch, cap = t["k"].shape[0], t["k"].shape[2]
-        n = B.ccgqa_decode_workspace_size(self.cfg, batch, cap)
+        n = B.ccgqa_decode_workspace_size(self.cfg, self.cache_batch, self.cache_cap)
         if self._dec_ws is None or self._dec_ws.numel() < n:
             self._dec_ws = torch.zeros(n, dtype=torch.uint8, device=self.device)
         return self._dec_ws

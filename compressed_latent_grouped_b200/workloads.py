@@ -144,6 +144,17 @@ def make_output_weights(w: Workload, seed: int = 0) -> torch.Tensor:
     return _normal(rng, (w.E, w.Hq * w.d), (1.0 / (w.Hq * w.d)) ** 0.5, w.dtype)
 
 
+def make_block_table(batch: int, pages_per_seq: int, n_pages: int, seed: int = 0) -> torch.Tensor:
+    """Block table of a paged cache: [batch, pages_per_seq] int32 page ids,
+    all distinct, drawn as the first batch * pages_per_seq entries of a seeded
+    permutation of the pool's n_pages pages (so a sequence's pages are
+    scattered over the pool in no order)."""
+    assert n_pages >= batch * pages_per_seq
+    rng = np.random.default_rng(seed + 104729)
+    ids = rng.permutation(n_pages)[: batch * pages_per_seq].astype(np.int32)
+    return torch.from_numpy(ids.reshape(batch, pages_per_seq))
+
+
 def sample_rows(S: int, n: int = 1024, tile: int = 128, seed: int = 1) -> np.ndarray:
     """Query positions checked one by one on full-size workloads: the first and
     last ``tile`` positions, positions on both sides of every ``tile`` boundary

@@ -112,10 +112,26 @@ typedef struct {
 
 /* Latent KV cache plus the decode state (device buffers, caller-owned).
    [Probleemstelling 2: the cache grows with the sequence; Resultaten 3: it
-   shrinks with C.] */
+   shrinks with C.]
+   Two layouts of k / v:
+    - contiguous (block_table == NULL): k, v are [batch, Hkv, cap, d];
+    - paged (block_table != NULL), after "Grouped Query Attention (GQA)",
+      section "GQA y tecnicas relacionadas" (PagedAttention: the cache is
+      allocated in fixed-size blocks, whatever number of heads fills them):
+      k, v are a pool of n_pages pages [n_pages, Hkv, page_size, d], each page
+      holding page_size consecutive tokens of one sequence for all Hkv heads.
+      Token t of sequence b lives in page block_table[b * (cap / page_size) +
+      t / page_size], row t % page_size.  page_size is a power of two from 16
+      to 4096 that divides cap; the table has cap / page_size int32 entries per
+      sequence, and only the entries of tokens a call reads or writes are
+      looked at (the rest may hold anything, e.g. -1 for pages not yet given).
+      Pages may be shared between sequences only if no call writes them.  An
+      entry outside [0, n_pages) that a kernel needs sets CCGQA_DEVERR_INDEX;
+      that access is skipped (writes) or reads zeros (reads), and the
+      sequence's output row is then undefined. */
 typedef struct {
-  void* k;            /* [batch, Hkv, cap, d]  post-RoPE keys */
-  void* v;            /* [batch, Hkv, cap, d]  value-shifted values */
+  void* k;            /* [batch, Hkv, cap, d]  post-RoPE keys (paged: [n_pages, Hkv, page_size, d]) */
+  void* v;            /* [batch, Hkv, cap, d]  value-shifted values (paged: as k) */
   int32_t* len;       /* [batch] tokens held (device int32) */
   void* conv_hist_q;  /* [batch, K-1, Hq d]  last K-1 pre-conv q~ rows, oldest first
                          (NULL allowed when K <= 1) */
@@ -124,6 +140,9 @@ typedef struct {
                          when value_shift == 0) */
   int32_t batch;
   int32_t cap;        /* token capacity per sequence */
+  const int32_t* block_table;  /* NULL = contiguous; else [batch, cap / page_size] page ids (device) */
+  int32_t page_size;  /* tokens per page (paged only) */
+  int32_t n_pages;    /* pages in the pool k / v (paged only; n_pages * Hkv < 2^31) */
 } ccgqa_kvcache;
 
 /* Bytes of workspace ccgqa_prefill needs for (batch, seq_len). */
@@ -144,7 +163,8 @@ CCGQA_API size_t ccgqa_decode_workspace_size(const ccgqa_config* cfg, int32_t ba
  *      overwritten, len[b] = seq_len, and the conv histories and v_prev are set
  *      so that ccgqa_decode_step continues the sequences.  Needs
  *      seq_len <= cache->cap and cache->batch == batch (else CCGQA_ERR_CAPACITY
- *      / CCGQA_ERR_INVALID_ARG).
+ *      / CCGQA_ERR_INVALID_ARG).  A paged cache is filled after the attention
+ *      (which reads k / v from the workspace) by one page-scatter kernel.
  * workspace: >= ccgqa_prefill_workspace_size bytes, 256-byte aligned.
  * Steps: projection (tcgen05 GEMM for bf16), fused conv + channel mix +
  * QK-mean + RoPE + value-shift, flash attention (tcgen05/TMEM/TMA for bf16). */
@@ -204,7 +224,8 @@ CCGQA_API ccgqa_status ccgqa_decode_step_noalloc(const ccgqa_config* cfg, const 
 CCGQA_API size_t ccgqa_decode_noalloc_max_bytes(void);
 
 /* Append n_new rows per sequence: cache->k[b, g, len[b] + i, :] = k_new[b, i, g, :]
- * (same for v), then len[b] += n_new.  Bit-exact copy.
+ * (same for v; in a paged cache, token len[b] + i of sequence b at its page
+ * and row), then len[b] += n_new.  Bit-exact copy.
  * k_new, v_new: [batch, n_new, Hkv, d].  n_new > cap returns CCGQA_ERR_CAPACITY
  * on the host; a sequence whose len[b] + n_new > cap is skipped on the device
  * and sets CCGQA_DEVERR_CAPACITY.  Conv histories and v_prev are not touched. */

@@ -39,6 +39,8 @@ int main(void) {
   printf("%zu %zu %zu %zu %zu\n", sizeof(ccgqa_config), offsetof(ccgqa_config, rope_base),
          offsetof(ccgqa_config, dtype), sizeof(ccgqa_weights), sizeof(ccgqa_kvcache));
   printf("%zu %zu\n", offsetof(ccgqa_kvcache, batch), offsetof(ccgqa_kvcache, cap));
+  printf("%zu %zu %zu\n", offsetof(ccgqa_kvcache, block_table), offsetof(ccgqa_kvcache, page_size),
+         offsetof(ccgqa_kvcache, n_pages));
   return 0;
 }
 """
@@ -56,6 +58,9 @@ int main(void) {
     assert vals[4] == ctypes.sizeof(B.ccgqa_kvcache)
     assert vals[5] == B.ccgqa_kvcache.batch.offset
     assert vals[6] == B.ccgqa_kvcache.cap.offset
+    assert vals[7] == B.ccgqa_kvcache.block_table.offset
+    assert vals[8] == B.ccgqa_kvcache.page_size.offset
+    assert vals[9] == B.ccgqa_kvcache.n_pages.offset
 
 
 def test_status_strings(lib):
@@ -172,6 +177,36 @@ def test_capacity_checked_on_host(lib):
                            ctypes.c_void_p(8192), ctypes.byref(cache), ctypes.c_void_p(1 << 20),
                            1 << 30, None, None)
     assert st == 1   # cache batch mismatch
+
+
+@pytest.mark.parametrize("page_size,cap,n_pages,table,why", [
+    (8, 64, 16, 1 << 16, "page below 16 tokens"),
+    (48, 96, 16, 1 << 16, "page size not a power of two"),
+    (8192, 8192, 16, 1 << 16, "page above 4096 tokens"),
+    (32, 80, 16, 1 << 16, "page size does not divide cap"),
+    (32, 64, 0, 1 << 16, "empty pool"),
+    (32, 64, 1 << 30, 1 << 16, "n_pages * Hkv past int32"),
+    (32, 64, 16, (1 << 16) + 2, "misaligned block table"),
+])
+def test_paged_cache_checked_on_host(lib, page_size, cap, n_pages, table, why):
+    """A paged cache's geometry is validated before any launch (append and
+    prefill both return CCGQA_ERR_INVALID_ARG)."""
+    cfg = _cfg(conv_width=0, qk_mean=0, value_shift=0)
+    cache = B.ccgqa_kvcache(4096, 8192, 12288, None, None, None, 1, cap, table, page_size,
+                            n_pages)
+    st = lib.ccgqa_kvcache_append(ctypes.byref(cfg), ctypes.byref(cache), ctypes.c_void_p(4096),
+                                  ctypes.c_void_p(8192), 1, None, None)
+    assert st == 1, why
+    w = B.make_weights()
+    st = lib.ccgqa_prefill(ctypes.byref(cfg), ctypes.byref(w), ctypes.c_void_p(4096), 1, 4,
+                           ctypes.c_void_p(8192), ctypes.byref(cache), ctypes.c_void_p(1 << 20),
+                           1 << 30, None, None)
+    assert st == 1, why
+    # the same cache with a valid geometry passes validation as far as capacity
+    good = B.ccgqa_kvcache(4096, 8192, 12288, None, None, None, 1, 64, 1 << 16, 32, 16)
+    st = lib.ccgqa_kvcache_append(ctypes.byref(cfg), ctypes.byref(good), ctypes.c_void_p(4096),
+                                  ctypes.c_void_p(8192), 65, None, None)
+    assert st == 3   # 65 tokens > cap 64: capacity, not geometry
 
 
 def test_launch_count_starts_at_zero(lib):
