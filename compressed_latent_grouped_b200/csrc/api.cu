@@ -1,6 +1,7 @@
 // C ABI of the CCGQA hot path: host-side validation, workspace layout and
 // kernel dispatch.  Every entry point validates all arguments before the first
 // launch and returns a status; the kernels themselves never trap.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdio>
@@ -309,7 +310,8 @@ ccgqa_status run_prefill(const Geo& g, const ccgqa_weights* w, const void* x, in
 }
 
 struct BwdWs {
-  size_t z, q, k, v, dq, dk, dv, lse, dsum, dy, dzm, du, u, dz, total;
+  size_t z, q, k, v, o, dq, dk, dv, lse, dsum, dy, dzm, du, u, dz, total;
+  int64_t lse_ld;   // packed log-sum-exp rows per (sequence, kv group), tensor-core path
 };
 BwdWs backward_ws(const Geo& g, int64_t B, int64_t S, bool has_proj) {
   BwdWs w;
@@ -326,11 +328,17 @@ BwdWs backward_ws(const Geo& g, int64_t B, int64_t S, bool has_proj) {
   w.q = take(qn * g.es);
   w.k = take(kvn * g.es);
   w.v = take(kvn * g.es);
+  w.o = take(g.dtype == CCGQA_BF16 ? qn * g.es : 0);
   w.dq = take(qn * 4);
   w.dk = take(kvn * 4);
   w.dv = take(kvn * 4);
-  w.lse = take(static_cast<size_t>(B) * g.Hq * S * 4);
-  w.dsum = take(static_cast<size_t>(B) * g.Hq * S * 4);
+  // [B, Hq, S] for the CUDA-core kernels; [B Hkv, lse_ld] packed rows (S G
+  // rounded up to 64) for the tensor-core ones
+  w.lse_ld = (S * g.G + 63) / 64 * 64;
+  const size_t n_lse = std::max(static_cast<size_t>(B) * g.Hq * S,
+                                static_cast<size_t>(B) * g.Hkv * static_cast<size_t>(w.lse_ld));
+  w.lse = take(n_lse * 4);
+  w.dsum = take(n_lse * 4);
   w.dy = take(cqk * 4);
   w.dzm = take(cqk * 4);
   w.du = take(cqk * 4);
@@ -430,6 +438,9 @@ ccgqa_status run_backward(const Geo& g, const ccgqa_weights* w, const void* x, i
   a.dv = reinterpret_cast<float*>(ws + L.dv);
   a.lse = reinterpret_cast<float*>(ws + L.lse);
   a.dsum = reinterpret_cast<float*>(ws + L.dsum);
+  a.lse_ld = L.lse_ld;
+  a.o = g.dtype == CCGQA_BF16 ? reinterpret_cast<T*>(ws + L.o) : nullptr;
+  a.dev_err = dev_err;
   a.dy = reinterpret_cast<float*>(ws + L.dy);
   a.dzm = reinterpret_cast<float*>(ws + L.dzm);
   a.du = reinterpret_cast<float*>(ws + L.du);

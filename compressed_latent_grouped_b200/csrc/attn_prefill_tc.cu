@@ -150,7 +150,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
                            const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, bf16* __restrict__ out,
                            int B, int S, int Hq, int Hkv, int G, int G_log2, int n_groups,
-                           int causal, int32_t* dev_err) {
+                           int causal, int32_t* dev_err, float* __restrict__ lse,
+                           int64_t lse_ld) {
   pdl_enter();
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -446,6 +447,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool store = row_ok && t < S;
+      if (lse != nullptr && store)
+        lse[static_cast<int64_t>(bg) * lse_ld + static_cast<int64_t>(t) * G + hl] = m_used + log2f(l);
       bf16* dst = out + ((static_cast<int64_t>(b) * S + t) * Hq + g * G + hl) * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
@@ -525,7 +528,8 @@ cudaError_t launch_d(const AttnArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const cudaError_t el = launch_pdl(kernel, dim3(grid), dim3(C::kThreads), C::kSmem, stream, tmQ,
                                     tmK, tmV, static_cast<bf16*>(a.out), a.B, a.S, a.Hq, a.Hkv,
-                                    a.G, G_log2, n_groups, a.causal, a.dev_err);
+                                    a.G, G_log2, n_groups, a.causal, a.dev_err, a.lse,
+                                    a.lse_ld);
   count_launches(1);
   return el != cudaSuccess ? el : cudaGetLastError();
 }

@@ -501,6 +501,51 @@ int blocks_for(int64_t n, int per) { return static_cast<int>((n + per - 1) / per
 
 template <typename T, int D>
 cudaError_t launch_attn_bwd_d(const BwdArgs<T>& a, cudaStream_t st) {
+  if constexpr (sizeof(T) == 2 && D >= 32) {
+    if (a.o != nullptr && a.lse_ld > 0 && attn_bwd_tc_supported(D, a.G)) {
+      // tensor core: the forward kernel recomputes o and the log-sum-exp, then
+      // the dq pass and the dk / dv pass
+      AttnArgs f{};
+      f.q = a.q;
+      f.k = a.k;
+      f.v = a.v;
+      f.out = a.o;
+      f.B = a.B;
+      f.S = a.S;
+      f.Hq = a.Hq;
+      f.Hkv = a.Hkv;
+      f.d = D;
+      f.G = a.G;
+      f.kv_cap = a.S;
+      f.causal = a.causal;
+      f.dev_err = a.dev_err;
+      f.lse = a.lse;
+      f.lse_ld = a.lse_ld;
+      cudaError_t e = launch_attn_prefill_tc(f, st);
+      if (e != cudaSuccess) return e;
+      AttnBwdTcArgs t{};
+      t.q = a.q;
+      t.k = a.k;
+      t.v = a.v;
+      t.o = a.o;
+      t.dout = a.dout;
+      t.lse = a.lse;
+      t.dsum = a.dsum;
+      t.ld = a.lse_ld;
+      t.dq = a.dq;
+      t.dk = a.dk;
+      t.dv = a.dv;
+      t.B = a.B;
+      t.S = a.S;
+      t.Hq = a.Hq;
+      t.Hkv = a.Hkv;
+      t.d = D;
+      t.G = a.G;
+      t.causal = a.causal;
+      t.dev_err = a.dev_err;
+      return launch_attn_bwd_tc(t, st);
+    }
+  }
   dim3 g1((a.S + kRows - 1) / kRows, a.Hq, a.B);
   attn_bwd_dq_kernel<T, D><<<g1, kRows * kSub, 0, st>>>(a.q, a.k, a.v, a.dout, a.dq, a.lse,
                                                          a.dsum, a.S, a.Hq, a.Hkv, a.G, a.causal);

@@ -76,10 +76,31 @@ struct AttnArgs {
   int64_t kv_cap;
   int causal;
   int32_t* dev_err;
+  // optional (tensor-core kernel only): each stored row's log-sum-exp in base
+  // 2 of the scaled scores, log2(sum_s 2^(log2(e) q.k_s / sqrt(d))), at
+  // lse[(b Hkv + g) lse_ld + t G + head in group]
+  float* lse = nullptr;
+  int64_t lse_ld = 0;
 };
 // bf16, d in {32, 64, 128}, any G <= 128 (a tile holds floor(128 / G)
 // positions of the group's G heads): tcgen05/TMEM/TMA flash attention.
 cudaError_t launch_attn_prefill_tc(const AttnArgs& a, cudaStream_t stream);
+
+// Attention backward on the tensor core (bf16, d in {32, 64, 128}, G a power
+// of two up to 64).  lse / dsum: [B Hkv, ld] packed per (sequence, kv group),
+// row t G + head in group, ld a multiple of 64 of at least S G; lse from the
+// forward kernel, dsum written here (D = rowsum(dO o)).
+struct AttnBwdTcArgs {
+  const void *q, *k, *v, *o, *dout;   // q, o, dout [B, S, Hq, d]; k, v [B, Hkv, S, d]
+  const float* lse;
+  float* dsum;
+  int64_t ld;
+  float *dq, *dk, *dv;                // fp32, like q, k, v
+  int B, S, Hq, Hkv, d, G, causal;
+  int32_t* dev_err;
+};
+bool attn_bwd_tc_supported(int d, int G);
+cudaError_t launch_attn_bwd_tc(const AttnBwdTcArgs& a, cudaStream_t stream);
 // CUDA-core flash attention (the fp32 path; bf16 where the tensor-core kernel
 // does not apply: d = 16 or G > 128).
 template <typename T>
@@ -174,6 +195,10 @@ struct BwdArgs {
   const T* dout;               // [B, S, Hq, d]
   float *dq, *dk, *dv;         // like q, k, v
   float *lse, *dsum;           // [B, Hq, S]: log-sum-exp and rowsum(dO * O)
+                               // (tensor-core path: [B Hkv, lse_ld] packed rows)
+  int64_t lse_ld;
+  T* o;                        // [B, S, Hq, d] forward output (tensor-core path)
+  int32_t* dev_err;
   float *dy, *dzm, *du, *u;    // [B S, (Hq + Hkv) d]
   float* dz;                   // [B S, N]
   T* dx;                       // [B S, E] (or [B S, N] for packed input)

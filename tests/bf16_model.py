@@ -195,11 +195,48 @@ def check_within_one_ulp(gpu, model, what=""):
     assert worst <= 0.0, f"{what}: a stored value is {worst:.3e} beyond one ulp (+ one ulp of RMS)"
 
 
+def _attention_backward_bf16_tc(q, k, v, G, causal, dout):
+    """The oracle's attention backward with the roundings of the tensor-core
+    backward kernels: D = rowsum(dout o) from the forward output o rounded to
+    bf16 (as the forward kernel stores it), and P and dS rounded to bf16
+    before the products that form dv, dk and dq (the MMA operands); the rest
+    in float64 (the kernels accumulate in fp32)."""
+    S, Hq, d = q.shape
+    scale = 1.0 / np.sqrt(d)
+    keys = np.arange(k.shape[0])
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for h in range(Hq):
+        g = h // G
+        sc = (q[:, h, :] @ k[:, g, :].T) * scale
+        if causal:
+            sc = np.where(keys[None, :] <= np.arange(S)[:, None], sc, -np.inf)
+        p = np.exp(sc - sc.max(axis=1, keepdims=True))
+        p = p / p.sum(axis=1, keepdims=True)
+        do = dout[:, h, :]
+        o = bf(p @ v[:, g, :])
+        dp = do @ v[:, g, :].T
+        ds = p * (dp - (do * o).sum(axis=1, keepdims=True))
+        pb, dsb = bf(p), bf(ds)
+        dv[:, g, :] += pb.T @ do
+        dq[:, h, :] = (dsb @ k[:, g, :]) * scale
+        dk[:, g, :] += (dsb.T @ q[:, h, :]) * scale
+    return dq, dk, dv
+
+
+def backward_takes_tensor_core(layer: O.Layer) -> bool:
+    """Whether the bf16 backward runs its attention on the tensor-core kernels
+    (d of 32, 64 or 128 and a power-of-two group of at most 64 heads)."""
+    d, G = layer.sh.d, layer.sh.G
+    return d in (32, 64, 128) and 1 <= G <= 64 and (G & (G - 1)) == 0
+
+
 def model_prefill_backward(layer: O.Layer, x: np.ndarray, dout: np.ndarray):
     """The oracle's backward with the forward values it uses rounded to bf16
     where the bf16 path rounds them (q~, k~, v~ and q, k, v), and dx rounded
     to bf16 as the bf16 path stores it; the gradients themselves in float64
     (the weight gradients stay unrounded: the kernel writes them in fp32).
+    Where the attention backward runs on the tensor core, its P, dS and the
+    forward output are rounded as those kernels round them.
     Returns the same dict as O.prefill_backward."""
     sh = layer.sh
     S = x.shape[0]
@@ -229,7 +266,10 @@ def model_prefill_backward(layer: O.Layer, x: np.ndarray, dout: np.ndarray):
     q = bf(O.rope(qm, pos, layer.rope_base))
     k = bf(O.rope(km, pos, layer.rope_base))
     v = O._shift_values(layer, v_lat)
-    dq, dk, dv = O.attention_backward(q, k, v, G, layer.causal, dout.reshape(S, Hq, d))
+    if backward_takes_tensor_core(layer):
+        dq, dk, dv = _attention_backward_bf16_tc(q, k, v, G, layer.causal, dout.reshape(S, Hq, d))
+    else:
+        dq, dk, dv = O.attention_backward(q, k, v, G, layer.causal, dout.reshape(S, Hq, d))
     dv_lat = O._value_shift_backward(layer, dv)
     dqm = O._rope_backward(dq, pos, layer.rope_base)
     dkm = O._rope_backward(dk, pos, layer.rope_base)

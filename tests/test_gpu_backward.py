@@ -36,6 +36,15 @@ CASES = {
     "bf16_d64_variants": W3.with_(name="bwd_d64var", S=90, qk_mean=2, value_shift=2,
                                   channel_conv=True),
     "bf16_d32_conv2_nochan": W2.with_(name="bwd_k2", B=1, S=77, conv_width=2),
+    # CUDA-core attention backward in bf16: a group of 3 heads, and d = 16
+    "bf16_d32_g3_simt": W2.with_(name="bwd_g3", B=1, S=90, E=768, C=4, Hq=6, Hkv=2),
+    "bf16_d16_simt": W1.with_(name="bwd_d16", dtype="bf16", S=80),
+    # tensor-core attention backward over several tiles and a ragged tail:
+    # two CTAs of query tiles and of key tiles, non-causal, a group of 1 and 8
+    "bf16_d64_tiles": W3.with_(name="bwd_d64_tiles", S=700),
+    "bf16_d32_noncausal": W2.with_(name="bwd_d32_nc", B=1, S=300, causal=False),
+    "bf16_d64_g1": W3.with_(name="bwd_d64_g1", S=333, Hq=2, Hkv=2, E=1024),
+    "bf16_d128_g8": W5.with_(name="bwd_d128_g8", B=1, S=260, Hq=32, Hkv=4),
 }
 
 
