@@ -310,7 +310,8 @@ ccgqa_status run_prefill(const Geo& g, const ccgqa_weights* w, const void* x, in
 }
 
 struct BwdWs {
-  size_t z, q, k, v, o, dq, dk, dv, lse, dsum, dy, dzm, du, u, dz, total;
+  size_t z, q, k, v, o, dq, dk, dv, lse, dsum, dy, dzm, du, u, dz, dz_b, wt, dzt, xt, total;
+  int64_t ldr;      // rows of the transposed gradient-GEMM operands (B S rounded up to 8)
   int64_t lse_ld;   // packed log-sum-exp rows per (sequence, kv group), tensor-core path
 };
 BwdWs backward_ws(const Geo& g, int64_t B, int64_t S, bool has_proj) {
@@ -344,6 +345,13 @@ BwdWs backward_ws(const Geo& g, int64_t B, int64_t S, bool has_proj) {
   w.du = take(cqk * 4);
   w.u = take(cqk * 4);
   w.dz = take(rows * g.N * 4);
+  // bf16 with a projection: operands of the tensor-core gradient GEMMs
+  const bool tc_gemm = g.dtype == CCGQA_BF16 && has_proj;
+  w.ldr = (static_cast<int64_t>(rows) + 7) / 8 * 8;
+  w.dz_b = take(tc_gemm ? rows * g.N * 2 : 0);
+  w.wt = take(tc_gemm ? static_cast<size_t>(g.E) * g.N * 2 : 0);
+  w.dzt = take(tc_gemm ? static_cast<size_t>(g.N) * w.ldr * 2 : 0);
+  w.xt = take(tc_gemm ? static_cast<size_t>(g.E) * w.ldr * 2 : 0);
   w.total = off;
   return w;
 }
@@ -441,6 +449,13 @@ ccgqa_status run_backward(const Geo& g, const ccgqa_weights* w, const void* x, i
   a.lse_ld = L.lse_ld;
   a.o = g.dtype == CCGQA_BF16 ? reinterpret_cast<T*>(ws + L.o) : nullptr;
   a.dev_err = dev_err;
+  if (g.dtype == CCGQA_BF16 && w->W_qkv) {
+    a.dz_b = reinterpret_cast<T*>(ws + L.dz_b);
+    a.WT = reinterpret_cast<T*>(ws + L.wt);
+    a.dzT = reinterpret_cast<T*>(ws + L.dzt);
+    a.xT = reinterpret_cast<T*>(ws + L.xt);
+    a.ldr = L.ldr;
+  }
   a.dy = reinterpret_cast<float*>(ws + L.dy);
   a.dzm = reinterpret_cast<float*>(ws + L.dzm);
   a.du = reinterpret_cast<float*>(ws + L.du);

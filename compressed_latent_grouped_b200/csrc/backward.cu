@@ -413,6 +413,8 @@ struct GemmArgs {
   int64_t bza, bzb, bzc;   // batch offsets (elements)
   int seg, seg_stride, off_a, off_b;
   int accumulate;
+  int ksplit;              // -1: cut K into ranges whose partial sums are added atomically
+                           // into C (fp32 C, zeroed by the caller); else one range
 };
 constexpr int kGBM = 64, kGBN = 64, kGBK = 16;
 
@@ -420,18 +422,25 @@ template <typename TA, typename TB, typename TC>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(const GemmArgs g) {
   __shared__ float As[kGBK][kGBM + 1];
   __shared__ float Bs[kGBK][kGBN + 1];
-  const TA* A = static_cast<const TA*>(g.A) + blockIdx.z * g.bza;
-  const TB* B = static_cast<const TB*>(g.B) + blockIdx.z * g.bzb;
-  TC* C = static_cast<TC*>(g.C) + blockIdx.z * g.bzc;
+  const int ks = g.ksplit > 1 ? g.ksplit : 1;
+  const int bz = blockIdx.z / ks, kpart = blockIdx.z % ks;
+  const TA* A = static_cast<const TA*>(g.A) + bz * g.bza;
+  const TB* B = static_cast<const TB*>(g.B) + bz * g.bzb;
+  TC* C = static_cast<TC*>(g.C) + bz * g.bzc;
   const int m0 = blockIdx.y * kGBM, n0 = blockIdx.x * kGBN;
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  // this CTA's K range: whole kGBK blocks, the last range takes the rest
+  const int kblocks = (g.K + kGBK - 1) / kGBK;
+  const int per = (kblocks + ks - 1) / ks;
+  const int k_begin = kpart * per * kGBK;
+  const int k_end = min(g.K, (kpart + 1) * per * kGBK);
   float acc[4][4] = {};
-  for (int k0 = 0; k0 < g.K; k0 += kGBK) {
+  for (int k0 = k_begin; k0 < k_end; k0 += kGBK) {
     for (int idx = threadIdx.x; idx < kGBK * kGBM; idx += 256) {
       const int kk = idx / kGBM, mm = idx % kGBM;
       const int k = k0 + kk, m = m0 + mm;
       float val = 0.f;
-      if (k < g.K && m < g.M) {
+      if (k < k_end && m < g.M) {
         const int64_t r = static_cast<int64_t>(k / g.seg) * g.seg_stride + g.off_a + k % g.seg;
         val = to_f32(A[m * g.sam + r * g.sak]);
       }
@@ -441,7 +450,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const GemmArgs g) {
       const int kk = idx / kGBN, nn = idx % kGBN;
       const int k = k0 + kk, n = n0 + nn;
       float val = 0.f;
-      if (k < g.K && n < g.N) {
+      if (k < k_end && n < g.N) {
         const int64_t r = static_cast<int64_t>(k / g.seg) * g.seg_stride + g.off_b + k % g.seg;
         val = to_f32(B[r * g.sbk + n * g.sbn]);
       }
@@ -472,6 +481,12 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const GemmArgs g) {
       if (n >= g.N) continue;
       TC* p = C + m * g.scm + n * g.scn;
       float val = acc[r][cc];
+      if constexpr (sizeof(TC) == 4) {
+        if (ks > 1) {
+          atomicAdd(reinterpret_cast<float*>(p), val);
+          continue;
+        }
+      }
       if (g.accumulate) val += to_f32(*p);
       *p = from_f32<TC>(val);
     }
@@ -485,7 +500,18 @@ cudaError_t gemm(GemmArgs g, int batch, cudaStream_t st) {
     g.seg_stride = 0;
   }
   if (g.M <= 0 || g.N <= 0 || batch <= 0) return cudaSuccess;
-  dim3 grid((g.N + kGBN - 1) / kGBN, (g.M + kGBM - 1) / kGBM, batch);
+  const int tiles = ((g.N + kGBN - 1) / kGBN) * ((g.M + kGBM - 1) / kGBM) * batch;
+  if (sizeof(TC) == 4 && !g.accumulate && g.ksplit == -1) {
+    // few output tiles over a long K (the weight gradients): split K so that
+    // about two waves of CTAs run, each range at least 32 K blocks long; the
+    // caller zeroed C, so the atomic sums start from zero
+    int ks = (2 * 148 + tiles - 1) / tiles;
+    const int max_ks = (g.K + 32 * kGBK - 1) / (32 * kGBK);
+    if (ks > max_ks) ks = max_ks;
+    g.ksplit = ks < 1 ? 1 : ks;
+  }
+  if (g.ksplit < 1) g.ksplit = 1;
+  dim3 grid((g.N + kGBN - 1) / kGBN, (g.M + kGBM - 1) / kGBM, batch * g.ksplit);
   gemm_simt_kernel<TA, TB, TC><<<grid, 256, 0, st>>>(g);
   count_launches(1);
   return cudaGetLastError();
@@ -498,6 +524,35 @@ __global__ void cast_kernel(const float* __restrict__ src, T* __restrict__ dst, 
 }
 
 int blocks_for(int64_t n, int per) { return static_cast<int>((n + per - 1) / per); }
+
+// out[c, r] = in[r, c] as bf16 for r < R, zero for R <= r < ldo (in: [R, C],
+// leading dimension C; out: [C, ldo]).  32 x 32 tiles through shared memory.
+template <typename TI>
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(const TI* __restrict__ in,
+                                                             bf16* __restrict__ out, int64_t R,
+                                                             int64_t C, int64_t ldo) {
+  __shared__ float tile[32][33];
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 32, c0 = static_cast<int64_t>(blockIdx.x) * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
+#pragma unroll
+  for (int i = 0; i < 32; i += 8) {
+    const int64_t r = r0 + ty + i, c = c0 + tx;
+    tile[ty + i][tx] = (r < R && c < C) ? to_f32(in[r * C + c]) : 0.f;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < 32; i += 8) {
+    const int64_t c = c0 + ty + i, r = r0 + tx;
+    if (c < C && r < ldo) out[c * ldo + r] = __float2bfloat16_rn(tile[tx][ty + i]);
+  }
+}
+
+template <typename TI>
+void transpose_bf16(const TI* in, bf16* out, int64_t R, int64_t C, int64_t ldo, cudaStream_t st) {
+  dim3 grid(static_cast<unsigned>((C + 31) / 32), static_cast<unsigned>((ldo + 31) / 32));
+  transpose_bf16_kernel<TI><<<grid, 256, 0, st>>>(in, out, R, C, ldo);
+  count_launches(1);
+}
 
 template <typename T, int D>
 cudaError_t launch_attn_bwd_d(const BwdArgs<T>& a, cudaStream_t st) {
@@ -588,7 +643,28 @@ cudaError_t launch_backward(const BwdArgs<T>& a, cudaStream_t st) {
   count_launches(1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // dx = dz W (or dz itself for packed input)
-  if (a.W) {
+  bool gw_done = false;
+  if constexpr (sizeof(T) == 2) {
+    if (a.W && a.dz_b && a.WT && a.dzT && a.xT) {
+      // tensor core: dx = bf16(dz) (W^T)^T, dW = bf16(dz)^T x as (dz^T)(x^T)^T
+      cast_kernel<T><<<blocks_for(rows * a.N, 256), 256, 0, st>>>(a.dz, a.dz_b, rows * a.N);
+      count_launches(1);
+      transpose_bf16<T>(a.W, a.WT, a.N, a.E, a.N, st);
+      if ((e = launch_proj_gemm_bf16(a.dz_b, a.WT, a.dx, static_cast<int>(rows), a.E, a.N,
+                                     a.dev_err, st)) != cudaSuccess)
+        return e;
+      if (a.g_W) {
+        transpose_bf16<float>(a.dz, a.dzT, rows, a.N, a.ldr, st);
+        transpose_bf16<T>(a.x, a.xT, rows, a.E, a.ldr, st);
+        if ((e = launch_gemm_bf16_f32out(a.dzT, a.xT, a.g_W, a.N, a.E, static_cast<int>(a.ldr),
+                                         a.dev_err, st)) != cudaSuccess)
+          return e;
+      }
+      gw_done = true;
+    }
+  }
+  if (gw_done) {
+  } else if (a.W) {
     GemmArgs g{};
     g.A = a.dz; g.B = a.W; g.C = a.dx;
     g.M = static_cast<int>(rows); g.N = a.E; g.K = a.N;
@@ -599,11 +675,12 @@ cudaError_t launch_backward(const BwdArgs<T>& a, cudaStream_t st) {
     count_launches(1);
   }
   // weight gradients (each optional; the buffers were zeroed by the caller)
-  if (a.g_W && a.W) {
+  if (a.g_W && a.W && !gw_done) {
     GemmArgs g{};
     g.A = a.dz; g.B = a.x; g.C = a.g_W;
     g.M = a.N; g.N = a.E; g.K = static_cast<int>(rows);
     g.sam = 1; g.sak = a.N; g.sbk = a.E; g.sbn = 1; g.scm = a.E; g.scn = 1;
+    g.ksplit = -1;
     if ((e = gemm<float, T, float>(g, 1, st)) != cudaSuccess) return e;
   }
   if (depthwise && a.g_q_seq && a.g_k_seq) {
@@ -624,6 +701,7 @@ cudaError_t launch_backward(const BwdArgs<T>& a, cudaStream_t st) {
       g.M = d; g.N = d; g.K = static_cast<int>(rows);
       g.sam = 1; g.sak = Cqk; g.sbk = Cqk; g.sbn = 1; g.scm = d; g.scn = 1;
       g.bza = d; g.bzb = d; g.bzc = static_cast<int64_t>(d) * d;
+      g.ksplit = -1;
       if ((e = gemm<float, float, float>(g, nh, st)) != cudaSuccess) return e;
     }
   }
@@ -639,6 +717,7 @@ cudaError_t launch_backward(const BwdArgs<T>& a, cudaStream_t st) {
         g.sam = 1; g.sak = Cqk; g.sbk = a.N; g.sbn = 1; g.scm = d; g.scn = 1;
         g.bza = d; g.bzb = d; g.bzc = static_cast<int64_t>(K) * d * d;
         g.seg = a.S - j; g.seg_stride = a.S; g.off_a = j; g.off_b = 0;
+        g.ksplit = -1;
         if ((e = gemm<float, T, float>(g, nh, st)) != cudaSuccess) return e;
       }
     }

@@ -25,6 +25,9 @@ bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank, co
 // returns cudaErrorInvalidValue).
 cudaError_t launch_proj_gemm_bf16(const bf16* A, const bf16* W, bf16* C, int M, int N, int K,
                                   int32_t* dev_err, cudaStream_t stream);
+// The same tensor-core GEMM with an fp32 output (N % 4 == 0).
+cudaError_t launch_gemm_bf16_f32out(const bf16* A, const bf16* W, float* C, int M, int N, int K,
+                                    int32_t* dev_err, cudaStream_t stream);
 // Same contraction in fp32 on the CUDA cores.
 cudaError_t launch_proj_gemm_f32(const float* A, const float* W, float* C, int M, int N, int K,
                                  cudaStream_t stream);
@@ -199,6 +202,11 @@ struct BwdArgs {
   int64_t lse_ld;
   T* o;                        // [B, S, Hq, d] forward output (tensor-core path)
   int32_t* dev_err;
+  // bf16 with a projection: the gradient GEMMs on the tensor core read
+  // dz_b = bf16(dz) [B S, N], W^T [E, N], and dz^T [N, ldr], x^T [E, ldr]
+  // (ldr = B S rounded up to a multiple of 8, zero past B S); null otherwise
+  T *dz_b, *WT, *dzT, *xT;
+  int64_t ldr;
   float *dy, *dzm, *du, *u;    // [B S, (Hq + Hkv) d]
   float* dz;                   // [B S, N]
   T* dx;                       // [B S, E] (or [B S, N] for packed input)

@@ -8,9 +8,10 @@
 //   shared-memory ring; warp 1 allocates 2 x 256 TMEM columns and one thread
 //   issues tcgen05.mma (M=128, N=256, K=16, fp32 accumulate) into them in turn;
 //   warps 2-5 read a finished accumulator back with tcgen05.ld, 32 x 32 at a
-//   time, into a 64B-swizzled bf16 staging buffer (two per warp, alternating)
-//   that a TMA tile store writes out as whole output rows (clipped at M and N),
-//   while the next tile accumulates into the other.
+//   time, into a swizzled staging buffer (two per warp, alternating; bf16, or
+//   fp32 for the weight gradients of the backward pass) that a TMA tile store
+//   writes out as whole output rows (clipped at M and N), while the next tile
+//   accumulates into the other.
 // fp32: a plain shared-memory tiled GEMM on the CUDA cores.
 #include "kernels.h"
 #include "sm100.cuh"
@@ -27,8 +28,13 @@ constexpr uint32_t kBTile = kBN * kBK * 2;      // 32 KB
 constexpr uint32_t kStageBytes = kATile + kBTile;
 constexpr uint32_t kOffBar = kStages * kStageBytes;          // barriers, TMEM slot (< 1 KB)
 constexpr uint32_t kOffOut = kOffBar + 1024;                  // output staging, 1024-aligned
-constexpr uint32_t kOutBuf = 32 * 32 * 2;                     // one 32 x 32 bf16 chunk
-constexpr size_t kGemmSmem = size_t(kOffOut) + 4 * 2 * kOutBuf + 1024;   // + alignment slack
+// one 32 x 32 output chunk: bf16 rows of 64 B (64B swizzle), fp32 rows of 128 B
+// (128B swizzle)
+template <typename TC>
+__host__ __device__ constexpr uint32_t out_buf() { return 32 * 32 * static_cast<uint32_t>(sizeof(TC)); }
+template <typename TC>
+constexpr size_t gemm_smem() { return size_t(kOffOut) + 4 * 2 * out_buf<TC>() + 1024; }  // + slack
+static_assert(gemm_smem<float>() <= 232448, "fp32 staging exceeds shared memory");
 
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int c0,
                                              int c1) {
@@ -53,6 +59,7 @@ __device__ __forceinline__ void bulk_wait_all() {
 // through L2).  The TMA ring and the k-block counter run on across tiles, and
 // the accumulator alternates between two 256-column TMEM buffers, so the
 // epilogue of one tile overlaps the main loop of the next.
+template <typename TC>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     proj_gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA,
                           const __grid_constant__ CUtensorMap tmB,
@@ -155,6 +162,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // Epilogue: warp w may only touch TMEM lanes [32 (w % 4), 32 (w % 4) + 32).
     const int q4 = warp & 3;
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    constexpr uint32_t kOutBuf = out_buf<TC>();
     uint8_t* stage = smem + kOffOut + (warp - 2) * 2 * kOutBuf;
     int i = 0, nst = 0;   // tiles read back, chunks stored by this warp
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
@@ -177,17 +185,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (lane == 0) bulk_wait_read_1();
           __syncwarp();
         }
+        if constexpr (sizeof(TC) == 4) {
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          uint4 pk;
-          uint32_t* pw = reinterpret_cast<uint32_t*>(&pk);
+          for (int v = 0; v < 8; ++v)
+            *reinterpret_cast<uint4*>(buf + swz_offset(lane, v * 16, 128)) =
+                make_uint4(r[v * 4], r[v * 4 + 1], r[v * 4 + 2], r[v * 4 + 3]);
+        } else {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[v * 8 + 2 * e]),
-                                                      __uint_as_float(r[v * 8 + 2 * e + 1]));
-            pw[e] = *reinterpret_cast<uint32_t*>(&h2);
+          for (int v = 0; v < 4; ++v) {
+            uint4 pk;
+            uint32_t* pw = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[v * 8 + 2 * e]),
+                                                        __uint_as_float(r[v * 8 + 2 * e + 1]));
+              pw[e] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+            *reinterpret_cast<uint4*>(buf + swz_offset(lane, v * 16, 64)) = pk;
           }
-          *reinterpret_cast<uint4*>(buf + swz_offset(lane, v * 16, 64)) = pk;
         }
         fence_proxy_async_smem();   // the TMA unit reads what the threads wrote
         __syncwarp();
@@ -267,37 +282,52 @@ __global__ void __launch_bounds__(256)
 
 }  // namespace
 
-cudaError_t launch_proj_gemm_bf16(const bf16* A, const bf16* W, bf16* C, int M, int N, int K,
-                                  int32_t* dev_err, cudaStream_t stream) {
+namespace {
+template <typename TC>
+cudaError_t launch_tc_gemm(const bf16* A, const bf16* W, TC* C, int M, int N, int K,
+                           int32_t* dev_err, cudaStream_t stream) {
+  constexpr bool f32 = sizeof(TC) == 4;
   CUtensorMap tmA, tmB, tmC;
   const uint64_t dA[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
   const uint64_t sA[1] = {static_cast<uint64_t>(K) * 2};
   const uint32_t bA[2] = {kBK, kBM};
   const uint64_t dB[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
   const uint32_t bB[2] = {kBK, kBN};
-  if (N % 8 != 0) return cudaErrorInvalidValue;   // 16-byte output row pitch for the TMA store
+  // 16-byte output row pitch for the TMA store
+  if (N % (f32 ? 4 : 8) != 0) return cudaErrorInvalidValue;
   const uint64_t dC[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(M)};
-  const uint64_t sC[1] = {static_cast<uint64_t>(N) * 2};
+  const uint64_t sC[1] = {static_cast<uint64_t>(N) * sizeof(TC)};
   const uint32_t bC[2] = {32, 32};
   if (!encode_tensor_map(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, dA, sA, bA,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tensor_map(&tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, dB, sA, bB,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tensor_map(&tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, dC, sC, bC,
-                         CU_TENSOR_MAP_SWIZZLE_64B))
+      !encode_tensor_map(&tmC, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                         2, C, dC, sC, bC, f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
-  cudaError_t e = allow_smem(reinterpret_cast<const void*>(proj_gemm_bf16_kernel),
-                             static_cast<int>(kGemmSmem));
+  cudaError_t e = allow_smem(reinterpret_cast<const void*>(proj_gemm_bf16_kernel<TC>),
+                             static_cast<int>(gemm_smem<TC>()));
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int tiles = ((N + kBN - 1) / kBN) * ((M + kBM - 1) / kBM);
   const int grid = tiles < sms ? tiles : sms;   // one persistent CTA per SM
-  const cudaError_t el = launch_pdl(proj_gemm_bf16_kernel, dim3(grid), dim3(kGemmThreads),
-                                    kGemmSmem, stream, tmA, tmB, tmC, M, N, K, dev_err);
+  const cudaError_t el = launch_pdl(proj_gemm_bf16_kernel<TC>, dim3(grid), dim3(kGemmThreads),
+                                    gemm_smem<TC>(), stream, tmA, tmB, tmC, M, N, K, dev_err);
   count_launches(1);
   return el != cudaSuccess ? el : cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_proj_gemm_bf16(const bf16* A, const bf16* W, bf16* C, int M, int N, int K,
+                                  int32_t* dev_err, cudaStream_t stream) {
+  return launch_tc_gemm<bf16>(A, W, C, M, N, K, dev_err, stream);
+}
+
+cudaError_t launch_gemm_bf16_f32out(const bf16* A, const bf16* W, float* C, int M, int N, int K,
+                                    int32_t* dev_err, cudaStream_t stream) {
+  return launch_tc_gemm<float>(A, W, C, M, N, K, dev_err, stream);
 }
 
 cudaError_t launch_proj_gemm_f32(const float* A, const float* W, float* C, int M, int N, int K,

@@ -236,7 +236,9 @@ def model_prefill_backward(layer: O.Layer, x: np.ndarray, dout: np.ndarray):
     to bf16 as the bf16 path stores it; the gradients themselves in float64
     (the weight gradients stay unrounded: the kernel writes them in fp32).
     Where the attention backward runs on the tensor core, its P, dS and the
-    forward output are rounded as those kernels round them.
+    forward output are rounded as those kernels round them; the projection's
+    gradients (dx and dW_qkv) take dz rounded to bf16, as the tensor-core GEMMs
+    that form them do.
     Returns the same dict as O.prefill_backward."""
     sh = layer.sh
     S = x.shape[0]
@@ -308,4 +310,6 @@ def model_prefill_backward(layer: O.Layer, x: np.ndarray, dout: np.ndarray):
     dzq = np.concatenate([dq_pre.reshape(S, -1), dk_pre.reshape(S, -1), dv_lat.reshape(S, -1)], axis=1)
     if layer.W_qkv is None:
         return {"dx": bf(dzq), "W_qkv": None, **grads}
-    return {"dx": bf(dzq @ layer.W_qkv), "W_qkv": dzq.T @ x, **grads}
+    # the projection's gradients run on the tensor core from dz rounded to bf16
+    dzb = bf(dzq)
+    return {"dx": bf(dzb @ layer.W_qkv), "W_qkv": dzb.T @ x, **grads}
