@@ -72,12 +72,14 @@ struct BwdTcCfg {
   static constexpr uint32_t kKOffBar = kKOffL + kKStages * 512;
   static constexpr size_t kKSmem = kKOffBar + 256 + 1024;
   // TMEM columns.  dq pass: S and dP (64 each) per tile, then dQ per tile.
-  // dkv pass: S^T and dP^T per tile, then dV | dK per tile.
+  // dkv pass: per tile two buffers of S^T | dP^T (32 + 32 columns), then
+  // dV | dK per tile.
   __device__ static constexpr uint32_t col_s(int x) { return x * 128; }
   __device__ static constexpr uint32_t col_dp(int x) { return x * 128 + 64; }
   __device__ static constexpr uint32_t col_dq(int x) { return kTiles * 128 + x * D; }
-  __device__ static constexpr uint32_t col_dv(int x) { return kTiles * 128 + x * 2 * D; }
-  __device__ static constexpr uint32_t col_dk(int x) { return kTiles * 128 + x * 2 * D + D; }
+  __device__ static constexpr uint32_t col_dkv_buf(int x, int b) { return x * 128 + b * 64; }
+  __device__ static constexpr uint32_t col_dkv_v(int x) { return kTiles * 128 + x * 2 * D; }
+  __device__ static constexpr uint32_t col_dkv_k(int x) { return kTiles * 128 + x * 2 * D + D; }
   static_assert(kTiles * 128 + kTiles * 2 * D <= 512, "TMEM columns");
   static_assert(kQSmem <= 227 * 1024 && kKSmem <= 227 * 1024, "shared memory");
 };
@@ -86,6 +88,16 @@ __device__ __forceinline__ float ex2f(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Four consecutive floats of shared memory, read where they are used (volatile:
+// not hoisted, so a row's 64 column constants never sit in registers at once).
+__device__ __forceinline__ float4 lds4(const float* p) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(smem_addr(p)));
+  return v;
 }
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
@@ -380,6 +392,10 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::kThreads, 1)
 }
 
 // ================================================================ dkv pass
+// Each 64-row query half is worked as two 32-row sub-halves, and each tile has
+// two TMEM buffers (S^T | dP^T, 32 columns each, P^T and dS^T written back as
+// bf16 over them), so the next sub-half's scores are computed into the other
+// buffer while the dV / dK MMAs of this one run.
 template <int D>
 __global__ void __launch_bounds__(BwdTcCfg<D>::kThreads, 1)
     attn_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQh,
@@ -399,11 +415,10 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::kThreads, 1)
   uint64_t* kv_full = bars;                       // K and V tiles
   uint64_t* h_full = kv_full + 1;                 // [kKStages] Q / dO halves, lse2 / D
   uint64_t* h_empty = h_full + C::kKStages;       // [kKStages], one commit per tile
-  uint64_t* s_full = h_empty + C::kKStages;       // [T]
-  uint64_t* dp_full = s_full + T;                 // [T]
-  uint64_t* ds_full = dp_full + T;                // [T], 128 arrivals
-  uint64_t* o_done = ds_full + T;                 // [T]
-  uint64_t* drain = o_done + T;
+  uint64_t* st_full = h_empty + C::kKStages;      // [T][2] S^T and dP^T of a buffer
+  uint64_t* ds_full = st_full + 2 * T;            // [T][2] 128 arrivals: P^T, dS^T written
+  uint64_t* o_done = ds_full + 2 * T;             // [T][2] dV / dK of a buffer complete
+  uint64_t* drain = o_done + 2 * T;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   __shared__ int abort_flag;
 
@@ -415,7 +430,8 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::kThreads, 1)
   const int k_start = kgrp * T * 128;
   const int64_t rows_all = static_cast<int64_t>(S) << G_log2;   // packed query rows of (b, g)
   const int u0 = causal ? static_cast<int>((static_cast<int64_t>(k_start) << G_log2) >> 6) : 0;
-  const int n_h = static_cast<int>((rows_all + 63) >> 6) - u0;
+  const int n_h = static_cast<int>((rows_all + 63) >> 6) - u0;  // 64-row halves
+  const int n_s = 2 * n_h;                                      // 32-row sub-halves
   const int pos_per_half = 64 >> G_log2;
 
   if (threadIdx.x == 0) {
@@ -424,11 +440,10 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::kThreads, 1)
       mbar_init(&h_full[s], 1);
       mbar_init(&h_empty[s], T);
     }
-    for (int x = 0; x < T; ++x) {
-      mbar_init(&s_full[x], 1);
-      mbar_init(&dp_full[x], 1);
-      mbar_init(&ds_full[x], 128);
-      mbar_init(&o_done[x], 1);
+    for (int i = 0; i < 2 * T; ++i) {
+      mbar_init(&st_full[i], 1);
+      mbar_init(&ds_full[i], 128);
+      mbar_init(&o_done[i], 1);
     }
     mbar_init(drain, T);
     abort_flag = 0;
@@ -479,47 +494,63 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::kThreads, 1)
     }
   } else if (warp >= 1 && warp <= T) {
     // ------------------------------------------------------------ MMA issuer
-    // Half i: S^T(i), dP^T(i); after the softmax wrote P^T and dS^T over them:
-    // dV += P^T dO, dK += dS^T Q; the next half's S^T and dP^T once those
-    // have read the buffers.
+    // Sub-half s (buffer s & 1): S^T(s) = K Q_s^T and dP^T(s) = V dO_s^T
+    // (M = 128 keys, N = 32 rows); once the softmax wrote P^T(s) / dS^T(s):
+    // dV += P^T(s) dO_s and dK += dS^T(s) Q_s (TS, K = 32), and, once those
+    // have read the buffer, S^T(s + 2) / dP^T(s + 2) into it.
     if (lane == 0) {
       const int x = warp - 1;
-      const uint32_t idesc_s = make_idesc_bf16(128, 64, false);
+      const uint32_t idesc_s = make_idesc_bf16(128, 32, false);
       const uint32_t idesc_o = make_idesc_bf16(128, D, true);
       const uint32_t k_base = smem_addr(smem + C::kKOffK) + x * C::kTile;
       const uint32_t v_base = smem_addr(smem + C::kKOffV) + x * C::kTile;
-      auto half_at = [&](uint32_t off, int i) {
-        return smem_addr(smem + off + (i % C::kKStages) * C::kHalf);
+      // rows of sub-half s inside its half's stage
+      auto sub_at = [&](uint32_t off, int s) {
+        return smem_addr(smem + off + ((s >> 1) % C::kKStages) * C::kHalf) +
+               (s & 1) * 32 * C::kRowBytes;
       };
-      auto issue_s = [&](int i) {
-        mma_rows_x_cols<D>(tmem + C::col_s(x), k_base, half_at(C::kKOffQ, i), C::kPanel64, idesc_s);
-        mma_commit(&s_full[x]);
-        mma_rows_x_cols<D>(tmem + C::col_dp(x), v_base, half_at(C::kKOffDO, i), C::kPanel64,
-                           idesc_s);
-        mma_commit(&dp_full[x]);
+      auto issue_st = [&](int s) {
+        const uint32_t buf = C::col_dkv_buf(x, s & 1);
+        mma_rows_x_cols<D>(tmem + buf, k_base, sub_at(C::kKOffQ, s), C::kPanel64, idesc_s);
+        mma_rows_x_cols<D>(tmem + buf + 32, v_base, sub_at(C::kKOffDO, s), C::kPanel64, idesc_s);
+        mma_commit(&st_full[x * 2 + (s & 1)]);
+      };
+      auto issue_out = [&](int s) {
+        const uint32_t buf = C::col_dkv_buf(x, s & 1);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint64_t bdo =
+              make_smem_desc(sub_at(C::kKOffDO, s) + kk * 16 * C::kRowBytes, C::kPanel64, C::kSbo, C::kSwz);
+          mma_ts(tmem + C::col_dkv_v(x), tmem + buf + kk * 8, bdo, idesc_o, (s > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t bq =
+              make_smem_desc(sub_at(C::kKOffQ, s) + kk * 16 * C::kRowBytes, C::kPanel64, C::kSbo, C::kSwz);
+          mma_ts(tmem + C::col_dkv_k(x), tmem + buf + 32 + kk * 8, bq, idesc_o,
+                 (s > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&o_done[x * 2 + (s & 1)]);
+        if (s & 1) mma_commit(&h_empty[(s >> 1) % C::kKStages]);
       };
       bool ok = mbar_wait(kv_full, 0, &abort_flag, dev_err) &&
                 mbar_wait(&h_full[0], 0, &abort_flag, dev_err);
       if (ok) {
         tc_fence_after();
-        issue_s(0);
+        issue_st(0);
+        issue_st(1);
       }
-      for (int i = 0; ok && i < n_h; ++i) {
-        if (!mbar_wait(&ds_full[x], i & 1, &abort_flag, dev_err)) break;
+      for (int s = 0; ok && s < n_s; ++s) {
+        const int bsel = x * 2 + (s & 1);
+        if (!mbar_wait(&ds_full[bsel], (s >> 1) & 1, &abort_flag, dev_err)) break;
         tc_fence_after();
-        mma_tmem_x_rows<D>(tmem + C::col_dv(x), tmem + C::col_s(x), half_at(C::kKOffDO, i),
-                           C::kPanel64, idesc_o, i == 0);
-        mma_tmem_x_rows<D>(tmem + C::col_dk(x), tmem + C::col_dp(x), half_at(C::kKOffQ, i),
-                           C::kPanel64, idesc_o, i == 0);
-        mma_commit(&o_done[x]);
-        mma_commit(&h_empty[i % C::kKStages]);
-        if (i + 1 < n_h) {
-          if (!mbar_wait(&h_full[(i + 1) % C::kKStages], ((i + 1) / C::kKStages) & 1, &abort_flag,
-                         dev_err) ||
-              !mbar_wait(&o_done[x], i & 1, &abort_flag, dev_err))
+        issue_out(s);
+        if (s + 2 < n_s) {
+          // S^T(s + 2) reuses this buffer: the dV / dK MMAs just issued read it
+          if (((s + 2) & 1) == 0 &&
+              !mbar_wait(&h_full[((s + 2) >> 1) % C::kKStages], (((s + 2) >> 1) / C::kKStages) & 1,
+                         &abort_flag, dev_err))
             break;
+          if (!mbar_wait(&o_done[bsel], (s >> 1) & 1, &abort_flag, dev_err)) break;
           tc_fence_after();
-          issue_s(i + 1);
+          issue_st(s + 2);
         }
       }
     }
@@ -533,78 +564,71 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::kThreads, 1)
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const float c = kLog2eB * rsqrtf(static_cast<float>(D));
     bool ok = true;
-    for (int i = 0; i < n_h; ++i) {
-      const int st = i % C::kKStages;
-      const int64_t row0 = static_cast<int64_t>(u0 + i) * 64;   // first packed row of the half
-      // columns e of the half are visible when lo <= e < hi
+    for (int s = 0; s < n_s; ++s) {
+      const int i = s >> 1, st = i % C::kKStages;
+      const int64_t row0 = static_cast<int64_t>(u0 + i) * 64 + (s & 1) * 32;   // first row
+      // columns e of the sub-half are visible when lo <= e < hi
       int lo = 0;
       if (causal) {
         const int64_t first = (static_cast<int64_t>(s_pos) << G_log2) - row0;
-        lo = first <= 0 ? 0 : (first >= 64 ? 64 : static_cast<int>(first));
+        lo = first <= 0 ? 0 : (first >= 32 ? 32 : static_cast<int>(first));
       }
       const int64_t left = rows_all - row0;
-      const int hi = left >= 64 ? 64 : static_cast<int>(left);
-      if (!key_in) lo = 64;
-      const bool full = __all_sync(0xffffffffu, lo == 0 && hi == 64);
+      const int hi = left >= 32 ? 32 : (left <= 0 ? 0 : static_cast<int>(left));
+      if (!key_in) lo = 32;
+      const bool full = __all_sync(0xffffffffu, lo == 0 && hi == 32);
+      const int bsel = x * 2 + (s & 1);
+      const uint32_t buf = C::col_dkv_buf(x, s & 1);
       // lse2 / D of the half (h_full: the bulk copies have landed)
       if (!mbar_wait(&h_full[st], (i / C::kKStages) & 1, &abort_flag, dev_err) ||
-          !mbar_wait(&s_full[x], i & 1, &abort_flag, dev_err)) {
+          !mbar_wait(&st_full[bsel], (s >> 1) & 1, &abort_flag, dev_err)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float* Ls = reinterpret_cast<const float*>(smem + C::kKOffL + st * 512);
+      const float* Ls = reinterpret_cast<const float*>(smem + C::kKOffL + st * 512) + (s & 1) * 32;
       const float* Ds = Ls + 64;
-      uint32_t pt[32];
-      float p[64];
+      uint32_t sv[32], dpv[32], pt[16], dt[16];
+      tmem_ld32(trow + buf, sv);
+      tmem_ld32(trow + buf + 32, dpv);
+      tmem_wait_ld();
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t sv[32];
-        tmem_ld32(trow + C::col_s(x) + ch * 32, sv);
-        tmem_wait_ld();
+      for (int e4 = 0; e4 < 32; e4 += 4) {
+        const float4 l4 = lds4(Ls + e4);
+        const float4 d4 = lds4(Ds + e4);
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+        const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+        float pe[4], de[4];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int col = ch * 32 + e;
-          const float pv = ex2f(fmaf(__uint_as_float(sv[e]), c, -Ls[col]));
-          p[col] = (full || (col >= lo && col < hi)) ? pv : 0.f;
+        for (int u = 0; u < 4; ++u) {
+          const int e = e4 + u;
+          const bool vis = full || (e >= lo && e < hi);
+          const float pv = ex2f(fmaf(__uint_as_float(sv[e]), c, -lv[u]));
+          pe[u] = vis ? pv : 0.f;
+          de[u] = vis ? pv * (__uint_as_float(dpv[e]) - dv4[u]) : 0.f;
         }
+        pt[e4 / 2] = pack2(pe[0], pe[1]);
+        pt[e4 / 2 + 1] = pack2(pe[2], pe[3]);
+        dt[e4 / 2] = pack2(de[0], de[1]);
+        dt[e4 / 2 + 1] = pack2(de[2], de[3]);
       }
-#pragma unroll
-      for (int e = 0; e < 32; ++e) pt[e] = pack2(p[2 * e], p[2 * e + 1]);
-      tmem_st32(trow + C::col_s(x), pt);
-      if (!mbar_wait(&dp_full[x], i & 1, &abort_flag, dev_err)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-#pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t dpv[32], ds[16];
-        tmem_ld32(trow + C::col_dp(x) + ch * 32, dpv);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c0 = ch * 32 + 2 * e, c1 = c0 + 1;
-          const float d0 = p[c0] * (__uint_as_float(dpv[2 * e]) - Ds[c0]);
-          const float d1 = p[c1] * (__uint_as_float(dpv[2 * e + 1]) - Ds[c1]);
-          ds[e] = pack2((full || (c0 >= lo && c0 < hi)) ? d0 : 0.f,
-                        (full || (c1 >= lo && c1 < hi)) ? d1 : 0.f);
-        }
-        tmem_st16(trow + C::col_dp(x) + ch * 16, ds);
-      }
+      tmem_st16(trow + buf, pt);
+      tmem_st16(trow + buf + 32, dt);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&ds_full[x]);
+      mbar_arrive(&ds_full[bsel]);
     }
-    if (ok && n_h > 0 && mbar_wait(&o_done[x], (n_h - 1) & 1, &abort_flag, dev_err)) {
+    // the last sub-half's dV / dK complete after all earlier ones
+    if (ok && n_s > 0 &&
+        mbar_wait(&o_done[x * 2 + ((n_s - 1) & 1)], ((n_s - 1) >> 1) & 1, &abort_flag, dev_err)) {
       tc_fence_after();
       const float sc = rsqrtf(static_cast<float>(D));
       const int64_t krow = (static_cast<int64_t>(bg) * S + s_pos) * D;
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t vv[32], kv[32];
-        tmem_ld32(trow + C::col_dv(x) + cc * 32, vv);
-        tmem_ld32(trow + C::col_dk(x) + cc * 32, kv);
+        tmem_ld32(trow + C::col_dkv_v(x) + cc * 32, vv);
+        tmem_ld32(trow + C::col_dkv_k(x) + cc * 32, kv);
         tmem_wait_ld();
         if (key_in) {
 #pragma unroll
