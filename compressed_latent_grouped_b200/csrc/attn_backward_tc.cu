@@ -29,6 +29,8 @@
 //             all G heads, so the group's sum comes from the MMA itself.
 // The 1 / sqrt(d) of dq and dk is applied at the store; P and dS are rounded
 // to bf16 for the MMAs, everything else is fp32.
+#include <algorithm>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -404,10 +406,24 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::kThreads, 1)
                            const __grid_constant__ CUtensorMap tmV,
                            const float* __restrict__ lse, const float* __restrict__ dsum,
                            float* __restrict__ dk, float* __restrict__ dv, int B, int S, int Hkv,
-                           int G_log2, int causal, int64_t ld, int32_t* dev_err) {
+                           int G_log2, int causal, int64_t ld, int chunk_halves, int max_chunks,
+                           int32_t* dev_err) {
   pdl_enter();
   using C = BwdTcCfg<D>;
   constexpr int T = C::kTiles;
+  // CTA = (key group, chunk of at most chunk_halves query halves, sequence x
+  // kv group); the chunks' dK / dV are summed atomically into zeroed buffers
+  const int BH = B * Hkv;
+  const int bg = static_cast<int>(blockIdx.x) % BH;
+  const int chunk = (static_cast<int>(blockIdx.x) / BH) % max_chunks;
+  const int kgrp = static_cast<int>(blockIdx.x) / BH / max_chunks;   // ascending: longest first
+  const int k_start = kgrp * T * 128;
+  const int64_t rows_all = static_cast<int64_t>(S) << G_log2;   // packed query rows of (b, g)
+  const int u_first = causal ? static_cast<int>((static_cast<int64_t>(k_start) << G_log2) >> 6) : 0;
+  const int n_h_all = static_cast<int>((rows_all + 63) >> 6) - u_first;
+  if (chunk * chunk_halves >= n_h_all) return;   // nothing left for this chunk
+  const int u0 = u_first + chunk * chunk_halves;
+  const int n_h = min(chunk_halves, n_h_all - chunk * chunk_halves);   // 64-row halves
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -423,14 +439,7 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::kThreads, 1)
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int BH = B * Hkv;
-  const int kgrp = static_cast<int>(blockIdx.x) / BH;    // ascending: the longest first
-  const int bg = static_cast<int>(blockIdx.x) % BH;
   const int b = bg / Hkv, g = bg % Hkv;
-  const int k_start = kgrp * T * 128;
-  const int64_t rows_all = static_cast<int64_t>(S) << G_log2;   // packed query rows of (b, g)
-  const int u0 = causal ? static_cast<int>((static_cast<int64_t>(k_start) << G_log2) >> 6) : 0;
-  const int n_h = static_cast<int>((rows_all + 63) >> 6) - u0;  // 64-row halves
   const int n_s = 2 * n_h;                                      // 32-row sub-halves
   const int pos_per_half = 64 >> G_log2;
 
@@ -633,12 +642,12 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::kThreads, 1)
         if (key_in) {
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
-            *reinterpret_cast<float4*>(dv + krow + cc * 32 + e) =
-                make_float4(__uint_as_float(vv[e]), __uint_as_float(vv[e + 1]),
-                            __uint_as_float(vv[e + 2]), __uint_as_float(vv[e + 3]));
-            *reinterpret_cast<float4*>(dk + krow + cc * 32 + e) =
-                make_float4(__uint_as_float(kv[e]) * sc, __uint_as_float(kv[e + 1]) * sc,
-                            __uint_as_float(kv[e + 2]) * sc, __uint_as_float(kv[e + 3]) * sc);
+            atomicAdd(reinterpret_cast<float4*>(dv + krow + cc * 32 + e),
+                      make_float4(__uint_as_float(vv[e]), __uint_as_float(vv[e + 1]),
+                                  __uint_as_float(vv[e + 2]), __uint_as_float(vv[e + 3])));
+            atomicAdd(reinterpret_cast<float4*>(dk + krow + cc * 32 + e),
+                      make_float4(__uint_as_float(kv[e]) * sc, __uint_as_float(kv[e + 1]) * sc,
+                                  __uint_as_float(kv[e + 2]) * sc, __uint_as_float(kv[e + 3]) * sc));
           }
         }
       }
@@ -713,16 +722,36 @@ cudaError_t launch_bwd_tc(const AttnBwdTcArgs& a, cudaStream_t stream) {
     count_launches(1);
     if (e != cudaSuccess) return e;
   }
-  // dkv pass
+  // dkv pass: the query halves of a key group are cut into chunks of at most
+  // L halves, L sized for about six waves of one CTA per SM (at least 16, so
+  // a chunk's K / V load and atomic epilogue stay small beside its work)
   {
     const int n_kgroups = (a.S + C::kTiles * 128 - 1) / (C::kTiles * 128);
-    cudaError_t e = allow_smem(reinterpret_cast<const void*>(attn_bwd_dkv_tc_kernel<D>),
-                               static_cast<int>(C::kKSmem));
+    const int64_t rows_all = static_cast<int64_t>(a.S) << G_log2;
+    const int64_t halves_all = (rows_all + 63) >> 6;
+    int64_t work = 0, longest = 0;
+    for (int kg = 0; kg < n_kgroups; ++kg) {
+      const int64_t u_first =
+          a.causal ? ((static_cast<int64_t>(kg) * C::kTiles * 128) << G_log2) >> 6 : 0;
+      work += halves_all - u_first;
+      longest = std::max<int64_t>(longest, halves_all - u_first);
+    }
+    work *= BH;
+    int64_t L = (work + 6 * 148 - 1) / (6 * 148);
+    if (L < 16) L = 16;
+    if (L > longest) L = longest;
+    const int max_chunks = static_cast<int>((longest + L - 1) / L);
+    const size_t kv_bytes = static_cast<size_t>(BH) * a.S * D * sizeof(float);
+    cudaError_t e = cudaMemsetAsync(a.dk, 0, kv_bytes, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(a.dv, 0, kv_bytes, stream);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(attn_bwd_dkv_tc_kernel<D>, dim3(n_kgroups * BH), dim3(C::kThreads), C::kKSmem,
-                   stream, tmQh, tmDOh, tmK, tmV, static_cast<const float*>(a.lse),
+    e = allow_smem(reinterpret_cast<const void*>(attn_bwd_dkv_tc_kernel<D>),
+                   static_cast<int>(C::kKSmem));
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(attn_bwd_dkv_tc_kernel<D>, dim3(n_kgroups * max_chunks * BH), dim3(C::kThreads),
+                   C::kKSmem, stream, tmQh, tmDOh, tmK, tmV, static_cast<const float*>(a.lse),
                    static_cast<const float*>(a.dsum), a.dk, a.dv, a.B, a.S, a.Hkv, G_log2,
-                   a.causal, a.ld, a.dev_err);
+                   a.causal, a.ld, static_cast<int>(L), max_chunks, a.dev_err);
     count_launches(1);
     if (e != cudaSuccess) return e;
   }
