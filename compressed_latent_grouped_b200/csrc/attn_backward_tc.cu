@@ -6,9 +6,11 @@
 // Inputs: q [B, S, Hq, d], k, v [B, Hkv, S, d], the forward output o and the
 // upstream gradient dO [B, S, Hq, d] (bf16), and the forward's log-sum-exp in
 // base 2 per query row, lse2 = log2(sum_s 2^(c s_ts)) with c = log2(e) / sqrt(d),
-// in the packed row order of the forward (row t G + head-in-group, a stride of
-// ld floats per (sequence, kv group)).  With P = 2^(c S - lse2) the softmax of
-// the scores S = q k^T and D = rowsum(dO o):
+// stored negated in the packed row order of the forward (row t G + head in
+// group, a stride of ld floats per (sequence, kv group)); D is stored negated
+// the same way, so that each score costs one packed FMA before the exponential
+// and one packed add and multiply after it.  With P = 2^(c S - lse2) the
+// softmax of the scores S = q k^T and D = rowsum(dO o):
 //   dP = dO v^T,  dS = P (dP - D),  dq = dS k / sqrt(d),
 //   dk = dS^T q / sqrt(d),  dv = P^T dO   (summed over the G heads of a group).
 //
@@ -70,7 +72,7 @@ struct BwdTcCfg {
   static constexpr uint32_t kKOffV = kKOffK + kTiles * kTile;
   static constexpr uint32_t kKOffQ = kKOffV + kTiles * kTile;
   static constexpr uint32_t kKOffDO = kKOffQ + kKStages * kHalf;
-  static constexpr uint32_t kKOffL = kKOffDO + kKStages * kHalf;   // [stage][lse2 64 | D 64]
+  static constexpr uint32_t kKOffL = kKOffDO + kKStages * kHalf;   // [stage][-lse2 64 | -D 64]
   static constexpr uint32_t kKOffBar = kKOffL + kKStages * 512;
   static constexpr size_t kKSmem = kKOffBar + 256 + 1024;
   // TMEM columns.  dq pass: S and dP (64 each) per tile, then dQ per tile.
@@ -100,6 +102,30 @@ __device__ __forceinline__ float4 lds4(const float* p) {
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                : "r"(smem_addr(p)));
   return v;
+}
+
+// Packed fp32 pairs on the FMA pipe (one instruction for two values).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)),
+        "l"(*reinterpret_cast<const uint64_t*>(&c)));
+  return *reinterpret_cast<float2*>(&d);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)));
+  return *reinterpret_cast<float2*>(&d);
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)));
+  return *reinterpret_cast<float2*>(&d);
 }
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
@@ -297,9 +323,9 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::kThreads, 1)
     const int64_t prow = static_cast<int64_t>(bg) * ld + (static_cast<int64_t>(t) << G_log2) + hl;
     const int64_t grow = ((static_cast<int64_t>(b) * S + t) * Hq + g * G + hl) * D;
     // D = rowsum(dO o) of this row (bf16 inputs, fp32 sum), kept for the dkv pass
-    float lse2 = 0.f, Dr = 0.f;
+    float nlse = 0.f, Dr = 0.f;   // -lse2, D
     if (row_in) {
-      lse2 = lse[prow];
+      nlse = lse[prow];
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < D / 8; ++i) {
@@ -315,9 +341,11 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::kThreads, 1)
         }
       }
       Dr = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-      dsum[prow] = Dr;
+      dsum[prow] = -Dr;
     }
+    const float2 nl2 = make_float2(nlse, nlse), nd2 = make_float2(-Dr, -Dr);
     const float c = kLog2eB * rsqrtf(static_cast<float>(D));
+    const float2 c2 = make_float2(c, c);
     bool ok = true;
     for (int k = 0; k < n_h; ++k) {
       const int kb = k * 64;
@@ -335,7 +363,11 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::kThreads, 1)
       tmem_ld32(trow + C::col_s(x) + 32, *reinterpret_cast<uint32_t(*)[32]>(&p[32]));
       tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 64; ++e) p[e] = ex2f(fmaf(p[e], c, -lse2));
+      for (int e = 0; e < 64; e += 2) {
+        const float2 a2 = ffma2(make_float2(p[e], p[e + 1]), c2, nl2);
+        p[e] = ex2f(a2.x);
+        p[e + 1] = ex2f(a2.y);
+      }
       if (!full) {
 #pragma unroll
         for (int e = 0; e < 64; ++e) p[e] = (e <= lim) ? p[e] : 0.f;
@@ -351,9 +383,13 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::kThreads, 1)
         tmem_ld32(trow + C::col_dp(x) + ch * 32, dp);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          ds[e] = pack2(p[ch * 32 + 2 * e] * (__uint_as_float(dp[2 * e]) - Dr),
-                        p[ch * 32 + 2 * e + 1] * (__uint_as_float(dp[2 * e + 1]) - Dr));
+        for (int e = 0; e < 16; ++e) {
+          const float2 d2 = fmul2(make_float2(p[ch * 32 + 2 * e], p[ch * 32 + 2 * e + 1]),
+                                  fadd2(make_float2(__uint_as_float(dp[2 * e]),
+                                                    __uint_as_float(dp[2 * e + 1])),
+                                        nd2));
+          ds[e] = pack2(d2.x, d2.y);
+        }
         tmem_st16(trow + C::col_dp(x) + ch * 16, ds);
       }
       tmem_wait_st();
@@ -588,7 +624,7 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::kThreads, 1)
       const bool full = __all_sync(0xffffffffu, lo == 0 && hi == 32);
       const int bsel = x * 2 + (s & 1);
       const uint32_t buf = C::col_dkv_buf(x, s & 1);
-      // lse2 / D of the half (h_full: the bulk copies have landed)
+      // -lse2 / -D of the half (h_full: the bulk copies have landed)
       if (!mbar_wait(&h_full[st], (i / C::kKStages) & 1, &abort_flag, dev_err) ||
           !mbar_wait(&st_full[bsel], (s >> 1) & 1, &abort_flag, dev_err)) {
         ok = false;
@@ -601,25 +637,49 @@ __global__ void __launch_bounds__(BwdTcCfg<D>::kThreads, 1)
       tmem_ld32(trow + buf, sv);
       tmem_ld32(trow + buf + 32, dpv);
       tmem_wait_ld();
+      // Ls / Ds hold -lse2 and -D per column: p = 2^(c s - lse2), ds = p (dp - D)
+      const float2 c2 = make_float2(c, c);
+      if (full) {
 #pragma unroll
-      for (int e4 = 0; e4 < 32; e4 += 4) {
-        const float4 l4 = lds4(Ls + e4);
-        const float4 d4 = lds4(Ds + e4);
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-        const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
-        float pe[4], de[4];
+        for (int e4 = 0; e4 < 32; e4 += 4) {
+          const float4 l4 = lds4(Ls + e4);
+          const float4 d4 = lds4(Ds + e4);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int e = e4 + u;
-          const bool vis = full || (e >= lo && e < hi);
-          const float pv = ex2f(fmaf(__uint_as_float(sv[e]), c, -lv[u]));
-          pe[u] = vis ? pv : 0.f;
-          de[u] = vis ? pv * (__uint_as_float(dpv[e]) - dv4[u]) : 0.f;
+          for (int u = 0; u < 2; ++u) {
+            const int e = e4 + 2 * u;
+            const float2 a2 = ffma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])),
+                                    c2, u ? make_float2(l4.z, l4.w) : make_float2(l4.x, l4.y));
+            const float2 p2 = make_float2(ex2f(a2.x), ex2f(a2.y));
+            const float2 d2 =
+                fmul2(p2, fadd2(make_float2(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])),
+                                u ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y)));
+            pt[e / 2] = pack2(p2.x, p2.y);
+            dt[e / 2] = pack2(d2.x, d2.y);
+          }
         }
-        pt[e4 / 2] = pack2(pe[0], pe[1]);
-        pt[e4 / 2 + 1] = pack2(pe[2], pe[3]);
-        dt[e4 / 2] = pack2(de[0], de[1]);
-        dt[e4 / 2 + 1] = pack2(de[2], de[3]);
+      } else {
+        // columns outside [lo, hi) are masked (past the sequence, the padding's
+        // -lse2 / -D may hold anything, so the results are selected, not scaled)
+#pragma unroll
+        for (int e4 = 0; e4 < 32; e4 += 4) {
+          const float4 l4 = lds4(Ls + e4);
+          const float4 d4 = lds4(Ds + e4);
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+          const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pe[4], de[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int e = e4 + u;
+            const bool vis = e >= lo && e < hi;
+            const float pv = ex2f(fmaf(__uint_as_float(sv[e]), c, lv[u]));
+            pe[u] = vis ? pv : 0.f;
+            de[u] = vis ? pv * (__uint_as_float(dpv[e]) + dv4[u]) : 0.f;
+          }
+          pt[e4 / 2] = pack2(pe[0], pe[1]);
+          pt[e4 / 2 + 1] = pack2(pe[2], pe[3]);
+          dt[e4 / 2] = pack2(de[0], de[1]);
+          dt[e4 / 2 + 1] = pack2(de[2], de[3]);
+        }
       }
       tmem_st16(trow + buf, pt);
       tmem_st16(trow + buf + 32, dt);

@@ -448,7 +448,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
       const float inv_l = 1.f / l;
       const bool store = row_ok && t < S;
       if (lse != nullptr && store)
-        lse[static_cast<int64_t>(bg) * lse_ld + static_cast<int64_t>(t) * G + hl] = m_used + log2f(l);
+        lse[static_cast<int64_t>(bg) * lse_ld + static_cast<int64_t>(t) * G + hl] = -(m_used + log2f(l));
       bf16* dst = out + ((static_cast<int64_t>(b) * S + t) * Hq + g * G + hl) * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {

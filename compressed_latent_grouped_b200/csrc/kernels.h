@@ -80,8 +80,8 @@ struct AttnArgs {
   int causal;
   int32_t* dev_err;
   // optional (tensor-core kernel only): each stored row's log-sum-exp in base
-  // 2 of the scaled scores, log2(sum_s 2^(log2(e) q.k_s / sqrt(d))), at
-  // lse[(b Hkv + g) lse_ld + t G + head in group]
+  // 2 of the scaled scores, negated, -log2(sum_s 2^(log2(e) q.k_s / sqrt(d))),
+  // at lse[(b Hkv + g) lse_ld + t G + head in group]
   float* lse = nullptr;
   int64_t lse_ld = 0;
 };
@@ -91,8 +91,8 @@ cudaError_t launch_attn_prefill_tc(const AttnArgs& a, cudaStream_t stream);
 
 // Attention backward on the tensor core (bf16, d in {32, 64, 128}, G a power
 // of two up to 64).  lse / dsum: [B Hkv, ld] packed per (sequence, kv group),
-// row t G + head in group, ld a multiple of 64 of at least S G; lse from the
-// forward kernel, dsum written here (D = rowsum(dO o)).
+// row t G + head in group, ld a multiple of 64 of at least S G, both negated:
+// lse from the forward kernel, dsum written here (-D, D = rowsum(dO o)).
 struct AttnBwdTcArgs {
   const void *q, *k, *v, *o, *dout;   // q, o, dout [B, S, Hq, d]; k, v [B, Hkv, S, d]
   const float* lse;
