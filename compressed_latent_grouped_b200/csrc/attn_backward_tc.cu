@@ -25,10 +25,14 @@
 //             form D for their rows (read by the second kernel).
 //   dkv pass  key-major: per 128-key tile (T tiles per CTA), the packed query
 //             rows that see it in halves of 64 rows (Q and dO halves, lse2 and
-//             D of the half by bulk copy).  S^T = K Q^T, dP^T = V dO^T; P^T is
-//             written as bf16 over the S^T buffer and dS^T over the dP^T
-//             buffer; dV += P^T dO and dK += dS^T Q (TS).  A half holds rows of
-//             all G heads, so the group's sum comes from the MMA itself.
+//             D of the half by bulk copy), each worked as two 32-row
+//             sub-halves in two TMEM buffers per tile.  S^T = K Q^T,
+//             dP^T = V dO^T; P^T is written as bf16 over S^T and dS^T over
+//             dP^T; dV += P^T dO and dK += dS^T Q (TS) while the next
+//             sub-half's scores go into the other buffer.  A half holds rows of
+//             all G heads, so the group's sum comes from the MMA itself.  A key
+//             tile's halves are cut into chunks, one CTA each, whose dK / dV
+//             are added atomically into zeroed buffers.
 // The 1 / sqrt(d) of dq and dk is applied at the store; P and dS are rounded
 // to bf16 for the MMAs, everything else is fp32.
 #include <algorithm>
