@@ -327,6 +327,10 @@ def measure_prefill_workload(w, steps, dev):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     for _ in range(3):
         lay.prefill(x, out)
+    # two kernels per call: the projection ran fused with the pre-attention
+    n0 = B.ccgqa_launch_count()
+    lay.prefill(x, out)
+    fused = B.ccgqa_launch_count() - n0 == 2 and not w.packed_input
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     for e in evs:
         flush.zero_()
@@ -344,7 +348,12 @@ def measure_prefill_workload(w, steps, dev):
            "attn_exp_unit_frac": exp_roofline(w, ms[2], peaks)["frac"],
            "pre_attn_ms": ms[1], "prefill_ms": sum(ms),
            "tokens_per_s": w.B * w.S / (sum(ms) / 1e3)}
-    if not w.packed_input:
+    if fused:
+        # one kernel: the projection GEMM's FLOPs over its time
+        res.pop("pre_attn_ms")
+        res["proj_pre_fused_ms"] = ms[0] + ms[1]
+        res["proj_pre_tflops"] = 2.0 * w.B * w.S * w.E * w.n_qkv / ((ms[0] + ms[1]) / 1e3) / 1e12
+    elif not w.packed_input:
         res["proj_ms"] = ms[0]
         res["proj_tflops"] = 2.0 * w.B * w.S * w.E * w.n_qkv / (ms[0] / 1e3) / 1e12
         pre_bytes = 2 * w.B * w.S * w.n_qkv * 2
@@ -515,6 +524,9 @@ def run_workload_only(args, local):
         w = w.with_(S=args.seq)
     if args.decode:
         w = w.with_(decode=True)
+    if args.unfused:
+        from compressed_latent_grouped_b200 import binding as B
+        B.ccgqa_set_fused_projection(False)
     if args.output_projection:
         res = measure_output_projection(w, args.steps, dev)
     elif args.backward:
@@ -815,6 +827,8 @@ def main():
     ap.add_argument("--seq", type=int, default=0, help="with --workload: override S (or L)")
     ap.add_argument("--decode", action="store_true",
                     help="with --workload: time a decode step against a cache of S tokens")
+    ap.add_argument("--unfused", action="store_true",
+                    help="with --workload: run the projection and pre-attention as separate kernels")
     ap.add_argument("--paged", type=int, default=0,
                     help="with --workload and a decode: a paged cache of this many tokens per page")
     ap.add_argument("--output-projection", action="store_true",

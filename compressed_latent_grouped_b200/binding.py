@@ -106,6 +106,8 @@ def load() -> ctypes.CDLL:
     lib.ccgqa_last_error_string.restype = c_char_p
     lib.ccgqa_set_phase_events.argtypes = [c_void_p, c_int32]
     lib.ccgqa_set_phase_events.restype = None
+    lib.ccgqa_set_fused_projection.argtypes = [c_int32]
+    lib.ccgqa_set_fused_projection.restype = None
     lib.ccgqa_selftest_wait_timeout.argtypes = [ctypes.c_int64, c_void_p, c_void_p]
     lib.ccgqa_selftest_wait_timeout.restype = c_int
     lib.ccgqa_graph_begin.argtypes = [c_void_p]
@@ -325,6 +327,12 @@ def ccgqa_graph_destroy(graph) -> None:
 
 
 _phase_keep = None
+
+
+def ccgqa_set_fused_projection(enable: bool) -> None:
+    """Process-wide: let ccgqa_prefill fuse the projection with the
+    pre-attention where that kernel applies (default on)."""
+    load().ccgqa_set_fused_projection(1 if enable else 0)
 
 
 def ccgqa_set_phase_events(events) -> None:

@@ -56,6 +56,10 @@ static ccgqa_status cuda_fail(cudaError_t e) {
   return CCGQA_ERR_CUDA;
 }
 
+// Whether ccgqa_prefill may fuse the projection with the pre-attention
+// (ccgqa_set_fused_projection; on unless switched off).
+static std::atomic<int> g_fuse_proj{1};
+
 // Optional phase events of the calling thread (ccgqa_set_phase_events).
 static thread_local void* const* t_phase_events = nullptr;
 static void phase_mark(int i, cudaStream_t st) {
@@ -222,21 +226,10 @@ ccgqa_status run_prefill(const Geo& g, const ccgqa_weights* w, const void* x, in
                          void* out, const ccgqa_kvcache* cache, uint8_t* ws, int32_t* dev_err,
                          cudaStream_t st) {
   const PrefillWs L = prefill_ws(g, B, S);
-  const T* src = static_cast<const T*>(x);
+  T* proj = reinterpret_cast<T*>(ws + L.proj);
+  const T* src = w->W_qkv ? proj : static_cast<const T*>(x);
   cudaError_t e = cudaSuccess;
   phase_mark(0, st);
-  if (w->W_qkv) {
-    T* proj = reinterpret_cast<T*>(ws + L.proj);
-    if constexpr (sizeof(T) == 2)
-      e = launch_proj_gemm_bf16(static_cast<const bf16*>(x), static_cast<const bf16*>(w->W_qkv),
-                                proj, B * S, g.N, g.E, dev_err, st);
-    else
-      e = launch_proj_gemm_f32(static_cast<const float*>(x), static_cast<const float*>(w->W_qkv),
-                               proj, B * S, g.N, g.E, st);
-    if (e != cudaSuccess) return cuda_fail(e);
-    src = proj;
-  }
-  phase_mark(1, st);
   PreAttnArgs<T> a{};
   a.src = src;
   a.src_ld = g.N;
@@ -277,7 +270,32 @@ ccgqa_status run_prefill(const Geo& g, const ccgqa_weights* w, const void* x, in
     a.len = cache->len;
   }
   a.dev_err = dev_err;
-  if ((e = launch_pre_attn<T>(a, st)) != cudaSuccess) return cuda_fail(e);
+  bool fused = false;
+  if constexpr (sizeof(T) == 2)
+    fused = w->W_qkv && g_fuse_proj.load() &&
+            proj_pre_tc_supported(a, static_cast<const bf16*>(x),
+                                  static_cast<const bf16*>(w->W_qkv), g.E);
+  if (fused) {
+    // projection and pre-attention in one kernel (no q~ | k~ | v~ in HBM)
+    if constexpr (sizeof(T) == 2)
+      e = launch_proj_pre_tc(static_cast<const bf16*>(x), static_cast<const bf16*>(w->W_qkv), g.E,
+                             a, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    phase_mark(1, st);
+  } else {
+    if (w->W_qkv) {
+      if constexpr (sizeof(T) == 2)
+        e = launch_proj_gemm_bf16(static_cast<const bf16*>(x),
+                                  static_cast<const bf16*>(w->W_qkv), proj, B * S, g.N, g.E,
+                                  dev_err, st);
+      else
+        e = launch_proj_gemm_f32(static_cast<const float*>(x),
+                                 static_cast<const float*>(w->W_qkv), proj, B * S, g.N, g.E, st);
+      if (e != cudaSuccess) return cuda_fail(e);
+    }
+    phase_mark(1, st);
+    if ((e = launch_pre_attn<T>(a, st)) != cudaSuccess) return cuda_fail(e);
+  }
   phase_mark(2, st);
   AttnArgs at{};
   at.q = a.q_out;
@@ -765,6 +783,8 @@ CCGQA_API const char* ccgqa_status_string(ccgqa_status s) {
 CCGQA_API uint64_t ccgqa_launch_count(void) { return g_launches.load(); }
 
 CCGQA_API const char* ccgqa_last_error_string(void) { return t_last_error; }
+
+CCGQA_API void ccgqa_set_fused_projection(int32_t enable) { g_fuse_proj.store(enable ? 1 : 0); }
 
 CCGQA_API void ccgqa_set_phase_events(void* const* events, int32_t n) {
   t_phase_events = (events != nullptr && n >= 4) ? events : nullptr;

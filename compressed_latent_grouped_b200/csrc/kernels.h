@@ -68,6 +68,11 @@ bool pre_attn_fits(int K, int G, int d, int es, bool has_mix);
 // on tcgen05, staging by TMA (launch_pre_attn dispatches there when this holds).
 bool pre_attn_tc_supported(const PreAttnArgs<bf16>& a);
 cudaError_t launch_pre_attn_tc(const PreAttnArgs<bf16>& a, cudaStream_t stream);
+// The projection fused with the pre-attention (bf16, d = 32, G <= 6, conv 1..4
+// taps with both channel-mix weights): x [B, S, E] and W [N, E] in, a.src unused.
+bool proj_pre_tc_supported(const PreAttnArgs<bf16>& a, const bf16* x, const bf16* W, int E);
+cudaError_t launch_proj_pre_tc(const bf16* x, const bf16* W, int E, const PreAttnArgs<bf16>& a,
+                               cudaStream_t stream);
 
 // ----------------------------------------------------------------- attention
 struct AttnArgs {

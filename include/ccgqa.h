@@ -321,6 +321,17 @@ CCGQA_API uint64_t ccgqa_launch_count(void);
  * turns it off.  Only the pointer is kept; the caller keeps the events alive. */
 CCGQA_API void ccgqa_set_phase_events(void* const* events, int32_t n);
 
+/* Process-wide switch (default 1 = on).  When on, ccgqa_prefill runs the
+ * latent projection and the pre-attention steps as ONE kernel where that
+ * kernel applies: bf16, d = 32, a projection weight, conv width 1..4 with
+ * depthwise taps and both channel-mix weights, G <= 6, 16-byte aligned x, W
+ * and conv weights ("Compressed Convolutional Attention", Methodologie: the
+ * projected q~ | k~ | v~ never reach HBM).  Its phase events [1] and [2] then
+ * both fall after that kernel.  0 runs the projection GEMM and the
+ * pre-attention kernel separately (the results agree within the bf16 rounding
+ * of the projection output).  For measurement and testing. */
+CCGQA_API void ccgqa_set_fused_projection(int32_t enable);
+
 /* Self-test of the device-side failure reporting (no counterpart in the
  * papers; it exercises the bounded wait every kernel of this library uses).
  * Launches one small kernel on `stream` whose threads wait on an mbarrier that

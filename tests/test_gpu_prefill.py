@@ -173,7 +173,15 @@ def test_launches_are_counted():
     inp = make_inputs(w, seed=0)
     n0 = B.ccgqa_launch_count()
     _run(w, inp)
-    assert B.ccgqa_launch_count() - n0 == 3   # projection, pre-attention, attention
+    # d = 32: the projection fused with the pre-attention, then attention
+    assert B.ccgqa_launch_count() - n0 == 2
+    B.ccgqa_set_fused_projection(False)
+    try:
+        n0 = B.ccgqa_launch_count()
+        _run(w, inp)
+        assert B.ccgqa_launch_count() - n0 == 3   # projection, pre-attention, attention
+    finally:
+        B.ccgqa_set_fused_projection(True)
 
 
 def _growing_score_inputs(w, slope, seed=0):
