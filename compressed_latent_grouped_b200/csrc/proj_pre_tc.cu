@@ -102,6 +102,507 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// ------------------------------------------------------------------ persistent
+// The persistent, warp-specialised form (G <= 5): one CTA per SM walks tiles
+// c, c + grid, ...; warp 0 streams the GEMM operands through a ring that runs
+// on across tiles, warp 1 accumulates tile i into one of two TMEM accumulators
+// (2 (G + 2) d columns, then the two mix accumulators), and warps 2-9 (256
+// threads) do the heads of tile i - 1 meanwhile, so the pre-attention work
+// hides behind the next tile's GEMM.
+constexpr int kPwStages = 3;
+constexpr int kPwThreads = 64 + 256;
+
+struct PwLayout {
+  uint32_t nz, a_bytes, b_bytes, stage_bytes, zh_bytes, u_bytes, w_bytes;
+  uint32_t off_z, off_u, off_w, off_ws, off_bar, bytes;
+};
+
+// ring | staged head rows (G + 2 slots of 128 x 64 B) | U_hi, U_lo | mix
+// weights (G + 1 tiles of 32 x 64 B) | taps [(G + 1) d][4] bf16 | barriers
+__host__ __device__ inline PwLayout pw_layout(int G) {
+  PwLayout L;
+  L.nz = static_cast<uint32_t>(G + 2) * kPpD;
+  L.a_bytes = kPpM * kPpBK * 2;
+  L.b_bytes = L.nz * kPpBK * 2;
+  L.stage_bytes = (L.a_bytes + L.b_bytes + 1023u) & ~1023u;
+  L.zh_bytes = kPpM * kPpRow;
+  L.u_bytes = kPpM * kPpRow;
+  L.w_bytes = kPpD * kPpRow;
+  L.off_z = kPwStages * L.stage_bytes;
+  L.off_u = L.off_z + static_cast<uint32_t>(G + 2) * L.zh_bytes;
+  L.off_w = L.off_u + 2 * L.u_bytes;
+  L.off_ws = L.off_w + static_cast<uint32_t>(G + 1) * L.w_bytes;
+  L.off_bar = L.off_ws + static_cast<uint32_t>(G + 1) * kPpD * 8;
+  L.bytes = L.off_bar + 8 * (2 * kPwStages + 8) + 16 + 1024;   // barriers, TMEM slot, slack
+  return L;
+}
+
+__global__ void __launch_bounds__(kPwThreads, 1)
+    proj_pre_ws_kernel(const __grid_constant__ CUtensorMap tmX,
+                       const __grid_constant__ CUtensorMap tmWq,
+                       const __grid_constant__ CUtensorMap tmWkv, int E, int n_rb,
+                       const __grid_constant__ PreAttnArgs<bf16> a) {
+  pdl_enter();
+  constexpr int D = kPpD;
+  constexpr uint32_t kRowBytes = kPpRow;                // 64-byte rows, 64B swizzle
+  constexpr uint32_t kSwz = kSwizzle64B;
+  constexpr uint32_t kSbo = 8 * kRowBytes;
+  constexpr int NCH = D / 8;                            // 16-byte chunks per row
+  constexpr int Q4 = D / 4;                             // rotary pairs per epilogue thread
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int G = a.G, S = a.S, K = a.K;
+  const PwLayout L = pw_layout(G);
+  const int NH = G + 1, QC = G * D, NZ = static_cast<int>(L.nz);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_tiles = n_rb * a.Hkv * a.B;
+  uint8_t* z = smem + L.off_z;                           // slot h: z + h zh_bytes
+  uint2* ws = reinterpret_cast<uint2*>(smem + L.off_ws);   // taps of a channel: 4 bf16
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.off_bar);   // [kPwStages]
+  uint64_t* empty = full + kPwStages;                                // [kPwStages]
+  uint64_t* acc_full = empty + kPwStages;                            // [2]
+  uint64_t* acc_empty = acc_full + 2;                                // [2], 256 arrivals
+  uint64_t* mma_done = acc_empty + 2;                                // [2] mix MMAs
+  uint64_t* drain = mma_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  __shared__ int abort_flag, n_issued;
+  const int nkb = (E + kPpBK - 1) / kPpBK;
+  // tile t: sequence b, row block rb (positions [125 rb, 125 rb + 125)), kv group g
+  auto tile_of = [&](int t, int& b, int& rb, int& g) {
+    g = t % a.Hkv;
+    rb = (t / a.Hkv) % n_rb;
+    b = t / (a.Hkv * n_rb);
+  };
+
+  if (tid == 0) {
+    for (int s = 0; s < kPwStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 256);
+      mbar_init(&mma_done[i], 1);
+    }
+    mbar_init(drain, 2);   // one commit from each MMA issuer (GEMM, mix)
+    abort_flag = 0;
+    n_issued = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);   // accumulators at 0 and NZ, the mix accumulators at 2 NZ
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t col_mix = 2 * static_cast<uint32_t>(NZ);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmX);
+      prefetch_tensormap(&tmWq);
+      prefetch_tensormap(&tmWkv);
+      int kg = 0;   // k-blocks issued so far (the ring runs on across tiles)
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+        int b, rb, g;
+        tile_of(t, b, rb, g);
+        const int rq = g * QC, rk = a.Hq * D + g * D, rv = (a.Hq + a.Hkv) * D + g * D;
+        for (int kb = 0; kb < nkb; ++kb, ++kg) {
+          const int s = kg % kPwStages;
+          if (!mbar_wait(&empty[s], ((kg / kPwStages) & 1) ^ 1, &abort_flag, a.dev_err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], L.a_bytes + L.b_bytes);
+          uint8_t* sa = smem + s * L.stage_bytes;
+          uint8_t* sb = sa + L.a_bytes;
+          tma_load_3d(sa, &tmX, &full[s], kb * kPpBK, rb * kPpOut - kPpHalo, b);
+          tma_load_2d(sb, &tmWq, &full[s], kb * kPpBK, rq);
+          tma_load_2d(sb + QC * 128, &tmWkv, &full[s], kb * kPpBK, rk);
+          tma_load_2d(sb + (QC + D) * 128, &tmWkv, &full[s], kb * kPpBK, rv);
+          n_issued = kg + 1;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ GEMM MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc_bf16(kPpM, NZ, false);
+      int kg = 0, i = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++i) {
+        const int buf = i & 1;
+        // the head workers have read this accumulator's previous tile back
+        if (!mbar_wait(&acc_empty[buf], ((i >> 1) & 1) ^ 1, &abort_flag, a.dev_err)) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + buf * NZ;
+        for (int kb = 0; kb < nkb; ++kb, ++kg) {
+          const int s = kg % kPwStages;
+          if (!mbar_wait(&full[s], (kg / kPwStages) & 1, &abort_flag, a.dev_err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_addr(smem + s * L.stage_bytes);
+          const uint32_t b_base = a_base + L.a_bytes;
+#pragma unroll
+          for (int k = 0; k < kPpBK / 16; ++k) {
+            const uint64_t ad = make_smem_desc(a_base + k * 32, 16, 1024, kSwizzle128B);
+            const uint64_t bd = make_smem_desc(b_base + k * 32, 16, 1024, kSwizzle128B);
+            mma_ss(acc, ad, bd, idesc, (kb | k) != 0);
+          }
+          mma_commit(&empty[s]);
+        }
+        if (ok) mma_commit(&acc_full[buf]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ head workers
+    const int ptid = tid - 64;                 // 0..255
+    const int wq = warp & 3;                   // TMEM lane quadrant of this warp
+    const int r = wq * 32 + lane;              // row == TMEM lane (position t0 + r)
+    const int part = (warp - 2) >> 2;          // conv chunks j = part (mod 2); pairs of half `part`
+    const bool row_out = r < kPpOut;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const uint32_t u_hi = smem_addr(smem + L.off_u);
+    const uint32_t u_lo = u_hi + L.u_bytes;
+    const uint32_t w_base = smem_addr(smem + L.off_w);
+    const uint32_t idesc = make_idesc_bf16(kPpM, D, false);
+    auto zchunk = [&](int h, int rr, int c) -> const uint4* {
+      return reinterpret_cast<const uint4*>(z + h * L.zh_bytes + swz_offset(rr, c * 16, kRowBytes));
+    };
+    bool ok = true;
+    int mix_base = 0;                           // mix MMAs issued by this CTA before this tile
+    for (int t = blockIdx.x, i = 0; ok && t < n_tiles; t += gridDim.x, ++i) {
+      int b, rb, g;
+      tile_of(t, b, rb, g);
+      const int t0 = rb * kPpOut, tp = t0 + r;
+      const int buf = i & 1;
+      // (every worker is done with the previous tile's staged rows, U and W:
+      // the barrier that ends each tile)
+      // mix weights W_h [d_out][d_in] of group g into the K-major 64B-swizzled
+      // B layout (the previous tile's mix MMAs have completed), and the taps
+      for (int idx = ptid; idx < NH * D * NCH; idx += 256) {
+        const int h = idx / (D * NCH), row = (idx / NCH) % D, c = idx % NCH;
+        const bf16* src = h < G ? a.wq_chan + (static_cast<int64_t>(g * G + h) * D + row) * D
+                                : a.wk_chan + (static_cast<int64_t>(g) * D + row) * D;
+        *reinterpret_cast<uint4*>(smem + L.off_w + h * L.w_bytes + swz_offset(row, c * 16, kRowBytes)) =
+            *reinterpret_cast<const uint4*>(src + c * 8);
+      }
+      for (int hc = ptid; hc < NH * D; hc += 256) {
+        const int h = hc / D, ch = hc % D;
+        const bf16* src = h < G ? a.wq_seq + (static_cast<int64_t>(g * G + h) * D + ch) * K
+                                : a.wk_seq + (static_cast<int64_t>(g) * D + ch) * K;
+        uint16_t w4[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) w4[k] = k < K ? __bfloat16_as_ushort(src[k]) : static_cast<uint16_t>(0);
+        ws[hc] = make_uint2(w4[0] | (static_cast<uint32_t>(w4[1]) << 16),
+                            w4[2] | (static_cast<uint32_t>(w4[3]) << 16));
+      }
+      // rotary (cos, sin) of this thread's pairs at position t0 + r (angle
+      // reduced modulo one turn exactly in 64-bit fixed point)
+      float rc[Q4], rs[Q4];
+      {
+        const int ip = part * Q4;
+#pragma unroll
+        for (int e = 0; e < Q4; ++e) {
+          rc[e] = 1.f;
+          rs[e] = 0.f;
+          if (a.rope_on) {
+            const uint64_t ph = static_cast<uint64_t>(tp) * a.rope_frac[ip + e];
+            const float f = static_cast<float>(static_cast<int64_t>(ph)) * 5.42101086242752217e-20f;
+            __sincosf(6.28318530717958648f * f, &rs[e], &rc[e]);
+          }
+        }
+      }
+      // the tile's accumulator -> staged bf16 head rows; then it is free again
+      ok = mbar_wait(&acc_full[buf], (i >> 1) & 1, &abort_flag, a.dev_err);
+      tc_fence_after();
+      {
+        const int n_slots = G + 2, half_slots = (n_slots + 1) / 2;
+        const int s_lo = part == 0 ? 0 : half_slots, s_hi = part == 0 ? half_slots : n_slots;
+        for (int sl = s_lo; sl < s_hi; ++sl) {
+          uint32_t v[32];
+          tmem_ld32(trow + buf * NZ + sl * D, v);
+          tmem_wait_ld();
+          if (ok) {
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+              uint4 pk;
+              pk.x = pack2(__uint_as_float(v[c * 8 + 0]), __uint_as_float(v[c * 8 + 1]));
+              pk.y = pack2(__uint_as_float(v[c * 8 + 2]), __uint_as_float(v[c * 8 + 3]));
+              pk.z = pack2(__uint_as_float(v[c * 8 + 4]), __uint_as_float(v[c * 8 + 5]));
+              pk.w = pack2(__uint_as_float(v[c * 8 + 6]), __uint_as_float(v[c * 8 + 7]));
+              *reinterpret_cast<uint4*>(z + sl * L.zh_bytes + swz_offset(r, c * 16, kRowBytes)) = pk;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
+      fence_proxy_async_smem();   // W is read by the tensor core
+      // one answer for all 256 workers (a worker leaving the loop alone would
+      // leave the others at a named barrier)
+      ok = !named_barrier_or(1, 256, !ok || abort_flag);
+      if (!ok) break;
+
+      // per head, as the one-tile kernel; mix MMA m (m = mix_base + head) goes
+      // into accumulator m & 1 and completes on mma_done[m & 1]
+      auto conv_part = [&](int hh, auto part_c) {
+        constexpr int P = decltype(part_c)::value;
+#pragma unroll
+        for (int j = P; j < NCH; j += 2) {
+          uint4 hi4 = make_uint4(0, 0, 0, 0), lo4 = make_uint4(0, 0, 0, 0);
+          if (row_out) {
+            const uint4* tw = reinterpret_cast<const uint4*>(ws + hh * D + j * 8);
+            uint4 t4[4], zz[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) t4[q] = tw[q];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) zz[k] = *zchunk(hh, r + kPpHalo - k, j);
+            float acc[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const uint4& tq = t4[e >> 1];
+              uint16_t w[4], zv[4];
+              halves((e & 1) ? tq.z : tq.x, w[0], w[1]);
+              halves((e & 1) ? tq.w : tq.y, w[2], w[3]);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const uint32_t* zw = reinterpret_cast<const uint32_t*>(&zz[k]);
+                uint16_t lo, hi;
+                halves(zw[e >> 1], lo, hi);
+                zv[k] = (e & 1) ? hi : lo;
+              }
+              float s = fma_bf16(zv[0], w[0], 0.f);
+#pragma unroll
+              for (int k = 1; k < 4; ++k) s = fma_bf16(zv[k], w[k], s);
+              acc[e] = s;
+            }
+            uint32_t* hp = reinterpret_cast<uint32_t*>(&hi4);
+            uint32_t* lp = reinterpret_cast<uint32_t*>(&lo4);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              hp[e] = pack2(acc[2 * e], acc[2 * e + 1]);
+              uint16_t h0, h1;
+              halves(hp[e], h0, h1);
+              lp[e] = pack2(fma_bf16(h0, kBf16MinusOne, acc[2 * e]),
+                            fma_bf16(h1, kBf16MinusOne, acc[2 * e + 1]));
+            }
+          }
+          const uint32_t off = swz_offset(r, j * 16, kRowBytes);
+          *reinterpret_cast<uint4*>(smem + L.off_u + off) = hi4;
+          *reinterpret_cast<uint4*>(smem + L.off_u + L.u_bytes + off) = lo4;
+        }
+      };
+      auto issue_mma = [&](int hh, int m) {
+        const uint32_t dt = tmem + col_mix + (m & 1) * D;
+        const uint32_t wb = w_base + hh * L.w_bytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(dt, make_smem_desc(u_hi + kk * 32, 16, kSbo, kSwz),
+                 make_smem_desc(wb + kk * 32, 16, kSbo, kSwz), idesc, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(dt, make_smem_desc(u_lo + kk * 32, 16, kSbo, kSwz),
+                 make_smem_desc(wb + kk * 32, 16, kSbo, kSwz), idesc, 1u);
+        mma_commit(&mma_done[m & 1]);
+      };
+
+      auto epilogue = [&](int hh, int m) {
+        const uint32_t col = col_mix + (m & 1) * D + part * Q4;
+        uint32_t ya[Q4], yb[Q4];               // channels part*Q4 + e and D/2 + part*Q4 + e
+        tmem_ld8(trow + col, ya);
+        tmem_ld8(trow + col + D / 2, yb);
+        tmem_wait_ld();
+        if (tp >= S || !row_out) return;
+        const int i0 = part * Q4;
+        float lo[Q4], hi[Q4];
+#pragma unroll
+        for (int e = 0; e < Q4; ++e) {
+          lo[e] = __uint_as_float(ya[e]);
+          hi[e] = __uint_as_float(yb[e]);
+        }
+        const int rr = r + kPpHalo;            // this position's staged row
+        if (a.qk_mean == 2) {
+          auto self_mean = [&](float (&y)[Q4], int c0) {
+            const uint4 ow = *zchunk(hh, rr, c0 / 8);
+            const uint32_t* op = reinterpret_cast<const uint32_t*>(&ow);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              uint16_t o0, o1;
+              halves(op[e], o0, o1);
+              y[2 * e] = fma_bf16(o0, kBf16Half, 0.5f * y[2 * e]);
+              y[2 * e + 1] = fma_bf16(o1, kBf16Half, 0.5f * y[2 * e + 1]);
+            }
+          };
+          self_mean(lo, i0);
+          self_mean(hi, i0 + D / 2);
+        } else if (a.qk_mean) {
+          const bool is_q = hh < G;
+          auto add_mean = [&](float (&y)[Q4], int c0) {
+            const uint4 kw = *zchunk(G, rr, c0 / 8);
+            const uint32_t* kp = reinterpret_cast<const uint32_t*>(&kw);
+            if (is_q) {
+              const uint4 qw = *zchunk(hh, rr, c0 / 8);
+              const uint32_t* qp = reinterpret_cast<const uint32_t*>(&qw);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                uint16_t q0, q1, k0, k1;
+                halves(qp[e], q0, q1);
+                halves(kp[e], k0, k1);
+                y[2 * e] = fma_bf16(k0, kBf16Half, fma_bf16(q0, kBf16Half, y[2 * e]));
+                y[2 * e + 1] = fma_bf16(k1, kBf16Half, fma_bf16(q1, kBf16Half, y[2 * e + 1]));
+              }
+            } else {
+              float sq[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) sq[e] = 0.f;
+              for (int hl = 0; hl < G; ++hl) {
+                const uint4 qw = *zchunk(hl, rr, c0 / 8);
+                const uint32_t* qp = reinterpret_cast<const uint32_t*>(&qw);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  uint16_t q0, q1;
+                  halves(qp[e], q0, q1);
+                  sq[2 * e] = add_bf16(q0, sq[2 * e]);
+                  sq[2 * e + 1] = add_bf16(q1, sq[2 * e + 1]);
+                }
+              }
+              const float hg = 0.5f / static_cast<float>(G);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                uint16_t k0, k1;
+                halves(kp[e], k0, k1);
+                y[2 * e] = fma_bf16(k0, kBf16Half, fmaf(sq[2 * e], hg, y[2 * e]));
+                y[2 * e + 1] = fma_bf16(k1, kBf16Half, fmaf(sq[2 * e + 1], hg, y[2 * e + 1]));
+              }
+            }
+          };
+          add_mean(lo, i0);
+          add_mean(hi, i0 + D / 2);
+        }
+        if (a.rope_on) {
+#pragma unroll
+          for (int e = 0; e < Q4; ++e) {
+            const float x0 = lo[e], x1 = hi[e];
+            lo[e] = x0 * rc[e] - x1 * rs[e];
+            hi[e] = x0 * rs[e] + x1 * rc[e];
+          }
+        }
+        bf16* dst = hh < G ? a.q_out + ((static_cast<int64_t>(b) * S + tp) * a.Hq + g * G + hh) * D
+                           : a.k_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + tp) * D;
+        uint4 pl, ph;
+        pl.x = pack2(lo[0], lo[1]);
+        pl.y = pack2(lo[2], lo[3]);
+        pl.z = pack2(lo[4], lo[5]);
+        pl.w = pack2(lo[6], lo[7]);
+        ph.x = pack2(hi[0], hi[1]);
+        ph.y = pack2(hi[2], hi[3]);
+        ph.z = pack2(hi[4], hi[5]);
+        ph.w = pack2(hi[6], hi[7]);
+        *reinterpret_cast<uint4*>(dst + i0) = pl;
+        *reinterpret_cast<uint4*>(dst + D / 2 + i0) = ph;
+      };
+
+      for (int hh = 0; hh < NH; ++hh) {
+        const int m = mix_base + hh;
+        if (hh > 0) {
+          // MMA m - 1 complete: U may be overwritten, accumulator (m - 1) & 1 is final
+          ok = ok && mbar_wait(&mma_done[(m - 1) & 1], ((m - 1) >> 1) & 1, &abort_flag, a.dev_err);
+          tc_fence_after();
+        }
+        if (ok) {
+          if (part == 0)
+            conv_part(hh, std::integral_constant<int, 0>{});
+          else
+            conv_part(hh, std::integral_constant<int, 1>{});
+        }
+        fence_proxy_async_smem();   // U is read by the tensor core
+        tc_fence_before();
+        ok = !named_barrier_or(1, 256, !ok || abort_flag);
+        tc_fence_after();
+        if (ok && ptid == 0) issue_mma(hh, m);
+        __syncwarp();
+        if (ok && hh > 0) epilogue(hh - 1, m - 1);
+      }
+      const int m_last = mix_base + NH - 1;
+      ok = ok && mbar_wait(&mma_done[m_last & 1], (m_last >> 1) & 1, &abort_flag, a.dev_err);
+      ok = __all_sync(0xffffffffu, ok);   // the epilogue's TMEM loads are warp-collective
+      tc_fence_after();
+      if (ok) epilogue(NH - 1, m_last);
+      mix_base += NH;
+
+      // value-shift rows (the whole-head reading: every channel from t - 1
+      // when the group's kv head is one of the last floor(Hkv / 2))
+      const bool shift_head = a.value_shift == 2 && g >= a.Hkv - a.Hkv / 2;
+      for (int idx = ptid; idx < kPpOut * NCH; idx += 256) {
+        const int tl = idx / NCH, c = idx % NCH;
+        const int tv = t0 + tl;
+        if (tv >= S) continue;
+        const bool prev = (a.value_shift == 1 && c * 8 >= D / 2) || shift_head;
+        const uint4 v = *zchunk(G + 1, tl + kPpHalo - (prev ? 1 : 0), c);
+        *reinterpret_cast<uint4*>(a.v_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + tv) *
+                                                D + c * 8) = v;
+      }
+      // decode state, from the tile holding position S - 1
+      if (a.len != nullptr && t0 <= S - 1 && S - 1 < t0 + kPpOut) {
+        const int KH = K - 1, Hq = a.Hq, Hkv = a.Hkv, qcol0 = g * QC;
+        for (int rr = 0; rr < KH; ++rr) {
+          const int srow = S - KH + rr - t0 + kPpHalo;
+          for (int c = ptid; c < QC + D; c += 256) {
+            const int h = c / D, ch = c % D;
+            const bf16 v = reinterpret_cast<const bf16*>(zchunk(h, srow, ch / 8))[ch % 8];
+            if (c < QC)
+              a.hist_q[(static_cast<int64_t>(b) * KH + rr) * Hq * D + qcol0 + c] = v;
+            else
+              a.hist_k[(static_cast<int64_t>(b) * KH + rr) * Hkv * D + g * D + (c - QC)] = v;
+          }
+        }
+        if (a.v_prev)
+          for (int i2 = ptid; i2 < D; i2 += 256)
+            a.v_prev[static_cast<int64_t>(b) * Hkv * D + g * D + i2] =
+                reinterpret_cast<const bf16*>(zchunk(G + 1, S - 1 - t0 + kPpHalo, i2 / 8))[i2 % 8];
+        if (g == 0 && ptid == 0) a.len[b] = S;
+      }
+      // end of the tile: the staged rows are free, and one answer for all workers
+      ok = !named_barrier_or(1, 256, !ok || abort_flag);
+    }
+  }
+
+  if (abort_flag) {
+    // Do not release TMEM while an MMA might still write it (the GEMM issuer's
+    // and the mix issuer's own MMAs), nor leave while the ring's last loads
+    // are in flight (bounded waits).
+    if ((warp == 1 && lane == 0) || tid == 64) {
+      mma_commit(drain);
+      const long long c0 = clock64();
+      while (!mbar_try_wait(drain, 0) && clock64() - c0 < kWaitLimitCycles) {
+      }
+    }
+    if (tid == 0) {
+      const int n = n_issued;
+      for (int kg = n > kPwStages ? n - kPwStages : 0; kg < n; ++kg) {
+        const long long c2 = clock64();
+        while (!mbar_try_wait(&full[kg % kPwStages], (kg / kPwStages) & 1) &&
+               clock64() - c2 < kWaitLimitCycles) {
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // kPpStages = 3 (one CTA per SM) when the grid is at most one wave; 2 (about
 // 97 KB of shared memory at G = 4, so two CTAs share an SM and one's GEMM runs
 // while the other works on its heads) otherwise.
@@ -152,7 +653,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     mbar_init(wl_bar, 1);
     mbar_init(&mma_done[0], 1);
     mbar_init(&mma_done[1], 1);
-    mbar_init(drain, 1);
+    mbar_init(drain, 2);   // one commit from each MMA issuer (GEMM: thread 32, mix: thread 0)
     abort_flag = 0;
     n_issued = 0;
     fence_barrier_init();
@@ -479,13 +980,13 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    ok = ok && !abort_flag;
+    ok = __all_sync(0xffffffffu, ok && !abort_flag);   // warp-uniform for the TMEM loads
     if (ok && tid == 0) issue_mma(hh);
     __syncwarp();
     if (ok && hh > 0) epilogue(hh - 1);
   }
   ok = ok && mbar_wait(&mma_done[(NH - 1) & 1], ((NH - 1) >> 1) & 1, &abort_flag, a.dev_err);
-  __syncwarp();
+  ok = __all_sync(0xffffffffu, ok);   // the epilogue's TMEM loads are warp-collective
   tc_fence_after();
   if (ok) epilogue(NH - 1);
 
@@ -526,13 +1027,16 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     if (g == 0 && tid == 0) a.len[b] = S;
   }
 
-  if (abort_flag && tid == 0) {
-    // Do not release TMEM while an MMA might still write it, nor leave while
-    // copies into this CTA's shared memory are in flight (bounded waits).
+  if (abort_flag && (tid == 0 || tid == 32)) {
+    // Do not release TMEM while an MMA might still write it (each issuer
+    // commits its own), nor leave while copies into this CTA's shared memory
+    // are in flight (bounded waits).
     mma_commit(drain);
     const long long c0 = clock64();
     while (!mbar_try_wait(drain, 0) && clock64() - c0 < kWaitLimitCycles) {
     }
+  }
+  if (abort_flag && tid == 0) {
     const long long c1 = clock64();
     while (!mbar_try_wait(wl_bar, 0) && clock64() - c1 < kWaitLimitCycles) {
     }
@@ -611,6 +1115,20 @@ cudaError_t launch_proj_pre_tc(const bf16* x, const bf16* W, int E, const PreAtt
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (2 * (a.G + 2) * D + 2 * D <= 512 && pw_layout(a.G).bytes <= 227 * 1024) {
+    // persistent: two GEMM accumulators and the two mix accumulators fit in TMEM
+    const int n_rb = static_cast<int>(grid.x);
+    const int n_tiles = n_rb * a.Hkv * a.B;
+    const int pgrid = n_tiles < sms ? n_tiles : sms;
+    const PwLayout P = pw_layout(a.G);
+    cudaError_t e = allow_smem(reinterpret_cast<const void*>(proj_pre_ws_kernel),
+                               static_cast<int>(P.bytes));
+    if (e != cudaSuccess) return e;
+    const cudaError_t el = launch_pdl(proj_pre_ws_kernel, dim3(pgrid), dim3(kPwThreads), P.bytes,
+                                      stream, tmX, tmWq, tmWkv, E, n_rb, a);
+    count_launches(1);
+    return el != cudaSuccess ? el : cudaGetLastError();
+  }
   const bool one_wave = static_cast<int64_t>(grid.x) * grid.y * grid.z <= sms;
   auto kernel = one_wave ? proj_pre_tc_kernel<3> : proj_pre_tc_kernel<2>;
   const PpLayout L = pp_layout(a.G, one_wave ? 3 : 2);
