@@ -49,6 +49,21 @@ cudaError_t allow_smem(const void* func, int bytes) {
   return e;
 }
 
+int sm_count() {
+  static std::mutex mu;
+  static std::map<int, int> counts;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = counts.find(dev);
+  if (it != counts.end()) return it->second;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  counts[dev] = n;
+  return n;
+}
+
 // Last CUDA error met by an entry point on this thread.
 static thread_local char t_last_error[256] = "no error";
 static ccgqa_status cuda_fail(cudaError_t e) {

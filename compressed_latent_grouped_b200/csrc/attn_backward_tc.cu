@@ -801,7 +801,8 @@ cudaError_t launch_bwd_tc(const AttnBwdTcArgs& a, cudaStream_t stream) {
       longest = std::max<int64_t>(longest, halves_all - u_first);
     }
     work *= BH;
-    int64_t L = (work + 6 * 148 - 1) / (6 * 148);
+    const int64_t waves6 = 6 * static_cast<int64_t>(sm_count());
+    int64_t L = (work + waves6 - 1) / waves6;
     if (L < 16) L = 16;
     if (L > longest) L = longest;
     const int max_chunks = static_cast<int>((longest + L - 1) / L);

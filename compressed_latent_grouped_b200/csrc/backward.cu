@@ -505,7 +505,7 @@ cudaError_t gemm(GemmArgs g, int batch, cudaStream_t st) {
     // few output tiles over a long K (the weight gradients): split K so that
     // about two waves of CTAs run, each range at least 32 K blocks long; the
     // caller zeroed C, so the atomic sums start from zero
-    int ks = (2 * 148 + tiles - 1) / tiles;
+    int ks = (2 * sm_count() + tiles - 1) / tiles;
     const int max_ks = (g.K + 32 * kGBK - 1) / (32 * kGBK);
     if (ks > max_ks) ks = max_ks;
     g.ksplit = ks < 1 ? 1 : ks;

@@ -38,6 +38,11 @@ bool stream_allowed(cudaStream_t st);
 // (the attribute is per device, the check costs a lock and a map lookup).
 cudaError_t allow_smem(const void* func, int bytes);
 
+// Streaming multiprocessors of the current device (looked up once per device;
+// 148, a B200's count, when no device answers, e.g. for a workspace-size query
+// on a machine without one).
+int sm_count();
+
 // Programmatic dependent launch.  A kernel launched by launch_pdl may be
 // scheduled while the kernel before it on the stream is still finishing (once
 // every CTA of that kernel has run pdl_trigger() or exited).  Every such kernel

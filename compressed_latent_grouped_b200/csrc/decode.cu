@@ -51,7 +51,8 @@ static int decode_proj_e_len(int E, int e_splits) {
 
 void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int es,
                  int* e_splits, int* splits, int* chunk) {
-  const int target = 2 * 148;
+  const int sms = sm_count();
+  const int target = 2 * sms;
   if (has_proj && decode_use_gemv(B, E, es)) {
     *e_splits = 1;   // one weight-streaming pass, no partials to sum
   } else if (has_proj && decode_use_proj_tc(E, es)) {
@@ -67,13 +68,13 @@ void decode_plan(int B, int Hkv, int E, int N, int64_t cap, bool has_proj, int e
     *e_splits = 0;
   }
   // Splits of whole 128-key chunks.  The CTAs of one launch should fill a whole
-  // number of waves of the resident slots (148 SMs x 2 CTAs), each CTA
+  // number of waves of the resident slots (SMs x 2 CTAs), each CTA
   // streaming at least ~1024 keys so its start-up cost stays small, and never
   // fewer than 4 chunks (512 keys) when the cache has that many: measured on
   // B200, a launch of a few hundred 2-chunk CTAs spends longer starting them
   // (about 37 per microsecond) and merging their partials than streaming keys.
   const int64_t bh = static_cast<int64_t>(B) * Hkv;
-  const int64_t slots = 148 * 2;
+  const int64_t slots = static_cast<int64_t>(sms) * 2;
   const int64_t max_sp = (cap + 127) / 128;
   int64_t best_sp = 1;
   double best = -1.0;

@@ -308,9 +308,7 @@ cudaError_t launch_tc_gemm(const bf16* A, const bf16* W, TC* C, int M, int N, in
   cudaError_t e = allow_smem(reinterpret_cast<const void*>(proj_gemm_bf16_kernel<TC>),
                              static_cast<int>(gemm_smem<TC>()));
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = sm_count();
   const int tiles = ((N + kBN - 1) / kBN) * ((M + kBM - 1) / kBM);
   const int grid = tiles < sms ? tiles : sms;   // one persistent CTA per SM
   const cudaError_t el = launch_pdl(proj_gemm_bf16_kernel<TC>, dim3(grid), dim3(kGemmThreads),

@@ -1112,9 +1112,7 @@ cudaError_t launch_proj_pre_tc(const bf16* x, const bf16* W, int E, const PreAtt
       return cudaErrorInvalidValue;
   }
   dim3 grid((a.S + kPpOut - 1) / kPpOut, a.Hkv, a.B);
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = sm_count();
   if (2 * (a.G + 2) * D + 2 * D <= 512 && pw_layout(a.G).bytes <= 227 * 1024) {
     // persistent: two GEMM accumulators and the two mix accumulators fit in TMEM
     const int n_rb = static_cast<int>(grid.x);
