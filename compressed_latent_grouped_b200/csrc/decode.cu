@@ -450,18 +450,6 @@ cudaError_t launch_decode_proj_tc(const bf16* x, const bf16* W, float* part, int
 }
 
 // ----------------------------------------------------------------- pre-step
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
-               "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit_group() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all_groups() {
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-}
 
 // Shared memory of the pre-step (byte offsets, each 16-byte aligned): fp32
 // rows (current pre-conv row zc[AC], conv out u[HC], mix out y[HC], taps

@@ -103,7 +103,8 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 }
 
 // ------------------------------------------------------------------ persistent
-// The persistent, warp-specialised form (G <= 5): one CTA per SM walks tiles
+// The persistent, warp-specialised form (G <= 4, where its buffers fit in shared
+// memory): one CTA per SM walks tiles
 // c, c + grid, ...; warp 0 streams the GEMM operands through a ring that runs
 // on across tiles, warp 1 accumulates tile i into one of two TMEM accumulators
 // (2 (G + 2) d columns, then the two mix accumulators), and warps 2-9 (256
@@ -114,11 +115,14 @@ constexpr int kPwThreads = 64 + 256;
 
 struct PwLayout {
   uint32_t nz, a_bytes, b_bytes, stage_bytes, zh_bytes, u_bytes, w_bytes;
-  uint32_t off_z, off_u, off_w, off_ws, off_bar, bytes;
+  uint32_t wset_bytes, rt_bytes;   // one buffer of mix weights, of raw taps
+  uint32_t off_z, off_u, off_w, off_rt, off_ws, off_bar, bytes;
 };
 
-// ring | staged head rows (G + 2 slots of 128 x 64 B) | U_hi, U_lo | mix
-// weights (G + 1 tiles of 32 x 64 B) | taps [(G + 1) d][4] bf16 | barriers
+// ring | staged head rows (G + 2 slots of 128 x 64 B) | U_hi, U_lo | two
+// buffers of mix weights (G + 1 tiles of 32 x 64 B each; the next tile's are
+// copied in while this tile's are in use) | two buffers of raw taps
+// [(G + 1) d][K] | packed taps [(G + 1) d][4] bf16 | barriers
 __host__ __device__ inline PwLayout pw_layout(int G) {
   PwLayout L;
   L.nz = static_cast<uint32_t>(G + 2) * kPpD;
@@ -128,10 +132,13 @@ __host__ __device__ inline PwLayout pw_layout(int G) {
   L.zh_bytes = kPpM * kPpRow;
   L.u_bytes = kPpM * kPpRow;
   L.w_bytes = kPpD * kPpRow;
+  L.wset_bytes = static_cast<uint32_t>(G + 1) * L.w_bytes;
+  L.rt_bytes = static_cast<uint32_t>(G + 1) * kPpD * 4 * 2;   // room for K = 4
   L.off_z = kPwStages * L.stage_bytes;
   L.off_u = L.off_z + static_cast<uint32_t>(G + 2) * L.zh_bytes;
   L.off_w = L.off_u + 2 * L.u_bytes;
-  L.off_ws = L.off_w + static_cast<uint32_t>(G + 1) * L.w_bytes;
+  L.off_rt = L.off_w + 2 * L.wset_bytes;
+  L.off_ws = L.off_rt + 2 * L.rt_bytes;
   L.off_bar = L.off_ws + static_cast<uint32_t>(G + 1) * kPpD * 8;
   L.bytes = L.off_bar + 8 * (2 * kPwStages + 8) + 16 + 1024;   // barriers, TMEM slot, slack
   return L;
@@ -276,31 +283,45 @@ __global__ void __launch_bounds__(kPwThreads, 1)
     auto zchunk = [&](int h, int rr, int c) -> const uint4* {
       return reinterpret_cast<const uint4*>(z + h * L.zh_bytes + swz_offset(rr, c * 16, kRowBytes));
     };
+    // mix weights W_h [d_out][d_in] of group g into weight buffer wb (the
+    // K-major 64B-swizzled B layout) and the group's raw taps into tap buffer
+    // wb, by 16-byte asynchronous copies (all four sources 16-byte aligned)
+    auto prefetch_weights = [&](int g, int wb) {
+      uint8_t* wdst = smem + L.off_w + wb * L.wset_bytes;
+      for (int idx = ptid; idx < NH * D * NCH; idx += 256) {
+        const int h = idx / (D * NCH), row = (idx / NCH) % D, c = idx % NCH;
+        const bf16* src = h < G ? a.wq_chan + (static_cast<int64_t>(g * G + h) * D + row) * D
+                                : a.wk_chan + (static_cast<int64_t>(g) * D + row) * D;
+        cp_async16(wdst + h * L.w_bytes + swz_offset(row, c * 16, kRowBytes), src + c * 8);
+      }
+      uint8_t* tdst = smem + L.off_rt + wb * L.rt_bytes;
+      const int qb = G * D * K * 2, kbytes = D * K * 2;   // multiples of 64
+      const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(a.wq_seq + static_cast<int64_t>(g) * G * D * K);
+      const uint8_t* ksrc = reinterpret_cast<const uint8_t*>(a.wk_seq + static_cast<int64_t>(g) * D * K);
+      for (int o = ptid * 16; o < qb + kbytes; o += 256 * 16)
+        cp_async16(tdst + o, o < qb ? qsrc + o : ksrc + (o - qb));
+      cp_async_commit_group();
+    };
     bool ok = true;
     int mix_base = 0;                           // mix MMAs issued by this CTA before this tile
+    if (blockIdx.x < n_tiles) {
+      prefetch_weights(static_cast<int>(blockIdx.x) % a.Hkv, 0);
+      cp_async_wait_all_groups();
+      named_barrier_sync(1, 256);
+    }
     for (int t = blockIdx.x, i = 0; ok && t < n_tiles; t += gridDim.x, ++i) {
       int b, rb, g;
       tile_of(t, b, rb, g);
       const int t0 = rb * kPpOut, tp = t0 + r;
       const int buf = i & 1;
-      // (every worker is done with the previous tile's staged rows, U and W:
-      // the barrier that ends each tile)
-      // mix weights W_h [d_out][d_in] of group g into the K-major 64B-swizzled
-      // B layout (the previous tile's mix MMAs have completed), and the taps
-      for (int idx = ptid; idx < NH * D * NCH; idx += 256) {
-        const int h = idx / (D * NCH), row = (idx / NCH) % D, c = idx % NCH;
-        const bf16* src = h < G ? a.wq_chan + (static_cast<int64_t>(g * G + h) * D + row) * D
-                                : a.wk_chan + (static_cast<int64_t>(g) * D + row) * D;
-        *reinterpret_cast<uint4*>(smem + L.off_w + h * L.w_bytes + swz_offset(row, c * 16, kRowBytes)) =
-            *reinterpret_cast<const uint4*>(src + c * 8);
-      }
+      // (every worker is done with the previous tile's staged rows, U and taps,
+      // and this tile's weights and raw taps have landed: the barrier that ends
+      // each tile)  Taps as bf16 [channel][4], zero past K.
+      const bf16* rt = reinterpret_cast<const bf16*>(smem + L.off_rt + buf * L.rt_bytes);
       for (int hc = ptid; hc < NH * D; hc += 256) {
-        const int h = hc / D, ch = hc % D;
-        const bf16* src = h < G ? a.wq_seq + (static_cast<int64_t>(g * G + h) * D + ch) * K
-                                : a.wk_seq + (static_cast<int64_t>(g) * D + ch) * K;
         uint16_t w4[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) w4[k] = k < K ? __bfloat16_as_ushort(src[k]) : static_cast<uint16_t>(0);
+        for (int k = 0; k < 4; ++k) w4[k] = k < K ? __bfloat16_as_ushort(rt[hc * K + k]) : static_cast<uint16_t>(0);
         ws[hc] = make_uint2(w4[0] | (static_cast<uint32_t>(w4[1]) << 16),
                             w4[2] | (static_cast<uint32_t>(w4[3]) << 16));
       }
@@ -345,7 +366,11 @@ __global__ void __launch_bounds__(kPwThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
-      fence_proxy_async_smem();   // W is read by the tensor core
+      // the next tile's weights into the other buffers (their last reader, the
+      // tile before this one, is done), landing while this tile's heads run
+      if (t + static_cast<int>(gridDim.x) < n_tiles)
+        prefetch_weights((t + static_cast<int>(gridDim.x)) % a.Hkv, buf ^ 1);
+      fence_proxy_async_smem();   // W (copied in at the end of the previous tile) is read by the tensor core
       // one answer for all 256 workers (a worker leaving the loop alone would
       // leave the others at a named barrier)
       ok = !named_barrier_or(1, 256, !ok || abort_flag);
@@ -402,7 +427,7 @@ __global__ void __launch_bounds__(kPwThreads, 1)
       };
       auto issue_mma = [&](int hh, int m) {
         const uint32_t dt = tmem + col_mix + (m & 1) * D;
-        const uint32_t wb = w_base + hh * L.w_bytes;
+        const uint32_t wb = w_base + buf * L.wset_bytes + hh * L.w_bytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(dt, make_smem_desc(u_hi + kk * 32, 16, kSbo, kSwz),
@@ -570,9 +595,12 @@ __global__ void __launch_bounds__(kPwThreads, 1)
                 reinterpret_cast<const bf16*>(zchunk(G + 1, S - 1 - t0 + kPpHalo, i2 / 8))[i2 % 8];
         if (g == 0 && ptid == 0) a.len[b] = S;
       }
-      // end of the tile: the staged rows are free, and one answer for all workers
+      // end of the tile: the next tile's weights have landed, the staged rows
+      // are free, and one answer for all workers
+      cp_async_wait_all_groups();
       ok = !named_barrier_or(1, 256, !ok || abort_flag);
     }
+    cp_async_wait_all_groups();   // no copy into shared memory outlives the loop
   }
 
   if (abort_flag) {
