@@ -102,6 +102,229 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// ------------------------------------------------------------------ per-head work
+// Shared by both forms.  Staged head rows: slot h (0..G-1 the query heads, G
+// the key head, G+1 the value head) holds 128 rows of 64 bytes at z + h zh,
+// row rr = position t0 - 3 + rr, 64B-swizzled.
+
+// 16 bytes at channel chunk c of slot h, staged row rr
+__device__ __forceinline__ const uint4* pp_zchunk(const uint8_t* z, uint32_t zh, int h, int rr,
+                                                  int c) {
+  return reinterpret_cast<const uint4*>(z + h * zh + swz_offset(rr, c * 16, kPpRow));
+}
+
+// conv of head hh for chunks j = P, P + 2, ... of output row r: u = sum_k w[c, k]
+// z[t - k, c] by fp32 FMAs on the bf16 operands (taps in order k = 0..3), then
+// u = hi + lo in bf16 into the U_hi / U_lo A tiles; rows past the CTA's output
+// get zeros
+template <int P>
+__device__ __forceinline__ void pp_conv(const uint8_t* z, uint32_t zh, const uint2* ws,
+                                        uint8_t* u_hi, uint32_t u_bytes, int hh, int r,
+                                        bool row_out) {
+  constexpr int D = kPpD, NCH = D / 8;
+#pragma unroll
+  for (int j = P; j < NCH; j += 2) {
+    uint4 hi4 = make_uint4(0, 0, 0, 0), lo4 = make_uint4(0, 0, 0, 0);
+    if (row_out) {
+      const uint4* tw = reinterpret_cast<const uint4*>(ws + hh * D + j * 8);   // 2 channels each
+      uint4 t4[4], zz[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) t4[q] = tw[q];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) zz[k] = *pp_zchunk(z, zh, hh, r + kPpHalo - k, j);
+      float acc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint4& tq = t4[e >> 1];
+        uint16_t w[4], zv[4];
+        halves((e & 1) ? tq.z : tq.x, w[0], w[1]);
+        halves((e & 1) ? tq.w : tq.y, w[2], w[3]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t* zw = reinterpret_cast<const uint32_t*>(&zz[k]);
+          uint16_t lo, hi;
+          halves(zw[e >> 1], lo, hi);
+          zv[k] = (e & 1) ? hi : lo;
+        }
+        float s = fma_bf16(zv[0], w[0], 0.f);
+#pragma unroll
+        for (int k = 1; k < 4; ++k) s = fma_bf16(zv[k], w[k], s);
+        acc[e] = s;
+      }
+      uint32_t* hp = reinterpret_cast<uint32_t*>(&hi4);
+      uint32_t* lp = reinterpret_cast<uint32_t*>(&lo4);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        hp[e] = pack2(acc[2 * e], acc[2 * e + 1]);
+        uint16_t h0, h1;
+        halves(hp[e], h0, h1);
+        // u - hi is exact in fp32
+        lp[e] = pack2(fma_bf16(h0, kBf16MinusOne, acc[2 * e]),
+                      fma_bf16(h1, kBf16MinusOne, acc[2 * e + 1]));
+      }
+    }
+    const uint32_t off = swz_offset(r, j * 16, kPpRow);
+    *reinterpret_cast<uint4*>(u_hi + off) = hi4;
+    *reinterpret_cast<uint4*>(u_hi + u_bytes + off) = lo4;
+  }
+}
+
+// epilogue of head hh for output row r (position t): the mixed channels
+// part*Q4 + e and d/2 + part*Q4 + e from TMEM at column tcol (warp-collective
+// loads), QK-mean from the staged pre-conv rows, RoPE with this thread's
+// (cos, sin), bf16 store into q (query heads) or the cache's k rows
+__device__ __forceinline__ void pp_epilogue(const uint8_t* z, uint32_t zh, uint32_t tcol, int hh,
+                                            int r, int part, int t, bool row_out,
+                                            const float (&rc)[kPpD / 4],
+                                            const float (&rs)[kPpD / 4],
+                                            const PreAttnArgs<bf16>& a, int b, int g) {
+  constexpr int D = kPpD, Q4 = D / 4;
+  const int G = a.G;
+  uint32_t ya[Q4], yb[Q4];
+  tmem_ld8(tcol, ya);
+  tmem_ld8(tcol + D / 2, yb);
+  tmem_wait_ld();
+  if (t >= a.S || !row_out) return;
+  const int i0 = part * Q4;
+  float lo[Q4], hi[Q4];
+#pragma unroll
+  for (int e = 0; e < Q4; ++e) {
+    lo[e] = __uint_as_float(ya[e]);
+    hi[e] = __uint_as_float(yb[e]);
+  }
+  const int rr = r + kPpHalo;                // this position's staged row
+  if (a.qk_mean == 2) {
+    // "self" reading: y = (y + own pre-conv value) / 2 over channels c0 + e
+    auto self_mean = [&](float (&y)[Q4], int c0) {
+      const uint4 ow = *pp_zchunk(z, zh, hh, rr, c0 / 8);
+      const uint32_t* op = reinterpret_cast<const uint32_t*>(&ow);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        uint16_t o0, o1;
+        halves(op[e], o0, o1);
+        y[2 * e] = fma_bf16(o0, kBf16Half, 0.5f * y[2 * e]);
+        y[2 * e + 1] = fma_bf16(o1, kBf16Half, 0.5f * y[2 * e + 1]);
+      }
+    };
+    self_mean(lo, i0);
+    self_mean(hi, i0 + D / 2);
+  } else if (a.qk_mean) {
+    const bool is_q = hh < G;
+    // y[e] += (q~ + k~) / 2 over channels c0 + e (q~: this head, or the mean of
+    // the group's query heads for the key head), as fp32 FMAs on the bf16 rows
+    auto add_mean = [&](float (&y)[Q4], int c0) {
+      const uint4 kw = *pp_zchunk(z, zh, G, rr, c0 / 8);
+      const uint32_t* kp = reinterpret_cast<const uint32_t*>(&kw);
+      if (is_q) {
+        const uint4 qw = *pp_zchunk(z, zh, hh, rr, c0 / 8);
+        const uint32_t* qp = reinterpret_cast<const uint32_t*>(&qw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          uint16_t q0, q1, k0, k1;
+          halves(qp[e], q0, q1);
+          halves(kp[e], k0, k1);
+          y[2 * e] = fma_bf16(k0, kBf16Half, fma_bf16(q0, kBf16Half, y[2 * e]));
+          y[2 * e + 1] = fma_bf16(k1, kBf16Half, fma_bf16(q1, kBf16Half, y[2 * e + 1]));
+        }
+      } else {
+        float sq[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sq[e] = 0.f;
+        for (int hl = 0; hl < G; ++hl) {
+          const uint4 qw = *pp_zchunk(z, zh, hl, rr, c0 / 8);
+          const uint32_t* qp = reinterpret_cast<const uint32_t*>(&qw);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint16_t q0, q1;
+            halves(qp[e], q0, q1);
+            sq[2 * e] = add_bf16(q0, sq[2 * e]);
+            sq[2 * e + 1] = add_bf16(q1, sq[2 * e + 1]);
+          }
+        }
+        const float hg = 0.5f / static_cast<float>(G);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          uint16_t k0, k1;
+          halves(kp[e], k0, k1);
+          y[2 * e] = fma_bf16(k0, kBf16Half, fmaf(sq[2 * e], hg, y[2 * e]));
+          y[2 * e + 1] = fma_bf16(k1, kBf16Half, fmaf(sq[2 * e + 1], hg, y[2 * e + 1]));
+        }
+      }
+    };
+    add_mean(lo, i0);
+    add_mean(hi, i0 + D / 2);
+  }
+  if (a.rope_on) {
+#pragma unroll
+    for (int e = 0; e < Q4; ++e) {
+      const float x0 = lo[e], x1 = hi[e];
+      lo[e] = x0 * rc[e] - x1 * rs[e];
+      hi[e] = x0 * rs[e] + x1 * rc[e];
+    }
+  }
+  bf16* dst = hh < G ? a.q_out + ((static_cast<int64_t>(b) * a.S + t) * a.Hq + g * G + hh) * D
+                     : a.k_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + t) * D;
+  uint4 pl, ph;
+  pl.x = pack2(lo[0], lo[1]);
+  pl.y = pack2(lo[2], lo[3]);
+  pl.z = pack2(lo[4], lo[5]);
+  pl.w = pack2(lo[6], lo[7]);
+  ph.x = pack2(hi[0], hi[1]);
+  ph.y = pack2(hi[2], hi[3]);
+  ph.z = pack2(hi[4], hi[5]);
+  ph.w = pack2(hi[6], hi[7]);
+  *reinterpret_cast<uint4*>(dst + i0) = pl;
+  *reinterpret_cast<uint4*>(dst + D / 2 + i0) = ph;
+}
+
+// value-shift rows of positions [t0, t0 + 125): v[t, :d/2] = v~[t, :d/2],
+// v[t, d/2:] = v~[t-1, d/2:] (whole-head reading: every channel from t - 1 when
+// the group's kv head is one of the last floor(Hkv / 2)); v~ of position -1 is
+// the zero row the TMA unit filled in.  Work items first, first + step, ...
+__device__ __forceinline__ void pp_value_shift(const uint8_t* z, uint32_t zh,
+                                               const PreAttnArgs<bf16>& a, int b, int g, int t0,
+                                               int first, int step) {
+  constexpr int D = kPpD, NCH = D / 8;
+  const bool shift_head = a.value_shift == 2 && g >= a.Hkv - a.Hkv / 2;
+  for (int idx = first; idx < kPpOut * NCH; idx += step) {
+    const int tl = idx / NCH, c = idx % NCH;
+    const int tv = t0 + tl;
+    if (tv >= a.S) continue;
+    const bool prev = (a.value_shift == 1 && c * 8 >= D / 2) || shift_head;
+    const uint4 v = *pp_zchunk(z, zh, a.G + 1, tl + kPpHalo - (prev ? 1 : 0), c);
+    *reinterpret_cast<uint4*>(a.v_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + tv) * D +
+                              c * 8) = v;
+  }
+}
+
+// decode state, written by the tile that holds position S - 1: the last K - 1
+// pre-conv q~ / k~ rows (staged rows; rows before position 0 are zero), v~ of
+// position S - 1 and len
+__device__ __forceinline__ void pp_decode_state(const uint8_t* z, uint32_t zh,
+                                                const PreAttnArgs<bf16>& a, int b, int g, int t0,
+                                                int first, int step) {
+  constexpr int D = kPpD;
+  const int S = a.S, G = a.G, QC = G * D;
+  if (a.len == nullptr || t0 > S - 1 || S - 1 >= t0 + kPpOut) return;
+  const int KH = a.K - 1, Hq = a.Hq, Hkv = a.Hkv, qcol0 = g * QC;
+  for (int rr = 0; rr < KH; ++rr) {
+    const int srow = S - KH + rr - t0 + kPpHalo;
+    for (int c = first; c < QC + D; c += step) {
+      const int h = c / D, ch = c % D;   // slot G: the key head
+      const bf16 v = reinterpret_cast<const bf16*>(pp_zchunk(z, zh, h, srow, ch / 8))[ch % 8];
+      if (c < QC)
+        a.hist_q[(static_cast<int64_t>(b) * KH + rr) * Hq * D + qcol0 + c] = v;
+      else
+        a.hist_k[(static_cast<int64_t>(b) * KH + rr) * Hkv * D + g * D + (c - QC)] = v;
+    }
+  }
+  if (a.v_prev)
+    for (int i = first; i < D; i += step)
+      a.v_prev[static_cast<int64_t>(b) * Hkv * D + g * D + i] =
+          reinterpret_cast<const bf16*>(pp_zchunk(z, zh, G + 1, S - 1 - t0 + kPpHalo, i / 8))[i % 8];
+  if (g == 0 && first == 0) a.len[b] = S;
+}
+
 // ------------------------------------------------------------------ persistent
 // The persistent, warp-specialised form (G <= 4, where its buffers fit in shared
 // memory): one CTA per SM walks tiles
@@ -159,7 +382,7 @@ __global__ void __launch_bounds__(kPwThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int G = a.G, S = a.S, K = a.K;
+  const int G = a.G, K = a.K;
   const PwLayout L = pw_layout(G);
   const int NH = G + 1, QC = G * D, NZ = static_cast<int>(L.nz);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -280,9 +503,6 @@ __global__ void __launch_bounds__(kPwThreads, 1)
     const uint32_t u_lo = u_hi + L.u_bytes;
     const uint32_t w_base = smem_addr(smem + L.off_w);
     const uint32_t idesc = make_idesc_bf16(kPpM, D, false);
-    auto zchunk = [&](int h, int rr, int c) -> const uint4* {
-      return reinterpret_cast<const uint4*>(z + h * L.zh_bytes + swz_offset(rr, c * 16, kRowBytes));
-    };
     // mix weights W_h [d_out][d_in] of group g into weight buffer wb (the
     // K-major 64B-swizzled B layout) and the group's raw taps into tap buffer
     // wb, by 16-byte asynchronous copies (all four sources 16-byte aligned)
@@ -378,53 +598,6 @@ __global__ void __launch_bounds__(kPwThreads, 1)
 
       // per head, as the one-tile kernel; mix MMA m (m = mix_base + head) goes
       // into accumulator m & 1 and completes on mma_done[m & 1]
-      auto conv_part = [&](int hh, auto part_c) {
-        constexpr int P = decltype(part_c)::value;
-#pragma unroll
-        for (int j = P; j < NCH; j += 2) {
-          uint4 hi4 = make_uint4(0, 0, 0, 0), lo4 = make_uint4(0, 0, 0, 0);
-          if (row_out) {
-            const uint4* tw = reinterpret_cast<const uint4*>(ws + hh * D + j * 8);
-            uint4 t4[4], zz[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) t4[q] = tw[q];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) zz[k] = *zchunk(hh, r + kPpHalo - k, j);
-            float acc[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const uint4& tq = t4[e >> 1];
-              uint16_t w[4], zv[4];
-              halves((e & 1) ? tq.z : tq.x, w[0], w[1]);
-              halves((e & 1) ? tq.w : tq.y, w[2], w[3]);
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const uint32_t* zw = reinterpret_cast<const uint32_t*>(&zz[k]);
-                uint16_t lo, hi;
-                halves(zw[e >> 1], lo, hi);
-                zv[k] = (e & 1) ? hi : lo;
-              }
-              float s = fma_bf16(zv[0], w[0], 0.f);
-#pragma unroll
-              for (int k = 1; k < 4; ++k) s = fma_bf16(zv[k], w[k], s);
-              acc[e] = s;
-            }
-            uint32_t* hp = reinterpret_cast<uint32_t*>(&hi4);
-            uint32_t* lp = reinterpret_cast<uint32_t*>(&lo4);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              hp[e] = pack2(acc[2 * e], acc[2 * e + 1]);
-              uint16_t h0, h1;
-              halves(hp[e], h0, h1);
-              lp[e] = pack2(fma_bf16(h0, kBf16MinusOne, acc[2 * e]),
-                            fma_bf16(h1, kBf16MinusOne, acc[2 * e + 1]));
-            }
-          }
-          const uint32_t off = swz_offset(r, j * 16, kRowBytes);
-          *reinterpret_cast<uint4*>(smem + L.off_u + off) = hi4;
-          *reinterpret_cast<uint4*>(smem + L.off_u + L.u_bytes + off) = lo4;
-        }
-      };
       auto issue_mma = [&](int hh, int m) {
         const uint32_t dt = tmem + col_mix + (m & 1) * D;
         const uint32_t wb = w_base + buf * L.wset_bytes + hh * L.w_bytes;
@@ -440,99 +613,8 @@ __global__ void __launch_bounds__(kPwThreads, 1)
       };
 
       auto epilogue = [&](int hh, int m) {
-        const uint32_t col = col_mix + (m & 1) * D + part * Q4;
-        uint32_t ya[Q4], yb[Q4];               // channels part*Q4 + e and D/2 + part*Q4 + e
-        tmem_ld8(trow + col, ya);
-        tmem_ld8(trow + col + D / 2, yb);
-        tmem_wait_ld();
-        if (tp >= S || !row_out) return;
-        const int i0 = part * Q4;
-        float lo[Q4], hi[Q4];
-#pragma unroll
-        for (int e = 0; e < Q4; ++e) {
-          lo[e] = __uint_as_float(ya[e]);
-          hi[e] = __uint_as_float(yb[e]);
-        }
-        const int rr = r + kPpHalo;            // this position's staged row
-        if (a.qk_mean == 2) {
-          auto self_mean = [&](float (&y)[Q4], int c0) {
-            const uint4 ow = *zchunk(hh, rr, c0 / 8);
-            const uint32_t* op = reinterpret_cast<const uint32_t*>(&ow);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              uint16_t o0, o1;
-              halves(op[e], o0, o1);
-              y[2 * e] = fma_bf16(o0, kBf16Half, 0.5f * y[2 * e]);
-              y[2 * e + 1] = fma_bf16(o1, kBf16Half, 0.5f * y[2 * e + 1]);
-            }
-          };
-          self_mean(lo, i0);
-          self_mean(hi, i0 + D / 2);
-        } else if (a.qk_mean) {
-          const bool is_q = hh < G;
-          auto add_mean = [&](float (&y)[Q4], int c0) {
-            const uint4 kw = *zchunk(G, rr, c0 / 8);
-            const uint32_t* kp = reinterpret_cast<const uint32_t*>(&kw);
-            if (is_q) {
-              const uint4 qw = *zchunk(hh, rr, c0 / 8);
-              const uint32_t* qp = reinterpret_cast<const uint32_t*>(&qw);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                uint16_t q0, q1, k0, k1;
-                halves(qp[e], q0, q1);
-                halves(kp[e], k0, k1);
-                y[2 * e] = fma_bf16(k0, kBf16Half, fma_bf16(q0, kBf16Half, y[2 * e]));
-                y[2 * e + 1] = fma_bf16(k1, kBf16Half, fma_bf16(q1, kBf16Half, y[2 * e + 1]));
-              }
-            } else {
-              float sq[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) sq[e] = 0.f;
-              for (int hl = 0; hl < G; ++hl) {
-                const uint4 qw = *zchunk(hl, rr, c0 / 8);
-                const uint32_t* qp = reinterpret_cast<const uint32_t*>(&qw);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  uint16_t q0, q1;
-                  halves(qp[e], q0, q1);
-                  sq[2 * e] = add_bf16(q0, sq[2 * e]);
-                  sq[2 * e + 1] = add_bf16(q1, sq[2 * e + 1]);
-                }
-              }
-              const float hg = 0.5f / static_cast<float>(G);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                uint16_t k0, k1;
-                halves(kp[e], k0, k1);
-                y[2 * e] = fma_bf16(k0, kBf16Half, fmaf(sq[2 * e], hg, y[2 * e]));
-                y[2 * e + 1] = fma_bf16(k1, kBf16Half, fmaf(sq[2 * e + 1], hg, y[2 * e + 1]));
-              }
-            }
-          };
-          add_mean(lo, i0);
-          add_mean(hi, i0 + D / 2);
-        }
-        if (a.rope_on) {
-#pragma unroll
-          for (int e = 0; e < Q4; ++e) {
-            const float x0 = lo[e], x1 = hi[e];
-            lo[e] = x0 * rc[e] - x1 * rs[e];
-            hi[e] = x0 * rs[e] + x1 * rc[e];
-          }
-        }
-        bf16* dst = hh < G ? a.q_out + ((static_cast<int64_t>(b) * S + tp) * a.Hq + g * G + hh) * D
-                           : a.k_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + tp) * D;
-        uint4 pl, ph;
-        pl.x = pack2(lo[0], lo[1]);
-        pl.y = pack2(lo[2], lo[3]);
-        pl.z = pack2(lo[4], lo[5]);
-        pl.w = pack2(lo[6], lo[7]);
-        ph.x = pack2(hi[0], hi[1]);
-        ph.y = pack2(hi[2], hi[3]);
-        ph.z = pack2(hi[4], hi[5]);
-        ph.w = pack2(hi[6], hi[7]);
-        *reinterpret_cast<uint4*>(dst + i0) = pl;
-        *reinterpret_cast<uint4*>(dst + D / 2 + i0) = ph;
+        pp_epilogue(z, L.zh_bytes, trow + col_mix + (m & 1) * D + part * Q4, hh, r, part, tp,
+                    row_out, rc, rs, a, b, g);
       };
 
       for (int hh = 0; hh < NH; ++hh) {
@@ -544,9 +626,9 @@ __global__ void __launch_bounds__(kPwThreads, 1)
         }
         if (ok) {
           if (part == 0)
-            conv_part(hh, std::integral_constant<int, 0>{});
+            pp_conv<0>(z, L.zh_bytes, ws, smem + L.off_u, L.u_bytes, hh, r, row_out);
           else
-            conv_part(hh, std::integral_constant<int, 1>{});
+            pp_conv<1>(z, L.zh_bytes, ws, smem + L.off_u, L.u_bytes, hh, r, row_out);
         }
         fence_proxy_async_smem();   // U is read by the tensor core
         tc_fence_before();
@@ -563,38 +645,8 @@ __global__ void __launch_bounds__(kPwThreads, 1)
       if (ok) epilogue(NH - 1, m_last);
       mix_base += NH;
 
-      // value-shift rows (the whole-head reading: every channel from t - 1
-      // when the group's kv head is one of the last floor(Hkv / 2))
-      const bool shift_head = a.value_shift == 2 && g >= a.Hkv - a.Hkv / 2;
-      for (int idx = ptid; idx < kPpOut * NCH; idx += 256) {
-        const int tl = idx / NCH, c = idx % NCH;
-        const int tv = t0 + tl;
-        if (tv >= S) continue;
-        const bool prev = (a.value_shift == 1 && c * 8 >= D / 2) || shift_head;
-        const uint4 v = *zchunk(G + 1, tl + kPpHalo - (prev ? 1 : 0), c);
-        *reinterpret_cast<uint4*>(a.v_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + tv) *
-                                                D + c * 8) = v;
-      }
-      // decode state, from the tile holding position S - 1
-      if (a.len != nullptr && t0 <= S - 1 && S - 1 < t0 + kPpOut) {
-        const int KH = K - 1, Hq = a.Hq, Hkv = a.Hkv, qcol0 = g * QC;
-        for (int rr = 0; rr < KH; ++rr) {
-          const int srow = S - KH + rr - t0 + kPpHalo;
-          for (int c = ptid; c < QC + D; c += 256) {
-            const int h = c / D, ch = c % D;
-            const bf16 v = reinterpret_cast<const bf16*>(zchunk(h, srow, ch / 8))[ch % 8];
-            if (c < QC)
-              a.hist_q[(static_cast<int64_t>(b) * KH + rr) * Hq * D + qcol0 + c] = v;
-            else
-              a.hist_k[(static_cast<int64_t>(b) * KH + rr) * Hkv * D + g * D + (c - QC)] = v;
-          }
-        }
-        if (a.v_prev)
-          for (int i2 = ptid; i2 < D; i2 += 256)
-            a.v_prev[static_cast<int64_t>(b) * Hkv * D + g * D + i2] =
-                reinterpret_cast<const bf16*>(zchunk(G + 1, S - 1 - t0 + kPpHalo, i2 / 8))[i2 % 8];
-        if (g == 0 && ptid == 0) a.len[b] = S;
-      }
+      pp_value_shift(z, L.zh_bytes, a, b, g, t0, ptid, 256);
+      pp_decode_state(z, L.zh_bytes, a, b, g, t0, ptid, 256);
       // end of the tile: the next tile's weights have landed, the staged rows
       // are free, and one answer for all workers
       cp_async_wait_all_groups();
@@ -635,7 +687,7 @@ __global__ void __launch_bounds__(kPwThreads, 1)
 // 97 KB of shared memory at G = 4, so two CTAs share an SM and one's GEMM runs
 // while the other works on its heads) otherwise.
 template <int kPpStages>
-__global__ void __launch_bounds__(kPpThreads, 1)
+__global__ void __launch_bounds__(kPpThreads, kPpStages == 2 ? 2 : 1)
     proj_pre_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                        const __grid_constant__ CUtensorMap tmWq,
                        const __grid_constant__ CUtensorMap tmWkv,
@@ -652,7 +704,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int G = a.G, S = a.S, K = a.K;
+  const int G = a.G, K = a.K;
   const PpLayout L = pp_layout(G, kPpStages);
   const int NH = G + 1, QC = G * D, NZ = static_cast<int>(L.nz);
   const int b = blockIdx.z, g = blockIdx.y, t0 = blockIdx.x * kPpOut;
@@ -670,7 +722,6 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   __shared__ int abort_flag, n_issued;   // n_issued: k-blocks whose loads the producer issued
 
   const int nkb = (E + kPpBK - 1) / kPpBK;
-  const int qcol0 = g * QC;
 
   if (tid == 0) {
     for (int s = 0; s < kPpStages; ++s) {
@@ -821,67 +872,11 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   const uint32_t idesc = make_idesc_bf16(kPpM, D, false);
   const int t = t0 + r;
   const bool row_out = r < kPpOut;         // rows 125..127 of the MMA tile are not written
-  // 16 bytes at channel chunk c of slot h, staged row rr (position t0 - 3 + rr)
-  auto zchunk = [&](int h, int rr, int c) -> const uint4* {
-    return reinterpret_cast<const uint4*>(z + h * L.zh_bytes + swz_offset(rr, c * 16, kRowBytes));
-  };
-
-  // conv of head hh for chunks j = P, P + 2, ... of row r: u = sum_k w[c, k]
-  // z[t - k, c] by fp32 FMAs on the bf16 operands (taps in order k = 0..3),
-  // then u = hi + lo in bf16; rows past the CTA's output get zeros
-  auto conv_part = [&](int hh, auto part_c) {
-    constexpr int P = decltype(part_c)::value;
-#pragma unroll
-    for (int j = P; j < NCH; j += 2) {
-      uint4 hi4 = make_uint4(0, 0, 0, 0), lo4 = make_uint4(0, 0, 0, 0);
-      if (row_out) {
-        const uint4* tw = reinterpret_cast<const uint4*>(ws + hh * D + j * 8);   // 2 channels each
-        uint4 t4[4], zz[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) t4[q] = tw[q];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) zz[k] = *zchunk(hh, r + kPpHalo - k, j);
-        float acc[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint4& tq = t4[e >> 1];
-          uint16_t w[4], zv[4];
-          halves((e & 1) ? tq.z : tq.x, w[0], w[1]);
-          halves((e & 1) ? tq.w : tq.y, w[2], w[3]);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t* zw = reinterpret_cast<const uint32_t*>(&zz[k]);
-            uint16_t lo, hi;
-            halves(zw[e >> 1], lo, hi);
-            zv[k] = (e & 1) ? hi : lo;
-          }
-          float s = fma_bf16(zv[0], w[0], 0.f);
-#pragma unroll
-          for (int k = 1; k < 4; ++k) s = fma_bf16(zv[k], w[k], s);
-          acc[e] = s;
-        }
-        uint32_t* hp = reinterpret_cast<uint32_t*>(&hi4);
-        uint32_t* lp = reinterpret_cast<uint32_t*>(&lo4);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          hp[e] = pack2(acc[2 * e], acc[2 * e + 1]);
-          uint16_t h0, h1;
-          halves(hp[e], h0, h1);
-          // u - hi is exact in fp32
-          lp[e] = pack2(fma_bf16(h0, kBf16MinusOne, acc[2 * e]),
-                        fma_bf16(h1, kBf16MinusOne, acc[2 * e + 1]));
-        }
-      }
-      const uint32_t off = swz_offset(r, j * 16, kRowBytes);
-      *reinterpret_cast<uint4*>(smem + L.off_u + off) = hi4;
-      *reinterpret_cast<uint4*>(smem + L.off_u + L.u_bytes + off) = lo4;
-    }
-  };
   auto conv = [&](int hh) {
     if (part == 0)
-      conv_part(hh, std::integral_constant<int, 0>{});
+      pp_conv<0>(z, L.zh_bytes, ws, smem + L.off_u, L.u_bytes, hh, r, row_out);
     else
-      conv_part(hh, std::integral_constant<int, 1>{});
+      pp_conv<1>(z, L.zh_bytes, ws, smem + L.off_u, L.u_bytes, hh, r, row_out);
   };
 
   auto issue_mma = [&](int hh) {
@@ -899,102 +894,8 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   };
 
   auto epilogue = [&](int hh) {
-    const uint32_t col = (hh & 1) * D + part * Q4;
-    uint32_t ya[Q4], yb[Q4];                 // channels part*Q4 + e and D/2 + part*Q4 + e
-    tmem_ld8(trow + col, ya);
-    tmem_ld8(trow + col + D / 2, yb);
-    tmem_wait_ld();
-    if (t >= S || !row_out) return;
-    const int i0 = part * Q4;
-    float lo[Q4], hi[Q4];
-#pragma unroll
-    for (int e = 0; e < Q4; ++e) {
-      lo[e] = __uint_as_float(ya[e]);
-      hi[e] = __uint_as_float(yb[e]);
-    }
-    const int rr = r + kPpHalo;              // this position's staged row
-    if (a.qk_mean == 2) {
-      // "self" reading: y = (y + own pre-conv value) / 2 over channels c0 + e
-      auto self_mean = [&](float (&y)[Q4], int c0) {
-        const uint4 ow = *zchunk(hh, rr, c0 / 8);
-        const uint32_t* op = reinterpret_cast<const uint32_t*>(&ow);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          uint16_t o0, o1;
-          halves(op[e], o0, o1);
-          y[2 * e] = fma_bf16(o0, kBf16Half, 0.5f * y[2 * e]);
-          y[2 * e + 1] = fma_bf16(o1, kBf16Half, 0.5f * y[2 * e + 1]);
-        }
-      };
-      self_mean(lo, i0);
-      self_mean(hi, i0 + D / 2);
-    } else if (a.qk_mean) {
-      const bool is_q = hh < G;
-      // y[e] += (q~ + k~) / 2 over channels c0 + e (q~: this head, or the mean
-      // of the group's query heads for the key head)
-      auto add_mean = [&](float (&y)[Q4], int c0) {
-        const uint4 kw = *zchunk(G, rr, c0 / 8);
-        const uint32_t* kp = reinterpret_cast<const uint32_t*>(&kw);
-        if (is_q) {
-          const uint4 qw = *zchunk(hh, rr, c0 / 8);
-          const uint32_t* qp = reinterpret_cast<const uint32_t*>(&qw);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            uint16_t q0, q1, k0, k1;
-            halves(qp[e], q0, q1);
-            halves(kp[e], k0, k1);
-            y[2 * e] = fma_bf16(k0, kBf16Half, fma_bf16(q0, kBf16Half, y[2 * e]));
-            y[2 * e + 1] = fma_bf16(k1, kBf16Half, fma_bf16(q1, kBf16Half, y[2 * e + 1]));
-          }
-        } else {
-          float sq[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) sq[e] = 0.f;
-          for (int hl = 0; hl < G; ++hl) {
-            const uint4 qw = *zchunk(hl, rr, c0 / 8);
-            const uint32_t* qp = reinterpret_cast<const uint32_t*>(&qw);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              uint16_t q0, q1;
-              halves(qp[e], q0, q1);
-              sq[2 * e] = add_bf16(q0, sq[2 * e]);
-              sq[2 * e + 1] = add_bf16(q1, sq[2 * e + 1]);
-            }
-          }
-          const float hg = 0.5f / static_cast<float>(G);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            uint16_t k0, k1;
-            halves(kp[e], k0, k1);
-            y[2 * e] = fma_bf16(k0, kBf16Half, fmaf(sq[2 * e], hg, y[2 * e]));
-            y[2 * e + 1] = fma_bf16(k1, kBf16Half, fmaf(sq[2 * e + 1], hg, y[2 * e + 1]));
-          }
-        }
-      };
-      add_mean(lo, i0);
-      add_mean(hi, i0 + D / 2);
-    }
-    if (a.rope_on) {
-#pragma unroll
-      for (int e = 0; e < Q4; ++e) {
-        const float x0 = lo[e], x1 = hi[e];
-        lo[e] = x0 * rc[e] - x1 * rs[e];
-        hi[e] = x0 * rs[e] + x1 * rc[e];
-      }
-    }
-    bf16* dst = hh < G ? a.q_out + ((static_cast<int64_t>(b) * S + t) * a.Hq + g * G + hh) * D
-                       : a.k_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + t) * D;
-    uint4 pl, ph;
-    pl.x = pack2(lo[0], lo[1]);
-    pl.y = pack2(lo[2], lo[3]);
-    pl.z = pack2(lo[4], lo[5]);
-    pl.w = pack2(lo[6], lo[7]);
-    ph.x = pack2(hi[0], hi[1]);
-    ph.y = pack2(hi[2], hi[3]);
-    ph.z = pack2(hi[4], hi[5]);
-    ph.w = pack2(hi[6], hi[7]);
-    *reinterpret_cast<uint4*>(dst + i0) = pl;
-    *reinterpret_cast<uint4*>(dst + D / 2 + i0) = ph;
+    pp_epilogue(z, L.zh_bytes, trow + (hh & 1) * D + part * Q4, hh, r, part, t, row_out, rc, rs,
+                a, b, g);
   };
 
   for (int hh = 0; hh < NH; ++hh) {
@@ -1018,42 +919,9 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   tc_fence_after();
   if (ok) epilogue(NH - 1);
 
-  // 4. value-shift rows: v[t, :d/2] = v~[t, :d/2], v[t, d/2:] = v~[t-1, d/2:]
-  // (whole-head reading: every channel from t - 1 when the group's kv head is
-  // one of the last floor(Hkv / 2)); v~ of position -1 is the zero row the
-  // TMA unit filled in
-  const bool shift_head = a.value_shift == 2 && g >= a.Hkv - a.Hkv / 2;
-  for (int idx = tid; idx < kPpOut * NCH; idx += kPpThreads) {
-    const int tl = idx / NCH, c = idx % NCH;
-    const int tv = t0 + tl;
-    if (tv >= S) continue;
-    const bool prev = (a.value_shift == 1 && c * 8 >= D / 2) || shift_head;
-    const uint4 v = *zchunk(G + 1, tl + kPpHalo - (prev ? 1 : 0), c);
-    *reinterpret_cast<uint4*>(a.v_out + ((static_cast<int64_t>(b) * a.Hkv + g) * a.kv_cap + tv) * D +
-                              c * 8) = v;
-  }
-
-  // 5. decode state, written by the CTA that holds position S - 1 (staged rows
-  // of positions S - K + 1 .. S - 1; rows before position 0 are zero)
-  if (a.len != nullptr && t0 <= S - 1 && S - 1 < t0 + kPpOut) {
-    const int KH = K - 1, Hq = a.Hq, Hkv = a.Hkv;
-    for (int rr = 0; rr < KH; ++rr) {
-      const int srow = S - KH + rr - t0 + kPpHalo;
-      for (int c = tid; c < QC + D; c += kPpThreads) {
-        const int h = c / D, ch = c % D;   // slot G: the key head
-        const bf16 v = reinterpret_cast<const bf16*>(zchunk(h, srow, ch / 8))[ch % 8];
-        if (c < QC)
-          a.hist_q[(static_cast<int64_t>(b) * KH + rr) * Hq * D + qcol0 + c] = v;
-        else
-          a.hist_k[(static_cast<int64_t>(b) * KH + rr) * Hkv * D + g * D + (c - QC)] = v;
-      }
-    }
-    if (a.v_prev)
-      for (int i = tid; i < D; i += kPpThreads)
-        a.v_prev[static_cast<int64_t>(b) * Hkv * D + g * D + i] =
-            reinterpret_cast<const bf16*>(zchunk(G + 1, S - 1 - t0 + kPpHalo, i / 8))[i % 8];
-    if (g == 0 && tid == 0) a.len[b] = S;
-  }
+  // 4. value-shift rows; 5. decode state (the CTA holding position S - 1)
+  pp_value_shift(z, L.zh_bytes, a, b, g, t0, tid, kPpThreads);
+  pp_decode_state(z, L.zh_bytes, a, b, g, t0, tid, kPpThreads);
 
   if (abort_flag && (tid == 0 || tid == 32)) {
     // Do not release TMEM while an MMA might still write it (each issuer

@@ -108,3 +108,19 @@ def test_fused_full_size_bit_identical_to_unfused():
     assert torch.equal(bits(out_f), bits(out_u))
     for key in ("k", "v", "hist_q", "hist_k", "v_prev", "len"):
         assert torch.equal(bits(t_f[key]), bits(t_u[key])), key
+
+
+def test_fused_one_tile_multi_wave_bit_identical_to_unfused():
+    """Six query heads per group (too many accumulators for the persistent
+    form) over more CTAs than one wave: the one-tile kernel with the 2-stage
+    ring, two CTAs per SM.  Bit-identical to the separate kernels."""
+    w = W2.with_(name="fu_g6_waves", B=2, S=5000, E=1536, C=4, Hq=12, Hkv=2)
+    assert -(-w.S // 125) * w.Hkv * w.B > 148
+    inp = make_inputs(w, seed=3)
+    out_f, t_f, n_f, _ = _run(w, inp, True)
+    out_u, t_u, n_u, _ = _run(w, inp, False)
+    assert n_f == n_u - 1, (n_f, n_u)
+    bits = lambda t: t.contiguous().view(torch.int16) if t.dtype == torch.bfloat16 else t  # noqa: E731
+    assert torch.equal(bits(out_f), bits(out_u))
+    for key in ("k", "v", "hist_q", "hist_k", "v_prev", "len"):
+        assert torch.equal(bits(t_f[key]), bits(t_u[key])), key
