@@ -16,8 +16,11 @@
  * Conventions for every entry point
  *  - All tensor pointers are DEVICE pointers, row-major, densely packed, owned
  *    by the caller; the library allocates no memory and keeps no state beyond
- *    a launch counter, the last CUDA error of each thread and the optional
- *    per-thread timing hook below.  Element type is cfg->dtype (fp32 or bf16)
+ *    a launch counter, the last CUDA error of each thread, the optional
+ *    per-thread timing hook, the process-wide fused-projection switch and the
+ *    allocation-free decode entry point's scratch array (all below), and a
+ *    record of the kernels whose shared-memory limit it has already raised.
+ *    Element type is cfg->dtype (fp32 or bf16)
  *    unless stated.  Every pointer must be 16-byte aligned.
  *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the
  *    legacy default stream).  Host-side validation happens first: on any
