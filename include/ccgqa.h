@@ -170,7 +170,11 @@ CCGQA_API size_t ccgqa_decode_workspace_size(const ccgqa_config* cfg, int32_t ba
  *      (which reads k / v from the workspace) by one page-scatter kernel.
  * workspace: >= ccgqa_prefill_workspace_size bytes, 256-byte aligned.
  * Steps: projection (tcgen05 GEMM for bf16), fused conv + channel mix +
- * QK-mean + RoPE + value-shift, flash attention (tcgen05/TMEM/TMA for bf16). */
+ * QK-mean + RoPE + value-shift, flash attention (tcgen05/TMEM/TMA for bf16).
+ * For bf16 at d = 32 with the depthwise conv (conv_width 1-4, both channel
+ * mixes given, G <= 6) the projection and the steps after it run as one
+ * kernel whose projected rows stay in shared memory; its results equal the
+ * separate kernels' bit for bit (ccgqa_set_fused_projection turns it off). */
 CCGQA_API ccgqa_status ccgqa_prefill(const ccgqa_config* cfg, const ccgqa_weights* w,
                                      const void* x, int32_t batch, int32_t seq_len,
                                      void* out, const ccgqa_kvcache* cache,
@@ -331,8 +335,9 @@ CCGQA_API void ccgqa_set_phase_events(void* const* events, int32_t n);
  * and conv weights ("Compressed Convolutional Attention", Methodologie: the
  * projected q~ | k~ | v~ never reach HBM).  Its phase events [1] and [2] then
  * both fall after that kernel.  0 runs the projection GEMM and the
- * pre-attention kernel separately (the results agree within the bf16 rounding
- * of the projection output).  For measurement and testing. */
+ * pre-attention kernel separately (the same results, bit for bit: the fused
+ * kernel rounds the projection to bf16 as the GEMM does and repeats the later
+ * steps' arithmetic).  For measurement and testing. */
 CCGQA_API void ccgqa_set_fused_projection(int32_t enable);
 
 /* Self-test of the device-side failure reporting (no counterpart in the
