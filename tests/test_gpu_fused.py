@@ -115,7 +115,7 @@ def test_fused_one_tile_multi_wave_bit_identical_to_unfused():
     form) over more CTAs than one wave: the one-tile kernel with the 2-stage
     ring, two CTAs per SM.  Bit-identical to the separate kernels."""
     w = W2.with_(name="fu_g6_waves", B=2, S=5000, E=1536, C=4, Hq=12, Hkv=2)
-    assert -(-w.S // 125) * w.Hkv * w.B > 148
+    assert -(-w.S // 125) * w.Hkv * w.B > torch.cuda.get_device_properties(0).multi_processor_count
     inp = make_inputs(w, seed=3)
     out_f, t_f, n_f, _ = _run(w, inp, True)
     out_u, t_u, n_u, _ = _run(w, inp, False)
